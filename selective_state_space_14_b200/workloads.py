@@ -1,0 +1,272 @@
+"""Seeded synthetic inputs for the selective-scan library and for its oracle.
+
+This module is the one piece shared by the CUDA path's tests/benchmark and the
+f64 oracle.  It draws random tensors and rounds them to the storage dtype; it
+holds none of the scan's arithmetic.  The only transforms applied here are the
+input *distributions* the workloads are defined with:
+
+* Mamba-1: x, z, B, C, D, dout ~ N(0,1); delta_raw = 0.5*N(0,1) - 2 (softplus is
+  applied by the scan, not here); A[c, n] = -exp(log(n + 1)); the delta bias of
+  the model-shaped workloads ~ U(ln 1e-3, ln 1e-1), the "targeted range" the
+  state-spaces/mamba README ("Troubleshooting / Initialization") describes.
+* Mamba-3 SISO: x, z, dout ~ N(0,1); B, C ~ N(0,1) then RMS-normalised over
+  d_state (the BCNorm stage that precedes the scan in the mamba-rs 0.4.2
+  ``Mamba3Scratch`` stage list, B5); alpha = exp(-softplus(N(0,1))); beta,
+  gamma ~ U(0, 0.5); theta (per-step rotation angle increments) ~ U(0, 0.1);
+  D ~ N(0,1) per head.
+
+Values are drawn in float32 from numpy's PCG64 with a fixed seed and rounded
+to the io dtype with round-to-nearest-even.  ``as_f64`` widens the rounded
+values, so the GPU path and the oracle see bit-identical inputs.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+from typing import Dict, Optional
+
+import numpy as np
+
+SEED_BASE = 20261202
+
+F32 = "f32"
+BF16 = "bf16"
+
+
+def round_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """float32 -> bfloat16 bit patterns (uint16), round-to-nearest-even."""
+    f = np.ascontiguousarray(x, dtype=np.float32)
+    bits = f.view(np.uint32).astype(np.uint64)
+    bits = (bits + 0x7FFF + ((bits >> 16) & 1)) >> 16
+    return bits.astype(np.uint16)
+
+
+def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
+    return (bits.astype(np.uint32) << 16).view(np.float32)
+
+
+@dataclass
+class Tensor:
+    """A stored tensor: its io dtype and its payload.
+
+    ``data`` is float32 for f32 tensors and uint16 bit patterns for bf16.
+    """
+
+    dtype: str
+    data: np.ndarray
+
+    @property
+    def shape(self):
+        return self.data.shape
+
+    def as_f32(self) -> np.ndarray:
+        if self.dtype == BF16:
+            return bf16_bits_to_f32(self.data)
+        return self.data
+
+    def as_f64(self) -> np.ndarray:
+        return self.as_f32().astype(np.float64)
+
+    @property
+    def nbytes(self) -> int:
+        return self.data.nbytes
+
+
+def store(x: np.ndarray, dtype: str) -> Tensor:
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    if dtype == BF16:
+        return Tensor(BF16, round_to_bf16_bits(x))
+    if dtype == F32:
+        return Tensor(F32, x)
+    raise ValueError(dtype)
+
+
+def _normal(rng, shape):
+    return rng.standard_normal(size=shape, dtype=np.float32)
+
+
+def _uniform(rng, lo, hi, shape):
+    return (lo + (hi - lo) * rng.random(size=shape, dtype=np.float32)).astype(np.float32)
+
+
+# --------------------------------------------------------------------------
+# Mamba-1 selective scan
+# --------------------------------------------------------------------------
+@dataclass
+class M1Problem:
+    batch: int
+    dim: int
+    dstate: int
+    seqlen: int
+    ngroups: int
+    io: str
+    delta_softplus: bool
+    u: Tensor
+    delta: Tensor
+    A: np.ndarray            # float32 [D, N]
+    B: Tensor                # [B, G, N, L]
+    C: Tensor                # [B, G, N, L]
+    D: Optional[np.ndarray]  # float32 [D]
+    delta_bias: Optional[np.ndarray]  # float32 [D]
+    z: Optional[Tensor]
+    h0: Optional[np.ndarray]  # float32 [B, D, N]
+    dout: Tensor
+    meta: Dict[str, object] = field(default_factory=dict)
+
+    @property
+    def token_channels(self) -> int:
+        return self.batch * self.dim * self.seqlen
+
+
+def m1_problem(batch, dim, dstate, seqlen, io=F32, seed=SEED_BASE, ngroups=1,
+               bias=False, with_z=True, with_D=True, with_h0=False,
+               delta_softplus=True) -> M1Problem:
+    """Mamba-1 scan inputs.
+
+    bias=False follows the small parity workload (no delta bias);
+    bias=True follows the model-shaped workloads (bias ~ U(ln 1e-3, ln 1e-1)).
+    """
+    rng = np.random.Generator(np.random.PCG64(seed))
+    Bsz, D, N, L, G = batch, dim, dstate, seqlen, ngroups
+    u = store(_normal(rng, (Bsz, D, L)), io)
+    delta = store(0.5 * _normal(rng, (Bsz, D, L)) - 2.0, io)
+    z = store(_normal(rng, (Bsz, D, L)), io) if with_z else None
+    Bm = store(_normal(rng, (Bsz, G, N, L)), io)
+    Cm = store(_normal(rng, (Bsz, G, N, L)), io)
+    A = np.ascontiguousarray(
+        np.broadcast_to(-np.exp(np.log(np.arange(1, N + 1, dtype=np.float64))), (D, N))
+    ).astype(np.float32)
+    Dp = _normal(rng, (D,)) if with_D else None
+    db = _uniform(rng, np.log(1e-3), np.log(1e-1), (D,)) if bias else None
+    h0 = _normal(rng, (Bsz, D, N)) if with_h0 else None
+    dout = store(_normal(rng, (Bsz, D, L)), io)
+    return M1Problem(Bsz, D, N, L, G, io, delta_softplus, u, delta, A, Bm, Cm, Dp, db, z,
+                     h0, dout)
+
+
+# --------------------------------------------------------------------------
+# Mamba-3 SISO scan
+# --------------------------------------------------------------------------
+@dataclass
+class M3Problem:
+    batch: int
+    seqlen: int
+    nheads: int
+    headdim: int
+    dstate: int
+    ngroups: int
+    nangles: int
+    io: str
+    x: Tensor          # [B, L, H, P]
+    z: Optional[Tensor]
+    B: Tensor          # [B, L, G, N]
+    C: Tensor          # [B, L, G, N]
+    alpha: Tensor      # [B, L, H]
+    beta: Tensor       # [B, L, H]
+    gamma: Tensor      # [B, L, H]
+    theta: Tensor      # [B, L, H, K]
+    D: Optional[np.ndarray]  # float32 [H]
+    h0: Optional[np.ndarray]  # float32 [B, H, P, N]
+    dout: Tensor
+
+    @property
+    def token_channels(self) -> int:
+        return self.batch * self.seqlen * self.nheads * self.headdim
+
+
+def _rms_normalise(v: np.ndarray, eps=1e-5) -> np.ndarray:
+    v64 = v.astype(np.float64)
+    return (v64 / np.sqrt(np.mean(v64 * v64, axis=-1, keepdims=True) + eps)).astype(np.float32)
+
+
+def m3_problem(batch, seqlen, nheads, headdim, dstate, ngroups=1, nangles=None, io=F32,
+               seed=SEED_BASE + 3, with_z=True, with_D=True, with_h0=False) -> M3Problem:
+    rng = np.random.Generator(np.random.PCG64(seed))
+    Bsz, L, H, P, N, G = batch, seqlen, nheads, headdim, dstate, ngroups
+    K = N // 2 if nangles is None else nangles
+    x = store(_normal(rng, (Bsz, L, H, P)), io)
+    z = store(_normal(rng, (Bsz, L, H, P)), io) if with_z else None
+    Bm = store(_rms_normalise(_normal(rng, (Bsz, L, G, N))), io)
+    Cm = store(_rms_normalise(_normal(rng, (Bsz, L, G, N))), io)
+    r = _normal(rng, (Bsz, L, H)).astype(np.float64)
+    alpha = store(np.exp(-np.logaddexp(0.0, r)), io)
+    beta = store(_uniform(rng, 0.0, 0.5, (Bsz, L, H)), io)
+    gamma = store(_uniform(rng, 0.0, 0.5, (Bsz, L, H)), io)
+    theta = store(_uniform(rng, 0.0, 0.1, (Bsz, L, H, K)), io)
+    Dp = _normal(rng, (H,)) if with_D else None
+    h0 = _normal(rng, (Bsz, H, P, N)) if with_h0 else None
+    dout = store(_normal(rng, (Bsz, L, H, P)), io)
+    return M3Problem(Bsz, L, H, P, N, G, K, io, x, z, Bm, Cm, alpha, beta, gamma, theta, Dp,
+                     h0, dout)
+
+
+# --------------------------------------------------------------------------
+# Single-token state update (decode)
+# --------------------------------------------------------------------------
+@dataclass
+class SUProblem:
+    batch: int
+    dim: int
+    dstate: int
+    ngroups: int
+    io: str
+    delta_softplus: bool
+    A: np.ndarray
+    D: Optional[np.ndarray]
+    delta_bias: Optional[np.ndarray]
+    state0: np.ndarray           # float32 [B, D, N]
+    steps: list                  # list of dicts: x, delta, z, B, C (Tensors)
+
+
+def su_problem(batch, dim, dstate, io=BF16, seed=SEED_BASE + 4, n_pool=8, ngroups=1,
+               random_state=False) -> SUProblem:
+    """Decode-step inputs: a pool of ``n_pool`` step input sets, cycled by the caller."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    Bsz, D, N, G = batch, dim, dstate, ngroups
+    A = np.ascontiguousarray(
+        np.broadcast_to(-np.exp(np.log(np.arange(1, N + 1, dtype=np.float64))), (D, N))
+    ).astype(np.float32)
+    Dp = _normal(rng, (D,))
+    db = _uniform(rng, np.log(1e-3), np.log(1e-1), (D,))
+    state0 = _normal(rng, (Bsz, D, N)) if random_state else np.zeros((Bsz, D, N), np.float32)
+    steps = []
+    for _ in range(n_pool):
+        steps.append(dict(
+            x=store(_normal(rng, (Bsz, D)), io),
+            delta=store(0.5 * _normal(rng, (Bsz, D)) - 2.0, io),
+            z=store(_normal(rng, (Bsz, D)), io),
+            B=store(_normal(rng, (Bsz, G, N)), io),
+            C=store(_normal(rng, (Bsz, G, N)), io),
+        ))
+    return SUProblem(Bsz, D, N, G, io, True, A, Dp, db, state0, steps)
+
+
+# --------------------------------------------------------------------------
+# The named workloads
+# --------------------------------------------------------------------------
+WORKLOADS = {
+    "m1_f32_b1_d64_n16_l256": dict(kind="m1", batch=1, dim=64, dstate=16, seqlen=256, io=F32,
+                                   bias=False, seed=SEED_BASE + 0),
+    "m1_bf16_b8_d1536_n16_l2048": dict(kind="m1", batch=8, dim=1536, dstate=16, seqlen=2048,
+                                       io=BF16, bias=True, seed=SEED_BASE + 1),
+    "m1_bf16_b4_d5120_n16_l4096": dict(kind="m1", batch=4, dim=5120, dstate=16, seqlen=4096,
+                                       io=BF16, bias=True, seed=SEED_BASE + 2),
+    "m3_bf16_b8_h24_p64_n64_k32_l2048": dict(kind="m3", batch=8, seqlen=2048, nheads=24,
+                                             headdim=64, dstate=64, nangles=32, io=BF16,
+                                             seed=SEED_BASE + 3),
+    "su_bf16_b256_d5120_n16_x1000": dict(kind="su", batch=256, dim=5120, dstate=16, io=BF16,
+                                         steps=1000, seed=SEED_BASE + 4),
+}
+
+
+def make(name: str):
+    w = dict(WORKLOADS[name])
+    kind = w.pop("kind")
+    if kind == "m1":
+        return m1_problem(w["batch"], w["dim"], w["dstate"], w["seqlen"], io=w["io"],
+                          seed=w["seed"], bias=w["bias"])
+    if kind == "m3":
+        return m3_problem(w["batch"], w["seqlen"], w["nheads"], w["headdim"], w["dstate"],
+                          nangles=w["nangles"], io=w["io"], seed=w["seed"])
+    if kind == "su":
+        return su_problem(w["batch"], w["dim"], w["dstate"], io=w["io"], seed=w["seed"])
+    raise ValueError(kind)
