@@ -1,0 +1,507 @@
+#!/usr/bin/env python3
+"""Benchmark of the selective-scan hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--no-extra] [--no-cpu-baseline]
+
+One step = the Mamba-1 selective scan forward + backward over one batch of the
+Mamba-130M-layer-shaped workload (bf16 storage, f32 accumulation; batch 8,
+d_inner 1536, d_state 16, L 2048), inputs resident in HBM.  Metric:
+tokens*channels per second (B*L*D per step / step time), whole job over all
+ranks.  Under torchrun each rank runs its own batch (independent problems, no
+data-path collective: weak scaling); timing is taken with CUDA events on the
+launching stream, bracketed by a barrier and a synchronize, max over ranks.
+
+The JSON line also carries: the roofline of the dominant launch (algorithmic
+bytes / measured duration vs the measured HBM copy bandwidth), the e2e figure
+(the same step through the C ABI starting from pinned host buffers, copies
+inside the timed region), the CPU oracle timed on a bounded sample, SM clocks
+sampled during the timed region, and per-workload figures for the other
+workloads (2.8B-layer-shaped Mamba-1, Mamba-3 SISO, decode step).
+
+--impl reference runs the f64 CPU oracle (the reference arm of this build) on a
+bounded sample of the same workload and prints the same metric.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from selective_state_space_14_b200 import workloads as W  # noqa: E402
+
+METRIC = "selective-scan tokens·channels/s (fwd+bwd) and achieved HBM GB/s vs ~8 TB/s peak"
+UNIT = "tokens*channels/s"
+HEADLINE = "m1_bf16_b8_d1536_n16_l2048"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return dict(hbm_gbs=float(d["hbm_gbs"]), bf16_tflops=float(d["bf16_tflops"]),
+                    bf16_tflops_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    sm_max_mhz=float(d.get("sm_max_mhz", 1965.0)), source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0,
+                sm_max_mhz=1965.0, source="fallback")
+
+
+# ---------------------------------------------------------------------------
+# algorithmic bytes (inputs read once + outputs written once)
+# ---------------------------------------------------------------------------
+def m1_bytes(Bsz, D, N, L, io_bytes, G=1):
+    tc = Bsz * D * L
+    bt = Bsz * G * L
+    params = D * N * 4 + 2 * D * 4
+    fwd = 4 * io_bytes * tc + 2 * N * io_bytes * bt + params + Bsz * D * N * 4  # x,dt,z,out; B,C; final
+    bwd = 7 * io_bytes * tc + 2 * N * io_bytes * bt + 2 * N * 4 * bt + params + D * N * 4 + 2 * D * 4
+    return fwd, bwd
+
+
+def m3_bytes(Bsz, L, H, P, N, G, K, io_bytes):
+    tc = Bsz * L * H * P
+    th = Bsz * L * H
+    bt = Bsz * L * G
+    fwd = 3 * io_bytes * tc + (3 + K) * io_bytes * th + 2 * N * io_bytes * bt + Bsz * H * P * N * 4
+    bwd = (5 * io_bytes * tc + (3 + K) * io_bytes * th + 2 * N * io_bytes * bt
+           + (3 + K) * 4 * th + 2 * N * 4 * bt + H * 4)
+    return fwd, bwd
+
+
+def su_bytes(Bsz, D, N, io_bytes, G=1):
+    return Bsz * D * (2 * N * 4 + 4 * io_bytes) + 2 * Bsz * G * N * io_bytes
+
+
+# ---------------------------------------------------------------------------
+# clocks sampling
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (FileNotFoundError, OSError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return dict(sm_mhz=None, sm_max_mhz=None, reasons=["nvidia-smi unavailable"])
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=2)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return dict(sm_mhz=None, sm_max_mhz=None, reasons=["no samples"])
+        return dict(sm_mhz=statistics.median(sm), sm_max_mhz=max(smax), reasons=sorted(reasons),
+                    samples=len(sm))
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (one process per GPU; no data-path collective)
+# ---------------------------------------------------------------------------
+def dist_init(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=None)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(world, value):
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def to_dev(t):
+    import torch
+    if t is None:
+        return None
+    if isinstance(t, np.ndarray):
+        return torch.from_numpy(np.ascontiguousarray(t, dtype=np.float32)).cuda()
+    if t.dtype == "bf16":
+        return torch.from_numpy(t.data.view(np.int16)).cuda().view(torch.bfloat16)
+    return torch.from_numpy(t.data).cuda()
+
+
+def to_pinned(t):
+    import torch
+    if t is None:
+        return None
+    if isinstance(t, np.ndarray):
+        return torch.from_numpy(np.ascontiguousarray(t, dtype=np.float32)).pin_memory()
+    if t.dtype == "bf16":
+        return torch.from_numpy(t.data.view(np.int16)).view(torch.bfloat16).pin_memory()
+    return torch.from_numpy(t.data).pin_memory()
+
+
+class M1Step:
+    """Device-resident Mamba-1 fwd+bwd step with all buffers preallocated."""
+
+    def __init__(self, p, msc):
+        import torch
+        self.msc = msc
+        self.p = p
+        self.a = dict(u=to_dev(p.u), delta=to_dev(p.delta), A=to_dev(p.A), B=to_dev(p.B),
+                      C=to_dev(p.C), D=to_dev(p.D), delta_bias=to_dev(p.delta_bias),
+                      z=to_dev(p.z), h0=None, delta_softplus=p.delta_softplus)
+        self.dout = to_dev(p.dout)
+        u = self.a["u"]
+        Bsz, D, L, N, G = p.batch, p.dim, p.seqlen, p.dstate, p.ngroups
+        f32 = dict(device="cuda", dtype=torch.float32)
+        self.out = torch.empty_like(u)
+        self.fs = torch.empty((Bsz, D, N), **f32)
+        self.saved = torch.empty((Bsz, D, (L + 255) // 256, N), **f32)
+        self.grads = dict(du=torch.empty_like(u), ddelta=torch.empty_like(u), dz=torch.empty_like(u),
+                          dA=torch.empty((D, N), **f32), dB=torch.empty((Bsz, G, N, L), **f32),
+                          dC=torch.empty((Bsz, G, N, L), **f32), dD=torch.empty((D,), **f32),
+                          ddelta_bias=torch.empty((D,), **f32), dh0=None)
+        self.ws = torch.empty(max(msc.msc_selective_scan_bwd_workspace_bytes(Bsz, D, N, L, G), 16),
+                              device="cuda", dtype=torch.uint8)
+
+    def fwd(self):
+        self.msc.msc_selective_scan_fwd(**self.a, out=self.out, final_state=self.fs,
+                                        saved_states=self.saved)
+
+    def bwd(self):
+        self.msc.msc_selective_scan_bwd(**self.a, saved_states=self.saved, dout=self.dout,
+                                        workspace=self.ws, grads=self.grads, want_dh0=False)
+
+
+def time_steps(step_fns, steps, warmup, world):
+    """Run warmup, then time `steps` iterations; per-phase CUDA-event times."""
+    import torch
+    for _ in range(warmup):
+        for f in step_fns:
+            f()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(step_fns) + 1)]
+          for _ in range(steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for k in range(steps):
+        ev[k][0].record(stream)
+        for i, f in enumerate(step_fns):
+            f()
+            ev[k][i + 1].record(stream)
+    end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    total_ms = start.elapsed_time(end)
+    phase_ms = [sum(ev[k][i].elapsed_time(ev[k][i + 1]) for k in range(steps)) / steps
+                for i in range(len(step_fns))]
+    return total_ms, phase_ms
+
+
+def cpu_baseline(budget_s=12.0):
+    """The f64 oracle (as it stands) on a bounded sample of the headline workload:
+    batch row 0, the first 96 channels, all 2048 steps, forward + backward."""
+    import oracle
+    p = W.make(HEADLINE)
+    nch = 96
+    sub = W.M1Problem(1, nch, p.dstate, p.seqlen, 1, p.io, p.delta_softplus,
+                      W.Tensor(p.io, p.u.data[:1, :nch]), W.Tensor(p.io, p.delta.data[:1, :nch]),
+                      p.A[:nch], W.Tensor(p.io, p.B.data[:1]), W.Tensor(p.io, p.C.data[:1]),
+                      p.D[:nch], p.delta_bias[:nch], W.Tensor(p.io, p.z.data[:1, :nch]), None,
+                      W.Tensor(p.io, p.dout.data[:1, :nch]))
+    args = oracle.m1_problem_args(sub)
+    dout = sub.dout.as_f64()
+    threads = oracle.default_threads()
+    reps, t_total = 0, 0.0
+    while t_total < budget_s and reps < 50:
+        t0 = time.perf_counter()
+        oracle.m1_fwd(**args, nthreads=threads)
+        oracle.m1_bwd(dout=dout, **args, nthreads=threads)
+        t_total += time.perf_counter() - t0
+        reps += 1
+    units = nch * p.seqlen * reps
+    return dict(value=units / t_total, unit=UNIT, cores=threads, kind="oracle",
+                sample=f"batch row 0, channels 0..{nch - 1}, L={p.seqlen}, fwd+bwd, {reps} reps, "
+                       f"{t_total:.1f} s")
+
+
+def run_e2e(p, msc, steps, warmup, world):
+    """Same step through the C ABI from pinned host buffers: H2D of the step's
+    inputs, fwd, bwd, D2H of every gradient and of the output, all timed."""
+    import torch
+    st = M1Step(p, msc)
+    host_in = dict(u=to_pinned(p.u), delta=to_pinned(p.delta), z=to_pinned(p.z), B=to_pinned(p.B),
+                   C=to_pinned(p.C), dout=to_pinned(p.dout))
+    dev_in = dict(u=st.a["u"], delta=st.a["delta"], z=st.a["z"], B=st.a["B"], C=st.a["C"],
+                  dout=st.dout)
+    outs = [st.out] + [v for v in st.grads.values() if v is not None]
+    host_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+    h2d = sum(v.numel() * v.element_size() for v in host_in.values())
+    d2h = sum(v.numel() * v.element_size() for v in host_out)
+
+    def step():
+        for k, v in host_in.items():
+            dev_in[k].copy_(v, non_blocking=True)
+        st.fwd()
+        st.bwd()
+        for d, h in zip(outs, host_out):
+            h.copy_(d, non_blocking=True)
+
+    total_ms, _ = time_steps([step], steps, warmup, world)
+    total_ms = max_over_ranks(world, total_ms)
+    return total_ms / steps, h2d, d2h
+
+
+def run_ours(args):
+    import torch
+    world, rank, local = dist_init(args.gpus)
+    torch.cuda.set_device(local)
+    from selective_state_space_14_b200 import msc
+    msc.lib()
+    peaks = load_peaks()
+    p = W.make(HEADLINE)
+    st = M1Step(p, msc)
+    sampler = ClockSampler(local)
+    sampler.start()
+    total_ms, (fwd_ms, bwd_ms) = time_steps([st.fwd, st.bwd], args.steps, args.warmup, world)
+    clocks = sampler.stop()
+    total_ms = max_over_ranks(world, total_ms)
+    ms_per_step = total_ms / args.steps
+    units = p.token_channels
+    value = units * world / (ms_per_step / 1e3)
+    fwd_b, bwd_b = m1_bytes(p.batch, p.dim, p.dstate, p.seqlen, 2)
+    dom = "bwd" if bwd_ms >= fwd_ms else "fwd"
+    dom_ms, dom_b = (bwd_ms, bwd_b) if dom == "bwd" else (fwd_ms, fwd_b)
+    achieved = dom_b / (dom_ms / 1e3) / 1e9
+    roofline = dict(bound="hbm", achieved=round(achieved, 1), peak=peaks["hbm_gbs"], unit="GB/s",
+                    frac=round(achieved / peaks["hbm_gbs"], 4), traffic=None,
+                    kernel=("msc_selective_scan_bwd (m1_bwd_kernel + m1_bwd_reduce_kernel)"
+                            if dom == "bwd" else "msc_selective_scan_fwd (m1_fwd_kernel)"),
+                    algorithmic_bytes=dom_b, launch_ms=round(dom_ms, 4),
+                    peak_source=peaks["source"])
+    e2e_ms, h2d, d2h = run_e2e(p, msc, max(2, args.steps // 2), 3, world)
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": HEADLINE, "batch": p.batch, "d_inner": p.dim, "d_state": p.dstate,
+                   "seq_len": p.seqlen, "io": "bf16 storage, f32 accumulation",
+                   "parallelism": f"independent batch per rank x{world}",
+                   "l2": "per-step working set > 126 MB L2 (inputs larger than L2)"},
+        "phases_ms": {"fwd": round(fwd_ms, 4), "bwd": round(bwd_ms, 4)},
+        "achieved_gbs": {"fwd": round(fwd_b / fwd_ms / 1e6, 1), "bwd": round(bwd_b / bwd_ms / 1e6, 1)},
+        "roofline": roofline,
+        "e2e": {"value": round(units * world / (e2e_ms / 1e3), 1), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(e2e_ms, 4)},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline()
+    if not args.no_extra:
+        line["workloads"] = extra_workloads(msc, args, world, peaks)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def extra_workloads(msc, args, world, peaks):
+    """Per-workload figures beside the headline (each timed like the headline)."""
+    import torch
+    res = {}
+    # Mamba-2.8B-layer-shaped Mamba-1 scan (bf16, B4 D5120 N16 L4096, final state)
+    p = W.make("m1_bf16_b4_d5120_n16_l4096")
+    st = M1Step(p, msc)
+    total_ms, (fwd_ms, bwd_ms) = time_steps([st.fwd, st.bwd], max(3, args.steps // 2), 3, world)
+    fb, bb = m1_bytes(p.batch, p.dim, p.dstate, p.seqlen, 2)
+    res["m1_bf16_b4_d5120_n16_l4096"] = dict(
+        fwd_ms=round(fwd_ms, 4), bwd_ms=round(bwd_ms, 4),
+        value=round(p.token_channels / ((fwd_ms + bwd_ms) / 1e3), 1), unit=UNIT,
+        fwd_hbm_frac=round(fb / fwd_ms / 1e6 / peaks["hbm_gbs"], 4),
+        bwd_hbm_frac=round(bb / bwd_ms / 1e6 / peaks["hbm_gbs"], 4))
+    del st
+    torch.cuda.empty_cache()
+    # decode step (B256 D5120 N16, 1000 consecutive steps cycling 8 input sets)
+    q = W.make("su_bf16_b256_d5120_n16_x1000")
+    state = torch.from_numpy(q.state0).cuda()
+    A, Dp, bias = to_dev(q.A), to_dev(q.D), to_dev(q.delta_bias)
+    pool = [{k: to_dev(v) for k, v in s.items()} for s in q.steps]
+    outs = [torch.empty_like(pool[0]["x"]) for _ in range(8)]
+
+    def decode_1000():
+        for t in range(1000):
+            s = pool[t % 8]
+            msc.msc_ssm_state_update(state, s["x"], s["delta"], A, s["B"], s["C"], D=Dp,
+                                     delta_bias=bias, z=s["z"], out=outs[t % 8])
+
+    total_ms, (ms,) = time_steps([decode_1000], 2, 1, world)
+    sb = su_bytes(q.batch, q.dim, q.dstate, 2)
+    res["su_bf16_b256_d5120_n16_x1000"] = dict(
+        ms_per_1000_steps=round(ms, 3), us_per_step=round(ms, 3),
+        value=round(q.batch * q.dim * 1000 / (ms / 1e3), 1), unit="channel-steps/s",
+        hbm_frac=round(sb * 1000 / (ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+        note="84 MB state can stay L2-resident between steps")
+    # Mamba-3 SISO
+    try:
+        m3 = W.make("m3_bf16_b8_h24_p64_n64_k32_l2048")
+        a = dict(x=to_dev(m3.x), B=to_dev(m3.B), C=to_dev(m3.C), alpha=to_dev(m3.alpha),
+                 beta=to_dev(m3.beta), gamma=to_dev(m3.gamma), theta=to_dev(m3.theta),
+                 D=to_dev(m3.D), z=to_dev(m3.z), h0=None)
+        dout = to_dev(m3.dout)
+        holder = {}
+
+        def f3():
+            holder["o"] = msc.msc_mamba3_siso_scan_fwd(**a, out=holder.get("out"),
+                                                       saved_states=holder.get("saved"))
+            holder["out"], holder["saved"] = holder["o"][0], holder["o"][2]
+
+        f3()
+        ws = torch.empty(max(msc.msc_mamba3_siso_scan_bwd_workspace_bytes(
+            m3.batch, m3.seqlen, m3.nheads, m3.headdim, m3.dstate, m3.ngroups, m3.nangles), 16),
+            device="cuda", dtype=torch.uint8)
+        grads = msc.msc_mamba3_siso_scan_bwd(**a, saved_states=holder["saved"], dout=dout,
+                                             workspace=ws)
+
+        def b3():
+            msc.msc_mamba3_siso_scan_bwd(**a, saved_states=holder["saved"], dout=dout,
+                                         workspace=ws, grads=grads)
+
+        total_ms, (f_ms, b_ms) = time_steps([f3, b3], max(3, args.steps // 2), 3, world)
+        fb, bb = m3_bytes(m3.batch, m3.seqlen, m3.nheads, m3.headdim, m3.dstate, m3.ngroups,
+                          m3.nangles, 2)
+        res["m3_bf16_b8_h24_p64_n64_k32_l2048"] = dict(
+            fwd_ms=round(f_ms, 4), bwd_ms=round(b_ms, 4),
+            value=round(m3.token_channels / ((f_ms + b_ms) / 1e3), 1), unit=UNIT,
+            fwd_hbm_frac=round(fb / f_ms / 1e6 / peaks["hbm_gbs"], 4),
+            bwd_hbm_frac=round(bb / b_ms / 1e6 / peaks["hbm_gbs"], 4))
+    except Exception as e:  # noqa: BLE001 -- report, keep the headline line
+        res["m3_bf16_b8_h24_p64_n64_k32_l2048"] = dict(error=str(e)[:200])
+    return res
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the f64 CPU oracle
+# ---------------------------------------------------------------------------
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    p = W.make(HEADLINE)
+    nch = 24
+    sub = W.M1Problem(1, nch, p.dstate, p.seqlen, 1, p.io, p.delta_softplus,
+                      W.Tensor(p.io, p.u.data[:1, :nch]), W.Tensor(p.io, p.delta.data[:1, :nch]),
+                      p.A[:nch], W.Tensor(p.io, p.B.data[:1]), W.Tensor(p.io, p.C.data[:1]),
+                      p.D[:nch], p.delta_bias[:nch], W.Tensor(p.io, p.z.data[:1, :nch]), None,
+                      W.Tensor(p.io, p.dout.data[:1, :nch]))
+    a = oracle.m1_problem_args(sub)
+    dout = sub.dout.as_f64()
+    threads = oracle.default_threads()
+    for _ in range(args.warmup):
+        oracle.m1_fwd(**a, nthreads=threads)
+        oracle.m1_bwd(dout=dout, **a, nthreads=threads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.m1_fwd(**a, nthreads=threads)
+        oracle.m1_bwd(dout=dout, **a, nthreads=threads)
+    dt = time.perf_counter() - t0
+    units = nch * p.seqlen * args.steps
+    value = units / dt
+    sample = f"batch row 0, channels 0..{nch - 1} of {HEADLINE}, fwd+bwd per step"
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 1), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": HEADLINE, "sample": sample},
+            "cpu_baseline": {"value": round(value, 1), "unit": UNIT, "cores": threads,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 1), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-extra", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,300 @@
+/*
+ * msc.h -- C ABI of the B200 selective state-space scan library (libmsc.so).
+ *
+ * The library computes the hot path of the Mamba family's selective SSM:
+ *
+ *   - the Mamba-1 selective scan, forward and backward (the selective SSM
+ *     layer of "Mamba: Linear-Time Sequence Modeling with Selective State
+ *     Spaces", Section 3 / Algorithm 2, as the state-spaces/mamba README's
+ *     "Usage / Selective SSM" section names it; "Mamba SSM (Gu and Dao,
+ *     2023)" with a "full backward pass through the recurrent SSM state" in
+ *     the mamba-rs 0.7.0 README, "Features");
+ *   - the Mamba-3 SISO scan, forward and backward (mamba-rs 0.7.0 README,
+ *     "Features"; backward stages B2 output gating, B3 BPTT and B4 RoPE of
+ *     Mamba3Scratch in mamba-rs 0.4.2 src/mamba3_siso/cpu/scratch.rs);
+ *   - the single-token recurrent state update used in decoding (mamba_step /
+ *     GpuMambaBackbone::step, mamba-rs 0.7.0 README, "Quick start").
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *   * Every function returns an msc_status.  On failure nothing is launched
+ *     and msc_last_error() returns a message (thread-local, valid until the
+ *     next call on the same thread) that names the offending argument.  The
+ *     one exception is MSC_ERR_CUDA, returned when a launch itself fails.
+ *   * Every tensor pointer is a caller-owned DEVICE pointer to a dense,
+ *     contiguous, row-major array with the layout stated below.  The library
+ *     allocates no memory, never synchronises, and launches all of its work
+ *     on the caller's stream; results are ready when the stream reaches them.
+ *   * Optional pointers may be NULL, meaning "absent": no h0 (zero initial
+ *     state), no z (no gate), no D (no skip), no delta_bias, no final state.
+ *   * io tensors (MSC_F32 or MSC_BF16, chosen per call) are read and written
+ *     in that dtype; every accumulation is f32 (the mamba-rs README,
+ *     "Features": "every kernel accumulates in f32"), and recurrent states and
+ *     reduced gradients are always f32.
+ *   * Results are bit-identical from run to run for the same inputs on the
+ *     same GPU and build: there are no atomics and every cross-thread
+ *     reduction has a fixed order (the "same bits run to run" guarantee of
+ *     mamba-rs docs/gemm-modes.md, "What is guaranteed").
+ *   * Argument structs begin with struct_size; callers set it to
+ *     sizeof(the struct) so that later fields can be added compatibly.
+ *   * Scratch memory, where an operation needs it, is passed in by the caller
+ *     (the "zero-allocation rule" of Mamba3Scratch: hot-path buffers are
+ *     preallocated once and reused); its size comes from the matching
+ *     *_bytes() query.
+ *   * Pointers must be 16-byte aligned.  Sequences of any length are
+ *     accepted; when a row's byte length is not a multiple of 16 the kernels
+ *     fall back to element loads for it.
+ */
+#ifndef MSC_H_
+#define MSC_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st *msc_stream_t;
+
+typedef enum {
+  MSC_OK = 0,
+  MSC_ERR_INVALID_ARG = 1, /* a NULL required pointer, a bad size or flag       */
+  MSC_ERR_UNSUPPORTED = 2, /* a valid request this build does not implement     */
+  MSC_ERR_ALIGNMENT = 3,   /* a pointer not 16-byte aligned                     */
+  MSC_ERR_CUDA = 4,        /* a CUDA launch error (message carries the reason)  */
+  MSC_ERR_WORKSPACE = 5    /* workspace pointer NULL or smaller than required   */
+} msc_status;
+
+typedef enum { MSC_F32 = 0, MSC_BF16 = 1 } msc_dtype;
+
+/* Message for the last failure on this thread ("" after a success). */
+const char *msc_last_error(void);
+
+/* Library version, e.g. "msc 0.1.0 sm_100a". */
+const char *msc_version(void);
+
+/* ======================================================================
+ * Mamba-1 selective scan
+ * ======================================================================
+ * Shapes: B = batch, D = dim (d_inner channels), N = dstate, L = seqlen,
+ * G = ngroups (B/C are shared by the D/G channels of a group; G divides D).
+ *
+ *   u, delta, z, out          io  [B, D, L]
+ *   Bm, Cm                    io  [B, G, N, L]
+ *   A                         f32 [D, N]
+ *   D, delta_bias             f32 [D]
+ *   h0, final_state           f32 [B, D, N]
+ *   saved_states              f32 [B, D, ceil(L / MSC_M1_SAVE_INTERVAL), N]
+ *
+ * Forward, per (b, c) and t = 0..L-1, with g the group of channel c:
+ *   delta_t = softplus(delta[b,c,t] + delta_bias[c])  if delta_softplus,
+ *             delta[b,c,t] + delta_bias[c]            otherwise
+ *   h[n]    = exp(delta_t * A[c,n]) * h[n] + delta_t * Bm[b,g,n,t] * u[b,c,t]
+ *   y       = sum_n Cm[b,g,n,t] * h[n] + D[c] * u[b,c,t]
+ *   out     = y * silu(z[b,c,t])                        (y if z is NULL)
+ * starting from h = h0[b,c,:] (or 0).  final_state receives h after the last
+ * step.  saved_states receives h at the start of every block of
+ * MSC_M1_SAVE_INTERVAL steps (the first is h0); the backward pass needs it.
+ * N may be 1..64; L >= 1.
+ */
+#define MSC_M1_SAVE_INTERVAL 256
+#define MSC_M1_MAX_DSTATE 64
+
+typedef struct {
+  uint32_t struct_size;
+  int32_t io_dtype;       /* msc_dtype of u, delta, z, Bm, Cm, out              */
+  int64_t batch, dim, dstate, seqlen, ngroups;
+  int32_t delta_softplus; /* 0 or 1                                            */
+  const void *u, *delta;
+  const float *A;
+  const void *Bm, *Cm;
+  const float *D;          /* optional */
+  const float *delta_bias; /* optional */
+  const void *z;           /* optional */
+  const float *h0;         /* optional */
+  void *out;
+  float *final_state;      /* optional */
+  float *saved_states;     /* optional; required if the backward pass follows */
+} msc_ss_fwd_args;
+
+/* Bytes of the saved_states array for these sizes. */
+size_t msc_selective_scan_saved_states_bytes(int64_t batch, int64_t dim, int64_t dstate,
+                                             int64_t seqlen);
+
+msc_status msc_selective_scan_fwd(const msc_ss_fwd_args *args, msc_stream_t stream);
+
+/*
+ * Backward (BPTT through the recurrent state).  Inputs are the forward's
+ * inputs, the saved_states it wrote, and dout [B, D, L] (io).  With
+ * g_t = dout_t * silu(z_t) and the state adjoint
+ *   lambda_t[n] = g_t Cm_t[n] + exp(delta_{t+1} A[c,n]) lambda_{t+1}[n]
+ * (lambda after the last step = 0: the final state is not differentiated):
+ *   du[b,c,t]        = g_t D[c] + delta_t sum_n lambda_t[n] Bm_t[n]       io
+ *   ddelta[b,c,t]    = d loss / d delta (raw, before bias and softplus)  io
+ *   dz[b,c,t]        = dout_t y_t silu'(z_t)                              io
+ *   dA[c,n]          = sum_{b,t} lambda_t delta_t exp(delta_t A) h_{t-1}  f32
+ *   dB[b,g,n,t]      = sum_{c in g} lambda_t[n] delta_t u_t               f32
+ *   dC[b,g,n,t]      = sum_{c in g} g_t h_t[n]                            f32
+ *   dD[c]            = sum_{b,t} g_t u_t                                  f32
+ *   ddelta_bias[c]   = sum_{b,t} ddelta[b,c,t]                            f32
+ *   dh0[b,c,n]       = exp(delta_0 A) lambda_0[n]                         f32
+ * dD, ddelta_bias, dz and dh0 are optional outputs (NULL: not computed).
+ * Every output is overwritten (not accumulated into).
+ * Workspace: msc_selective_scan_bwd_workspace_bytes() bytes of device memory,
+ * contents on entry irrelevant.
+ */
+typedef struct {
+  uint32_t struct_size;
+  int32_t io_dtype;
+  int64_t batch, dim, dstate, seqlen, ngroups;
+  int32_t delta_softplus;
+  const void *u, *delta;
+  const float *A;
+  const void *Bm, *Cm;
+  const float *D;          /* optional */
+  const float *delta_bias; /* optional */
+  const void *z;           /* optional */
+  const float *h0;         /* optional */
+  const float *saved_states; /* required: written by the forward            */
+  const void *dout;
+  void *du, *ddelta;
+  void *dz;                /* optional (only meaningful with z)              */
+  float *dA, *dB, *dC;
+  float *dD;               /* optional */
+  float *ddelta_bias;      /* optional */
+  float *dh0;              /* optional */
+} msc_ss_bwd_args;
+
+size_t msc_selective_scan_bwd_workspace_bytes(int64_t batch, int64_t dim, int64_t dstate,
+                                              int64_t seqlen, int64_t ngroups);
+
+msc_status msc_selective_scan_bwd(const msc_ss_bwd_args *args, void *workspace,
+                                  size_t workspace_bytes, msc_stream_t stream);
+
+/* ======================================================================
+ * Single-token state update (decode)
+ * ======================================================================
+ *   state                     f32 [B, D, N]   read and written in place
+ *   x, delta, z, out          io  [B, D]
+ *   Bm, Cm                    io  [B, G, N]
+ *   A f32 [D, N]; D, delta_bias f32 [D]
+ * One step of the Mamba-1 recurrence above, for every (b, c):
+ *   state[b,c,n] <- exp(delta A[c,n]) state[b,c,n] + delta Bm[b,g,n] x[b,c]
+ *   out[b,c]      = (sum_n Cm[b,g,n] state[b,c,n] + D[c] x[b,c]) silu(z[b,c])
+ * It equals the scan's step exactly in arithmetic order per element.
+ */
+typedef struct {
+  uint32_t struct_size;
+  int32_t io_dtype;
+  int64_t batch, dim, dstate, ngroups;
+  int32_t delta_softplus;
+  float *state;
+  const void *x, *delta;
+  const float *A;
+  const void *Bm, *Cm;
+  const float *D;          /* optional */
+  const float *delta_bias; /* optional */
+  const void *z;           /* optional */
+  void *out;
+} msc_su_args;
+
+msc_status msc_ssm_state_update(const msc_su_args *args, msc_stream_t stream);
+
+/* ======================================================================
+ * Mamba-3 SISO scan
+ * ======================================================================
+ * Shapes: B = batch, L = seqlen, H = nheads, P = headdim, N = dstate,
+ * G = ngroups (G divides H), K = nangles (2K <= N).
+ *
+ *   x, z, out                 io  [B, L, H, P]
+ *   Bm, Cm                    io  [B, L, G, N]
+ *   alpha, beta, gamma        io  [B, L, H]
+ *   theta                     io  [B, L, H, K]   per-step angle increments
+ *   D                         f32 [H]
+ *   h0, final_state           f32 [B, H, P, N]
+ *
+ * Per (b, h), with g the group of head h and t = 0..L-1:
+ *   phi_t[k] = sum_{s<=t} theta[b,s,h,k]
+ *   Bt_t = R(phi_t) Bm[b,t,g,:],  Ct_t = R(phi_t) Cm[b,t,g,:]
+ *      (R rotates each pair (2k, 2k+1), k < K, counter-clockwise by phi_t[k];
+ *       components 2K..N-1 are not rotated)
+ *   K_t  = x[b,t,h,:] (outer) Bt_t                                  [P, N]
+ *   S_t  = alpha_t S_{t-1} + beta_t K_{t-1} + gamma_t K_t,   K_{-1} = 0,
+ *          S_{-1} = h0 (or 0)
+ *   y_t  = S_t Ct_t + D[h] x[b,t,h,:];  out = y_t * silu(z[b,t,h,:])
+ * final_state receives S_{L-1}.
+ * Supported: P in {16, 32, 64, 128}, N in {16, 32, 64, 128}; L >= 1.
+ */
+typedef struct {
+  uint32_t struct_size;
+  int32_t io_dtype;
+  int64_t batch, seqlen, nheads, headdim, dstate, ngroups, nangles;
+  const void *x;
+  const void *z;           /* optional */
+  const void *Bm, *Cm;
+  const void *alpha, *beta, *gamma, *theta;
+  const float *D;          /* optional */
+  const float *h0;         /* optional */
+  void *out;
+  float *final_state;      /* optional */
+  float *saved_states;     /* optional; required if the backward pass follows */
+} msc_m3_fwd_args;
+
+/* saved_states holds S at the start of every block of MSC_M3_CHUNK steps,
+ * f32 [B, H, ceil(L / MSC_M3_CHUNK), P, N]; this returns its size in bytes. */
+#define MSC_M3_CHUNK 64
+size_t msc_mamba3_siso_saved_states_bytes(int64_t batch, int64_t seqlen, int64_t nheads,
+                                          int64_t headdim, int64_t dstate);
+
+msc_status msc_mamba3_siso_scan_fwd(const msc_m3_fwd_args *args, msc_stream_t stream);
+
+/*
+ * Backward.  Inputs are the forward's inputs, the saved_states it wrote and
+ * dout [B, L, H, P] (io).  With g_t = dout_t * silu(z_t) and the state adjoint
+ *   Lambda_t = g_t (outer) Ct_t + alpha_{t+1} Lambda_{t+1}:
+ *   dK_t        = gamma_t Lambda_t + beta_{t+1} Lambda_{t+1}
+ *   dx          = dK_t Bt_t + D g_t                                     io
+ *   dz          = dout_t y_t silu'(z_t)                                 io
+ *   dalpha_t    = <Lambda_t, S_{t-1}>, dbeta_t = <Lambda_t, K_{t-1}>,
+ *   dgamma_t    = <Lambda_t, K_t>                                       f32 [B,L,H]
+ *   dB, dC      = R(phi_t)^T (dK_t^T x_t), R(phi_t)^T (S_t^T g_t),
+ *                 summed over the heads of the group                    f32 [B,L,G,N]
+ *   dtheta_t[k] = sum_{s>=t} dphi_s[k]                                  f32 [B,L,H,K]
+ *   dD[h]       = sum g_t . x_t                                         f32 [H]
+ *   dh0         = alpha_0 Lambda_0                                      f32 [B,H,P,N]
+ * dz, dD and dh0 are optional outputs.  Every output is overwritten.
+ */
+typedef struct {
+  uint32_t struct_size;
+  int32_t io_dtype;
+  int64_t batch, seqlen, nheads, headdim, dstate, ngroups, nangles;
+  const void *x;
+  const void *z;           /* optional */
+  const void *Bm, *Cm;
+  const void *alpha, *beta, *gamma, *theta;
+  const float *D;          /* optional */
+  const float *h0;         /* optional */
+  const float *saved_states; /* required: written by the forward            */
+  const void *dout;
+  void *dx;
+  void *dz;                /* optional */
+  float *dB, *dC;
+  float *dalpha, *dbeta, *dgamma, *dtheta;
+  float *dD;               /* optional */
+  float *dh0;              /* optional */
+} msc_m3_bwd_args;
+
+size_t msc_mamba3_siso_scan_bwd_workspace_bytes(int64_t batch, int64_t seqlen, int64_t nheads,
+                                                int64_t headdim, int64_t dstate,
+                                                int64_t ngroups, int64_t nangles);
+
+msc_status msc_mamba3_siso_scan_bwd(const msc_m3_bwd_args *args, void *workspace,
+                                    size_t workspace_bytes, msc_stream_t stream);
+
+#ifdef __cplusplus
+} /* extern "C" */
+#endif
+
+#endif /* MSC_H_ */

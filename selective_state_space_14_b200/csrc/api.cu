@@ -1,0 +1,261 @@
+// api.cu -- the extern "C" entry points of libmsc.so (declared in msc.h).
+//
+// Each entry point checks its arguments on the host, translates them into the
+// internal launch parameters and enqueues the kernels on the caller's stream.
+// Nothing here allocates device memory or synchronises.  Errors are reported
+// as msc_status codes plus a thread-local message that names the argument
+// (the mamba-rs docs/gemm-modes.md "Errors" section: messages name the call or
+// value that failed).
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "../../include/msc.h"
+#include "kernels.h"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+msc_status fail(msc_status st, const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+msc_status ok() {
+  g_err[0] = '\0';
+  return MSC_OK;
+}
+
+msc_status cuda_status(cudaError_t e, const char *what) {
+  if (e == cudaSuccess) return ok();
+  return fail(MSC_ERR_CUDA, "%s: CUDA error %s (%s)", what, cudaGetErrorName(e),
+              cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+#define REQUIRE_PTR(fn, name, ptr)                                                   \
+  do {                                                                              \
+    if ((ptr) == nullptr) return fail(MSC_ERR_INVALID_ARG, "%s: %s is NULL", fn, name); \
+    if (!aligned16(ptr))                                                            \
+      return fail(MSC_ERR_ALIGNMENT, "%s: %s is not 16-byte aligned", fn, name);    \
+  } while (0)
+
+#define OPTIONAL_PTR(fn, name, ptr)                                                 \
+  do {                                                                              \
+    if ((ptr) != nullptr && !aligned16(ptr))                                        \
+      return fail(MSC_ERR_ALIGNMENT, "%s: %s is not 16-byte aligned", fn, name);    \
+  } while (0)
+
+size_t io_size(int32_t dt) { return dt == MSC_BF16 ? 2 : 4; }
+
+msc_status check_dtype(const char *fn, int32_t dt) {
+  if (dt != MSC_F32 && dt != MSC_BF16)
+    return fail(MSC_ERR_INVALID_ARG, "%s: io_dtype %d is not MSC_F32 (0) or MSC_BF16 (1)", fn,
+                (int)dt);
+  return MSC_OK;
+}
+
+msc_status check_flag(const char *fn, const char *name, int32_t v) {
+  if (v != 0 && v != 1) return fail(MSC_ERR_INVALID_ARG, "%s: %s must be 0 or 1, got %d", fn, name, (int)v);
+  return MSC_OK;
+}
+
+// Shared size checks of the Mamba-1 scans.
+msc_status check_m1_sizes(const char *fn, int64_t B, int64_t D, int64_t N, int64_t L, int64_t G) {
+  if (B < 0 || D < 0 || L < 0)
+    return fail(MSC_ERR_INVALID_ARG, "%s: batch, dim and seqlen must be >= 0 (got %lld, %lld, %lld)",
+                fn, (long long)B, (long long)D, (long long)L);
+  if (N < 1 || N > MSC_M1_MAX_DSTATE)
+    return fail(MSC_ERR_UNSUPPORTED, "%s: dstate %lld outside the supported range 1..%d", fn,
+                (long long)N, MSC_M1_MAX_DSTATE);
+  if (G < 1 || (D > 0 && D % G != 0))
+    return fail(MSC_ERR_INVALID_ARG, "%s: ngroups %lld must be >= 1 and divide dim %lld", fn,
+                (long long)G, (long long)D);
+  if (B > 65535)
+    return fail(MSC_ERR_UNSUPPORTED, "%s: batch %lld exceeds 65535", fn, (long long)B);
+  return MSC_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *msc_last_error(void) { return g_err; }
+
+const char *msc_version(void) { return "msc 0.1.0 sm_100a"; }
+
+// ============================================================== Mamba-1 ====
+size_t msc_selective_scan_saved_states_bytes(int64_t batch, int64_t dim, int64_t dstate,
+                                             int64_t seqlen) {
+  if (batch <= 0 || dim <= 0 || dstate <= 0 || seqlen <= 0) return 0;
+  const int64_t n_save = (seqlen + MSC_M1_SAVE_INTERVAL - 1) / MSC_M1_SAVE_INTERVAL;
+  return sizeof(float) * (size_t)(batch * dim * n_save * dstate);
+}
+
+msc_status msc_selective_scan_fwd(const msc_ss_fwd_args *a, msc_stream_t stream) {
+  const char *fn = "msc_selective_scan_fwd";
+  if (!a) return fail(MSC_ERR_INVALID_ARG, "%s: args is NULL", fn);
+  if (a->struct_size < sizeof(msc_ss_fwd_args))
+    return fail(MSC_ERR_INVALID_ARG, "%s: struct_size %u < sizeof(msc_ss_fwd_args) %zu", fn,
+                a->struct_size, sizeof(msc_ss_fwd_args));
+  msc_status st;
+  if ((st = check_dtype(fn, a->io_dtype)) != MSC_OK) return st;
+  if ((st = check_flag(fn, "delta_softplus", a->delta_softplus)) != MSC_OK) return st;
+  if ((st = check_m1_sizes(fn, a->batch, a->dim, a->dstate, a->seqlen, a->ngroups)) != MSC_OK)
+    return st;
+  const int64_t B = a->batch, D = a->dim, N = a->dstate, L = a->seqlen;
+  if (B == 0 || D == 0) return ok();
+  REQUIRE_PTR(fn, "A", a->A);
+  OPTIONAL_PTR(fn, "D", a->D);
+  OPTIONAL_PTR(fn, "delta_bias", a->delta_bias);
+  OPTIONAL_PTR(fn, "h0", a->h0);
+  OPTIONAL_PTR(fn, "final_state", a->final_state);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (L == 0) {  // no steps: the final state is the initial state
+    if (a->final_state) {
+      const size_t bytes = sizeof(float) * (size_t)(B * D * N);
+      cudaError_t e = a->h0 ? cudaMemcpyAsync(a->final_state, a->h0, bytes,
+                                              cudaMemcpyDeviceToDevice, s)
+                            : cudaMemsetAsync(a->final_state, 0, bytes, s);
+      return cuda_status(e, fn);
+    }
+    return ok();
+  }
+  REQUIRE_PTR(fn, "u", a->u);
+  REQUIRE_PTR(fn, "delta", a->delta);
+  REQUIRE_PTR(fn, "Bm", a->Bm);
+  REQUIRE_PTR(fn, "Cm", a->Cm);
+  REQUIRE_PTR(fn, "out", a->out);
+  OPTIONAL_PTR(fn, "z", a->z);
+  OPTIONAL_PTR(fn, "saved_states", a->saved_states);
+
+  msc::M1Params p = {};
+  p.io_bf16 = a->io_dtype == MSC_BF16;
+  p.B = B; p.D = D; p.N = N; p.L = L; p.G = a->ngroups;
+  p.softplus = a->delta_softplus;
+  p.vec = (L * (int64_t)io_size(a->io_dtype)) % 16 == 0;
+  p.u = a->u; p.delta = a->delta; p.Bm = a->Bm; p.Cm = a->Cm; p.z = a->z;
+  p.A = a->A; p.Dp = a->D; p.bias = a->delta_bias; p.h0 = a->h0;
+  p.out = a->out; p.final_state = a->final_state; p.saved = a->saved_states;
+  return cuda_status(msc::launch_m1_fwd(p, s), fn);
+}
+
+size_t msc_selective_scan_bwd_workspace_bytes(int64_t batch, int64_t dim, int64_t dstate,
+                                              int64_t seqlen, int64_t ngroups) {
+  if (batch <= 0 || dim <= 0 || dstate <= 0 || seqlen <= 0) return 0;
+  return msc::m1_bwd_workspace_bytes(batch, dim, dstate, seqlen, ngroups);
+}
+
+msc_status msc_selective_scan_bwd(const msc_ss_bwd_args *a, void *workspace,
+                                  size_t workspace_bytes, msc_stream_t stream) {
+  const char *fn = "msc_selective_scan_bwd";
+  if (!a) return fail(MSC_ERR_INVALID_ARG, "%s: args is NULL", fn);
+  if (a->struct_size < sizeof(msc_ss_bwd_args))
+    return fail(MSC_ERR_INVALID_ARG, "%s: struct_size %u < sizeof(msc_ss_bwd_args) %zu", fn,
+                a->struct_size, sizeof(msc_ss_bwd_args));
+  msc_status st;
+  if ((st = check_dtype(fn, a->io_dtype)) != MSC_OK) return st;
+  if ((st = check_flag(fn, "delta_softplus", a->delta_softplus)) != MSC_OK) return st;
+  if ((st = check_m1_sizes(fn, a->batch, a->dim, a->dstate, a->seqlen, a->ngroups)) != MSC_OK)
+    return st;
+  const int64_t B = a->batch, D = a->dim, N = a->dstate, L = a->seqlen, G = a->ngroups;
+  if (G > 1 && (D / G) % msc::kM1BwdBlock != 0)
+    return fail(MSC_ERR_UNSUPPORTED,
+                "%s: with ngroups > 1 the channels per group (%lld) must be a multiple of %d",
+                fn, (long long)(D / G), msc::kM1BwdBlock);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (D == 0) return ok();
+  REQUIRE_PTR(fn, "A", a->A);
+  REQUIRE_PTR(fn, "dA", a->dA);
+  OPTIONAL_PTR(fn, "dD", a->dD);
+  OPTIONAL_PTR(fn, "ddelta_bias", a->ddelta_bias);
+  OPTIONAL_PTR(fn, "dh0", a->dh0);
+  if (B == 0 || L == 0) {  // nothing depends on any parameter: zero gradients
+    cudaError_t e = cudaMemsetAsync(a->dA, 0, sizeof(float) * (size_t)(D * N), s);
+    if (e == cudaSuccess && a->dD) e = cudaMemsetAsync(a->dD, 0, sizeof(float) * (size_t)D, s);
+    if (e == cudaSuccess && a->ddelta_bias)
+      e = cudaMemsetAsync(a->ddelta_bias, 0, sizeof(float) * (size_t)D, s);
+    if (e == cudaSuccess && a->dh0 && B > 0)
+      e = cudaMemsetAsync(a->dh0, 0, sizeof(float) * (size_t)(B * D * N), s);
+    return cuda_status(e, fn);
+  }
+  REQUIRE_PTR(fn, "u", a->u);
+  REQUIRE_PTR(fn, "delta", a->delta);
+  REQUIRE_PTR(fn, "Bm", a->Bm);
+  REQUIRE_PTR(fn, "Cm", a->Cm);
+  REQUIRE_PTR(fn, "saved_states", a->saved_states);
+  REQUIRE_PTR(fn, "dout", a->dout);
+  REQUIRE_PTR(fn, "du", a->du);
+  REQUIRE_PTR(fn, "ddelta", a->ddelta);
+  REQUIRE_PTR(fn, "dB", a->dB);
+  REQUIRE_PTR(fn, "dC", a->dC);
+  OPTIONAL_PTR(fn, "D", a->D);
+  OPTIONAL_PTR(fn, "delta_bias", a->delta_bias);
+  OPTIONAL_PTR(fn, "z", a->z);
+  OPTIONAL_PTR(fn, "h0", a->h0);
+  OPTIONAL_PTR(fn, "dz", a->dz);
+  const size_t need = msc::m1_bwd_workspace_bytes(B, D, N, L, G);
+  if (workspace == nullptr || workspace_bytes < need)
+    return fail(MSC_ERR_WORKSPACE, "%s: workspace of %zu bytes given, %zu required", fn,
+                workspace ? workspace_bytes : (size_t)0, need);
+  if (!aligned16(workspace))
+    return fail(MSC_ERR_ALIGNMENT, "%s: workspace is not 16-byte aligned", fn);
+
+  msc::M1Params p = {};
+  p.io_bf16 = a->io_dtype == MSC_BF16;
+  p.B = B; p.D = D; p.N = N; p.L = L; p.G = G;
+  p.softplus = a->delta_softplus;
+  p.vec = (L * (int64_t)io_size(a->io_dtype)) % 16 == 0;
+  p.u = a->u; p.delta = a->delta; p.Bm = a->Bm; p.Cm = a->Cm; p.z = a->z;
+  p.A = a->A; p.Dp = a->D; p.bias = a->delta_bias; p.h0 = a->h0;
+  p.saved_in = a->saved_states; p.dout = a->dout;
+  p.du = a->du; p.ddelta = a->ddelta; p.dz = a->z ? a->dz : nullptr;
+  p.dA = a->dA; p.dB = a->dB; p.dC = a->dC; p.dD = a->dD; p.dbias = a->ddelta_bias;
+  p.dh0 = a->dh0;
+  p.n_part = (D + msc::kM1BwdBlock - 1) / msc::kM1BwdBlock;
+  const size_t bc = ((sizeof(float) * (size_t)(p.n_part * B * 2 * N * L)) + 255) / 256 * 256;
+  p.ws_bc = static_cast<float *>(workspace);
+  p.ws_misc = reinterpret_cast<float *>(static_cast<char *>(workspace) + bc);
+  return cuda_status(msc::launch_m1_bwd(p, s), fn);
+}
+
+// ======================================================== decode step ====
+msc_status msc_ssm_state_update(const msc_su_args *a, msc_stream_t stream) {
+  const char *fn = "msc_ssm_state_update";
+  if (!a) return fail(MSC_ERR_INVALID_ARG, "%s: args is NULL", fn);
+  if (a->struct_size < sizeof(msc_su_args))
+    return fail(MSC_ERR_INVALID_ARG, "%s: struct_size %u < sizeof(msc_su_args) %zu", fn,
+                a->struct_size, sizeof(msc_su_args));
+  msc_status st;
+  if ((st = check_dtype(fn, a->io_dtype)) != MSC_OK) return st;
+  if ((st = check_flag(fn, "delta_softplus", a->delta_softplus)) != MSC_OK) return st;
+  if ((st = check_m1_sizes(fn, 0, a->dim, a->dstate, 0, a->ngroups)) != MSC_OK) return st;
+  if (a->batch < 0) return fail(MSC_ERR_INVALID_ARG, "%s: batch must be >= 0", fn);
+  if (a->batch == 0 || a->dim == 0) return ok();
+  REQUIRE_PTR(fn, "state", a->state);
+  REQUIRE_PTR(fn, "x", a->x);
+  REQUIRE_PTR(fn, "delta", a->delta);
+  REQUIRE_PTR(fn, "A", a->A);
+  REQUIRE_PTR(fn, "Bm", a->Bm);
+  REQUIRE_PTR(fn, "Cm", a->Cm);
+  REQUIRE_PTR(fn, "out", a->out);
+  OPTIONAL_PTR(fn, "D", a->D);
+  OPTIONAL_PTR(fn, "delta_bias", a->delta_bias);
+  OPTIONAL_PTR(fn, "z", a->z);
+  msc::SUParams p = {};
+  p.io_bf16 = a->io_dtype == MSC_BF16;
+  p.B = a->batch; p.D = a->dim; p.N = a->dstate; p.G = a->ngroups;
+  p.softplus = a->delta_softplus;
+  p.state = a->state; p.x = a->x; p.delta = a->delta; p.Bm = a->Bm; p.Cm = a->Cm; p.z = a->z;
+  p.A = a->A; p.Dp = a->D; p.bias = a->delta_bias; p.out = a->out;
+  return cuda_status(msc::launch_state_update(p, reinterpret_cast<cudaStream_t>(stream)), fn);
+}
+
+}  // extern "C"

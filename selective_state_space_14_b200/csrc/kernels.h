@@ -1,0 +1,75 @@
+// kernels.h -- internal launch interface between the C ABI layer (api.cu) and
+// the kernel translation units.  Not installed; msc.h is the public surface.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace msc {
+
+// ---------------------------------------------------------------- Mamba-1 --
+struct M1Params {
+  int io_bf16;
+  int64_t B, D, N, L, G;
+  int softplus;
+  bool vec;  // rows of length L are 16-byte aligned for vector access
+  const void *u, *delta, *Bm, *Cm, *z;
+  const float *A, *Dp, *bias, *h0;
+  // forward outputs
+  void *out;
+  float *final_state, *saved;
+  // backward
+  const float *saved_in;
+  const void *dout;
+  void *du, *ddelta, *dz;
+  float *dA, *dB, *dC, *dD, *dbias, *dh0;
+  float *ws_bc;    // [n_part][B][2][N][L] partial sums of dB, dC
+  float *ws_misc;  // [B][D][N + 2]: per-(b, c) dA row, dD, dbias
+  int64_t n_part;  // partials per batch row (channel blocks of kM1BwdBlock)
+};
+
+constexpr int MSC_MAX_N = 64;             // largest Mamba-1 d_state
+constexpr int kM1SaveInterval = 256;      // saved-state spacing (time steps)
+constexpr int kM1BwdWarps = 8;            // channels per CTA in the backward
+constexpr int kM1BwdCluster = 8;          // CTAs per cluster in the backward
+constexpr int kM1BwdBlock = kM1BwdWarps * kM1BwdCluster;  // channels per partial
+
+cudaError_t launch_m1_fwd(const M1Params &p, cudaStream_t s);
+cudaError_t launch_m1_bwd(const M1Params &p, cudaStream_t s);
+size_t m1_bwd_workspace_bytes(int64_t B, int64_t D, int64_t N, int64_t L, int64_t G);
+
+// ------------------------------------------------------------ decode step --
+struct SUParams {
+  int io_bf16;
+  int64_t B, D, N, G;
+  int softplus;
+  float *state;
+  const void *x, *delta, *Bm, *Cm, *z;
+  const float *A, *Dp, *bias;
+  void *out;
+};
+cudaError_t launch_state_update(const SUParams &p, cudaStream_t s);
+
+// ---------------------------------------------------------- Mamba-3 SISO --
+struct M3Params {
+  int io_bf16;
+  int64_t B, L, H, P, N, G, K;
+  const void *x, *z, *Bm, *Cm, *alpha, *beta, *gamma, *theta;
+  const float *Dp, *h0;
+  void *out;
+  float *final_state;
+  // backward
+  const void *dout;
+  void *dx, *dz;
+  float *dB, *dC, *dalpha, *dbeta, *dgamma, *dtheta, *dD, *dh0;
+  void *ws;
+  size_t ws_bytes;
+};
+cudaError_t launch_m3_fwd(const M3Params &p, cudaStream_t s);
+cudaError_t launch_m3_bwd(const M3Params &p, cudaStream_t s);
+size_t m3_bwd_workspace_bytes(int64_t B, int64_t L, int64_t H, int64_t P, int64_t N, int64_t G,
+                              int64_t K);
+bool m3_supported(int64_t P, int64_t N);
+
+}  // namespace msc

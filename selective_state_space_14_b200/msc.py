@@ -1,0 +1,322 @@
+"""Thin Python binding of libmsc.so (the C ABI declared in include/msc.h).
+
+Argument marshalling only: every step of the scans runs in the library's CUDA
+kernels.  torch supplies device memory and the current stream.  There is no
+CPU fallback: if libmsc.so is missing or cannot be loaded, every call raises.
+
+The functions carry the C entry points' names and take torch tensors laid out
+as msc.h states (contiguous, on the current CUDA device).  Outputs not passed
+in are allocated with torch and returned.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmsc.so")
+
+MSC_F32, MSC_BF16 = 0, 1
+MSC_M1_SAVE_INTERVAL = 256
+
+STATUS = {0: "MSC_OK", 1: "MSC_ERR_INVALID_ARG", 2: "MSC_ERR_UNSUPPORTED", 3: "MSC_ERR_ALIGNMENT",
+          4: "MSC_ERR_CUDA", 5: "MSC_ERR_WORKSPACE"}
+
+
+class MscError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+_vp = ctypes.c_void_p
+_i64 = ctypes.c_int64
+_i32 = ctypes.c_int32
+_u32 = ctypes.c_uint32
+
+
+class SsFwdArgs(ctypes.Structure):
+    _fields_ = [("struct_size", _u32), ("io_dtype", _i32), ("batch", _i64), ("dim", _i64),
+                ("dstate", _i64), ("seqlen", _i64), ("ngroups", _i64), ("delta_softplus", _i32),
+                ("u", _vp), ("delta", _vp), ("A", _vp), ("Bm", _vp), ("Cm", _vp), ("D", _vp),
+                ("delta_bias", _vp), ("z", _vp), ("h0", _vp), ("out", _vp), ("final_state", _vp),
+                ("saved_states", _vp)]
+
+
+class SsBwdArgs(ctypes.Structure):
+    _fields_ = [("struct_size", _u32), ("io_dtype", _i32), ("batch", _i64), ("dim", _i64),
+                ("dstate", _i64), ("seqlen", _i64), ("ngroups", _i64), ("delta_softplus", _i32),
+                ("u", _vp), ("delta", _vp), ("A", _vp), ("Bm", _vp), ("Cm", _vp), ("D", _vp),
+                ("delta_bias", _vp), ("z", _vp), ("h0", _vp), ("saved_states", _vp),
+                ("dout", _vp), ("du", _vp), ("ddelta", _vp), ("dz", _vp), ("dA", _vp),
+                ("dB", _vp), ("dC", _vp), ("dD", _vp), ("ddelta_bias", _vp), ("dh0", _vp)]
+
+
+class SuArgs(ctypes.Structure):
+    _fields_ = [("struct_size", _u32), ("io_dtype", _i32), ("batch", _i64), ("dim", _i64),
+                ("dstate", _i64), ("ngroups", _i64), ("delta_softplus", _i32), ("state", _vp),
+                ("x", _vp), ("delta", _vp), ("A", _vp), ("Bm", _vp), ("Cm", _vp), ("D", _vp),
+                ("delta_bias", _vp), ("z", _vp), ("out", _vp)]
+
+
+class M3FwdArgs(ctypes.Structure):
+    _fields_ = [("struct_size", _u32), ("io_dtype", _i32), ("batch", _i64), ("seqlen", _i64),
+                ("nheads", _i64), ("headdim", _i64), ("dstate", _i64), ("ngroups", _i64),
+                ("nangles", _i64), ("x", _vp), ("z", _vp), ("Bm", _vp), ("Cm", _vp),
+                ("alpha", _vp), ("beta", _vp), ("gamma", _vp), ("theta", _vp), ("D", _vp),
+                ("h0", _vp), ("out", _vp), ("final_state", _vp), ("saved_states", _vp)]
+
+
+class M3BwdArgs(ctypes.Structure):
+    _fields_ = [("struct_size", _u32), ("io_dtype", _i32), ("batch", _i64), ("seqlen", _i64),
+                ("nheads", _i64), ("headdim", _i64), ("dstate", _i64), ("ngroups", _i64),
+                ("nangles", _i64), ("x", _vp), ("z", _vp), ("Bm", _vp), ("Cm", _vp),
+                ("alpha", _vp), ("beta", _vp), ("gamma", _vp), ("theta", _vp), ("D", _vp),
+                ("h0", _vp), ("saved_states", _vp), ("dout", _vp), ("dx", _vp), ("dz", _vp),
+                ("dB", _vp), ("dC", _vp), ("dalpha", _vp), ("dbeta", _vp), ("dgamma", _vp),
+                ("dtheta", _vp), ("dD", _vp), ("dh0", _vp)]
+
+
+EXPORTS = ["msc_last_error", "msc_version", "msc_selective_scan_saved_states_bytes",
+           "msc_selective_scan_fwd", "msc_selective_scan_bwd_workspace_bytes",
+           "msc_selective_scan_bwd", "msc_ssm_state_update", "msc_mamba3_siso_saved_states_bytes",
+           "msc_mamba3_siso_scan_fwd", "msc_mamba3_siso_scan_bwd_workspace_bytes",
+           "msc_mamba3_siso_scan_bwd"]
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmsc.so (raises if it is missing: there is no fallback)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing; build it with "
+                               "`python -m selective_state_space_14_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        L.msc_last_error.restype = ctypes.c_char_p
+        L.msc_version.restype = ctypes.c_char_p
+        for name, argt in (("msc_selective_scan_fwd", [ctypes.POINTER(SsFwdArgs), _vp]),
+                           ("msc_selective_scan_bwd",
+                            [ctypes.POINTER(SsBwdArgs), _vp, ctypes.c_size_t, _vp]),
+                           ("msc_ssm_state_update", [ctypes.POINTER(SuArgs), _vp]),
+                           ("msc_mamba3_siso_scan_fwd", [ctypes.POINTER(M3FwdArgs), _vp]),
+                           ("msc_mamba3_siso_scan_bwd",
+                            [ctypes.POINTER(M3BwdArgs), _vp, ctypes.c_size_t, _vp])):
+            f = getattr(L, name)
+            f.argtypes = argt
+            f.restype = ctypes.c_int
+        L.msc_selective_scan_saved_states_bytes.argtypes = [_i64] * 4
+        L.msc_selective_scan_saved_states_bytes.restype = ctypes.c_size_t
+        L.msc_selective_scan_bwd_workspace_bytes.argtypes = [_i64] * 5
+        L.msc_selective_scan_bwd_workspace_bytes.restype = ctypes.c_size_t
+        L.msc_mamba3_siso_saved_states_bytes.argtypes = [_i64] * 5
+        L.msc_mamba3_siso_saved_states_bytes.restype = ctypes.c_size_t
+        L.msc_mamba3_siso_scan_bwd_workspace_bytes.argtypes = [_i64] * 7
+        L.msc_mamba3_siso_scan_bwd_workspace_bytes.restype = ctypes.c_size_t
+        _lib = L
+    return _lib
+
+
+def version() -> str:
+    return lib().msc_version().decode()
+
+
+def _check(status: int):
+    if status != 0:
+        raise MscError(status, lib().msc_last_error().decode())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libmsc must be contiguous")
+    return t.data_ptr()
+
+
+def _io(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return MSC_BF16
+    if t.dtype == torch.float32:
+        return MSC_F32
+    raise TypeError(f"unsupported io dtype {t.dtype}")
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+# ---------------------------------------------------------------------------
+# Mamba-1 selective scan
+# ---------------------------------------------------------------------------
+def msc_selective_scan_saved_states_bytes(batch, dim, dstate, seqlen) -> int:
+    return int(lib().msc_selective_scan_saved_states_bytes(batch, dim, dstate, seqlen))
+
+
+def msc_selective_scan_bwd_workspace_bytes(batch, dim, dstate, seqlen, ngroups=1) -> int:
+    return int(lib().msc_selective_scan_bwd_workspace_bytes(batch, dim, dstate, seqlen, ngroups))
+
+
+def msc_selective_scan_fwd(u, delta, A, B, C, D=None, delta_bias=None, z=None, h0=None,
+                           delta_softplus=True, out=None, final_state=None, saved_states=None,
+                           want_final_state=True, want_saved_states=True, stream=None):
+    """Mamba-1 forward.  u, delta, z: [B, D, L]; A: f32 [D, N]; B, C: [B, G, N, L].
+
+    Returns (out, final_state, saved_states)."""
+    Bsz, Dm, L = u.shape
+    G, N = B.shape[1], B.shape[2]
+    dev = u.device
+    if out is None:
+        out = torch.empty_like(u)
+    if final_state is None and want_final_state:
+        final_state = torch.empty((Bsz, Dm, N), device=dev, dtype=torch.float32)
+    if saved_states is None and want_saved_states:
+        n_save = (L + MSC_M1_SAVE_INTERVAL - 1) // MSC_M1_SAVE_INTERVAL
+        saved_states = torch.empty((Bsz, Dm, max(n_save, 1), N), device=dev, dtype=torch.float32)
+    a = SsFwdArgs(ctypes.sizeof(SsFwdArgs), _io(u), Bsz, Dm, N, L, G, int(delta_softplus),
+                  _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(delta_bias),
+                  _ptr(z), _ptr(h0), _ptr(out), _ptr(final_state), _ptr(saved_states))
+    _check(lib().msc_selective_scan_fwd(ctypes.byref(a), _stream(stream)))
+    return out, final_state, saved_states
+
+
+def msc_selective_scan_bwd(u, delta, A, B, C, saved_states, dout, D=None, delta_bias=None, z=None,
+                           h0=None, delta_softplus=True, workspace=None, want_dh0=True,
+                           grads=None, stream=None):
+    """Mamba-1 backward.  Returns dict du, ddelta, dA, dB, dC, dD, ddelta_bias, dz, dh0."""
+    Bsz, Dm, L = u.shape
+    G, N = B.shape[1], B.shape[2]
+    dev = u.device
+    f32 = dict(device=dev, dtype=torch.float32)
+    g = dict(grads or {})
+    if "du" not in g:
+        g["du"] = torch.empty_like(u)
+    if "ddelta" not in g:
+        g["ddelta"] = torch.empty_like(u)
+    if "dA" not in g:
+        g["dA"] = torch.empty((Dm, N), **f32)
+    if "dB" not in g:
+        g["dB"] = torch.empty((Bsz, G, N, L), **f32)
+    if "dC" not in g:
+        g["dC"] = torch.empty((Bsz, G, N, L), **f32)
+    if "dD" not in g:
+        g["dD"] = torch.empty((Dm,), **f32)
+    if "ddelta_bias" not in g:
+        g["ddelta_bias"] = torch.empty((Dm,), **f32)
+    if "dz" not in g:
+        g["dz"] = torch.empty_like(u) if z is not None else None
+    if "dh0" not in g:
+        g["dh0"] = torch.empty((Bsz, Dm, N), **f32) if want_dh0 else None
+    need = msc_selective_scan_bwd_workspace_bytes(Bsz, Dm, N, L, G)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), device=dev, dtype=torch.uint8)
+    a = SsBwdArgs(ctypes.sizeof(SsBwdArgs), _io(u), Bsz, Dm, N, L, G, int(delta_softplus),
+                  _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(delta_bias),
+                  _ptr(z), _ptr(h0), _ptr(saved_states), _ptr(dout), _ptr(g["du"]),
+                  _ptr(g["ddelta"]), _ptr(g["dz"]), _ptr(g["dA"]), _ptr(g["dB"]), _ptr(g["dC"]),
+                  _ptr(g["dD"]), _ptr(g["ddelta_bias"]), _ptr(g["dh0"]))
+    _check(lib().msc_selective_scan_bwd(ctypes.byref(a), _ptr(workspace), workspace.numel(),
+                                        _stream(stream)))
+    return g
+
+
+# ---------------------------------------------------------------------------
+# single-token state update
+# ---------------------------------------------------------------------------
+def msc_ssm_state_update(state, x, delta, A, B, C, D=None, delta_bias=None, z=None,
+                         delta_softplus=True, out=None, stream=None):
+    """In-place decode step.  state f32 [B, D, N]; x, delta, z [B, D]; B, C [B, G, N]."""
+    Bsz, Dm, N = state.shape
+    G = B.shape[1]
+    if out is None:
+        out = torch.empty_like(x)
+    a = SuArgs(ctypes.sizeof(SuArgs), _io(x), Bsz, Dm, N, G, int(delta_softplus), _ptr(state),
+               _ptr(x), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(delta_bias),
+               _ptr(z), _ptr(out))
+    _check(lib().msc_ssm_state_update(ctypes.byref(a), _stream(stream)))
+    return out
+
+
+# ---------------------------------------------------------------------------
+# Mamba-3 SISO
+# ---------------------------------------------------------------------------
+def msc_mamba3_siso_saved_states_bytes(batch, seqlen, nheads, headdim, dstate) -> int:
+    return int(lib().msc_mamba3_siso_saved_states_bytes(batch, seqlen, nheads, headdim, dstate))
+
+
+def msc_mamba3_siso_scan_bwd_workspace_bytes(batch, seqlen, nheads, headdim, dstate, ngroups,
+                                             nangles) -> int:
+    return int(lib().msc_mamba3_siso_scan_bwd_workspace_bytes(batch, seqlen, nheads, headdim,
+                                                                 dstate, ngroups, nangles))
+
+
+def msc_mamba3_siso_scan_fwd(x, B, C, alpha, beta, gamma, theta, D=None, z=None, h0=None,
+                             out=None, final_state=None, saved_states=None,
+                             want_final_state=True, want_saved_states=True, stream=None):
+    """Mamba-3 SISO forward.  x, z [B, L, H, P]; B, C [B, L, G, N]; alpha, beta, gamma
+    [B, L, H]; theta [B, L, H, K].  Returns (out, final_state, saved_states)."""
+    Bsz, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    K = theta.shape[3]
+    dev = x.device
+    if out is None:
+        out = torch.empty_like(x)
+    if final_state is None and want_final_state:
+        final_state = torch.empty((Bsz, H, P, N), device=dev, dtype=torch.float32)
+    if saved_states is None and want_saved_states:
+        nb = msc_mamba3_siso_saved_states_bytes(Bsz, L, H, P, N)
+        saved_states = torch.empty(max(nb // 4, 4), device=dev, dtype=torch.float32)
+    a = M3FwdArgs(ctypes.sizeof(M3FwdArgs), _io(x), Bsz, L, H, P, N, G, K, _ptr(x), _ptr(z),
+                  _ptr(B), _ptr(C), _ptr(alpha), _ptr(beta), _ptr(gamma), _ptr(theta), _ptr(D),
+                  _ptr(h0), _ptr(out), _ptr(final_state), _ptr(saved_states))
+    _check(lib().msc_mamba3_siso_scan_fwd(ctypes.byref(a), _stream(stream)))
+    return out, final_state, saved_states
+
+
+def msc_mamba3_siso_scan_bwd(x, B, C, alpha, beta, gamma, theta, saved_states, dout, D=None,
+                             z=None, h0=None, workspace=None, want_dh0=True, grads=None,
+                             stream=None):
+    """Mamba-3 SISO backward.  Returns dict dx, dz, dB, dC, dalpha, dbeta, dgamma, dtheta, dD, dh0."""
+    Bsz, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    K = theta.shape[3]
+    dev = x.device
+    f32 = dict(device=dev, dtype=torch.float32)
+    g = dict(grads or {})
+    if "dx" not in g:
+        g["dx"] = torch.empty_like(x)
+    if "dz" not in g:
+        g["dz"] = torch.empty_like(x) if z is not None else None
+    if "dB" not in g:
+        g["dB"] = torch.empty((Bsz, L, G, N), **f32)
+    if "dC" not in g:
+        g["dC"] = torch.empty((Bsz, L, G, N), **f32)
+    if "dalpha" not in g:
+        g["dalpha"] = torch.empty((Bsz, L, H), **f32)
+    if "dbeta" not in g:
+        g["dbeta"] = torch.empty((Bsz, L, H), **f32)
+    if "dgamma" not in g:
+        g["dgamma"] = torch.empty((Bsz, L, H), **f32)
+    if "dtheta" not in g:
+        g["dtheta"] = torch.empty((Bsz, L, H, K), **f32)
+    if "dD" not in g:
+        g["dD"] = torch.empty((H,), **f32)
+    if "dh0" not in g:
+        g["dh0"] = torch.empty((Bsz, H, P, N), **f32) if want_dh0 else None
+    need = msc_mamba3_siso_scan_bwd_workspace_bytes(Bsz, L, H, P, N, G, K)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), device=dev, dtype=torch.uint8)
+    a = M3BwdArgs(ctypes.sizeof(M3BwdArgs), _io(x), Bsz, L, H, P, N, G, K, _ptr(x), _ptr(z),
+                  _ptr(B), _ptr(C), _ptr(alpha), _ptr(beta), _ptr(gamma), _ptr(theta), _ptr(D),
+                  _ptr(h0), _ptr(saved_states), _ptr(dout), _ptr(g["dx"]), _ptr(g["dz"]),
+                  _ptr(g["dB"]), _ptr(g["dC"]), _ptr(g["dalpha"]), _ptr(g["dbeta"]),
+                  _ptr(g["dgamma"]), _ptr(g["dtheta"]), _ptr(g["dD"]), _ptr(g["dh0"]))
+    _check(lib().msc_mamba3_siso_scan_bwd(ctypes.byref(a), _ptr(workspace), workspace.numel(),
+                                          _stream(stream)))
+    return g
