@@ -213,7 +213,7 @@ class M1Step:
         f32 = dict(device="cuda", dtype=torch.float32)
         self.out = torch.empty_like(u)
         self.fs = torch.empty((Bsz, D, N), **f32)
-        self.saved = torch.empty((Bsz, D, (L + 255) // 256, N), **f32)
+        self.saved = torch.empty((Bsz, D, (L + msc.MSC_M1_SAVE_INTERVAL - 1) // msc.MSC_M1_SAVE_INTERVAL, N), **f32)
         self.grads = dict(du=torch.empty_like(u), ddelta=torch.empty_like(u), dz=torch.empty_like(u),
                           dA=torch.empty((D, N), **f32), dB=torch.empty((Bsz, G, N, L), **f32),
                           dC=torch.empty((Bsz, G, N, L), **f32), dD=torch.empty((D,), **f32),

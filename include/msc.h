@@ -99,7 +99,7 @@ const char *msc_version(void);
  * MSC_M1_SAVE_INTERVAL steps (the first is h0); the backward pass needs it.
  * N may be 1..64; L >= 1.
  */
-#define MSC_M1_SAVE_INTERVAL 256
+#define MSC_M1_SAVE_INTERVAL 8
 #define MSC_M1_MAX_DSTATE 64
 
 typedef struct {

@@ -166,10 +166,10 @@ msc_status msc_selective_scan_bwd(const msc_ss_bwd_args *a, void *workspace,
   if ((st = check_m1_sizes(fn, a->batch, a->dim, a->dstate, a->seqlen, a->ngroups)) != MSC_OK)
     return st;
   const int64_t B = a->batch, D = a->dim, N = a->dstate, L = a->seqlen, G = a->ngroups;
-  if (G > 1 && (D / G) % msc::kM1BwdBlock != 0)
+  if (G > 1 && (D / G) % msc::m1_bwd_block(N) != 0)
     return fail(MSC_ERR_UNSUPPORTED,
-                "%s: with ngroups > 1 the channels per group (%lld) must be a multiple of %d",
-                fn, (long long)(D / G), msc::kM1BwdBlock);
+                "%s: with ngroups > 1 the channels per group (%lld) must be a multiple of %lld",
+                fn, (long long)(D / G), (long long)msc::m1_bwd_block(N));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (D == 0) return ok();
   REQUIRE_PTR(fn, "A", a->A);
@@ -219,7 +219,7 @@ msc_status msc_selective_scan_bwd(const msc_ss_bwd_args *a, void *workspace,
   p.du = a->du; p.ddelta = a->ddelta; p.dz = a->z ? a->dz : nullptr;
   p.dA = a->dA; p.dB = a->dB; p.dC = a->dC; p.dD = a->dD; p.dbias = a->ddelta_bias;
   p.dh0 = a->dh0;
-  p.n_part = (D + msc::kM1BwdBlock - 1) / msc::kM1BwdBlock;
+  p.n_part = msc::m1_bwd_partials(D, N, G);
   const size_t bc = ((sizeof(float) * (size_t)(p.n_part * B * 2 * N * L)) + 255) / 256 * 256;
   p.ws_bc = static_cast<float *>(workspace);
   p.ws_misc = reinterpret_cast<float *>(static_cast<char *>(workspace) + bc);

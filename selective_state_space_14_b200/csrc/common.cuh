@@ -22,18 +22,77 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// softplus(v) = log(1 + e^v); for v > 20 it equals v to f32 precision.
-__device__ __forceinline__ float softplus(float v) { return v > 20.f ? v : log1pf(expf(v)); }
+// softplus(v) = log(1 + e^v), e = e^v.  For e < 1/4, log(1 + e) is taken from
+// the series of 2 atanh(s), s = e / (2 + e) <= 1/9 (log(1 + e) =
+// log((1 + s) / (1 - s)) = 2 (s + s^3/3 + s^5/5 + ...); the terms kept leave a
+// relative truncation error below s^10/11 < 3e-11), which keeps full relative
+// accuracy for tiny e where log(1 + e) would cancel; otherwise 1 + e >= 1.25
+// and the hardware logarithm is accurate.  For v > 20, softplus(v) = v in f32.
+__device__ __forceinline__ float softplus(float v) {
+  if (v > 20.f) return v;
+  const float e = __expf(v);
+  if (e < 0.25f) {
+    const float s = __fdividef(e, 2.f + e);
+    const float s2 = s * s;
+    float r = fmaf(s2, 1.f / 9.f, 1.f / 7.f);
+    r = fmaf(s2, r, 1.f / 5.f);
+    r = fmaf(s2, r, 1.f / 3.f);
+    r = fmaf(s2, r, 1.f);
+    return 2.f * s * r;
+  }
+  return __logf(1.f + e);
+}
 
-__device__ __forceinline__ float sigmoid(float v) { return 1.f / (1.f + expf(-v)); }
+// sigmoid(v) = 1 / (1 + e^-v), evaluated from e^-|v| so that it stays finite.
+__device__ __forceinline__ float sigmoid(float v) {
+  const float e = __expf(-fabsf(v));
+  const float s = __fdividef(1.f, 1.f + e);
+  return v >= 0.f ? s : e * s;
+}
 
 __device__ __forceinline__ float silu(float v) { return v * sigmoid(v); }
 
 // d/dv silu(v) = s (1 + v (1 - s)), s = sigmoid(v)
 __device__ __forceinline__ float dsilu(float v) {
-  float s = sigmoid(v);
+  const float s = sigmoid(v);
   return s * (1.f + v * (1.f - s));
 }
+
+// ---------------------------------------------------------------------------
+// packed pairs of f32 (PTX add/mul/fma .f32x2, sm_100+): one instruction
+// computes two IEEE round-to-nearest results, bit-identical to two scalar ops
+// ---------------------------------------------------------------------------
+// Operands are packed into 64-bit registers inside the asm (mov.b64 {lo, hi}),
+// so that no value is type-punned through memory.
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float2 splat2(float v) { return make_float2(v, v); }
+__device__ __forceinline__ float2 ex2_2(float2 v) { return make_float2(ex2(v.x), ex2(v.y)); }
 
 // ---------------------------------------------------------------------------
 // element conversion
@@ -140,6 +199,60 @@ __device__ __forceinline__ void store_run(bf16 *p, int64_t t0, int64_t n, bool v
     for (int i = 0; i < K; ++i)
       if (t0 + i < n) p[t0 + i] = __float2bfloat16_rn(v[i]);
   }
+}
+
+// ---------------------------------------------------------------------------
+// scans of the linear-recurrence monoid over the kW lanes of a lane group
+// (kW = 8: four independent 8-lane groups per warp), on packed pairs
+//   (p, h) o (p', h') = (p p', p' h + h')   -- "earlier o later"
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float2 shfl_up2(float2 v, int off, int width) {
+  return make_float2(__shfl_up_sync(0xffffffffu, v.x, off, width),
+                     __shfl_up_sync(0xffffffffu, v.y, off, width));
+}
+__device__ __forceinline__ float2 shfl_down2(float2 v, int off, int width) {
+  return make_float2(__shfl_down_sync(0xffffffffu, v.x, off, width),
+                     __shfl_down_sync(0xffffffffu, v.y, off, width));
+}
+__device__ __forceinline__ float2 shfl2(float2 v, int src, int width) {
+  return make_float2(__shfl_sync(0xffffffffu, v.x, src, width),
+                     __shfl_sync(0xffffffffu, v.y, src, width));
+}
+
+// Exclusive prefix within the group (lane order = time order): (pe, he) is the
+// composition of all earlier lanes of the group, identity for its first lane.
+template <int kW>
+__device__ __forceinline__ void group_scan_fwd2(float2 p, float2 h, int j, float2 &pe, float2 &he) {
+#pragma unroll
+  for (int off = 1; off < kW; off <<= 1) {
+    const float2 pu = shfl_up2(p, off, kW);
+    const float2 hu = shfl_up2(h, off, kW);
+    if (j >= off) {
+      h = fma2(p, hu, h);
+      p = mul2(p, pu);
+    }
+  }
+  pe = shfl_up2(p, 1, kW);
+  he = shfl_up2(h, 1, kW);
+  if (j == 0) { pe = splat2(1.f); he = splat2(0.f); }
+}
+
+// Suffix version for the adjoint: a lane maps the carry entering from its
+// right, mu_in, to p * mu_in + m; (ps, ms) composes all later lanes.
+template <int kW>
+__device__ __forceinline__ void group_scan_rev2(float2 p, float2 m, int j, float2 &ps, float2 &ms) {
+#pragma unroll
+  for (int off = 1; off < kW; off <<= 1) {
+    const float2 pd = shfl_down2(p, off, kW);
+    const float2 md = shfl_down2(m, off, kW);
+    if (j + off < kW) {
+      m = fma2(p, md, m);
+      p = mul2(p, pd);
+    }
+  }
+  ps = shfl_down2(p, 1, kW);
+  ms = shfl_down2(m, 1, kW);
+  if (j == kW - 1) { ps = splat2(1.f); ms = splat2(0.f); }
 }
 
 // ---------------------------------------------------------------------------

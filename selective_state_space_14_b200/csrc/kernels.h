@@ -26,15 +26,20 @@ struct M1Params {
   float *dA, *dB, *dC, *dD, *dbias, *dh0;
   float *ws_bc;    // [n_part][B][2][N][L] partial sums of dB, dC
   float *ws_misc;  // [B][D][N + 2]: per-(b, c) dA row, dD, dbias
-  int64_t n_part;  // partials per batch row (channel blocks of kM1BwdBlock)
+  int64_t n_part;  // dB/dC partials per batch row (one per cluster of CTAs)
 };
 
 constexpr int MSC_MAX_N = 64;             // largest Mamba-1 d_state
-constexpr int kM1SaveInterval = 256;      // saved-state spacing (time steps)
-constexpr int kM1BwdWarps = 8;            // channels per CTA in the backward
+constexpr int kM1SaveInterval = 8;        // saved-state spacing (time steps)
 constexpr int kM1BwdCluster = 8;          // CTAs per cluster in the backward
-constexpr int kM1BwdBlock = kM1BwdWarps * kM1BwdCluster;  // channels per partial
+// channels summed into one dB/dC partial by a cluster of backward CTAs:
+// 4 warps x (32 lanes / (padded d_state / 2)) channels per CTA, times the cluster
+inline int64_t m1_bwd_block(int64_t N) {
+  const int64_t kn = N <= 16 ? 16 : (N <= 32 ? 32 : 64);
+  return 4 * (32 / (kn / 2)) * kM1BwdCluster;
+}
 
+int64_t m1_bwd_partials(int64_t D, int64_t N, int64_t G);
 cudaError_t launch_m1_fwd(const M1Params &p, cudaStream_t s);
 cudaError_t launch_m1_bwd(const M1Params &p, cudaStream_t s);
 size_t m1_bwd_workspace_bytes(int64_t B, int64_t D, int64_t N, int64_t L, int64_t G);

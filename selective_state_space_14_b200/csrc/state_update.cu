@@ -19,7 +19,7 @@
 namespace msc {
 namespace {
 
-template <typename T, bool kVec4>
+template <typename T>
 __global__ void __launch_bounds__(256) state_update_kernel(const SUParams p) {
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t D = p.D, N = p.N;
@@ -34,26 +34,33 @@ __global__ void __launch_bounds__(256) state_update_kernel(const SUParams p) {
   const T *Cp = static_cast<const T *>(p.Cm) + (b * p.G + g) * N;
   const float *Ap = p.A + c * N;
   float *st = p.state + i * N;
-  if constexpr (kVec4) {
+  if (N % 4 == 0) {
     for (int64_t n = 0; n < N; n += 4) {
-      float4 h = *reinterpret_cast<const float4 *>(st + n);
+      const float4 h4 = *reinterpret_cast<const float4 *>(st + n);
       const float4 A4 = __ldg(reinterpret_cast<const float4 *>(Ap + n));
-      float hv[4] = {h.x, h.y, h.z, h.w};
-      const float Av[4] = {A4.x, A4.y, A4.z, A4.w};
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float a = ex2(d * (Av[k] * kLog2e));
-        hv[k] = fmaf(a, hv[k], dtx * to_f32(Bp[n + k]));
-        y = fmaf(to_f32(Cp[n + k]), hv[k], y);
-      }
-      *reinterpret_cast<float4 *>(st + n) = make_float4(hv[0], hv[1], hv[2], hv[3]);
+      float2 h01 = make_float2(h4.x, h4.y), h23 = make_float2(h4.z, h4.w);
+      const float2 a01 = ex2_2(mul2(splat2(d), mul2(make_float2(A4.x, A4.y), splat2(kLog2e))));
+      const float2 a23 = ex2_2(mul2(splat2(d), mul2(make_float2(A4.z, A4.w), splat2(kLog2e))));
+      h01 = fma2(a01, h01, mul2(splat2(dtx), make_float2(to_f32(Bp[n]), to_f32(Bp[n + 1]))));
+      h23 = fma2(a23, h23, mul2(splat2(dtx), make_float2(to_f32(Bp[n + 2]), to_f32(Bp[n + 3]))));
+      y = fmaf(to_f32(Cp[n]), h01.x, y);
+      y = fmaf(to_f32(Cp[n + 1]), h01.y, y);
+      y = fmaf(to_f32(Cp[n + 2]), h23.x, y);
+      y = fmaf(to_f32(Cp[n + 3]), h23.y, y);
+      *reinterpret_cast<float4 *>(st + n) = make_float4(h01.x, h01.y, h23.x, h23.y);
     }
   } else {
-    for (int64_t n = 0; n < N; ++n) {
-      const float a = ex2(d * (Ap[n] * kLog2e));
-      const float h = fmaf(a, st[n], dtx * to_f32(Bp[n]));
-      st[n] = h;
-      y = fmaf(to_f32(Cp[n]), h, y);
+    for (int64_t n = 0; n < N; n += 2) {
+      const bool two = n + 1 < N;
+      float2 h = make_float2(st[n], two ? st[n + 1] : 0.f);
+      const float2 A2 = mul2(make_float2(Ap[n], two ? Ap[n + 1] : 0.f), splat2(kLog2e));
+      const float2 a = ex2_2(mul2(splat2(d), A2));
+      const float2 Bv = make_float2(to_f32(Bp[n]), two ? to_f32(Bp[n + 1]) : 0.f);
+      const float2 Cv = make_float2(to_f32(Cp[n]), two ? to_f32(Cp[n + 1]) : 0.f);
+      h = fma2(a, h, mul2(splat2(dtx), Bv));
+      y = fmaf(Cv.y, h.y, fmaf(Cv.x, h.x, y));
+      st[n] = h.x;
+      if (two) st[n + 1] = h.y;
     }
   }
   if (p.z) y *= silu(to_f32(static_cast<const T *>(p.z)[i]));
@@ -64,10 +71,7 @@ template <typename T>
 cudaError_t launch_t(const SUParams &p, cudaStream_t s) {
   const int64_t rows = p.B * p.D;
   const unsigned blocks = (unsigned)((rows + 255) / 256);
-  if (p.N % 4 == 0)
-    state_update_kernel<T, true><<<blocks, 256, 0, s>>>(p);
-  else
-    state_update_kernel<T, false><<<blocks, 256, 0, s>>>(p);
+  state_update_kernel<T><<<blocks, 256, 0, s>>>(p);
   return cudaGetLastError();
 }
 

@@ -20,7 +20,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmsc.so")
 
 MSC_F32, MSC_BF16 = 0, 1
-MSC_M1_SAVE_INTERVAL = 256
+MSC_M1_SAVE_INTERVAL = 8
 
 STATUS = {0: "MSC_OK", 1: "MSC_ERR_INVALID_ARG", 2: "MSC_ERR_UNSUPPORTED", 3: "MSC_ERR_ALIGNMENT",
           4: "MSC_ERR_CUDA", 5: "MSC_ERR_WORKSPACE"}

@@ -68,7 +68,7 @@ CASES = [
     (2, 65, 16, 600, 1, "f32", True, True, True, True, True),
     (1, 8, 64, 300, 1, "f32", True, True, True, True, True),
     (1, 7, 5, 513, 1, "f32", False, True, True, False, True),
-    (2, 128, 8, 130, 2, "f32", True, True, True, True, True),
+    (2, 256, 8, 130, 2, "f32", True, True, True, True, True),
     (2, 96, 16, 700, 1, "bf16", True, True, True, True, True),
     (1, 40, 16, 9, 1, "bf16", True, True, True, False, True),
 ]
@@ -97,11 +97,11 @@ def test_determinism(msc):
 def test_resume_is_bit_continuous(msc):
     """A scan over L equals a scan over L1 followed by one over L - L1 started
     from the first one's final state; bit-equal when L1 is a multiple of the
-    forward's 512-step chunk."""
+    forward's 128-step chunk."""
     p = W.m1_problem(1, 12, 16, 1536, io="f32", seed=9, bias=True)
     a = m1_device_args(p)
     full, fs_full, _ = msc.msc_selective_scan_fwd(**a)
-    L1 = 1024
+    L1 = 1024  # a multiple of the 128-step chunk
     part = {k: (v[..., :L1].contiguous() if k in ("u", "delta", "z") else v) for k, v in a.items()}
     part["B"], part["C"] = a["B"][..., :L1].contiguous(), a["C"][..., :L1].contiguous()
     o1, fs1, _ = msc.msc_selective_scan_fwd(**part)
