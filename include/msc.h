@@ -225,7 +225,7 @@ msc_status msc_ssm_state_update(const msc_su_args *args, msc_stream_t stream);
  *          S_{-1} = h0 (or 0)
  *   y_t  = S_t Ct_t + D[h] x[b,t,h,:];  out = y_t * silu(z[b,t,h,:])
  * final_state receives S_{L-1}.
- * Supported: P in {16, 32, 64, 128}, N in {16, 32, 64, 128}; L >= 1.
+ * Supported: P and N each in {16, 32, 64}; L >= 0 (L = 0 copies h0 to final_state).
  */
 typedef struct {
   uint32_t struct_size;

@@ -85,6 +85,19 @@ msc_status check_m1_sizes(const char *fn, int64_t B, int64_t D, int64_t N, int64
 
 }  // namespace
 
+namespace msc {
+// shared with the Mamba-3 entry points (api_m3.cu): one thread-local message
+msc_status api_fail(msc_status st, const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return st;
+}
+msc_status api_ok() { return ok(); }
+msc_status api_cuda(cudaError_t e, const char *what) { return cuda_status(e, what); }
+}  // namespace msc
+
 extern "C" {
 
 const char *msc_last_error(void) { return g_err; }

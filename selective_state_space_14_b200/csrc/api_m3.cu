@@ -1,14 +1,74 @@
 // api_m3.cu -- extern "C" entry points of the Mamba-3 SISO scan (msc.h).
+//
+// Argument checks on the host, then the launch on the caller's stream.  Same
+// conventions as api.cu: status codes, a thread-local message naming the
+// argument, no allocation, no synchronisation.
 #include <cuda_runtime.h>
 
+#include <cstdarg>
 #include <cstdio>
 
 #include "../../include/msc.h"
 #include "kernels.h"
 
+static_assert(MSC_M3_CHUNK == MSC_M3_CHUNK_STEPS, "saved-state interval");
+
+namespace msc {
+msc_status api_fail(msc_status st, const char *fmt, ...);
+msc_status api_ok();
+msc_status api_cuda(cudaError_t e, const char *what);
+}  // namespace msc
+
 namespace {
-thread_local char g_m3_err[256];
+
+using msc::api_cuda;
+using msc::api_fail;
+using msc::api_ok;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+#define M3_REQUIRE(fn, name, ptr)                                                        \
+  do {                                                                                   \
+    if ((ptr) == nullptr) return api_fail(MSC_ERR_INVALID_ARG, "%s: %s is NULL", fn, name); \
+    if (!aligned16(ptr))                                                                 \
+      return api_fail(MSC_ERR_ALIGNMENT, "%s: %s is not 16-byte aligned", fn, name);     \
+  } while (0)
+
+#define M3_OPTIONAL(fn, name, ptr)                                                       \
+  do {                                                                                   \
+    if ((ptr) != nullptr && !aligned16(ptr))                                             \
+      return api_fail(MSC_ERR_ALIGNMENT, "%s: %s is not 16-byte aligned", fn, name);     \
+  } while (0)
+
+template <typename Args>
+msc_status check_m3(const char *fn, const Args *a) {
+  if (!a) return api_fail(MSC_ERR_INVALID_ARG, "%s: args is NULL", fn);
+  if (a->struct_size < sizeof(Args))
+    return api_fail(MSC_ERR_INVALID_ARG, "%s: struct_size %u is smaller than the struct (%zu)",
+                    fn, a->struct_size, sizeof(Args));
+  if (a->io_dtype != MSC_F32 && a->io_dtype != MSC_BF16)
+    return api_fail(MSC_ERR_INVALID_ARG, "%s: io_dtype %d is not MSC_F32 (0) or MSC_BF16 (1)",
+                    fn, (int)a->io_dtype);
+  if (a->batch < 0 || a->seqlen < 0 || a->nheads < 1 || a->ngroups < 1 || a->nangles < 0)
+    return api_fail(MSC_ERR_INVALID_ARG,
+                    "%s: need batch >= 0, seqlen >= 0, nheads >= 1, ngroups >= 1, nangles >= 0",
+                    fn);
+  if (a->nheads % a->ngroups != 0)
+    return api_fail(MSC_ERR_INVALID_ARG, "%s: ngroups %lld does not divide nheads %lld", fn,
+                    (long long)a->ngroups, (long long)a->nheads);
+  if (!msc::m3_supported(a->headdim, a->dstate))
+    return api_fail(MSC_ERR_UNSUPPORTED,
+                    "%s: headdim %lld / dstate %lld not supported (each must be 16, 32 or 64)", fn,
+                    (long long)a->headdim, (long long)a->dstate);
+  if (2 * a->nangles > a->dstate)
+    return api_fail(MSC_ERR_INVALID_ARG, "%s: 2 * nangles (%lld) exceeds dstate (%lld)", fn,
+                    (long long)(2 * a->nangles), (long long)a->dstate);
+  if (a->batch > 65535 || a->nheads > 65535)
+    return api_fail(MSC_ERR_UNSUPPORTED, "%s: batch and nheads must be <= 65535", fn);
+  return MSC_OK;
 }
+
+}  // namespace
 
 extern "C" {
 
@@ -19,17 +79,113 @@ size_t msc_mamba3_siso_saved_states_bytes(int64_t batch, int64_t seqlen, int64_t
   return sizeof(float) * (size_t)(batch * nheads * nc * headdim * dstate);
 }
 
-size_t msc_mamba3_siso_scan_bwd_workspace_bytes(int64_t, int64_t, int64_t, int64_t, int64_t,
-                                                int64_t, int64_t) {
-  return 0;
+msc_status msc_mamba3_siso_scan_fwd(const msc_m3_fwd_args *a, msc_stream_t stream) {
+  const char *fn = "msc_mamba3_siso_scan_fwd";
+  msc_status st = check_m3(fn, a);
+  if (st != MSC_OK) return st;
+  if (a->batch == 0) return api_ok();
+  M3_OPTIONAL(fn, "D", a->D);
+  M3_OPTIONAL(fn, "h0", a->h0);
+  M3_OPTIONAL(fn, "final_state", a->final_state);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t B = a->batch, H = a->nheads, P = a->headdim, N = a->dstate;
+  if (a->seqlen == 0) {
+    if (a->final_state) {
+      const size_t bytes = sizeof(float) * (size_t)(B * H * P * N);
+      return api_cuda(a->h0 ? cudaMemcpyAsync(a->final_state, a->h0, bytes,
+                                              cudaMemcpyDeviceToDevice, s)
+                            : cudaMemsetAsync(a->final_state, 0, bytes, s),
+                      fn);
+    }
+    return api_ok();
+  }
+  M3_REQUIRE(fn, "x", a->x);
+  M3_REQUIRE(fn, "Bm", a->Bm);
+  M3_REQUIRE(fn, "Cm", a->Cm);
+  M3_REQUIRE(fn, "alpha", a->alpha);
+  M3_REQUIRE(fn, "beta", a->beta);
+  M3_REQUIRE(fn, "gamma", a->gamma);
+  if (a->nangles > 0) M3_REQUIRE(fn, "theta", a->theta);
+  M3_REQUIRE(fn, "out", a->out);
+  M3_OPTIONAL(fn, "z", a->z);
+  M3_OPTIONAL(fn, "saved_states", a->saved_states);
+  msc::M3Params p = {};
+  p.io_bf16 = a->io_dtype == MSC_BF16;
+  p.B = B; p.L = a->seqlen; p.H = H; p.P = P; p.N = N; p.G = a->ngroups; p.K = a->nangles;
+  p.x = a->x; p.z = a->z; p.Bm = a->Bm; p.Cm = a->Cm;
+  p.alpha = a->alpha; p.beta = a->beta; p.gamma = a->gamma; p.theta = a->theta;
+  p.Dp = a->D; p.h0 = a->h0; p.out = a->out; p.final_state = a->final_state;
+  p.saved = a->saved_states;
+  return api_cuda(msc::launch_m3_fwd(p, s), fn);
 }
 
-msc_status msc_mamba3_siso_scan_fwd(const msc_m3_fwd_args *, msc_stream_t) {
-  return MSC_ERR_UNSUPPORTED;
+size_t msc_mamba3_siso_scan_bwd_workspace_bytes(int64_t batch, int64_t seqlen, int64_t nheads,
+                                                int64_t headdim, int64_t dstate,
+                                                int64_t ngroups, int64_t nangles) {
+  if (batch <= 0 || seqlen <= 0 || nheads <= 0 || headdim <= 0 || dstate <= 0 || ngroups <= 0)
+    return 0;
+  return msc::m3_bwd_workspace_bytes(batch, seqlen, nheads, headdim, dstate, ngroups, nangles);
 }
 
-msc_status msc_mamba3_siso_scan_bwd(const msc_m3_bwd_args *, void *, size_t, msc_stream_t) {
-  return MSC_ERR_UNSUPPORTED;
+msc_status msc_mamba3_siso_scan_bwd(const msc_m3_bwd_args *a, void *workspace,
+                                    size_t workspace_bytes, msc_stream_t stream) {
+  const char *fn = "msc_mamba3_siso_scan_bwd";
+  msc_status st = check_m3(fn, a);
+  if (st != MSC_OK) return st;
+  const int64_t B = a->batch, L = a->seqlen, H = a->nheads, P = a->headdim, N = a->dstate;
+  const int64_t G = a->ngroups, K = a->nangles;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (B == 0) {
+    if (a->dD) return api_cuda(cudaMemsetAsync(a->dD, 0, sizeof(float) * (size_t)H, s), fn);
+    return api_ok();
+  }
+  M3_OPTIONAL(fn, "dD", a->dD);
+  M3_OPTIONAL(fn, "dh0", a->dh0);
+  if (L == 0) {
+    cudaError_t e = cudaSuccess;
+    if (a->dD) e = cudaMemsetAsync(a->dD, 0, sizeof(float) * (size_t)H, s);
+    if (e == cudaSuccess && a->dh0)
+      e = cudaMemsetAsync(a->dh0, 0, sizeof(float) * (size_t)(B * H * P * N), s);
+    return api_cuda(e, fn);
+  }
+  M3_REQUIRE(fn, "x", a->x);
+  M3_REQUIRE(fn, "Bm", a->Bm);
+  M3_REQUIRE(fn, "Cm", a->Cm);
+  M3_REQUIRE(fn, "alpha", a->alpha);
+  M3_REQUIRE(fn, "beta", a->beta);
+  M3_REQUIRE(fn, "gamma", a->gamma);
+  if (K > 0) {
+    M3_REQUIRE(fn, "theta", a->theta);
+    M3_REQUIRE(fn, "dtheta", a->dtheta);
+  }
+  M3_REQUIRE(fn, "saved_states", a->saved_states);
+  M3_REQUIRE(fn, "dout", a->dout);
+  M3_REQUIRE(fn, "dx", a->dx);
+  M3_REQUIRE(fn, "dB", a->dB);
+  M3_REQUIRE(fn, "dC", a->dC);
+  M3_REQUIRE(fn, "dalpha", a->dalpha);
+  M3_REQUIRE(fn, "dbeta", a->dbeta);
+  M3_REQUIRE(fn, "dgamma", a->dgamma);
+  M3_OPTIONAL(fn, "z", a->z);
+  M3_OPTIONAL(fn, "dz", a->dz);
+  M3_OPTIONAL(fn, "D", a->D);
+  M3_OPTIONAL(fn, "h0", a->h0);
+  const size_t need = msc::m3_bwd_workspace_bytes(B, L, H, P, N, G, K);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need))
+    return api_fail(MSC_ERR_WORKSPACE, "%s: workspace of %zu bytes given, %zu required", fn,
+                    workspace ? workspace_bytes : (size_t)0, need);
+  if (workspace && !aligned16(workspace))
+    return api_fail(MSC_ERR_ALIGNMENT, "%s: workspace is not 16-byte aligned", fn);
+  msc::M3Params p = {};
+  p.io_bf16 = a->io_dtype == MSC_BF16;
+  p.B = B; p.L = L; p.H = H; p.P = P; p.N = N; p.G = G; p.K = K;
+  p.x = a->x; p.z = a->z; p.Bm = a->Bm; p.Cm = a->Cm;
+  p.alpha = a->alpha; p.beta = a->beta; p.gamma = a->gamma; p.theta = a->theta;
+  p.Dp = a->D; p.h0 = a->h0; p.saved_in = a->saved_states; p.dout = a->dout;
+  p.dx = a->dx; p.dz = a->z ? a->dz : nullptr; p.dB = a->dB; p.dC = a->dC;
+  p.dalpha = a->dalpha; p.dbeta = a->dbeta; p.dgamma = a->dgamma; p.dtheta = a->dtheta;
+  p.dD = a->dD; p.dh0 = a->dh0; p.ws = workspace; p.ws_bytes = workspace_bytes;
+  return api_cuda(msc::launch_m3_bwd(p, s), fn);
 }
 
 }  // extern "C"

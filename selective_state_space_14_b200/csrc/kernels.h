@@ -57,14 +57,16 @@ struct SUParams {
 cudaError_t launch_state_update(const SUParams &p, cudaStream_t s);
 
 // ---------------------------------------------------------- Mamba-3 SISO --
+#define MSC_M3_CHUNK_STEPS 64  // steps per chunk (= the saved-state interval)
 struct M3Params {
   int io_bf16;
   int64_t B, L, H, P, N, G, K;
   const void *x, *z, *Bm, *Cm, *alpha, *beta, *gamma, *theta;
   const float *Dp, *h0;
   void *out;
-  float *final_state;
+  float *final_state, *saved;
   // backward
+  const float *saved_in;
   const void *dout;
   void *dx, *dz;
   float *dB, *dC, *dalpha, *dbeta, *dgamma, *dtheta, *dD, *dh0;
