@@ -1,12 +1,509 @@
-// m3_bwd.cu -- Mamba-3 SISO scan, backward (sm_100a).  (in progress)
+// m3_bwd.cu -- Mamba-3 SISO scan, backward (sm_100a): backward stages B2
+// (output gating), B3 (BPTT through the trapezoidal state) and B4 (RoPE) of
+// Mamba3Scratch in mamba-rs 0.4.2 src/mamba3_siso/cpu/scratch.rs.
+//
+// Chunk-local notation as in m3_common.cuh (t, s, tau in [0, Q); g_t the
+// gradient of y_t, i.e. dout_t silu(z_t)).  The state adjoint
+// Lambda_t = dL/dS_t is never formed step by step: with U the adjoint of the
+// first state of the next chunk (its alpha, beta written alpha_Q, beta_Q),
+//   Lambda_t = sum_{tau>=t} d(tau,t) g_tau (outer) Ct_tau + d(Q-1,t) alpha_Q U,
+// and every gradient is a contraction of chunk tiles:
+//   dK_t   = sum_tau c(tau,t) g_tau (outer) Ct_tau + wU_t U,
+//            wU_t = alpha_Q c(Q-1,t) + [t = Q-1] beta_Q
+//   dX     = W^T G + diag(wU) Bt U^T + D G                       (W = c o Ct Bt^T)
+//   dBt    = (c o G X^T)^T Ct + diag(wU) X U
+//   dCt    = diag(d(.,-1)) G S_in + (c o G X^T) Bt + beta_0 diag(d(.,0)) (G x_prev) Bt_prev^T
+//   U_prev = G^T diag(d(.,0)) Ct + d(Q-1,0) alpha_Q U             (adjoint of the chunk's S_0)
+//   dgamma_s = sum_{tau>=s} d(tau,s) (Ct_tau.Bt_s)(g_tau.x_s) + alpha_Q d(Q-1,s) v_s
+//   dbeta_s  = sum_{tau>=s} d(tau,s) (Ct_tau.Bt_{s-1})(g_tau.x_{s-1}) + alpha_Q d(Q-1,s) v_{s-1}
+//     (v_s = x_s^T U Bt_s; index -1 is the previous chunk's last step)
+//   dalpha_r = (1/alpha_r) sum_{t>=r} [rowsum_t(E) - colsum_t(E)],  E(tau,s) = d(tau,s) dL/dd(tau,s)
+// The RoPE backward rotates dBt, dCt back (R^T) per head, forms dphi and
+// the reverse cumulative sum dtheta; the per-head dB, dC go to the workspace
+// and a second kernel adds the heads of each group in ascending order.
+// One CTA per (b, h) walks the chunks from last to first; the chunk-start
+// states come from the forward's saved states, the chunk-start angles from a
+// sequential sum per angle identical to the forward's.
 #include "m3_common.cuh"
 
 namespace msc {
+namespace {
 
-size_t m3_bwd_workspace_bytes(int64_t, int64_t, int64_t, int64_t, int64_t, int64_t, int64_t) {
-  return 0;
+using namespace m3;
+
+template <int P, int N>
+struct BwdSmem {
+  static constexpr int kK = N / 2;
+  static constexpr int kMx = (P > N ? P : N) > kQ ? (P > N ? P : N) : kQ;  // widest row
+  static constexpr int X = 0;                          // [Q][P]
+  static constexpr int Gm = X + kQ * P;                // [Q][P]  g = dout silu(z)
+  static constexpr int Bt = Gm + kQ * P;               // [Q][N]
+  static constexpr int Ct = Bt + kQ * N;               // [Q][N]
+  static constexpr int Sin = Ct + kQ * N;              // [P][N]
+  static constexpr int U = Sin + P * N;                // [P][N]
+  static constexpr int CB = U + P * N;                 // [Q][Q]  Ct Bt^T, later c o G X^T
+  static constexpr int W = CB + kQ * kQ;               // [Q][Q]  c o Ct Bt^T, later dBt [Q][N]
+  static constexpr int T1 = W + kQ * kQ;               // [Q][kMx] Y, dX, dCt
+  static constexpr int T2 = T1 + kQ * kMx;             // [Q][kMx] G X^T, X U
+  static constexpr int T3 = T2 + kQ * kMx;             // [kMx][kMx] G S_in, U_prev
+  static constexpr int Dm = T3 + kMx * kMx;            // [Q][Q+1]
+  static constexpr int Phi = Dm + kQ * (kQ + 1);       // [Q][kK] angles, later dphi
+  static constexpr int vec = Phi + kQ * kK;
+  static constexpr int al = vec, be = al + kQ, ga = be + kQ, d1 = ga + kQ, d0 = d1 + kQ,
+                       crow = d0 + kQ, wu = crow + kQ, cbp = wu + kQ, gxp = cbp + kQ,
+                       vv = gxp + kQ /* v_{-1..Q-1}: Q + 1 */, dgam = vv + kQ + 4,
+                       dbet = dgam + kQ, rowe = dbet + kQ, cole = rowe + kQ, xprev = cole + kQ,
+                       bprev = xprev + P, phist = bprev + N, dth = phist + kK,
+                       red = dth + kK /* kThreads */;
+  static constexpr int total = red + kThreads;
+};
+
+template <typename T, int P, int N>
+__global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, float *ws_phi,
+                                                             float *ws_dB, float *ws_dC,
+                                                             float *ws_dD) {
+  using S = BwdSmem<P, N>;
+  constexpr int kK = S::kK;
+  extern __shared__ float4 smem4[];
+  float *sm = reinterpret_cast<float *>(smem4);
+  float *sX = sm + S::X, *sG = sm + S::Gm, *sBt = sm + S::Bt, *sCt = sm + S::Ct;
+  float *sSin = sm + S::Sin, *sU = sm + S::U, *sCB = sm + S::CB, *sW = sm + S::W;
+  float *sT1 = sm + S::T1, *sT2 = sm + S::T2, *sT3 = sm + S::T3, *sDm = sm + S::Dm;
+  float *sPhi = sm + S::Phi;
+  float *sAl = sm + S::al, *sBe = sm + S::be, *sGa = sm + S::ga, *sD1 = sm + S::d1;
+  float *sD0 = sm + S::d0, *sCrow = sm + S::crow, *sWu = sm + S::wu, *sCbp = sm + S::cbp;
+  float *sGxp = sm + S::gxp, *sV = sm + S::vv + 1 /* sV[-1] valid */, *sDgam = sm + S::dgam;
+  float *sDbet = sm + S::dbet, *sRowE = sm + S::rowe, *sColE = sm + S::cole;
+  float *sXprev = sm + S::xprev, *sBprev = sm + S::bprev, *sPhiSt = sm + S::phist;
+  float *sDth = sm + S::dth, *sRed = sm + S::red;
+
+  const int tid = threadIdx.x;
+  const int64_t h = blockIdx.x, b = blockIdx.y;
+  const int64_t L = p.L, H = p.H, G = p.G, K = p.K;
+  const int64_t g = h / (H / G);
+  const float Dh = p.Dp ? p.Dp[h] : 0.f;
+  const int64_t n_chunks = (L + kQ - 1) / kQ;
+  float *phi_start = ws_phi + (b * H + h) * n_chunks * (K > 0 ? K : 1);
+
+  // chunk-start angles: sum_{s < chunk start} theta_s, accumulated exactly as
+  // the forward does (one f32 sum per angle, in step order)
+  if (tid < K) {
+    float acc = 0.f;
+    for (int64_t t = 0; t < L; ++t) {
+      if (t % kQ == 0) phi_start[(t / kQ) * K + tid] = acc;
+      acc += ldv<T>(p.theta, ((b * L + t) * H + h) * K + tid);
+    }
+  }
+  for (int i = tid; i < P * N; i += kThreads) sU[i] = 0.f;
+  for (int i = tid; i < kK; i += kThreads) sDth[i] = 0.f;
+  float alQ = 1.f, beQ = 0.f;  // alpha, beta of the next chunk's first step
+  float dD_l = 0.f;
+  __syncthreads();  // phi_start is read back by other threads (global, same CTA)
+
+  for (int64_t ch = n_chunks - 1; ch >= 0; --ch) {
+    const int64_t t0 = ch * kQ;
+    const int Qc = (int)((L - t0) < kQ ? (L - t0) : kQ);
+    // ---- A. stage the chunk ---------------------------------------------------
+    for (int i = tid; i < kQ * P; i += kThreads) {
+      const int t = i / P, pp = i % P;
+      float x = 0.f, gv = 0.f;
+      if (t < Qc) {
+        const int64_t j = ((b * L + t0 + t) * H + h) * P + pp;
+        x = ldv<T>(p.x, j);
+        const float dy = ldv<T>(p.dout, j);
+        gv = p.z ? dy * silu(ldv<T>(p.z, j)) : dy;
+      }
+      sX[i] = x;
+      sG[i] = gv;
+      dD_l = fmaf(gv, x, dD_l);
+    }
+    for (int i = tid; i < kQ * N; i += kThreads) {
+      const int t = i / N, n = i % N;
+      const bool in = t < Qc;
+      const int64_t j = ((b * L + t0 + t) * G + g) * N + n;
+      sBt[i] = in ? ldv<T>(p.Bm, j) : 0.f;
+      sCt[i] = in ? ldv<T>(p.Cm, j) : 0.f;
+    }
+    for (int t = tid; t < kQ; t += kThreads) {
+      const bool in = t < Qc;
+      const int64_t j = (b * L + t0 + t) * H + h;
+      sAl[t] = in ? ldv<T>(p.alpha, j) : 1.f;
+      sBe[t] = in ? ldv<T>(p.beta, j) : 0.f;
+      sGa[t] = in ? ldv<T>(p.gamma, j) : 0.f;
+    }
+    for (int i = tid; i < kQ * K; i += kThreads) {
+      const int t = i / (int)K, k = i % (int)K;
+      sPhi[t * kK + k] = t < Qc ? ldv<T>(p.theta, ((b * L + t0 + t) * H + h) * K + k) : 0.f;
+    }
+    for (int i = tid; i < P * N; i += kThreads)
+      sSin[i] = p.saved_in[((b * H + h) * n_chunks + ch) * P * N + i];
+    for (int i = tid; i < kK; i += kThreads) sPhiSt[i] = i < K ? phi_start[ch * K + i] : 0.f;
+    for (int i = tid; i < P; i += kThreads)
+      sXprev[i] = t0 > 0 ? ldv<T>(p.x, ((b * L + t0 - 1) * H + h) * P + i) : 0.f;
+    for (int i = tid; i < N; i += kThreads)
+      sBprev[i] = t0 > 0 ? ldv<T>(p.Bm, ((b * L + t0 - 1) * G + g) * N + i) : 0.f;
+    __syncthreads();
+    // ---- B. angles, decays, rotations -----------------------------------------
+    if (tid < K) {
+      float acc = sPhiSt[tid];
+      for (int t = 0; t < kQ; ++t) {
+        acc += sPhi[t * kK + tid];
+        sPhi[t * kK + tid] = acc;
+      }
+    }
+    for (int col = tid; col <= kQ; col += kThreads) {
+      const int s = col - 1;
+      float v = 1.f;
+      if (s >= 0) sDm[s * (kQ + 1) + col] = 1.f;
+      for (int t = s + 1; t < kQ; ++t) {
+        v *= sAl[t];
+        sDm[t * (kQ + 1) + col] = v;
+      }
+    }
+    __syncthreads();
+    for (int i = tid; i < (kQ + 1) * (N / 2); i += kThreads) {
+      // rows 0..Q-1: the chunk's B and C; row Q: the previous step's B
+      const int t = i / (N / 2), k = i % (N / 2);
+      float *bb = t < kQ ? sBt + t * N : sBprev;
+      const float b0 = bb[2 * k], b1 = bb[2 * k + 1];
+      float c0 = 0.f, c1 = 0.f;
+      if (t < kQ) { c0 = sCt[t * N + 2 * k]; c1 = sCt[t * N + 2 * k + 1]; }
+      if (k < K) {
+        float sn, cs;
+        sincosf(t < kQ ? sPhi[t * kK + k] : sPhiSt[k], &sn, &cs);
+        bb[2 * k] = cs * b0 - sn * b1;
+        bb[2 * k + 1] = sn * b0 + cs * b1;
+        if (t < kQ) {
+          sCt[t * N + 2 * k] = cs * c0 - sn * c1;
+          sCt[t * N + 2 * k + 1] = sn * c0 + cs * c1;
+        }
+      }
+    }
+    __syncthreads();
+    // ---- C. Ct Bt^T, per-step vectors, W ---------------------------------------
+    mm<kQ, kQ, N, false, true>(sCB, kQ, sCt, N, sBt, N, nullptr, nullptr, false);
+    for (int t = tid; t < kQ; t += kThreads) {
+      sD1[t] = sDm[t * (kQ + 1)];
+      sD0[t] = sDm[t * (kQ + 1) + 1];
+      sCrow[t] = (t == kQ - 1) ? sGa[t]
+                               : sDm[(kQ - 1) * (kQ + 1) + t + 2] * (sAl[t + 1] * sGa[t] + sBe[t + 1]);
+      float cb = 0.f, gx = 0.f;
+      for (int n = 0; n < N; ++n) cb = fmaf(sCt[t * N + n], sBprev[n], cb);
+      for (int q = 0; q < P; ++q) gx = fmaf(sG[t * P + q], sXprev[q], gx);
+      sCbp[t] = cb;
+      sGxp[t] = gx;
+    }
+    __syncthreads();
+    for (int t = tid; t < kQ; t += kThreads) sWu[t] = alQ * sCrow[t] + (t == kQ - 1 ? beQ : 0.f);
+    for (int i = tid; i < kQ * kQ; i += kThreads) {
+      const int t = i / kQ, s = i % kQ;
+      float w = 0.f;
+      if (s == t) w = sGa[t] * sCB[i];
+      else if (s < t) w = sDm[t * (kQ + 1) + s + 2] * (sAl[s + 1] * sGa[s] + sBe[s + 1]) * sCB[i];
+      sW[i] = w;
+    }
+    __syncthreads();
+    // ---- D. y (for dz) -----------------------------------------------------------
+    mm<kQ, P, kQ, false, false>(sT1, S::kMx, sW, kQ, sX, P, nullptr, nullptr, false);
+    mm<kQ, P, N, false, true>(sT1, S::kMx, sCt, N, sSin, N, sD1, nullptr, true);
+    __syncthreads();
+    if (p.dz) {
+      for (int i = tid; i < kQ * P; i += kThreads) {
+        const int t = i / P, pp = i % P;
+        if (t < Qc) {
+          const float y = sT1[t * S::kMx + pp] + sBe[0] * sD0[t] * sCbp[t] * sXprev[pp] + Dh * sX[i];
+          const int64_t j = ((b * L + t0 + t) * H + h) * P + pp;
+          const float dy = ldv<T>(p.dout, j);
+          static_cast<T *>(p.dz)[j] = from_f32<T>(y * dy * dsilu(ldv<T>(p.z, j)));
+        }
+      }
+    }
+    // ---- E. G X^T, G S_in; first scalar pass -----------------------------------
+    mm<kQ, kQ, P, false, true>(sT2, S::kMx, sG, P, sX, P, nullptr, nullptr, false);
+    mm<kQ, N, P, false, false>(sT3, S::kMx, sG, P, sSin, N, nullptr, nullptr, false);
+    __syncthreads();
+    for (int s = tid; s < kQ; s += kThreads) {
+      // column s of E, dgamma_s and dbeta_s (chunk-internal parts)
+      float dg = 0.f, db = 0.f;
+      for (int tau = s; tau < kQ; ++tau) {
+        const float d = sDm[tau * (kQ + 1) + s + 1];
+        dg = fmaf(d, sCB[tau * kQ + s] * sT2[tau * S::kMx + s], dg);
+        const float m1 = s > 0 ? sCB[tau * kQ + s - 1] * sT2[tau * S::kMx + s - 1]
+                               : sCbp[tau] * sGxp[tau];
+        db = fmaf(d, m1, db);
+      }
+      sDgam[s] = dg;
+      sDbet[s] = db;
+      sColE[s] = sGa[s] * dg + sBe[s] * db;
+    }
+    for (int tau = tid; tau < kQ; tau += kThreads) {
+      // row tau of E: columns -1..tau
+      float gs = 0.f;
+      for (int n = 0; n < N; ++n) gs = fmaf(sT3[tau * S::kMx + n], sCt[tau * N + n], gs);
+      float r = sDm[tau * (kQ + 1)] * gs;
+      for (int s = 0; s <= tau; ++s) {
+        const float m0 = sCB[tau * kQ + s] * sT2[tau * S::kMx + s];
+        const float m1 = s > 0 ? sCB[tau * kQ + s - 1] * sT2[tau * S::kMx + s - 1]
+                               : sCbp[tau] * sGxp[tau];
+        r = fmaf(sDm[tau * (kQ + 1) + s + 1], fmaf(sGa[s], m0, sBe[s] * m1), r);
+      }
+      sRowE[tau] = r;
+    }
+    __syncthreads();
+    // c o G X^T replaces Ct Bt^T
+    for (int i = tid; i < kQ * kQ; i += kThreads) {
+      const int t = i / kQ, s = i % kQ;
+      float w = 0.f;
+      if (s == t) w = sGa[t] * sT2[t * S::kMx + s];
+      else if (s < t)
+        w = sDm[t * (kQ + 1) + s + 2] * (sAl[s + 1] * sGa[s] + sBe[s + 1]) * sT2[t * S::kMx + s];
+      sCB[i] = w;
+    }
+    __syncthreads();
+    // ---- F. dx; X U; dBt; second scalar pass --------------------------------------
+    mm<kQ, P, kQ, true, false>(sT1, S::kMx, sW, kQ, sG, P, nullptr, nullptr, false);
+    mm<kQ, P, N, false, true>(sT1, S::kMx, sBt, N, sU, N, sWu, nullptr, true);
+    mm<kQ, N, P, false, false>(sT2, S::kMx, sX, P, sU, N, nullptr, nullptr, false);
+    __syncthreads();
+    for (int i = tid; i < kQ * P; i += kThreads) {
+      const int t = i / P, pp = i % P;
+      if (t < Qc)
+        static_cast<T *>(p.dx)[((b * L + t0 + t) * H + h) * P + pp] =
+            from_f32<T>(fmaf(Dh, sG[i], sT1[t * S::kMx + pp]));
+    }
+    mm<kQ, N, kQ, true, false>(sW, N, sCB, kQ, sCt, N, nullptr, nullptr, false);
+    // v_s = x_s^T U Bt_s (s >= 0), v_{-1} with the previous step; <U, S_in>
+    for (int s = tid; s < kQ; s += kThreads) {
+      float v = 0.f;
+      for (int n = 0; n < N; ++n) v = fmaf(sT2[s * S::kMx + n], sBt[s * N + n], v);
+      sV[s] = v;
+    }
+    {
+      float part = 0.f;
+      for (int i = tid; i < P * N; i += kThreads) part = fmaf(sU[i], sSin[i], part);
+      sRed[tid] = part;
+    }
+    __syncthreads();
+    for (int i = tid; i < kQ * N; i += kThreads) {
+      const int t = i / N, n = i % N;
+      sW[i] = fmaf(sWu[t], sT2[t * S::kMx + n], sW[i]);  // dBt
+    }
+    if (tid == 0) {
+      float v = 0.f;
+      for (int n = 0; n < N; ++n) {
+        float xu = 0.f;
+        for (int q = 0; q < P; ++q) xu = fmaf(sXprev[q], sU[q * N + n], xu);
+        v = fmaf(xu, sBprev[n], v);
+      }
+      sV[-1] = v;
+      float us = 0.f;
+      for (int i = 0; i < kThreads; ++i) us += sRed[i];
+      sRed[0] = us;
+    }
+    __syncthreads();
+    for (int s = tid; s < kQ; s += kThreads) {
+      // parts that reach the next chunk through the last state
+      const float dl = sDm[(kQ - 1) * (kQ + 1) + s + 1];
+      const float fg = alQ * dl * sV[s], fb = alQ * dl * sV[s - 1];
+      sDgam[s] += fg;
+      sDbet[s] += fb;
+      sColE[s] += sGa[s] * fg + sBe[s] * fb;
+    }
+    if (tid == 0) {
+      float extra = alQ * sDm[(kQ - 1) * (kQ + 1)] * sRed[0];  // column -1 of row Q-1
+      for (int s = 0; s < kQ; ++s) {
+        const float dl = sDm[(kQ - 1) * (kQ + 1) + s + 1];
+        extra = fmaf(alQ * dl, fmaf(sGa[s], sV[s], sBe[s] * sV[s - 1]), extra);
+      }
+      sRowE[kQ - 1] += extra;
+    }
+    __syncthreads();
+    // ---- G. dCt ---------------------------------------------------------------------
+    mm<kQ, N, kQ, false, false>(sT1, S::kMx, sCB, kQ, sBt, N, nullptr, nullptr, false);
+    __syncthreads();
+    for (int i = tid; i < kQ * N; i += kThreads) {
+      const int t = i / N, n = i % N;
+      float v = sT1[t * S::kMx + n] + sD1[t] * sT3[t * S::kMx + n];
+      v = fmaf(sBe[0] * sD0[t] * sGxp[t], sBprev[n], v);
+      sT1[t * S::kMx + n] = v;
+    }
+    // dalpha, dbeta, dgamma of this chunk
+    if (tid == 0) {
+      float acc = 0.f;
+      for (int r = kQ - 1; r >= 0; --r) {
+        acc += sRowE[r] - sColE[r];
+        if (r < Qc) {
+          const int64_t j = (b * L + t0 + r) * H + h;
+          p.dalpha[j] = acc / sAl[r];
+          p.dbeta[j] = sDbet[r];
+          p.dgamma[j] = sDgam[r];
+        }
+      }
+    }
+    __syncthreads();
+    // ---- H. U_prev = G^T diag(d(.,0)) Ct + d(Q-1,0) alpha_Q U --------------------------
+    mm<P, N, kQ, true, false>(sT3, S::kMx, sG, P, sCt, N, nullptr, sD0, false);
+    // ---- J. RoPE backward: per-head dB, dC and dphi -----------------------------------
+    for (int i = tid; i < kQ * (N / 2); i += kThreads) {
+      const int t = i / (N / 2), k = i % (N / 2);
+      const float db0 = sW[t * N + 2 * k], db1 = sW[t * N + 2 * k + 1];
+      const float dc0 = sT1[t * S::kMx + 2 * k], dc1 = sT1[t * S::kMx + 2 * k + 1];
+      float rb0 = db0, rb1 = db1, rc0 = dc0, rc1 = dc1;
+      if (k < K) {
+        float sn, cs;
+        sincosf(sPhi[t * kK + k], &sn, &cs);
+        rb0 = cs * db0 + sn * db1;
+        rb1 = -sn * db0 + cs * db1;
+        rc0 = cs * dc0 + sn * dc1;
+        rc1 = -sn * dc0 + cs * dc1;
+      }
+      if (t < Qc) {
+        const int64_t j = ((b * L + t0 + t) * H + h) * N + 2 * k;
+        ws_dB[j] = rb0;
+        ws_dB[j + 1] = rb1;
+        ws_dC[j] = rc0;
+        ws_dC[j + 1] = rc1;
+      }
+    }
+    __syncthreads();
+    for (int i = tid; i < kQ * K; i += kThreads) {
+      const int t = i / (int)K, k = i % (int)K;
+      const float b0 = sBt[t * N + 2 * k], b1 = sBt[t * N + 2 * k + 1];
+      const float c0 = sCt[t * N + 2 * k], c1 = sCt[t * N + 2 * k + 1];
+      const float db0 = sW[t * N + 2 * k], db1 = sW[t * N + 2 * k + 1];
+      const float dc0 = sT1[t * S::kMx + 2 * k], dc1 = sT1[t * S::kMx + 2 * k + 1];
+      sPhi[t * kK + k] = (db1 * b0 - db0 * b1) + (dc1 * c0 - dc0 * c1);  // dphi_t[k]
+    }
+    __syncthreads();
+    if (tid < K) {
+      float acc = sDth[tid];
+      for (int t = Qc - 1; t >= 0; --t) {
+        acc += sPhi[t * kK + tid];
+        p.dtheta[((b * L + t0 + t) * H + h) * K + tid] = acc;
+      }
+      sDth[tid] = acc;
+    }
+    // ---- K. hand the adjoint to the previous chunk ----------------------------------
+    {
+      const float c = sD0[kQ - 1] * alQ;
+      for (int i = tid; i < P * N; i += kThreads) {
+        const int pp = i / N, n = i % N;
+        sU[i] = fmaf(c, sU[i], sT3[pp * S::kMx + n]);
+      }
+    }
+    alQ = sAl[0];
+    beQ = sBe[0];
+    __syncthreads();
+  }
+
+  if (p.dh0) {
+    for (int i = tid; i < P * N; i += kThreads)
+      p.dh0[(b * H + h) * P * N + i] = alQ * sU[i];  // alpha_0 Lambda_0
+  }
+  sRed[tid] = dD_l;
+  __syncthreads();
+  if (tid == 0) {
+    float s = 0.f;
+    for (int i = 0; i < kThreads; ++i) s += sRed[i];
+    ws_dD[b * H + h] = s;
+  }
 }
 
-cudaError_t launch_m3_bwd(const M3Params &, cudaStream_t) { return cudaErrorNotSupported; }
+// dB, dC: the heads of each group added in ascending head order; dD: the
+// batch rows added in ascending order.
+__global__ void m3_bwd_reduce_kernel(const M3Params p, const float *ws_dB, const float *ws_dC,
+                                     const float *ws_dD) {
+  const int64_t Bsz = p.B, L = p.L, H = p.H, G = p.G, N = p.N;
+  const int64_t hpg = H / G;
+  const int64_t n_bc = Bsz * L * G * N;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_bc + H;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    if (i < n_bc) {
+      const int64_t n = i % N, g = (i / N) % G, bt = i / (N * G);  // bt = b * L + t
+      float sb = 0.f, sc = 0.f;
+      for (int64_t hh = g * hpg; hh < (g + 1) * hpg; ++hh) {
+        sb += ws_dB[(bt * H + hh) * N + n];
+        sc += ws_dC[(bt * H + hh) * N + n];
+      }
+      p.dB[i] = sb;
+      p.dC[i] = sc;
+    } else if (p.dD) {
+      const int64_t h = i - n_bc;
+      float s = 0.f;
+      for (int64_t b = 0; b < Bsz; ++b) s += ws_dD[b * H + h];
+      p.dD[h] = s;
+    }
+  }
+}
+
+struct WsLayout {
+  size_t phi, dB, dC, dD, total;
+};
+
+WsLayout ws_layout(int64_t B, int64_t L, int64_t H, int64_t N, int64_t K) {
+  auto up = [](size_t v) { return (v + 255) / 256 * 256; };
+  const int64_t nc = (L + kQ - 1) / kQ;
+  WsLayout w;
+  w.phi = 0;
+  w.dB = up(sizeof(float) * (size_t)(B * H * nc * (K > 0 ? K : 1)));
+  w.dC = w.dB + up(sizeof(float) * (size_t)(B * L * H * N));
+  w.dD = w.dC + up(sizeof(float) * (size_t)(B * L * H * N));
+  w.total = w.dD + up(sizeof(float) * (size_t)(B * H));
+  return w;
+}
+
+template <typename T, int P, int N>
+cudaError_t launch_t(const M3Params &p, cudaStream_t s) {
+  const size_t smem = sizeof(float) * (size_t)BwdSmem<P, N>::total;
+  cudaError_t e = cudaFuncSetAttribute(m3_bwd_kernel<T, P, N>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const WsLayout w = ws_layout(p.B, p.L, p.H, p.N, p.K);
+  char *ws = static_cast<char *>(p.ws);
+  float *phi = reinterpret_cast<float *>(ws + w.phi);
+  float *dB = reinterpret_cast<float *>(ws + w.dB);
+  float *dC = reinterpret_cast<float *>(ws + w.dC);
+  float *dD = reinterpret_cast<float *>(ws + w.dD);
+  m3_bwd_kernel<T, P, N><<<dim3((unsigned)p.H, (unsigned)p.B), kThreads, smem, s>>>(p, phi, dB,
+                                                                                  dC, dD);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int64_t total = p.B * p.L * p.G * p.N + p.H;
+  int64_t blocks = (total + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  m3_bwd_reduce_kernel<<<(unsigned)blocks, 256, 0, s>>>(p, dB, dC, dD);
+  return cudaGetLastError();
+}
+
+template <typename T, int P>
+cudaError_t launch_n(const M3Params &p, cudaStream_t s) {
+  switch (p.N) {
+    case 16: return launch_t<T, P, 16>(p, s);
+    case 32: return launch_t<T, P, 32>(p, s);
+    default: return launch_t<T, P, 64>(p, s);
+  }
+}
+
+template <typename T>
+cudaError_t launch_p(const M3Params &p, cudaStream_t s) {
+  switch (p.P) {
+    case 16: return launch_n<T, 16>(p, s);
+    case 32: return launch_n<T, 32>(p, s);
+    default: return launch_n<T, 64>(p, s);
+  }
+}
+
+}  // namespace
+
+size_t m3_bwd_workspace_bytes(int64_t B, int64_t L, int64_t H, int64_t P, int64_t N, int64_t G,
+                              int64_t K) {
+  (void)P;
+  (void)G;
+  return ws_layout(B, L, H, N, K).total;
+}
+
+cudaError_t launch_m3_bwd(const M3Params &p, cudaStream_t s) {
+  return p.io_bf16 ? launch_p<bf16>(p, s) : launch_p<float>(p, s);
+}
 
 }  // namespace msc

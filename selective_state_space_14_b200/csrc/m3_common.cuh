@@ -23,13 +23,16 @@ namespace m3 {
 constexpr int kQ = MSC_M3_CHUNK_STEPS;   // steps per chunk
 constexpr int kThreads = 256;
 
-// C[m][n] (+)= rowscale[m] * sum_k kscale[k] * At[k][m] * B[k][n]
-// At is stored k-major ([K][M], row stride lda), B is [K][N] (row stride ldb),
-// C is [M][N] (row stride ldc).  M and N are multiples of 4; each thread owns
-// 4 x 4 outputs.  Executed by all kThreads threads of the CTA; the caller
-// separates it from producers and consumers with block barriers.
-template <int M, int N, int K>
-__device__ __forceinline__ void mm(float *C, int ldc, const float *At, int lda, const float *B,
+// C[m][n] (+)= rowscale[m] * sum_k kscale[k] * A(m, k) * B(k, n), with
+//   A(m, k) = kAT ? A[k * lda + m] : A[m * lda + k]
+//   B(k, n) = kBT ? B[n * ldb + k] : B[k * ldb + n]
+// C is [M][N] with row stride ldc.  M, N, K are multiples of 4; each thread
+// owns a 4 x 4 block of C and walks K four at a time with 16-byte loads.
+// Executed by all kThreads threads of the CTA, each on its own output blocks
+// (the same blocks on every call with the same M, N); callers separate it
+// from producers and consumers of its operands with block barriers.
+template <int M, int N, int K, bool kAT, bool kBT>
+__device__ __forceinline__ void mm(float *C, int ldc, const float *A, int lda, const float *B,
                                    int ldb, const float *rowscale, const float *kscale,
                                    bool accumulate) {
   constexpr int kTiles = (M / 4) * (N / 4);
@@ -41,20 +44,42 @@ __device__ __forceinline__ void mm(float *C, int ldc, const float *At, int lda, 
     for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int jj = 0; jj < 4; ++jj) acc[i][jj] = 0.f;
-#pragma unroll 4
-    for (int k = 0; k < K; ++k) {
-      float4 a = *reinterpret_cast<const float4 *>(At + k * lda + m0);
-      const float4 b = *reinterpret_cast<const float4 *>(B + k * ldb + n0);
-      if (kscale) {
-        const float ks = kscale[k];
-        a.x *= ks; a.y *= ks; a.z *= ks; a.w *= ks;
+#pragma unroll 2
+    for (int k0 = 0; k0 < K; k0 += 4) {
+      float a[4][4], bv[4][4];  // a[m][k], bv[k][n] of this 4 x 4 x 4 step
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const float4 v = kAT ? *reinterpret_cast<const float4 *>(A + (k0 + r) * lda + m0)
+                             : *reinterpret_cast<const float4 *>(A + (m0 + r) * lda + k0);
+        const float e[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          if (kAT) a[q][r] = e[q];
+          else a[r][q] = e[q];
+        }
+        const float4 w = kBT ? *reinterpret_cast<const float4 *>(B + (n0 + r) * ldb + k0)
+                             : *reinterpret_cast<const float4 *>(B + (k0 + r) * ldb + n0);
+        const float f[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          if (kBT) bv[q][r] = f[q];
+          else bv[r][q] = f[q];
+        }
       }
-      const float av[4] = {a.x, a.y, a.z, a.w};
-      const float bv[4] = {b.x, b.y, b.z, b.w};
+      if (kscale) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+        for (int q = 0; q < 4; ++q) {
+          const float ks = kscale[k0 + q];
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj) acc[i][jj] = fmaf(av[i], bv[jj], acc[i][jj]);
+          for (int r = 0; r < 4; ++r) a[r][q] *= ks;
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) acc[i][jj] = fmaf(a[i][q], bv[q][jj], acc[i][jj]);
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i) {

@@ -137,7 +137,7 @@ __global__ void __launch_bounds__(kThreads, 1) m3_fwd_kernel(const M3Params p) {
     }
     __syncthreads();
     // ---- 4. G = Ct Bt^T; per-step vectors --------------------------------------
-    mm<kQ, kQ, N>(sG, kQ, sCtT, kQ, sBtT, kQ, nullptr, nullptr, false);
+    mm<kQ, kQ, N, true, false>(sG, kQ, sCtT, kQ, sBtT, kQ, nullptr, nullptr, false);
     for (int t = tid; t < kQ; t += kThreads) {
       sDlast[t] = sDm[t * (kQ + 1)];                       // d(t, -1)
       float dot = 0.f;
@@ -159,8 +159,8 @@ __global__ void __launch_bounds__(kThreads, 1) m3_fwd_kernel(const M3Params p) {
     }
     __syncthreads();
     // ---- 6. Y = W X + diag(d(., -1)) Ct S_in^T ---------------------------------
-    mm<kQ, P, kQ>(sY, P, sWT, kQ, sX, P, nullptr, nullptr, false);
-    mm<kQ, P, N>(sY, P, sCtT, kQ, sST, P, sDlast, nullptr, true);
+    mm<kQ, P, kQ, true, false>(sY, P, sWT, kQ, sX, P, nullptr, nullptr, false);
+    mm<kQ, P, N, true, false>(sY, P, sCtT, kQ, sST, P, sDlast, nullptr, true);
     __syncthreads();
     // ---- 7. outputs; the state entering this chunk goes to `saved` -------------
     for (int i = tid; i < kQ * P; i += kThreads) {
@@ -190,7 +190,7 @@ __global__ void __launch_bounds__(kThreads, 1) m3_fwd_kernel(const M3Params p) {
       }
     }
     __syncthreads();
-    mm<N, P, kQ>(sST, P, sBt, N, sX, P, nullptr, sCrow, true);
+    mm<N, P, kQ, true, false>(sST, P, sBt, N, sX, P, nullptr, sCrow, true);
     __syncthreads();
     // ---- 9. carry the last step's key and angles into the next chunk ----------
     for (int i = tid; i < P; i += kThreads) sXprev[i] = sX[(Qc - 1) * P + i];

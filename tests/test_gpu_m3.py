@@ -90,3 +90,73 @@ def test_fwd_model_shaped_full_size(msc):
     r = _oracle_fwd(p)
     assert_close("out", g["out"], r["out"], TOL["bf16"])
     assert_close("final_state", g["final_state"], r["final_state"], TOL["bf16"])
+
+
+# ---------------------------------------------------------------------------
+# backward
+# ---------------------------------------------------------------------------
+def _gpu_bwd(msc, p):
+    a = m3_device_args(p)
+    out, fs, saved = msc.msc_mamba3_siso_scan_fwd(**a)
+    g = msc.msc_mamba3_siso_scan_bwd(saved_states=saved, dout=dev(p.dout), **a)
+    torch.cuda.synchronize()
+    return {k: host(v) for k, v in g.items() if v is not None}
+
+
+def _oracle_bwd(p):
+    return oracle.m3_bwd(dout=p.dout.as_f64(), **oracle.m3_problem_args(p))
+
+
+BWD_CASES = [
+    # (B, L, H, P, N, G, K, io, z, D, h0)
+    (1, 1, 1, 16, 16, 1, 8, "f32", True, True, True),
+    (2, 7, 2, 16, 16, 1, 4, "f32", True, True, True),
+    (1, 64, 2, 32, 16, 1, 8, "f32", False, False, False),
+    (1, 65, 3, 16, 32, 3, 16, "f32", True, True, True),
+    (2, 200, 4, 64, 64, 2, 32, "f32", True, True, True),
+    (1, 130, 2, 32, 64, 1, 0, "f32", True, False, True),
+    (2, 300, 4, 64, 64, 1, 32, "bf16", True, True, False),
+]
+
+
+@pytest.mark.parametrize("case", BWD_CASES,
+                         ids=[f"B{c[0]}L{c[1]}H{c[2]}P{c[3]}N{c[4]}G{c[5]}K{c[6]}{c[7]}" for c in BWD_CASES])
+def test_bwd_parity_shapes(msc, case):
+    Bsz, L, H, P, N, G, K, io, z, Dp, h0 = case
+    p = W.m3_problem(Bsz, L, H, P, N, ngroups=G, nangles=K, io=io, seed=91 + L + H, with_z=z,
+                     with_D=Dp, with_h0=h0)
+    g = _gpu_bwd(msc, p)
+    r = _oracle_bwd(p)
+    for k in M3_GRADS:
+        if k not in g:
+            continue
+        if k == "dtheta" and K == 0:
+            continue
+        if k == "dz" and not z:
+            continue
+        if k == "dD" and not Dp:
+            continue
+        assert_close(k, g[k], r[k], TOL[io])
+
+
+def test_bwd_determinism(msc):
+    p = W.m3_problem(2, 150, 3, 64, 64, nangles=32, io="bf16", seed=4, with_h0=True)
+    runs = [_gpu_bwd(msc, p) for _ in range(3)]
+    for r in runs[1:]:
+        for k in runs[0]:
+            np.testing.assert_array_equal(r[k], runs[0][k], err_msg=k)
+
+
+def test_bwd_model_shaped_full_size(msc):
+    """The Mamba-3 SISO workload at full size (bf16, B8 H24 P64 N64 K32 L2048):
+    the GPU runs all of it; the oracle recomputes batch row 0 (all 24 heads, so
+    the group sums of dB and dC are complete) and that row is compared."""
+    p = W.make("m3_bf16_b8_h24_p64_n64_k32_l2048")
+    g = _gpu_bwd(msc, p)
+    T = lambda t: W.Tensor(t.dtype, t.data[:1])
+    p0 = W.M3Problem(1, p.seqlen, p.nheads, p.headdim, p.dstate, p.ngroups, p.nangles, p.io,
+                     T(p.x), T(p.z), T(p.B), T(p.C), T(p.alpha), T(p.beta), T(p.gamma),
+                     T(p.theta), p.D, None, T(p.dout))
+    r = _oracle_bwd(p0)
+    for k in ("dx", "dz", "dB", "dC", "dalpha", "dbeta", "dgamma", "dtheta", "dh0"):
+        assert_close(k, g[k][:1], r[k], TOL["bf16"])
