@@ -211,18 +211,21 @@ def test_state_update_decode_workload_sampled(msc):
         if t % 100 == 99 or t == 999:
             outs.append((t, host(o)[rows_b, rows_c]))
     final = host(st)[rows_b, rows_c]
-    # oracle: each sampled row as its own (batch=1, dim=1) problem
+    # oracle: each sampled row as its own (batch=1, dim=1) problem; the pool's
+    # sampled rows are widened to f64 once
+    pool = [dict(x=s["x"].as_f64()[rows_b, rows_c], delta=s["delta"].as_f64()[rows_b, rows_c],
+                 z=s["z"].as_f64()[rows_b, rows_c], B=s["B"].as_f64()[rows_b],
+                 C=s["C"].as_f64()[rows_b]) for s in q.steps]
+    D64 = q.D.astype(np.float64)[rows_c]
+    bias64 = q.delta_bias.astype(np.float64)[rows_c]
     for t in range(1000):
-        s = q.steps[t % 8]
+        s = pool[t % 8]
         ref_out = np.zeros(64)
         for r in range(64):
-            b, c = rows_b[r], rows_c[r]
             ns, o = oracle.ssm_state_update(
-                st_ref[r:r + 1], s["x"].as_f64()[b:b + 1, c:c + 1],
-                s["delta"].as_f64()[b:b + 1, c:c + 1], A64[r:r + 1],
-                s["B"].as_f64()[b:b + 1], s["C"].as_f64()[b:b + 1],
-                D=q.D.astype(np.float64)[c:c + 1], delta_bias=q.delta_bias.astype(np.float64)[c:c + 1],
-                z=s["z"].as_f64()[b:b + 1, c:c + 1])
+                st_ref[r:r + 1], s["x"][r:r + 1, None], s["delta"][r:r + 1, None], A64[r:r + 1],
+                s["B"][r:r + 1], s["C"][r:r + 1], D=D64[r:r + 1], delta_bias=bias64[r:r + 1],
+                z=s["z"][r:r + 1, None])
             st_ref[r:r + 1] = ns
             ref_out[r] = o[0, 0]
         for (tt, got) in outs:
