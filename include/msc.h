@@ -173,6 +173,26 @@ size_t msc_selective_scan_bwd_workspace_bytes(int64_t batch, int64_t dim, int64_
 msc_status msc_selective_scan_bwd(const msc_ss_bwd_args *args, void *workspace,
                                   size_t workspace_bytes, msc_stream_t stream);
 
+/*
+ * The same backward pass without a workspace argument, for callers that may
+ * not allocate device memory when they run it (a fixed memory budget
+ * reserved up front, a pooled allocator that must not be bypassed, a path
+ * that must not synchronise the device).  This entry point has no
+ * counterpart in the pages; it is an addition of this library.
+ *
+ * The scratch lives in a static device array of MSC_STATIC_SCRATCH_BYTES
+ * inside the library, held on every GPU that loads the library until the
+ * process exits.  Sizes whose msc_selective_scan_bwd_workspace_bytes()
+ * exceeds it are rejected with MSC_ERR_WORKSPACE (nothing launched).  The
+ * first call on a device looks up the array's device address on that device
+ * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * All calls share the array: calls that may overlap on the GPU race on it
+ * and must be serialised by the caller.  Results equal those of
+ * msc_selective_scan_bwd.  Allocates nothing, never synchronises.
+ */
+#define MSC_STATIC_SCRATCH_BYTES (32u << 20)
+msc_status msc_selective_scan_bwd_static(const msc_ss_bwd_args *args, msc_stream_t stream);
+
 /* ======================================================================
  * Single-token state update (decode)
  * ======================================================================

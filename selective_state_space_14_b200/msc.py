@@ -82,7 +82,8 @@ class M3BwdArgs(ctypes.Structure):
 
 EXPORTS = ["msc_last_error", "msc_version", "msc_selective_scan_saved_states_bytes",
            "msc_selective_scan_fwd", "msc_selective_scan_bwd_workspace_bytes",
-           "msc_selective_scan_bwd", "msc_ssm_state_update", "msc_mamba3_siso_saved_states_bytes",
+           "msc_selective_scan_bwd", "msc_selective_scan_bwd_static", "msc_ssm_state_update",
+           "msc_mamba3_siso_saved_states_bytes",
            "msc_mamba3_siso_scan_fwd", "msc_mamba3_siso_scan_bwd_workspace_bytes",
            "msc_mamba3_siso_scan_bwd"]
 
@@ -102,6 +103,7 @@ def lib() -> ctypes.CDLL:
         for name, argt in (("msc_selective_scan_fwd", [ctypes.POINTER(SsFwdArgs), _vp]),
                            ("msc_selective_scan_bwd",
                             [ctypes.POINTER(SsBwdArgs), _vp, ctypes.c_size_t, _vp]),
+                           ("msc_selective_scan_bwd_static", [ctypes.POINTER(SsBwdArgs), _vp]),
                            ("msc_ssm_state_update", [ctypes.POINTER(SuArgs), _vp]),
                            ("msc_mamba3_siso_scan_fwd", [ctypes.POINTER(M3FwdArgs), _vp]),
                            ("msc_mamba3_siso_scan_bwd",
@@ -223,6 +225,40 @@ def msc_selective_scan_bwd(u, delta, A, B, C, saved_states, dout, D=None, delta_
                   _ptr(g["dD"]), _ptr(g["ddelta_bias"]), _ptr(g["dh0"]))
     _check(lib().msc_selective_scan_bwd(ctypes.byref(a), _ptr(workspace), workspace.numel(),
                                         _stream(stream)))
+    return g
+
+
+MSC_STATIC_SCRATCH_BYTES = 32 << 20
+
+
+def msc_selective_scan_bwd_static(u, delta, A, B, C, saved_states, dout, D=None,
+                                  delta_bias=None, z=None, h0=None, delta_softplus=True,
+                                  want_dh0=True, grads=None, stream=None):
+    """Mamba-1 backward with the library's static scratch instead of a workspace
+    (for callers that may not allocate device memory; see msc.h)."""
+    Bsz, Dm, L = u.shape
+    G, N = B.shape[1], B.shape[2]
+    dev = u.device
+    f32 = dict(device=dev, dtype=torch.float32)
+    g = dict(grads or {})
+    for k, shape in (("dA", (Dm, N)), ("dB", (Bsz, G, N, L)), ("dC", (Bsz, G, N, L)),
+                     ("dD", (Dm,)), ("ddelta_bias", (Dm,))):
+        if k not in g:
+            g[k] = torch.empty(shape, **f32)
+    if "du" not in g:
+        g["du"] = torch.empty_like(u)
+    if "ddelta" not in g:
+        g["ddelta"] = torch.empty_like(u)
+    if "dz" not in g:
+        g["dz"] = torch.empty_like(u) if z is not None else None
+    if "dh0" not in g:
+        g["dh0"] = torch.empty((Bsz, Dm, N), **f32) if want_dh0 else None
+    a = SsBwdArgs(ctypes.sizeof(SsBwdArgs), _io(u), Bsz, Dm, N, L, G, int(delta_softplus),
+                  _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(delta_bias),
+                  _ptr(z), _ptr(h0), _ptr(saved_states), _ptr(dout), _ptr(g["du"]),
+                  _ptr(g["ddelta"]), _ptr(g["dz"]), _ptr(g["dA"]), _ptr(g["dB"]), _ptr(g["dC"]),
+                  _ptr(g["dD"]), _ptr(g["ddelta_bias"]), _ptr(g["dh0"]))
+    _check(lib().msc_selective_scan_bwd_static(ctypes.byref(a), _stream(stream)))
     return g
 
 
