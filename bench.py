@@ -144,15 +144,18 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # distributed plumbing (one process per GPU; no data-path collective)
 # ---------------------------------------------------------------------------
-def dist_init(n_gpus):
+def dist_init(n_gpus, backend="nccl"):
+    """Rank, world size and local rank from the launcher's environment; one
+    process group (short timeout) when there is more than one rank."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}: launch one process per GPU")
     if world > 1:
         import datetime
         import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=None)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
     return world, rank, local
 
 
@@ -162,12 +165,12 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(world, value):
+def max_over_ranks(world, value, device="cuda"):
     if world == 1:
         return value
     import torch
     import torch.distributed as dist
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    t = torch.tensor([value], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -261,10 +264,11 @@ def time_steps(step_fns, steps, warmup, world):
 
 def cpu_baseline(budget_s=12.0):
     """The f64 oracle (as it stands) on a bounded sample of the headline workload:
-    batch row 0, the first 96 channels, all 2048 steps, forward + backward."""
+    batch row 0 (all its channels, all steps), forward + backward, repeated for
+    about ``budget_s`` seconds."""
     import oracle
     p = W.make(HEADLINE)
-    nch = 96
+    nch = p.dim
     sub = W.M1Problem(1, nch, p.dstate, p.seqlen, 1, p.io, p.delta_softplus,
                       W.Tensor(p.io, p.u.data[:1, :nch]), W.Tensor(p.io, p.delta.data[:1, :nch]),
                       p.A[:nch], W.Tensor(p.io, p.B.data[:1]), W.Tensor(p.io, p.C.data[:1]),
@@ -274,7 +278,7 @@ def cpu_baseline(budget_s=12.0):
     dout = sub.dout.as_f64()
     threads = oracle.default_threads()
     reps, t_total = 0, 0.0
-    while t_total < budget_s and reps < 50:
+    while t_total < budget_s and reps < 1000:
         t0 = time.perf_counter()
         oracle.m1_fwd(**args, nthreads=threads)
         oracle.m1_bwd(dout=dout, **args, nthreads=threads)
@@ -320,7 +324,7 @@ def run_ours(args):
     from selective_state_space_14_b200 import msc
     msc.lib()
     peaks = load_peaks()
-    p = W.make(HEADLINE)
+    p = W.make(HEADLINE, shard=rank)  # each rank its own batch of the same shape
     st = M1Step(p, msc)
     sampler = ClockSampler(local)
     sampler.start()
@@ -445,6 +449,61 @@ def extra_workloads(msc, args, world, peaks):
 
 
 # ---------------------------------------------------------------------------
+# one phase alone (for profilers): launches only that phase's kernels
+# ---------------------------------------------------------------------------
+def run_only(args):
+    """``--only PHASE``: the named phase of ``--workload`` (default: the headline
+    Mamba-1 workload, or the Mamba-3 one for m3 phases), ``warmup`` untimed and
+    ``steps`` timed launches; prints one JSON line with the per-launch time.  Not
+    a bench line: the setup launches (e.g. the forward whose saved states a
+    backward needs) run before the warm-up."""
+    import torch
+    from selective_state_space_14_b200 import msc
+    msc.lib()
+    phase = args.only
+    if phase.startswith("m1"):
+        p = W.make(args.workload or HEADLINE)
+        st = M1Step(p, msc)
+        st.fwd()
+        fn = st.fwd if phase == "m1_fwd" else st.bwd
+        units = p.token_channels
+    elif phase.startswith("m3"):
+        m3 = W.make(args.workload or "m3_bf16_b8_h24_p64_n64_k32_l2048")
+        a = dict(x=to_dev(m3.x), B=to_dev(m3.B), C=to_dev(m3.C), alpha=to_dev(m3.alpha),
+                 beta=to_dev(m3.beta), gamma=to_dev(m3.gamma), theta=to_dev(m3.theta),
+                 D=to_dev(m3.D), z=to_dev(m3.z), h0=None)
+        dout = to_dev(m3.dout)
+        out, _, saved = msc.msc_mamba3_siso_scan_fwd(**a)
+        ws = torch.empty(max(msc.msc_mamba3_siso_scan_bwd_workspace_bytes(
+            m3.batch, m3.seqlen, m3.nheads, m3.headdim, m3.dstate, m3.ngroups, m3.nangles), 16),
+            device="cuda", dtype=torch.uint8)
+        grads = msc.msc_mamba3_siso_scan_bwd(**a, saved_states=saved, dout=dout, workspace=ws)
+        if phase == "m3_fwd":
+            def fn():
+                msc.msc_mamba3_siso_scan_fwd(**a, out=out, saved_states=saved)
+        else:
+            def fn():
+                msc.msc_mamba3_siso_scan_bwd(**a, saved_states=saved, dout=dout, workspace=ws,
+                                             grads=grads)
+        units = m3.token_channels
+    else:  # decode
+        q = W.make(args.workload or "su_bf16_b256_d5120_n16_x1000")
+        state = torch.from_numpy(q.state0).cuda()
+        A, Dp, bias = to_dev(q.A), to_dev(q.D), to_dev(q.delta_bias)
+        s = {k: to_dev(v) for k, v in q.steps[0].items()}
+        out = torch.empty_like(s["x"])
+
+        def fn():
+            msc.msc_ssm_state_update(state, s["x"], s["delta"], A, s["B"], s["C"], D=Dp,
+                                     delta_bias=bias, z=s["z"], out=out)
+        units = q.batch * q.dim
+    torch.cuda.synchronize()
+    total_ms, (ms,) = time_steps([fn], args.steps, args.warmup, 1)
+    print(json.dumps({"only": phase, "workload": args.workload, "ms_per_launch": round(ms, 5),
+                      "units_per_s": round(units / (ms / 1e3), 1)}), flush=True)
+
+
+# ---------------------------------------------------------------------------
 # reference arm: the f64 CPU oracle
 # ---------------------------------------------------------------------------
 def run_reference(args):
@@ -454,7 +513,7 @@ def run_reference(args):
         return
     import oracle
     p = W.make(HEADLINE)
-    nch = 24
+    nch = 256  # channels of batch row 0 per step: a step is ~50 ms of oracle work
     sub = W.M1Problem(1, nch, p.dstate, p.seqlen, 1, p.io, p.delta_softplus,
                       W.Tensor(p.io, p.u.data[:1, :nch]), W.Tensor(p.io, p.delta.data[:1, :nch]),
                       p.A[:nch], W.Tensor(p.io, p.B.data[:1]), W.Tensor(p.io, p.C.data[:1]),
@@ -494,10 +553,15 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extra", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=["m1_fwd", "m1_bwd", "m3_fwd", "m3_bwd", "decode"],
+                    help="time one phase alone (for profiling); prints no bench line")
+    ap.add_argument("--workload", default=None, help="workload name for --only")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    if args.impl == "reference":
+    if args.only:
+        run_only(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

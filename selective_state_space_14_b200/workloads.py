@@ -258,9 +258,13 @@ WORKLOADS = {
 }
 
 
-def make(name: str):
+def make(name: str, shard: int = 0):
+    """The named workload.  ``shard`` > 0 draws another batch of the same shape
+    and distributions (seed + 1000 * shard): one per rank when ranks process
+    independent batches."""
     w = dict(WORKLOADS[name])
     kind = w.pop("kind")
+    w["seed"] += 1000 * shard
     if kind == "m1":
         return m1_problem(w["batch"], w["dim"], w["dstate"], w["seqlen"], io=w["io"],
                           seed=w["seed"], bias=w["bias"])

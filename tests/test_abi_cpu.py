@@ -1,0 +1,134 @@
+"""The C ABI on the host: the library loads without a GPU, exports every
+function include/msc.h declares, and refuses bad arguments with the documented
+status and a message naming the argument, before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from selective_state_space_14_b200 import msc
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+OK, INVALID, UNSUPPORTED, ALIGNMENT, CUDA, WORKSPACE = 0, 1, 2, 3, 4, 5
+
+
+def _header_functions():
+    text = open(os.path.join(ROOT, "include", "msc.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(msc_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_binding_exports():
+    assert _header_functions() == sorted(msc.EXPORTS)
+
+
+def test_library_exports_every_declared_function():
+    lib = ctypes.CDLL(msc.LIB_PATH)
+    for name in _header_functions():
+        assert hasattr(lib, name), name
+
+
+def test_version_string():
+    assert msc.lib().msc_version().decode().startswith("msc ")
+
+
+def _err():
+    return msc.lib().msc_last_error().decode()
+
+
+def _fwd_args(**kw):
+    a = msc.SsFwdArgs()
+    a.struct_size = ctypes.sizeof(msc.SsFwdArgs)
+    a.io_dtype, a.batch, a.dim, a.dstate, a.seqlen, a.ngroups, a.delta_softplus = (
+        msc.MSC_BF16, 2, 64, 16, 128, 1, 1)
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: the checks fail first
+    for f in ("u", "delta", "A", "Bm", "Cm", "out"):
+        setattr(a, f, fake)
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+def _call_fwd(a):
+    return msc.lib().msc_selective_scan_fwd(ctypes.byref(a) if a is not None else None, None)
+
+
+def test_fwd_rejects_null_args():
+    assert _call_fwd(None) == INVALID and "args is NULL" in _err()
+
+
+def test_fwd_rejects_short_struct():
+    assert _call_fwd(_fwd_args(struct_size=8)) == INVALID and "struct_size" in _err()
+
+
+def test_fwd_rejects_bad_dtype():
+    assert _call_fwd(_fwd_args(io_dtype=7)) == INVALID and "io_dtype" in _err()
+
+
+@pytest.mark.parametrize("field,value,status,word", [
+    ("batch", -1, INVALID, "batch"),
+    ("seqlen", -5, INVALID, "seqlen"),
+    ("dstate", 0, UNSUPPORTED, "dstate"),
+    ("dstate", 65, UNSUPPORTED, "dstate"),
+    ("ngroups", 3, INVALID, "ngroups"),
+    ("delta_softplus", 2, INVALID, "delta_softplus"),
+])
+def test_fwd_rejects_bad_sizes(field, value, status, word):
+    assert _call_fwd(_fwd_args(**{field: value})) == status
+    assert word in _err()
+
+
+def test_fwd_rejects_missing_input():
+    assert _call_fwd(_fwd_args(u=None)) == INVALID and "u" in _err()
+
+
+def test_fwd_rejects_misaligned_pointer():
+    assert _call_fwd(_fwd_args(A=ctypes.c_void_p((1 << 20) + 2))) == ALIGNMENT
+    assert "A" in _err()
+
+
+def test_bwd_rejects_small_workspace():
+    a = msc.SsBwdArgs()
+    a.struct_size = ctypes.sizeof(msc.SsBwdArgs)
+    a.io_dtype, a.batch, a.dim, a.dstate, a.seqlen, a.ngroups, a.delta_softplus = (
+        msc.MSC_F32, 1, 64, 16, 64, 1, 1)
+    fake = ctypes.c_void_p(1 << 20)
+    for f in ("u", "delta", "A", "Bm", "Cm", "saved_states", "dout", "du", "ddelta", "dA",
+              "dB", "dC"):
+        setattr(a, f, fake)
+    need = msc.msc_selective_scan_bwd_workspace_bytes(1, 64, 16, 64, 1)
+    st = msc.lib().msc_selective_scan_bwd(ctypes.byref(a), fake, need - 256, None)
+    assert st == WORKSPACE and "workspace" in _err()
+
+
+def test_m3_rejects_unsupported_headdim():
+    a = msc.M3FwdArgs()
+    a.struct_size = ctypes.sizeof(msc.M3FwdArgs)
+    a.io_dtype, a.batch, a.seqlen, a.nheads, a.headdim, a.dstate, a.ngroups, a.nangles = (
+        msc.MSC_BF16, 1, 64, 2, 24, 64, 1, 8)
+    st = msc.lib().msc_mamba3_siso_scan_fwd(ctypes.byref(a), None)
+    assert st == UNSUPPORTED and "headdim" in _err()
+
+
+def test_m3_rejects_too_many_angles():
+    a = msc.M3FwdArgs()
+    a.struct_size = ctypes.sizeof(msc.M3FwdArgs)
+    a.io_dtype, a.batch, a.seqlen, a.nheads, a.headdim, a.dstate, a.ngroups, a.nangles = (
+        msc.MSC_BF16, 1, 64, 2, 64, 16, 1, 9)
+    st = msc.lib().msc_mamba3_siso_scan_fwd(ctypes.byref(a), None)
+    assert st == INVALID and "nangles" in _err()
+
+
+def test_state_update_rejects_null():
+    assert msc.lib().msc_ssm_state_update(None, None) == INVALID
+
+
+def test_size_functions():
+    # saved states: f32 [B, D, ceil(L / 8), N]
+    assert msc.msc_selective_scan_saved_states_bytes(2, 3, 16, 17) == 4 * 2 * 3 * 3 * 16
+    # M3 saved states: f32 [B, H, ceil(L / 64), P, N]
+    assert int(msc.lib().msc_mamba3_siso_saved_states_bytes(2, 65, 3, 16, 32)) == \
+        4 * 2 * 3 * 2 * 16 * 32
+    assert msc.msc_selective_scan_bwd_workspace_bytes(8, 1536, 16, 2048, 1) <= \
+        msc.MSC_STATIC_SCRATCH_BYTES
