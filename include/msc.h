@@ -190,7 +190,7 @@ msc_status msc_selective_scan_bwd(const msc_ss_bwd_args *args, void *workspace,
  * and must be serialised by the caller.  Results equal those of
  * msc_selective_scan_bwd.  Allocates nothing, never synchronises.
  */
-#define MSC_STATIC_SCRATCH_BYTES (32u << 20)
+#define MSC_STATIC_SCRATCH_BYTES (64u << 20)
 msc_status msc_selective_scan_bwd_static(const msc_ss_bwd_args *args, msc_stream_t stream);
 
 /* ======================================================================

@@ -179,10 +179,6 @@ msc_status msc_selective_scan_bwd(const msc_ss_bwd_args *a, void *workspace,
   if ((st = check_m1_sizes(fn, a->batch, a->dim, a->dstate, a->seqlen, a->ngroups)) != MSC_OK)
     return st;
   const int64_t B = a->batch, D = a->dim, N = a->dstate, L = a->seqlen, G = a->ngroups;
-  if (G > 1 && (D / G) % msc::m1_bwd_block(N) != 0)
-    return fail(MSC_ERR_UNSUPPORTED,
-                "%s: with ngroups > 1 the channels per group (%lld) must be a multiple of %lld",
-                fn, (long long)(D / G), (long long)msc::m1_bwd_block(N));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (D == 0) return ok();
   REQUIRE_PTR(fn, "A", a->A);

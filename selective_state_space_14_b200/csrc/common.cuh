@@ -202,6 +202,24 @@ __device__ __forceinline__ void store_run(bf16 *p, int64_t t0, int64_t n, bool v
 }
 
 // ---------------------------------------------------------------------------
+// asynchronous global -> shared copies (cp.async, 16 bytes; bytes past
+// src_bytes are zero-filled).  Both addresses must be 16-byte aligned.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src, int src_bytes) {
+  const uint32_t d = (uint32_t)__cvta_generic_to_shared(smem_dst);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(d), "l"(gmem_src),
+               "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;\n" ::: "memory");
+}
+template <int kPending>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(kPending) : "memory");
+}
+
+// ---------------------------------------------------------------------------
 // scans of the linear-recurrence monoid over the kW lanes of a lane group
 // (kW = 8: four independent 8-lane groups per warp), on packed pairs
 //   (p, h) o (p', h') = (p p', p' h + h')   -- "earlier o later"

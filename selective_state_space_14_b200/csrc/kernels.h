@@ -32,11 +32,11 @@ struct M1Params {
 constexpr int MSC_MAX_N = 64;             // largest Mamba-1 d_state
 constexpr int kM1SaveInterval = 8;        // saved-state spacing (time steps)
 constexpr int kM1BwdCluster = 8;          // CTAs per cluster in the backward
-// channels summed into one dB/dC partial by a cluster of backward CTAs:
-// 4 warps x (32 lanes / (padded d_state / 2)) channels per CTA, times the cluster
-inline int64_t m1_bwd_block(int64_t N) {
+constexpr int kM1BwdWarps = 3;            // warps per backward CTA
+// channels of one backward CTA: kM1BwdWarps x (32 lanes / (padded d_state / 2))
+inline int64_t m1_bwd_cta_channels(int64_t N) {
   const int64_t kn = N <= 16 ? 16 : (N <= 32 ? 32 : 64);
-  return 4 * (32 / (kn / 2)) * kM1BwdCluster;
+  return kM1BwdWarps * (32 / (kn / 2));
 }
 
 int64_t m1_bwd_partials(int64_t D, int64_t N, int64_t G);

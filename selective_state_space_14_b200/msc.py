@@ -228,7 +228,7 @@ def msc_selective_scan_bwd(u, delta, A, B, C, saved_states, dout, D=None, delta_
     return g
 
 
-MSC_STATIC_SCRATCH_BYTES = 32 << 20
+MSC_STATIC_SCRATCH_BYTES = 64 << 20
 
 
 def msc_selective_scan_bwd_static(u, delta, A, B, C, saved_states, dout, D=None,
