@@ -73,9 +73,12 @@ struct BwdSmem {
   // byte offsets
   static constexpr int stage = 0;                                   // [2][kStageBytes]
   static constexpr int bcf = stage + 2 * kStageBytes;               // [2][kBlk][kP] float4
+  // per (warp channel, step): (d, d, d x, d x) and (g, g), pairs ready for
+  // the packed arithmetic of the state pairs
   static constexpr int tok = bcf + 2 * kBlk * kP * 16;              // [kWarps][kChW][kS] float4
+  static constexpr int tokg = tok + kWarps * kChW * kS * 16;        // [kWarps][kChW][kS] float2
   static constexpr int kTileRow = kP + 1;                           // float4 per (chw, step) row
-  static constexpr int tile = tok + kWarps * kChW * kS * 16;        // [kWarps][kChW][kS][kP+1] float4
+  static constexpr int tile = tokg + kWarps * kChW * kS * 8;        // [kWarps][kChW][kS][kP+1] float4
   static constexpr int rbc = tile + kWarps * kChW * kS * kTileRow * 16;  // [kCh][kS][kP] float4
   static constexpr int kAccRow = kBlk + 1;                          // floats per (tensor, n) row
   static constexpr int acc = rbc + kCh * kS * kP * 16;              // [2][kN][kBlk+1] f32
@@ -103,60 +106,67 @@ __device__ __forceinline__ void issue_stage(const M1Params &p, unsigned char *st
                                             bool vec_sav, int tid) {
   using S = BwdSmem<T, kN>;
   constexpr int kCh = S::kCh;
+  constexpr int kThreads = kWarps * 32;
   constexpr int E = 16 / (int)sizeof(T);  // elements per 16-byte piece
   constexpr int kPieces = kBlk / E;       // pieces per token / B / C run
-  constexpr int kTokU = 4 * kCh * kPieces;
-  constexpr int kBCU = 2 * kN * kPieces;
-  constexpr int kSavU = kCh * kWin * (kN / 4);
-  const int64_t D = p.D, L = p.L, N = p.N;
+  const int64_t L = p.L, N = p.N;
   const int64_t t0 = kb * kBlk;
-  for (int u = tid; u < kTokU + kBCU + kSavU; u += kWarps * 32) {
-    if (u < kTokU + kBCU) {
-      const T *row;
-      int64_t t = t0;
-      T *dst;
-      bool ok;
-      if (u < kTokU) {
-        const int j = u % kPieces, cl = (u / kPieces) % kCh, k = u / (kPieces * kCh);
-        const int64_t c = c_first + cl;
-        const void *src = k == 0 ? p.u : (k == 1 ? p.delta : (k == 2 ? p.z : p.dout));
-        ok = src != nullptr && c < c_end;
-        row = ok ? static_cast<const T *>(src) + (b * D + c) * L : static_cast<const T *>(p.u);
-        t += j * E;
-        dst = reinterpret_cast<T *>(st) + (k * kCh + cl) * kBlk + j * E;
-      } else {
-        const int v = u - kTokU;
-        const int j = v % kPieces, n = (v / kPieces) % kN, k = v / (kPieces * kN);
-        ok = n < N;
-        row = ok ? (k == 0 ? Bg : Cg) + n * L : Bg;
-        t += j * E;
-        dst = reinterpret_cast<T *>(st + S::kTokBytes) + (k * kN + n) * kBlk + j * E;
-      }
-      const int64_t left = L - t;
-      const int valid = !ok || left <= 0 ? 0 : (left >= E ? E : (int)left);
-      if (p.vec) {
-        cp_async16(dst, valid > 0 ? row + t : row, valid * (int)sizeof(T));
-      } else {
-#pragma unroll
-        for (int i = 0; i < E; ++i) dst[i] = i < valid ? row[t + i] : from_f32<T>(0.f);
-      }
+  // token runs: (tensor k, channel cl, piece j)
+#pragma unroll 1
+  for (int u = tid; u < 4 * kCh * kPieces; u += kThreads) {
+    const int j = u % kPieces, r = u / kPieces;
+    const int cl = r % kCh, k = r / kCh;
+    const int64_t c = c_first + cl;
+    const void *src = k == 0 ? p.u : (k == 1 ? p.delta : (k == 2 ? p.z : p.dout));
+    const bool ok = src != nullptr && c < c_end;
+    const T *row = ok ? static_cast<const T *>(src) + (b * p.D + c) * L : static_cast<const T *>(p.u);
+    const int64_t t = t0 + j * E;
+    const int64_t left = L - t;
+    const int valid = !ok || left <= 0 ? 0 : (left >= E ? E : (int)left);
+    T *dst = reinterpret_cast<T *>(st) + r * kBlk + j * E;
+    if (p.vec) {
+      cp_async16(dst, valid > 0 ? row + t : row, valid * (int)sizeof(T));
     } else {
-      const int v = u - kTokU - kBCU;
-      const int j = v % (kN / 4), w = (v / (kN / 4)) % kWin, cl = v / ((kN / 4) * kWin);
-      const int64_t c = c_first + cl;
-      const int64_t chunk = kb * kWin + w;
-      const int64_t n = 4 * j;
-      float *dst = reinterpret_cast<float *>(st + S::kTokBytes + S::kBCBytes) +
-                   (cl * kWin + w) * kN + n;
-      const bool ok = c < c_end && chunk < n_chunks && n < N;
-      const float *src = p.saved_in + ((b * D + (ok ? c : 0)) * n_chunks + (ok ? chunk : 0)) * N;
-      const int valid = ok ? (int)(N - n < 4 ? N - n : 4) : 0;
-      if (vec_sav) {
-        cp_async16(dst, ok ? src + n : p.saved_in, valid * 4);
-      } else {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) dst[i] = i < valid ? src[n + i] : 0.f;
-      }
+      for (int i = 0; i < E; ++i) dst[i] = i < valid ? row[t + i] : from_f32<T>(0.f);
+    }
+  }
+  // B and C rows: (tensor k, state n, piece j)
+#pragma unroll 1
+  for (int u = tid; u < 2 * kN * kPieces; u += kThreads) {
+    const int j = u % kPieces, r = u / kPieces;
+    const int n = r % kN, k = r / kN;
+    const bool ok = n < N;
+    const T *row = ok ? (k == 0 ? Bg : Cg) + n * L : Bg;
+    const int64_t t = t0 + j * E;
+    const int64_t left = L - t;
+    const int valid = !ok || left <= 0 ? 0 : (left >= E ? E : (int)left);
+    T *dst = reinterpret_cast<T *>(st + S::kTokBytes) + r * kBlk + j * E;
+    if (p.vec) {
+      cp_async16(dst, valid > 0 ? row + t : row, valid * (int)sizeof(T));
+    } else {
+#pragma unroll
+      for (int i = 0; i < E; ++i) dst[i] = i < valid ? row[t + i] : from_f32<T>(0.f);
+    }
+  }
+  // saved states: (channel cl, window w, 4 states); a channel's windows are
+  // consecutive in memory, kWin * N floats from chunk kb * kWin on
+#pragma unroll 1
+  for (int u = tid; u < kCh * kWin * (kN / 4); u += kThreads) {
+    const int j = u % (kWin * (kN / 4)), cl = u / (kWin * (kN / 4));
+    const int w = j / (kN / 4);
+    const int64_t n = 4 * (j % (kN / 4));
+    const int64_t c = c_first + cl;
+    const int64_t chunk = kb * kWin + w;
+    float *dst = reinterpret_cast<float *>(st + S::kTokBytes + S::kBCBytes) + (cl * kWin + w) * kN + n;
+    const bool ok = c < c_end && chunk < n_chunks && n < N;
+    const float *src = ok ? p.saved_in + ((b * p.D + c) * n_chunks + chunk) * N + n : p.saved_in;
+    const int valid = ok ? (int)(N - n < 4 ? N - n : 4) : 0;
+    if (vec_sav) {
+      cp_async16(dst, src, valid * 4);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) dst[i] = i < valid ? src[i] : 0.f;
     }
   }
   cp_async_commit();
@@ -204,6 +214,7 @@ __global__ void __launch_bounds__(kWarps * 32, 4) m1_bwd_kernel(const M1Params p
   const int chw = lane / kP;
   const int chl = warp * kChW + chw;
   float4 *const sTok = reinterpret_cast<float4 *>(smem + S::tok) + (warp * kChW + chw) * kS;
+  float2 *const sTokG = reinterpret_cast<float2 *>(smem + S::tokg) + (warp * kChW + chw) * kS;
   float4 *const sTile =
       reinterpret_cast<float4 *>(smem + S::tile) + (warp * kChW + chw) * kS * S::kTileRow;
   const int64_t D = p.D, L = p.L, N = p.N, Bsz = p.B;
@@ -269,6 +280,7 @@ __global__ void __launch_bounds__(kWarps * 32, 4) m1_bwd_kernel(const M1Params p
       float tx = 0.f, tD = 0.f, tdx = 0.f, tsig = 0.f, tdzf = 0.f, tg = 0.f;
       if (pr < kS) {
         float4 tk = make_float4(0.f, 0.f, 0.f, 0.f);
+        float2 tk2 = make_float2(0.f, 0.f);
         const int tb = tw + pr;
         if (active && t_win + pr < L) {
           const float x = ldsm<T>(st, (0 * kCh + chl) * kBlk + tb);
@@ -282,11 +294,13 @@ __global__ void __launch_bounds__(kWarps * 32, 4) m1_bwd_kernel(const M1Params p
             gz = dy * (zv * sz);
             dzf = dy * (sz * fmaf(zv, 1.f - sz, 1.f));
           }
-          tk = make_float4(d, d * x, gz, 0.f);
+          tk = make_float4(d, d, d * x, d * x);
+          tk2 = make_float2(gz, gz);
           tx = x; tD = d; tdx = D_c * x; tg = gz; tdzf = dzf;
           tsig = p.softplus ? sigmoid(v) : 1.f;
         }
         sTok[pr] = tk;
+        sTokG[pr] = tk2;
       }
       __syncwarp();
 
@@ -297,29 +311,31 @@ __global__ void __launch_bounds__(kWarps * 32, 4) m1_bwd_kernel(const M1Params p
         h = make_float2(n0 < N ? sv.x : 0.f, n1 < N ? sv.y : 0.f);
       }
       float2 a[kS], hp[kS];
-      float tdt[kS], tdtx[kS], tgz[kS], yv[kS];
+      float yv[kS];
 #pragma unroll
       for (int t = 0; t < kS; ++t) {
         const float4 tk = sTok[t];
         const float4 bcv = bcf[(tw + t) * kP + pr];
-        tdt[t] = tk.x; tdtx[t] = tk.y; tgz[t] = tk.z;
-        a[t] = ex2_2(mul2(splat2(tk.x), A2));
+        a[t] = ex2_2(mul2(make_float2(tk.x, tk.y), A2));
         hp[t] = h;
-        h = fma2(a[t], h, mul2(splat2(tk.y), make_float2(bcv.x, bcv.y)));
+        h = fma2(a[t], h, mul2(make_float2(tk.z, tk.w), make_float2(bcv.x, bcv.y)));
         yv[t] = fmaf(bcv.w, h.y, bcv.z * h.x);
       }
       // ---- backwards over the window ----------------------------------------
 #pragma unroll
       for (int t = kS - 1; t >= 0; --t) {
         const float4 bcv = bcf[(tw + t) * kP + pr];
+        const float4 tk = sTok[t];
+        const float2 g2 = sTokG[t];
+        const float2 dt2 = make_float2(tk.x, tk.y), dtx2 = make_float2(tk.z, tk.w);
         const float2 Bv = make_float2(bcv.x, bcv.y), Cv = make_float2(bcv.z, bcv.w);
-        const float2 lam = fma2(splat2(tgz[t]), Cv, mu);
+        const float2 lam = fma2(g2, Cv, mu);
         const float2 q = mul2(a[t], hp[t]);
-        const float2 hcur = fma2(splat2(tdtx[t]), Bv, q);
-        const float2 dC = mul2(splat2(tgz[t]), hcur);
-        const float2 dB = mul2(lam, splat2(tdtx[t]));
+        const float2 hcur = fma2(dtx2, Bv, q);
+        const float2 dC = mul2(g2, hcur);
+        const float2 dB = mul2(lam, dtx2);
         const float2 lq = mul2(lam, q);
-        dA = fma2(splat2(tdt[t]), lq, dA);
+        dA = fma2(dt2, lq, dA);
         sTile[t * S::kTileRow + pr] =
             make_float4(yv[t], fmaf(Ap.y, lq.y, Ap.x * lq.x), fmaf(lam.y, Bv.y, lam.x * Bv.x), 0.f);
         sRbc[(chl * kS + t) * kP + pr] = make_float4(dB.x, dB.y, dC.x, dC.y);
@@ -384,7 +400,11 @@ __global__ void __launch_bounds__(kWarps * 32, 4) m1_bwd_kernel(const M1Params p
     if (kb >= 2)
       issue_stage<T, kN>(p, stage0 + (kb & 1) * S::kStageBytes, b, c_first, c_end, Bg, Cg, kb - 2,
                          n_chunks, vec_sav, tid);
-    cluster.sync();  // peers are done reading; the new B/C table is visible
+    // peers are done reading (the values read are consumed before the arrive);
+    // the new B/C table is visible CTA-wide
+    __syncthreads();
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;\n" ::: "memory");
+    asm volatile("barrier.cluster.wait.aligned;\n" ::: "memory");
   }
 
   // per-(b, c) partials: dA (per thread), dD and dbias (the lanes of a channel
