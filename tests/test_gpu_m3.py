@@ -43,6 +43,12 @@ FWD_CASES = [
     (1, 130, 2, 32, 64, 1, 0, "f32", True, False, True),
     (2, 300, 4, 64, 64, 1, 32, "bf16", True, True, False),
     (1, 129, 2, 64, 32, 1, 10, "bf16", True, True, True),
+    (1, 1, 1, 16, 16, 1, 8, "bf16", True, True, True),
+    (2, 7, 2, 16, 32, 1, 4, "bf16", True, True, True),
+    (1, 65, 3, 32, 64, 3, 16, "bf16", False, False, True),
+    (2, 200, 4, 64, 64, 2, 32, "bf16", True, True, True),
+    (1, 130, 2, 32, 16, 1, 0, "bf16", True, False, True),
+    (1, 640, 2, 64, 64, 1, 32, "bf16", True, True, True),
 ]
 
 
