@@ -263,7 +263,10 @@ typedef struct {
 } msc_m3_fwd_args;
 
 /* saved_states holds S at the start of every block of MSC_M3_CHUNK steps,
- * f32 [B, H, ceil(L / MSC_M3_CHUNK), P, N]; this returns its size in bytes. */
+ * f32 [B, H, ceil(L / MSC_M3_CHUNK), P, N], followed by the cumulative angles
+ * phi at the start of every block, f32 [B, H, ceil(L / MSC_M3_CHUNK), N / 2]
+ * (entries k >= K are zero); the backward pass reads both.  This returns its
+ * size in bytes. */
 #define MSC_M3_CHUNK 64
 size_t msc_mamba3_siso_saved_states_bytes(int64_t batch, int64_t seqlen, int64_t nheads,
                                           int64_t headdim, int64_t dstate);

@@ -76,7 +76,8 @@ size_t msc_mamba3_siso_saved_states_bytes(int64_t batch, int64_t seqlen, int64_t
                                           int64_t headdim, int64_t dstate) {
   if (batch <= 0 || seqlen <= 0 || nheads <= 0 || headdim <= 0 || dstate <= 0) return 0;
   const int64_t nc = (seqlen + MSC_M3_CHUNK - 1) / MSC_M3_CHUNK;
-  return sizeof(float) * (size_t)(batch * nheads * nc * headdim * dstate);
+  // chunk-start states, then chunk-start cumulative angles
+  return sizeof(float) * (size_t)(batch * nheads * nc * (headdim * dstate + dstate / 2));
 }
 
 msc_status msc_mamba3_siso_scan_fwd(const msc_m3_fwd_args *a, msc_stream_t stream) {

@@ -24,12 +24,42 @@
 // One CTA per (b, h) walks the chunks from last to first; the chunk-start
 // states come from the forward's saved states, the chunk-start angles from a
 // sequential sum per angle identical to the forward's.
-#include "m3_common.cuh"
+#include <type_traits>
+
+#include "m3_tc.cuh"
 
 namespace msc {
 namespace {
 
 using namespace m3;
+
+// Chunk contractions: tensor cores (split tf32, f32-class products) for bf16
+// io, f32 on the CUDA cores for f32 io.
+template <typename T, int M, int N, int K, bool kAT, bool kBT, bool kSplitA = true,
+          bool kSplitB = true>
+__device__ __forceinline__ void mmx(float *C, int ldc, const float *A, int lda, const float *B,
+                                    int ldb, const float *rowscale, const float *kscale,
+                                    bool accumulate) {
+  if constexpr (std::is_same_v<T, bf16>)
+    mmt<M, N, K, kAT, kBT, kSplitA, kSplitB>(C, ldc, A, lda, B, ldb, rowscale, kscale, accumulate);
+  else
+    mm<M, N, K, kAT, kBT>(C, ldc, A, lda, B, ldb, rowscale, kscale, accumulate);
+}
+
+// Sum over the CTA's kThreads threads in a fixed order (warp butterflies, then
+// the warp sums in warp order); every thread gets the sum.  Contains block
+// barriers: call from uniform control flow.
+__device__ __forceinline__ float block_sum(float v, float *sRed) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  if ((threadIdx.x & 31) == 0) sRed[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float s = 0.f;
+#pragma unroll
+  for (int w = 0; w < kThreads / 32; ++w) s += sRed[w];
+  __syncthreads();
+  return s;
+}
 
 template <int P, int N>
 struct BwdSmem {
@@ -59,9 +89,8 @@ struct BwdSmem {
 };
 
 template <typename T, int P, int N>
-__global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, float *ws_phi,
-                                                             float *ws_dB, float *ws_dC,
-                                                             float *ws_dD) {
+__global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, float *ws_dB,
+                                                             float *ws_dC, float *ws_dD) {
   using S = BwdSmem<P, N>;
   constexpr int kK = S::kK;
   extern __shared__ float4 smem4[];
@@ -83,22 +112,13 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
   const int64_t g = h / (H / G);
   const float Dh = p.Dp ? p.Dp[h] : 0.f;
   const int64_t n_chunks = (L + kQ - 1) / kQ;
-  float *phi_start = ws_phi + (b * H + h) * n_chunks * (K > 0 ? K : 1);
+  // chunk-start angles, as the forward accumulated them (after the states)
+  const float *phi_start = p.saved_in + p.B * H * n_chunks * P * N + (b * H + h) * n_chunks * kK;
 
-  // chunk-start angles: sum_{s < chunk start} theta_s, accumulated exactly as
-  // the forward does (one f32 sum per angle, in step order)
-  if (tid < K) {
-    float acc = 0.f;
-    for (int64_t t = 0; t < L; ++t) {
-      if (t % kQ == 0) phi_start[(t / kQ) * K + tid] = acc;
-      acc += ldv<T>(p.theta, ((b * L + t) * H + h) * K + tid);
-    }
-  }
   for (int i = tid; i < P * N; i += kThreads) sU[i] = 0.f;
   for (int i = tid; i < kK; i += kThreads) sDth[i] = 0.f;
   float alQ = 1.f, beQ = 0.f;  // alpha, beta of the next chunk's first step
   float dD_l = 0.f;
-  __syncthreads();  // phi_start is read back by other threads (global, same CTA)
 
   for (int64_t ch = n_chunks - 1; ch >= 0; --ch) {
     const int64_t t0 = ch * kQ;
@@ -137,7 +157,7 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
     }
     for (int i = tid; i < P * N; i += kThreads)
       sSin[i] = p.saved_in[((b * H + h) * n_chunks + ch) * P * N + i];
-    for (int i = tid; i < kK; i += kThreads) sPhiSt[i] = i < K ? phi_start[ch * K + i] : 0.f;
+    for (int i = tid; i < kK; i += kThreads) sPhiSt[i] = i < K ? phi_start[ch * kK + i] : 0.f;
     for (int i = tid; i < P; i += kThreads)
       sXprev[i] = t0 > 0 ? ldv<T>(p.x, ((b * L + t0 - 1) * H + h) * P + i) : 0.f;
     for (int i = tid; i < N; i += kThreads)
@@ -181,7 +201,7 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
     }
     __syncthreads();
     // ---- C. Ct Bt^T, per-step vectors, W ---------------------------------------
-    mm<kQ, kQ, N, false, true>(sCB, kQ, sCt, N, sBt, N, nullptr, nullptr, false);
+    mmx<T, kQ, kQ, N, false, true>(sCB, kQ, sCt, N, sBt, N, nullptr, nullptr, false);
     for (int t = tid; t < kQ; t += kThreads) {
       sD1[t] = sDm[t * (kQ + 1)];
       sD0[t] = sDm[t * (kQ + 1) + 1];
@@ -204,8 +224,8 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
     }
     __syncthreads();
     // ---- D. y (for dz) -----------------------------------------------------------
-    mm<kQ, P, kQ, false, false>(sT1, S::kMx, sW, kQ, sX, P, nullptr, nullptr, false);
-    mm<kQ, P, N, false, true>(sT1, S::kMx, sCt, N, sSin, N, sD1, nullptr, true);
+    mmx<T, kQ, P, kQ, false, false, true, false>(sT1, S::kMx, sW, kQ, sX, P, nullptr, nullptr, false);
+    mmx<T, kQ, P, N, false, true>(sT1, S::kMx, sCt, N, sSin, N, sD1, nullptr, true);
     __syncthreads();
     if (p.dz) {
       for (int i = tid; i < kQ * P; i += kThreads) {
@@ -219,8 +239,8 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
       }
     }
     // ---- E. G X^T, G S_in; first scalar pass -----------------------------------
-    mm<kQ, kQ, P, false, true>(sT2, S::kMx, sG, P, sX, P, nullptr, nullptr, false);
-    mm<kQ, N, P, false, false>(sT3, S::kMx, sG, P, sSin, N, nullptr, nullptr, false);
+    mmx<T, kQ, kQ, P, false, true, true, false>(sT2, S::kMx, sG, P, sX, P, nullptr, nullptr, false);
+    mmx<T, kQ, N, P, false, false>(sT3, S::kMx, sG, P, sSin, N, nullptr, nullptr, false);
     __syncthreads();
     for (int s = tid; s < kQ; s += kThreads) {
       // column s of E, dgamma_s and dbeta_s (chunk-internal parts)
@@ -261,9 +281,9 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
     }
     __syncthreads();
     // ---- F. dx; X U; dBt; second scalar pass --------------------------------------
-    mm<kQ, P, kQ, true, false>(sT1, S::kMx, sW, kQ, sG, P, nullptr, nullptr, false);
-    mm<kQ, P, N, false, true>(sT1, S::kMx, sBt, N, sU, N, sWu, nullptr, true);
-    mm<kQ, N, P, false, false>(sT2, S::kMx, sX, P, sU, N, nullptr, nullptr, false);
+    mmx<T, kQ, P, kQ, true, false>(sT1, S::kMx, sW, kQ, sG, P, nullptr, nullptr, false);
+    mmx<T, kQ, P, N, false, true>(sT1, S::kMx, sBt, N, sU, N, sWu, nullptr, true);
+    mmx<T, kQ, N, P, false, false, false, true>(sT2, S::kMx, sX, P, sU, N, nullptr, nullptr, false);
     __syncthreads();
     for (int i = tid; i < kQ * P; i += kThreads) {
       const int t = i / P, pp = i % P;
@@ -271,36 +291,35 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
         static_cast<T *>(p.dx)[((b * L + t0 + t) * H + h) * P + pp] =
             from_f32<T>(fmaf(Dh, sG[i], sT1[t * S::kMx + pp]));
     }
-    mm<kQ, N, kQ, true, false>(sW, N, sCB, kQ, sCt, N, nullptr, nullptr, false);
+    mmx<T, kQ, N, kQ, true, false>(sW, N, sCB, kQ, sCt, N, nullptr, nullptr, false);
     // v_s = x_s^T U Bt_s (s >= 0), v_{-1} with the previous step; <U, S_in>
     for (int s = tid; s < kQ; s += kThreads) {
       float v = 0.f;
       for (int n = 0; n < N; ++n) v = fmaf(sT2[s * S::kMx + n], sBt[s * N + n], v);
       sV[s] = v;
     }
+    __syncthreads();
+    // v_{-1} = x_prev^T U Bt_prev and <U, S_in>, as fixed-order block sums
+    float us, vm1;
     {
       float part = 0.f;
       for (int i = tid; i < P * N; i += kThreads) part = fmaf(sU[i], sSin[i], part);
-      sRed[tid] = part;
+      float xb = 0.f;
+      if (tid < N) {
+        float xu = 0.f;
+        for (int q = 0; q < P; ++q) xu = fmaf(sXprev[q], sU[q * N + tid], xu);
+        xb = xu * sBprev[tid];
+      }
+      us = block_sum(part, sRed);
+      vm1 = block_sum(xb, sRed);
     }
-    __syncthreads();
     for (int i = tid; i < kQ * N; i += kThreads) {
       const int t = i / N, n = i % N;
       sW[i] = fmaf(sWu[t], sT2[t * S::kMx + n], sW[i]);  // dBt
     }
-    if (tid == 0) {
-      float v = 0.f;
-      for (int n = 0; n < N; ++n) {
-        float xu = 0.f;
-        for (int q = 0; q < P; ++q) xu = fmaf(sXprev[q], sU[q * N + n], xu);
-        v = fmaf(xu, sBprev[n], v);
-      }
-      sV[-1] = v;
-      float us = 0.f;
-      for (int i = 0; i < kThreads; ++i) us += sRed[i];
-      sRed[0] = us;
-    }
+    if (tid == 0) sV[-1] = vm1;
     __syncthreads();
+    float ex = 0.f;
     for (int s = tid; s < kQ; s += kThreads) {
       // parts that reach the next chunk through the last state
       const float dl = sDm[(kQ - 1) * (kQ + 1) + s + 1];
@@ -308,18 +327,15 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
       sDgam[s] += fg;
       sDbet[s] += fb;
       sColE[s] += sGa[s] * fg + sBe[s] * fb;
+      ex = fmaf(alQ * dl, fmaf(sGa[s], sV[s], sBe[s] * sV[s - 1]), ex);
     }
-    if (tid == 0) {
-      float extra = alQ * sDm[(kQ - 1) * (kQ + 1)] * sRed[0];  // column -1 of row Q-1
-      for (int s = 0; s < kQ; ++s) {
-        const float dl = sDm[(kQ - 1) * (kQ + 1) + s + 1];
-        extra = fmaf(alQ * dl, fmaf(sGa[s], sV[s], sBe[s] * sV[s - 1]), extra);
-      }
-      sRowE[kQ - 1] += extra;
+    {
+      const float extra = block_sum(ex, sRed) + alQ * sDm[(kQ - 1) * (kQ + 1)] * us;
+      if (tid == 0) sRowE[kQ - 1] += extra;  // column -1 and the U terms of row Q-1
     }
     __syncthreads();
     // ---- G. dCt ---------------------------------------------------------------------
-    mm<kQ, N, kQ, false, false>(sT1, S::kMx, sCB, kQ, sBt, N, nullptr, nullptr, false);
+    mmx<T, kQ, N, kQ, false, false>(sT1, S::kMx, sCB, kQ, sBt, N, nullptr, nullptr, false);
     __syncthreads();
     for (int i = tid; i < kQ * N; i += kThreads) {
       const int t = i / N, n = i % N;
@@ -327,22 +343,37 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
       v = fmaf(sBe[0] * sD0[t] * sGxp[t], sBprev[n], v);
       sT1[t * S::kMx + n] = v;
     }
-    // dalpha, dbeta, dgamma of this chunk
-    if (tid == 0) {
-      float acc = 0.f;
-      for (int r = kQ - 1; r >= 0; --r) {
-        acc += sRowE[r] - sColE[r];
-        if (r < Qc) {
-          const int64_t j = (b * L + t0 + r) * H + h;
-          p.dalpha[j] = acc / sAl[r];
-          p.dbeta[j] = sDbet[r];
-          p.dgamma[j] = sDgam[r];
-        }
+    // dalpha, dbeta, dgamma of this chunk: dalpha_r = (1/alpha_r) sum_{t>=r}
+    // (rowE_t - colE_t), a suffix scan over the chunk in warp 0 (lane l: steps
+    // 2l, 2l+1)
+    if (tid < 32) {
+      const int r0 = 2 * tid, r1 = 2 * tid + 1;
+      const float v0 = sRowE[r0] - sColE[r0], v1 = sRowE[r1] - sColE[r1];
+      float incl = v0 + v1;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const float o = __shfl_down_sync(0xffffffffu, incl, off);
+        if (tid + off < 32) incl += o;
+      }
+      float excl = __shfl_down_sync(0xffffffffu, incl, 1);
+      if (tid == 31) excl = 0.f;
+      const float a1 = excl + v1, a0 = a1 + v0;
+      if (r0 < Qc) {
+        const int64_t j = (b * L + t0 + r0) * H + h;
+        p.dalpha[j] = a0 / sAl[r0];
+        p.dbeta[j] = sDbet[r0];
+        p.dgamma[j] = sDgam[r0];
+      }
+      if (r1 < Qc) {
+        const int64_t j = (b * L + t0 + r1) * H + h;
+        p.dalpha[j] = a1 / sAl[r1];
+        p.dbeta[j] = sDbet[r1];
+        p.dgamma[j] = sDgam[r1];
       }
     }
     __syncthreads();
     // ---- H. U_prev = G^T diag(d(.,0)) Ct + d(Q-1,0) alpha_Q U --------------------------
-    mm<P, N, kQ, true, false>(sT3, S::kMx, sG, P, sCt, N, nullptr, sD0, false);
+    mmx<T, P, N, kQ, true, false>(sT3, S::kMx, sG, P, sCt, N, nullptr, sD0, false);
     // ---- J. RoPE backward: per-head dB, dC and dphi -----------------------------------
     for (int i = tid; i < kQ * (N / 2); i += kThreads) {
       const int t = i / (N / 2), k = i % (N / 2);
@@ -400,13 +431,8 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
     for (int i = tid; i < P * N; i += kThreads)
       p.dh0[(b * H + h) * P * N + i] = alQ * sU[i];  // alpha_0 Lambda_0
   }
-  sRed[tid] = dD_l;
-  __syncthreads();
-  if (tid == 0) {
-    float s = 0.f;
-    for (int i = 0; i < kThreads; ++i) s += sRed[i];
-    ws_dD[b * H + h] = s;
-  }
+  const float dD = block_sum(dD_l, sRed);
+  if (tid == 0) ws_dD[b * H + h] = dD;
 }
 
 // dB, dC: the heads of each group added in ascending head order; dD: the
@@ -437,15 +463,13 @@ __global__ void m3_bwd_reduce_kernel(const M3Params p, const float *ws_dB, const
 }
 
 struct WsLayout {
-  size_t phi, dB, dC, dD, total;
+  size_t dB, dC, dD, total;
 };
 
-WsLayout ws_layout(int64_t B, int64_t L, int64_t H, int64_t N, int64_t K) {
+WsLayout ws_layout(int64_t B, int64_t L, int64_t H, int64_t N) {
   auto up = [](size_t v) { return (v + 255) / 256 * 256; };
-  const int64_t nc = (L + kQ - 1) / kQ;
   WsLayout w;
-  w.phi = 0;
-  w.dB = up(sizeof(float) * (size_t)(B * H * nc * (K > 0 ? K : 1)));
+  w.dB = 0;
   w.dC = w.dB + up(sizeof(float) * (size_t)(B * L * H * N));
   w.dD = w.dC + up(sizeof(float) * (size_t)(B * L * H * N));
   w.total = w.dD + up(sizeof(float) * (size_t)(B * H));
@@ -458,14 +482,13 @@ cudaError_t launch_t(const M3Params &p, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(m3_bwd_kernel<T, P, N>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const WsLayout w = ws_layout(p.B, p.L, p.H, p.N, p.K);
+  const WsLayout w = ws_layout(p.B, p.L, p.H, p.N);
   char *ws = static_cast<char *>(p.ws);
-  float *phi = reinterpret_cast<float *>(ws + w.phi);
   float *dB = reinterpret_cast<float *>(ws + w.dB);
   float *dC = reinterpret_cast<float *>(ws + w.dC);
   float *dD = reinterpret_cast<float *>(ws + w.dD);
-  m3_bwd_kernel<T, P, N><<<dim3((unsigned)p.H, (unsigned)p.B), kThreads, smem, s>>>(p, phi, dB,
-                                                                                  dC, dD);
+  m3_bwd_kernel<T, P, N><<<dim3((unsigned)p.H, (unsigned)p.B), kThreads, smem, s>>>(p, dB, dC,
+                                                                                  dD);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int64_t total = p.B * p.L * p.G * p.N + p.H;
@@ -499,7 +522,8 @@ size_t m3_bwd_workspace_bytes(int64_t B, int64_t L, int64_t H, int64_t P, int64_
                               int64_t K) {
   (void)P;
   (void)G;
-  return ws_layout(B, L, H, N, K).total;
+  (void)K;
+  return ws_layout(B, L, H, N).total;
 }
 
 cudaError_t launch_m3_bwd(const M3Params &p, cudaStream_t s) {

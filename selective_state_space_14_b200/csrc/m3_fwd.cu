@@ -178,6 +178,9 @@ __global__ void __launch_bounds__(kThreads, 1) m3_fwd_kernel(const M3Params p) {
         const int pp = i / N, n = i % N;
         dst[i] = sST[n * P + pp];
       }
+      // the cumulative angles at the chunk start, after all states
+      float *ang = p.saved + p.B * H * n_chunks * P * N + ((b * H + h) * n_chunks + ch) * S::kK;
+      for (int i = tid; i < S::kK; i += kThreads) ang[i] = sPhiPrev[i];
     }
     __syncthreads();
     // ---- 8. S_out = d(Q-1,-1) S_in + beta_0 d(Q-1,0) K_prev + X^T diag(c) Bt ----

@@ -289,6 +289,9 @@ __global__ void __launch_bounds__(kThreads, 2) m3_fwd_tc_kernel(const M3Params p
         if ((j & 1) == 0)
           *reinterpret_cast<float2 *>(dst + pp * N + n) = make_float2(s_acc[i][j], s_acc[i][j + 1]);
       });
+      // the cumulative angles at the chunk start, after all states
+      float *ang = p.saved + p.B * H * nc * P * N + ((b * H + h) * nc + ch) * kKmax;
+      if (tid < kKmax) ang[tid] = sPhi0[tid];
     }
     __syncthreads();  // (D) Ct is consumed; the per-step vectors are visible
 

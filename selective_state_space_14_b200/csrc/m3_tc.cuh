@@ -124,3 +124,38 @@ __device__ __forceinline__ void for_acc(F f) {
 
 }  // namespace m3
 }  // namespace msc
+
+namespace msc {
+namespace m3 {
+
+// Drop-in for mm() of m3_common.cuh on the tensor cores:
+//   C[m][n] (+)= rowscale[m] * sum_k kscale[k] * A(m, k) * B(k, n)
+// with the same operand conventions; operands that are exact in tf32 may be
+// declared unsplit.  Executed by all threads of the CTA; callers separate it
+// from producers and consumers of its operands with block barriers.
+template <int M, int N, int K, bool kAT, bool kBT, bool kSplitA = true, bool kSplitB = true>
+__device__ __forceinline__ void mmt(float *C, int ldc, const float *A, int lda, const float *B,
+                                    int ldb, const float *rowscale, const float *kscale,
+                                    bool accumulate) {
+  float acc[TileSplit<M, N>::kPerWarp][4];
+  zero_acc<M, N>(acc);
+  auto fa = [&](int m, int k) {
+    const float v = kAT ? A[k * lda + m] : A[m * lda + k];
+    return kscale ? v * kscale[k] : v;
+  };
+  auto fb = [&](int k, int n) { return kBT ? B[n * ldb + k] : B[k * ldb + n]; };
+  if (kscale) {
+    mma_tiles<M, N, K, true, kSplitB>(acc, fa, fb);
+  } else {
+    mma_tiles<M, N, K, kSplitA, kSplitB>(acc, fa, fb);
+  }
+  for_acc<M, N>([&](int i, int j, int m, int n) {
+    float v = acc[i][j];
+    if (rowscale) v *= rowscale[m];
+    float *dst = C + m * ldc + n;
+    *dst = accumulate ? *dst + v : v;
+  });
+}
+
+}  // namespace m3
+}  // namespace msc

@@ -127,8 +127,8 @@ def test_state_update_rejects_null():
 def test_size_functions():
     # saved states: f32 [B, D, ceil(L / 8), N]
     assert msc.msc_selective_scan_saved_states_bytes(2, 3, 16, 17) == 4 * 2 * 3 * 3 * 16
-    # M3 saved states: f32 [B, H, ceil(L / 64), P, N]
+    # M3 saved states: f32 [B, H, ceil(L / 64), P, N] + angles f32 [B, H, ceil(L / 64), N / 2]
     assert int(msc.lib().msc_mamba3_siso_saved_states_bytes(2, 65, 3, 16, 32)) == \
-        4 * 2 * 3 * 2 * 16 * 32
+        4 * 2 * 3 * 2 * (16 * 32 + 16)
     assert msc.msc_selective_scan_bwd_workspace_bytes(8, 1536, 16, 2048, 1) <= \
         msc.MSC_STATIC_SCRATCH_BYTES
