@@ -46,6 +46,29 @@ __device__ __forceinline__ void mmx(float *C, int ldc, const float *A, int lda, 
     mm<M, N, K, kAT, kBT>(C, ldc, A, lda, B, ldb, rowscale, kscale, accumulate);
 }
 
+// 8 consecutive io elements from global memory at index j (16-byte aligned
+// for bf16), or zeros when !valid
+template <typename T>
+__device__ __forceinline__ void ld8(const void *base, int64_t j, bool valid, float (&v)[8]) {
+  if (!valid) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = 0.f;
+    return;
+  }
+  if constexpr (std::is_same_v<T, bf16>) {
+    const uint4 r = __ldg(reinterpret_cast<const uint4 *>(static_cast<const bf16 *>(base) + j));
+    unpack_bf16x2(r.x, v[0], v[1]);
+    unpack_bf16x2(r.y, v[2], v[3]);
+    unpack_bf16x2(r.z, v[4], v[5]);
+    unpack_bf16x2(r.w, v[6], v[7]);
+  } else {
+    const float4 a = __ldg(reinterpret_cast<const float4 *>(static_cast<const float *>(base) + j));
+    const float4 c = __ldg(reinterpret_cast<const float4 *>(static_cast<const float *>(base) + j + 4));
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = c.x; v[5] = c.y; v[6] = c.z; v[7] = c.w;
+  }
+}
+
 // Sum over the CTA's kThreads threads in a fixed order (warp butterflies, then
 // the warp sums in warp order); every thread gets the sum.  Contains block
 // barriers: call from uniform control flow.
@@ -65,18 +88,21 @@ template <int P, int N>
 struct BwdSmem {
   static constexpr int kK = N / 2;
   static constexpr int kMx = (P > N ? P : N) > kQ ? (P > N ? P : N) : kQ;  // widest row
-  static constexpr int X = 0;                          // [Q][P]
-  static constexpr int Gm = X + kQ * P;                // [Q][P]  g = dout silu(z)
-  static constexpr int Bt = Gm + kQ * P;               // [Q][N]
-  static constexpr int Ct = Bt + kQ * N;               // [Q][N]
-  static constexpr int Sin = Ct + kQ * N;              // [P][N]
-  static constexpr int U = Sin + P * N;                // [P][N]
-  static constexpr int CB = U + P * N;                 // [Q][Q]  Ct Bt^T, later c o G X^T
-  static constexpr int W = CB + kQ * kQ;               // [Q][Q]  c o Ct Bt^T, later dBt [Q][N]
-  static constexpr int T1 = W + kQ * kQ;               // [Q][kMx] Y, dX, dCt
-  static constexpr int T2 = T1 + kQ * kMx;             // [Q][kMx] G X^T, X U
-  static constexpr int T3 = T2 + kQ * kMx;             // [kMx][kMx] G S_in, U_prev
-  static constexpr int Dm = T3 + kMx * kMx;            // [Q][Q+1]
+  // row strides, padded by 4 floats so that the tensor-core fragment loads
+  // (8 rows x 4 columns per instruction) spread over the banks
+  static constexpr int lP = P + 4, lN = N + 4, lQ = kQ + 4, lMx = kMx + 4;
+  static constexpr int X = 0;                          // [Q][lP]
+  static constexpr int Gm = X + kQ * lP;               // [Q][lP]  g = dout silu(z)
+  static constexpr int Bt = Gm + kQ * lP;              // [Q][lN]
+  static constexpr int Ct = Bt + kQ * lN;              // [Q][lN]
+  static constexpr int Sin = Ct + kQ * lN;             // [P][lN]
+  static constexpr int U = Sin + P * lN;               // [P][lN]
+  static constexpr int CB = U + P * lN;                // [Q][lQ]  Ct Bt^T, later c o G X^T
+  static constexpr int W = CB + kQ * lQ;               // [Q][lQ]  c o Ct Bt^T, later dBt [Q][lN]
+  static constexpr int T1 = W + kQ * lQ;               // [Q][lMx] Y, dX, dCt
+  static constexpr int T2 = T1 + kQ * lMx;             // [Q][lMx] G X^T, X U
+  static constexpr int T3 = T2 + kQ * lMx;             // [kMx][lMx] G S_in, U_prev
+  static constexpr int Dm = T3 + kMx * lMx;            // [Q][Q+1]
   static constexpr int Phi = Dm + kQ * (kQ + 1);       // [Q][kK] angles, later dphi
   static constexpr int vec = Phi + kQ * kK;
   static constexpr int al = vec, be = al + kQ, ga = be + kQ, d1 = ga + kQ, d0 = d1 + kQ,
@@ -93,6 +119,7 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
                                                              float *ws_dC, float *ws_dD) {
   using S = BwdSmem<P, N>;
   constexpr int kK = S::kK;
+  constexpr int lP = S::lP, lN = S::lN, lQ = S::lQ, lMx = S::lMx;
   extern __shared__ float4 smem4[];
   float *sm = reinterpret_cast<float *>(smem4);
   float *sX = sm + S::X, *sG = sm + S::Gm, *sBt = sm + S::Bt, *sCt = sm + S::Ct;
@@ -115,7 +142,7 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
   // chunk-start angles, as the forward accumulated them (after the states)
   const float *phi_start = p.saved_in + p.B * H * n_chunks * P * N + (b * H + h) * n_chunks * kK;
 
-  for (int i = tid; i < P * N; i += kThreads) sU[i] = 0.f;
+  for (int i = tid; i < P * lN; i += kThreads) sU[i] = 0.f;
   for (int i = tid; i < kK; i += kThreads) sDth[i] = 0.f;
   float alQ = 1.f, beQ = 0.f;  // alpha, beta of the next chunk's first step
   float dD_l = 0.f;
@@ -124,25 +151,55 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
     const int64_t t0 = ch * kQ;
     const int Qc = (int)((L - t0) < kQ ? (L - t0) : kQ);
     // ---- A. stage the chunk ---------------------------------------------------
-    for (int i = tid; i < kQ * P; i += kThreads) {
-      const int t = i / P, pp = i % P;
-      float x = 0.f, gv = 0.f;
-      if (t < Qc) {
-        const int64_t j = ((b * L + t0 + t) * H + h) * P + pp;
-        x = ldv<T>(p.x, j);
-        const float dy = ldv<T>(p.dout, j);
-        gv = p.z ? dy * silu(ldv<T>(p.z, j)) : dy;
+    // the chunk's starting state by cp.async, straight into its padded rows
+    {
+      const float *src = p.saved_in + ((b * H + h) * n_chunks + ch) * P * N;
+      for (int u = tid; u < P * (N / 4); u += kThreads) {
+        const int r = u / (N / 4), pc = u % (N / 4);
+        cp_async16(sSin + r * lN + pc * 4, src + r * N + pc * 4, 16);
       }
-      sX[i] = x;
-      sG[i] = gv;
-      dD_l = fmaf(gv, x, dD_l);
+      cp_async_commit();
     }
-    for (int i = tid; i < kQ * N; i += kThreads) {
-      const int t = i / N, n = i % N;
+    // x, dout, z: runs of 8 along p, all loads of a thread issued first
+    for (int u0 = tid; u0 < kQ * (P / 8); u0 += 2 * kThreads) {
+      float xv[2][8], dv[2][8], zv[2][8];
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int u = u0 + r * kThreads;
+        const int t = u / (P / 8), pc = u % (P / 8);
+        const bool in = u < kQ * (P / 8) && t < Qc;
+        const int64_t j = ((b * L + t0 + t) * H + h) * P + pc * 8;
+        ld8<T>(p.x, j, in, xv[r]);
+        ld8<T>(p.dout, j, in, dv[r]);
+        ld8<T>(p.z, j, in && p.z, zv[r]);
+      }
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int u = u0 + r * kThreads;
+        if (u >= kQ * (P / 8)) continue;
+        const int t = u / (P / 8), pc = u % (P / 8);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float gv = p.z ? dv[r][e] * silu(zv[r][e]) : dv[r][e];
+          sX[t * lP + pc * 8 + e] = xv[r][e];
+          sG[t * lP + pc * 8 + e] = gv;
+          dD_l = fmaf(gv, xv[r][e], dD_l);
+        }
+      }
+    }
+    // B and C rows: runs of 8 along n
+    for (int u = tid; u < kQ * (N / 8); u += kThreads) {
+      const int t = u / (N / 8), pc = u % (N / 8);
       const bool in = t < Qc;
-      const int64_t j = ((b * L + t0 + t) * G + g) * N + n;
-      sBt[i] = in ? ldv<T>(p.Bm, j) : 0.f;
-      sCt[i] = in ? ldv<T>(p.Cm, j) : 0.f;
+      const int64_t j = ((b * L + t0 + t) * G + g) * N + pc * 8;
+      float bv[8], cv[8];
+      ld8<T>(p.Bm, j, in, bv);
+      ld8<T>(p.Cm, j, in, cv);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        sBt[t * lN + pc * 8 + e] = bv[e];
+        sCt[t * lN + pc * 8 + e] = cv[e];
+      }
     }
     for (int t = tid; t < kQ; t += kThreads) {
       const bool in = t < Qc;
@@ -155,13 +212,31 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
       const int t = i / (int)K, k = i % (int)K;
       sPhi[t * kK + k] = t < Qc ? ldv<T>(p.theta, ((b * L + t0 + t) * H + h) * K + k) : 0.f;
     }
-    for (int i = tid; i < P * N; i += kThreads)
-      sSin[i] = p.saved_in[((b * H + h) * n_chunks + ch) * P * N + i];
     for (int i = tid; i < kK; i += kThreads) sPhiSt[i] = i < K ? phi_start[ch * kK + i] : 0.f;
     for (int i = tid; i < P; i += kThreads)
       sXprev[i] = t0 > 0 ? ldv<T>(p.x, ((b * L + t0 - 1) * H + h) * P + i) : 0.f;
     for (int i = tid; i < N; i += kThreads)
       sBprev[i] = t0 > 0 ? ldv<T>(p.Bm, ((b * L + t0 - 1) * G + g) * N + i) : 0.f;
+    // the previous chunk's rows into L2 while this one computes
+    if (ch > 0) {
+      const int64_t tp = t0 - kQ;
+      for (int u = tid; u < 4 * kQ; u += kThreads) {
+        const int k = u / kQ, t = u % kQ;
+        const void *ptr;
+        if (k < 3) {
+          const void *base = k == 0 ? p.x : (k == 1 ? p.dout : p.z);
+          if (!base) continue;
+          ptr = static_cast<const T *>(base) + ((b * L + tp + t) * H + h) * P;
+        } else {
+          ptr = static_cast<const T *>(p.Bm) + ((b * L + tp + t) * G + g) * N;
+        }
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(ptr));
+      }
+      const float *sv = p.saved_in + ((b * H + h) * n_chunks + ch - 1) * P * N;
+      for (int u = tid; u < P * N / 32; u += kThreads)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(sv + u * 32));
+    }
+    cp_async_wait<0>();
     __syncthreads();
     // ---- B. angles, decays, rotations -----------------------------------------
     if (tid < K) {
@@ -184,32 +259,32 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
     for (int i = tid; i < (kQ + 1) * (N / 2); i += kThreads) {
       // rows 0..Q-1: the chunk's B and C; row Q: the previous step's B
       const int t = i / (N / 2), k = i % (N / 2);
-      float *bb = t < kQ ? sBt + t * N : sBprev;
+      float *bb = t < kQ ? sBt + t * lN : sBprev;
       const float b0 = bb[2 * k], b1 = bb[2 * k + 1];
       float c0 = 0.f, c1 = 0.f;
-      if (t < kQ) { c0 = sCt[t * N + 2 * k]; c1 = sCt[t * N + 2 * k + 1]; }
+      if (t < kQ) { c0 = sCt[t * lN + 2 * k]; c1 = sCt[t * lN + 2 * k + 1]; }
       if (k < K) {
         float sn, cs;
         sincosf(t < kQ ? sPhi[t * kK + k] : sPhiSt[k], &sn, &cs);
         bb[2 * k] = cs * b0 - sn * b1;
         bb[2 * k + 1] = sn * b0 + cs * b1;
         if (t < kQ) {
-          sCt[t * N + 2 * k] = cs * c0 - sn * c1;
-          sCt[t * N + 2 * k + 1] = sn * c0 + cs * c1;
+          sCt[t * lN + 2 * k] = cs * c0 - sn * c1;
+          sCt[t * lN + 2 * k + 1] = sn * c0 + cs * c1;
         }
       }
     }
     __syncthreads();
     // ---- C. Ct Bt^T, per-step vectors, W ---------------------------------------
-    mmx<T, kQ, kQ, N, false, true>(sCB, kQ, sCt, N, sBt, N, nullptr, nullptr, false);
+    mmx<T, kQ, kQ, N, false, true>(sCB, lQ, sCt, lN, sBt, lN, nullptr, nullptr, false);
     for (int t = tid; t < kQ; t += kThreads) {
       sD1[t] = sDm[t * (kQ + 1)];
       sD0[t] = sDm[t * (kQ + 1) + 1];
       sCrow[t] = (t == kQ - 1) ? sGa[t]
                                : sDm[(kQ - 1) * (kQ + 1) + t + 2] * (sAl[t + 1] * sGa[t] + sBe[t + 1]);
       float cb = 0.f, gx = 0.f;
-      for (int n = 0; n < N; ++n) cb = fmaf(sCt[t * N + n], sBprev[n], cb);
-      for (int q = 0; q < P; ++q) gx = fmaf(sG[t * P + q], sXprev[q], gx);
+      for (int n = 0; n < N; ++n) cb = fmaf(sCt[t * lN + n], sBprev[n], cb);
+      for (int q = 0; q < P; ++q) gx = fmaf(sG[t * lP + q], sXprev[q], gx);
       sCbp[t] = cb;
       sGxp[t] = gx;
     }
@@ -218,20 +293,22 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
     for (int i = tid; i < kQ * kQ; i += kThreads) {
       const int t = i / kQ, s = i % kQ;
       float w = 0.f;
-      if (s == t) w = sGa[t] * sCB[i];
-      else if (s < t) w = sDm[t * (kQ + 1) + s + 2] * (sAl[s + 1] * sGa[s] + sBe[s + 1]) * sCB[i];
-      sW[i] = w;
+      if (s == t) w = sGa[t] * sCB[t * lQ + s];
+      else if (s < t)
+        w = sDm[t * (kQ + 1) + s + 2] * (sAl[s + 1] * sGa[s] + sBe[s + 1]) * sCB[t * lQ + s];
+      sW[t * lQ + s] = w;
     }
     __syncthreads();
     // ---- D. y (for dz) -----------------------------------------------------------
-    mmx<T, kQ, P, kQ, false, false, true, false>(sT1, S::kMx, sW, kQ, sX, P, nullptr, nullptr, false);
-    mmx<T, kQ, P, N, false, true>(sT1, S::kMx, sCt, N, sSin, N, sD1, nullptr, true);
+    mmx<T, kQ, P, kQ, false, false, true, false>(sT1, lMx, sW, lQ, sX, lP, nullptr, nullptr, false);
+    mmx<T, kQ, P, N, false, true>(sT1, lMx, sCt, lN, sSin, lN, sD1, nullptr, true);
     __syncthreads();
     if (p.dz) {
       for (int i = tid; i < kQ * P; i += kThreads) {
         const int t = i / P, pp = i % P;
         if (t < Qc) {
-          const float y = sT1[t * S::kMx + pp] + sBe[0] * sD0[t] * sCbp[t] * sXprev[pp] + Dh * sX[i];
+          const float y =
+              sT1[t * lMx + pp] + sBe[0] * sD0[t] * sCbp[t] * sXprev[pp] + Dh * sX[t * lP + pp];
           const int64_t j = ((b * L + t0 + t) * H + h) * P + pp;
           const float dy = ldv<T>(p.dout, j);
           static_cast<T *>(p.dz)[j] = from_f32<T>(y * dy * dsilu(ldv<T>(p.z, j)));
@@ -239,16 +316,16 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
       }
     }
     // ---- E. G X^T, G S_in; first scalar pass -----------------------------------
-    mmx<T, kQ, kQ, P, false, true, true, false>(sT2, S::kMx, sG, P, sX, P, nullptr, nullptr, false);
-    mmx<T, kQ, N, P, false, false>(sT3, S::kMx, sG, P, sSin, N, nullptr, nullptr, false);
+    mmx<T, kQ, kQ, P, false, true, true, false>(sT2, lMx, sG, lP, sX, lP, nullptr, nullptr, false);
+    mmx<T, kQ, N, P, false, false>(sT3, lMx, sG, lP, sSin, lN, nullptr, nullptr, false);
     __syncthreads();
     for (int s = tid; s < kQ; s += kThreads) {
       // column s of E, dgamma_s and dbeta_s (chunk-internal parts)
       float dg = 0.f, db = 0.f;
       for (int tau = s; tau < kQ; ++tau) {
         const float d = sDm[tau * (kQ + 1) + s + 1];
-        dg = fmaf(d, sCB[tau * kQ + s] * sT2[tau * S::kMx + s], dg);
-        const float m1 = s > 0 ? sCB[tau * kQ + s - 1] * sT2[tau * S::kMx + s - 1]
+        dg = fmaf(d, sCB[tau * lQ + s] * sT2[tau * lMx + s], dg);
+        const float m1 = s > 0 ? sCB[tau * lQ + s - 1] * sT2[tau * lMx + s - 1]
                                : sCbp[tau] * sGxp[tau];
         db = fmaf(d, m1, db);
       }
@@ -259,11 +336,11 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
     for (int tau = tid; tau < kQ; tau += kThreads) {
       // row tau of E: columns -1..tau
       float gs = 0.f;
-      for (int n = 0; n < N; ++n) gs = fmaf(sT3[tau * S::kMx + n], sCt[tau * N + n], gs);
+      for (int n = 0; n < N; ++n) gs = fmaf(sT3[tau * lMx + n], sCt[tau * lN + n], gs);
       float r = sDm[tau * (kQ + 1)] * gs;
       for (int s = 0; s <= tau; ++s) {
-        const float m0 = sCB[tau * kQ + s] * sT2[tau * S::kMx + s];
-        const float m1 = s > 0 ? sCB[tau * kQ + s - 1] * sT2[tau * S::kMx + s - 1]
+        const float m0 = sCB[tau * lQ + s] * sT2[tau * lMx + s];
+        const float m1 = s > 0 ? sCB[tau * lQ + s - 1] * sT2[tau * lMx + s - 1]
                                : sCbp[tau] * sGxp[tau];
         r = fmaf(sDm[tau * (kQ + 1) + s + 1], fmaf(sGa[s], m0, sBe[s] * m1), r);
       }
@@ -274,28 +351,28 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
     for (int i = tid; i < kQ * kQ; i += kThreads) {
       const int t = i / kQ, s = i % kQ;
       float w = 0.f;
-      if (s == t) w = sGa[t] * sT2[t * S::kMx + s];
+      if (s == t) w = sGa[t] * sT2[t * lMx + s];
       else if (s < t)
-        w = sDm[t * (kQ + 1) + s + 2] * (sAl[s + 1] * sGa[s] + sBe[s + 1]) * sT2[t * S::kMx + s];
-      sCB[i] = w;
+        w = sDm[t * (kQ + 1) + s + 2] * (sAl[s + 1] * sGa[s] + sBe[s + 1]) * sT2[t * lMx + s];
+      sCB[t * lQ + s] = w;
     }
     __syncthreads();
     // ---- F. dx; X U; dBt; second scalar pass --------------------------------------
-    mmx<T, kQ, P, kQ, true, false>(sT1, S::kMx, sW, kQ, sG, P, nullptr, nullptr, false);
-    mmx<T, kQ, P, N, false, true>(sT1, S::kMx, sBt, N, sU, N, sWu, nullptr, true);
-    mmx<T, kQ, N, P, false, false, false, true>(sT2, S::kMx, sX, P, sU, N, nullptr, nullptr, false);
+    mmx<T, kQ, P, kQ, true, false>(sT1, lMx, sW, lQ, sG, lP, nullptr, nullptr, false);
+    mmx<T, kQ, P, N, false, true>(sT1, lMx, sBt, lN, sU, lN, sWu, nullptr, true);
+    mmx<T, kQ, N, P, false, false, false, true>(sT2, lMx, sX, lP, sU, lN, nullptr, nullptr, false);
     __syncthreads();
     for (int i = tid; i < kQ * P; i += kThreads) {
       const int t = i / P, pp = i % P;
       if (t < Qc)
         static_cast<T *>(p.dx)[((b * L + t0 + t) * H + h) * P + pp] =
-            from_f32<T>(fmaf(Dh, sG[i], sT1[t * S::kMx + pp]));
+            from_f32<T>(fmaf(Dh, sG[t * lP + pp], sT1[t * lMx + pp]));
     }
-    mmx<T, kQ, N, kQ, true, false>(sW, N, sCB, kQ, sCt, N, nullptr, nullptr, false);
+    mmx<T, kQ, N, kQ, true, false>(sW, lN, sCB, lQ, sCt, lN, nullptr, nullptr, false);
     // v_s = x_s^T U Bt_s (s >= 0), v_{-1} with the previous step; <U, S_in>
     for (int s = tid; s < kQ; s += kThreads) {
       float v = 0.f;
-      for (int n = 0; n < N; ++n) v = fmaf(sT2[s * S::kMx + n], sBt[s * N + n], v);
+      for (int n = 0; n < N; ++n) v = fmaf(sT2[s * lMx + n], sBt[s * lN + n], v);
       sV[s] = v;
     }
     __syncthreads();
@@ -303,11 +380,14 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
     float us, vm1;
     {
       float part = 0.f;
-      for (int i = tid; i < P * N; i += kThreads) part = fmaf(sU[i], sSin[i], part);
+      for (int i = tid; i < P * N; i += kThreads) {
+        const int o = (i / N) * lN + i % N;
+        part = fmaf(sU[o], sSin[o], part);
+      }
       float xb = 0.f;
       if (tid < N) {
         float xu = 0.f;
-        for (int q = 0; q < P; ++q) xu = fmaf(sXprev[q], sU[q * N + tid], xu);
+        for (int q = 0; q < P; ++q) xu = fmaf(sXprev[q], sU[q * lN + tid], xu);
         xb = xu * sBprev[tid];
       }
       us = block_sum(part, sRed);
@@ -315,7 +395,7 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
     }
     for (int i = tid; i < kQ * N; i += kThreads) {
       const int t = i / N, n = i % N;
-      sW[i] = fmaf(sWu[t], sT2[t * S::kMx + n], sW[i]);  // dBt
+      sW[t * lN + n] = fmaf(sWu[t], sT2[t * lMx + n], sW[t * lN + n]);  // dBt
     }
     if (tid == 0) sV[-1] = vm1;
     __syncthreads();
@@ -335,13 +415,13 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
     }
     __syncthreads();
     // ---- G. dCt ---------------------------------------------------------------------
-    mmx<T, kQ, N, kQ, false, false>(sT1, S::kMx, sCB, kQ, sBt, N, nullptr, nullptr, false);
+    mmx<T, kQ, N, kQ, false, false>(sT1, lMx, sCB, lQ, sBt, lN, nullptr, nullptr, false);
     __syncthreads();
     for (int i = tid; i < kQ * N; i += kThreads) {
       const int t = i / N, n = i % N;
-      float v = sT1[t * S::kMx + n] + sD1[t] * sT3[t * S::kMx + n];
+      float v = sT1[t * lMx + n] + sD1[t] * sT3[t * lMx + n];
       v = fmaf(sBe[0] * sD0[t] * sGxp[t], sBprev[n], v);
-      sT1[t * S::kMx + n] = v;
+      sT1[t * lMx + n] = v;
     }
     // dalpha, dbeta, dgamma of this chunk: dalpha_r = (1/alpha_r) sum_{t>=r}
     // (rowE_t - colE_t), a suffix scan over the chunk in warp 0 (lane l: steps
@@ -373,12 +453,12 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
     }
     __syncthreads();
     // ---- H. U_prev = G^T diag(d(.,0)) Ct + d(Q-1,0) alpha_Q U --------------------------
-    mmx<T, P, N, kQ, true, false>(sT3, S::kMx, sG, P, sCt, N, nullptr, sD0, false);
+    mmx<T, P, N, kQ, true, false>(sT3, lMx, sG, lP, sCt, lN, nullptr, sD0, false);
     // ---- J. RoPE backward: per-head dB, dC and dphi -----------------------------------
     for (int i = tid; i < kQ * (N / 2); i += kThreads) {
       const int t = i / (N / 2), k = i % (N / 2);
-      const float db0 = sW[t * N + 2 * k], db1 = sW[t * N + 2 * k + 1];
-      const float dc0 = sT1[t * S::kMx + 2 * k], dc1 = sT1[t * S::kMx + 2 * k + 1];
+      const float db0 = sW[t * lN + 2 * k], db1 = sW[t * lN + 2 * k + 1];
+      const float dc0 = sT1[t * lMx + 2 * k], dc1 = sT1[t * lMx + 2 * k + 1];
       float rb0 = db0, rb1 = db1, rc0 = dc0, rc1 = dc1;
       if (k < K) {
         float sn, cs;
@@ -399,10 +479,10 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
     __syncthreads();
     for (int i = tid; i < kQ * K; i += kThreads) {
       const int t = i / (int)K, k = i % (int)K;
-      const float b0 = sBt[t * N + 2 * k], b1 = sBt[t * N + 2 * k + 1];
-      const float c0 = sCt[t * N + 2 * k], c1 = sCt[t * N + 2 * k + 1];
-      const float db0 = sW[t * N + 2 * k], db1 = sW[t * N + 2 * k + 1];
-      const float dc0 = sT1[t * S::kMx + 2 * k], dc1 = sT1[t * S::kMx + 2 * k + 1];
+      const float b0 = sBt[t * lN + 2 * k], b1 = sBt[t * lN + 2 * k + 1];
+      const float c0 = sCt[t * lN + 2 * k], c1 = sCt[t * lN + 2 * k + 1];
+      const float db0 = sW[t * lN + 2 * k], db1 = sW[t * lN + 2 * k + 1];
+      const float dc0 = sT1[t * lMx + 2 * k], dc1 = sT1[t * lMx + 2 * k + 1];
       sPhi[t * kK + k] = (db1 * b0 - db0 * b1) + (dc1 * c0 - dc0 * c1);  // dphi_t[k]
     }
     __syncthreads();
@@ -419,7 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
       const float c = sD0[kQ - 1] * alQ;
       for (int i = tid; i < P * N; i += kThreads) {
         const int pp = i / N, n = i % N;
-        sU[i] = fmaf(c, sU[i], sT3[pp * S::kMx + n]);
+        sU[pp * lN + n] = fmaf(c, sU[pp * lN + n], sT3[pp * lMx + n]);
       }
     }
     alQ = sAl[0];
@@ -429,7 +509,7 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
 
   if (p.dh0) {
     for (int i = tid; i < P * N; i += kThreads)
-      p.dh0[(b * H + h) * P * N + i] = alQ * sU[i];  // alpha_0 Lambda_0
+      p.dh0[(b * H + h) * P * N + i] = alQ * sU[(i / N) * lN + i % N];  // alpha_0 Lambda_0
   }
   const float dD = block_sum(dD_l, sRed);
   if (tid == 0) ws_dD[b * H + h] = dD;
