@@ -85,6 +85,31 @@ def su_bytes(Bsz, D, N, io_bytes, G=1):
 
 
 # ---------------------------------------------------------------------------
+# DRAM traffic of the dominant kernel from an ncu capture (dram__bytes_read.sum
+# + dram__bytes_write.sum, one launch of the named workload), valid only for
+# the kernel source it was taken on: reported when the source file's hash
+# still matches, else null.
+# ---------------------------------------------------------------------------
+NCU_TRAFFIC = {
+    # kernel source file: (sha256 prefix of the file, workload, bytes per launch)
+}
+
+
+def ncu_traffic(src_name):
+    import hashlib
+    ent = NCU_TRAFFIC.get(src_name)
+    if ent is None:
+        return None
+    path = os.path.join(ROOT, "selective_state_space_14_b200", "csrc", src_name)
+    try:
+        with open(path, "rb") as f:
+            digest = hashlib.sha256(f.read()).hexdigest()
+    except OSError:
+        return None
+    return ent[2] if digest.startswith(ent[0]) else None
+
+
+# ---------------------------------------------------------------------------
 # clocks sampling
 # ---------------------------------------------------------------------------
 class ClockSampler:
@@ -339,7 +364,8 @@ def run_ours(args):
     dom_ms, dom_b = (bwd_ms, bwd_b) if dom == "bwd" else (fwd_ms, fwd_b)
     achieved = dom_b / (dom_ms / 1e3) / 1e9
     roofline = dict(bound="hbm", achieved=round(achieved, 1), peak=peaks["hbm_gbs"], unit="GB/s",
-                    frac=round(achieved / peaks["hbm_gbs"], 4), traffic=None,
+                    frac=round(achieved / peaks["hbm_gbs"], 4),
+                    traffic=ncu_traffic("m1_bwd.cu" if dom == "bwd" else "m1_fwd.cu"),
                     kernel=("msc_selective_scan_bwd (m1_bwd_kernel + m1_bwd_reduce_kernel)"
                             if dom == "bwd" else "msc_selective_scan_fwd (m1_fwd_kernel)"),
                     algorithmic_bytes=dom_b, launch_ms=round(dom_ms, 4),

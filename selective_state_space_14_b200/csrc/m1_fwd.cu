@@ -9,10 +9,11 @@
 //
 // Work decomposition (m1_common.cuh): a thread owns a (b, c) sequence and one
 // pair of state indices, and steps through time with the pair of states in
-// registers; exp(delta A) is taken as 2^(delta * A log2 e) on the SFU.  Per
-// 64-step chunk the CTA stages the per-token values of its channels (softplus
-// and the silu gate computed once per token) and the batch row's B, C in
-// shared memory.  y_t sums over the state pairs of a channel: every kP steps
+// registers; exp(delta A) is taken as 2^(delta * A log2 e) on the SFU.  The
+// raw inputs of a 32-step chunk (u, delta, z of the CTA's channels and the
+// batch row's B, C) arrive by cp.async one chunk ahead; per chunk the CTA
+// turns them into per-token values (softplus and the silu gate computed once
+// per token) and an f32 table of B, C pairs in shared memory.  y_t sums over the state pairs of a channel: every kP steps
 // each lane writes its kP pair partials to a padded shared-memory tile and
 // then sums one step's partials in pair order (a transpose through shared
 // memory, no shuffles).  Gated outputs collect in shared memory and leave in
@@ -26,6 +27,8 @@ namespace {
 using namespace m1;
 
 constexpr int kWarps = 4;
+constexpr int kTF = 32;  // steps per forward chunk
+static_assert(kTF % kM1SaveInterval == 0, "chunk must hold whole saved-state intervals");
 
 template <int kN>
 struct FwdSmem {
@@ -37,22 +40,82 @@ struct FwdSmem {
   static constexpr int kRow = kP + 4;
   static constexpr int kChBlock = kP * kRow + (kP == 8 ? 8 : (kP == 16 ? 16 : 0));
   // float offsets
-  static constexpr int kOut = kT + 8;  // output tile channel stride (bank spread)
-  static constexpr int tok = 0;                               // [kT][kCh] float4
-  static constexpr int bc = tok + kCh * kT * 4;               // [kT][kP] float4
-  static constexpr int ytile = bc + kT * kP * 4;              // [kWarps][32/kP][kChBlock]
+  static constexpr int kOut = kTF + 8;  // output tile channel stride (bank spread)
+  static constexpr int tok = 0;                               // [kTF][kCh] float4
+  static constexpr int bc = tok + kCh * kTF * 4;              // [kTF][kP] float4
+  static constexpr int ytile = bc + kTF * kP * 4;             // [kWarps][32/kP][kChBlock]
   static constexpr int out = ytile + kWarps * (32 / kP) * kChBlock;  // [kCh][kOut]
-  static constexpr int total = out + kCh * kOut;
+  static constexpr int raw = (out + kCh * kOut + 3) / 4 * 4;  // raw inputs (16-byte aligned)
+  static constexpr int total_floats = raw;
 };
+
+// raw inputs of one chunk, bytes: u, delta, z [3][kCh][kTF] T; B, C [2][kN][kTF] T
+template <typename T, int kN>
+struct FwdRaw {
+  static constexpr int kCh = Layout<kN, kWarps>::kCh;
+  static constexpr int tok = 0;
+  static constexpr int bc = 3 * kCh * kTF * (int)sizeof(T);
+  static constexpr int bytes = bc + 2 * kN * kTF * (int)sizeof(T);
+};
+
+// Issue the copies of the chunk starting at tc into the raw buffer: 16-byte
+// cp.async pieces (zero-filled past the end of a row) when rows are 16-byte
+// aligned, element copies otherwise.  Entries past L, past the last channel
+// or past d_state are never read as data.
+template <typename T, int kN>
+__device__ __forceinline__ void fwd_issue_raw(const M1Params &p, unsigned char *raw, int64_t b,
+                                              int64_t c_first, int64_t c_end, const T *Bg,
+                                              const T *Cg, int64_t tc, int tid) {
+  using R = FwdRaw<T, kN>;
+  constexpr int kCh = R::kCh;
+  constexpr int kThreads = kWarps * 32;
+  constexpr int E = 16 / (int)sizeof(T);
+  constexpr int kPieces = kTF / E;
+  const int64_t L = p.L, N = p.N;
+  for (int u = tid; u < 3 * kCh * kPieces + 2 * kN * kPieces; u += kThreads) {
+    const T *row;
+    bool ok;
+    int r, j;
+    T *dst;
+    if (u < 3 * kCh * kPieces) {
+      j = u % kPieces;
+      r = u / kPieces;
+      const int cl = r % kCh, k = r / kCh;
+      const int64_t c = c_first + cl;
+      const void *src = k == 0 ? p.u : (k == 1 ? p.delta : p.z);
+      ok = src != nullptr && c < c_end;
+      row = ok ? static_cast<const T *>(src) + (b * p.D + c) * L : static_cast<const T *>(p.u);
+      dst = reinterpret_cast<T *>(raw + R::tok) + r * kTF + j * E;
+    } else {
+      const int v = u - 3 * kCh * kPieces;
+      j = v % kPieces;
+      r = v / kPieces;
+      const int n = r % kN, k = r / kN;
+      ok = n < N;
+      row = ok ? (k == 0 ? Bg : Cg) + n * L : Bg;
+      dst = reinterpret_cast<T *>(raw + R::bc) + r * kTF + j * E;
+    }
+    const int64_t t = tc + j * E;
+    const int64_t left = L - t;
+    const int valid = !ok || left <= 0 ? 0 : (left >= E ? E : (int)left);
+    if (p.vec) {
+      cp_async16(dst, valid > 0 ? row + t : row, valid * (int)sizeof(T));
+    } else {
+#pragma unroll
+      for (int i = 0; i < E; ++i) dst[i] = i < valid ? row[t + i] : from_f32<T>(0.f);
+    }
+  }
+  cp_async_commit();
+}
 
 // Store the gated outputs of the chunk starting at tc from shared memory.
 template <typename T, int kCh, int kOut>
 __device__ __forceinline__ void store_chunk(T *out_base, const float *sout, int64_t c_first,
                                             int64_t c_end, int64_t b, int64_t D, int64_t L,
                                             int64_t tc, bool vec, int tid, int nthreads) {
-  for (int u = tid; u < kCh * (kT / 8); u += nthreads) {
-    const int chl = u / (kT / 8);
-    const int seg = u % (kT / 8);
+  for (int u = tid; u < kCh * (kTF / 8); u += nthreads) {
+    const int chl = u / (kTF / 8);
+    const int seg = u % (kTF / 8);
     const int64_t c = c_first + chl;
     if (c >= c_end) continue;
     float v[8];
@@ -94,8 +157,10 @@ __global__ void __launch_bounds__(kWarps * 32, 6) m1_fwd_kernel(const M1Params p
   const bool active = c < c_end;
   const T *Bg = static_cast<const T *>(p.Bm) + (b * p.G + g) * N * L;
   const T *Cg = static_cast<const T *>(p.Cm) + (b * p.G + g) * N * L;
-  const int64_t n_chunks = (L + kT - 1) / kT;
+  const int64_t n_chunks = (L + kTF - 1) / kTF;
   const int64_t n_save = (L + kM1SaveInterval - 1) / kM1SaveInterval;
+  using R = FwdRaw<T, kN>;
+  unsigned char *raw = reinterpret_cast<unsigned char *>(smem + S::raw);
 
   // this thread's state pair and its A * log2(e)
   const int n0 = 2 * pr, n1 = 2 * pr + 1;
@@ -108,47 +173,67 @@ __global__ void __launch_bounds__(kWarps * 32, 6) m1_fwd_kernel(const M1Params p
       if (n1 < N) h.y = p.h0[(b * D + c) * N + n1];
     }
   }
+  // token conversion role: channel tcl, a run of kRun steps tseg (one run per thread)
+  constexpr int kRun = kCh * kTF / kThreads;  // 4, 2, 1 for d_state 16, 32, 64
+  static_assert(kRun >= 1 && kCh * kTF == kRun * kThreads, "one token run per thread");
+  const int tcl = tid % kCh, tseg = tid / kCh;
+  const int64_t tcc = c_first + tcl;
+  const bool tact = tcc < c_end;
+  const float tDc = (tact && p.Dp) ? p.Dp[tcc] : 0.f;
+  const float tbias = (tact && p.bias) ? p.bias[tcc] : 0.f;
 
+  fwd_issue_raw<T, kN>(p, raw, b, c_first, c_end, Bg, Cg, 0, tid);
   for (int64_t ch = 0; ch <= n_chunks; ++ch) {
-    const int64_t tc = ch * kT;
-    // ---- outputs of the previous chunk, and staging of this chunk ----------
+    const int64_t tc = ch * kTF;
+    cp_async_wait<0>();
+    __syncthreads();  // this chunk's raw inputs are in; the last chunk is done
     if (ch > 0)
       store_chunk<T, kCh, S::kOut>(static_cast<T *>(p.out), sOut, c_first, c_end, b, D, L,
-                                   tc - kT, p.vec, tid, kThreads);
+                                   tc - kTF, p.vec, tid, kThreads);
     if (ch == n_chunks) break;
-    // (channel fastest: stores to the [step][channel] tile are contiguous, and
-    // lanes cl and cl + kCh read the two halves of one 32-byte sector)
-    for (int u = tid; u < kCh * (kT / 8); u += kThreads) {
-      const int cl = u % kCh, seg = u / kCh;
-      const int64_t cc = c_first + cl;
-      const int64_t t = tc + seg * 8;
-      float x[8], v[8], zv[8];
-      const bool act = cc < c_end;
-      if (act) {
-        const int64_t row = (b * D + cc) * L;
-        load_run<8>(static_cast<const T *>(p.u) + row, t, L, p.vec, x, 0.f);
-        load_run<8>(static_cast<const T *>(p.delta) + row, t, L, p.vec, v, 0.f);
-        if (p.z) load_run<8>(static_cast<const T *>(p.z) + row, t, L, p.vec, zv, 0.f);
-      }
-      const float Dc = (act && p.Dp) ? p.Dp[cc] : 0.f;
-      const float bias = (act && p.bias) ? p.bias[cc] : 0.f;
+    // ---- per-token values: kRun steps of one channel per thread ---------------
+    {
+      const T *ru = reinterpret_cast<const T *>(raw + R::tok);
+      float x[kRun], v[kRun], zv[kRun];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
+      for (int i = 0; i < kRun; ++i) {
+        const int o = tcl * kTF + tseg * kRun + i;
+        x[i] = to_f32(ru[o]);
+        v[i] = to_f32(ru[kCh * kTF + o]);
+        zv[i] = p.z ? to_f32(ru[2 * kCh * kTF + o]) : 0.f;
+      }
+#pragma unroll
+      for (int i = 0; i < kRun; ++i) {
         float4 tk = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (act && t + i < L) {
-          const float vv = v[i] + bias;
+        if (tact && tc + tseg * kRun + i < L) {
+          const float vv = v[i] + tbias;
           const float d = p.softplus ? softplus(vv) : vv;
-          tk = make_float4(d, d * x[i], Dc * x[i], p.z ? silu(zv[i]) : 1.f);
+          tk = make_float4(d, d * x[i], tDc * x[i], p.z ? silu(zv[i]) : 1.f);
         }
-        sTok[(seg * 8 + i) * kCh + cl] = tk;
+        sTok[(tseg * kRun + i) * kCh + tcl] = tk;
       }
     }
-    stage_bc<T, kN, kT>(sBC, Bg, Cg, N, L, tc, p.vec, tid, kThreads);
-    __syncthreads();
+    // ---- B, C pairs in f32 ------------------------------------------------------
+    {
+      const T *rb = reinterpret_cast<const T *>(raw + R::bc);
+      for (int u = tid; u < kTF * kP; u += kThreads) {
+        const int t = u % kTF, q = u / kTF;
+        const bool in = tc + t < L;
+        float e[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int n = 2 * q + (k & 1);
+          e[k] = (in && n < N) ? to_f32(rb[((k >> 1) * kN + n) * kTF + t]) : 0.f;
+        }
+        sBC[t * kP + q] = make_float4(e[0], e[1], e[2], e[3]);
+      }
+    }
+    __syncthreads();  // tables ready; the raw buffer and the output tile are free
+    if (ch + 1 < n_chunks) fwd_issue_raw<T, kN>(p, raw, b, c_first, c_end, Bg, Cg, tc + kTF, tid);
 
     // ---- the recurrence over the chunk -------------------------------------
 #pragma unroll 1
-    for (int grp = 0; grp < kT / kP; ++grp) {
+    for (int grp = 0; grp < kTF / kP; ++grp) {
       float yp[kP];
 #pragma unroll
       for (int k = 0; k < kP; ++k) {
@@ -178,7 +263,6 @@ __global__ void __launch_bounds__(kWarps * 32, 6) m1_fwd_kernel(const M1Params p
       sOut[chl * S::kOut + t] = y * tk.w;
       __syncwarp();
     }
-    __syncthreads();
   }
 
   if (active && p.final_state) {
@@ -191,7 +275,7 @@ __global__ void __launch_bounds__(kWarps * 32, 6) m1_fwd_kernel(const M1Params p
 template <typename T, int kN>
 cudaError_t launch_t(const M1Params &p, cudaStream_t s) {
   using Lay = Layout<kN, kWarps>;
-  const size_t smem = sizeof(float) * (size_t)FwdSmem<kN>::total;
+  const size_t smem = sizeof(float) * (size_t)FwdSmem<kN>::total_floats + FwdRaw<T, kN>::bytes;
   cudaError_t e = cudaFuncSetAttribute(m1_fwd_kernel<T, kN>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
