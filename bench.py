@@ -92,6 +92,7 @@ def su_bytes(Bsz, D, N, io_bytes, G=1):
 # ---------------------------------------------------------------------------
 NCU_TRAFFIC = {
     # kernel source file: (sha256 prefix of the file, workload, bytes per launch)
+    "m1_bwd.cu": ("11a659c65d88cc6a", "m1_bf16_b8_d1536_n16_l2048", 404215040 + 157788672),
 }
 
 
@@ -113,57 +114,58 @@ def ncu_traffic(src_name):
 # clocks sampling
 # ---------------------------------------------------------------------------
 class ClockSampler:
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and throttle reasons of one GPU, polled through NVML every
+    ``period_s`` from a thread while the timed region runs (read-only)."""
 
-    def __init__(self, gpu_index):
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4}
+
+    def __init__(self, gpu_index, period_s=0.002):
         self.gpu = gpu_index
-        self.proc = None
-        self.lines = []
+        self.period = period_s
+        self.samples = []
+        self.err = None
+        self._stop = threading.Event()
+        self.thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.handle = pynvml.nvmlDeviceGetHandleByIndex(gpu_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # noqa: BLE001 -- no NVML: report it, keep the run
+            self.nvml = None
+            self.err = f"nvml unavailable: {e}"[:120]
+
+    def _poll(self):
+        n = self.nvml
+        while not self._stop.is_set():
+            try:
+                sm = n.nvmlDeviceGetClockInfo(self.handle, n.NVML_CLOCK_SM)
+                rs = n.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                self.samples.append((sm, rs))
+            except Exception as e:  # noqa: BLE001
+                self.err = str(e)[:120]
+                return
+            time.sleep(self.period)
 
     def start(self):
-        try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
-            self.thread.start()
-        except (FileNotFoundError, OSError):
-            self.proc = None
-
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+        if self.nvml is None:
+            return
+        self.thread = threading.Thread(target=self._poll, daemon=True)
+        self.thread.start()
 
     def stop(self):
-        if self.proc is None:
-            return dict(sm_mhz=None, sm_max_mhz=None, reasons=["nvidia-smi unavailable"])
-        time.sleep(0.15)
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=2)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            f = [x.strip() for x in ln.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                smax.append(float(f[2]))
-            except ValueError:
-                continue
-            for nm, v in zip(names, f[5:9]):
-                if v.lower() == "active":
-                    reasons.add(nm)
-        if not sm:
-            return dict(sm_mhz=None, sm_max_mhz=None, reasons=["no samples"])
-        return dict(sm_mhz=statistics.median(sm), sm_max_mhz=max(smax), reasons=sorted(reasons),
-                    samples=len(sm))
+        if self.nvml is None:
+            return dict(sm_mhz=None, sm_max_mhz=None, reasons=[self.err])
+        self._stop.set()
+        self.thread.join(timeout=2)
+        if not self.samples:
+            return dict(sm_mhz=None, sm_max_mhz=self.max_mhz, reasons=["no samples"])
+        reasons = sorted({name for _, rs in self.samples for name, bit in self.REASONS.items()
+                          if rs & bit})
+        return dict(sm_mhz=statistics.median(s for s, _ in self.samples), sm_max_mhz=self.max_mhz,
+                    reasons=reasons, samples=len(self.samples))
 
 
 # ---------------------------------------------------------------------------
@@ -258,8 +260,9 @@ class M1Step:
                                         workspace=self.ws, grads=self.grads, want_dh0=False)
 
 
-def time_steps(step_fns, steps, warmup, world):
-    """Run warmup, then time `steps` iterations; per-phase CUDA-event times."""
+def time_steps(step_fns, steps, warmup, world, sampler=None):
+    """Run warmup, then time `steps` iterations; per-phase CUDA-event times.
+    A clock sampler, if given, runs during the timed region only."""
     import torch
     for _ in range(warmup):
         for f in step_fns:
@@ -272,6 +275,8 @@ def time_steps(step_fns, steps, warmup, world):
           for _ in range(steps)]
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
+    if sampler is not None:
+        sampler.start()
     start.record(stream)
     for k in range(steps):
         ev[k][0].record(stream)
@@ -280,6 +285,8 @@ def time_steps(step_fns, steps, warmup, world):
             ev[k][i + 1].record(stream)
     end.record(stream)
     torch.cuda.synchronize()
+    if sampler is not None:
+        sampler.clocks = sampler.stop()
     barrier(world)
     total_ms = start.elapsed_time(end)
     phase_ms = [sum(ev[k][i].elapsed_time(ev[k][i + 1]) for k in range(steps)) / steps
@@ -352,9 +359,9 @@ def run_ours(args):
     p = W.make(HEADLINE, shard=rank)  # each rank its own batch of the same shape
     st = M1Step(p, msc)
     sampler = ClockSampler(local)
-    sampler.start()
-    total_ms, (fwd_ms, bwd_ms) = time_steps([st.fwd, st.bwd], args.steps, args.warmup, world)
-    clocks = sampler.stop()
+    total_ms, (fwd_ms, bwd_ms) = time_steps([st.fwd, st.bwd], args.steps, args.warmup, world,
+                                            sampler=sampler)
+    clocks = sampler.clocks
     total_ms = max_over_ranks(world, total_ms)
     ms_per_step = total_ms / args.steps
     units = p.token_channels
