@@ -71,6 +71,12 @@ CASES = [
     (2, 256, 8, 130, 2, "f32", True, True, True, True, True),
     (2, 96, 16, 700, 1, "bf16", True, True, True, True, True),
     (1, 40, 16, 9, 1, "bf16", True, True, True, False, True),
+    # 16-byte-aligned rows (cp.async staging) with a ragged last block, groups
+    # that do not fill whole CTAs or clusters, d_state 32 and 64
+    (2, 100, 32, 1000, 2, "bf16", True, True, True, True, True),
+    (1, 24, 64, 96, 1, "bf16", True, True, True, True, True),
+    (3, 36, 16, 1024, 3, "bf16", True, False, True, True, True),
+    (1, 20, 16, 40, 1, "f32", True, True, True, True, True),
 ]
 
 
