@@ -64,6 +64,26 @@ def test_fwd_parity_shapes(msc, case):
     assert_close("final_state", g["final_state"], r["final_state"], TOL[io])
 
 
+@pytest.mark.parametrize("case", [c for c in FWD_CASES if c[7] == "bf16"],
+                         ids=[f"B{c[0]}L{c[1]}H{c[2]}P{c[3]}N{c[4]}G{c[5]}K{c[6]}" for c in FWD_CASES
+                              if c[7] == "bf16"])
+def test_fwd_without_saved_states(msc, case):
+    """bf16 forward without saved states against the oracle, and against the
+    same forward with saved states."""
+    Bsz, L, H, P, N, G, K, io, z, Dp, h0 = case
+    p = W.m3_problem(Bsz, L, H, P, N, ngroups=G, nangles=K, io=io, seed=77 + L + H, with_z=z,
+                     with_D=Dp, with_h0=h0)
+    a = m3_device_args(p)
+    out1, fs1, sv = msc.msc_mamba3_siso_scan_fwd(**a, want_saved_states=False)
+    out2, fs2, _ = msc.msc_mamba3_siso_scan_fwd(**a)
+    torch.cuda.synchronize()
+    assert sv is None
+    r = _oracle_fwd(p)
+    assert_close("out", host(out1), r["out"], TOL[io])
+    assert_close("final_state", host(fs1), r["final_state"], TOL[io])
+    assert torch.equal(out1, out2) and torch.equal(fs1, fs2)
+
+
 def test_fwd_determinism(msc):
     p = W.m3_problem(2, 150, 3, 64, 64, nangles=32, io="bf16", seed=3)
     a = m3_device_args(p)
