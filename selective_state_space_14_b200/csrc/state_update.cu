@@ -34,7 +34,29 @@ __global__ void __launch_bounds__(256) state_update_kernel(const SUParams p) {
   const T *Cp = static_cast<const T *>(p.Cm) + (b * p.G + g) * N;
   const float *Ap = p.A + c * N;
   float *st = p.state + i * N;
-  if (N % 4 == 0) {
+  if (N % 8 == 0) {
+    // B and C in 16-byte runs (8 io elements) next to the state's 16-byte pieces
+    for (int64_t n = 0; n < N; n += 8) {
+      float bv[8], cv[8];
+      load_run<8, Cache::kKeep>(Bp, n, N, true, bv, 0.f);
+      load_run<8, Cache::kKeep>(Cp, n, N, true, cv, 0.f);
+#pragma unroll
+      for (int q = 0; q < 8; q += 4) {
+        const float4 h4 = *reinterpret_cast<const float4 *>(st + n + q);
+        const float4 A4 = __ldg(reinterpret_cast<const float4 *>(Ap + n + q));
+        float2 h01 = make_float2(h4.x, h4.y), h23 = make_float2(h4.z, h4.w);
+        const float2 a01 = ex2_2(mul2(splat2(d), mul2(make_float2(A4.x, A4.y), splat2(kLog2e))));
+        const float2 a23 = ex2_2(mul2(splat2(d), mul2(make_float2(A4.z, A4.w), splat2(kLog2e))));
+        h01 = fma2(a01, h01, mul2(splat2(dtx), make_float2(bv[q], bv[q + 1])));
+        h23 = fma2(a23, h23, mul2(splat2(dtx), make_float2(bv[q + 2], bv[q + 3])));
+        y = fmaf(cv[q], h01.x, y);
+        y = fmaf(cv[q + 1], h01.y, y);
+        y = fmaf(cv[q + 2], h23.x, y);
+        y = fmaf(cv[q + 3], h23.y, y);
+        *reinterpret_cast<float4 *>(st + n + q) = make_float4(h01.x, h01.y, h23.x, h23.y);
+      }
+    }
+  } else if (N % 4 == 0) {
     for (int64_t n = 0; n < N; n += 4) {
       const float4 h4 = *reinterpret_cast<const float4 *>(st + n);
       const float4 A4 = __ldg(reinterpret_cast<const float4 *>(Ap + n));
