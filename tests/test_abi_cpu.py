@@ -132,3 +132,11 @@ def test_size_functions():
         4 * 2 * 3 * 2 * (16 * 32 + 16)
     assert msc.msc_selective_scan_bwd_workspace_bytes(8, 1536, 16, 2048, 1) <= \
         msc.MSC_STATIC_SCRATCH_BYTES
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    """No silent fallback: without libmsc.so the binding raises."""
+    monkeypatch.setattr(msc, "LIB_PATH", str(tmp_path / "missing" / "libmsc.so"))
+    monkeypatch.setattr(msc, "_lib", None)
+    with pytest.raises(RuntimeError, match="missing"):
+        msc.lib()

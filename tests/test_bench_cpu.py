@@ -1,0 +1,53 @@
+"""Host-side pieces of bench.py: the algorithmic byte counts the roofline
+divides by, the source-hash gate on the recorded ncu traffic, and the clock
+sampler's behaviour without a GPU."""
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+def test_m1_bytes_per_unit():
+    # bwd: 7 io values per token-channel; B, C in and dB, dC (f32) out per
+    # (b, t); A, D, bias in and dA, dD, dbias out
+    B, D, N, L, io = 8, 1536, 16, 2048, 2
+    fwd, bwd = bench.m1_bytes(B, D, N, L, io)
+    tc, bt = B * D * L, B * L
+    params = D * N * 4 + 2 * D * 4
+    assert bwd == 7 * io * tc + 2 * N * io * bt + 2 * N * 4 * bt + params + D * N * 4 + 2 * D * 4
+    assert fwd == 4 * io * tc + 2 * N * io * bt + params + B * D * N * 4
+    assert bwd == 355688448  # the figure the bench line and DESIGN quote
+
+
+def test_m3_bytes_per_unit():
+    B, L, H, P, N, G, K, io = 8, 2048, 24, 64, 64, 1, 32, 2
+    fwd, bwd = bench.m3_bytes(B, L, H, P, N, G, K, io)
+    assert fwd == 3 * io * B * L * H * P + (3 + K) * io * B * L * H + 2 * N * io * B * L * G \
+        + B * H * P * N * 4
+    assert round(fwd / 1e6, 1) == 185.9 and round(bwd / 1e6, 1) == 346.8
+
+
+def test_decode_bytes():
+    assert round(bench.su_bytes(256, 5120, 16, 2) / 1e6, 1) == 178.3
+
+
+def test_traffic_gated_by_source_hash(monkeypatch):
+    assert bench.ncu_traffic("no_such_kernel.cu") is None
+    monkeypatch.setitem(bench.NCU_TRAFFIC, "m1_fwd.cu", ("0000000000000000", "w", 123))
+    assert bench.ncu_traffic("m1_fwd.cu") is None  # stale capture: not reported
+    import hashlib
+    path = os.path.join(ROOT, "selective_state_space_14_b200", "csrc", "m1_fwd.cu")
+    h = hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+    monkeypatch.setitem(bench.NCU_TRAFFIC, "m1_fwd.cu", (h, "w", 123))
+    assert bench.ncu_traffic("m1_fwd.cu") == 123
+
+
+def test_clock_sampler_without_gpu():
+    s = bench.ClockSampler(0)
+    s.start()
+    r = s.stop()
+    assert set(r) >= {"sm_mhz", "sm_max_mhz", "reasons"}
