@@ -1,0 +1,543 @@
+// m3_fwd_umma.cu -- Mamba-3 SISO scan, forward, bf16 io, on the sm_100a
+// tensor cores through tcgen05 (umma.cuh).
+//
+// Same recurrence, chunked form (m3_common.cuh) and outputs as m3_fwd_tc.cu
+// (mamba-rs 0.7.0 README, "Features"; the three-term update and per-head
+// cumulative angles whose gradients stages B3 and B4 of Mamba3Scratch,
+// mamba-rs 0.4.2 src/mamba3_siso/cpu/scratch.rs, hold).  One CTA of 8 warps
+// per (b, h) walks the 64-step chunks in order, two CTAs per SM.  A chunk is
+// two rounds of tensor-core work:
+//
+//   round 1   G  = Ct Bt^T        (A: Ct [t][n], B: Bt [s][n])
+//             Y1 = Ct S^T         (A: Ct,        B: S  [p][n])
+//   epilogue  W  = c o G          (into Ct's planes)
+//             Bc = diag(c(Q-1, .)) Bt   (into Bt's planes)
+//   round 2   Y2 = W X            (A: W [t][s],  B: X^T [p][s])
+//             dS = X^T Bc         (A: X^T,       B: Bc read MN-major)
+//   epilogue  out = (d(t,-1) Y1 + Y2 + beta_0 d(t,0) (Ct.Bt_prev) x_prev + D x) silu(z)
+//             S   = d(Q-1,-1) S + beta_0 d(Q-1,0) x_prev (outer) Bt_prev + dS
+//
+// f32 operands live in shared memory as three bf16 parts, the bf16 inputs as
+// one, so every product carries f32 accuracy.  Thread 0 issues the MMAs; the
+// CTA waits on an mbarrier (bounded) and reads the f32 accumulators from
+// TMEM.  The state stays in registers, row r of the accumulator layout per
+// thread, with its parts in shared memory for the next chunk's Y1.  x, B, C of
+// the next chunk arrive by cp.async, and theta, alpha, beta, gamma into
+// registers, while a chunk computes.
+//
+// Shared-memory access patterns follow the core-matrix layout: a warp stores
+// a core matrix (8 rows x 16 bytes) per instruction, so that no two lanes
+// share a bank.  The cumulative angles come from a scan over each warp's 8
+// steps (lanes 4 i + q hold step i of angle pairs q, q + 4, ...) and the
+// per-warp totals, which is also the layout the rotation writes in.
+#include "m3_common.cuh"
+#include "umma.cuh"
+
+namespace msc {
+namespace {
+
+using namespace m3;
+using umma::koff;
+
+template <int P, int N>
+struct UmFwdSmem {
+  static constexpr int kK = N / 2;
+  static constexpr int kRS = N * 2 + 16;   // raw B, C row stride in bytes (padded: no bank conflicts)
+  // bytes; bf16 part planes, K-major core-matrix layout (umma.cuh)
+  static constexpr int kCW = 64 * 64 * 2;  // one part of Ct (K = N) or W (K = Q)
+  static constexpr int kBt = 64 * N * 2;   // one part of Bt / Bc [s][n]
+  static constexpr int kSp = P * N * 2;    // one part of S [p][n]
+  static constexpr int cw = 0;
+  static constexpr int bt = cw + 3 * kCW;
+  static constexpr int sp = bt + 3 * kBt;
+  static constexpr int xp = sp + 3 * kSp;       // X^T [p][s], exact bf16, 64 rows (rows >= P zero)
+  static constexpr int rx = xp + 64 * 64 * 2;   // raw x [t][p]
+  static constexpr int rB = rx + 64 * P * 2;    // raw B [t][n]
+  static constexpr int rC = rB + 64 * kRS;      // raw C [t][n]
+  // f32 vectors
+  static constexpr int vec = rC + 64 * kRS;
+  static constexpr int al = vec, be = al + 256, ga = be + 256, lc = ga + 256, ev = lc + 256,
+                       dl = ev + 256, crow = dl + 256, wcd = crow + 256,
+                       xprev = wcd + 256,        // [2][P], by chunk parity
+                       bprev = xprev + 2 * P * 4,  // [2][N]
+                       phi0 = bprev + 2 * N * 4, seg = phi0 + kK * 4, misc = seg + 8 * kK * 4;
+  static constexpr int total = misc + 32;  // tmem slot, mbarrier, error flag
+};
+
+// cp.async the raw x, B, C rows of the chunk at t0 (rows past L zero-filled)
+template <int P, int N>
+__device__ __forceinline__ void um_issue_raw(const M3Params &p, unsigned char *sm, int64_t b,
+                                             int64_t h, int64_t g, int64_t t0) {
+  using S = UmFwdSmem<P, N>;
+  const int64_t L = p.L, H = p.H, G = p.G;
+  const bf16 *x = static_cast<const bf16 *>(p.x);
+  const bf16 *Bm = static_cast<const bf16 *>(p.Bm);
+  const bf16 *Cm = static_cast<const bf16 *>(p.Cm);
+  for (int u = threadIdx.x; u < kQ * (P / 8) + 2 * kQ * (N / 8); u += kThreads) {
+    if (u < kQ * (P / 8)) {
+      const int t = u / (P / 8), pc = u % (P / 8);
+      const bool in = t0 + t < L;
+      cp_async16(sm + S::rx + (t * P + pc * 8) * 2,
+                 in ? x + ((b * L + t0 + t) * H + h) * P + pc * 8 : x, in ? 16 : 0);
+    } else {
+      const int v = u - kQ * (P / 8);
+      const int k = v / (kQ * (N / 8)), w = v % (kQ * (N / 8));
+      const int t = w / (N / 8), pc = w % (N / 8);
+      const bool in = t0 + t < L;
+      const bf16 *src = k == 0 ? Bm : Cm;
+      cp_async16(sm + (k == 0 ? S::rB : S::rC) + t * S::kRS + pc * 16,
+                 in ? src + ((b * L + t0 + t) * G + g) * N + pc * 8 : src, in ? 16 : 0);
+    }
+  }
+  cp_async_commit();
+}
+
+__device__ __forceinline__ uint32_t bf16pair(bf16 lo, bf16 hi) {
+  return (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
+}
+
+// the three parts of (v0, v1) at byte offset `off` of the planes at `base`
+// (plane stride `stride`), one 4-byte store per plane
+__device__ __forceinline__ void put3x2(unsigned char *base, int stride, int off, float v0,
+                                       float v1) {
+  bf16 a[3], c[3];
+  umma::split3(v0, a);
+  umma::split3(v1, c);
+#pragma unroll
+  for (int q = 0; q < 3; ++q)
+    *reinterpret_cast<uint32_t *>(base + q * stride + off) = bf16pair(a[q], c[q]);
+}
+
+// the three parts of v[0..7] (one core-matrix row), one 16-byte store per plane
+__device__ __forceinline__ void put3x8(unsigned char *base, int stride, int off, const float *v) {
+  uint32_t w[3][4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    bf16 a[3], c[3];
+    umma::split3(v[2 * e], a);
+    umma::split3(v[2 * e + 1], c);
+#pragma unroll
+    for (int q = 0; q < 3; ++q) w[q][e] = bf16pair(a[q], c[q]);
+  }
+#pragma unroll
+  for (int q = 0; q < 3; ++q)
+    *reinterpret_cast<uint4 *>(base + q * stride + off) = make_uint4(w[q][0], w[q][1], w[q][2], w[q][3]);
+}
+
+// Issue one product into TMEM column `col`: parts of A (nA of them, planes at
+// aA, stride sA, K-major with Ka columns, 64 rows) times parts of B (nB,
+// planes at aB, stride sB; K-major with Kb columns, or with kBMN the same
+// bytes read MN-major, Kb then being the MN extent), over K / 16 steps.  Part
+// pairs whose order is below f32 rounding are left out; the smallest go first.
+template <int NMMA, bool kBMN>
+__device__ __forceinline__ void issue_product(uint32_t tmem, int col, uint32_t aA, int sA, int nA,
+                                              int Ka, uint32_t aB, int sB, int nB, int Kb, int K) {
+  const uint32_t id = umma::idesc_bf16<NMMA, kBMN>();
+  const int pa[6] = {2, 1, 0, 1, 0, 0}, pb[6] = {0, 1, 2, 0, 1, 0};
+  bool first = true;
+  for (int u = 0; u < 6; ++u) {
+    if (pa[u] >= nA || pb[u] >= nB) continue;
+    for (int ks = 0; ks < K / 16; ++ks) {
+      const uint64_t da = umma::desc(aA + pa[u] * sA + ks * 256, 128, Ka * 16);
+      const uint64_t db = kBMN ? umma::desc(aB + pb[u] * sB + ks * 2 * (Kb * 16), Kb * 16, 128)
+                               : umma::desc(aB + pb[u] * sB + ks * 256, 128, Kb * 16);
+      umma::mma(tmem + col, da, db, id, !first);
+      first = false;
+    }
+  }
+}
+
+template <int P, int N>
+__global__ void __launch_bounds__(kThreads, 2) m3_fwd_umma_kernel(const M3Params p) {
+  using S = UmFwdSmem<P, N>;
+  constexpr int kK = N / 2;
+  constexpr int kJ = kK / 4;  // angle pairs per rotation lane
+  extern __shared__ __align__(1024) unsigned char sm[];
+  float *sAl = reinterpret_cast<float *>(sm + S::al), *sBe = reinterpret_cast<float *>(sm + S::be);
+  float *sGa = reinterpret_cast<float *>(sm + S::ga), *sLc = reinterpret_cast<float *>(sm + S::lc);
+  float *sEv = reinterpret_cast<float *>(sm + S::ev), *sDl = reinterpret_cast<float *>(sm + S::dl);
+  float *sCrow = reinterpret_cast<float *>(sm + S::crow);
+  float *sWcd = reinterpret_cast<float *>(sm + S::wcd);
+  float *sXprev = reinterpret_cast<float *>(sm + S::xprev);
+  float *sBprev = reinterpret_cast<float *>(sm + S::bprev);
+  float *sPhi0 = reinterpret_cast<float *>(sm + S::phi0), *sSeg = reinterpret_cast<float *>(sm + S::seg);
+  uint32_t *sTmem = reinterpret_cast<uint32_t *>(sm + S::misc);
+  uint64_t *sMbar = reinterpret_cast<uint64_t *>(sm + S::misc + 8);
+  int *sErr = reinterpret_cast<int *>(sm + S::misc + 16);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t h = blockIdx.x, b = blockIdx.y;
+  const int64_t L = p.L, H = p.H, G = p.G;
+  const int K = (int)p.K;
+  const int64_t g = h / (H / G);
+  const float Dh = p.Dp ? p.Dp[h] : 0.f;
+  const int64_t nc = (L + kQ - 1) / kQ;
+  const bf16 *x_g = static_cast<const bf16 *>(p.x);
+  const bf16 *al_g = static_cast<const bf16 *>(p.alpha);
+  const bf16 *be_g = static_cast<const bf16 *>(p.beta);
+  const bf16 *ga_g = static_cast<const bf16 *>(p.gamma);
+  const bf16 *th_g = static_cast<const bf16 *>(p.theta);
+  const bf16 *z_g = static_cast<const bf16 *>(p.z);
+  bf16 *out_g = static_cast<bf16 *>(p.out);
+  const uint32_t base = umma::smem_addr(sm);
+  const uint32_t mbar = umma::smem_addr(sMbar);
+
+  // Roles.  Rotation: step sg * 8 + ri of the chunk, angle pairs rq + 4 j.
+  // Accumulator rows: lanes 0..15 of warp w hold row r = 16 (w % 4) + lane
+  // (TMEM lane quarter w % 4) and the column half cb = w / 4.
+  const int sg = warp, ri = lane >> 2, rq = lane & 3;
+  const int r = 16 * (warp & 3) + (lane & 15), cb = warp >> 2;
+  const bool rlive = lane < 16;
+  const bool srow = rlive && r < P;
+  const uint32_t tq = (uint32_t)(32 * (warp & 3)) << 16;
+
+  if (warp == 0) umma::tmem_alloc(sTmem, 256);
+  if (tid == 0) {
+    umma::mbar_init(mbar);
+    *sErr = 0;
+  }
+  // the state: row r of S, columns cb * kK .. cb * kK + kK - 1
+  float sreg[kK];
+#pragma unroll
+  for (int j = 0; j < kK; ++j) {
+    const int n = cb * kK + j;
+    sreg[j] = (srow && p.h0) ? p.h0[((b * H + h) * P + r) * N + n] : 0.f;
+  }
+  if (srow) {
+#pragma unroll
+    for (int q = 0; q < kK / 8; ++q) put3x8(sm + S::sp, S::kSp, koff(r, cb * kK + 8 * q, N), sreg + 8 * q);
+  }
+  for (int i = tid; i < 2 * P; i += kThreads) sXprev[i] = 0.f;
+  for (int i = tid; i < 2 * N; i += kThreads) sBprev[i] = 0.f;
+  for (int i = tid; i < kK; i += kThreads) sPhi0[i] = 0.f;
+  // rows P..63 of X^T take part in dS (rows of the result that are dropped)
+  for (int i = tid; i < (64 - P) * 64 / 8; i += kThreads)
+    *reinterpret_cast<uint4 *>(sm + S::xp + P * 128 + i * 16) = make_uint4(0, 0, 0, 0);
+
+  // next chunk's theta (rotation roles) and alpha, beta, gamma (warp 0, steps 2 lane, 2 lane + 1)
+  float thv[kJ];
+  float pa0, pa1, pb0, pb1, pg0, pg1;
+  auto load_small = [&](int64_t t0) {
+    const int64_t t = t0 + sg * 8 + ri;
+#pragma unroll
+    for (int j = 0; j < kJ; ++j) {
+      const int k = rq + 4 * j;
+      thv[j] = (k < K && t < L) ? __bfloat162float(th_g[((b * L + t) * H + h) * K + k]) : 0.f;
+    }
+    pa0 = pa1 = 1.f;
+    pb0 = pb1 = pg0 = pg1 = 0.f;
+    if (warp == 0) {
+      const int64_t s = t0 + 2 * lane;
+      if (s < L) {
+        const int64_t j = (b * L + s) * H + h;
+        pa0 = __bfloat162float(al_g[j]);
+        pb0 = __bfloat162float(be_g[j]);
+        pg0 = __bfloat162float(ga_g[j]);
+      }
+      if (s + 1 < L) {
+        const int64_t j = (b * L + s + 1) * H + h;
+        pa1 = __bfloat162float(al_g[j]);
+        pb1 = __bfloat162float(be_g[j]);
+        pg1 = __bfloat162float(ga_g[j]);
+      }
+    }
+  };
+  um_issue_raw<P, N>(p, sm, b, h, g, 0);
+  load_small(0);
+  umma::fence_before();
+  __syncthreads();
+  umma::fence_after();
+  const uint32_t tmem = *sTmem;
+  float2 brot[kJ];  // this lane's rotated B pairs
+
+  for (int64_t ch = 0; ch < nc; ++ch) {
+    const int64_t t0 = ch * kQ;
+    const int Qc = (int)((L - t0) < kQ ? (L - t0) : kQ);
+    const int cur = (int)(ch & 1);
+    const float *xp_c = sXprev + cur * P, *bp_c = sBprev + cur * N;
+    float *xp_n = sXprev + (cur ^ 1) * P, *bp_n = sBprev + (cur ^ 1) * N;
+    cp_async_wait<0>();
+    __syncthreads();  // (A) this chunk's raw inputs are in; the last chunk is done
+    if (*sErr) break;
+
+    // ---- 1. state and angles entering the chunk; X^T; per-step vectors; angle scan
+    if (p.saved) {
+      if (srow) {
+        float *dst = p.saved + (((b * H + h) * nc + ch) * P + r) * N + cb * kK;
+#pragma unroll
+        for (int q = 0; q < kK / 4; ++q)
+          reinterpret_cast<float4 *>(dst)[q] =
+              make_float4(sreg[4 * q], sreg[4 * q + 1], sreg[4 * q + 2], sreg[4 * q + 3]);
+      }
+      float *ang = p.saved + p.B * H * nc * P * N + ((b * H + h) * nc + ch) * kK;
+      if (tid < kK) ang[tid] = sPhi0[tid];
+    }
+    for (int u = tid; u < P * 8; u += kThreads) {
+      const int pp = u % P, t8 = u / P;
+      const bf16 *src = reinterpret_cast<const bf16 *>(sm + S::rx) + t8 * 8 * P + pp;
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) w[e] = bf16pair(src[2 * e * P], src[(2 * e + 1) * P]);
+      *reinterpret_cast<uint4 *>(sm + S::xp + koff(pp, t8 * 8, 64)) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    for (int i = tid; i < P; i += kThreads)
+      xp_n[i] = __bfloat162float(reinterpret_cast<const bf16 *>(sm + S::rx)[(Qc - 1) * P + i]);
+    if (warp == 0) {
+      const int s0 = 2 * lane;
+      sAl[s0] = pa0; sAl[s0 + 1] = pa1;
+      sBe[s0] = pb0; sBe[s0 + 1] = pb1;
+      sGa[s0] = pg0; sGa[s0 + 1] = pg1;
+      // inclusive scan of log2(alpha)
+      float la0, la1;
+      asm("lg2.approx.f32 %0, %1;" : "=f"(la0) : "f"(pa0));
+      asm("lg2.approx.f32 %0, %1;" : "=f"(la1) : "f"(pa1));
+      la0 = fmaxf(la0, -126.f);
+      la1 = fmaxf(la1, -126.f);
+      float incl = la0 + la1;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const float v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
+      }
+      float excl = __shfl_up_sync(0xffffffffu, incl, 1);
+      if (lane == 0) excl = 0.f;
+      sLc[s0] = excl + la0;
+      sLc[s0 + 1] = incl;
+      __syncwarp();
+      const float lcl = sLc[kQ - 1];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int t = s0 + e;
+        const float ev = t + 1 < kQ ? fmaf(sAl[t + 1], sGa[t], sBe[t + 1]) : 0.f;
+        sDl[t] = ex2(sLc[t]);
+        sEv[t] = ev;
+        sCrow[t] = t + 1 < kQ ? ex2(lcl - sLc[t + 1]) * ev : sGa[t];
+      }
+    }
+    // theta: inclusive sums over this warp's 8 steps, per angle; the totals
+#pragma unroll
+    for (int j = 0; j < kJ; ++j) {
+      float v = thv[j];
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        const float u = __shfl_up_sync(0xffffffffu, v, off);
+        if (lane >= off) v += u;
+      }
+      thv[j] = v;
+      if (ri == 7) sSeg[sg * kK + rq + 4 * j] = v;
+    }
+    __syncthreads();  // (B)
+
+    // ---- 2. rotate B and C by the cumulative angles into the Bt and Ct planes
+    {
+      const int t = sg * 8 + ri;
+      const unsigned char *rb = sm + S::rB + t * S::kRS, *rc = sm + S::rC + t * S::kRS;
+      float dot = 0.f;
+#pragma unroll
+      for (int j = 0; j < kJ; ++j) {
+        const int k = rq + 4 * j;
+        float b0, b1, c0, c1;
+        unpack_bf16x2(*reinterpret_cast<const uint32_t *>(rb + 4 * k), b0, b1);
+        unpack_bf16x2(*reinterpret_cast<const uint32_t *>(rc + 4 * k), c0, c1);
+        if (k < K) {
+          float phi = sPhi0[k];
+          for (int s2 = 0; s2 < sg; ++s2) phi += sSeg[s2 * kK + k];
+          phi += thv[j];
+          float sn, cs;
+          sincosf(phi, &sn, &cs);
+          const float rb0 = cs * b0 - sn * b1, rb1 = sn * b0 + cs * b1;
+          const float rc0 = cs * c0 - sn * c1, rc1 = sn * c0 + cs * c1;
+          b0 = rb0; b1 = rb1; c0 = rc0; c1 = rc1;
+        }
+        brot[j] = make_float2(b0, b1);
+        put3x2(sm + S::bt, S::kBt, koff(t, 2 * k, N), b0, b1);
+        put3x2(sm + S::cw, S::kCW, koff(t, 2 * k, N), c0, c1);
+        dot = fmaf(c0, bp_c[2 * k], fmaf(c1, bp_c[2 * k + 1], dot));
+        if (t == Qc - 1) {
+          bp_n[2 * k] = b0;
+          bp_n[2 * k + 1] = b1;
+        }
+      }
+      dot += __shfl_xor_sync(0xffffffffu, dot, 1);
+      dot += __shfl_xor_sync(0xffffffffu, dot, 2);
+      if (rq == 0) sWcd[t] = dot;
+    }
+    umma::fence_async_smem();
+    __syncthreads();  // (C) operands of round 1 in place; raw stage consumed
+
+    if (tid == 0) {
+      umma::fence_after();
+      issue_product<64, false>(tmem, 0, base + S::cw, S::kCW, 3, N, base + S::bt, S::kBt, 3, N, N);
+      issue_product<P, false>(tmem, 64, base + S::cw, S::kCW, 3, N, base + S::sp, S::kSp, 3, N, N);
+      umma::commit(mbar);
+    }
+    if (ch + 1 < nc) {
+      um_issue_raw<P, N>(p, sm, b, h, g, t0 + kQ);
+      load_small(t0 + kQ);
+    }
+    if (tid < kK) {  // angles after this chunk
+      float phi = sPhi0[tid];
+#pragma unroll
+      for (int s2 = 0; s2 < 8; ++s2) phi += sSeg[s2 * kK + tid];
+      sPhi0[tid] = phi;
+    }
+
+    // ---- 3. W = c o G over Ct's planes; Bc = diag(c(Q-1, .)) Bt over Bt's planes
+    if (!umma::mbar_wait(mbar, 0)) *sErr = 1;
+    umma::fence_after();
+    {
+      const int t = r;
+      const float lct = sLc[t], gt = sGa[t];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float gv[8];
+        umma::tmem_ld8(tmem + tq + cb * 32 + 8 * q, gv);
+        if (rlive) {
+          float wv[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int s = cb * 32 + 8 * q + e;
+            wv[e] = s == t ? gt * gv[e] : (s < t ? ex2(lct - sLc[s + 1]) * sEv[s] * gv[e] : 0.f);
+          }
+          put3x8(sm + S::cw, S::kCW, koff(t, cb * 32 + 8 * q, 64), wv);
+        }
+      }
+    }
+    {
+      const int t = sg * 8 + ri;
+      const float cr = sCrow[t];
+#pragma unroll
+      for (int j = 0; j < kJ; ++j)
+        put3x2(sm + S::bt, S::kBt, koff(t, 2 * (rq + 4 * j), N), cr * brot[j].x, cr * brot[j].y);
+    }
+    umma::fence_async_smem();
+    umma::fence_before();
+    __syncthreads();  // (D) operands of round 2 in place
+    if (*sErr) break;
+    if (tid == 0) {
+      umma::fence_after();
+      issue_product<P, false>(tmem, 128, base + S::cw, S::kCW, 3, 64, base + S::xp, 0, 1, 64, 64);
+      issue_product<N, true>(tmem, 192, base + S::xp, 0, 1, 64, base + S::bt, S::kBt, 3, N, 64);
+      umma::commit(mbar);
+    }
+
+    // ---- 4. outputs; the state update
+    if (!umma::mbar_wait(mbar, 1)) *sErr = 1;
+    umma::fence_after();
+    {
+      const int t = r;
+      const float dlt = sDl[t], wct = sBe[0] * ex2(sLc[t] - sLc[0]) * sWcd[t];
+      const bool live = rlive && t < Qc;
+      const int64_t o = ((b * L + t0 + t) * H + h) * P + cb * (P / 2);
+#pragma unroll
+      for (int q = 0; q < P / 16; ++q) {
+        float y1[8], y2[8];
+        umma::tmem_ld8(tmem + tq + 64 + cb * (P / 2) + 8 * q, y1);
+        umma::tmem_ld8(tmem + tq + 128 + cb * (P / 2) + 8 * q, y2);
+        if (live) {
+          const uint4 xv = *reinterpret_cast<const uint4 *>(x_g + o + 8 * q);
+          float xf[8];
+          unpack_bf16x2(xv.x, xf[0], xf[1]);
+          unpack_bf16x2(xv.y, xf[2], xf[3]);
+          unpack_bf16x2(xv.z, xf[4], xf[5]);
+          unpack_bf16x2(xv.w, xf[6], xf[7]);
+          float y[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int pp = cb * (P / 2) + 8 * q + e;
+            y[e] = fmaf(dlt, y1[e], y2[e]) + wct * xp_c[pp] + Dh * xf[e];
+          }
+          if (z_g) {
+            const uint4 zv = *reinterpret_cast<const uint4 *>(z_g + o + 8 * q);
+            float zf[8];
+            unpack_bf16x2(zv.x, zf[0], zf[1]);
+            unpack_bf16x2(zv.y, zf[2], zf[3]);
+            unpack_bf16x2(zv.z, zf[4], zf[5]);
+            unpack_bf16x2(zv.w, zf[6], zf[7]);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) y[e] *= silu(zf[e]);
+          }
+          *reinterpret_cast<uint4 *>(out_g + o + 8 * q) =
+              make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
+                         pack_bf16x2(y[6], y[7]));
+        }
+      }
+    }
+    {
+      const float dlast = sDl[kQ - 1], w0 = sBe[0] * ex2(sLc[kQ - 1] - sLc[0]);
+      const float wx = srow ? w0 * xp_c[r] : 0.f;
+#pragma unroll
+      for (int q = 0; q < kK / 8; ++q) {
+        float dv[8];
+        umma::tmem_ld8(tmem + tq + 192 + cb * kK + 8 * q, dv);
+        if (srow) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            float &sv = sreg[8 * q + e];
+            sv = fmaf(dlast, sv, wx * bp_c[cb * kK + 8 * q + e]) + dv[e];
+          }
+          put3x8(sm + S::sp, S::kSp, koff(r, cb * kK + 8 * q, N), sreg + 8 * q);
+        }
+      }
+    }
+    umma::fence_async_smem();
+    umma::fence_before();
+  }
+
+  cp_async_wait<0>();
+  __syncthreads();
+  const bool failed = *sErr != 0;
+  if (p.final_state && srow) {
+    float *dst = p.final_state + ((b * H + h) * P + r) * N + cb * kK;
+    const float nan = __int_as_float(0x7fc00000);
+#pragma unroll
+    for (int q = 0; q < kK / 4; ++q)
+      reinterpret_cast<float4 *>(dst)[q] =
+          failed ? make_float4(nan, nan, nan, nan)
+                 : make_float4(sreg[4 * q], sreg[4 * q + 1], sreg[4 * q + 2], sreg[4 * q + 3]);
+  }
+  if (failed) {  // a tensor-core round never completed: the outputs of this (b, h) are NaN
+    const bf16 qnan = __ushort_as_bfloat16((unsigned short)0x7fc0);
+    for (int64_t i = tid; i < L * P; i += kThreads)
+      out_g[((b * L + i / P) * H + h) * P + i % P] = qnan;
+  }
+  umma::fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    umma::fence_after();
+    umma::tmem_dealloc(tmem, 256);
+  }
+}
+
+template <int P, int N>
+cudaError_t launch_um(const M3Params &p, cudaStream_t s) {
+  // at least 80 KB of shared memory per CTA, so that no more than two CTAs
+  // (2 x 256 TMEM columns) share an SM
+  const size_t smem = UmFwdSmem<P, N>::total > 80 * 1024 ? (size_t)UmFwdSmem<P, N>::total : 80 * 1024;
+  cudaError_t e = cudaFuncSetAttribute(m3_fwd_umma_kernel<P, N>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  m3_fwd_umma_kernel<P, N><<<dim3((unsigned)p.H, (unsigned)p.B), kThreads, smem, s>>>(p);
+  return cudaGetLastError();
+}
+
+template <int P>
+cudaError_t launch_um_n(const M3Params &p, cudaStream_t s) {
+  switch (p.N) {
+    case 16: return launch_um<P, 16>(p, s);
+    case 32: return launch_um<P, 32>(p, s);
+    default: return launch_um<P, 64>(p, s);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_m3_fwd_umma(const M3Params &p, cudaStream_t s) {
+  switch (p.P) {
+    case 16: return launch_um_n<16>(p, s);
+    case 32: return launch_um_n<32>(p, s);
+    default: return launch_um_n<64>(p, s);
+  }
+}
+
+}  // namespace msc
