@@ -42,7 +42,8 @@ using umma::koff;
 template <int P, int N>
 struct UmFwdSmem {
   static constexpr int kK = N / 2;
-  static constexpr int kRS = N * 2 + 16;   // raw B, C row stride in bytes (padded: no bank conflicts)
+  static constexpr int kG = kK / 4;         // groups of 4 angle pairs
+  static constexpr int kRS = N * 2 + 16;    // raw B, C row stride in bytes (padded: no bank conflicts)
   // bytes; bf16 part planes, K-major core-matrix layout (umma.cuh)
   static constexpr int kCW = 64 * 64 * 2;  // one part of Ct (K = N) or W (K = Q)
   static constexpr int kBt = 64 * N * 2;   // one part of Bt / Bc [s][n]
@@ -57,10 +58,11 @@ struct UmFwdSmem {
   // f32 vectors
   static constexpr int vec = rC + 64 * kRS;
   static constexpr int al = vec, be = al + 256, ga = be + 256, lc = ga + 256, ev = lc + 256,
-                       dl = ev + 256, crow = dl + 256, wcd = crow + 256,
-                       xprev = wcd + 256,        // [2][P], by chunk parity
+                       dl = ev + 256, crow = dl + 256,
+                       wcd = crow + 256,           // [kG][Q] partial Ct_t . Bt_prev per angle group
+                       xprev = wcd + kG * 256,     // [2][P], by chunk parity
                        bprev = xprev + 2 * P * 4,  // [2][N]
-                       phi0 = bprev + 2 * N * 4, seg = phi0 + kK * 4, misc = seg + 8 * kK * 4;
+                       misc = bprev + 2 * N * 4;
   static constexpr int total = misc + 32;  // tmem slot, mbarrier, error flag
 };
 
@@ -100,28 +102,21 @@ __device__ __forceinline__ uint32_t bf16pair(bf16 lo, bf16 hi) {
 // (plane stride `stride`), one 4-byte store per plane
 __device__ __forceinline__ void put3x2(unsigned char *base, int stride, int off, float v0,
                                        float v1) {
-  bf16 a[3], c[3];
-  umma::split3(v0, a);
-  umma::split3(v1, c);
+  uint32_t w[3];
+  umma::split3x2(v0, v1, w);
 #pragma unroll
-  for (int q = 0; q < 3; ++q)
-    *reinterpret_cast<uint32_t *>(base + q * stride + off) = bf16pair(a[q], c[q]);
+  for (int q = 0; q < 3; ++q) *reinterpret_cast<uint32_t *>(base + q * stride + off) = w[q];
 }
 
-// the three parts of v[0..7] (one core-matrix row), one 16-byte store per plane
-__device__ __forceinline__ void put3x8(unsigned char *base, int stride, int off, const float *v) {
-  uint32_t w[3][4];
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    bf16 a[3], c[3];
-    umma::split3(v[2 * e], a);
-    umma::split3(v[2 * e + 1], c);
-#pragma unroll
-    for (int q = 0; q < 3; ++q) w[q][e] = bf16pair(a[q], c[q]);
-  }
-#pragma unroll
-  for (int q = 0; q < 3; ++q)
-    *reinterpret_cast<uint4 *>(base + q * stride + off) = make_uint4(w[q][0], w[q][1], w[q][2], w[q][3]);
+// sin and cos of a cumulative angle: Cody and Waite's additive reduction by
+// 2 pi, the constant split as 6.28125 (8 significant bits, so n * 6.28125 is
+// exact for |n| < 2^16) plus the remainder 2 pi - 6.28125, then the SFU's sin
+// and cos on [-pi, pi] (absolute error about 2^-21)
+__device__ __forceinline__ void sincos_reduced(float phi, float &sn, float &cs) {
+  const float n = rintf(phi * 0.15915494309189535f);
+  float r = fmaf(-n, 6.28125f, phi);
+  r = fmaf(-n, 1.9353071795864769e-3f, r);
+  __sincosf(r, &sn, &cs);
 }
 
 // Issue one product into TMEM column `col`: parts of A (nA of them, planes at
@@ -151,7 +146,11 @@ template <int P, int N>
 __global__ void __launch_bounds__(kThreads, 2) m3_fwd_umma_kernel(const M3Params p) {
   using S = UmFwdSmem<P, N>;
   constexpr int kK = N / 2;
-  constexpr int kJ = kK / 4;  // angle pairs per rotation lane
+  constexpr int kG = S::kG;    // angle groups
+  constexpr int kWG = 8 / kG;  // warps per angle group
+  constexpr int kM = 8 / kWG;  // 8-step segments a warp rotates
+  constexpr int kSR = kK / 8;  // 8-column blocks of a state row half
+  constexpr int kPR = P / 16;  // 8-column blocks of an output row half
   extern __shared__ __align__(1024) unsigned char sm[];
   float *sAl = reinterpret_cast<float *>(sm + S::al), *sBe = reinterpret_cast<float *>(sm + S::be);
   float *sGa = reinterpret_cast<float *>(sm + S::ga), *sLc = reinterpret_cast<float *>(sm + S::lc);
@@ -160,7 +159,6 @@ __global__ void __launch_bounds__(kThreads, 2) m3_fwd_umma_kernel(const M3Params
   float *sWcd = reinterpret_cast<float *>(sm + S::wcd);
   float *sXprev = reinterpret_cast<float *>(sm + S::xprev);
   float *sBprev = reinterpret_cast<float *>(sm + S::bprev);
-  float *sPhi0 = reinterpret_cast<float *>(sm + S::phi0), *sSeg = reinterpret_cast<float *>(sm + S::seg);
   uint32_t *sTmem = reinterpret_cast<uint32_t *>(sm + S::misc);
   uint64_t *sMbar = reinterpret_cast<uint64_t *>(sm + S::misc + 8);
   int *sErr = reinterpret_cast<int *>(sm + S::misc + 16);
@@ -182,47 +180,69 @@ __global__ void __launch_bounds__(kThreads, 2) m3_fwd_umma_kernel(const M3Params
   const uint32_t base = umma::smem_addr(sm);
   const uint32_t mbar = umma::smem_addr(sMbar);
 
-  // Roles.  Rotation: step sg * 8 + ri of the chunk, angle pairs rq + 4 j.
-  // Accumulator rows: lanes 0..15 of warp w hold row r = 16 (w % 4) + lane
-  // (TMEM lane quarter w % 4) and the column half cb = w / 4.
-  const int sg = warp, ri = lane >> 2, rq = lane & 3;
-  const int r = 16 * (warp & 3) + (lane & 15), cb = warp >> 2;
-  const bool rlive = lane < 16;
-  const bool srow = rlive && r < P;
-  const uint32_t tq = (uint32_t)(32 * (warp & 3)) << 16;
+  // Roles.  Angles: lane (ri, rq) = (lane / 4, lane % 4) of warp w holds
+  // angle pair ka = 4 (w % kG) + rq at steps 8 m + ri of the chunk, for all
+  // eight segments m, and rotates segments sp kM .. sp kM + kM - 1 (sp = w /
+  // kG).  Accumulators: warp w reads rows ra = 16 (w % 4) + ri and rb = ra + 8
+  // (TMEM lane quarter w % 4), column half cb = w / 4, columns 2 rq, 2 rq + 1
+  // of each 8-column block.
+  const int ri = lane >> 2, rq = lane & 3;
+  const int ag = warp % kG, sp = warp / kG;
+  const int ka = 4 * ag + rq;
+  const int q4 = warp & 3, cb = warp >> 2;
+  const int ra = 16 * q4 + ri, rb = ra + 8, c2 = 2 * rq;
+  const bool srow = 16 * q4 < P;
+  const uint32_t tq = (uint32_t)(32 * q4) << 16;
 
   if (warp == 0) umma::tmem_alloc(sTmem, 256);
   if (tid == 0) {
     umma::mbar_init(mbar);
     *sErr = 0;
   }
-  // the state: row r of S, columns cb * kK .. cb * kK + kK - 1
-  float sreg[kK];
+  // the state: rows ra (sreg[4 i], [4 i + 1]) and rb (sreg[4 i + 2], [4 i + 3]),
+  // columns cb * kK + 8 i + c2 + 0, 1
+  float sreg[kK / 2];
+  const float *h0 = p.h0 ? p.h0 + (b * H + h) * P * N : nullptr;
 #pragma unroll
-  for (int j = 0; j < kK; ++j) {
-    const int n = cb * kK + j;
-    sreg[j] = (srow && p.h0) ? p.h0[((b * H + h) * P + r) * N + n] : 0.f;
+  for (int i = 0; i < kSR; ++i) {
+    const int n = cb * kK + 8 * i + c2;
+    const float2 va = (srow && h0) ? *reinterpret_cast<const float2 *>(h0 + ra * N + n) : make_float2(0.f, 0.f);
+    const float2 vb = (srow && h0) ? *reinterpret_cast<const float2 *>(h0 + rb * N + n) : make_float2(0.f, 0.f);
+    sreg[4 * i] = va.x; sreg[4 * i + 1] = va.y;
+    sreg[4 * i + 2] = vb.x; sreg[4 * i + 3] = vb.y;
   }
-  if (srow) {
+  auto put_state = [&]() {
 #pragma unroll
-    for (int q = 0; q < kK / 8; ++q) put3x8(sm + S::sp, S::kSp, koff(r, cb * kK + 8 * q, N), sreg + 8 * q);
-  }
+    for (int i = 0; i < kSR; ++i) {
+      const int n = cb * kK + 8 * i + c2;
+      put3x2(sm + S::sp, S::kSp, koff(ra, n, N), sreg[4 * i], sreg[4 * i + 1]);
+      put3x2(sm + S::sp, S::kSp, koff(rb, n, N), sreg[4 * i + 2], sreg[4 * i + 3]);
+    }
+  };
+  auto store_state = [&](float *dst) {  // dst: this (b, h)'s P x N block
+#pragma unroll
+    for (int i = 0; i < kSR; ++i) {
+      const int n = cb * kK + 8 * i + c2;
+      *reinterpret_cast<float2 *>(dst + ra * N + n) = make_float2(sreg[4 * i], sreg[4 * i + 1]);
+      *reinterpret_cast<float2 *>(dst + rb * N + n) = make_float2(sreg[4 * i + 2], sreg[4 * i + 3]);
+    }
+  };
+  if (srow) put_state();
   for (int i = tid; i < 2 * P; i += kThreads) sXprev[i] = 0.f;
   for (int i = tid; i < 2 * N; i += kThreads) sBprev[i] = 0.f;
-  for (int i = tid; i < kK; i += kThreads) sPhi0[i] = 0.f;
   // rows P..63 of X^T take part in dS (rows of the result that are dropped)
   for (int i = tid; i < (64 - P) * 64 / 8; i += kThreads)
     *reinterpret_cast<uint4 *>(sm + S::xp + P * 128 + i * 16) = make_uint4(0, 0, 0, 0);
 
-  // next chunk's theta (rotation roles) and alpha, beta, gamma (warp 0, steps 2 lane, 2 lane + 1)
-  float thv[kJ];
+  // the next chunk's theta (angle roles) and alpha, beta, gamma (warp 0: steps
+  // 2 lane, 2 lane + 1)
+  float thv[8];
   float pa0, pa1, pb0, pb1, pg0, pg1;
   auto load_small = [&](int64_t t0) {
-    const int64_t t = t0 + sg * 8 + ri;
 #pragma unroll
-    for (int j = 0; j < kJ; ++j) {
-      const int k = rq + 4 * j;
-      thv[j] = (k < K && t < L) ? __bfloat162float(th_g[((b * L + t) * H + h) * K + k]) : 0.f;
+    for (int m = 0; m < 8; ++m) {
+      const int64_t t = t0 + 8 * m + ri;
+      thv[m] = (ka < K && t < L) ? __bfloat162float(th_g[((b * L + t) * H + h) * K + ka]) : 0.f;
     }
     pa0 = pa1 = 1.f;
     pb0 = pb1 = pg0 = pg1 = 0.f;
@@ -248,7 +268,8 @@ __global__ void __launch_bounds__(kThreads, 2) m3_fwd_umma_kernel(const M3Params
   __syncthreads();
   umma::fence_after();
   const uint32_t tmem = *sTmem;
-  float2 brot[kJ];  // this lane's rotated B pairs
+  float phi_c = 0.f;  // cumulative angle of pair ka before the chunk
+  float2 brot[8];     // rotated B of pair ka at steps 8 m + ri (this warp's segments)
 
   for (int64_t ch = 0; ch < nc; ++ch) {
     const int64_t t0 = ch * kQ;
@@ -260,17 +281,11 @@ __global__ void __launch_bounds__(kThreads, 2) m3_fwd_umma_kernel(const M3Params
     __syncthreads();  // (A) this chunk's raw inputs are in; the last chunk is done
     if (*sErr) break;
 
-    // ---- 1. state and angles entering the chunk; X^T; per-step vectors; angle scan
+    // ---- 1. state and angles entering the chunk; X^T; per-step vectors ----------
     if (p.saved) {
-      if (srow) {
-        float *dst = p.saved + (((b * H + h) * nc + ch) * P + r) * N + cb * kK;
-#pragma unroll
-        for (int q = 0; q < kK / 4; ++q)
-          reinterpret_cast<float4 *>(dst)[q] =
-              make_float4(sreg[4 * q], sreg[4 * q + 1], sreg[4 * q + 2], sreg[4 * q + 3]);
-      }
-      float *ang = p.saved + p.B * H * nc * P * N + ((b * H + h) * nc + ch) * kK;
-      if (tid < kK) ang[tid] = sPhi0[tid];
+      if (srow) store_state(p.saved + ((b * H + h) * nc + ch) * P * N);
+      if (sp == 0 && ri == 0)
+        p.saved[p.B * H * nc * P * N + ((b * H + h) * nc + ch) * kK + ka] = phi_c;
     }
     for (int u = tid; u < P * 8; u += kThreads) {
       const int pp = u % P, t8 = u / P;
@@ -314,53 +329,51 @@ __global__ void __launch_bounds__(kThreads, 2) m3_fwd_umma_kernel(const M3Params
         sCrow[t] = t + 1 < kQ ? ex2(lcl - sLc[t + 1]) * ev : sGa[t];
       }
     }
-    // theta: inclusive sums over this warp's 8 steps, per angle; the totals
-#pragma unroll
-    for (int j = 0; j < kJ; ++j) {
-      float v = thv[j];
-#pragma unroll
-      for (int off = 4; off < 32; off <<= 1) {
-        const float u = __shfl_up_sync(0xffffffffu, v, off);
-        if (lane >= off) v += u;
-      }
-      thv[j] = v;
-      if (ri == 7) sSeg[sg * kK + rq + 4 * j] = v;
-    }
-    __syncthreads();  // (B)
 
-    // ---- 2. rotate B and C by the cumulative angles into the Bt and Ct planes
+    // ---- 2. cumulative angles; rotate B and C into the Bt and Ct planes ------------
     {
-      const int t = sg * 8 + ri;
-      const unsigned char *rb = sm + S::rB + t * S::kRS, *rc = sm + S::rC + t * S::kRS;
-      float dot = 0.f;
+      float T[8];  // segment totals
 #pragma unroll
-      for (int j = 0; j < kJ; ++j) {
-        const int k = rq + 4 * j;
-        float b0, b1, c0, c1;
-        unpack_bf16x2(*reinterpret_cast<const uint32_t *>(rb + 4 * k), b0, b1);
-        unpack_bf16x2(*reinterpret_cast<const uint32_t *>(rc + 4 * k), c0, c1);
-        if (k < K) {
-          float phi = sPhi0[k];
-          for (int s2 = 0; s2 < sg; ++s2) phi += sSeg[s2 * kK + k];
-          phi += thv[j];
-          float sn, cs;
-          sincosf(phi, &sn, &cs);
-          const float rb0 = cs * b0 - sn * b1, rb1 = sn * b0 + cs * b1;
-          const float rc0 = cs * c0 - sn * c1, rc1 = sn * c0 + cs * c1;
-          b0 = rb0; b1 = rb1; c0 = rc0; c1 = rc1;
+      for (int m = 0; m < 8; ++m) {
+        float v = thv[m];
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+          const float u = __shfl_up_sync(0xffffffffu, v, off);
+          if (lane >= off) v += u;
         }
-        brot[j] = make_float2(b0, b1);
-        put3x2(sm + S::bt, S::kBt, koff(t, 2 * k, N), b0, b1);
-        put3x2(sm + S::cw, S::kCW, koff(t, 2 * k, N), c0, c1);
-        dot = fmaf(c0, bp_c[2 * k], fmaf(c1, bp_c[2 * k + 1], dot));
-        if (t == Qc - 1) {
-          bp_n[2 * k] = b0;
-          bp_n[2 * k + 1] = b1;
-        }
+        thv[m] = v;  // inclusive within segment m
+        T[m] = __shfl_sync(0xffffffffu, v, 28 + rq);
       }
-      dot += __shfl_xor_sync(0xffffffffu, dot, 1);
-      dot += __shfl_xor_sync(0xffffffffu, dot, 2);
-      if (rq == 0) sWcd[t] = dot;
+      float phi = phi_c;
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        if (m >= sp * kM && m < sp * kM + kM) {
+          const int t = 8 * m + ri;
+          float b0, b1, c0, c1;
+          unpack_bf16x2(*reinterpret_cast<const uint32_t *>(sm + S::rB + t * S::kRS + 4 * ka), b0, b1);
+          unpack_bf16x2(*reinterpret_cast<const uint32_t *>(sm + S::rC + t * S::kRS + 4 * ka), c0, c1);
+          if (ka < K) {
+            float sn, cs;
+            sincos_reduced(phi + thv[m], sn, cs);
+            const float rb0 = cs * b0 - sn * b1, rb1 = sn * b0 + cs * b1;
+            const float rc0 = cs * c0 - sn * c1, rc1 = sn * c0 + cs * c1;
+            b0 = rb0; b1 = rb1; c0 = rc0; c1 = rc1;
+          }
+          brot[m] = make_float2(b0, b1);
+          put3x2(sm + S::bt, S::kBt, koff(t, 2 * ka, N), b0, b1);
+          put3x2(sm + S::cw, S::kCW, koff(t, 2 * ka, N), c0, c1);
+          float d = fmaf(c0, bp_c[2 * ka], c1 * bp_c[2 * ka + 1]);
+          d += __shfl_xor_sync(0xffffffffu, d, 1);
+          d += __shfl_xor_sync(0xffffffffu, d, 2);
+          if (rq == 0) sWcd[ag * kQ + t] = d;
+          if (t == Qc - 1) {
+            bp_n[2 * ka] = b0;
+            bp_n[2 * ka + 1] = b1;
+          }
+        }
+        phi += T[m];
+      }
+      phi_c = phi;
     }
     umma::fence_async_smem();
     __syncthreads();  // (C) operands of round 1 in place; raw stage consumed
@@ -375,40 +388,50 @@ __global__ void __launch_bounds__(kThreads, 2) m3_fwd_umma_kernel(const M3Params
       um_issue_raw<P, N>(p, sm, b, h, g, t0 + kQ);
       load_small(t0 + kQ);
     }
-    if (tid < kK) {  // angles after this chunk
-      float phi = sPhi0[tid];
+    // x and z of this thread's outputs (rows ra, rb)
+    uint32_t xo[2 * kPR], zo[2 * kPR];
 #pragma unroll
-      for (int s2 = 0; s2 < 8; ++s2) phi += sSeg[s2 * kK + tid];
-      sPhi0[tid] = phi;
-    }
+    for (int i = 0; i < kPR; ++i)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int t = e ? rb : ra;
+        const int64_t o = ((b * L + t0 + t) * H + h) * P + cb * (P / 2) + 8 * i + c2;
+        const bool in = t < Qc;
+        xo[2 * i + e] = in ? *reinterpret_cast<const uint32_t *>(x_g + o) : 0u;
+        zo[2 * i + e] = (in && z_g) ? *reinterpret_cast<const uint32_t *>(z_g + o) : 0u;
+      }
 
     // ---- 3. W = c o G over Ct's planes; Bc = diag(c(Q-1, .)) Bt over Bt's planes
     if (!umma::mbar_wait(mbar, 0)) *sErr = 1;
     umma::fence_after();
     {
-      const int t = r;
-      const float lct = sLc[t], gt = sGa[t];
+      float gv[16];
+      umma::tmem_ld16<4>(tmem + tq + cb * 32, gv);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        float gv[8];
-        umma::tmem_ld8(tmem + tq + cb * 32 + 8 * q, gv);
-        if (rlive) {
-          float wv[8];
+      for (int e = 0; e < 2; ++e) {
+        const int t = e ? rb : ra;
+        const float lct = sLc[t], gt = sGa[t];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int s = cb * 32 + 8 * q + e;
-            wv[e] = s == t ? gt * gv[e] : (s < t ? ex2(lct - sLc[s + 1]) * sEv[s] * gv[e] : 0.f);
+        for (int i = 0; i < 4; ++i) {
+          const int s0 = cb * 32 + 8 * i + c2;
+          float w[2];
+#pragma unroll
+          for (int f = 0; f < 2; ++f) {
+            const int s = s0 + f;
+            const float gval = gv[4 * i + 2 * e + f];
+            w[f] = s == t ? gt * gval : (s < t ? ex2(lct - sLc[s + 1]) * sEv[s] * gval : 0.f);
           }
-          put3x8(sm + S::cw, S::kCW, koff(t, cb * 32 + 8 * q, 64), wv);
+          put3x2(sm + S::cw, S::kCW, koff(t, s0, 64), w[0], w[1]);
         }
       }
     }
-    {
-      const int t = sg * 8 + ri;
-      const float cr = sCrow[t];
 #pragma unroll
-      for (int j = 0; j < kJ; ++j)
-        put3x2(sm + S::bt, S::kBt, koff(t, 2 * (rq + 4 * j), N), cr * brot[j].x, cr * brot[j].y);
+    for (int m = 0; m < 8; ++m) {
+      if (m >= sp * kM && m < sp * kM + kM) {
+        const int t = 8 * m + ri;
+        const float cr = sCrow[t];
+        put3x2(sm + S::bt, S::kBt, koff(t, 2 * ka, N), cr * brot[m].x, cr * brot[m].y);
+      }
     }
     umma::fence_async_smem();
     umma::fence_before();
@@ -421,63 +444,57 @@ __global__ void __launch_bounds__(kThreads, 2) m3_fwd_umma_kernel(const M3Params
       umma::commit(mbar);
     }
 
-    // ---- 4. outputs; the state update
+    // ---- 4. outputs; the state update ------------------------------------------------
     if (!umma::mbar_wait(mbar, 1)) *sErr = 1;
     umma::fence_after();
     {
-      const int t = r;
-      const float dlt = sDl[t], wct = sBe[0] * ex2(sLc[t] - sLc[0]) * sWcd[t];
-      const bool live = rlive && t < Qc;
-      const int64_t o = ((b * L + t0 + t) * H + h) * P + cb * (P / 2);
+      float y1[4 * kPR], y2[4 * kPR];
+      umma::tmem_ld16_pair<kPR>(tmem + tq + 64 + cb * (P / 2), tmem + tq + 128 + cb * (P / 2), y1, y2);
 #pragma unroll
-      for (int q = 0; q < P / 16; ++q) {
-        float y1[8], y2[8];
-        umma::tmem_ld8(tmem + tq + 64 + cb * (P / 2) + 8 * q, y1);
-        umma::tmem_ld8(tmem + tq + 128 + cb * (P / 2) + 8 * q, y2);
-        if (live) {
-          const uint4 xv = *reinterpret_cast<const uint4 *>(x_g + o + 8 * q);
-          float xf[8];
-          unpack_bf16x2(xv.x, xf[0], xf[1]);
-          unpack_bf16x2(xv.y, xf[2], xf[3]);
-          unpack_bf16x2(xv.z, xf[4], xf[5]);
-          unpack_bf16x2(xv.w, xf[6], xf[7]);
-          float y[8];
+      for (int e = 0; e < 2; ++e) {
+        const int t = e ? rb : ra;
+        if (t < Qc) {
+          float wcd = 0.f;
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int pp = cb * (P / 2) + 8 * q + e;
-            y[e] = fmaf(dlt, y1[e], y2[e]) + wct * xp_c[pp] + Dh * xf[e];
+          for (int a = 0; a < kG; ++a) wcd += sWcd[a * kQ + t];
+          const float dlt = sDl[t], wct = sBe[0] * ex2(sLc[t] - sLc[0]) * wcd;
+#pragma unroll
+          for (int i = 0; i < kPR; ++i) {
+            const int p0 = cb * (P / 2) + 8 * i + c2;
+            float xf0, xf1;
+            unpack_bf16x2(xo[2 * i + e], xf0, xf1);
+            float o0 = fmaf(dlt, y1[4 * i + 2 * e], y2[4 * i + 2 * e]) + wct * xp_c[p0] + Dh * xf0;
+            float o1 = fmaf(dlt, y1[4 * i + 2 * e + 1], y2[4 * i + 2 * e + 1]) + wct * xp_c[p0 + 1] + Dh * xf1;
+            if (z_g) {
+              float zf0, zf1;
+              unpack_bf16x2(zo[2 * i + e], zf0, zf1);
+              o0 *= silu(zf0);
+              o1 *= silu(zf1);
+            }
+            *reinterpret_cast<uint32_t *>(out_g + ((b * L + t0 + t) * H + h) * P + p0) = pack_bf16x2(o0, o1);
           }
-          if (z_g) {
-            const uint4 zv = *reinterpret_cast<const uint4 *>(z_g + o + 8 * q);
-            float zf[8];
-            unpack_bf16x2(zv.x, zf[0], zf[1]);
-            unpack_bf16x2(zv.y, zf[2], zf[3]);
-            unpack_bf16x2(zv.z, zf[4], zf[5]);
-            unpack_bf16x2(zv.w, zf[6], zf[7]);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) y[e] *= silu(zf[e]);
-          }
-          *reinterpret_cast<uint4 *>(out_g + o + 8 * q) =
-              make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
-                         pack_bf16x2(y[6], y[7]));
         }
       }
     }
     {
-      const float dlast = sDl[kQ - 1], w0 = sBe[0] * ex2(sLc[kQ - 1] - sLc[0]);
-      const float wx = srow ? w0 * xp_c[r] : 0.f;
+      float dv[kK / 2];
+      umma::tmem_ld16<kSR>(tmem + tq + 192 + cb * kK, dv);
+      if (srow) {
+        const float dlast = sDl[kQ - 1], w0 = sBe[0] * ex2(sLc[kQ - 1] - sLc[0]);
 #pragma unroll
-      for (int q = 0; q < kK / 8; ++q) {
-        float dv[8];
-        umma::tmem_ld8(tmem + tq + 192 + cb * kK + 8 * q, dv);
-        if (srow) {
+        for (int e = 0; e < 2; ++e) {
+          const float wx = w0 * xp_c[e ? rb : ra];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            float &sv = sreg[8 * q + e];
-            sv = fmaf(dlast, sv, wx * bp_c[cb * kK + 8 * q + e]) + dv[e];
+          for (int i = 0; i < kSR; ++i) {
+            const int n = cb * kK + 8 * i + c2;
+#pragma unroll
+            for (int f = 0; f < 2; ++f) {
+              float &sv = sreg[4 * i + 2 * e + f];
+              sv = fmaf(dlast, sv, wx * bp_c[n + f]) + dv[4 * i + 2 * e + f];
+            }
           }
-          put3x8(sm + S::sp, S::kSp, koff(r, cb * kK + 8 * q, N), sreg + 8 * q);
         }
+        put_state();
       }
     }
     umma::fence_async_smem();
@@ -488,13 +505,11 @@ __global__ void __launch_bounds__(kThreads, 2) m3_fwd_umma_kernel(const M3Params
   __syncthreads();
   const bool failed = *sErr != 0;
   if (p.final_state && srow) {
-    float *dst = p.final_state + ((b * H + h) * P + r) * N + cb * kK;
-    const float nan = __int_as_float(0x7fc00000);
+    if (failed) {
 #pragma unroll
-    for (int q = 0; q < kK / 4; ++q)
-      reinterpret_cast<float4 *>(dst)[q] =
-          failed ? make_float4(nan, nan, nan, nan)
-                 : make_float4(sreg[4 * q], sreg[4 * q + 1], sreg[4 * q + 2], sreg[4 * q + 3]);
+      for (int j = 0; j < kK / 2; ++j) sreg[j] = __int_as_float(0x7fc00000);
+    }
+    store_state(p.final_state + (b * H + h) * P * N);
   }
   if (failed) {  // a tensor-core round never completed: the outputs of this (b, h) are NaN
     const bf16 qnan = __ushort_as_bfloat16((unsigned short)0x7fc0);

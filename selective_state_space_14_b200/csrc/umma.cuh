@@ -18,9 +18,12 @@
 // Exact bf16 operands (the inputs) go as one part.
 //
 // Accumulators with M = 64 rows occupy TMEM lanes 16 w .. 16 w + 15 of each
-// 32-lane quarter w (row 16 w + i at lane 32 w + i); warp w of a CTA reads its
-// quarter w % 4 with tcgen05.ld.32x32b, lanes 0..15 of the warp receiving
-// rows 16 (w % 4) + lane.
+// 32-lane quarter w (row 16 w + i at lane 32 w + i).  Warp w of a CTA reads
+// the 16 rows of its quarter w % 4 with tcgen05.ld.16x256b, which spreads
+// them over all 32 threads: per block of 8 columns, thread i receives rows
+// i / 4 and 8 + i / 4 (of the 16), columns 2 (i % 4) and 2 (i % 4) + 1.
+// Each load and its tcgen05.wait::ld sit in one asm statement, so that no use
+// of the registers can be scheduled ahead of the wait.
 //
 // Every wait on an mbarrier is bounded; a wait that runs out reports failure
 // and the caller turns its outputs into NaN rather than hang.
@@ -113,27 +116,119 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols));
 }
 
-// 8 consecutive f32 columns of this warp's TMEM quarter: thread i gets lane
-// (32 (warp % 4) + i), columns col .. col + 7
-__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
+// 16 TMEM lanes x 8 R columns from the lane and column in taddr (tcgen05.ld
+// .16x256b.xR), waited for: per block c of 8 columns, thread i gets v[4 c],
+// v[4 c + 1] = (lane i / 4, columns 8 c + 2 (i % 4) + 0, 1) and v[4 c + 2],
+// v[4 c + 3] = (lane 8 + i / 4, the same columns).
+template <int R>
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float *v);
+// two such loads (ta into va, tb into vb) in flight together
+template <int R>
+__device__ __forceinline__ void tmem_ld16_pair(uint32_t ta, uint32_t tb, float *va, float *vb);
+
+template <>
+__device__ __forceinline__ void tmem_ld16<1>(uint32_t taddr, float *v) {
+  uint32_t r[4];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x1.b32 {%0,%1,%2,%3}, [%4];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 4; ++i) v[i] = __uint_as_float(r[i]);
+}
+template <>
+__device__ __forceinline__ void tmem_ld16_pair<1>(uint32_t ta, uint32_t tb, float *va, float *vb) {
+  uint32_t a[4], b[4];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x1.b32 {%0,%1,%2,%3}, [%8];\n\t"
+      "tcgen05.ld.sync.aligned.16x256b.x1.b32 {%4,%5,%6,%7}, [%9];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3]),
+        "=r"(b[0]), "=r"(b[1]), "=r"(b[2]), "=r"(b[3])
+      : "r"(ta), "r"(tb)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    va[i] = __uint_as_float(a[i]);
+    vb[i] = __uint_as_float(b[i]);
+  }
+}
+
+template <>
+__device__ __forceinline__ void tmem_ld16<2>(uint32_t taddr, float *v) {
   uint32_t r[8];
   asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+      "tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+      : "r"(taddr)
+      : "memory");
 #pragma unroll
   for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }
+template <>
+__device__ __forceinline__ void tmem_ld16_pair<2>(uint32_t ta, uint32_t tb, float *va, float *vb) {
+  uint32_t a[8], b[8];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%16];\n\t"
+      "tcgen05.ld.sync.aligned.16x256b.x2.b32 {%8,%9,%10,%11,%12,%13,%14,%15}, [%17];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3]), "=r"(a[4]), "=r"(a[5]), "=r"(a[6]), "=r"(a[7]),
+        "=r"(b[0]), "=r"(b[1]), "=r"(b[2]), "=r"(b[3]), "=r"(b[4]), "=r"(b[5]), "=r"(b[6]), "=r"(b[7])
+      : "r"(ta), "r"(tb)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    va[i] = __uint_as_float(a[i]);
+    vb[i] = __uint_as_float(b[i]);
+  }
+}
 
-// the three bf16 parts of v
-__device__ __forceinline__ void split3(float v, __nv_bfloat16 (&p)[3]) {
-  p[0] = __float2bfloat16_rn(v);
-  float r = v - __bfloat162float(p[0]);
-  p[1] = __float2bfloat16_rn(r);
-  r -= __bfloat162float(p[1]);
-  p[2] = __float2bfloat16_rn(r);
+template <>
+__device__ __forceinline__ void tmem_ld16<4>(uint32_t taddr, float *v) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x4.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+template <>
+__device__ __forceinline__ void tmem_ld16_pair<4>(uint32_t ta, uint32_t tb, float *va, float *vb) {
+  uint32_t a[16], b[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x4.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%32];\n\t"
+      "tcgen05.ld.sync.aligned.16x256b.x4.b32 {%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%33];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3]), "=r"(a[4]), "=r"(a[5]), "=r"(a[6]), "=r"(a[7]), "=r"(a[8]), "=r"(a[9]), "=r"(a[10]), "=r"(a[11]), "=r"(a[12]), "=r"(a[13]), "=r"(a[14]), "=r"(a[15]),
+        "=r"(b[0]), "=r"(b[1]), "=r"(b[2]), "=r"(b[3]), "=r"(b[4]), "=r"(b[5]), "=r"(b[6]), "=r"(b[7]), "=r"(b[8]), "=r"(b[9]), "=r"(b[10]), "=r"(b[11]), "=r"(b[12]), "=r"(b[13]), "=r"(b[14]), "=r"(b[15])
+      : "r"(ta), "r"(tb)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    va[i] = __uint_as_float(a[i]);
+    vb[i] = __uint_as_float(b[i]);
+  }
+}
+
+// the three bf16 parts of v0 and v1, packed per part: w[q] holds part q of
+// v0 in its low half and of v1 in its high half (the memory order of two
+// consecutive bf16)
+__device__ __forceinline__ void split3x2(float v0, float v1, uint32_t (&w)[3]) {
+  const __nv_bfloat162 p0 = __floats2bfloat162_rn(v0, v1);
+  const float2 f0 = __bfloat1622float2(p0);
+  const float r0 = v0 - f0.x, r1 = v1 - f0.y;
+  const __nv_bfloat162 p1 = __floats2bfloat162_rn(r0, r1);
+  const float2 f1 = __bfloat1622float2(p1);
+  const __nv_bfloat162 p2 = __floats2bfloat162_rn(r0 - f1.x, r1 - f1.y);
+  w[0] = *reinterpret_cast<const uint32_t *>(&p0);
+  w[1] = *reinterpret_cast<const uint32_t *>(&p1);
+  w[2] = *reinterpret_cast<const uint32_t *>(&p2);
 }
 
 }  // namespace umma
