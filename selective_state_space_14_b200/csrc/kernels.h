@@ -74,7 +74,6 @@ struct M3Params {
   size_t ws_bytes;
 };
 cudaError_t launch_m3_fwd(const M3Params &p, cudaStream_t s);
-cudaError_t launch_m3_fwd_tc(const M3Params &p, cudaStream_t s);    // bf16 io, mma.sync tf32
 cudaError_t launch_m3_fwd_umma(const M3Params &p, cudaStream_t s);  // bf16 io, tcgen05
 cudaError_t launch_m3_bwd(const M3Params &p, cudaStream_t s);
 size_t m3_bwd_workspace_bytes(int64_t B, int64_t L, int64_t H, int64_t P, int64_t N, int64_t G,

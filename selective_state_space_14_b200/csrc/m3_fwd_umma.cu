@@ -1,7 +1,7 @@
 // m3_fwd_umma.cu -- Mamba-3 SISO scan, forward, bf16 io, on the sm_100a
 // tensor cores through tcgen05 (umma.cuh).
 //
-// Same recurrence, chunked form (m3_common.cuh) and outputs as m3_fwd_tc.cu
+// Same recurrence, chunked form (m3_common.cuh) and outputs as m3_fwd.cu
 // (mamba-rs 0.7.0 README, "Features"; the three-term update and per-head
 // cumulative angles whose gradients stages B3 and B4 of Mamba3Scratch,
 // mamba-rs 0.4.2 src/mamba3_siso/cpu/scratch.rs, hold).  One CTA of 8 warps
