@@ -316,6 +316,49 @@ size_t msc_mamba3_siso_scan_bwd_workspace_bytes(int64_t batch, int64_t seqlen, i
 msc_status msc_mamba3_siso_scan_bwd(const msc_m3_bwd_args *args, void *workspace,
                                     size_t workspace_bytes, msc_stream_t stream);
 
+/* ======================================================================
+ * Mamba-3 SISO single-token state update (decode)
+ * ======================================================================
+ * The step that mamba3_step applies to a Mamba3State (mamba-rs 0.7.0 README,
+ * "Quick start (CPU)", Mamba-3), reduced to the scan: one step t of the
+ * Mamba-3 SISO recurrence above for every (b, h).  The recurrent state is
+ * everything that step needs from the past:
+ *
+ *   state     f32 [B, H, P, N]   S_{t-1} in, S_t out
+ *   x_prev    f32 [B, H, P]      x_{t-1} in, x_t out      (K_{t-1} = x_prev (outer) bt_prev)
+ *   bt_prev   f32 [B, H, N]      Bt_{t-1} in, Bt_t out    (the rotated B of the last step)
+ *   phi       f32 [B, H, K]      phi_{t-1} in, phi_t out  (cumulative angles)
+ * all read and written in place; a fresh sequence starts from zeros (then
+ * L steps equal msc_mamba3_siso_scan_fwd over those L tokens with h0 = 0).
+ * Inputs of the step:
+ *   x, z, out                 io  [B, H, P]
+ *   Bm, Cm                    io  [B, G, N]
+ *   alpha, beta, gamma        io  [B, H]
+ *   theta                     io  [B, H, K]
+ *   D                         f32 [H]
+ * Per (b, h), with g the group of head h:
+ *   phi   <- phi + theta;  Bt = R(phi) Bm[b,g,:],  Ct = R(phi) Cm[b,g,:]
+ *   S     <- alpha S + beta x_prev (outer) bt_prev + gamma x (outer) Bt
+ *   out    = (S Ct + D[h] x) * silu(z)
+ *   x_prev <- x,  bt_prev <- Bt
+ * Supported: P and N each in {16, 32, 64}, 2K <= N.  Every pointer is
+ * 16-byte aligned; z and D are optional, theta and phi may be NULL when K = 0.
+ */
+typedef struct {
+  uint32_t struct_size;
+  int32_t io_dtype;
+  int64_t batch, nheads, headdim, dstate, ngroups, nangles;
+  float *state, *x_prev, *bt_prev, *phi;
+  const void *x;
+  const void *z;           /* optional */
+  const void *Bm, *Cm;
+  const void *alpha, *beta, *gamma, *theta;
+  const float *D;          /* optional */
+  void *out;
+} msc_m3_su_args;
+
+msc_status msc_mamba3_siso_state_update(const msc_m3_su_args *args, msc_stream_t stream);
+
 #ifdef __cplusplus
 } /* extern "C" */
 #endif

@@ -43,8 +43,10 @@ def _load():
         _lib.oracle_ssm_state_update.argtypes = [i64] * 4 + [ci] + [dp] * 10
         _lib.oracle_m3_fwd.argtypes = [i64] * 7 + [dp] * 12 + [ci]
         _lib.oracle_m3_bwd.argtypes = [i64] * 7 + [dp] * 21 + [ci]
+        _lib.oracle_m3_state_update.argtypes = [i64] * 6 + [dp] * 14
         for f in (_lib.oracle_m1_fwd, _lib.oracle_m1_fwd_tree, _lib.oracle_m1_bwd,
-                  _lib.oracle_ssm_state_update, _lib.oracle_m3_fwd, _lib.oracle_m3_bwd):
+                  _lib.oracle_ssm_state_update, _lib.oracle_m3_fwd, _lib.oracle_m3_bwd,
+                  _lib.oracle_m3_state_update):
             f.restype = ctypes.c_int
         _lib.oracle_default_threads.restype = ctypes.c_int
     return _lib
@@ -174,6 +176,24 @@ def m3_bwd(x, B, C, alpha, beta, gamma, theta, dout, D=None, z=None, h0=None, nt
                              p1, p2, p3, p4, p5, p6, p7, p8, p9, p10, nthreads))
     return dict(dx=dx, dz=dz, dB=dB, dC=dC, dalpha=da, dbeta=db, dgamma=dg, dtheta=dth, dD=dD,
                 dh0=dh0)
+
+
+def m3_state_update(state, x_prev, bt_prev, phi, x, B, C, alpha, beta, gamma, theta, D=None,
+                    z=None):
+    """One Mamba-3 SISO decode step.  state [B, H, P, N], x_prev [B, H, P],
+    bt_prev [B, H, N], phi [B, H, K] (updated copies are returned); x, z [B, H, P];
+    B, C [B, G, N]; alpha/beta/gamma [B, H]; theta [B, H, K].
+    Returns (state, x_prev, bt_prev, phi, out [B, H, P])."""
+    lib = _load()
+    carried = [np.array(a, dtype=np.float64, copy=True) for a in (state, x_prev, bt_prev, phi)]
+    Bsz, H, P, N = carried[0].shape
+    G = B.shape[1]
+    K = carried[3].shape[2]
+    keep = [_in(v) for v in (x, z, B, C, alpha, beta, gamma, theta, D)]
+    out, po = _out((Bsz, H, P))
+    _check(lib.oracle_m3_state_update(Bsz, H, P, N, G, K, *[a.ctypes.data for a in carried],
+                                      *[k[1] for k in keep], po))
+    return (*carried, out)
 
 
 # ---------------------------------------------------------------------------

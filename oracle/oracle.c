@@ -39,7 +39,9 @@
  *
  *   Single-token state update: one step of the Mamba-1 recurrence applied to
  *   a stored state (mamba_step / GpuMambaBackbone::step, mamba-rs 0.7.0
- *   README, "Quick start").
+ *   README, "Quick start"), and one step of the Mamba-3 SISO recurrence
+ *   applied to a stored state with its last key and cumulative angles
+ *   (mamba3_step on a Mamba3State, the same README, "Quick start (CPU)").
  */
 #include <math.h>
 #include <pthread.h>
@@ -633,5 +635,52 @@ int oracle_m3_bwd(int64_t Bsz, int64_t L, int64_t H, int64_t P, int64_t N, int64
     fold_parts(c.dB_part, nt, Bsz * L * G * N, dB);
     fold_parts(c.dC_part, nt, Bsz * L * G * N, dC);
     fold_parts(c.dD_part, nt, H, dD);
+    return 0;
+}
+
+/*
+ * Mamba-3 SISO single-token state update (the step mamba3_step applies to a
+ * Mamba3State, mamba-rs 0.7.0 README, "Quick start (CPU)", Mamba-3): one step
+ * of the recurrence above for every (batch, head), written out on its own.
+ * The carried state is S [B, H, P, N], the last step's input x_prev [B, H, P],
+ * its rotated B bt_prev [B, H, N] (so that K_{t-1} = x_prev (outer) bt_prev)
+ * and the cumulative angles phi [B, H, K]; all are updated in place.
+ * Inputs: x, z, out [B, H, P]; B, C [B, G, N]; alpha, beta, gamma [B, H];
+ * theta [B, H, K]; D [H].
+ *   phi += theta;  Bt = R(phi) B;  Ct = R(phi) C
+ *   S    = alpha S + beta x_prev (outer) bt_prev + gamma x (outer) Bt
+ *   out  = (S Ct + D x) silu(z);   x_prev = x;  bt_prev = Bt
+ */
+int oracle_m3_state_update(int64_t Bsz, int64_t H, int64_t P, int64_t N, int64_t G, int64_t K,
+                           double *S, double *x_prev, double *bt_prev, double *phi,
+                           const double *x, const double *z, const double *Bm,
+                           const double *Cm, const double *alpha, const double *beta,
+                           const double *gamma, const double *theta, const double *Dp,
+                           double *out) {
+    if (N > ORACLE_MAX_N || 2 * K > N || G < 1 || H % G) return -1;
+    double Bt[ORACLE_MAX_N], Ct[ORACLE_MAX_N];
+    for (int64_t b = 0; b < Bsz; ++b) {
+        for (int64_t h = 0; h < H; ++h) {
+            const int64_t bh = b * H + h, g = h / (H / G);
+            double *ph = &phi[bh * K];
+            for (int64_t k = 0; k < K; ++k) ph[k] += theta[bh * K + k];
+            rope_apply(&Bm[(b * G + g) * N], ph, N, K, Bt);
+            rope_apply(&Cm[(b * G + g) * N], ph, N, K, Ct);
+            const double al = alpha[bh], be = beta[bh], ga = gamma[bh];
+            for (int64_t p = 0; p < P; ++p) {
+                const double xp = x[bh * P + p], xq = x_prev[bh * P + p];
+                double y = 0.0;
+                for (int64_t n = 0; n < N; ++n) {
+                    double *s = &S[(bh * P + p) * N + n];
+                    *s = al * *s + be * xq * bt_prev[bh * N + n] + ga * xp * Bt[n];
+                    y += Ct[n] * *s;
+                }
+                if (Dp) y += Dp[h] * xp;
+                out[bh * P + p] = z ? y * silu(z[bh * P + p]) : y;
+            }
+            for (int64_t p = 0; p < P; ++p) x_prev[bh * P + p] = x[bh * P + p];
+            for (int64_t n = 0; n < N; ++n) bt_prev[bh * N + n] = Bt[n];
+        }
+    }
     return 0;
 }

@@ -240,6 +240,62 @@ def su_problem(batch, dim, dstate, io=BF16, seed=SEED_BASE + 4, n_pool=8, ngroup
     return SUProblem(Bsz, D, N, G, io, True, A, Dp, db, state0, steps)
 
 
+@dataclass
+class M3SUProblem:
+    """Mamba-3 SISO decode: the carried state and a pool of step inputs."""
+    batch: int
+    nheads: int
+    headdim: int
+    dstate: int
+    ngroups: int
+    nangles: int
+    io: str
+    D: Optional[np.ndarray]      # float32 [H]
+    state0: np.ndarray           # float32 [B, H, P, N]
+    x_prev0: np.ndarray          # float32 [B, H, P]
+    bt_prev0: np.ndarray         # float32 [B, H, N]
+    phi0: np.ndarray             # float32 [B, H, K]
+    steps: list                  # dicts: x, z [B,H,P]; B, C [B,G,N]; alpha, beta, gamma [B,H]; theta [B,H,K]
+
+
+def m3su_problem(batch, nheads, headdim, dstate, ngroups=1, nangles=None, io=BF16,
+                 seed=SEED_BASE + 5, n_pool=8, random_state=False, with_z=True,
+                 with_D=True) -> M3SUProblem:
+    """Mamba-3 decode-step inputs with the distributions of the Mamba-3 scan
+    workload, a pool of ``n_pool`` step input sets cycled by the caller.  The
+    carried state starts at zero (a fresh sequence) or, with ``random_state``,
+    at random values (the middle of a sequence: N(0,1) state and last input,
+    a unit-RMS last rotated key, angles in [0, 10))."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    Bsz, H, P, N, G = batch, nheads, headdim, dstate, ngroups
+    K = N // 2 if nangles is None else nangles
+    Dp = _normal(rng, (H,)) if with_D else None
+    if random_state:
+        state0 = _normal(rng, (Bsz, H, P, N))
+        x_prev0 = _normal(rng, (Bsz, H, P))
+        bt_prev0 = _rms_normalise(_normal(rng, (Bsz, H, N)))
+        phi0 = _uniform(rng, 0.0, 10.0, (Bsz, H, K))
+    else:
+        state0 = np.zeros((Bsz, H, P, N), np.float32)
+        x_prev0 = np.zeros((Bsz, H, P), np.float32)
+        bt_prev0 = np.zeros((Bsz, H, N), np.float32)
+        phi0 = np.zeros((Bsz, H, K), np.float32)
+    steps = []
+    for _ in range(n_pool):
+        r = _normal(rng, (Bsz, H)).astype(np.float64)
+        steps.append(dict(
+            x=store(_normal(rng, (Bsz, H, P)), io),
+            z=store(_normal(rng, (Bsz, H, P)), io) if with_z else None,
+            B=store(_rms_normalise(_normal(rng, (Bsz, G, N))), io),
+            C=store(_rms_normalise(_normal(rng, (Bsz, G, N))), io),
+            alpha=store(np.exp(-np.logaddexp(0.0, r)), io),
+            beta=store(_uniform(rng, 0.0, 0.5, (Bsz, H)), io),
+            gamma=store(_uniform(rng, 0.0, 0.5, (Bsz, H)), io),
+            theta=store(_uniform(rng, 0.0, 0.1, (Bsz, H, K)), io),
+        ))
+    return M3SUProblem(Bsz, H, P, N, G, K, io, Dp, state0, x_prev0, bt_prev0, phi0, steps)
+
+
 # --------------------------------------------------------------------------
 # The named workloads
 # --------------------------------------------------------------------------
@@ -255,6 +311,9 @@ WORKLOADS = {
                                              seed=SEED_BASE + 3),
     "su_bf16_b256_d5120_n16_x1000": dict(kind="su", batch=256, dim=5120, dstate=16, io=BF16,
                                          steps=1000, seed=SEED_BASE + 4),
+    "m3su_bf16_b256_h24_p64_n64_k32_x1000": dict(kind="m3su", batch=256, nheads=24, headdim=64,
+                                                 dstate=64, nangles=32, io=BF16, steps=1000,
+                                                 seed=SEED_BASE + 5),
 }
 
 
@@ -273,4 +332,7 @@ def make(name: str, shard: int = 0):
                           nangles=w["nangles"], io=w["io"], seed=w["seed"])
     if kind == "su":
         return su_problem(w["batch"], w["dim"], w["dstate"], io=w["io"], seed=w["seed"])
+    if kind == "m3su":
+        return m3su_problem(w["batch"], w["nheads"], w["headdim"], w["dstate"],
+                            nangles=w["nangles"], io=w["io"], seed=w["seed"])
     raise ValueError(kind)

@@ -371,3 +371,74 @@ def test_m3_dD_closed_form():
     g = oracle.m3_bwd(dout=dout, **a)
     np.testing.assert_allclose(g["dD"], np.sum(dout * _silu(a["z"]) * a["x"], axis=(0, 1, 3)),
                                rtol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# Mamba-3 single-token state update
+# ---------------------------------------------------------------------------
+def _m3_decode_chain(a, G, state0=None):
+    """Run the oracle's decode step over every token of the scan inputs `a`
+    (x [B,L,H,P], ...) from a fresh carried state; returns outs [B,L,H,P] and
+    the final carried state."""
+    Bsz, L, H, P = a["x"].shape
+    N, K = a["B"].shape[3], a["theta"].shape[3]
+    S = np.zeros((Bsz, H, P, N)) if state0 is None else state0.copy()
+    xp, bp, ph = np.zeros((Bsz, H, P)), np.zeros((Bsz, H, N)), np.zeros((Bsz, H, K))
+    outs = np.zeros_like(a["x"])
+    for t in range(L):
+        S, xp, bp, ph, o = oracle.m3_state_update(
+            S, xp, bp, ph, a["x"][:, t], a["B"][:, t], a["C"][:, t], a["alpha"][:, t],
+            a["beta"][:, t], a["gamma"][:, t], a["theta"][:, t], D=a["D"], z=a["z"][:, t])
+        outs[:, t] = o
+    return outs, S, xp, bp, ph
+
+
+@pytest.mark.parametrize("G,H", [(1, 2), (2, 4)])
+def test_m3_state_update_chain_equals_scan(G, H):
+    """L decode steps from a fresh carried state (S = h0, no last key, zero
+    angles) reproduce the scan's outputs and final state: the step carries
+    exactly K_{t-1} and the cumulative angles."""
+    a = _m3_tiny(Bsz=2, L=9, H=H, P=3, N=6, K=2, G=G, h0=True)
+    r = oracle.m3_fwd(**a)
+    outs, S, xp, bp, ph = _m3_decode_chain(a, G, state0=a["h0"])
+    np.testing.assert_allclose(outs, r["out"], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(S, r["final_state"], rtol=1e-12, atol=1e-13)
+    np.testing.assert_array_equal(xp, a["x"][:, -1])
+    np.testing.assert_allclose(ph, np.cumsum(a["theta"], axis=1)[:, -1], rtol=1e-14)
+    for b in range(2):
+        for h in range(H):
+            g = h // (H // G)
+            np.testing.assert_allclose(bp[b, h], _rot(a["B"][b, -1, g], ph[b, h], 2), rtol=1e-13)
+
+
+def test_m3_state_update_identity_step():
+    """alpha = 1, beta = gamma = 0 leaves S as it was; y = S R(phi+theta) C + D x,
+    and the carried x and rotated B become this step's."""
+    Bsz, H, P, N, K = 1, 2, 3, 4, 2
+    S0, xp0, bp0 = _rand(Bsz, H, P, N), _rand(Bsz, H, P), _rand(Bsz, H, N)
+    ph0, th = _rand(Bsz, H, K), _rand(Bsz, H, K)
+    x, Bm, Cm, D = _rand(Bsz, H, P), _rand(Bsz, 1, N), _rand(Bsz, 1, N), _rand(H)
+    S, xp, bp, ph, out = oracle.m3_state_update(
+        S0, xp0, bp0, ph0, x, Bm, Cm, np.ones((Bsz, H)), np.zeros((Bsz, H)), np.zeros((Bsz, H)),
+        th, D=D)
+    np.testing.assert_array_equal(S, S0)
+    for h in range(H):
+        Ct = _rot(Cm[0, 0], ph0[0, h] + th[0, h], K)
+        np.testing.assert_allclose(out[0, h], S0[0, h] @ Ct + D[h] * x[0, h], rtol=1e-13)
+        np.testing.assert_allclose(bp[0, h], _rot(Bm[0, 0], ph0[0, h] + th[0, h], K), rtol=1e-14)
+    np.testing.assert_array_equal(xp, x)
+
+
+def test_m3_state_update_angle_offset_invariance():
+    """From a fresh state, adding one constant to the carried angles changes no
+    output: only differences of cumulative angles reach y."""
+    a = _m3_tiny(Bsz=1, L=6, H=2, P=2, N=4, K=2, h0=False)
+    o1 = _m3_decode_chain(a, 1)[0]
+    Bsz, L, H, P = a["x"].shape
+    S, xp, bp = np.zeros((1, H, P, 4)), np.zeros((1, H, P)), np.zeros((1, H, 4))
+    ph = np.full((1, H, 2), 2.5)
+    for t in range(L):
+        S, xp, bp, ph, o = oracle.m3_state_update(
+            S, xp, bp, ph, a["x"][:, t], a["B"][:, t], a["C"][:, t], a["alpha"][:, t],
+            a["beta"][:, t], a["gamma"][:, t], a["theta"][:, t], D=a["D"], z=a["z"][:, t])
+        np.testing.assert_allclose(o, o1[:, t], rtol=1e-11, atol=1e-12)
