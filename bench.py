@@ -84,6 +84,14 @@ def su_bytes(Bsz, D, N, io_bytes, G=1):
     return Bsz * D * (2 * N * 4 + 4 * io_bytes) + 2 * Bsz * G * N * io_bytes
 
 
+def m3su_bytes(Bsz, H, P, N, G, K, io_bytes):
+    """One Mamba-3 decode step: the carried state, last input, last rotated key
+    and angles read and written (f32); x, z, out, alpha, beta, gamma, theta per
+    (b, h) and B, C per (b, g) in io."""
+    per_head = 2 * 4 * (P * N + P + N + K) + io_bytes * (3 * P + 3 + K)
+    return Bsz * H * per_head + 2 * Bsz * G * N * io_bytes
+
+
 # ---------------------------------------------------------------------------
 # DRAM traffic of the dominant kernel from an ncu capture (dram__bytes_read.sum
 # + dram__bytes_write.sum, one launch of the named workload), valid only for
@@ -476,6 +484,30 @@ def extra_workloads(msc, args, world, peaks):
         value=round(q.batch * q.dim * 1000 / (ms / 1e3), 1), unit="channel-steps/s",
         hbm_frac=round(sb * 1000 / (ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
         note="84 MB state can stay L2-resident between steps")
+    # Mamba-3 SISO decode step (B256 H24 P64 N64 K32, 1000 steps cycling 8 input sets)
+    q3 = W.make("m3su_bf16_b256_h24_p64_n64_k32_x1000")
+    carried = [torch.from_numpy(v).cuda() for v in (q3.state0, q3.x_prev0, q3.bt_prev0, q3.phi0)]
+    D3 = to_dev(q3.D)
+    pool3 = [{k: to_dev(v) for k, v in s.items()} for s in q3.steps]
+    outs3 = [torch.empty_like(pool3[0]["x"]) for _ in range(8)]
+
+    def m3_decode_1000():
+        for t in range(1000):
+            s = pool3[t % 8]
+            msc.msc_mamba3_siso_state_update(*carried, s["x"], s["B"], s["C"], s["alpha"],
+                                             s["beta"], s["gamma"], s["theta"], D=D3, z=s["z"],
+                                             out=outs3[t % 8])
+
+    total_ms, (ms,) = time_steps([m3_decode_1000], 2, 1, world)
+    sb3 = m3su_bytes(q3.batch, q3.nheads, q3.headdim, q3.dstate, q3.ngroups, q3.nangles, 2)
+    res["m3su_bf16_b256_h24_p64_n64_k32_x1000"] = dict(
+        ms_per_1000_steps=round(ms, 3), us_per_step=round(ms, 3),
+        value=round(q3.batch * q3.nheads * q3.headdim * 1000 / (ms / 1e3), 1),
+        unit="token-channel steps/s",
+        hbm_frac=round(sb3 * 1000 / (ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+        note="101 MB state: most of it can stay in the 126 MB L2 between steps")
+    del carried, pool3, outs3
+    torch.cuda.empty_cache()
     # Mamba-3 SISO
     try:
         m3 = W.make("m3_bf16_b8_h24_p64_n64_k32_l2048")
@@ -533,7 +565,7 @@ def run_only(args):
         st.fwd()
         fn = st.fwd if phase == "m1_fwd" else st.bwd
         units = p.token_channels
-    elif phase.startswith("m3"):
+    elif phase in ("m3_fwd", "m3_bwd"):
         m3 = W.make(args.workload or "m3_bf16_b8_h24_p64_n64_k32_l2048")
         a = dict(x=to_dev(m3.x), B=to_dev(m3.B), C=to_dev(m3.C), alpha=to_dev(m3.alpha),
                  beta=to_dev(m3.beta), gamma=to_dev(m3.gamma), theta=to_dev(m3.theta),
@@ -552,6 +584,18 @@ def run_only(args):
                 msc.msc_mamba3_siso_scan_bwd(**a, saved_states=saved, dout=dout, workspace=ws,
                                              grads=grads)
         units = m3.token_channels
+    elif phase == "m3_decode":
+        q = W.make(args.workload or "m3su_bf16_b256_h24_p64_n64_k32_x1000")
+        carried = [torch.from_numpy(v).cuda() for v in (q.state0, q.x_prev0, q.bt_prev0, q.phi0)]
+        D3 = to_dev(q.D)
+        s = {k: to_dev(v) for k, v in q.steps[0].items()}
+        out = torch.empty_like(s["x"])
+
+        def fn():
+            msc.msc_mamba3_siso_state_update(*carried, s["x"], s["B"], s["C"], s["alpha"],
+                                             s["beta"], s["gamma"], s["theta"], D=D3, z=s["z"],
+                                             out=out)
+        units = q.batch * q.nheads * q.headdim
     else:  # decode
         q = W.make(args.workload or "su_bf16_b256_d5120_n16_x1000")
         state = torch.from_numpy(q.state0).cuda()
@@ -619,7 +663,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extra", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["m1_fwd", "m1_bwd", "m3_fwd", "m3_bwd", "decode"],
+    ap.add_argument("--only", choices=["m1_fwd", "m1_bwd", "m3_fwd", "m3_bwd", "decode",
+                                       "m3_decode"],
                     help="time one phase alone (for profiling); prints no bench line")
     ap.add_argument("--workload", default=None, help="workload name for --only")
     args = ap.parse_args()

@@ -189,4 +189,56 @@ msc_status msc_mamba3_siso_scan_bwd(const msc_m3_bwd_args *a, void *workspace,
   return api_cuda(msc::launch_m3_bwd(p, s), fn);
 }
 
+msc_status msc_mamba3_siso_state_update(const msc_m3_su_args *a, msc_stream_t stream) {
+  const char *fn = "msc_mamba3_siso_state_update";
+  if (!a) return api_fail(MSC_ERR_INVALID_ARG, "%s: args is NULL", fn);
+  if (a->struct_size < sizeof(msc_m3_su_args))
+    return api_fail(MSC_ERR_INVALID_ARG, "%s: struct_size %u is smaller than the struct (%zu)",
+                    fn, a->struct_size, sizeof(msc_m3_su_args));
+  if (a->io_dtype != MSC_F32 && a->io_dtype != MSC_BF16)
+    return api_fail(MSC_ERR_INVALID_ARG, "%s: io_dtype %d is not MSC_F32 (0) or MSC_BF16 (1)",
+                    fn, (int)a->io_dtype);
+  if (a->batch < 0 || a->nheads < 1 || a->ngroups < 1 || a->nangles < 0)
+    return api_fail(MSC_ERR_INVALID_ARG,
+                    "%s: need batch >= 0, nheads >= 1, ngroups >= 1, nangles >= 0", fn);
+  if (a->nheads % a->ngroups != 0)
+    return api_fail(MSC_ERR_INVALID_ARG, "%s: ngroups %lld does not divide nheads %lld", fn,
+                    (long long)a->ngroups, (long long)a->nheads);
+  if (!msc::m3_supported(a->headdim, a->dstate))
+    return api_fail(MSC_ERR_UNSUPPORTED,
+                    "%s: headdim %lld / dstate %lld not supported (each must be 16, 32 or 64)", fn,
+                    (long long)a->headdim, (long long)a->dstate);
+  if (2 * a->nangles > a->dstate)
+    return api_fail(MSC_ERR_INVALID_ARG, "%s: 2 * nangles (%lld) exceeds dstate (%lld)", fn,
+                    (long long)(2 * a->nangles), (long long)a->dstate);
+  if (a->batch * a->nheads > ((int64_t)1 << 31))
+    return api_fail(MSC_ERR_UNSUPPORTED, "%s: batch * nheads must be <= 2^31", fn);
+  if (a->batch == 0) return api_ok();
+  M3_REQUIRE(fn, "state", a->state);
+  M3_REQUIRE(fn, "x_prev", a->x_prev);
+  M3_REQUIRE(fn, "bt_prev", a->bt_prev);
+  M3_REQUIRE(fn, "x", a->x);
+  M3_REQUIRE(fn, "Bm", a->Bm);
+  M3_REQUIRE(fn, "Cm", a->Cm);
+  M3_REQUIRE(fn, "alpha", a->alpha);
+  M3_REQUIRE(fn, "beta", a->beta);
+  M3_REQUIRE(fn, "gamma", a->gamma);
+  M3_REQUIRE(fn, "out", a->out);
+  if (a->nangles > 0) {
+    M3_REQUIRE(fn, "phi", a->phi);
+    M3_REQUIRE(fn, "theta", a->theta);
+  }
+  M3_OPTIONAL(fn, "z", a->z);
+  M3_OPTIONAL(fn, "D", a->D);
+  msc::M3SUParams p = {};
+  p.io_bf16 = a->io_dtype == MSC_BF16;
+  p.B = a->batch; p.H = a->nheads; p.P = a->headdim; p.N = a->dstate; p.G = a->ngroups;
+  p.K = a->nangles;
+  p.state = a->state; p.x_prev = a->x_prev; p.bt_prev = a->bt_prev; p.phi = a->phi;
+  p.x = a->x; p.z = a->z; p.Bm = a->Bm; p.Cm = a->Cm;
+  p.alpha = a->alpha; p.beta = a->beta; p.gamma = a->gamma; p.theta = a->theta;
+  p.Dp = a->D; p.out = a->out;
+  return api_cuda(msc::launch_m3_state_update(p, reinterpret_cast<cudaStream_t>(stream)), fn);
+}
+
 }  // extern "C"

@@ -80,4 +80,15 @@ size_t m3_bwd_workspace_bytes(int64_t B, int64_t L, int64_t H, int64_t P, int64_
                               int64_t K);
 bool m3_supported(int64_t P, int64_t N);
 
+// Mamba-3 SISO single-token state update (decode)
+struct M3SUParams {
+  int io_bf16;
+  int64_t B, H, P, N, G, K;
+  float *state, *x_prev, *bt_prev, *phi;
+  const void *x, *z, *Bm, *Cm, *alpha, *beta, *gamma, *theta;
+  const float *Dp;
+  void *out;
+};
+cudaError_t launch_m3_state_update(const M3SUParams &p, cudaStream_t s);
+
 }  // namespace msc

@@ -1,0 +1,149 @@
+// m3_state_update.cu -- Mamba-3 SISO single-token state update (decode).
+//
+// One step of the Mamba-3 SISO recurrence (mamba-rs 0.7.0 README, "Features";
+// the step mamba3_step applies to a Mamba3State, the same README, "Quick
+// start (CPU)") for every (b, h), on a carried state S [P][N], the last
+// input x_prev [P], the last rotated key bt_prev [N] and the cumulative
+// angles phi [K]:
+//   phi <- phi + theta;  Bt = R(phi) B;  Ct = R(phi) C
+//   S   <- alpha S + beta x_prev (outer) bt_prev + gamma x (outer) Bt
+//   out  = (S Ct + D x) silu(z);   x_prev <- x;  bt_prev <- Bt
+//
+// The step is bound by HBM: S is read and written once (2 P N 4 bytes per
+// head), everything else is a few hundred bytes per head.  A head is served
+// by P N / 16 threads, N / 16 per row of S, each holding 16 state entries as
+// four 16-byte pieces interleaved with its row neighbours' (so that the
+// threads of a row read and write one contiguous run per instruction).  A
+// CTA of 256 threads serves 256 / (P N / 16) heads.  Per head, the first N/2
+// threads rotate one pair of B and C each into shared memory; y sums a row's
+// partials over its N / 16 threads with shuffles in a fixed order.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace msc {
+namespace {
+
+constexpr int kSUThreads = 256;
+
+template <typename T>
+__device__ __forceinline__ float ldf(const void *base, int64_t i) {
+  return to_f32(static_cast<const T *>(base)[i]);
+}
+
+template <typename T, int P, int N>
+__global__ void __launch_bounds__(kSUThreads) m3_state_update_kernel(const M3SUParams p) {
+  constexpr int kTPR = N / 16;           // threads per row of S
+  constexpr int kTPH = P * kTPR;         // threads per head
+  constexpr int kHPC = kSUThreads / kTPH;  // heads per CTA
+  constexpr int kPer = 3 * N + P;        // shared floats per head: Bt, Ct, bt_prev, x_prev
+  __shared__ __align__(16) float sm[kHPC * kPer];
+
+  const int tid = threadIdx.x;
+  const int hl = tid / kTPH, j = tid % kTPH;
+  const int64_t BH = p.B * p.H;
+  const int64_t bh = (int64_t)blockIdx.x * kHPC + hl;
+  const bool live = bh < BH;
+  const int64_t b = bh / p.H, h = bh % p.H;
+  const int64_t g = h / (p.H / p.G);
+  const int K = (int)p.K;
+  float *sBt = sm + hl * kPer, *sCt = sBt + N, *sBp = sCt + N, *sXp = sBp + N;
+
+  // ---- the step's rotated B and C; the carried x_prev and bt_prev ----------
+  if (live) {
+    if (j < N / 2) {
+      const int64_t o = (b * p.G + g) * N + 2 * j;
+      float b0 = ldf<T>(p.Bm, o), b1 = ldf<T>(p.Bm, o + 1);
+      float c0 = ldf<T>(p.Cm, o), c1 = ldf<T>(p.Cm, o + 1);
+      if (j < K) {
+        const float phi = p.phi[bh * K + j] + ldf<T>(p.theta, bh * K + j);
+        p.phi[bh * K + j] = phi;
+        float sn, cs;
+        sincosf(phi, &sn, &cs);
+        const float rb0 = cs * b0 - sn * b1, rb1 = sn * b0 + cs * b1;
+        const float rc0 = cs * c0 - sn * c1, rc1 = sn * c0 + cs * c1;
+        b0 = rb0; b1 = rb1; c0 = rc0; c1 = rc1;
+      }
+      sBt[2 * j] = b0; sBt[2 * j + 1] = b1;
+      sCt[2 * j] = c0; sCt[2 * j + 1] = c1;
+    }
+    for (int i = j; i < N; i += kTPH) sBp[i] = p.bt_prev[bh * N + i];
+    for (int i = j; i < P; i += kTPH) sXp[i] = p.x_prev[bh * P + i];
+  }
+  __syncthreads();
+  if (!live) return;
+  // the carried key of the next step (every read of the old one is done)
+  for (int i = j; i < N; i += kTPH) p.bt_prev[bh * N + i] = sBt[i];
+  for (int i = j; i < P; i += kTPH) p.x_prev[bh * P + i] = ldf<T>(p.x, bh * P + i);
+
+  // ---- the state rows ---------------------------------------------------------
+  const int row = j / kTPR, q = j % kTPR;
+  const float al = ldf<T>(p.alpha, bh), be = ldf<T>(p.beta, bh), ga = ldf<T>(p.gamma, bh);
+  const float xv = ldf<T>(p.x, bh * P + row);
+  const float bxq = be * sXp[row], gx = ga * xv;
+  float4 *srow = reinterpret_cast<float4 *>(p.state + (bh * P + row) * N);
+  const float4 *vBt = reinterpret_cast<const float4 *>(sBt);
+  const float4 *vCt = reinterpret_cast<const float4 *>(sCt);
+  const float4 *vBp = reinterpret_cast<const float4 *>(sBp);
+  float4 s[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) s[i] = srow[i * kTPR + q];
+  float y = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int v = i * kTPR + q;
+    const float4 bt = vBt[v], ct = vCt[v], bp = vBp[v];
+    s[i].x = fmaf(al, s[i].x, fmaf(bxq, bp.x, gx * bt.x));
+    s[i].y = fmaf(al, s[i].y, fmaf(bxq, bp.y, gx * bt.y));
+    s[i].z = fmaf(al, s[i].z, fmaf(bxq, bp.z, gx * bt.z));
+    s[i].w = fmaf(al, s[i].w, fmaf(bxq, bp.w, gx * bt.w));
+    y = fmaf(ct.x, s[i].x, y);
+    y = fmaf(ct.y, s[i].y, y);
+    y = fmaf(ct.z, s[i].z, y);
+    y = fmaf(ct.w, s[i].w, y);
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) srow[i * kTPR + q] = s[i];
+  // (kTPR > 1 only for N >= 32, where a warp holds threads of one head only,
+  // so no lane of a shuffling warp has returned above)
+#pragma unroll
+  for (int off = 1; off < kTPR; off <<= 1) y += __shfl_xor_sync(0xffffffffu, y, off, kTPR);
+  if (q == 0) {
+    if (p.Dp) y = fmaf(p.Dp[h], xv, y);
+    if (p.z) y *= silu(ldf<T>(p.z, bh * P + row));
+    static_cast<T *>(p.out)[bh * P + row] = from_f32<T>(y);
+  }
+}
+
+template <typename T, int P, int N>
+cudaError_t launch_pn(const M3SUParams &p, cudaStream_t s) {
+  constexpr int kHPC = kSUThreads / (P * N / 16);
+  const int64_t blocks = (p.B * p.H + kHPC - 1) / kHPC;
+  m3_state_update_kernel<T, P, N><<<(unsigned)blocks, kSUThreads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+template <typename T, int P>
+cudaError_t launch_p(const M3SUParams &p, cudaStream_t s) {
+  switch (p.N) {
+    case 16: return launch_pn<T, P, 16>(p, s);
+    case 32: return launch_pn<T, P, 32>(p, s);
+    default: return launch_pn<T, P, 64>(p, s);
+  }
+}
+
+template <typename T>
+cudaError_t launch_t(const M3SUParams &p, cudaStream_t s) {
+  switch (p.P) {
+    case 16: return launch_p<T, 16>(p, s);
+    case 32: return launch_p<T, 32>(p, s);
+    default: return launch_p<T, 64>(p, s);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_m3_state_update(const M3SUParams &p, cudaStream_t s) {
+  return p.io_bf16 ? launch_t<bf16>(p, s) : launch_t<float>(p, s);
+}
+
+}  // namespace msc

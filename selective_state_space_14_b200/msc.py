@@ -80,12 +80,20 @@ class M3BwdArgs(ctypes.Structure):
                 ("dtheta", _vp), ("dD", _vp), ("dh0", _vp)]
 
 
+class M3SuArgs(ctypes.Structure):
+    _fields_ = [("struct_size", _u32), ("io_dtype", _i32), ("batch", _i64), ("nheads", _i64),
+                ("headdim", _i64), ("dstate", _i64), ("ngroups", _i64), ("nangles", _i64),
+                ("state", _vp), ("x_prev", _vp), ("bt_prev", _vp), ("phi", _vp), ("x", _vp),
+                ("z", _vp), ("Bm", _vp), ("Cm", _vp), ("alpha", _vp), ("beta", _vp),
+                ("gamma", _vp), ("theta", _vp), ("D", _vp), ("out", _vp)]
+
+
 EXPORTS = ["msc_last_error", "msc_version", "msc_selective_scan_saved_states_bytes",
            "msc_selective_scan_fwd", "msc_selective_scan_bwd_workspace_bytes",
            "msc_selective_scan_bwd", "msc_selective_scan_bwd_static", "msc_ssm_state_update",
            "msc_mamba3_siso_saved_states_bytes",
            "msc_mamba3_siso_scan_fwd", "msc_mamba3_siso_scan_bwd_workspace_bytes",
-           "msc_mamba3_siso_scan_bwd"]
+           "msc_mamba3_siso_scan_bwd", "msc_mamba3_siso_state_update"]
 
 _lib = None
 
@@ -107,7 +115,8 @@ def lib() -> ctypes.CDLL:
                            ("msc_ssm_state_update", [ctypes.POINTER(SuArgs), _vp]),
                            ("msc_mamba3_siso_scan_fwd", [ctypes.POINTER(M3FwdArgs), _vp]),
                            ("msc_mamba3_siso_scan_bwd",
-                            [ctypes.POINTER(M3BwdArgs), _vp, ctypes.c_size_t, _vp])):
+                            [ctypes.POINTER(M3BwdArgs), _vp, ctypes.c_size_t, _vp]),
+                           ("msc_mamba3_siso_state_update", [ctypes.POINTER(M3SuArgs), _vp])):
             f = getattr(L, name)
             f.argtypes = argt
             f.restype = ctypes.c_int
@@ -356,3 +365,21 @@ def msc_mamba3_siso_scan_bwd(x, B, C, alpha, beta, gamma, theta, saved_states, d
     _check(lib().msc_mamba3_siso_scan_bwd(ctypes.byref(a), _ptr(workspace), workspace.numel(),
                                           _stream(stream)))
     return g
+
+
+def msc_mamba3_siso_state_update(state, x_prev, bt_prev, phi, x, B, C, alpha, beta, gamma,
+                                 theta, D=None, z=None, out=None, stream=None):
+    """In-place Mamba-3 SISO decode step.  Carried: state f32 [B, H, P, N], x_prev f32
+    [B, H, P], bt_prev f32 [B, H, N], phi f32 [B, H, K].  Step inputs: x, z [B, H, P];
+    B, C [B, G, N]; alpha, beta, gamma [B, H]; theta [B, H, K].  Returns out [B, H, P]."""
+    Bsz, H, P, N = state.shape
+    G = B.shape[1]
+    K = phi.shape[2]
+    if out is None:
+        out = torch.empty_like(x)
+    a = M3SuArgs(ctypes.sizeof(M3SuArgs), _io(x), Bsz, H, P, N, G, K, _ptr(state), _ptr(x_prev),
+                 _ptr(bt_prev), _ptr(phi) if K > 0 else None, _ptr(x), _ptr(z), _ptr(B), _ptr(C),
+                 _ptr(alpha), _ptr(beta), _ptr(gamma), _ptr(theta) if K > 0 else None, _ptr(D),
+                 _ptr(out))
+    _check(lib().msc_mamba3_siso_state_update(ctypes.byref(a), _stream(stream)))
+    return out

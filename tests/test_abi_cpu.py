@@ -124,6 +124,43 @@ def test_state_update_rejects_null():
     assert msc.lib().msc_ssm_state_update(None, None) == INVALID
 
 
+def _m3su_args(**kw):
+    a = msc.M3SuArgs()
+    a.struct_size = ctypes.sizeof(msc.M3SuArgs)
+    a.io_dtype, a.batch, a.nheads, a.headdim, a.dstate, a.ngroups, a.nangles = (
+        msc.MSC_BF16, 2, 4, 64, 64, 1, 32)
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("field,value,status,word", [
+    ("headdim", 48, UNSUPPORTED, "headdim"),
+    ("dstate", 128, UNSUPPORTED, "dstate"),
+    ("nangles", 33, INVALID, "nangles"),
+    ("ngroups", 3, INVALID, "ngroups"),
+    ("nheads", 0, INVALID, "nheads"),
+    ("io_dtype", 7, INVALID, "io_dtype"),
+    ("struct_size", 8, INVALID, "struct_size"),
+])
+def test_m3_state_update_rejects_bad_sizes(field, value, status, word):
+    st = msc.lib().msc_mamba3_siso_state_update(ctypes.byref(_m3su_args(**{field: value})), None)
+    assert st == status and word in _err()
+
+
+def test_m3_state_update_rejects_missing_and_misaligned():
+    assert msc.lib().msc_mamba3_siso_state_update(None, None) == INVALID
+    st = msc.lib().msc_mamba3_siso_state_update(ctypes.byref(_m3su_args()), None)
+    assert st == INVALID and "state" in _err()
+    a = _m3su_args(state=0x1000, x_prev=0x2000, bt_prev=0x3008)
+    st = msc.lib().msc_mamba3_siso_state_update(ctypes.byref(a), None)
+    assert st == ALIGNMENT and "bt_prev" in _err()
+
+
+def test_m3_state_update_empty_batch_is_a_no_op():
+    assert msc.lib().msc_mamba3_siso_state_update(ctypes.byref(_m3su_args(batch=0)), None) == 0
+
+
 def test_size_functions():
     # saved states: f32 [B, D, ceil(L / 8), N]
     assert msc.msc_selective_scan_saved_states_bytes(2, 3, 16, 17) == 4 * 2 * 3 * 3 * 16

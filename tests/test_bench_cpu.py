@@ -35,6 +35,15 @@ def test_decode_bytes():
     assert round(bench.su_bytes(256, 5120, 16, 2) / 1e6, 1) == 178.3
 
 
+def test_m3_decode_bytes():
+    B, H, P, N, G, K, io = 256, 24, 64, 64, 1, 32, 2
+    # state, x_prev, bt_prev, phi read + written in f32; x, z, out, alpha,
+    # beta, gamma, theta per head and B, C per group in io
+    per_head = 2 * 4 * (P * N + P + N + K) + io * (3 * P + 3 + K)
+    assert bench.m3su_bytes(B, H, P, N, G, K, io) == B * H * per_head + 2 * B * G * N * io
+    assert round(bench.m3su_bytes(B, H, P, N, G, K, io) / 1e6, 1) == 212.0
+
+
 def test_traffic_gated_by_source_hash(monkeypatch):
     assert bench.ncu_traffic("no_such_kernel.cu") is None
     monkeypatch.setitem(bench.NCU_TRAFFIC, "m1_fwd.cu", ("0000000000000000", "w", 123))

@@ -186,3 +186,140 @@ def test_bwd_model_shaped_full_size(msc):
     r = _oracle_bwd(p0)
     for k in ("dx", "dz", "dB", "dC", "dalpha", "dbeta", "dgamma", "dtheta", "dh0"):
         assert_close(k, g[k][:1], r[k], TOL["bf16"])
+
+
+# ---------------------------------------------------------------------------
+# single-token state update (decode)
+# ---------------------------------------------------------------------------
+def _su_device_state(q):
+    return [torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).cuda()
+            for a in (q.state0, q.x_prev0, q.bt_prev0, q.phi0)]
+
+
+SU_CASES = [
+    # (B, H, P, N, G, K, io, random_state, z, D, steps)
+    (3, 4, 64, 64, 1, 32, "f32", True, True, True, 12),
+    (2, 6, 16, 16, 2, 8, "f32", True, True, False, 12),
+    (5, 3, 32, 64, 3, 5, "f32", False, False, True, 12),
+    (4, 8, 64, 64, 2, 32, "bf16", True, True, True, 40),
+    (7, 3, 16, 32, 1, 16, "bf16", True, True, True, 20),
+    (3, 5, 64, 16, 1, 0, "bf16", False, True, False, 20),
+    (9, 2, 16, 16, 1, 8, "bf16", True, False, True, 20),
+    (2, 4, 32, 32, 4, 16, "bf16", True, True, True, 20),
+]
+
+
+@pytest.mark.parametrize("case", SU_CASES,
+                         ids=[f"B{c[0]}H{c[1]}P{c[2]}N{c[3]}G{c[4]}K{c[5]}{c[6]}" for c in SU_CASES])
+def test_m3_state_update_chain(msc, case):
+    """Chained decode steps against the oracle's chained steps: every output
+    and, at the end, the four carried tensors."""
+    Bsz, H, P, N, G, K, io, rs, z, Dp, n = case
+    q = W.m3su_problem(Bsz, H, P, N, ngroups=G, nangles=K, io=io, seed=11 + Bsz + N, n_pool=n,
+                       random_state=rs, with_z=z, with_D=Dp)
+    S, xp, bp, ph = _su_device_state(q)
+    ref = [a.astype(np.float64) for a in (q.state0, q.x_prev0, q.bt_prev0, q.phi0)]
+    D = dev(q.D)
+    for s in q.steps:
+        o = msc.msc_mamba3_siso_state_update(S, xp, bp, ph, dev(s["x"]), dev(s["B"]), dev(s["C"]),
+                                             dev(s["alpha"]), dev(s["beta"]), dev(s["gamma"]),
+                                             dev(s["theta"]), D=D, z=dev(s["z"]))
+        f = lambda t: None if t is None else t.as_f64()
+        *ref, o_ref = oracle.m3_state_update(*ref, f(s["x"]), f(s["B"]), f(s["C"]),
+                                             f(s["alpha"]), f(s["beta"]), f(s["gamma"]),
+                                             f(s["theta"]),
+                                             D=None if q.D is None else q.D.astype(np.float64),
+                                             z=f(s["z"]))
+        assert_close("out", host(o), o_ref, TOL[io])
+    for name, g, r in zip(("state", "x_prev", "bt_prev", "phi"), (S, xp, bp, ph), ref):
+        assert_close(name, host(g), r, TOL[io])
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_m3_state_update_chain_equals_scan(msc, io):
+    """Decoding a sequence token by token from a fresh carried state (the state
+    set to h0) gives the outputs and final state of the scan of the same
+    tokens, within the storage tolerance (the scan's chunked tile products and
+    the step's per-row sums round differently)."""
+    p = W.m3_problem(2, 150, 4, 64, 64, ngroups=2, nangles=32, io=io, seed=5, with_h0=True)
+    a = m3_device_args(p)
+    out, fs, _ = msc.msc_mamba3_siso_scan_fwd(**a, want_saved_states=False)
+    S = a["h0"].clone()
+    xp = torch.zeros((2, 4, 64), device="cuda")
+    bp = torch.zeros((2, 4, 64), device="cuda")
+    ph = torch.zeros((2, 4, 32), device="cuda")
+    outs = []
+    for t in range(p.seqlen):
+        c = lambda k: a[k][:, t].contiguous()
+        outs.append(msc.msc_mamba3_siso_state_update(
+            S, xp, bp, ph, c("x"), c("B"), c("C"), c("alpha"), c("beta"), c("gamma"), c("theta"),
+            D=a["D"], z=c("z")))
+    torch.cuda.synchronize()
+    assert_close("out", host(torch.stack(outs, dim=1)), host(out), TOL[io])
+    assert_close("final_state", host(S), host(fs), TOL[io])
+
+
+def test_m3_state_update_deterministic(msc):
+    q = W.m3su_problem(4, 8, 64, 64, nangles=32, io="bf16", seed=2, n_pool=3, random_state=True)
+    runs = []
+    for _ in range(2):
+        S, xp, bp, ph = _su_device_state(q)
+        for s in q.steps:
+            o = msc.msc_mamba3_siso_state_update(S, xp, bp, ph, dev(s["x"]), dev(s["B"]),
+                                                 dev(s["C"]), dev(s["alpha"]), dev(s["beta"]),
+                                                 dev(s["gamma"]), dev(s["theta"]), D=dev(q.D),
+                                                 z=dev(s["z"]))
+        torch.cuda.synchronize()
+        runs.append((o.clone(), S.clone(), bp.clone(), ph.clone()))
+    for x, y in zip(*runs):
+        assert torch.equal(x, y)
+
+
+def test_m3_state_update_workload_sampled(msc):
+    """The Mamba-3 decode workload (B256 H24 P64 N64 K32, bf16 inputs, f32
+    state, 1000 steps cycling a pool of 8 input sets) on the GPU; the oracle
+    follows 6 fixed (b, h) rows through all 1000 steps (rows are independent)."""
+    q = W.make("m3su_bf16_b256_h24_p64_n64_k32_x1000")
+    S, xp, bp, ph = _su_device_state(q)
+    D = dev(q.D)
+    steps = [{k: dev(v) for k, v in s.items()} for s in q.steps]
+    rows = [(0, 0), (17, 5), (100, 23), (128, 12), (201, 7), (255, 23)]
+    bi = np.array([r[0] for r in rows])
+    hi = np.array([r[1] for r in rows])
+    outs = []
+    for t in range(1000):
+        s = steps[t % 8]
+        o = msc.msc_mamba3_siso_state_update(S, xp, bp, ph, s["x"], s["B"], s["C"], s["alpha"],
+                                             s["beta"], s["gamma"], s["theta"], D=D, z=s["z"])
+        if t % 250 == 249:
+            outs.append((t, host(o)[bi, hi]))
+    torch.cuda.synchronize()
+    # oracle: the sampled rows as one problem of 6 batch rows with one head each
+    f = lambda t: t.as_f64()
+    pool = [dict(x=f(s["x"])[bi, hi][:, None], z=f(s["z"])[bi, hi][:, None],
+                 B=f(s["B"])[bi], C=f(s["C"])[bi], alpha=f(s["alpha"])[bi, hi][:, None],
+                 beta=f(s["beta"])[bi, hi][:, None], gamma=f(s["gamma"])[bi, hi][:, None],
+                 theta=f(s["theta"])[bi, hi][:, None]) for s in q.steps]
+    Dh = q.D.astype(np.float64)[hi]
+    ref = [np.zeros((6, 1, 64, 64)), np.zeros((6, 1, 64)), np.zeros((6, 1, 64)),
+           np.zeros((6, 1, 32))]
+    k = 0
+    for t in range(1000):
+        s = pool[t % 8]
+        # per-row D: run each row as its own head-0 problem with its own D
+        new = [np.empty_like(r) for r in ref]
+        o_ref = np.empty((6, 1, 64))
+        for r in range(6):
+            res = oracle.m3_state_update(*[a[r:r + 1] for a in ref], s["x"][r:r + 1],
+                                         s["B"][r:r + 1], s["C"][r:r + 1], s["alpha"][r:r + 1],
+                                         s["beta"][r:r + 1], s["gamma"][r:r + 1],
+                                         s["theta"][r:r + 1], D=Dh[r:r + 1], z=s["z"][r:r + 1])
+            for a, b_ in zip(new, res[:4]):
+                a[r:r + 1] = b_
+            o_ref[r:r + 1] = res[4]
+        ref = new
+        if k < len(outs) and outs[k][0] == t:
+            assert_close(f"out@{t}", outs[k][1], o_ref[:, 0], TOL["bf16"])
+            k += 1
+    assert_close("state", host(S)[bi, hi], ref[0][:, 0], TOL["bf16"])
+    assert_close("phi", host(ph)[bi, hi], ref[3][:, 0], TOL["bf16"])
