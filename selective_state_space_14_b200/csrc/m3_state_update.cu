@@ -47,6 +47,21 @@ __global__ void __launch_bounds__(kSUThreads) m3_state_update_kernel(const M3SUP
   const int64_t g = h / (p.H / p.G);
   const int K = (int)p.K;
   float *sBt = sm + hl * kPer, *sCt = sBt + N, *sBp = sCt + N, *sXp = sBp + N;
+  const int row = j / kTPR, q = j % kTPR;
+  float4 *srow = reinterpret_cast<float4 *>(p.state + (bh * P + row) * N);
+
+  // this thread's state entries and scalars, in flight while the head's
+  // rotation runs
+  float4 s[4];
+  float al = 0.f, be = 0.f, ga = 0.f, xv = 0.f;
+  if (live) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) s[i] = srow[i * kTPR + q];
+    al = ldf<T>(p.alpha, bh);
+    be = ldf<T>(p.beta, bh);
+    ga = ldf<T>(p.gamma, bh);
+    xv = ldf<T>(p.x, bh * P + row);
+  }
 
   // ---- the step's rotated B and C; the carried x_prev and bt_prev ----------
   if (live) {
@@ -76,17 +91,10 @@ __global__ void __launch_bounds__(kSUThreads) m3_state_update_kernel(const M3SUP
   for (int i = j; i < P; i += kTPH) p.x_prev[bh * P + i] = ldf<T>(p.x, bh * P + i);
 
   // ---- the state rows ---------------------------------------------------------
-  const int row = j / kTPR, q = j % kTPR;
-  const float al = ldf<T>(p.alpha, bh), be = ldf<T>(p.beta, bh), ga = ldf<T>(p.gamma, bh);
-  const float xv = ldf<T>(p.x, bh * P + row);
   const float bxq = be * sXp[row], gx = ga * xv;
-  float4 *srow = reinterpret_cast<float4 *>(p.state + (bh * P + row) * N);
   const float4 *vBt = reinterpret_cast<const float4 *>(sBt);
   const float4 *vCt = reinterpret_cast<const float4 *>(sCt);
   const float4 *vBp = reinterpret_cast<const float4 *>(sBp);
-  float4 s[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) s[i] = srow[i * kTPR + q];
   float y = 0.f;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
