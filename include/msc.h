@@ -27,10 +27,12 @@
  *     on the caller's stream; results are ready when the stream reaches them.
  *   * Optional pointers may be NULL, meaning "absent": no h0 (zero initial
  *     state), no z (no gate), no D (no skip), no delta_bias, no final state.
- *   * io tensors (MSC_F32 or MSC_BF16, chosen per call) are read and written
- *     in that dtype; every accumulation is f32 (the mamba-rs README,
- *     "Features": "every kernel accumulates in f32"), and recurrent states and
- *     reduced gradients are always f32.
+ *   * io tensors (MSC_F32, MSC_BF16 or MSC_F16, chosen per call; "f32, bf16
+ *     and f16 storage", mamba-rs README, "Features") are read and written in
+ *     that dtype; every accumulation is f32 (the same README: "every kernel
+ *     accumulates in f32"), and recurrent states and reduced gradients are
+ *     always f32.  f16 values are IEEE binary16: results past its range
+ *     (65504) become infinite in the stored outputs.
  *   * Results are bit-identical from run to run for the same inputs on the
  *     same GPU and build: there are no atomics and every cross-thread
  *     reduction has a fixed order (the "same bits run to run" guarantee of
@@ -67,7 +69,7 @@ typedef enum {
   MSC_ERR_WORKSPACE = 5    /* workspace pointer NULL or smaller than required   */
 } msc_status;
 
-typedef enum { MSC_F32 = 0, MSC_BF16 = 1 } msc_dtype;
+typedef enum { MSC_F32 = 0, MSC_BF16 = 1, MSC_F16 = 2 } msc_dtype;
 
 /* Message for the last failure on this thread ("" after a success). */
 const char *msc_last_error(void);

@@ -53,11 +53,12 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
       return fail(MSC_ERR_ALIGNMENT, "%s: %s is not 16-byte aligned", fn, name);    \
   } while (0)
 
-size_t io_size(int32_t dt) { return dt == MSC_BF16 ? 2 : 4; }
+size_t io_size(int32_t dt) { return dt == MSC_F32 ? 4 : 2; }
 
 msc_status check_dtype(const char *fn, int32_t dt) {
-  if (dt != MSC_F32 && dt != MSC_BF16)
-    return fail(MSC_ERR_INVALID_ARG, "%s: io_dtype %d is not MSC_F32 (0) or MSC_BF16 (1)", fn,
+  if (dt != MSC_F32 && dt != MSC_BF16 && dt != MSC_F16)
+    return fail(MSC_ERR_INVALID_ARG,
+                "%s: io_dtype %d is not MSC_F32 (0), MSC_BF16 (1) or MSC_F16 (2)", fn,
                 (int)dt);
   return MSC_OK;
 }
@@ -150,7 +151,7 @@ msc_status msc_selective_scan_fwd(const msc_ss_fwd_args *a, msc_stream_t stream)
   OPTIONAL_PTR(fn, "saved_states", a->saved_states);
 
   msc::M1Params p = {};
-  p.io_bf16 = a->io_dtype == MSC_BF16;
+  p.io = a->io_dtype;
   p.B = B; p.D = D; p.N = N; p.L = L; p.G = a->ngroups;
   p.softplus = a->delta_softplus;
   p.vec = (L * (int64_t)io_size(a->io_dtype)) % 16 == 0;
@@ -218,7 +219,7 @@ msc_status msc_selective_scan_bwd(const msc_ss_bwd_args *a, void *workspace,
     return fail(MSC_ERR_ALIGNMENT, "%s: workspace is not 16-byte aligned", fn);
 
   msc::M1Params p = {};
-  p.io_bf16 = a->io_dtype == MSC_BF16;
+  p.io = a->io_dtype;
   p.B = B; p.D = D; p.N = N; p.L = L; p.G = G;
   p.softplus = a->delta_softplus;
   p.vec = (L * (int64_t)io_size(a->io_dtype)) % 16 == 0;
@@ -259,7 +260,7 @@ msc_status msc_ssm_state_update(const msc_su_args *a, msc_stream_t stream) {
   OPTIONAL_PTR(fn, "delta_bias", a->delta_bias);
   OPTIONAL_PTR(fn, "z", a->z);
   msc::SUParams p = {};
-  p.io_bf16 = a->io_dtype == MSC_BF16;
+  p.io = a->io_dtype;
   p.B = a->batch; p.D = a->dim; p.N = a->dstate; p.G = a->ngroups;
   p.softplus = a->delta_softplus;
   p.state = a->state; p.x = a->x; p.delta = a->delta; p.Bm = a->Bm; p.Cm = a->Cm; p.z = a->z;

@@ -46,8 +46,9 @@ msc_status check_m3(const char *fn, const Args *a) {
   if (a->struct_size < sizeof(Args))
     return api_fail(MSC_ERR_INVALID_ARG, "%s: struct_size %u is smaller than the struct (%zu)",
                     fn, a->struct_size, sizeof(Args));
-  if (a->io_dtype != MSC_F32 && a->io_dtype != MSC_BF16)
-    return api_fail(MSC_ERR_INVALID_ARG, "%s: io_dtype %d is not MSC_F32 (0) or MSC_BF16 (1)",
+  if (a->io_dtype != MSC_F32 && a->io_dtype != MSC_BF16 && a->io_dtype != MSC_F16)
+    return api_fail(MSC_ERR_INVALID_ARG,
+                    "%s: io_dtype %d is not MSC_F32 (0), MSC_BF16 (1) or MSC_F16 (2)",
                     fn, (int)a->io_dtype);
   if (a->batch < 0 || a->seqlen < 0 || a->nheads < 1 || a->ngroups < 1 || a->nangles < 0)
     return api_fail(MSC_ERR_INVALID_ARG,
@@ -111,7 +112,7 @@ msc_status msc_mamba3_siso_scan_fwd(const msc_m3_fwd_args *a, msc_stream_t strea
   M3_OPTIONAL(fn, "z", a->z);
   M3_OPTIONAL(fn, "saved_states", a->saved_states);
   msc::M3Params p = {};
-  p.io_bf16 = a->io_dtype == MSC_BF16;
+  p.io = a->io_dtype;
   p.B = B; p.L = a->seqlen; p.H = H; p.P = P; p.N = N; p.G = a->ngroups; p.K = a->nangles;
   p.x = a->x; p.z = a->z; p.Bm = a->Bm; p.Cm = a->Cm;
   p.alpha = a->alpha; p.beta = a->beta; p.gamma = a->gamma; p.theta = a->theta;
@@ -178,7 +179,7 @@ msc_status msc_mamba3_siso_scan_bwd(const msc_m3_bwd_args *a, void *workspace,
   if (workspace && !aligned16(workspace))
     return api_fail(MSC_ERR_ALIGNMENT, "%s: workspace is not 16-byte aligned", fn);
   msc::M3Params p = {};
-  p.io_bf16 = a->io_dtype == MSC_BF16;
+  p.io = a->io_dtype;
   p.B = B; p.L = L; p.H = H; p.P = P; p.N = N; p.G = G; p.K = K;
   p.x = a->x; p.z = a->z; p.Bm = a->Bm; p.Cm = a->Cm;
   p.alpha = a->alpha; p.beta = a->beta; p.gamma = a->gamma; p.theta = a->theta;
@@ -195,8 +196,9 @@ msc_status msc_mamba3_siso_state_update(const msc_m3_su_args *a, msc_stream_t st
   if (a->struct_size < sizeof(msc_m3_su_args))
     return api_fail(MSC_ERR_INVALID_ARG, "%s: struct_size %u is smaller than the struct (%zu)",
                     fn, a->struct_size, sizeof(msc_m3_su_args));
-  if (a->io_dtype != MSC_F32 && a->io_dtype != MSC_BF16)
-    return api_fail(MSC_ERR_INVALID_ARG, "%s: io_dtype %d is not MSC_F32 (0) or MSC_BF16 (1)",
+  if (a->io_dtype != MSC_F32 && a->io_dtype != MSC_BF16 && a->io_dtype != MSC_F16)
+    return api_fail(MSC_ERR_INVALID_ARG,
+                    "%s: io_dtype %d is not MSC_F32 (0), MSC_BF16 (1) or MSC_F16 (2)",
                     fn, (int)a->io_dtype);
   if (a->batch < 0 || a->nheads < 1 || a->ngroups < 1 || a->nangles < 0)
     return api_fail(MSC_ERR_INVALID_ARG,
@@ -231,7 +233,7 @@ msc_status msc_mamba3_siso_state_update(const msc_m3_su_args *a, msc_stream_t st
   M3_OPTIONAL(fn, "z", a->z);
   M3_OPTIONAL(fn, "D", a->D);
   msc::M3SUParams p = {};
-  p.io_bf16 = a->io_dtype == MSC_BF16;
+  p.io = a->io_dtype;
   p.B = a->batch; p.H = a->nheads; p.P = a->headdim; p.N = a->dstate; p.G = a->ngroups;
   p.K = a->nangles;
   p.state = a->state; p.x_prev = a->x_prev; p.bt_prev = a->bt_prev; p.phi = a->phi;

@@ -1,17 +1,21 @@
 // common.cuh -- device helpers shared by the sm_100a kernels of libmsc.
 //
-// io tensors are f32 or bf16; all arithmetic is f32.  Loads of a lane's run of
+// io tensors are f32, bf16 or f16; all arithmetic is f32.  Loads of a lane's run of
 // consecutive elements use 16-byte vector accesses when the run is aligned and
 // in bounds, element accesses otherwise (ragged tails, odd row lengths).
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+
+#include <type_traits>
 
 namespace msc {
 
 using bf16 = __nv_bfloat16;
+using f16 = __half;
 
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -99,10 +103,12 @@ __device__ __forceinline__ float2 ex2_2(float2 v) { return make_float2(ex2(v.x),
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float to_f32(float v) { return v; }
 __device__ __forceinline__ float to_f32(bf16 v) { return __bfloat162float(v); }
+__device__ __forceinline__ float to_f32(f16 v) { return __half2float(v); }
 
 template <typename T> __device__ __forceinline__ T from_f32(float v);
 template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
 template <> __device__ __forceinline__ bf16 from_f32<bf16>(float v) { return __float2bfloat16_rn(v); }
+template <> __device__ __forceinline__ f16 from_f32<f16>(float v) { return __float2half_rn(v); }
 
 // unpack one 32-bit word holding two bf16 (low half first in memory)
 __device__ __forceinline__ void unpack_bf16x2(uint32_t w, float &lo, float &hi) {
@@ -114,6 +120,27 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t l = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(lo));
   uint32_t h = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi));
   return l | (h << 16);
+}
+
+// the same for either 16-bit io type (bf16 or f16)
+template <typename T>
+__device__ __forceinline__ void unpack2(uint32_t w, float &lo, float &hi) {
+  if constexpr (std::is_same_v<T, bf16>) {
+    unpack_bf16x2(w, lo, hi);
+  } else {
+    lo = __half2float(__ushort_as_half((unsigned short)(w & 0xffffu)));
+    hi = __half2float(__ushort_as_half((unsigned short)(w >> 16)));
+  }
+}
+template <typename T>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+  if constexpr (std::is_same_v<T, bf16>) {
+    return pack_bf16x2(lo, hi);
+  } else {
+    const uint32_t l = (uint32_t)__half_as_ushort(__float2half_rn(lo));
+    const uint32_t h = (uint32_t)__half_as_ushort(__float2half_rn(hi));
+    return l | (h << 16);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -146,23 +173,33 @@ __device__ __forceinline__ void load_run(const float *p, int64_t t0, int64_t n, 
   }
 }
 
-template <int K, Cache C = Cache::kStream>
-__device__ __forceinline__ void load_run(const bf16 *p, int64_t t0, int64_t n, bool vec,
-                                         float (&v)[K], float fill) {
-  static_assert(K % 8 == 0, "bf16 run length must be a multiple of 8");
+template <int K, Cache C = Cache::kStream, typename T16>
+__device__ __forceinline__ void load_run16(const T16 *p, int64_t t0, int64_t n, bool vec,
+                                           float (&v)[K], float fill) {
+  static_assert(K % 8 == 0, "16-bit run length must be a multiple of 8");
   if (vec && t0 + K <= n) {
 #pragma unroll
     for (int j = 0; j < K / 8; ++j) {
       uint4 r = ld16<C>(p + t0 + 8 * j);
-      unpack_bf16x2(r.x, v[8 * j + 0], v[8 * j + 1]);
-      unpack_bf16x2(r.y, v[8 * j + 2], v[8 * j + 3]);
-      unpack_bf16x2(r.z, v[8 * j + 4], v[8 * j + 5]);
-      unpack_bf16x2(r.w, v[8 * j + 6], v[8 * j + 7]);
+      unpack2<T16>(r.x, v[8 * j + 0], v[8 * j + 1]);
+      unpack2<T16>(r.y, v[8 * j + 2], v[8 * j + 3]);
+      unpack2<T16>(r.z, v[8 * j + 4], v[8 * j + 5]);
+      unpack2<T16>(r.w, v[8 * j + 6], v[8 * j + 7]);
     }
   } else {
 #pragma unroll
-    for (int i = 0; i < K; ++i) v[i] = (t0 + i < n) ? __bfloat162float(p[t0 + i]) : fill;
+    for (int i = 0; i < K; ++i) v[i] = (t0 + i < n) ? to_f32(p[t0 + i]) : fill;
   }
+}
+template <int K, Cache C = Cache::kStream>
+__device__ __forceinline__ void load_run(const bf16 *p, int64_t t0, int64_t n, bool vec,
+                                         float (&v)[K], float fill) {
+  load_run16<K, C>(p, t0, n, vec, v, fill);
+}
+template <int K, Cache C = Cache::kStream>
+__device__ __forceinline__ void load_run(const f16 *p, int64_t t0, int64_t n, bool vec,
+                                         float (&v)[K], float fill) {
+  load_run16<K, C>(p, t0, n, vec, v, fill);
 }
 
 template <int K>
@@ -182,23 +219,33 @@ __device__ __forceinline__ void store_run(float *p, int64_t t0, int64_t n, bool 
   }
 }
 
-template <int K>
-__device__ __forceinline__ void store_run(bf16 *p, int64_t t0, int64_t n, bool vec,
-                                          const float (&v)[K]) {
+template <int K, typename T16>
+__device__ __forceinline__ void store_run16(T16 *p, int64_t t0, int64_t n, bool vec,
+                                            const float (&v)[K]) {
   if (vec && t0 + K <= n) {
 #pragma unroll
     for (int j = 0; j < K / 8; ++j) {
-      uint4 r = make_uint4(pack_bf16x2(v[8 * j + 0], v[8 * j + 1]),
-                           pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
-                           pack_bf16x2(v[8 * j + 4], v[8 * j + 5]),
-                           pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
+      uint4 r = make_uint4(pack2<T16>(v[8 * j + 0], v[8 * j + 1]),
+                           pack2<T16>(v[8 * j + 2], v[8 * j + 3]),
+                           pack2<T16>(v[8 * j + 4], v[8 * j + 5]),
+                           pack2<T16>(v[8 * j + 6], v[8 * j + 7]));
       __stcs(reinterpret_cast<uint4 *>(p + t0 + 8 * j), r);
     }
   } else {
 #pragma unroll
     for (int i = 0; i < K; ++i)
-      if (t0 + i < n) p[t0 + i] = __float2bfloat16_rn(v[i]);
+      if (t0 + i < n) p[t0 + i] = from_f32<T16>(v[i]);
   }
+}
+template <int K>
+__device__ __forceinline__ void store_run(bf16 *p, int64_t t0, int64_t n, bool vec,
+                                          const float (&v)[K]) {
+  store_run16<K>(p, t0, n, vec, v);
+}
+template <int K>
+__device__ __forceinline__ void store_run(f16 *p, int64_t t0, int64_t n, bool vec,
+                                          const float (&v)[K]) {
+  store_run16<K>(p, t0, n, vec, v);
 }
 
 // ---------------------------------------------------------------------------

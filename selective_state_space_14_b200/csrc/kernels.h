@@ -10,7 +10,7 @@ namespace msc {
 
 // ---------------------------------------------------------------- Mamba-1 --
 struct M1Params {
-  int io_bf16;
+  int io;  // msc_dtype: 0 f32, 1 bf16, 2 f16
   int64_t B, D, N, L, G;
   int softplus;
   bool vec;  // rows of length L are 16-byte aligned for vector access
@@ -46,7 +46,7 @@ size_t m1_bwd_workspace_bytes(int64_t B, int64_t D, int64_t N, int64_t L, int64_
 
 // ------------------------------------------------------------ decode step --
 struct SUParams {
-  int io_bf16;
+  int io;  // msc_dtype: 0 f32, 1 bf16, 2 f16
   int64_t B, D, N, G;
   int softplus;
   float *state;
@@ -59,7 +59,7 @@ cudaError_t launch_state_update(const SUParams &p, cudaStream_t s);
 // ---------------------------------------------------------- Mamba-3 SISO --
 #define MSC_M3_CHUNK_STEPS 64  // steps per chunk (= the saved-state interval)
 struct M3Params {
-  int io_bf16;
+  int io;  // msc_dtype: 0 f32, 1 bf16, 2 f16
   int64_t B, L, H, P, N, G, K;
   const void *x, *z, *Bm, *Cm, *alpha, *beta, *gamma, *theta;
   const float *Dp, *h0;
@@ -82,7 +82,7 @@ bool m3_supported(int64_t P, int64_t N);
 
 // Mamba-3 SISO single-token state update (decode)
 struct M3SUParams {
-  int io_bf16;
+  int io;  // msc_dtype: 0 f32, 1 bf16, 2 f16
   int64_t B, H, P, N, G, K;
   float *state, *x_prev, *bt_prev, *phi;
   const void *x, *z, *Bm, *Cm, *alpha, *beta, *gamma, *theta;

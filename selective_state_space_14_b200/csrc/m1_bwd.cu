@@ -522,7 +522,11 @@ size_t m1_bwd_workspace_bytes(int64_t B, int64_t D, int64_t N, int64_t L, int64_
 }
 
 cudaError_t launch_m1_bwd(const M1Params &p, cudaStream_t s) {
-  return p.io_bf16 ? launch_n<bf16>(p, s) : launch_n<float>(p, s);
+  switch (p.io) {
+    case 1: return launch_n<bf16>(p, s);
+    case 2: return launch_n<f16>(p, s);
+    default: return launch_n<float>(p, s);
+  }
 }
 
 }  // namespace msc

@@ -297,7 +297,11 @@ cudaError_t launch_n(const M1Params &p, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_m1_fwd(const M1Params &p, cudaStream_t s) {
-  return p.io_bf16 ? launch_n<bf16>(p, s) : launch_n<float>(p, s);
+  switch (p.io) {
+    case 1: return launch_n<bf16>(p, s);
+    case 2: return launch_n<f16>(p, s);
+    default: return launch_n<float>(p, s);
+  }
 }
 
 }  // namespace msc

@@ -55,12 +55,12 @@ __device__ __forceinline__ void ld8(const void *base, int64_t j, bool valid, flo
     for (int e = 0; e < 8; ++e) v[e] = 0.f;
     return;
   }
-  if constexpr (std::is_same_v<T, bf16>) {
-    const uint4 r = __ldg(reinterpret_cast<const uint4 *>(static_cast<const bf16 *>(base) + j));
-    unpack_bf16x2(r.x, v[0], v[1]);
-    unpack_bf16x2(r.y, v[2], v[3]);
-    unpack_bf16x2(r.z, v[4], v[5]);
-    unpack_bf16x2(r.w, v[6], v[7]);
+  if constexpr (sizeof(T) == 2) {
+    const uint4 r = __ldg(reinterpret_cast<const uint4 *>(static_cast<const T *>(base) + j));
+    unpack2<T>(r.x, v[0], v[1]);
+    unpack2<T>(r.y, v[2], v[3]);
+    unpack2<T>(r.z, v[4], v[5]);
+    unpack2<T>(r.w, v[6], v[7]);
   } else {
     const float4 a = __ldg(reinterpret_cast<const float4 *>(static_cast<const float *>(base) + j));
     const float4 c = __ldg(reinterpret_cast<const float4 *>(static_cast<const float *>(base) + j + 4));
@@ -607,7 +607,11 @@ size_t m3_bwd_workspace_bytes(int64_t B, int64_t L, int64_t H, int64_t P, int64_
 }
 
 cudaError_t launch_m3_bwd(const M3Params &p, cudaStream_t s) {
-  return p.io_bf16 ? launch_p<bf16>(p, s) : launch_p<float>(p, s);
+  switch (p.io) {
+    case 1: return launch_p<bf16>(p, s);
+    case 2: return launch_p<f16>(p, s);
+    default: return launch_p<float>(p, s);
+  }
 }
 
 }  // namespace msc

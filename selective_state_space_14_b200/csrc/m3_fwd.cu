@@ -244,10 +244,14 @@ bool m3_supported(int64_t P, int64_t N) {
   return (P == 16 || P == 32 || P == 64) && (N == 16 || N == 32 || N == 64);
 }
 
-// bf16 io runs the tcgen05 kernel (m3_fwd_umma.cu); f32 io this one, whose
-// contractions are f32 on the CUDA cores.
+// bf16 io runs the tcgen05 kernel (m3_fwd_umma.cu); f32 and f16 io this one,
+// whose contractions are f32 on the CUDA cores.
 cudaError_t launch_m3_fwd(const M3Params &p, cudaStream_t s) {
-  return p.io_bf16 ? launch_m3_fwd_umma(p, s) : launch_p<float>(p, s);
+  switch (p.io) {
+    case 1: return launch_m3_fwd_umma(p, s);
+    case 2: return launch_p<f16>(p, s);
+    default: return launch_p<float>(p, s);
+  }
 }
 
 }  // namespace msc

@@ -100,7 +100,11 @@ cudaError_t launch_t(const SUParams &p, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_state_update(const SUParams &p, cudaStream_t s) {
-  return p.io_bf16 ? launch_t<bf16>(p, s) : launch_t<float>(p, s);
+  switch (p.io) {
+    case 1: return launch_t<bf16>(p, s);
+    case 2: return launch_t<f16>(p, s);
+    default: return launch_t<float>(p, s);
+  }
 }
 
 }  // namespace msc

@@ -19,7 +19,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmsc.so")
 
-MSC_F32, MSC_BF16 = 0, 1
+MSC_F32, MSC_BF16, MSC_F16 = 0, 1, 2
 MSC_M1_SAVE_INTERVAL = 8
 
 STATUS = {0: "MSC_OK", 1: "MSC_ERR_INVALID_ARG", 2: "MSC_ERR_UNSUPPORTED", 3: "MSC_ERR_ALIGNMENT",
@@ -154,6 +154,8 @@ def _io(t: torch.Tensor) -> int:
         return MSC_BF16
     if t.dtype == torch.float32:
         return MSC_F32
+    if t.dtype == torch.float16:
+        return MSC_F16
     raise TypeError(f"unsupported io dtype {t.dtype}")
 
 

@@ -30,6 +30,7 @@ SEED_BASE = 20261202
 
 F32 = "f32"
 BF16 = "bf16"
+F16 = "f16"
 
 
 def round_to_bf16_bits(x: np.ndarray) -> np.ndarray:
@@ -48,7 +49,8 @@ def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
 class Tensor:
     """A stored tensor: its io dtype and its payload.
 
-    ``data`` is float32 for f32 tensors and uint16 bit patterns for bf16.
+    ``data`` is float32 for f32 tensors, uint16 bit patterns for bf16 and
+    float16 for f16 (IEEE binary16, numpy's round-to-nearest-even cast).
     """
 
     dtype: str
@@ -61,6 +63,8 @@ class Tensor:
     def as_f32(self) -> np.ndarray:
         if self.dtype == BF16:
             return bf16_bits_to_f32(self.data)
+        if self.dtype == F16:
+            return self.data.astype(np.float32)
         return self.data
 
     def as_f64(self) -> np.ndarray:
@@ -77,6 +81,8 @@ def store(x: np.ndarray, dtype: str) -> Tensor:
         return Tensor(BF16, round_to_bf16_bits(x))
     if dtype == F32:
         return Tensor(F32, x)
+    if dtype == F16:
+        return Tensor(F16, x.astype(np.float16))
     raise ValueError(dtype)
 
 

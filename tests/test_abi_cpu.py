@@ -64,6 +64,14 @@ def test_fwd_rejects_short_struct():
 
 def test_fwd_rejects_bad_dtype():
     assert _call_fwd(_fwd_args(io_dtype=7)) == INVALID and "io_dtype" in _err()
+    assert _call_fwd(_fwd_args(io_dtype=3)) == INVALID and "MSC_F16" in _err()
+
+
+def test_f16_is_an_io_dtype():
+    """MSC_F16 passes the dtype check: the call goes on to the pointer checks
+    (a NULL u stops it there, before any launch)."""
+    assert _call_fwd(_fwd_args(io_dtype=msc.MSC_F16, u=None)) == INVALID
+    assert "io_dtype" not in _err() and "u is NULL" in _err()
 
 
 @pytest.mark.parametrize("field,value,status,word", [

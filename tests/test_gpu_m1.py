@@ -77,6 +77,11 @@ CASES = [
     (1, 24, 64, 96, 1, "bf16", True, True, True, True, True),
     (3, 36, 16, 1024, 3, "bf16", True, False, True, True, True),
     (1, 20, 16, 40, 1, "f32", True, True, True, True, True),
+    # f16 storage: aligned rows with a ragged block, d_state 64, unaligned rows
+    (2, 96, 16, 700, 1, "f16", True, True, True, True, True),
+    (1, 24, 64, 96, 1, "f16", True, True, True, True, True),
+    (1, 7, 5, 513, 1, "f16", False, True, True, False, True),
+    (2, 100, 32, 1000, 2, "f16", True, True, True, True, True),
 ]
 
 
@@ -176,7 +181,7 @@ def test_state_update_equals_scan_step_bitwise(msc):
     assert torch.equal(st, fs)
 
 
-@pytest.mark.parametrize("io", ["f32", "bf16"])
+@pytest.mark.parametrize("io", ["f32", "bf16", "f16"])
 def test_state_update_chain(msc, io):
     """60 chained decode steps against the oracle's chained steps."""
     q = W.su_problem(3, 70, 16, io=io, seed=3, random_state=True, n_pool=60)

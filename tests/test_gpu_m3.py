@@ -49,6 +49,8 @@ FWD_CASES = [
     (2, 200, 4, 64, 64, 2, 32, "bf16", True, True, True),
     (1, 130, 2, 32, 16, 1, 0, "bf16", True, False, True),
     (1, 640, 2, 64, 64, 1, 32, "bf16", True, True, True),
+    (2, 200, 4, 64, 64, 2, 32, "f16", True, True, True),
+    (1, 65, 3, 16, 32, 3, 16, "f16", False, True, True),
 ]
 
 
@@ -142,6 +144,8 @@ BWD_CASES = [
     (2, 200, 4, 64, 64, 2, 32, "f32", True, True, True),
     (1, 130, 2, 32, 64, 1, 0, "f32", True, False, True),
     (2, 300, 4, 64, 64, 1, 32, "bf16", True, True, False),
+    (1, 130, 2, 32, 64, 1, 10, "f16", True, True, True),
+    (2, 70, 2, 64, 64, 1, 32, "f16", True, False, True),
 ]
 
 
@@ -206,6 +210,8 @@ SU_CASES = [
     (3, 5, 64, 16, 1, 0, "bf16", False, True, False, 20),
     (9, 2, 16, 16, 1, 8, "bf16", True, False, True, 20),
     (2, 4, 32, 32, 4, 16, "bf16", True, True, True, 20),
+    (3, 4, 64, 64, 1, 32, "f16", True, True, True, 12),
+    (2, 6, 16, 32, 2, 8, "f16", False, True, True, 12),
 ]
 
 
