@@ -16,11 +16,13 @@
 // row and walks the sequence backwards.
 //
 //   * Blocks of kBlk = 32 steps.  The raw inputs of a block (u, delta, z,
-//     dout of the CTA's channels, the B and C rows, and the forward's saved
-//     states) are brought into shared memory by cp.async one block ahead,
-//     into the other half of a double buffer, so no warp waits on a global
-//     load; B and C are converted once per block into an f32 table of
-//     (B[2p], B[2p+1], C[2p], C[2p+1]) per (step, pair).
+//     dout of the CTA's channels, the B and C rows) are brought into shared
+//     memory by cp.async one block ahead, into the other half of a double
+//     buffer, from a table of row addresses built once per CTA, so no warp
+//     waits on a global load; B and C are converted once per block, eight
+//     steps of a pair at a time, into an f32 table of (B[2p], B[2p+1], C[2p],
+//     C[2p+1]) per (step, pair).  Each thread loads its pair of the
+//     forward's saved state straight into registers, one window ahead.
 //   * Windows of kS = 8 steps (the forward's saved-state interval), walked
 //     in reverse.  Per window the lanes p < kS of a channel first derive the
 //     per-token values of step p (softplus, gates) and share them through a
@@ -65,11 +67,11 @@ struct BwdSmem {
   static constexpr int kCh = Lay::kCh;
   static constexpr int kChW = Lay::kChPerWarp;
   // raw stage (one buffer; two are kept): tokens [4][kCh][kBlk] T in the
-  // order u, delta, z, dout; bc [2][kN][kBlk] T; saved [kCh][kWin][kN] f32
+  // order u, delta, z, dout; bc [2][kN][kBlk] T
   static constexpr int kTokBytes = 4 * kCh * kBlk * (int)sizeof(T);
   static constexpr int kBCBytes = 2 * kN * kBlk * (int)sizeof(T);
-  static constexpr int kSavBytes = kCh * kWin * kN * 4;
-  static constexpr int kStageBytes = kTokBytes + kBCBytes + kSavBytes;
+  static constexpr int kStageBytes = kTokBytes + kBCBytes;
+  static constexpr int kRows = 4 * kCh + 2 * kN;  // staged rows: tokens, then B and C
   // byte offsets
   static constexpr int stage = 0;                                   // [2][kStageBytes]
   static constexpr int bcf = stage + 2 * kStageBytes;               // [2][kBlk][kP] float4
@@ -82,7 +84,9 @@ struct BwdSmem {
   static constexpr int rbc = tile + kWarps * kChW * kS * kTileRow * 16;  // [kCh][kS][kP] float4
   static constexpr int kAccRow = kBlk + 1;                          // floats per (tensor, n) row
   static constexpr int acc = rbc + kCh * kS * kP * 16;              // [2][kN][kBlk+1] f32
-  static constexpr int total = acc + 2 * kN * kAccRow * 4;
+  // global address of every staged row at t = 0 (0: absent row, zero-filled)
+  static constexpr int rows = (acc + 2 * kN * kAccRow * 4 + 7) / 8 * 8;  // [kRows] pointers
+  static constexpr int total = rows + kRows * 8;
   static_assert(kStageBytes % 16 == 0 && kTokBytes % 16 == 0 && kBCBytes % 16 == 0,
                 "stage regions must stay 16-byte aligned");
 };
@@ -92,104 +96,95 @@ __device__ __forceinline__ float ldsm(const unsigned char *base, int i) {
   return to_f32(reinterpret_cast<const T *>(base)[i]);
 }
 
-// Issue the copies of block kb's raw inputs into one stage buffer: token runs
-// of the CTA's channels, the B and C rows and the saved states of the block's
-// windows.  With vec (16-byte aligned rows) every 16-byte piece is one
-// cp.async that zero-fills what lies past the end of its row; otherwise the
-// elements are copied one by one (synchronously).  Entries past L, past the
-// last channel, past d_state or past the last saved state are never read as
-// data: the consumers test those bounds themselves.
+// The global address of every row the stage copies, at t = 0, once per CTA:
+// token rows (tensor k of u, delta, z, dout; channel cl) at k * kCh + cl, then
+// the B and C rows (state n) at 4 kCh + k * kN + n.  Rows that do not exist
+// (absent z, a channel past the group, a state past d_state) hold 0.
 template <typename T, int kN>
-__device__ __forceinline__ void issue_stage(const M1Params &p, unsigned char *st, int64_t b,
-                                            int64_t c_first, int64_t c_end, const T *Bg,
-                                            const T *Cg, int64_t kb, int64_t n_chunks,
-                                            bool vec_sav, int tid) {
+__device__ __forceinline__ void fill_rows(const M1Params &p, const T **rows, int64_t b,
+                                          int64_t c_first, int64_t c_end, const T *Bg,
+                                          const T *Cg, int tid) {
   using S = BwdSmem<T, kN>;
   constexpr int kCh = S::kCh;
-  constexpr int kThreads = kWarps * 32;
+  for (int r = tid; r < S::kRows; r += kWarps * 32) {
+    const T *row = nullptr;
+    if (r < 4 * kCh) {
+      const int k = r / kCh, cl = r % kCh;
+      const void *src = k == 0 ? p.u : (k == 1 ? p.delta : (k == 2 ? p.z : p.dout));
+      const int64_t c = c_first + cl;
+      if (src != nullptr && c < c_end) row = static_cast<const T *>(src) + (b * p.D + c) * p.L;
+    } else {
+      const int k = (r - 4 * kCh) / kN, n = (r - 4 * kCh) % kN;
+      if (n < p.N) row = (k == 0 ? Bg : Cg) + n * p.L;
+    }
+    rows[r] = row;
+  }
+}
+
+// Issue the copies of block kb's raw inputs into one stage buffer: the token
+// runs of the CTA's channels and the B and C rows, 16-byte pieces taken from
+// the row table.  With vec (16-byte aligned rows) every piece is one cp.async
+// that zero-fills what lies past the end of its row or past L; otherwise the
+// elements are copied one by one (synchronously).  Absent rows are zeros.
+template <typename T, int kN>
+__device__ __forceinline__ void issue_stage(const M1Params &p, unsigned char *st,
+                                            const T *const *rows, int64_t kb, int tid) {
+  using S = BwdSmem<T, kN>;
   constexpr int E = 16 / (int)sizeof(T);  // elements per 16-byte piece
-  constexpr int kPieces = kBlk / E;       // pieces per token / B / C run
-  const int64_t L = p.L, N = p.N;
+  constexpr int kPieces = kBlk / E;       // pieces per row
+  static_assert((kPieces & (kPieces - 1)) == 0, "pieces per row: a power of two");
+  const int64_t L = p.L;
   const int64_t t0 = kb * kBlk;
-  // token runs: (tensor k, channel cl, piece j)
+  const T *const fallback = static_cast<const T *>(p.Bm);  // a valid address for empty copies
 #pragma unroll 1
-  for (int u = tid; u < 4 * kCh * kPieces; u += kThreads) {
-    const int j = u % kPieces, r = u / kPieces;
-    const int cl = r % kCh, k = r / kCh;
-    const int64_t c = c_first + cl;
-    const void *src = k == 0 ? p.u : (k == 1 ? p.delta : (k == 2 ? p.z : p.dout));
-    const bool ok = src != nullptr && c < c_end;
-    const T *row = ok ? static_cast<const T *>(src) + (b * p.D + c) * L : static_cast<const T *>(p.u);
+  for (int u = tid; u < S::kRows * kPieces; u += kWarps * 32) {
+    const int j = u & (kPieces - 1), r = u / kPieces;
+    const T *row = rows[r];
     const int64_t t = t0 + j * E;
     const int64_t left = L - t;
-    const int valid = !ok || left <= 0 ? 0 : (left >= E ? E : (int)left);
+    const int valid = row == nullptr || left <= 0 ? 0 : (left >= E ? E : (int)left);
     T *dst = reinterpret_cast<T *>(st) + r * kBlk + j * E;
     if (p.vec) {
-      cp_async16(dst, valid > 0 ? row + t : row, valid * (int)sizeof(T));
+      cp_async16(dst, valid > 0 ? row + t : fallback, valid * (int)sizeof(T));
     } else {
 #pragma unroll
       for (int i = 0; i < E; ++i) dst[i] = i < valid ? row[t + i] : from_f32<T>(0.f);
-    }
-  }
-  // B and C rows: (tensor k, state n, piece j)
-#pragma unroll 1
-  for (int u = tid; u < 2 * kN * kPieces; u += kThreads) {
-    const int j = u % kPieces, r = u / kPieces;
-    const int n = r % kN, k = r / kN;
-    const bool ok = n < N;
-    const T *row = ok ? (k == 0 ? Bg : Cg) + n * L : Bg;
-    const int64_t t = t0 + j * E;
-    const int64_t left = L - t;
-    const int valid = !ok || left <= 0 ? 0 : (left >= E ? E : (int)left);
-    T *dst = reinterpret_cast<T *>(st + S::kTokBytes) + r * kBlk + j * E;
-    if (p.vec) {
-      cp_async16(dst, valid > 0 ? row + t : row, valid * (int)sizeof(T));
-    } else {
-#pragma unroll
-      for (int i = 0; i < E; ++i) dst[i] = i < valid ? row[t + i] : from_f32<T>(0.f);
-    }
-  }
-  // saved states: (channel cl, window w, 4 states); a channel's windows are
-  // consecutive in memory, kWin * N floats from chunk kb * kWin on
-#pragma unroll 1
-  for (int u = tid; u < kCh * kWin * (kN / 4); u += kThreads) {
-    const int j = u % (kWin * (kN / 4)), cl = u / (kWin * (kN / 4));
-    const int w = j / (kN / 4);
-    const int64_t n = 4 * (j % (kN / 4));
-    const int64_t c = c_first + cl;
-    const int64_t chunk = kb * kWin + w;
-    float *dst = reinterpret_cast<float *>(st + S::kTokBytes + S::kBCBytes) + (cl * kWin + w) * kN + n;
-    const bool ok = c < c_end && chunk < n_chunks && n < N;
-    const float *src = ok ? p.saved_in + ((b * p.D + c) * n_chunks + chunk) * N + n : p.saved_in;
-    const int valid = ok ? (int)(N - n < 4 ? N - n : 4) : 0;
-    if (vec_sav) {
-      cp_async16(dst, src, valid * 4);
-    } else {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) dst[i] = i < valid ? src[i] : 0.f;
     }
   }
   cp_async_commit();
 }
 
 // Block kb's B and C rows (raw stage) -> bcf[tt][p] = (B[2p], B[2p+1], C[2p],
-// C[2p+1]) in f32, zero past d_state and past L.
+// C[2p+1]) in f32.  The stage already holds zeros past d_state and past L.
+// One unit is a pair p and 8 consecutive steps: four 8-element row pieces in,
+// eight float4 out.
 template <typename T, int kN>
-__device__ __forceinline__ void convert_bc(const unsigned char *st, float4 *bcf, int64_t N,
-                                           int64_t L, int64_t kb, int tid) {
+__device__ __forceinline__ void convert_bc(const unsigned char *st, float4 *bcf, int tid) {
   using S = BwdSmem<T, kN>;
   constexpr int kP = S::kP;
-  const unsigned char *raw = st + S::kTokBytes;
-  for (int i = tid; i < kBlk * kP; i += kWarps * 32) {
-    const int tt = i % kBlk, pr = i / kBlk;
-    const bool tin = kb * kBlk + tt < L;
-    float v[4];
+  const T *raw = reinterpret_cast<const T *>(st + S::kTokBytes);
+  for (int u = tid; u < kP * (kBlk / 8); u += kWarps * 32) {
+    const int pr = u % kP, seg = u / kP;
+    float v[4][8];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      const int n = 2 * pr + (k & 1);
-      v[k] = (tin && n < N) ? ldsm<T>(raw, ((k >> 1) * kN + n) * kBlk + tt) : 0.f;
+      const T *src = raw + ((k >> 1) * kN + 2 * pr + (k & 1)) * kBlk + seg * 8;
+      if constexpr (sizeof(T) == 2) {
+        const uint4 w = *reinterpret_cast<const uint4 *>(src);
+        unpack2<T>(w.x, v[k][0], v[k][1]);
+        unpack2<T>(w.y, v[k][2], v[k][3]);
+        unpack2<T>(w.z, v[k][4], v[k][5]);
+        unpack2<T>(w.w, v[k][6], v[k][7]);
+      } else {
+        const float4 a = reinterpret_cast<const float4 *>(src)[0];
+        const float4 c = reinterpret_cast<const float4 *>(src)[1];
+        v[k][0] = a.x; v[k][1] = a.y; v[k][2] = a.z; v[k][3] = a.w;
+        v[k][4] = c.x; v[k][5] = c.y; v[k][6] = c.z; v[k][7] = c.w;
+      }
     }
-    bcf[tt * kP + pr] = make_float4(v[0], v[1], v[2], v[3]);
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      bcf[(seg * 8 + i) * kP + pr] = make_float4(v[0][i], v[1][i], v[2][i], v[3][i]);
   }
 }
 
@@ -234,9 +229,19 @@ __global__ void __launch_bounds__(kWarps * 32, 4) m1_bwd_kernel(const M1Params p
   const T *Cg = static_cast<const T *>(p.Cm) + (b * p.G + g) * N * L;
   const int64_t n_chunks = (L + kS - 1) / kS;
   const int64_t nb = (L + kBlk - 1) / kBlk;
-  const bool vec_sav = (N % 4 == 0) && ((reinterpret_cast<uintptr_t>(p.saved_in) & 15) == 0);
-
   const int n0 = 2 * pr, n1 = 2 * pr + 1;
+  // this thread's pair of the saved states, one window ahead (windows run
+  // backwards: chunk kb * kWin + w)
+  const float *const sav_row = p.saved_in + (b * D + c) * n_chunks * N;
+  auto load_saved = [&](int64_t chunk) {
+    float2 v = make_float2(0.f, 0.f);
+    if (active && chunk >= 0 && chunk < n_chunks) {
+      if (n0 < N) v.x = sav_row[chunk * N + n0];
+      if (n1 < N) v.y = sav_row[chunk * N + n1];
+    }
+    return v;
+  };
+
   float2 Ap = make_float2(0.f, 0.f);
   if (active) {
     if (n0 < N) Ap.x = p.A[c * N + n0];
@@ -251,26 +256,28 @@ __global__ void __launch_bounds__(kWarps * 32, 4) m1_bwd_kernel(const M1Params p
 
   unsigned char *const stage0 = smem + S::stage;
   float4 *const bcf0 = reinterpret_cast<float4 *>(smem + S::bcf);
+  const T **const rows = reinterpret_cast<const T **>(smem + S::rows);
 
-  // ---- prologue: the last block's inputs (and the one before, in flight) ----
-  issue_stage<T, kN>(p, stage0 + ((nb - 1) & 1) * S::kStageBytes, b, c_first, c_end, Bg, Cg,
-                     nb - 1, n_chunks, vec_sav, tid);
+  // ---- prologue: the row table; the last block's inputs (and the one
+  // before, in flight); the first window's saved state ------------------------
+  fill_rows<T, kN>(p, rows, b, c_first, c_end, Bg, Cg, tid);
+  __syncthreads();
+  issue_stage<T, kN>(p, stage0 + ((nb - 1) & 1) * S::kStageBytes, rows, nb - 1, tid);
   if (nb >= 2) {
-    issue_stage<T, kN>(p, stage0 + ((nb - 2) & 1) * S::kStageBytes, b, c_first, c_end, Bg, Cg,
-                       nb - 2, n_chunks, vec_sav, tid);
+    issue_stage<T, kN>(p, stage0 + ((nb - 2) & 1) * S::kStageBytes, rows, nb - 2, tid);
     cp_async_wait<1>();
   } else {
     cp_async_wait<0>();
   }
+  float2 sv_next = load_saved((nb - 1) * kWin + kWin - 1);
   __syncthreads();
   convert_bc<T, kN>(stage0 + ((nb - 1) & 1) * S::kStageBytes, bcf0 + ((nb - 1) & 1) * kBlk * kP,
-                    N, L, nb - 1, tid);
+                    tid);
   __syncthreads();
 
   for (int64_t kb = nb - 1; kb >= 0; --kb) {
     const unsigned char *const st = stage0 + (kb & 1) * S::kStageBytes;
     const float4 *const bcf = bcf0 + (kb & 1) * kBlk * kP;
-    const float *const sav = reinterpret_cast<const float *>(st + S::kTokBytes + S::kBCBytes);
 
     for (int w = kWin - 1; w >= 0; --w) {
       const int tw = w * kS;  // the window's first step within the block
@@ -305,11 +312,8 @@ __global__ void __launch_bounds__(kWarps * 32, 4) m1_bwd_kernel(const M1Params p
       __syncwarp();
 
       // ---- forward over the window from the saved state ---------------------
-      float2 h = make_float2(0.f, 0.f);
-      if (active && kb * kWin + w < n_chunks) {
-        const float2 sv = *reinterpret_cast<const float2 *>(sav + (chl * kWin + w) * kN + n0);
-        h = make_float2(n0 < N ? sv.x : 0.f, n1 < N ? sv.y : 0.f);
-      }
+      float2 h = sv_next;
+      sv_next = load_saved(kb * kWin + w - 1);  // the next window walked
       float2 a[kS], hp[kS];
       float yv[kS];
 #pragma unroll
@@ -396,10 +400,8 @@ __global__ void __launch_bounds__(kWarps * 32, 4) m1_bwd_kernel(const M1Params p
     }
     if (kb >= 1)
       convert_bc<T, kN>(stage0 + ((kb - 1) & 1) * S::kStageBytes, bcf0 + ((kb - 1) & 1) * kBlk * kP,
-                        N, L, kb - 1, tid);
-    if (kb >= 2)
-      issue_stage<T, kN>(p, stage0 + (kb & 1) * S::kStageBytes, b, c_first, c_end, Bg, Cg, kb - 2,
-                         n_chunks, vec_sav, tid);
+                        tid);
+    if (kb >= 2) issue_stage<T, kN>(p, stage0 + (kb & 1) * S::kStageBytes, rows, kb - 2, tid);
     // peers are done reading (the values read are consumed before the arrive);
     // the new B/C table is visible CTA-wide
     __syncthreads();
