@@ -83,9 +83,12 @@ struct BwdSmem {
   static constexpr int tile = tokg + kWarps * kChW * kS * 8;        // [kWarps][kChW][kS][kP+1] float4
   static constexpr int rbc = tile + kWarps * kChW * kS * kTileRow * 16;  // [kCh][kS][kP] float4
   static constexpr int kAccRow = kBlk + 1;                          // floats per (tensor, n) row
-  static constexpr int acc = rbc + kCh * kS * kP * 16;              // [2][kN][kBlk+1] f32
+  // the block's dB/dC sums over the CTA's channels, [2][kN][kBlk+1] f32, one
+  // buffer per block parity (the cluster reads one while the next fills)
+  static constexpr int kAccFloats = 2 * kN * kAccRow;
+  static constexpr int acc = rbc + kCh * kS * kP * 16;              // [2 parities]
   // global address of every staged row at t = 0 (0: absent row, zero-filled)
-  static constexpr int rows = (acc + 2 * kN * kAccRow * 4 + 7) / 8 * 8;  // [kRows] pointers
+  static constexpr int rows = (acc + 2 * kAccFloats * 4 + 7) / 8 * 8;  // [kRows] pointers
   static constexpr int total = rows + kRows * 8;
   static_assert(kStageBytes % 16 == 0 && kTokBytes % 16 == 0 && kBCBytes % 16 == 0,
                 "stage regions must stay 16-byte aligned");
@@ -199,7 +202,7 @@ __global__ void __launch_bounds__(kWarps * 32, 4) m1_bwd_kernel(const M1Params p
   extern __shared__ float4 smem4[];
   unsigned char *smem = reinterpret_cast<unsigned char *>(smem4);
   float4 *const sRbc = reinterpret_cast<float4 *>(smem + S::rbc);
-  float *const acc = reinterpret_cast<float *>(smem + S::acc);
+  float *const acc0 = reinterpret_cast<float *>(smem + S::acc);
   cg::cluster_group cluster = cg::this_cluster();
   const unsigned rank = cluster.block_rank();
 
@@ -278,6 +281,7 @@ __global__ void __launch_bounds__(kWarps * 32, 4) m1_bwd_kernel(const M1Params p
   for (int64_t kb = nb - 1; kb >= 0; --kb) {
     const unsigned char *const st = stage0 + (kb & 1) * S::kStageBytes;
     const float4 *const bcf = bcf0 + (kb & 1) * kBlk * kP;
+    float *const acc = acc0 + (kb & 1) * S::kAccFloats;
 
     for (int w = kWin - 1; w >= 0; --w) {
       const int tw = w * kS;  // the window's first step within the block
@@ -369,45 +373,56 @@ __global__ void __launch_bounds__(kWarps * 32, 4) m1_bwd_kernel(const M1Params p
       __syncthreads();  // every channel's dB/dC entries of the window are in place
 
       // ---- dB, dC of the window's steps: the CTA's channels in channel order --
-      const float2 *const r2 = reinterpret_cast<const float2 *>(sRbc);
-      for (int it = tid; it < kS * kP * 2; it += kThreads) {
-        const int half = it & 1, qq = (it >> 1) % kP, t = (it >> 1) / kP;
-        float2 s = r2[(t * kP + qq) * 2 + half];
+      for (int it = tid; it < kS * kP; it += kThreads) {
+        const int qq = it % kP, t = it / kP;
+        const float4 v0 = sRbc[t * kP + qq];
+        float2 sb = make_float2(v0.x, v0.y), sc = make_float2(v0.z, v0.w);
 #pragma unroll
-        for (int cl = 1; cl < kCh; ++cl) s = add2(s, r2[((cl * kS + t) * kP + qq) * 2 + half]);
-        float *row = acc + (half * kN + 2 * qq) * S::kAccRow + tw + t;
-        row[0] = s.x;
-        row[S::kAccRow] = s.y;
+        for (int cl = 1; cl < kCh; ++cl) {
+          const float4 v = sRbc[(cl * kS + t) * kP + qq];
+          sb = add2(sb, make_float2(v.x, v.y));
+          sc = add2(sc, make_float2(v.z, v.w));
+        }
+        float *rb = acc + 2 * qq * S::kAccRow + tw + t;
+        float *rc = acc + (kN + 2 * qq) * S::kAccRow + tw + t;
+        rb[0] = sb.x;
+        rb[S::kAccRow] = sb.y;
+        rc[0] = sc.x;
+        rc[S::kAccRow] = sc.y;
       }
       __syncthreads();  // the entries are free for the next window
     }
 
-    // ---- end of block: the cluster's sums in rank order, next block's inputs --
+    // ---- end of block: next block's inputs, the cluster's sums in rank order --
     cp_async_wait<0>();  // block kb - 1's inputs (issued one block ago) have landed
-    cluster.sync();      // accumulators complete; block kb's buffers free
-    {
-      constexpr int E = 2 * kN * kBlk;
-      constexpr int per = E / kCS;
-      for (int e = (int)rank * per + tid; e < ((int)rank + 1) * per; e += kThreads) {
-        const int te = e / (kN * kBlk), n = (e / kBlk) % kN, tt = e % kBlk;
-        const int off = (te * kN + n) * S::kAccRow + tt;
-        float s = *(cluster.map_shared_rank(acc, 0) + off);
-#pragma unroll
-        for (int qq = 1; qq < kCS; ++qq) s += *(cluster.map_shared_rank(acc, qq) + off);
-        const int64_t t = kb * kBlk + tt;
-        if (n < N && t < L) p.ws_bc[(((part * Bsz + b) * 2 + te) * N + n) * L + t] = s;
-      }
-    }
+    cluster.sync();      // every CTA's accumulators of block kb are complete; block kb's buffers free
     if (kb >= 1)
       convert_bc<T, kN>(stage0 + ((kb - 1) & 1) * S::kStageBytes, bcf0 + ((kb - 1) & 1) * kBlk * kP,
                         tid);
     if (kb >= 2) issue_stage<T, kN>(p, stage0 + (kb & 1) * S::kStageBytes, rows, kb - 2, tid);
-    // peers are done reading (the values read are consumed before the arrive);
-    // the new B/C table is visible CTA-wide
-    __syncthreads();
-    asm volatile("barrier.cluster.arrive.relaxed.aligned;\n" ::: "memory");
-    asm volatile("barrier.cluster.wait.aligned;\n" ::: "memory");
+    __syncthreads();  // the new B/C table is visible CTA-wide
+    // The peers' accumulators of block kb stay intact until their block kb - 2,
+    // which starts after the next cluster barrier: this CTA reaches that
+    // barrier only after these reads.
+    {
+      constexpr int E = 2 * kN * kBlk;
+      constexpr int per = E / kCS;
+      const float *racc[kCS];
+#pragma unroll
+      for (int qq = 0; qq < kCS; ++qq) racc[qq] = cluster.map_shared_rank(acc, qq);
+      for (int e = (int)rank * per + tid; e < ((int)rank + 1) * per; e += kThreads) {
+        const int te = e / (kN * kBlk), n = (e / kBlk) % kN, tt = e % kBlk;
+        const int off = (te * kN + n) * S::kAccRow + tt;
+        float s = racc[0][off];
+#pragma unroll
+        for (int qq = 1; qq < kCS; ++qq) s += racc[qq][off];
+        const int64_t t = kb * kBlk + tt;
+        if (n < N && t < L) p.ws_bc[(((part * Bsz + b) * 2 + te) * N + n) * L + t] = s;
+      }
+    }
   }
+  // no CTA leaves while a peer may still read its accumulators
+  cluster.sync();
 
   // per-(b, c) partials: dA (per thread), dD and dbias (the lanes of a channel
   // added by a fixed butterfly), dh0 = the carry left after step 0
