@@ -53,53 +53,59 @@ struct FwdSmem {
 template <typename T, int kN>
 struct FwdRaw {
   static constexpr int kCh = Layout<kN, kWarps>::kCh;
+  static constexpr int kRows = 3 * kCh + 2 * kN;  // staged rows: u, delta, z, then B and C
   static constexpr int tok = 0;
   static constexpr int bc = 3 * kCh * kTF * (int)sizeof(T);
-  static constexpr int bytes = bc + 2 * kN * kTF * (int)sizeof(T);
+  // global address of every staged row at t = 0 (0: absent row, zero-filled)
+  static constexpr int rows = (bc + 2 * kN * kTF * (int)sizeof(T) + 7) / 8 * 8;
+  static constexpr int bytes = rows + kRows * 8;
 };
 
-// Issue the copies of the chunk starting at tc into the raw buffer: 16-byte
-// cp.async pieces (zero-filled past the end of a row) when rows are 16-byte
-// aligned, element copies otherwise.  Entries past L, past the last channel
-// or past d_state are never read as data.
+// The row table, once per CTA: token rows (tensor k of u, delta, z; channel
+// cl) at k * kCh + cl, then the B and C rows (state n) at 3 kCh + k * kN + n.
 template <typename T, int kN>
-__device__ __forceinline__ void fwd_issue_raw(const M1Params &p, unsigned char *raw, int64_t b,
+__device__ __forceinline__ void fwd_fill_rows(const M1Params &p, const T **rows, int64_t b,
                                               int64_t c_first, int64_t c_end, const T *Bg,
-                                              const T *Cg, int64_t tc, int tid) {
+                                              const T *Cg, int tid) {
   using R = FwdRaw<T, kN>;
   constexpr int kCh = R::kCh;
-  constexpr int kThreads = kWarps * 32;
+  for (int r = tid; r < R::kRows; r += kWarps * 32) {
+    const T *row = nullptr;
+    if (r < 3 * kCh) {
+      const int k = r / kCh, cl = r % kCh;
+      const void *src = k == 0 ? p.u : (k == 1 ? p.delta : p.z);
+      const int64_t c = c_first + cl;
+      if (src != nullptr && c < c_end) row = static_cast<const T *>(src) + (b * p.D + c) * p.L;
+    } else {
+      const int k = (r - 3 * kCh) / kN, n = (r - 3 * kCh) % kN;
+      if (n < p.N) row = (k == 0 ? Bg : Cg) + n * p.L;
+    }
+    rows[r] = row;
+  }
+}
+
+// Issue the copies of the chunk starting at tc into the raw buffer: 16-byte
+// pieces of the rows in the row table, by cp.async (zero-filled past the end
+// of a row) when rows are 16-byte aligned, element copies otherwise.  Absent
+// rows are zeros.
+template <typename T, int kN>
+__device__ __forceinline__ void fwd_issue_raw(const M1Params &p, unsigned char *raw,
+                                              const T *const *rows, int64_t tc, int tid) {
+  using R = FwdRaw<T, kN>;
   constexpr int E = 16 / (int)sizeof(T);
   constexpr int kPieces = kTF / E;
-  const int64_t L = p.L, N = p.N;
-  for (int u = tid; u < 3 * kCh * kPieces + 2 * kN * kPieces; u += kThreads) {
-    const T *row;
-    bool ok;
-    int r, j;
-    T *dst;
-    if (u < 3 * kCh * kPieces) {
-      j = u % kPieces;
-      r = u / kPieces;
-      const int cl = r % kCh, k = r / kCh;
-      const int64_t c = c_first + cl;
-      const void *src = k == 0 ? p.u : (k == 1 ? p.delta : p.z);
-      ok = src != nullptr && c < c_end;
-      row = ok ? static_cast<const T *>(src) + (b * p.D + c) * L : static_cast<const T *>(p.u);
-      dst = reinterpret_cast<T *>(raw + R::tok) + r * kTF + j * E;
-    } else {
-      const int v = u - 3 * kCh * kPieces;
-      j = v % kPieces;
-      r = v / kPieces;
-      const int n = r % kN, k = r / kN;
-      ok = n < N;
-      row = ok ? (k == 0 ? Bg : Cg) + n * L : Bg;
-      dst = reinterpret_cast<T *>(raw + R::bc) + r * kTF + j * E;
-    }
+  static_assert((kPieces & (kPieces - 1)) == 0, "pieces per row: a power of two");
+  const int64_t L = p.L;
+  const T *const fallback = static_cast<const T *>(p.Bm);  // a valid address for empty copies
+  for (int u = tid; u < R::kRows * kPieces; u += kWarps * 32) {
+    const int j = u & (kPieces - 1), r = u / kPieces;
+    const T *row = rows[r];
     const int64_t t = tc + j * E;
     const int64_t left = L - t;
-    const int valid = !ok || left <= 0 ? 0 : (left >= E ? E : (int)left);
+    const int valid = row == nullptr || left <= 0 ? 0 : (left >= E ? E : (int)left);
+    T *dst = reinterpret_cast<T *>(raw) + r * kTF + j * E;
     if (p.vec) {
-      cp_async16(dst, valid > 0 ? row + t : row, valid * (int)sizeof(T));
+      cp_async16(dst, valid > 0 ? row + t : fallback, valid * (int)sizeof(T));
     } else {
 #pragma unroll
       for (int i = 0; i < E; ++i) dst[i] = i < valid ? row[t + i] : from_f32<T>(0.f);
@@ -182,7 +188,10 @@ __global__ void __launch_bounds__(kWarps * 32, 6) m1_fwd_kernel(const M1Params p
   const float tDc = (tact && p.Dp) ? p.Dp[tcc] : 0.f;
   const float tbias = (tact && p.bias) ? p.bias[tcc] : 0.f;
 
-  fwd_issue_raw<T, kN>(p, raw, b, c_first, c_end, Bg, Cg, 0, tid);
+  const T **const rows = reinterpret_cast<const T **>(raw + R::rows);
+  fwd_fill_rows<T, kN>(p, rows, b, c_first, c_end, Bg, Cg, tid);
+  __syncthreads();
+  fwd_issue_raw<T, kN>(p, raw, rows, 0, tid);
   for (int64_t ch = 0; ch <= n_chunks; ++ch) {
     const int64_t tc = ch * kTF;
     cp_async_wait<0>();
@@ -213,23 +222,37 @@ __global__ void __launch_bounds__(kWarps * 32, 6) m1_fwd_kernel(const M1Params p
         sTok[(tseg * kRun + i) * kCh + tcl] = tk;
       }
     }
-    // ---- B, C pairs in f32 ------------------------------------------------------
+    // ---- B, C pairs in f32 (the raw rows hold zeros past d_state and past L):
+    // a unit is a pair and 8 consecutive steps, four row pieces in, eight
+    // float4 out
     {
       const T *rb = reinterpret_cast<const T *>(raw + R::bc);
-      for (int u = tid; u < kTF * kP; u += kThreads) {
-        const int t = u % kTF, q = u / kTF;
-        const bool in = tc + t < L;
-        float e[4];
+      for (int u = tid; u < kP * (kTF / 8); u += kThreads) {
+        const int q = u % kP, seg = u / kP;
+        float e[4][8];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const int n = 2 * q + (k & 1);
-          e[k] = (in && n < N) ? to_f32(rb[((k >> 1) * kN + n) * kTF + t]) : 0.f;
+          const T *src = rb + ((k >> 1) * kN + 2 * q + (k & 1)) * kTF + seg * 8;
+          if constexpr (sizeof(T) == 2) {
+            const uint4 w = *reinterpret_cast<const uint4 *>(src);
+            unpack2<T>(w.x, e[k][0], e[k][1]);
+            unpack2<T>(w.y, e[k][2], e[k][3]);
+            unpack2<T>(w.z, e[k][4], e[k][5]);
+            unpack2<T>(w.w, e[k][6], e[k][7]);
+          } else {
+            const float4 a = reinterpret_cast<const float4 *>(src)[0];
+            const float4 c = reinterpret_cast<const float4 *>(src)[1];
+            e[k][0] = a.x; e[k][1] = a.y; e[k][2] = a.z; e[k][3] = a.w;
+            e[k][4] = c.x; e[k][5] = c.y; e[k][6] = c.z; e[k][7] = c.w;
+          }
         }
-        sBC[t * kP + q] = make_float4(e[0], e[1], e[2], e[3]);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          sBC[(seg * 8 + i) * kP + q] = make_float4(e[0][i], e[1][i], e[2][i], e[3][i]);
       }
     }
     __syncthreads();  // tables ready; the raw buffer and the output tile are free
-    if (ch + 1 < n_chunks) fwd_issue_raw<T, kN>(p, raw, b, c_first, c_end, Bg, Cg, tc + kTF, tid);
+    if (ch + 1 < n_chunks) fwd_issue_raw<T, kN>(p, raw, rows, tc + kTF, tid);
 
     // ---- the recurrence over the chunk -------------------------------------
 #pragma unroll 1
