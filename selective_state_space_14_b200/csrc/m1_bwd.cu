@@ -77,10 +77,13 @@ struct BwdSmem {
   static constexpr int bcf = stage + 2 * kStageBytes;               // [2][kBlk][kP] float4
   // per (warp channel, step): (d, d, d x, d x) and (g, g), pairs ready for
   // the packed arithmetic of the state pairs
-  static constexpr int tok = bcf + 2 * kBlk * kP * 16;              // [kWarps][kChW][kS] float4
-  static constexpr int tokg = tok + kWarps * kChW * kS * 16;        // [kWarps][kChW][kS] float2
+  // (per channel kS + 1 slots: the channels of a warp, read at the same step,
+  // fall on different banks)
+  static constexpr int kTokRow = kS + 1;
+  static constexpr int tok = bcf + 2 * kBlk * kP * 16;              // [kWarps][kChW][kTokRow] float4
+  static constexpr int tokg = tok + kWarps * kChW * kTokRow * 16;   // [kWarps][kChW][kTokRow] float2
   static constexpr int kTileRow = kP + 1;                           // float4 per (chw, step) row
-  static constexpr int tile = tokg + kWarps * kChW * kS * 8;        // [kWarps][kChW][kS][kP+1] float4
+  static constexpr int tile = (tokg + kWarps * kChW * kTokRow * 8 + 15) / 16 * 16;  // [kWarps][kChW][kS][kP+1] float4
   static constexpr int rbc = tile + kWarps * kChW * kS * kTileRow * 16;  // [kCh][kS][kP] float4
   static constexpr int kAccRow = kBlk + 1;                          // floats per (tensor, n) row
   // the block's dB/dC sums over the CTA's channels, [2][kN][kBlk+1] f32, one
@@ -211,8 +214,8 @@ __global__ void __launch_bounds__(kWarps * 32, 4) m1_bwd_kernel(const M1Params p
   const int pr = lane % kP;
   const int chw = lane / kP;
   const int chl = warp * kChW + chw;
-  float4 *const sTok = reinterpret_cast<float4 *>(smem + S::tok) + (warp * kChW + chw) * kS;
-  float2 *const sTokG = reinterpret_cast<float2 *>(smem + S::tokg) + (warp * kChW + chw) * kS;
+  float4 *const sTok = reinterpret_cast<float4 *>(smem + S::tok) + (warp * kChW + chw) * S::kTokRow;
+  float2 *const sTokG = reinterpret_cast<float2 *>(smem + S::tokg) + (warp * kChW + chw) * S::kTokRow;
   float4 *const sTile =
       reinterpret_cast<float4 *>(smem + S::tile) + (warp * kChW + chw) * kS * S::kTileRow;
   const int64_t D = p.D, L = p.L, N = p.N, Bsz = p.B;

@@ -49,13 +49,17 @@ struct FwdSmem {
   static constexpr int total_floats = raw;
 };
 
-// raw inputs of one chunk, bytes: u, delta, z [3][kCh][kTF] T; B, C [2][kN][kTF] T
+// raw inputs of one chunk, bytes: u, delta, z [3][kCh][kTokRow] T; B, C [2][kN][kTF] T;
+// then the row table
 template <typename T, int kN>
 struct FwdRaw {
   static constexpr int kCh = Layout<kN, kWarps>::kCh;
   static constexpr int kRows = 3 * kCh + 2 * kN;  // staged rows: u, delta, z, then B and C
+  // token rows padded by 16 bytes: the threads that convert one step of
+  // consecutive channels read from different banks
+  static constexpr int kTokRow = kTF + 16 / (int)sizeof(T);
   static constexpr int tok = 0;
-  static constexpr int bc = 3 * kCh * kTF * (int)sizeof(T);
+  static constexpr int bc = 3 * kCh * kTokRow * (int)sizeof(T);
   // global address of every staged row at t = 0 (0: absent row, zero-filled)
   static constexpr int rows = (bc + 2 * kN * kTF * (int)sizeof(T) + 7) / 8 * 8;
   static constexpr int bytes = rows + kRows * 8;
@@ -103,7 +107,8 @@ __device__ __forceinline__ void fwd_issue_raw(const M1Params &p, unsigned char *
     const int64_t t = tc + j * E;
     const int64_t left = L - t;
     const int valid = row == nullptr || left <= 0 ? 0 : (left >= E ? E : (int)left);
-    T *dst = reinterpret_cast<T *>(raw) + r * kTF + j * E;
+    T *dst = r < 3 * R::kCh ? reinterpret_cast<T *>(raw) + r * R::kTokRow + j * E
+                            : reinterpret_cast<T *>(raw + R::bc) + (r - 3 * R::kCh) * kTF + j * E;
     if (p.vec) {
       cp_async16(dst, valid > 0 ? row + t : fallback, valid * (int)sizeof(T));
     } else {
@@ -206,10 +211,10 @@ __global__ void __launch_bounds__(kWarps * 32, 6) m1_fwd_kernel(const M1Params p
       float x[kRun], v[kRun], zv[kRun];
 #pragma unroll
       for (int i = 0; i < kRun; ++i) {
-        const int o = tcl * kTF + tseg * kRun + i;
+        const int o = tcl * R::kTokRow + tseg * kRun + i;
         x[i] = to_f32(ru[o]);
-        v[i] = to_f32(ru[kCh * kTF + o]);
-        zv[i] = p.z ? to_f32(ru[2 * kCh * kTF + o]) : 0.f;
+        v[i] = to_f32(ru[kCh * R::kTokRow + o]);
+        zv[i] = p.z ? to_f32(ru[2 * kCh * R::kTokRow + o]) : 0.f;
       }
 #pragma unroll
       for (int i = 0; i < kRun; ++i) {
