@@ -49,19 +49,19 @@ struct FwdSmem {
   static constexpr int total_floats = raw;
 };
 
-// raw inputs of one chunk, bytes: u, delta, z [3][kCh][kTokRow] T; B, C [2][kN][kTF] T;
+// raw inputs of one chunk, bytes: u, delta, z [3][kCh][kTokRow] T; B, C [2][kN][kTokRow] T;
 // then the row table
 template <typename T, int kN>
 struct FwdRaw {
   static constexpr int kCh = Layout<kN, kWarps>::kCh;
   static constexpr int kRows = 3 * kCh + 2 * kN;  // staged rows: u, delta, z, then B and C
-  // token rows padded by 16 bytes: the threads that convert one step of
-  // consecutive channels read from different banks
+  // rows padded by 16 bytes: the threads that convert one step of
+  // consecutive channels (or state pairs) read from different banks
   static constexpr int kTokRow = kTF + 16 / (int)sizeof(T);
   static constexpr int tok = 0;
   static constexpr int bc = 3 * kCh * kTokRow * (int)sizeof(T);
   // global address of every staged row at t = 0 (0: absent row, zero-filled)
-  static constexpr int rows = (bc + 2 * kN * kTF * (int)sizeof(T) + 7) / 8 * 8;
+  static constexpr int rows = (bc + 2 * kN * kTokRow * (int)sizeof(T) + 7) / 8 * 8;
   static constexpr int bytes = rows + kRows * 8;
 };
 
@@ -108,7 +108,7 @@ __device__ __forceinline__ void fwd_issue_raw(const M1Params &p, unsigned char *
     const int64_t left = L - t;
     const int valid = row == nullptr || left <= 0 ? 0 : (left >= E ? E : (int)left);
     T *dst = r < 3 * R::kCh ? reinterpret_cast<T *>(raw) + r * R::kTokRow + j * E
-                            : reinterpret_cast<T *>(raw + R::bc) + (r - 3 * R::kCh) * kTF + j * E;
+                            : reinterpret_cast<T *>(raw + R::bc) + (r - 3 * R::kCh) * R::kTokRow + j * E;
     if (p.vec) {
       cp_async16(dst, valid > 0 ? row + t : fallback, valid * (int)sizeof(T));
     } else {
@@ -129,9 +129,9 @@ __device__ __forceinline__ void store_chunk(T *out_base, const float *sout, int6
     const int seg = u % (kTF / 8);
     const int64_t c = c_first + chl;
     if (c >= c_end) continue;
-    float v[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = sout[chl * kOut + seg * 8 + i];
+    const float4 a = *reinterpret_cast<const float4 *>(sout + chl * kOut + seg * 8);
+    const float4 e = *reinterpret_cast<const float4 *>(sout + chl * kOut + seg * 8 + 4);
+    const float v[8] = {a.x, a.y, a.z, a.w, e.x, e.y, e.z, e.w};
     store_run<8>(out_base + (b * D + c) * L, tc + seg * 8, L, vec, v);
   }
 }
@@ -237,7 +237,7 @@ __global__ void __launch_bounds__(kWarps * 32, 6) m1_fwd_kernel(const M1Params p
         float e[4][8];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const T *src = rb + ((k >> 1) * kN + 2 * q + (k & 1)) * kTF + seg * 8;
+          const T *src = rb + ((k >> 1) * kN + 2 * q + (k & 1)) * R::kTokRow + seg * 8;
           if constexpr (sizeof(T) == 2) {
             const uint4 w = *reinterpret_cast<const uint4 *>(src);
             unpack2<T>(w.x, e[k][0], e[k][1]);
