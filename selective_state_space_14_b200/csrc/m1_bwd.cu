@@ -67,9 +67,12 @@ struct BwdSmem {
   static constexpr int kCh = Lay::kCh;
   static constexpr int kChW = Lay::kChPerWarp;
   // raw stage (one buffer; two are kept): tokens [4][kCh][kBlk] T in the
-  // order u, delta, z, dout; bc [2][kN][kBlk] T
+  // order u, delta, z, dout; bc [2][kN][kBCRow] T
   static constexpr int kTokBytes = 4 * kCh * kBlk * (int)sizeof(T);
-  static constexpr int kBCBytes = 2 * kN * kBlk * (int)sizeof(T);
+  // B and C rows padded by 16 bytes: the eight rows a conversion reads at
+  // once fall on different banks
+  static constexpr int kBCRow = kBlk + 16 / (int)sizeof(T);
+  static constexpr int kBCBytes = 2 * kN * kBCRow * (int)sizeof(T);
   static constexpr int kStageBytes = kTokBytes + kBCBytes;
   static constexpr int kRows = 4 * kCh + 2 * kN;  // staged rows: tokens, then B and C
   // byte offsets
@@ -149,7 +152,9 @@ __device__ __forceinline__ void issue_stage(const M1Params &p, unsigned char *st
     const int64_t t = t0 + j * E;
     const int64_t left = L - t;
     const int valid = row == nullptr || left <= 0 ? 0 : (left >= E ? E : (int)left);
-    T *dst = reinterpret_cast<T *>(st) + r * kBlk + j * E;
+    T *dst = r < 4 * S::kCh
+                 ? reinterpret_cast<T *>(st) + r * kBlk + j * E
+                 : reinterpret_cast<T *>(st + S::kTokBytes) + (r - 4 * S::kCh) * S::kBCRow + j * E;
     if (p.vec) {
       cp_async16(dst, valid > 0 ? row + t : fallback, valid * (int)sizeof(T));
     } else {
@@ -174,7 +179,7 @@ __device__ __forceinline__ void convert_bc(const unsigned char *st, float4 *bcf,
     float v[4][8];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      const T *src = raw + ((k >> 1) * kN + 2 * pr + (k & 1)) * kBlk + seg * 8;
+      const T *src = raw + ((k >> 1) * kN + 2 * pr + (k & 1)) * S::kBCRow + seg * 8;
       if constexpr (sizeof(T) == 2) {
         const uint4 w = *reinterpret_cast<const uint4 *>(src);
         unpack2<T>(w.x, v[k][0], v[k][1]);
