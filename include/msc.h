@@ -99,10 +99,13 @@ const char *msc_version(void);
  * starting from h = h0[b,c,:] (or 0).  final_state receives h after the last
  * step.  saved_states receives h at the start of every block of
  * MSC_M1_SAVE_INTERVAL steps (the first is h0); the backward pass needs it.
- * N may be 1..64; L >= 1.
+ * N may be 1..256 ("state dimensions up to 256", mamba-rs README,
+ * "Features"); L >= 1.  Above 64 states the scan runs in slabs of 64 states
+ * and the forward needs a workspace of msc_selective_scan_fwd_workspace_bytes()
+ * bytes (0 up to 64 states) for the sums over the earlier slabs.
  */
 #define MSC_M1_SAVE_INTERVAL 8
-#define MSC_M1_MAX_DSTATE 64
+#define MSC_M1_MAX_DSTATE 256
 
 typedef struct {
   uint32_t struct_size;
@@ -119,7 +122,13 @@ typedef struct {
   void *out;
   float *final_state;      /* optional */
   float *saved_states;     /* optional; required if the backward pass follows */
+  void *workspace;         /* required when dstate > 64, else ignored (may be NULL) */
+  size_t workspace_bytes;
 } msc_ss_fwd_args;
+
+/* Bytes of the forward's workspace for these sizes (0 when dstate <= 64). */
+size_t msc_selective_scan_fwd_workspace_bytes(int64_t batch, int64_t dim, int64_t dstate,
+                                              int64_t seqlen);
 
 /* Bytes of the saved_states array for these sizes. */
 size_t msc_selective_scan_saved_states_bytes(int64_t batch, int64_t dim, int64_t dstate,

@@ -9,6 +9,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdarg>
+#include <cstddef>
 #include <cstdio>
 #include <cstring>
 
@@ -113,12 +114,23 @@ size_t msc_selective_scan_saved_states_bytes(int64_t batch, int64_t dim, int64_t
   return sizeof(float) * (size_t)(batch * dim * n_save * dstate);
 }
 
+size_t msc_selective_scan_fwd_workspace_bytes(int64_t batch, int64_t dim, int64_t dstate,
+                                              int64_t seqlen) {
+  if (batch <= 0 || dim <= 0 || dstate <= msc::kM1Slab || seqlen <= 0) return 0;
+  return sizeof(float) * (size_t)(batch * dim * seqlen);  // the sums over the earlier slabs
+}
+
 msc_status msc_selective_scan_fwd(const msc_ss_fwd_args *a, msc_stream_t stream) {
   const char *fn = "msc_selective_scan_fwd";
   if (!a) return fail(MSC_ERR_INVALID_ARG, "%s: args is NULL", fn);
-  if (a->struct_size < sizeof(msc_ss_fwd_args))
-    return fail(MSC_ERR_INVALID_ARG, "%s: struct_size %u < sizeof(msc_ss_fwd_args) %zu", fn,
-                a->struct_size, sizeof(msc_ss_fwd_args));
+  // callers built before the workspace fields pass a shorter struct: no workspace
+  constexpr size_t kNoWorkspaceSize = offsetof(msc_ss_fwd_args, workspace);
+  if (a->struct_size < kNoWorkspaceSize)
+    return fail(MSC_ERR_INVALID_ARG, "%s: struct_size %u < %zu", fn, a->struct_size,
+                kNoWorkspaceSize);
+  const bool has_ws_fields = a->struct_size >= sizeof(msc_ss_fwd_args);
+  void *const workspace = has_ws_fields ? a->workspace : nullptr;
+  const size_t workspace_bytes = has_ws_fields ? a->workspace_bytes : 0;
   msc_status st;
   if ((st = check_dtype(fn, a->io_dtype)) != MSC_OK) return st;
   if ((st = check_flag(fn, "delta_softplus", a->delta_softplus)) != MSC_OK) return st;
@@ -149,6 +161,11 @@ msc_status msc_selective_scan_fwd(const msc_ss_fwd_args *a, msc_stream_t stream)
   REQUIRE_PTR(fn, "out", a->out);
   OPTIONAL_PTR(fn, "z", a->z);
   OPTIONAL_PTR(fn, "saved_states", a->saved_states);
+  const size_t need = msc_selective_scan_fwd_workspace_bytes(B, D, N, L);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need))
+    return fail(MSC_ERR_WORKSPACE, "%s: dstate %lld needs a workspace of %zu bytes, %zu given",
+                fn, (long long)N, need, workspace ? workspace_bytes : (size_t)0);
+  OPTIONAL_PTR(fn, "workspace", workspace);
 
   msc::M1Params p = {};
   p.io = a->io_dtype;
@@ -158,6 +175,7 @@ msc_status msc_selective_scan_fwd(const msc_ss_fwd_args *a, msc_stream_t stream)
   p.u = a->u; p.delta = a->delta; p.Bm = a->Bm; p.Cm = a->Cm; p.z = a->z;
   p.A = a->A; p.Dp = a->D; p.bias = a->delta_bias; p.h0 = a->h0;
   p.out = a->out; p.final_state = a->final_state; p.saved = a->saved_states;
+  p.tok_part = need > 0 ? static_cast<float *>(workspace) : nullptr;
   return cuda_status(msc::launch_m1_fwd(p, s), fn);
 }
 
@@ -229,10 +247,12 @@ msc_status msc_selective_scan_bwd(const msc_ss_bwd_args *a, void *workspace,
   p.du = a->du; p.ddelta = a->ddelta; p.dz = a->z ? a->dz : nullptr;
   p.dA = a->dA; p.dB = a->dB; p.dC = a->dC; p.dD = a->dD; p.dbias = a->ddelta_bias;
   p.dh0 = a->dh0;
-  p.n_part = msc::m1_bwd_partials(D, N, G);
-  const size_t bc = ((sizeof(float) * (size_t)(p.n_part * B * 2 * N * L)) + 255) / 256 * 256;
-  p.ws_bc = static_cast<float *>(workspace);
-  p.ws_misc = reinterpret_cast<float *>(static_cast<char *>(workspace) + bc);
+  const msc::M1BwdWorkspace w = msc::m1_bwd_workspace(B, D, N, L, G);
+  char *const ws = static_cast<char *>(workspace);
+  p.n_part = w.n_part;
+  p.ws_bc = reinterpret_cast<float *>(ws + w.bc);
+  p.ws_misc = reinterpret_cast<float *>(ws + w.misc);
+  p.tok_part = N > msc::kM1Slab ? reinterpret_cast<float *>(ws + w.tok) : nullptr;
   return cuda_status(msc::launch_m1_bwd(p, s), fn);
 }
 

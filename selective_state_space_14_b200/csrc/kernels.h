@@ -24,12 +24,22 @@ struct M1Params {
   const void *dout;
   void *du, *ddelta, *dz;
   float *dA, *dB, *dC, *dD, *dbias, *dh0;
-  float *ws_bc;    // [n_part][B][2][N][L] partial sums of dB, dC
-  float *ws_misc;  // [B][D][N + 2]: per-(b, c) dA row, dD, dbias
+  float *ws_bc;    // [n_part][B][2][ldN][L] partial sums of dB, dC
+  float *ws_misc;  // [B][D][ldN + 2]: per-(b, c) dA row, dD, dbias
   int64_t n_part;  // dB/dC partials per batch row (one per cluster of CTAs)
+  // d_state above kM1Slab runs as slabs of at most kM1Slab states, one launch
+  // each: N is the slab's width, n0 its first state, ldN the full d_state
+  // (the row length of A, h0, the states and dA).  The per-token sums over
+  // the states (y, and in the backward also the dΔ and du sums) collect in
+  // tok_part across the slabs in slab order; the last slab finishes them.
+  int64_t n0, ldN;
+  int slab;         // kSlabWhole, kSlabFirst, kSlabMiddle or kSlabLast
+  float *tok_part;  // fwd: [B][D][L] (y); bwd: [3][B][D][L] (y, dΔ sum, Σ λ B)
 };
+constexpr int kM1Slab = 64;  // widest d_state one launch handles
+constexpr int kSlabWhole = 0, kSlabFirst = 1, kSlabMiddle = 2, kSlabLast = 3;
 
-constexpr int MSC_MAX_N = 64;             // largest Mamba-1 d_state
+constexpr int MSC_MAX_N = 256;            // largest Mamba-1 d_state (slabs of 64 above 64)
 constexpr int kM1SaveInterval = 8;        // saved-state spacing (time steps)
 constexpr int kM1BwdCluster = 8;          // CTAs per cluster in the backward
 constexpr int kM1BwdWarps = 3;            // warps per backward CTA
@@ -43,6 +53,11 @@ int64_t m1_bwd_partials(int64_t D, int64_t N, int64_t G);
 cudaError_t launch_m1_fwd(const M1Params &p, cudaStream_t s);
 cudaError_t launch_m1_bwd(const M1Params &p, cudaStream_t s);
 size_t m1_bwd_workspace_bytes(int64_t B, int64_t D, int64_t N, int64_t L, int64_t G);
+struct M1BwdWorkspace {
+  int64_t n_part;
+  size_t bc, misc, tok, bytes;  // byte offsets of the regions, total size
+};
+M1BwdWorkspace m1_bwd_workspace(int64_t B, int64_t D, int64_t N, int64_t L, int64_t G);
 
 // ------------------------------------------------------------ decode step --
 struct SUParams {

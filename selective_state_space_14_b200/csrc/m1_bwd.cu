@@ -224,6 +224,8 @@ __global__ void __launch_bounds__(kWarps * 32, 4) m1_bwd_kernel(const M1Params p
   float4 *const sTile =
       reinterpret_cast<float4 *>(smem + S::tile) + (warp * kChW + chw) * kS * S::kTileRow;
   const int64_t D = p.D, L = p.L, N = p.N, Bsz = p.B;
+  const int64_t ldN = p.ldN, ns = p.n0;  // row length of A and the states; this slab's first state
+  const bool finish = p.slab == kSlabWhole || p.slab == kSlabLast;  // this launch finishes the tokens
   const int64_t b = blockIdx.y;
   // a group's channels fill whole clusters; the CTAs past them own no channel
   const int64_t per_group = D / p.G;
@@ -236,31 +238,31 @@ __global__ void __launch_bounds__(kWarps * 32, 4) m1_bwd_kernel(const M1Params p
   const int64_t c = c_first + chl;
   const bool active = c < c_end;
   const int64_t part = blockIdx.x / kCS;  // dB/dC partial of this cluster
-  const T *Bg = static_cast<const T *>(p.Bm) + (b * p.G + g) * N * L;
-  const T *Cg = static_cast<const T *>(p.Cm) + (b * p.G + g) * N * L;
+  const T *Bg = static_cast<const T *>(p.Bm) + ((b * p.G + g) * ldN + ns) * L;
+  const T *Cg = static_cast<const T *>(p.Cm) + ((b * p.G + g) * ldN + ns) * L;
   const int64_t n_chunks = (L + kS - 1) / kS;
   const int64_t nb = (L + kBlk - 1) / kBlk;
   const int n0 = 2 * pr, n1 = 2 * pr + 1;
   // this thread's pair of the saved states, one window ahead (windows run
   // backwards: chunk kb * kWin + w)
-  const float *const sav_row = p.saved_in + (b * D + c) * n_chunks * N;
+  const float *const sav_row = p.saved_in + (b * D + c) * n_chunks * ldN + ns;
   auto load_saved = [&](int64_t chunk) {
     float2 v = make_float2(0.f, 0.f);
     if (active && chunk >= 0 && chunk < n_chunks) {
-      if (n0 < N) v.x = sav_row[chunk * N + n0];
-      if (n1 < N) v.y = sav_row[chunk * N + n1];
+      if (n0 < N) v.x = sav_row[chunk * ldN + n0];
+      if (n1 < N) v.y = sav_row[chunk * ldN + n1];
     }
     return v;
   };
 
   float2 Ap = make_float2(0.f, 0.f);
   if (active) {
-    if (n0 < N) Ap.x = p.A[c * N + n0];
-    if (n1 < N) Ap.y = p.A[c * N + n1];
+    if (n0 < N) Ap.x = p.A[c * ldN + ns + n0];
+    if (n1 < N) Ap.y = p.A[c * ldN + ns + n1];
   }
   const float2 A2 = mul2(Ap, splat2(kLog2e));
   const float bias_c = (active && p.bias) ? p.bias[c] : 0.f;
-  const float D_c = (active && p.Dp) ? p.Dp[c] : 0.f;
+  const float D_c = (active && p.Dp && finish) ? p.Dp[c] : 0.f;  // the D terms join once
   float2 mu = make_float2(0.f, 0.f);  // a_{t+1} lambda_{t+1}, handed backwards
   float2 dA = make_float2(0.f, 0.f);  // this (b, c)'s dA for the pair
   float dD_l = 0.f, dbias_l = 0.f;    // per lane (the tokens it finishes)
@@ -370,6 +372,23 @@ __global__ void __launch_bounds__(kWarps * 32, 4) m1_bwd_kernel(const M1Params p
         const int64_t t = t_win + pr;
         if (active && t < L) {
           const int64_t i = (b * D + c) * L + t;
+          if (p.slab != kSlabWhole) {  // the sums over the states cross the slabs
+            float *tp = p.tok_part + i;
+            const int64_t plane = Bsz * D * L;
+            if (p.slab != kSlabFirst) {
+              y = tp[0] + y;
+              dd = tp[plane] + dd;
+              sb = tp[2 * plane] + sb;
+            }
+            if (!finish) {
+              tp[0] = y;
+              tp[plane] = dd;
+              tp[2 * plane] = sb;
+            }
+          }
+        }
+        if (finish && active && t < L) {
+          const int64_t i = (b * D + c) * L + t;
           const float draw = fmaf(tx, sb, dd) * tsig;
           static_cast<T *>(p.du)[i] = from_f32<T>(fmaf(tD, sb, tg * D_c));
           static_cast<T *>(p.ddelta)[i] = from_f32<T>(draw);
@@ -425,7 +444,7 @@ __global__ void __launch_bounds__(kWarps * 32, 4) m1_bwd_kernel(const M1Params p
 #pragma unroll
         for (int qq = 1; qq < kCS; ++qq) s += racc[qq][off];
         const int64_t t = kb * kBlk + tt;
-        if (n < N && t < L) p.ws_bc[(((part * Bsz + b) * 2 + te) * N + n) * L + t] = s;
+        if (n < N && t < L) p.ws_bc[(((part * Bsz + b) * 2 + te) * ldN + ns + n) * L + t] = s;
       }
     }
   }
@@ -440,16 +459,16 @@ __global__ void __launch_bounds__(kWarps * 32, 4) m1_bwd_kernel(const M1Params p
     dbias_l += __shfl_xor_sync(0xffffffffu, dbias_l, off, kP);
   }
   if (active) {
-    float *m = p.ws_misc + (b * D + c) * (N + 2);
-    if (n0 < N) m[n0] = dA.x;
-    if (n1 < N) m[n1] = dA.y;
+    float *m = p.ws_misc + (b * D + c) * (ldN + 2);
+    if (n0 < N) m[ns + n0] = dA.x;
+    if (n1 < N) m[ns + n1] = dA.y;
     if (p.dh0) {
-      if (n0 < N) p.dh0[(b * D + c) * N + n0] = mu.x;
-      if (n1 < N) p.dh0[(b * D + c) * N + n1] = mu.y;
+      if (n0 < N) p.dh0[(b * D + c) * ldN + ns + n0] = mu.x;
+      if (n1 < N) p.dh0[(b * D + c) * ldN + ns + n1] = mu.y;
     }
-    if (pr == 0) {
-      m[N] = dD_l;
-      m[N + 1] = dbias_l;
+    if (pr == 0 && finish) {
+      m[ldN] = dD_l;
+      m[ldN + 1] = dbias_l;
     }
   }
 }
@@ -500,7 +519,7 @@ cudaError_t launch_t(const M1Params &p, cudaStream_t s) {
   cudaError_t err = cudaFuncSetAttribute(m1_bwd_kernel<T, kN>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
-  const int64_t grid_x = p.G * ctas_padded_per_group(p.D, p.N, p.G);
+  const int64_t grid_x = p.G * ctas_padded_per_group(p.D, kN, p.G);  // the layout's channels per CTA
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid_x, (unsigned)p.B);
   cfg.blockDim = dim3(Lay::kThreads);
@@ -513,19 +532,14 @@ cudaError_t launch_t(const M1Params &p, cudaStream_t s) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  err = cudaLaunchKernelEx(&cfg, m1_bwd_kernel<T, kN>, p);
-  if (err != cudaSuccess) return err;
-  const int64_t total = p.B * p.G * 2 * p.N * p.L + p.D * (p.N + 2);
-  const int threads = 256;
-  int64_t blocks = (total + threads - 1) / threads;
-  if (blocks > 148 * 16) blocks = 148 * 16;
-  m1_bwd_reduce_kernel<<<(unsigned)blocks, threads, 0, s>>>(p);
-  return cudaGetLastError();
+  return cudaLaunchKernelEx(&cfg, m1_bwd_kernel<T, kN>, p);
 }
 
+// one slab (or the whole d_state); slabs all run at the widest layout, so
+// that every slab has the same CTAs and dB/dC partials
 template <typename T>
 cudaError_t launch_n(const M1Params &p, cudaStream_t s) {
-  switch (pad_n(p.N)) {
+  switch (p.slab == kSlabWhole ? pad_n(p.N) : kM1Slab) {
     case 16: return launch_t<T, 16>(p, s);
     case 32: return launch_t<T, 32>(p, s);
     default: return launch_t<T, 64>(p, s);
@@ -536,22 +550,53 @@ cudaError_t launch_n(const M1Params &p, cudaStream_t s) {
 
 // Partials: one per cluster of CTAs; a group's channels fill whole clusters.
 int64_t m1_bwd_partials(int64_t D, int64_t N, int64_t G) {
-  return G * ctas_padded_per_group(D, N, G) / kM1BwdCluster;
+  return G * ctas_padded_per_group(D, N > kM1Slab ? kM1Slab : N, G) / kM1BwdCluster;
+}
+
+// Workspace: dB/dC partials [n_part][B][2][N][L], per-(b, c) partials
+// [B][D][N + 2], and above one slab the token sums [3][B][D][L].
+M1BwdWorkspace m1_bwd_workspace(int64_t B, int64_t D, int64_t N, int64_t L, int64_t G) {
+  auto up = [](size_t v) { return (v + 255) / 256 * 256; };
+  M1BwdWorkspace w;
+  w.n_part = m1_bwd_partials(D, N, G);
+  w.bc = 0;
+  w.misc = up(sizeof(float) * (size_t)(w.n_part * B * 2 * N * L));
+  w.tok = w.misc + up(sizeof(float) * (size_t)(B * D * (N + 2)));
+  w.bytes = w.tok + (N > kM1Slab ? sizeof(float) * (size_t)(3 * B * D * L) : 0);
+  return w;
 }
 
 size_t m1_bwd_workspace_bytes(int64_t B, int64_t D, int64_t N, int64_t L, int64_t G) {
-  const int64_t n_part = m1_bwd_partials(D, N, G);
-  size_t bc = sizeof(float) * (size_t)(n_part * B * 2 * N * L);
-  bc = (bc + 255) / 256 * 256;
-  return bc + sizeof(float) * (size_t)(B * D * (N + 2));
+  return m1_bwd_workspace(B, D, N, L, G).bytes;
 }
 
-cudaError_t launch_m1_bwd(const M1Params &p, cudaStream_t s) {
-  switch (p.io) {
-    case 1: return launch_n<bf16>(p, s);
-    case 2: return launch_n<f16>(p, s);
-    default: return launch_n<float>(p, s);
+// The whole d_state in one launch, or slabs of kM1Slab states in ascending
+// order (the token sums carried in tok_part), then the fixed-order reduction
+// of the partials over the full d_state.
+cudaError_t launch_m1_bwd(const M1Params &p0, cudaStream_t s) {
+  const int64_t n_tot = p0.N;
+  const int64_t slabs = (n_tot + kM1Slab - 1) / kM1Slab;
+  for (int64_t k = 0; k < slabs; ++k) {
+    M1Params p = p0;
+    p.ldN = n_tot;
+    p.n0 = k * kM1Slab;
+    p.N = n_tot - p.n0 < kM1Slab ? n_tot - p.n0 : kM1Slab;
+    p.slab = slabs == 1 ? kSlabWhole
+                        : (k == 0 ? kSlabFirst : (k == slabs - 1 ? kSlabLast : kSlabMiddle));
+    cudaError_t e;
+    switch (p.io) {
+      case 1: e = launch_n<bf16>(p, s); break;
+      case 2: e = launch_n<f16>(p, s); break;
+      default: e = launch_n<float>(p, s); break;
+    }
+    if (e != cudaSuccess) return e;
   }
+  const int64_t total = p0.B * p0.G * 2 * n_tot * p0.L + p0.D * (n_tot + 2);
+  const int threads = 256;
+  int64_t blocks = (total + threads - 1) / threads;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  m1_bwd_reduce_kernel<<<(unsigned)blocks, threads, 0, s>>>(p0);
+  return cudaGetLastError();
 }
 
 }  // namespace msc

@@ -45,7 +45,8 @@ struct FwdSmem {
   static constexpr int bc = tok + kCh * kTF * 4;              // [kTF][kP] float4
   static constexpr int ytile = bc + kTF * kP * 4;             // [kWarps][32/kP][kChBlock]
   static constexpr int out = ytile + kWarps * (32 / kP) * kChBlock;  // [kCh][kOut]
-  static constexpr int raw = (out + kCh * kOut + 3) / 4 * 4;  // raw inputs (16-byte aligned)
+  static constexpr int gate = out + kCh * kOut;               // [kCh][kOut] silu(z), last slab
+  static constexpr int raw = (gate + kCh * kOut + 3) / 4 * 4;  // raw inputs (16-byte aligned)
   static constexpr int total_floats = raw;
 };
 
@@ -119,11 +120,15 @@ __device__ __forceinline__ void fwd_issue_raw(const M1Params &p, unsigned char *
   cp_async_commit();
 }
 
-// Store the gated outputs of the chunk starting at tc from shared memory.
+// Store the outputs of the chunk starting at tc from shared memory.  Whole
+// d_state: the gated outputs.  Slabs: the first writes its sums over its
+// states to tok_part (f32), a middle one adds to them, the last adds them to
+// its own and stores the gated outputs.
 template <typename T, int kCh, int kOut>
-__device__ __forceinline__ void store_chunk(T *out_base, const float *sout, int64_t c_first,
-                                            int64_t c_end, int64_t b, int64_t D, int64_t L,
-                                            int64_t tc, bool vec, int tid, int nthreads) {
+__device__ __forceinline__ void store_chunk(const M1Params &p, const float *sout,
+                                            const float *sgate, int64_t c_first, int64_t c_end,
+                                            int64_t b, int64_t tc, int tid, int nthreads) {
+  const int64_t D = p.D, L = p.L;
   for (int u = tid; u < kCh * (kTF / 8); u += nthreads) {
     const int chl = u / (kTF / 8);
     const int seg = u % (kTF / 8);
@@ -131,8 +136,28 @@ __device__ __forceinline__ void store_chunk(T *out_base, const float *sout, int6
     if (c >= c_end) continue;
     const float4 a = *reinterpret_cast<const float4 *>(sout + chl * kOut + seg * 8);
     const float4 e = *reinterpret_cast<const float4 *>(sout + chl * kOut + seg * 8 + 4);
-    const float v[8] = {a.x, a.y, a.z, a.w, e.x, e.y, e.z, e.w};
-    store_run<8>(out_base + (b * D + c) * L, tc + seg * 8, L, vec, v);
+    float v[8] = {a.x, a.y, a.z, a.w, e.x, e.y, e.z, e.w};
+    const int64_t row = (b * D + c) * L, t0 = tc + seg * 8;
+    if (p.slab == kSlabWhole) {
+      store_run<8>(static_cast<T *>(p.out) + row, t0, L, p.vec, v);
+      continue;
+    }
+    if (p.slab != kSlabFirst) {
+      float prev[8];
+      load_run<8>(p.tok_part + row, t0, L, p.vec, prev, 0.f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = prev[i] + v[i];
+    }
+    if (p.slab == kSlabLast) {
+      const float4 ga = *reinterpret_cast<const float4 *>(sgate + chl * kOut + seg * 8);
+      const float4 ge = *reinterpret_cast<const float4 *>(sgate + chl * kOut + seg * 8 + 4);
+      const float g[8] = {ga.x, ga.y, ga.z, ga.w, ge.x, ge.y, ge.z, ge.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] *= g[i];
+      store_run<8>(static_cast<T *>(p.out) + row, t0, L, p.vec, v);
+    } else {
+      store_run<8>(p.tok_part + row, t0, L, p.vec, v);
+    }
   }
 }
 
@@ -148,6 +173,7 @@ __global__ void __launch_bounds__(kWarps * 32, 6) m1_fwd_kernel(const M1Params p
   float4 *sTok = reinterpret_cast<float4 *>(smem + S::tok);
   float4 *sBC = reinterpret_cast<float4 *>(smem + S::bc);
   float *sOut = smem + S::out;
+  float *sGate = smem + S::gate;
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -157,6 +183,7 @@ __global__ void __launch_bounds__(kWarps * 32, 6) m1_fwd_kernel(const M1Params p
   float *ytile = smem + S::ytile + (warp * Lay::kChPerWarp + chw) * S::kChBlock;
 
   const int64_t D = p.D, L = p.L, N = p.N;
+  const int64_t ldN = p.ldN, ns = p.n0;  // row length of A and the states; this slab's first state
   const int64_t b = blockIdx.y;
   // CTAs tile each B/C group separately, so a CTA never straddles two groups
   const int64_t per_group = D / p.G;
@@ -166,8 +193,8 @@ __global__ void __launch_bounds__(kWarps * 32, 6) m1_fwd_kernel(const M1Params p
   const int64_t c_end = (g + 1) * per_group;
   const int64_t c = c_first + chl;
   const bool active = c < c_end;
-  const T *Bg = static_cast<const T *>(p.Bm) + (b * p.G + g) * N * L;
-  const T *Cg = static_cast<const T *>(p.Cm) + (b * p.G + g) * N * L;
+  const T *Bg = static_cast<const T *>(p.Bm) + ((b * p.G + g) * ldN + ns) * L;
+  const T *Cg = static_cast<const T *>(p.Cm) + ((b * p.G + g) * ldN + ns) * L;
   const int64_t n_chunks = (L + kTF - 1) / kTF;
   const int64_t n_save = (L + kM1SaveInterval - 1) / kM1SaveInterval;
   using R = FwdRaw<T, kN>;
@@ -177,11 +204,11 @@ __global__ void __launch_bounds__(kWarps * 32, 6) m1_fwd_kernel(const M1Params p
   const int n0 = 2 * pr, n1 = 2 * pr + 1;
   float2 h = make_float2(0.f, 0.f), A2 = make_float2(0.f, 0.f);
   if (active) {
-    if (n0 < N) A2.x = p.A[c * N + n0] * kLog2e;
-    if (n1 < N) A2.y = p.A[c * N + n1] * kLog2e;
+    if (n0 < N) A2.x = p.A[c * ldN + ns + n0] * kLog2e;
+    if (n1 < N) A2.y = p.A[c * ldN + ns + n1] * kLog2e;
     if (p.h0) {
-      if (n0 < N) h.x = p.h0[(b * D + c) * N + n0];
-      if (n1 < N) h.y = p.h0[(b * D + c) * N + n1];
+      if (n0 < N) h.x = p.h0[(b * D + c) * ldN + ns + n0];
+      if (n1 < N) h.y = p.h0[(b * D + c) * ldN + ns + n1];
     }
   }
   // token conversion role: channel tcl, a run of kRun steps tseg (one run per thread)
@@ -190,7 +217,9 @@ __global__ void __launch_bounds__(kWarps * 32, 6) m1_fwd_kernel(const M1Params p
   const int tcl = tid % kCh, tseg = tid / kCh;
   const int64_t tcc = c_first + tcl;
   const bool tact = tcc < c_end;
-  const float tDc = (tact && p.Dp) ? p.Dp[tcc] : 0.f;
+  // the D x skip joins the sums once: in the whole or the last slab
+  const bool with_skip = p.slab == kSlabWhole || p.slab == kSlabLast;
+  const float tDc = (tact && p.Dp && with_skip) ? p.Dp[tcc] : 0.f;
   const float tbias = (tact && p.bias) ? p.bias[tcc] : 0.f;
 
   const T **const rows = reinterpret_cast<const T **>(raw + R::rows);
@@ -202,8 +231,7 @@ __global__ void __launch_bounds__(kWarps * 32, 6) m1_fwd_kernel(const M1Params p
     cp_async_wait<0>();
     __syncthreads();  // this chunk's raw inputs are in; the last chunk is done
     if (ch > 0)
-      store_chunk<T, kCh, S::kOut>(static_cast<T *>(p.out), sOut, c_first, c_end, b, D, L,
-                                   tc - kTF, p.vec, tid, kThreads);
+      store_chunk<T, kCh, S::kOut>(p, sOut, sGate, c_first, c_end, b, tc - kTF, tid, kThreads);
     if (ch == n_chunks) break;
     // ---- per-token values: kRun steps of one channel per thread ---------------
     {
@@ -267,7 +295,7 @@ __global__ void __launch_bounds__(kWarps * 32, 6) m1_fwd_kernel(const M1Params p
       for (int k = 0; k < kP; ++k) {
         const int t = grp * kP + k;
         if (t % kM1SaveInterval == 0 && active && p.saved && tc + t < L) {
-          float *dst = p.saved + ((b * D + c) * n_save + (tc + t) / kM1SaveInterval) * N;
+          float *dst = p.saved + ((b * D + c) * n_save + (tc + t) / kM1SaveInterval) * ldN + ns;
           if (n0 < N) dst[n0] = h.x;
           if (n1 < N) dst[n1] = h.y;
         }
@@ -288,13 +316,18 @@ __global__ void __launch_bounds__(kWarps * 32, 6) m1_fwd_kernel(const M1Params p
       float y = tk.z;
 #pragma unroll
       for (int q = 0; q < kP; ++q) y += ytile[q * S::kRow + pr];
-      sOut[chl * S::kOut + t] = y * tk.w;
+      if (p.slab == kSlabWhole) {
+        sOut[chl * S::kOut + t] = y * tk.w;
+      } else {
+        sOut[chl * S::kOut + t] = y;
+        sGate[chl * S::kOut + t] = tk.w;
+      }
       __syncwarp();
     }
   }
 
   if (active && p.final_state) {
-    float *dst = p.final_state + (b * D + c) * N;
+    float *dst = p.final_state + (b * D + c) * ldN + ns;
     if (n0 < N) dst[n0] = h.x;
     if (n1 < N) dst[n1] = h.y;
   }
@@ -315,7 +348,7 @@ cudaError_t launch_t(const M1Params &p, cudaStream_t s) {
 
 template <typename T>
 cudaError_t launch_n(const M1Params &p, cudaStream_t s) {
-  switch (pad_n(p.N)) {
+  switch (p.slab == kSlabWhole ? pad_n(p.N) : kM1Slab) {
     case 16: return launch_t<T, 16>(p, s);
     case 32: return launch_t<T, 32>(p, s);
     default: return launch_t<T, 64>(p, s);
@@ -324,12 +357,27 @@ cudaError_t launch_n(const M1Params &p, cudaStream_t s) {
 
 }  // namespace
 
-cudaError_t launch_m1_fwd(const M1Params &p, cudaStream_t s) {
-  switch (p.io) {
-    case 1: return launch_n<bf16>(p, s);
-    case 2: return launch_n<f16>(p, s);
-    default: return launch_n<float>(p, s);
+// The whole d_state in one launch, or slabs of kM1Slab states in ascending
+// order, the sums over the states carried in tok_part.
+cudaError_t launch_m1_fwd(const M1Params &p0, cudaStream_t s) {
+  const int64_t n_tot = p0.N;
+  const int64_t slabs = (n_tot + kM1Slab - 1) / kM1Slab;
+  for (int64_t k = 0; k < slabs; ++k) {
+    M1Params p = p0;
+    p.ldN = n_tot;
+    p.n0 = k * kM1Slab;
+    p.N = n_tot - p.n0 < kM1Slab ? n_tot - p.n0 : kM1Slab;
+    p.slab = slabs == 1 ? kSlabWhole
+                        : (k == 0 ? kSlabFirst : (k == slabs - 1 ? kSlabLast : kSlabMiddle));
+    cudaError_t e;
+    switch (p.io) {
+      case 1: e = launch_n<bf16>(p, s); break;
+      case 2: e = launch_n<f16>(p, s); break;
+      default: e = launch_n<float>(p, s); break;
+    }
+    if (e != cudaSuccess) return e;
   }
+  return cudaSuccess;
 }
 
 }  // namespace msc

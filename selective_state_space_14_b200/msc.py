@@ -43,7 +43,7 @@ class SsFwdArgs(ctypes.Structure):
                 ("dstate", _i64), ("seqlen", _i64), ("ngroups", _i64), ("delta_softplus", _i32),
                 ("u", _vp), ("delta", _vp), ("A", _vp), ("Bm", _vp), ("Cm", _vp), ("D", _vp),
                 ("delta_bias", _vp), ("z", _vp), ("h0", _vp), ("out", _vp), ("final_state", _vp),
-                ("saved_states", _vp)]
+                ("saved_states", _vp), ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t)]
 
 
 class SsBwdArgs(ctypes.Structure):
@@ -89,7 +89,7 @@ class M3SuArgs(ctypes.Structure):
 
 
 EXPORTS = ["msc_last_error", "msc_version", "msc_selective_scan_saved_states_bytes",
-           "msc_selective_scan_fwd", "msc_selective_scan_bwd_workspace_bytes",
+           "msc_selective_scan_fwd_workspace_bytes", "msc_selective_scan_fwd", "msc_selective_scan_bwd_workspace_bytes",
            "msc_selective_scan_bwd", "msc_selective_scan_bwd_static", "msc_ssm_state_update",
            "msc_mamba3_siso_saved_states_bytes",
            "msc_mamba3_siso_scan_fwd", "msc_mamba3_siso_scan_bwd_workspace_bytes",
@@ -122,6 +122,8 @@ def lib() -> ctypes.CDLL:
             f.restype = ctypes.c_int
         L.msc_selective_scan_saved_states_bytes.argtypes = [_i64] * 4
         L.msc_selective_scan_saved_states_bytes.restype = ctypes.c_size_t
+        L.msc_selective_scan_fwd_workspace_bytes.argtypes = [_i64] * 4
+        L.msc_selective_scan_fwd_workspace_bytes.restype = ctypes.c_size_t
         L.msc_selective_scan_bwd_workspace_bytes.argtypes = [_i64] * 5
         L.msc_selective_scan_bwd_workspace_bytes.restype = ctypes.c_size_t
         L.msc_mamba3_siso_saved_states_bytes.argtypes = [_i64] * 5
@@ -176,10 +178,16 @@ def msc_selective_scan_bwd_workspace_bytes(batch, dim, dstate, seqlen, ngroups=1
     return int(lib().msc_selective_scan_bwd_workspace_bytes(batch, dim, dstate, seqlen, ngroups))
 
 
+def msc_selective_scan_fwd_workspace_bytes(batch, dim, dstate, seqlen) -> int:
+    return int(lib().msc_selective_scan_fwd_workspace_bytes(batch, dim, dstate, seqlen))
+
+
 def msc_selective_scan_fwd(u, delta, A, B, C, D=None, delta_bias=None, z=None, h0=None,
                            delta_softplus=True, out=None, final_state=None, saved_states=None,
-                           want_final_state=True, want_saved_states=True, stream=None):
+                           want_final_state=True, want_saved_states=True, workspace=None,
+                           stream=None):
     """Mamba-1 forward.  u, delta, z: [B, D, L]; A: f32 [D, N]; B, C: [B, G, N, L].
+    Above 64 states a workspace is needed (allocated here if not given).
 
     Returns (out, final_state, saved_states)."""
     Bsz, Dm, L = u.shape
@@ -192,9 +200,14 @@ def msc_selective_scan_fwd(u, delta, A, B, C, D=None, delta_bias=None, z=None, h
     if saved_states is None and want_saved_states:
         n_save = (L + MSC_M1_SAVE_INTERVAL - 1) // MSC_M1_SAVE_INTERVAL
         saved_states = torch.empty((Bsz, Dm, max(n_save, 1), N), device=dev, dtype=torch.float32)
+    need = msc_selective_scan_fwd_workspace_bytes(Bsz, Dm, N, L)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, device=dev, dtype=torch.uint8)
     a = SsFwdArgs(ctypes.sizeof(SsFwdArgs), _io(u), Bsz, Dm, N, L, G, int(delta_softplus),
                   _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(delta_bias),
-                  _ptr(z), _ptr(h0), _ptr(out), _ptr(final_state), _ptr(saved_states))
+                  _ptr(z), _ptr(h0), _ptr(out), _ptr(final_state), _ptr(saved_states),
+                  _ptr(workspace), workspace.numel() * workspace.element_size()
+                  if workspace is not None else 0)
     _check(lib().msc_selective_scan_fwd(ctypes.byref(a), _stream(stream)))
     return out, final_state, saved_states
 

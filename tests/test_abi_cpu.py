@@ -78,13 +78,29 @@ def test_f16_is_an_io_dtype():
     ("batch", -1, INVALID, "batch"),
     ("seqlen", -5, INVALID, "seqlen"),
     ("dstate", 0, UNSUPPORTED, "dstate"),
-    ("dstate", 65, UNSUPPORTED, "dstate"),
+    ("dstate", 257, UNSUPPORTED, "dstate"),
     ("ngroups", 3, INVALID, "ngroups"),
     ("delta_softplus", 2, INVALID, "delta_softplus"),
 ])
 def test_fwd_rejects_bad_sizes(field, value, status, word):
     assert _call_fwd(_fwd_args(**{field: value})) == status
     assert word in _err()
+
+
+def test_fwd_wide_state_needs_a_workspace():
+    """Above 64 states the forward runs in slabs and needs its workspace; the
+    call stops at that check (no launch)."""
+    assert msc.msc_selective_scan_fwd_workspace_bytes(2, 64, 64, 128) == 0
+    assert msc.msc_selective_scan_fwd_workspace_bytes(2, 64, 65, 128) == 4 * 2 * 64 * 128
+    assert _call_fwd(_fwd_args(dstate=128)) == WORKSPACE and "workspace" in _err()
+
+
+def test_fwd_accepts_the_struct_without_workspace_fields():
+    """A struct that ends before the workspace fields is still read (a NULL u
+    stops the call at the pointer checks, before any launch)."""
+    short = msc.SsFwdArgs.workspace.offset
+    assert _call_fwd(_fwd_args(struct_size=short, u=None)) == INVALID and "u is NULL" in _err()
+    assert _call_fwd(_fwd_args(struct_size=short - 8)) == INVALID and "struct_size" in _err()
 
 
 def test_fwd_rejects_missing_input():

@@ -82,6 +82,13 @@ CASES = [
     (1, 24, 64, 96, 1, "f16", True, True, True, True, True),
     (1, 7, 5, 513, 1, "f16", False, True, True, False, True),
     (2, 100, 32, 1000, 2, "f16", True, True, True, True, True),
+    # d_state above 64: slabs of 64 states (first + last, first + middles + last,
+    # a narrow last slab)
+    (1, 8, 128, 300, 1, "f32", True, True, True, True, True),
+    (2, 12, 100, 257, 1, "f32", False, True, True, True, True),
+    (1, 16, 256, 130, 2, "bf16", True, True, True, True, True),
+    (2, 40, 96, 1000, 1, "bf16", True, False, True, True, True),
+    (1, 8, 200, 64, 1, "f16", True, True, True, True, True),
 ]
 
 
@@ -198,6 +205,24 @@ def test_state_update_chain(msc, io):
                                                 z=s["z"].as_f64())
         assert_close("out", host(o), o_ref, TOL[io])
     assert_close("state", host(st), st_ref, TOL[io])
+
+
+def test_state_update_wide_state(msc):
+    """The decode step with 200 states (the step has no d_state limit below 256)."""
+    q = W.su_problem(2, 24, 200, io="bf16", seed=8, random_state=True, n_pool=6)
+    st = torch.from_numpy(q.state0).cuda()
+    st_ref = q.state0.astype(np.float64)
+    A, Dp, bias = dev(q.A), dev(q.D), dev(q.delta_bias)
+    for s in q.steps:
+        o = msc.msc_ssm_state_update(st, dev(s["x"]), dev(s["delta"]), A, dev(s["B"]),
+                                     dev(s["C"]), D=Dp, delta_bias=bias, z=dev(s["z"]))
+        st_ref, o_ref = oracle.ssm_state_update(st_ref, s["x"].as_f64(), s["delta"].as_f64(),
+                                                q.A.astype(np.float64), s["B"].as_f64(),
+                                                s["C"].as_f64(), D=q.D.astype(np.float64),
+                                                delta_bias=q.delta_bias.astype(np.float64),
+                                                z=s["z"].as_f64())
+        assert_close("out", host(o), o_ref, TOL["bf16"])
+    assert_close("state", host(st), st_ref, TOL["bf16"])
 
 
 def test_state_update_decode_workload_sampled(msc):
