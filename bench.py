@@ -100,7 +100,7 @@ def m3su_bytes(Bsz, H, P, N, G, K, io_bytes):
 # ---------------------------------------------------------------------------
 NCU_TRAFFIC = {
     # kernel source file: (sha256 prefix of the file, workload, bytes per launch)
-    "m1_bwd.cu": ("11a659c65d88cc6a", "m1_bf16_b8_d1536_n16_l2048", 404215040 + 157788672),
+    "m1_bwd.cu": ("4523265612d28912", "m1_bf16_b8_d1536_n16_l2048", 404786688 + 159501312),
 }
 
 
