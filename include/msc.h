@@ -256,7 +256,11 @@ msc_status msc_ssm_state_update(const msc_su_args *args, msc_stream_t stream);
  *          S_{-1} = h0 (or 0)
  *   y_t  = S_t Ct_t + D[h] x[b,t,h,:];  out = y_t * silu(z[b,t,h,:])
  * final_state receives S_{L-1}.
- * Supported: P and N each in {16, 32, 64}; L >= 0 (L = 0 copies h0 to final_state).
+ * Supported: P in {16, 32, 64}; N in {16, 32, 64} and, as slabs of 64
+ * states, {128, 192, 256} ("state dimensions up to 256", mamba-rs README,
+ * "Features"; the Mamba README's Mamba-3 example uses 128); L >= 0 (L = 0
+ * copies h0 to final_state).  Above 64 states the forward needs a workspace
+ * of msc_mamba3_siso_scan_fwd_workspace_bytes() bytes (0 up to 64 states).
  */
 typedef struct {
   uint32_t struct_size;
@@ -271,7 +275,13 @@ typedef struct {
   void *out;
   float *final_state;      /* optional */
   float *saved_states;     /* optional; required if the backward pass follows */
+  void *workspace;         /* required when dstate > 64, else ignored (may be NULL) */
+  size_t workspace_bytes;
 } msc_m3_fwd_args;
+
+/* Bytes of the forward's workspace for these sizes (0 when dstate <= 64). */
+size_t msc_mamba3_siso_scan_fwd_workspace_bytes(int64_t batch, int64_t seqlen, int64_t nheads,
+                                                int64_t headdim, int64_t dstate);
 
 /* saved_states holds S at the start of every block of MSC_M3_CHUNK steps,
  * f32 [B, H, ceil(L / MSC_M3_CHUNK), P, N], followed by the cumulative angles
@@ -352,7 +362,7 @@ msc_status msc_mamba3_siso_scan_bwd(const msc_m3_bwd_args *args, void *workspace
  *   S     <- alpha S + beta x_prev (outer) bt_prev + gamma x (outer) Bt
  *   out    = (S Ct + D[h] x) * silu(z)
  *   x_prev <- x,  bt_prev <- Bt
- * Supported: P and N each in {16, 32, 64}, 2K <= N.  Every pointer is
+ * Supported: P in {16, 32, 64}, N in {16, 32, 64, 128, 192, 256}, 2K <= N.  Every pointer is
  * 16-byte aligned; z and D are optional, theta and phi may be NULL when K = 0.
  */
 typedef struct {

@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdarg>
+#include <cstddef>
 #include <cstdio>
 
 #include "../../include/msc.h"
@@ -41,11 +42,11 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
   } while (0)
 
 template <typename Args>
-msc_status check_m3(const char *fn, const Args *a) {
+msc_status check_m3(const char *fn, const Args *a, size_t min_size = sizeof(Args)) {
   if (!a) return api_fail(MSC_ERR_INVALID_ARG, "%s: args is NULL", fn);
-  if (a->struct_size < sizeof(Args))
+  if (a->struct_size < min_size)
     return api_fail(MSC_ERR_INVALID_ARG, "%s: struct_size %u is smaller than the struct (%zu)",
-                    fn, a->struct_size, sizeof(Args));
+                    fn, a->struct_size, min_size);
   if (a->io_dtype != MSC_F32 && a->io_dtype != MSC_BF16 && a->io_dtype != MSC_F16)
     return api_fail(MSC_ERR_INVALID_ARG,
                     "%s: io_dtype %d is not MSC_F32 (0), MSC_BF16 (1) or MSC_F16 (2)",
@@ -59,7 +60,8 @@ msc_status check_m3(const char *fn, const Args *a) {
                     (long long)a->ngroups, (long long)a->nheads);
   if (!msc::m3_supported(a->headdim, a->dstate))
     return api_fail(MSC_ERR_UNSUPPORTED,
-                    "%s: headdim %lld / dstate %lld not supported (each must be 16, 32 or 64)", fn,
+                    "%s: headdim %lld / dstate %lld not supported (headdim 16, 32 or 64; dstate 16, "
+                    "32, 64, 128, 192 or 256)", fn,
                     (long long)a->headdim, (long long)a->dstate);
   if (2 * a->nangles > a->dstate)
     return api_fail(MSC_ERR_INVALID_ARG, "%s: 2 * nangles (%lld) exceeds dstate (%lld)", fn,
@@ -81,10 +83,20 @@ size_t msc_mamba3_siso_saved_states_bytes(int64_t batch, int64_t seqlen, int64_t
   return sizeof(float) * (size_t)(batch * nheads * nc * (headdim * dstate + dstate / 2));
 }
 
+size_t msc_mamba3_siso_scan_fwd_workspace_bytes(int64_t batch, int64_t seqlen, int64_t nheads,
+                                                int64_t headdim, int64_t dstate) {
+  if (batch <= 0 || seqlen <= 0 || nheads <= 0 || headdim <= 0 || dstate <= msc::kM3Slab) return 0;
+  return sizeof(float) * (size_t)(batch * seqlen * nheads * headdim);  // y over the earlier slabs
+}
+
 msc_status msc_mamba3_siso_scan_fwd(const msc_m3_fwd_args *a, msc_stream_t stream) {
   const char *fn = "msc_mamba3_siso_scan_fwd";
-  msc_status st = check_m3(fn, a);
+  // callers built before the workspace fields pass a shorter struct: no workspace
+  msc_status st = check_m3(fn, a, offsetof(msc_m3_fwd_args, workspace));
   if (st != MSC_OK) return st;
+  const bool has_ws_fields = a->struct_size >= sizeof(msc_m3_fwd_args);
+  void *const workspace = has_ws_fields ? a->workspace : nullptr;
+  const size_t workspace_bytes = has_ws_fields ? a->workspace_bytes : 0;
   if (a->batch == 0) return api_ok();
   M3_OPTIONAL(fn, "D", a->D);
   M3_OPTIONAL(fn, "h0", a->h0);
@@ -111,6 +123,11 @@ msc_status msc_mamba3_siso_scan_fwd(const msc_m3_fwd_args *a, msc_stream_t strea
   M3_REQUIRE(fn, "out", a->out);
   M3_OPTIONAL(fn, "z", a->z);
   M3_OPTIONAL(fn, "saved_states", a->saved_states);
+  const size_t need = msc_mamba3_siso_scan_fwd_workspace_bytes(B, a->seqlen, H, P, N);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need))
+    return api_fail(MSC_ERR_WORKSPACE, "%s: dstate %lld needs a workspace of %zu bytes, %zu given",
+                    fn, (long long)N, need, workspace ? workspace_bytes : (size_t)0);
+  M3_OPTIONAL(fn, "workspace", workspace);
   msc::M3Params p = {};
   p.io = a->io_dtype;
   p.B = B; p.L = a->seqlen; p.H = H; p.P = P; p.N = N; p.G = a->ngroups; p.K = a->nangles;
@@ -118,6 +135,7 @@ msc_status msc_mamba3_siso_scan_fwd(const msc_m3_fwd_args *a, msc_stream_t strea
   p.alpha = a->alpha; p.beta = a->beta; p.gamma = a->gamma; p.theta = a->theta;
   p.Dp = a->D; p.h0 = a->h0; p.out = a->out; p.final_state = a->final_state;
   p.saved = a->saved_states;
+  p.tok_y = need > 0 ? static_cast<float *>(workspace) : nullptr;
   return api_cuda(msc::launch_m3_fwd(p, s), fn);
 }
 
@@ -208,7 +226,8 @@ msc_status msc_mamba3_siso_state_update(const msc_m3_su_args *a, msc_stream_t st
                     (long long)a->ngroups, (long long)a->nheads);
   if (!msc::m3_supported(a->headdim, a->dstate))
     return api_fail(MSC_ERR_UNSUPPORTED,
-                    "%s: headdim %lld / dstate %lld not supported (each must be 16, 32 or 64)", fn,
+                    "%s: headdim %lld / dstate %lld not supported (headdim 16, 32 or 64; dstate 16, "
+                    "32, 64, 128, 192 or 256)", fn,
                     (long long)a->headdim, (long long)a->dstate);
   if (2 * a->nangles > a->dstate)
     return api_fail(MSC_ERR_INVALID_ARG, "%s: 2 * nangles (%lld) exceeds dstate (%lld)", fn,

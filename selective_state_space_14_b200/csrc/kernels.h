@@ -87,7 +87,16 @@ struct M3Params {
   float *dB, *dC, *dalpha, *dbeta, *dgamma, *dtheta, *dD, *dh0;
   void *ws;
   size_t ws_bytes;
+  // d_state above kM3Slab runs as slabs (N the slab's width, n0 its first
+  // state, ldN the full d_state; angle pairs n0/2 .. n0/2 + N/2 - 1 of the
+  // K); the sums over the states of each output carry from slab to slab:
+  // fwd y in tok_y, bwd y (for dz) in tok_y and dx in tok_dx, dalpha, dbeta,
+  // dgamma in place.  The last slab finishes them.
+  int64_t n0, ldN;
+  int slab;  // kSlabWhole, kSlabFirst, kSlabMiddle or kSlabLast
+  float *tok_y, *tok_dx;  // [B, L, H, P] f32
 };
+constexpr int kM3Slab = 64;  // widest d_state one launch handles
 cudaError_t launch_m3_fwd(const M3Params &p, cudaStream_t s);
 cudaError_t launch_m3_fwd_umma(const M3Params &p, cudaStream_t s);  // bf16 io, tcgen05
 cudaError_t launch_m3_bwd(const M3Params &p, cudaStream_t s);

@@ -114,7 +114,9 @@ struct BwdSmem {
   static constexpr int total = red + kThreads;
 };
 
-template <typename T, int P, int N>
+// kSlab: one slab of a wider d_state (runtime row length and offsets);
+// otherwise the whole d_state with compile-time strides
+template <typename T, int P, int N, bool kSlab>
 __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, float *ws_dB,
                                                              float *ws_dC, float *ws_dD) {
   using S = BwdSmem<P, N>;
@@ -135,12 +137,18 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
 
   const int tid = threadIdx.x;
   const int64_t h = blockIdx.x, b = blockIdx.y;
-  const int64_t L = p.L, H = p.H, G = p.G, K = p.K;
+  const int64_t L = p.L, H = p.H, G = p.G;
+  // this slab's states n0 .. n0 + N - 1 of ldN; its angle pairs k0 .. k0 + K - 1 of Kt
+  const int64_t ldN = kSlab ? p.ldN : N, n0 = kSlab ? p.n0 : 0, Kt = p.K, k0 = n0 / 2;
+  const int64_t K = Kt - k0 < 0 ? 0 : (Kt - k0 > kK ? kK : Kt - k0);
+  const int slab = kSlab ? p.slab : kSlabWhole;
+  const bool finish = slab == kSlabWhole || slab == kSlabLast;
   const int64_t g = h / (H / G);
-  const float Dh = p.Dp ? p.Dp[h] : 0.f;
+  const float Dh = (p.Dp && finish) ? p.Dp[h] : 0.f;  // the D terms join once
   const int64_t n_chunks = (L + kQ - 1) / kQ;
   // chunk-start angles, as the forward accumulated them (after the states)
-  const float *phi_start = p.saved_in + p.B * H * n_chunks * P * N + (b * H + h) * n_chunks * kK;
+  const float *phi_start =
+      p.saved_in + p.B * H * n_chunks * P * ldN + (b * H + h) * n_chunks * (ldN / 2) + k0;
 
   for (int i = tid; i < P * lN; i += kThreads) sU[i] = 0.f;
   for (int i = tid; i < kK; i += kThreads) sDth[i] = 0.f;
@@ -153,10 +161,10 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
     // ---- A. stage the chunk ---------------------------------------------------
     // the chunk's starting state by cp.async, straight into its padded rows
     {
-      const float *src = p.saved_in + ((b * H + h) * n_chunks + ch) * P * N;
+      const float *src = p.saved_in + ((b * H + h) * n_chunks + ch) * P * ldN + n0;
       for (int u = tid; u < P * (N / 4); u += kThreads) {
         const int r = u / (N / 4), pc = u % (N / 4);
-        cp_async16(sSin + r * lN + pc * 4, src + r * N + pc * 4, 16);
+        cp_async16(sSin + r * lN + pc * 4, src + r * ldN + pc * 4, 16);
       }
       cp_async_commit();
     }
@@ -191,7 +199,7 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
     for (int u = tid; u < kQ * (N / 8); u += kThreads) {
       const int t = u / (N / 8), pc = u % (N / 8);
       const bool in = t < Qc;
-      const int64_t j = ((b * L + t0 + t) * G + g) * N + pc * 8;
+      const int64_t j = ((b * L + t0 + t) * G + g) * ldN + n0 + pc * 8;
       float bv[8], cv[8];
       ld8<T>(p.Bm, j, in, bv);
       ld8<T>(p.Cm, j, in, cv);
@@ -210,13 +218,13 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
     }
     for (int i = tid; i < kQ * K; i += kThreads) {
       const int t = i / (int)K, k = i % (int)K;
-      sPhi[t * kK + k] = t < Qc ? ldv<T>(p.theta, ((b * L + t0 + t) * H + h) * K + k) : 0.f;
+      sPhi[t * kK + k] = t < Qc ? ldv<T>(p.theta, ((b * L + t0 + t) * H + h) * Kt + k0 + k) : 0.f;
     }
-    for (int i = tid; i < kK; i += kThreads) sPhiSt[i] = i < K ? phi_start[ch * kK + i] : 0.f;
+    for (int i = tid; i < kK; i += kThreads) sPhiSt[i] = i < K ? phi_start[ch * (ldN / 2) + i] : 0.f;
     for (int i = tid; i < P; i += kThreads)
       sXprev[i] = t0 > 0 ? ldv<T>(p.x, ((b * L + t0 - 1) * H + h) * P + i) : 0.f;
     for (int i = tid; i < N; i += kThreads)
-      sBprev[i] = t0 > 0 ? ldv<T>(p.Bm, ((b * L + t0 - 1) * G + g) * N + i) : 0.f;
+      sBprev[i] = t0 > 0 ? ldv<T>(p.Bm, ((b * L + t0 - 1) * G + g) * ldN + n0 + i) : 0.f;
     // the previous chunk's rows into L2 while this one computes
     if (ch > 0) {
       const int64_t tp = t0 - kQ;
@@ -228,13 +236,14 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
           if (!base) continue;
           ptr = static_cast<const T *>(base) + ((b * L + tp + t) * H + h) * P;
         } else {
-          ptr = static_cast<const T *>(p.Bm) + ((b * L + tp + t) * G + g) * N;
+          ptr = static_cast<const T *>(p.Bm) + ((b * L + tp + t) * G + g) * ldN + n0;
         }
         asm volatile("prefetch.global.L2 [%0];" ::"l"(ptr));
       }
-      const float *sv = p.saved_in + ((b * H + h) * n_chunks + ch - 1) * P * N;
-      for (int u = tid; u < P * N / 32; u += kThreads)
-        asm volatile("prefetch.global.L2 [%0];" ::"l"(sv + u * 32));
+      const float *sv = p.saved_in + ((b * H + h) * n_chunks + ch - 1) * P * ldN + n0;
+      constexpr int kLines = (N + 31) / 32;  // 128-byte lines per row
+      for (int u = tid; u < P * kLines; u += kThreads)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(sv + (u / kLines) * ldN + (u % kLines) * 32));
     }
     cp_async_wait<0>();
     __syncthreads();
@@ -307,9 +316,16 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
       for (int i = tid; i < kQ * P; i += kThreads) {
         const int t = i / P, pp = i % P;
         if (t < Qc) {
-          const float y =
+          float y =
               sT1[t * lMx + pp] + sBe[0] * sD0[t] * sCbp[t] * sXprev[pp] + Dh * sX[t * lP + pp];
           const int64_t j = ((b * L + t0 + t) * H + h) * P + pp;
+          if (slab != kSlabWhole) {  // y sums over the states: across the slabs
+            if (slab != kSlabFirst) y = p.tok_y[j] + y;
+            if (!finish) {
+              p.tok_y[j] = y;
+              continue;
+            }
+          }
           const float dy = ldv<T>(p.dout, j);
           static_cast<T *>(p.dz)[j] = from_f32<T>(y * dy * dsilu(ldv<T>(p.z, j)));
         }
@@ -364,9 +380,18 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
     __syncthreads();
     for (int i = tid; i < kQ * P; i += kThreads) {
       const int t = i / P, pp = i % P;
-      if (t < Qc)
-        static_cast<T *>(p.dx)[((b * L + t0 + t) * H + h) * P + pp] =
-            from_f32<T>(fmaf(Dh, sG[t * lP + pp], sT1[t * lMx + pp]));
+      if (t < Qc) {
+        const int64_t j = ((b * L + t0 + t) * H + h) * P + pp;
+        float v = fmaf(Dh, sG[t * lP + pp], sT1[t * lMx + pp]);
+        if (slab != kSlabWhole) {  // dx sums over the states: across the slabs
+          if (slab != kSlabFirst) v = p.tok_dx[j] + v;
+          if (!finish) {
+            p.tok_dx[j] = v;
+            continue;
+          }
+        }
+        static_cast<T *>(p.dx)[j] = from_f32<T>(v);
+      }
     }
     mmx<T, kQ, N, kQ, true, false>(sW, lN, sCB, lQ, sCt, lN, nullptr, nullptr, false);
     // v_s = x_s^T U Bt_s (s >= 0), v_{-1} with the previous step; <U, S_in>
@@ -438,17 +463,19 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
       float excl = __shfl_down_sync(0xffffffffu, incl, 1);
       if (tid == 31) excl = 0.f;
       const float a1 = excl + v1, a0 = a1 + v0;
+      // (slabs after the first add their sums over the states in place)
+      const bool add = slab == kSlabMiddle || slab == kSlabLast;
       if (r0 < Qc) {
         const int64_t j = (b * L + t0 + r0) * H + h;
-        p.dalpha[j] = a0 / sAl[r0];
-        p.dbeta[j] = sDbet[r0];
-        p.dgamma[j] = sDgam[r0];
+        p.dalpha[j] = (add ? p.dalpha[j] : 0.f) + a0 / sAl[r0];
+        p.dbeta[j] = (add ? p.dbeta[j] : 0.f) + sDbet[r0];
+        p.dgamma[j] = (add ? p.dgamma[j] : 0.f) + sDgam[r0];
       }
       if (r1 < Qc) {
         const int64_t j = (b * L + t0 + r1) * H + h;
-        p.dalpha[j] = a1 / sAl[r1];
-        p.dbeta[j] = sDbet[r1];
-        p.dgamma[j] = sDgam[r1];
+        p.dalpha[j] = (add ? p.dalpha[j] : 0.f) + a1 / sAl[r1];
+        p.dbeta[j] = (add ? p.dbeta[j] : 0.f) + sDbet[r1];
+        p.dgamma[j] = (add ? p.dgamma[j] : 0.f) + sDgam[r1];
       }
     }
     __syncthreads();
@@ -469,7 +496,7 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
         rc1 = -sn * dc0 + cs * dc1;
       }
       if (t < Qc) {
-        const int64_t j = ((b * L + t0 + t) * H + h) * N + 2 * k;
+        const int64_t j = ((b * L + t0 + t) * H + h) * ldN + n0 + 2 * k;
         ws_dB[j] = rb0;
         ws_dB[j + 1] = rb1;
         ws_dC[j] = rc0;
@@ -490,7 +517,7 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
       float acc = sDth[tid];
       for (int t = Qc - 1; t >= 0; --t) {
         acc += sPhi[t * kK + tid];
-        p.dtheta[((b * L + t0 + t) * H + h) * K + tid] = acc;
+        p.dtheta[((b * L + t0 + t) * H + h) * Kt + k0 + tid] = acc;
       }
       sDth[tid] = acc;
     }
@@ -509,10 +536,10 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
 
   if (p.dh0) {
     for (int i = tid; i < P * N; i += kThreads)
-      p.dh0[(b * H + h) * P * N + i] = alQ * sU[(i / N) * lN + i % N];  // alpha_0 Lambda_0
+      p.dh0[((b * H + h) * P + i / N) * ldN + n0 + i % N] = alQ * sU[(i / N) * lN + i % N];  // alpha_0 Lambda_0
   }
   const float dD = block_sum(dD_l, sRed);
-  if (tid == 0) ws_dD[b * H + h] = dD;
+  if (tid == 0 && finish) ws_dD[b * H + h] = dD;
 }
 
 // dB, dC: the heads of each group added in ascending head order; dD: the
@@ -542,48 +569,48 @@ __global__ void m3_bwd_reduce_kernel(const M3Params p, const float *ws_dB, const
   }
 }
 
+// per-head dB, dC [B, L, H, N]; per-(b, h) dD [B, H]; above one slab the
+// sums over the states of y and dx [B, L, H, P]
 struct WsLayout {
-  size_t dB, dC, dD, total;
+  size_t dB, dC, dD, tok_y, tok_dx, total;
 };
 
-WsLayout ws_layout(int64_t B, int64_t L, int64_t H, int64_t N) {
+WsLayout ws_layout(int64_t B, int64_t L, int64_t H, int64_t P, int64_t N) {
   auto up = [](size_t v) { return (v + 255) / 256 * 256; };
   WsLayout w;
   w.dB = 0;
   w.dC = w.dB + up(sizeof(float) * (size_t)(B * L * H * N));
   w.dD = w.dC + up(sizeof(float) * (size_t)(B * L * H * N));
-  w.total = w.dD + up(sizeof(float) * (size_t)(B * H));
+  w.tok_y = w.dD + up(sizeof(float) * (size_t)(B * H));
+  const size_t tok = N > kM3Slab ? up(sizeof(float) * (size_t)(B * L * H * P)) : 0;
+  w.tok_dx = w.tok_y + tok;
+  w.total = w.tok_dx + tok;
   return w;
 }
 
-template <typename T, int P, int N>
+template <typename T, int P, int N, bool kSlab>
 cudaError_t launch_t(const M3Params &p, cudaStream_t s) {
   const size_t smem = sizeof(float) * (size_t)BwdSmem<P, N>::total;
-  cudaError_t e = cudaFuncSetAttribute(m3_bwd_kernel<T, P, N>,
+  cudaError_t e = cudaFuncSetAttribute(m3_bwd_kernel<T, P, N, kSlab>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const WsLayout w = ws_layout(p.B, p.L, p.H, p.N);
+  const WsLayout w = ws_layout(p.B, p.L, p.H, p.P, p.ldN);
   char *ws = static_cast<char *>(p.ws);
   float *dB = reinterpret_cast<float *>(ws + w.dB);
   float *dC = reinterpret_cast<float *>(ws + w.dC);
   float *dD = reinterpret_cast<float *>(ws + w.dD);
-  m3_bwd_kernel<T, P, N><<<dim3((unsigned)p.H, (unsigned)p.B), kThreads, smem, s>>>(p, dB, dC,
-                                                                                  dD);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  const int64_t total = p.B * p.L * p.G * p.N + p.H;
-  int64_t blocks = (total + 255) / 256;
-  if (blocks > 148 * 16) blocks = 148 * 16;
-  m3_bwd_reduce_kernel<<<(unsigned)blocks, 256, 0, s>>>(p, dB, dC, dD);
+  m3_bwd_kernel<T, P, N, kSlab><<<dim3((unsigned)p.H, (unsigned)p.B), kThreads, smem, s>>>(
+      p, dB, dC, dD);
   return cudaGetLastError();
 }
 
 template <typename T, int P>
 cudaError_t launch_n(const M3Params &p, cudaStream_t s) {
+  if (p.slab != kSlabWhole) return launch_t<T, P, kM3Slab, true>(p, s);
   switch (p.N) {
-    case 16: return launch_t<T, P, 16>(p, s);
-    case 32: return launch_t<T, P, 32>(p, s);
-    default: return launch_t<T, P, 64>(p, s);
+    case 16: return launch_t<T, P, 16, false>(p, s);
+    case 32: return launch_t<T, P, 32, false>(p, s);
+    default: return launch_t<T, P, 64, false>(p, s);
   }
 }
 
@@ -600,18 +627,45 @@ cudaError_t launch_p(const M3Params &p, cudaStream_t s) {
 
 size_t m3_bwd_workspace_bytes(int64_t B, int64_t L, int64_t H, int64_t P, int64_t N, int64_t G,
                               int64_t K) {
-  (void)P;
   (void)G;
   (void)K;
-  return ws_layout(B, L, H, N).total;
+  return ws_layout(B, L, H, P, N).total;
 }
 
-cudaError_t launch_m3_bwd(const M3Params &p, cudaStream_t s) {
-  switch (p.io) {
-    case 1: return launch_p<bf16>(p, s);
-    case 2: return launch_p<f16>(p, s);
-    default: return launch_p<float>(p, s);
+// The whole d_state in one launch, or slabs of kM3Slab states in ascending
+// order (sums over the states carried in the workspace and in dalpha, dbeta,
+// dgamma), then the fixed-order sum of dB, dC over the heads of a group and
+// of dD over the batch.
+cudaError_t launch_m3_bwd(const M3Params &p0, cudaStream_t s) {
+  const int64_t n_tot = p0.N;
+  const int64_t slabs = (n_tot + kM3Slab - 1) / kM3Slab;
+  const WsLayout w = ws_layout(p0.B, p0.L, p0.H, p0.P, n_tot);
+  char *ws = static_cast<char *>(p0.ws);
+  for (int64_t k = 0; k < slabs; ++k) {
+    M3Params p = p0;
+    p.ldN = n_tot;
+    p.n0 = k * kM3Slab;
+    p.N = n_tot - p.n0 < kM3Slab ? n_tot - p.n0 : kM3Slab;
+    p.slab = slabs == 1 ? kSlabWhole
+                        : (k == 0 ? kSlabFirst : (k == slabs - 1 ? kSlabLast : kSlabMiddle));
+    p.tok_y = slabs > 1 ? reinterpret_cast<float *>(ws + w.tok_y) : nullptr;
+    p.tok_dx = slabs > 1 ? reinterpret_cast<float *>(ws + w.tok_dx) : nullptr;
+    cudaError_t e;
+    switch (p.io) {
+      case 1: e = launch_p<bf16>(p, s); break;
+      case 2: e = launch_p<f16>(p, s); break;
+      default: e = launch_p<float>(p, s); break;
+    }
+    if (e != cudaSuccess) return e;
   }
+  float *dB = reinterpret_cast<float *>(ws + w.dB);
+  float *dC = reinterpret_cast<float *>(ws + w.dC);
+  float *dD = reinterpret_cast<float *>(ws + w.dD);
+  const int64_t total = p0.B * p0.L * p0.G * n_tot + p0.H;
+  int64_t blocks = (total + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  m3_bwd_reduce_kernel<<<(unsigned)blocks, 256, 0, s>>>(p0, dB, dC, dD);
+  return cudaGetLastError();
 }
 
 }  // namespace msc

@@ -41,7 +41,9 @@ struct FwdSmem {
   static constexpr int total = phiprev + kK;
 };
 
-template <typename T, int P, int N>
+// kSlab: one slab of a wider d_state (runtime row length and offsets);
+// otherwise the whole d_state with compile-time strides
+template <typename T, int P, int N, bool kSlab>
 __global__ void __launch_bounds__(kThreads, 1) m3_fwd_kernel(const M3Params p) {
   using S = FwdSmem<P, N>;
   extern __shared__ float4 smem4[];
@@ -55,14 +57,19 @@ __global__ void __launch_bounds__(kThreads, 1) m3_fwd_kernel(const M3Params p) {
 
   const int tid = threadIdx.x;
   const int64_t h = blockIdx.x, b = blockIdx.y;
-  const int64_t L = p.L, H = p.H, G = p.G, K = p.K;
+  const int64_t L = p.L, H = p.H, G = p.G;
+  // this slab's states n0 .. n0 + N - 1 of ldN; its angle pairs k0 .. k0 + K - 1 of Kt
+  const int64_t ldN = kSlab ? p.ldN : N, n0 = kSlab ? p.n0 : 0, Kt = p.K, k0 = n0 / 2;
+  const int64_t K = Kt - k0 < 0 ? 0 : (Kt - k0 > S::kK ? S::kK : Kt - k0);
+  const int slab = kSlab ? p.slab : kSlabWhole;
+  const bool finish = slab == kSlabWhole || slab == kSlabLast;
   const int64_t g = h / (H / G);
-  const float Dh = p.Dp ? p.Dp[h] : 0.f;
+  const float Dh = (p.Dp && finish) ? p.Dp[h] : 0.f;  // the D x skip joins once
   const int64_t n_chunks = (L + kQ - 1) / kQ;
 
   for (int i = tid; i < N * P; i += kThreads) {
     const int n = i / P, pp = i % P;
-    sST[i] = p.h0 ? p.h0[((b * H + h) * P + pp) * N + n] : 0.f;
+    sST[i] = p.h0 ? p.h0[((b * H + h) * P + pp) * ldN + n0 + n] : 0.f;
   }
   for (int i = tid; i < P; i += kThreads) sXprev[i] = 0.f;
   for (int i = tid; i < N; i += kThreads) sBprev[i] = 0.f;
@@ -80,7 +87,7 @@ __global__ void __launch_bounds__(kThreads, 1) m3_fwd_kernel(const M3Params p) {
     for (int i = tid; i < kQ * N; i += kThreads) {
       const int t = i / N, n = i % N;
       const bool in = t < Qc;
-      const int64_t j = ((b * L + t0 + t) * G + g) * N + n;
+      const int64_t j = ((b * L + t0 + t) * G + g) * ldN + n0 + n;
       sBt[i] = in ? ldv<T>(p.Bm, j) : 0.f;
       sG[i] = in ? ldv<T>(p.Cm, j) : 0.f;  // raw C, [Q][N], until the rotation
     }
@@ -93,7 +100,7 @@ __global__ void __launch_bounds__(kThreads, 1) m3_fwd_kernel(const M3Params p) {
     }
     for (int i = tid; i < kQ * K; i += kThreads) {
       const int t = i / (int)K, k = i % (int)K;
-      sPhi[t * S::kK + k] = t < Qc ? ldv<T>(p.theta, ((b * L + t0 + t) * H + h) * K + k) : 0.f;
+      sPhi[t * S::kK + k] = t < Qc ? ldv<T>(p.theta, ((b * L + t0 + t) * H + h) * Kt + k0 + k) : 0.f;
     }
     __syncthreads();
     // ---- 2. cumulative angles; decay products d(t, s) ------------------------
@@ -168,18 +175,25 @@ __global__ void __launch_bounds__(kThreads, 1) m3_fwd_kernel(const M3Params p) {
       if (t < Qc) {
         float y = sY[i] + sWc[t] * sXprev[pp] + Dh * sX[i];
         const int64_t j = ((b * L + t0 + t) * H + h) * P + pp;
+        if (slab != kSlabWhole) {  // the sums over the states cross the slabs
+          if (slab != kSlabFirst) y = p.tok_y[j] + y;
+          if (!finish) {
+            p.tok_y[j] = y;
+            continue;
+          }
+        }
         if (p.z) y *= silu(ldv<T>(p.z, j));
         static_cast<T *>(p.out)[j] = from_f32<T>(y);
       }
     }
     if (p.saved) {
-      float *dst = p.saved + ((b * H + h) * n_chunks + ch) * P * N;
+      float *dst = p.saved + ((b * H + h) * n_chunks + ch) * P * ldN + n0;
       for (int i = tid; i < P * N; i += kThreads) {
         const int pp = i / N, n = i % N;
-        dst[i] = sST[n * P + pp];
+        dst[pp * ldN + n] = sST[n * P + pp];
       }
       // the cumulative angles at the chunk start, after all states
-      float *ang = p.saved + p.B * H * n_chunks * P * N + ((b * H + h) * n_chunks + ch) * S::kK;
+      float *ang = p.saved + p.B * H * n_chunks * P * ldN + ((b * H + h) * n_chunks + ch) * (ldN / 2) + k0;
       for (int i = tid; i < S::kK; i += kThreads) ang[i] = sPhiPrev[i];
     }
     __syncthreads();
@@ -202,30 +216,31 @@ __global__ void __launch_bounds__(kThreads, 1) m3_fwd_kernel(const M3Params p) {
   }
   __syncthreads();
   if (p.final_state) {
-    float *dst = p.final_state + (b * H + h) * P * N;
+    float *dst = p.final_state + (b * H + h) * P * ldN + n0;
     for (int i = tid; i < P * N; i += kThreads) {
       const int pp = i / N, n = i % N;
-      dst[i] = sST[n * P + pp];
+      dst[pp * ldN + n] = sST[n * P + pp];
     }
   }
 }
 
-template <typename T, int P, int N>
+template <typename T, int P, int N, bool kSlab>
 cudaError_t launch_t(const M3Params &p, cudaStream_t s) {
   const size_t smem = sizeof(float) * (size_t)FwdSmem<P, N>::total;
-  cudaError_t e = cudaFuncSetAttribute(m3_fwd_kernel<T, P, N>,
+  cudaError_t e = cudaFuncSetAttribute(m3_fwd_kernel<T, P, N, kSlab>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  m3_fwd_kernel<T, P, N><<<dim3((unsigned)p.H, (unsigned)p.B), kThreads, smem, s>>>(p);
+  m3_fwd_kernel<T, P, N, kSlab><<<dim3((unsigned)p.H, (unsigned)p.B), kThreads, smem, s>>>(p);
   return cudaGetLastError();
 }
 
 template <typename T, int P>
 cudaError_t launch_n(const M3Params &p, cudaStream_t s) {
+  if (p.slab != kSlabWhole) return launch_t<T, P, kM3Slab, true>(p, s);
   switch (p.N) {
-    case 16: return launch_t<T, P, 16>(p, s);
-    case 32: return launch_t<T, P, 32>(p, s);
-    default: return launch_t<T, P, 64>(p, s);
+    case 16: return launch_t<T, P, 16, false>(p, s);
+    case 32: return launch_t<T, P, 32, false>(p, s);
+    default: return launch_t<T, P, 64, false>(p, s);
   }
 }
 
@@ -240,18 +255,35 @@ cudaError_t launch_p(const M3Params &p, cudaStream_t s) {
 
 }  // namespace
 
+// d_state 16, 32 or 64 in one launch; 128, 192 or 256 as slabs of 64 states
 bool m3_supported(int64_t P, int64_t N) {
-  return (P == 16 || P == 32 || P == 64) && (N == 16 || N == 32 || N == 64);
+  return (P == 16 || P == 32 || P == 64) &&
+         (N == 16 || N == 32 || N == 64 || (N > kM3Slab && N <= 4 * kM3Slab && N % kM3Slab == 0));
 }
 
 // bf16 io runs the tcgen05 kernel (m3_fwd_umma.cu); f32 and f16 io this one,
 // whose contractions are f32 on the CUDA cores.
-cudaError_t launch_m3_fwd(const M3Params &p, cudaStream_t s) {
-  switch (p.io) {
-    case 1: return launch_m3_fwd_umma(p, s);
-    case 2: return launch_p<f16>(p, s);
-    default: return launch_p<float>(p, s);
+// The whole d_state in one launch, or slabs of kM3Slab states in ascending
+// order, the output sums carried in tok_y.
+cudaError_t launch_m3_fwd(const M3Params &p0, cudaStream_t s) {
+  const int64_t n_tot = p0.N;
+  const int64_t slabs = (n_tot + kM3Slab - 1) / kM3Slab;
+  for (int64_t k = 0; k < slabs; ++k) {
+    M3Params p = p0;
+    p.ldN = n_tot;
+    p.n0 = k * kM3Slab;
+    p.N = n_tot - p.n0 < kM3Slab ? n_tot - p.n0 : kM3Slab;
+    p.slab = slabs == 1 ? kSlabWhole
+                        : (k == 0 ? kSlabFirst : (k == slabs - 1 ? kSlabLast : kSlabMiddle));
+    cudaError_t e;
+    switch (p.io) {
+      case 1: e = launch_m3_fwd_umma(p, s); break;
+      case 2: e = launch_p<f16>(p, s); break;
+      default: e = launch_p<float>(p, s); break;
+    }
+    if (e != cudaSuccess) return e;
   }
+  return cudaSuccess;
 }
 
 }  // namespace msc

@@ -67,7 +67,7 @@ struct UmFwdSmem {
 };
 
 // cp.async the raw x, B, C rows of the chunk at t0 (rows past L zero-filled)
-template <int P, int N>
+template <int P, int N, bool kSlab>
 __device__ __forceinline__ void um_issue_raw(const M3Params &p, unsigned char *sm, int64_t b,
                                              int64_t h, int64_t g, int64_t t0) {
   using S = UmFwdSmem<P, N>;
@@ -88,7 +88,9 @@ __device__ __forceinline__ void um_issue_raw(const M3Params &p, unsigned char *s
       const bool in = t0 + t < L;
       const bf16 *src = k == 0 ? Bm : Cm;
       cp_async16(sm + (k == 0 ? S::rB : S::rC) + t * S::kRS + pc * 16,
-                 in ? src + ((b * L + t0 + t) * G + g) * N + pc * 8 : src, in ? 16 : 0);
+                 in ? src + ((b * L + t0 + t) * G + g) * (kSlab ? p.ldN : N) + (kSlab ? p.n0 : 0) + pc * 8
+                    : src,
+                 in ? 16 : 0);
     }
   }
   cp_async_commit();
@@ -142,7 +144,9 @@ __device__ __forceinline__ void issue_product(uint32_t tmem, int col, uint32_t a
   }
 }
 
-template <int P, int N>
+// kSlab: one slab of a wider d_state (runtime row length and offsets);
+// otherwise the whole d_state with compile-time strides
+template <int P, int N, bool kSlab>
 __global__ void __launch_bounds__(kThreads, 2) m3_fwd_umma_kernel(const M3Params p) {
   using S = UmFwdSmem<P, N>;
   constexpr int kK = N / 2;
@@ -166,9 +170,15 @@ __global__ void __launch_bounds__(kThreads, 2) m3_fwd_umma_kernel(const M3Params
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t h = blockIdx.x, b = blockIdx.y;
   const int64_t L = p.L, H = p.H, G = p.G;
-  const int K = (int)p.K;
+  // this slab's states n0 .. n0 + N - 1 of ldN, and its angle pairs k0 ..
+  // k0 + K - 1 of the Kt
+  const int64_t ldN = kSlab ? p.ldN : N, n0 = kSlab ? p.n0 : 0;
+  const int Kt = (int)p.K, k0 = (int)(n0 / 2);
+  const int K = Kt - k0 < 0 ? 0 : (Kt - k0 > kK ? kK : Kt - k0);
+  const int slab = kSlab ? p.slab : kSlabWhole;
+  const bool finish = slab == kSlabWhole || slab == kSlabLast;
   const int64_t g = h / (H / G);
-  const float Dh = p.Dp ? p.Dp[h] : 0.f;
+  const float Dh = (p.Dp && finish) ? p.Dp[h] : 0.f;  // the D x skip joins once
   const int64_t nc = (L + kQ - 1) / kQ;
   const bf16 *x_g = static_cast<const bf16 *>(p.x);
   const bf16 *al_g = static_cast<const bf16 *>(p.alpha);
@@ -202,12 +212,12 @@ __global__ void __launch_bounds__(kThreads, 2) m3_fwd_umma_kernel(const M3Params
   // the state: rows ra (sreg[4 i], [4 i + 1]) and rb (sreg[4 i + 2], [4 i + 3]),
   // columns cb * kK + 8 i + c2 + 0, 1
   float sreg[kK / 2];
-  const float *h0 = p.h0 ? p.h0 + (b * H + h) * P * N : nullptr;
+  const float *h0 = p.h0 ? p.h0 + (b * H + h) * P * ldN + n0 : nullptr;  // rows of ldN
 #pragma unroll
   for (int i = 0; i < kSR; ++i) {
     const int n = cb * kK + 8 * i + c2;
-    const float2 va = (srow && h0) ? *reinterpret_cast<const float2 *>(h0 + ra * N + n) : make_float2(0.f, 0.f);
-    const float2 vb = (srow && h0) ? *reinterpret_cast<const float2 *>(h0 + rb * N + n) : make_float2(0.f, 0.f);
+    const float2 va = (srow && h0) ? *reinterpret_cast<const float2 *>(h0 + ra * ldN + n) : make_float2(0.f, 0.f);
+    const float2 vb = (srow && h0) ? *reinterpret_cast<const float2 *>(h0 + rb * ldN + n) : make_float2(0.f, 0.f);
     sreg[4 * i] = va.x; sreg[4 * i + 1] = va.y;
     sreg[4 * i + 2] = vb.x; sreg[4 * i + 3] = vb.y;
   }
@@ -219,12 +229,12 @@ __global__ void __launch_bounds__(kThreads, 2) m3_fwd_umma_kernel(const M3Params
       put3x2(sm + S::sp, S::kSp, koff(rb, n, N), sreg[4 * i + 2], sreg[4 * i + 3]);
     }
   };
-  auto store_state = [&](float *dst) {  // dst: this (b, h)'s P x N block
+  auto store_state = [&](float *dst) {  // dst: this (b, h, slab)'s P x N block, rows of ldN
 #pragma unroll
     for (int i = 0; i < kSR; ++i) {
       const int n = cb * kK + 8 * i + c2;
-      *reinterpret_cast<float2 *>(dst + ra * N + n) = make_float2(sreg[4 * i], sreg[4 * i + 1]);
-      *reinterpret_cast<float2 *>(dst + rb * N + n) = make_float2(sreg[4 * i + 2], sreg[4 * i + 3]);
+      *reinterpret_cast<float2 *>(dst + ra * ldN + n) = make_float2(sreg[4 * i], sreg[4 * i + 1]);
+      *reinterpret_cast<float2 *>(dst + rb * ldN + n) = make_float2(sreg[4 * i + 2], sreg[4 * i + 3]);
     }
   };
   if (srow) put_state();
@@ -242,7 +252,7 @@ __global__ void __launch_bounds__(kThreads, 2) m3_fwd_umma_kernel(const M3Params
 #pragma unroll
     for (int m = 0; m < 8; ++m) {
       const int64_t t = t0 + 8 * m + ri;
-      thv[m] = (ka < K && t < L) ? __bfloat162float(th_g[((b * L + t) * H + h) * K + ka]) : 0.f;
+      thv[m] = (ka < K && t < L) ? __bfloat162float(th_g[((b * L + t) * H + h) * Kt + k0 + ka]) : 0.f;
     }
     pa0 = pa1 = 1.f;
     pb0 = pb1 = pg0 = pg1 = 0.f;
@@ -262,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 2) m3_fwd_umma_kernel(const M3Params
       }
     }
   };
-  um_issue_raw<P, N>(p, sm, b, h, g, 0);
+  um_issue_raw<P, N, kSlab>(p, sm, b, h, g, 0);
   load_small(0);
   umma::fence_before();
   __syncthreads();
@@ -283,9 +293,9 @@ __global__ void __launch_bounds__(kThreads, 2) m3_fwd_umma_kernel(const M3Params
 
     // ---- 1. state and angles entering the chunk; X^T; per-step vectors ----------
     if (p.saved) {
-      if (srow) store_state(p.saved + ((b * H + h) * nc + ch) * P * N);
+      if (srow) store_state(p.saved + ((b * H + h) * nc + ch) * P * ldN + n0);
       if (sp == 0 && ri == 0)
-        p.saved[p.B * H * nc * P * N + ((b * H + h) * nc + ch) * kK + ka] = phi_c;
+        p.saved[p.B * H * nc * P * ldN + ((b * H + h) * nc + ch) * (ldN / 2) + k0 + ka] = phi_c;
     }
     for (int u = tid; u < P * 8; u += kThreads) {
       const int pp = u % P, t8 = u / P;
@@ -385,7 +395,7 @@ __global__ void __launch_bounds__(kThreads, 2) m3_fwd_umma_kernel(const M3Params
       umma::commit(mbar);
     }
     if (ch + 1 < nc) {
-      um_issue_raw<P, N>(p, sm, b, h, g, t0 + kQ);
+      um_issue_raw<P, N, kSlab>(p, sm, b, h, g, t0 + kQ);
       load_small(t0 + kQ);
     }
     // x and z of this thread's outputs (rows ra, rb)
@@ -465,13 +475,26 @@ __global__ void __launch_bounds__(kThreads, 2) m3_fwd_umma_kernel(const M3Params
             unpack_bf16x2(xo[2 * i + e], xf0, xf1);
             float o0 = fmaf(dlt, y1[4 * i + 2 * e], y2[4 * i + 2 * e]) + wct * xp_c[p0] + Dh * xf0;
             float o1 = fmaf(dlt, y1[4 * i + 2 * e + 1], y2[4 * i + 2 * e + 1]) + wct * xp_c[p0 + 1] + Dh * xf1;
+            const int64_t oi = ((b * L + t0 + t) * H + h) * P + p0;
+            if (slab != kSlabWhole) {  // the sums over the states cross the slabs
+              float2 *ty = reinterpret_cast<float2 *>(p.tok_y + oi);
+              if (slab != kSlabFirst) {
+                const float2 prev = *ty;
+                o0 = prev.x + o0;
+                o1 = prev.y + o1;
+              }
+              if (!finish) {
+                *ty = make_float2(o0, o1);
+                continue;
+              }
+            }
             if (z_g) {
               float zf0, zf1;
               unpack_bf16x2(zo[2 * i + e], zf0, zf1);
               o0 *= silu(zf0);
               o1 *= silu(zf1);
             }
-            *reinterpret_cast<uint32_t *>(out_g + ((b * L + t0 + t) * H + h) * P + p0) = pack_bf16x2(o0, o1);
+            *reinterpret_cast<uint32_t *>(out_g + oi) = pack_bf16x2(o0, o1);
           }
         }
       }
@@ -509,7 +532,7 @@ __global__ void __launch_bounds__(kThreads, 2) m3_fwd_umma_kernel(const M3Params
 #pragma unroll
       for (int j = 0; j < kK / 2; ++j) sreg[j] = __int_as_float(0x7fc00000);
     }
-    store_state(p.final_state + (b * H + h) * P * N);
+    store_state(p.final_state + (b * H + h) * P * ldN + n0);
   }
   if (failed) {  // a tensor-core round never completed: the outputs of this (b, h) are NaN
     const bf16 qnan = __ushort_as_bfloat16((unsigned short)0x7fc0);
@@ -524,24 +547,25 @@ __global__ void __launch_bounds__(kThreads, 2) m3_fwd_umma_kernel(const M3Params
   }
 }
 
-template <int P, int N>
+template <int P, int N, bool kSlab>
 cudaError_t launch_um(const M3Params &p, cudaStream_t s) {
   // at least 80 KB of shared memory per CTA, so that no more than two CTAs
   // (2 x 256 TMEM columns) share an SM
   const size_t smem = UmFwdSmem<P, N>::total > 80 * 1024 ? (size_t)UmFwdSmem<P, N>::total : 80 * 1024;
-  cudaError_t e = cudaFuncSetAttribute(m3_fwd_umma_kernel<P, N>,
+  cudaError_t e = cudaFuncSetAttribute(m3_fwd_umma_kernel<P, N, kSlab>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  m3_fwd_umma_kernel<P, N><<<dim3((unsigned)p.H, (unsigned)p.B), kThreads, smem, s>>>(p);
+  m3_fwd_umma_kernel<P, N, kSlab><<<dim3((unsigned)p.H, (unsigned)p.B), kThreads, smem, s>>>(p);
   return cudaGetLastError();
 }
 
 template <int P>
 cudaError_t launch_um_n(const M3Params &p, cudaStream_t s) {
+  if (p.slab != kSlabWhole) return launch_um<P, kM3Slab, true>(p, s);
   switch (p.N) {
-    case 16: return launch_um<P, 16>(p, s);
-    case 32: return launch_um<P, 32>(p, s);
-    default: return launch_um<P, 64>(p, s);
+    case 16: return launch_um<P, 16, false>(p, s);
+    case 32: return launch_um<P, 32, false>(p, s);
+    default: return launch_um<P, 64, false>(p, s);
   }
 }
 

@@ -16,7 +16,9 @@
 // threads of a row read and write one contiguous run per instruction).  A
 // CTA of 256 threads serves 256 / (P N / 16) heads.  Per head, the first N/2
 // threads rotate one pair of B and C each into shared memory; y sums a row's
-// partials over its N / 16 threads with shuffles in a fixed order.
+// partials over its N / 16 threads with shuffles in a fixed order.  Wider
+// states (128, 192, 256) are walked in slabs of 64 states with the 64-state
+// layout, y carried across the slabs in registers.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -32,10 +34,12 @@ __device__ __forceinline__ float ldf(const void *base, int64_t i) {
 
 template <typename T, int P, int N>
 __global__ void __launch_bounds__(kSUThreads) m3_state_update_kernel(const M3SUParams p) {
-  constexpr int kTPR = N / 16;           // threads per row of S
-  constexpr int kTPH = P * kTPR;         // threads per head
+  constexpr int kSN = N < 64 ? N : 64;     // states per slab (wider states: slabs of 64 in turn)
+  constexpr int kNS = N / kSN;             // slabs
+  constexpr int kTPR = kSN / 16;           // threads per row of a slab
+  constexpr int kTPH = P * kTPR;           // threads per head
   constexpr int kHPC = kSUThreads / kTPH;  // heads per CTA
-  constexpr int kPer = 3 * N + P;        // shared floats per head: Bt, Ct, bt_prev, x_prev
+  constexpr int kPer = 3 * kSN + P;        // shared floats per head: Bt, Ct, bt_prev (a slab), x_prev
   __shared__ __align__(16) float sm[kHPC * kPer];
 
   const int tid = threadIdx.x;
@@ -46,71 +50,75 @@ __global__ void __launch_bounds__(kSUThreads) m3_state_update_kernel(const M3SUP
   const int64_t b = bh / p.H, h = bh % p.H;
   const int64_t g = h / (p.H / p.G);
   const int K = (int)p.K;
-  float *sBt = sm + hl * kPer, *sCt = sBt + N, *sBp = sCt + N, *sXp = sBp + N;
+  float *sBt = sm + hl * kPer, *sCt = sBt + kSN, *sBp = sCt + kSN, *sXp = sBp + kSN;
   const int row = j / kTPR, q = j % kTPR;
   float4 *srow = reinterpret_cast<float4 *>(p.state + (bh * P + row) * N);
 
-  // this thread's state entries and scalars, in flight while the head's
-  // rotation runs
-  float4 s[4];
   float al = 0.f, be = 0.f, ga = 0.f, xv = 0.f;
   if (live) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) s[i] = srow[i * kTPR + q];
     al = ldf<T>(p.alpha, bh);
     be = ldf<T>(p.beta, bh);
     ga = ldf<T>(p.gamma, bh);
     xv = ldf<T>(p.x, bh * P + row);
-  }
-
-  // ---- the step's rotated B and C; the carried x_prev and bt_prev ----------
-  if (live) {
-    if (j < N / 2) {
-      const int64_t o = (b * p.G + g) * N + 2 * j;
-      float b0 = ldf<T>(p.Bm, o), b1 = ldf<T>(p.Bm, o + 1);
-      float c0 = ldf<T>(p.Cm, o), c1 = ldf<T>(p.Cm, o + 1);
-      if (j < K) {
-        const float phi = p.phi[bh * K + j] + ldf<T>(p.theta, bh * K + j);
-        p.phi[bh * K + j] = phi;
-        float sn, cs;
-        sincosf(phi, &sn, &cs);
-        const float rb0 = cs * b0 - sn * b1, rb1 = sn * b0 + cs * b1;
-        const float rc0 = cs * c0 - sn * c1, rc1 = sn * c0 + cs * c1;
-        b0 = rb0; b1 = rb1; c0 = rc0; c1 = rc1;
-      }
-      sBt[2 * j] = b0; sBt[2 * j + 1] = b1;
-      sCt[2 * j] = c0; sCt[2 * j + 1] = c1;
-    }
-    for (int i = j; i < N; i += kTPH) sBp[i] = p.bt_prev[bh * N + i];
     for (int i = j; i < P; i += kTPH) sXp[i] = p.x_prev[bh * P + i];
   }
-  __syncthreads();
-  if (!live) return;
-  // the carried key of the next step (every read of the old one is done)
-  for (int i = j; i < N; i += kTPH) p.bt_prev[bh * N + i] = sBt[i];
-  for (int i = j; i < P; i += kTPH) p.x_prev[bh * P + i] = ldf<T>(p.x, bh * P + i);
-
-  // ---- the state rows ---------------------------------------------------------
-  const float bxq = be * sXp[row], gx = ga * xv;
-  const float4 *vBt = reinterpret_cast<const float4 *>(sBt);
-  const float4 *vCt = reinterpret_cast<const float4 *>(sCt);
-  const float4 *vBp = reinterpret_cast<const float4 *>(sBp);
   float y = 0.f;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int v = i * kTPR + q;
-    const float4 bt = vBt[v], ct = vCt[v], bp = vBp[v];
-    s[i].x = fmaf(al, s[i].x, fmaf(bxq, bp.x, gx * bt.x));
-    s[i].y = fmaf(al, s[i].y, fmaf(bxq, bp.y, gx * bt.y));
-    s[i].z = fmaf(al, s[i].z, fmaf(bxq, bp.z, gx * bt.z));
-    s[i].w = fmaf(al, s[i].w, fmaf(bxq, bp.w, gx * bt.w));
-    y = fmaf(ct.x, s[i].x, y);
-    y = fmaf(ct.y, s[i].y, y);
-    y = fmaf(ct.z, s[i].z, y);
-    y = fmaf(ct.w, s[i].w, y);
-  }
+  for (int sl = 0; sl < kNS; ++sl) {
+    const int n0 = sl * kSN;
+    // this thread's state entries of the slab and the slab's rotated B and
+    // C; the carried bt_prev of the slab
+    float4 st[4];
+    if (live) {
 #pragma unroll
-  for (int i = 0; i < 4; ++i) srow[i * kTPR + q] = s[i];
+      for (int i = 0; i < 4; ++i) st[i] = srow[n0 / 4 + i * kTPR + q];
+      if (j < kSN / 2) {
+        const int ka = n0 / 2 + j;  // global angle pair
+        const int64_t o = (b * p.G + g) * N + n0 + 2 * j;
+        float b0 = ldf<T>(p.Bm, o), b1 = ldf<T>(p.Bm, o + 1);
+        float c0 = ldf<T>(p.Cm, o), c1 = ldf<T>(p.Cm, o + 1);
+        if (ka < K) {
+          const float phi = p.phi[bh * K + ka] + ldf<T>(p.theta, bh * K + ka);
+          p.phi[bh * K + ka] = phi;
+          float sn, cs;
+          sincosf(phi, &sn, &cs);
+          const float rb0 = cs * b0 - sn * b1, rb1 = sn * b0 + cs * b1;
+          const float rc0 = cs * c0 - sn * c1, rc1 = sn * c0 + cs * c1;
+          b0 = rb0; b1 = rb1; c0 = rc0; c1 = rc1;
+        }
+        sBt[2 * j] = b0; sBt[2 * j + 1] = b1;
+        sCt[2 * j] = c0; sCt[2 * j + 1] = c1;
+      }
+      for (int i = j; i < kSN; i += kTPH) sBp[i] = p.bt_prev[bh * N + n0 + i];
+    }
+    __syncthreads();
+    if (live) {
+      // the carried key of the next step (every read of the old one is done)
+      for (int i = j; i < kSN; i += kTPH) p.bt_prev[bh * N + n0 + i] = sBt[i];
+      const float bxq = be * sXp[row], gx = ga * xv;
+      const float4 *vBt = reinterpret_cast<const float4 *>(sBt);
+      const float4 *vCt = reinterpret_cast<const float4 *>(sCt);
+      const float4 *vBp = reinterpret_cast<const float4 *>(sBp);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int v = i * kTPR + q;
+        const float4 bt = vBt[v], ct = vCt[v], bp = vBp[v];
+        st[i].x = fmaf(al, st[i].x, fmaf(bxq, bp.x, gx * bt.x));
+        st[i].y = fmaf(al, st[i].y, fmaf(bxq, bp.y, gx * bt.y));
+        st[i].z = fmaf(al, st[i].z, fmaf(bxq, bp.z, gx * bt.z));
+        st[i].w = fmaf(al, st[i].w, fmaf(bxq, bp.w, gx * bt.w));
+        y = fmaf(ct.x, st[i].x, y);
+        y = fmaf(ct.y, st[i].y, y);
+        y = fmaf(ct.z, st[i].z, y);
+        y = fmaf(ct.w, st[i].w, y);
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) srow[n0 / 4 + i * kTPR + q] = st[i];
+    }
+    if (kNS > 1) __syncthreads();  // the slab's tables are free for the next slab
+  }
+  if (!live) return;
+  for (int i = j; i < P; i += kTPH) p.x_prev[bh * P + i] = ldf<T>(p.x, bh * P + i);
   // (kTPR > 1 only for N >= 32, where a warp holds threads of one head only,
   // so no lane of a shuffling warp has returned above)
 #pragma unroll
@@ -124,7 +132,7 @@ __global__ void __launch_bounds__(kSUThreads) m3_state_update_kernel(const M3SUP
 
 template <typename T, int P, int N>
 cudaError_t launch_pn(const M3SUParams &p, cudaStream_t s) {
-  constexpr int kHPC = kSUThreads / (P * N / 16);
+  constexpr int kHPC = kSUThreads / (P * (N < 64 ? N : 64) / 16);
   const int64_t blocks = (p.B * p.H + kHPC - 1) / kHPC;
   m3_state_update_kernel<T, P, N><<<(unsigned)blocks, kSUThreads, 0, s>>>(p);
   return cudaGetLastError();
@@ -135,7 +143,10 @@ cudaError_t launch_p(const M3SUParams &p, cudaStream_t s) {
   switch (p.N) {
     case 16: return launch_pn<T, P, 16>(p, s);
     case 32: return launch_pn<T, P, 32>(p, s);
-    default: return launch_pn<T, P, 64>(p, s);
+    case 64: return launch_pn<T, P, 64>(p, s);
+    case 128: return launch_pn<T, P, 128>(p, s);
+    case 192: return launch_pn<T, P, 192>(p, s);
+    default: return launch_pn<T, P, 256>(p, s);
   }
 }
 

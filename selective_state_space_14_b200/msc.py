@@ -67,7 +67,8 @@ class M3FwdArgs(ctypes.Structure):
                 ("nheads", _i64), ("headdim", _i64), ("dstate", _i64), ("ngroups", _i64),
                 ("nangles", _i64), ("x", _vp), ("z", _vp), ("Bm", _vp), ("Cm", _vp),
                 ("alpha", _vp), ("beta", _vp), ("gamma", _vp), ("theta", _vp), ("D", _vp),
-                ("h0", _vp), ("out", _vp), ("final_state", _vp), ("saved_states", _vp)]
+                ("h0", _vp), ("out", _vp), ("final_state", _vp), ("saved_states", _vp),
+                ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t)]
 
 
 class M3BwdArgs(ctypes.Structure):
@@ -91,7 +92,7 @@ class M3SuArgs(ctypes.Structure):
 EXPORTS = ["msc_last_error", "msc_version", "msc_selective_scan_saved_states_bytes",
            "msc_selective_scan_fwd_workspace_bytes", "msc_selective_scan_fwd", "msc_selective_scan_bwd_workspace_bytes",
            "msc_selective_scan_bwd", "msc_selective_scan_bwd_static", "msc_ssm_state_update",
-           "msc_mamba3_siso_saved_states_bytes",
+           "msc_mamba3_siso_saved_states_bytes", "msc_mamba3_siso_scan_fwd_workspace_bytes",
            "msc_mamba3_siso_scan_fwd", "msc_mamba3_siso_scan_bwd_workspace_bytes",
            "msc_mamba3_siso_scan_bwd", "msc_mamba3_siso_state_update"]
 
@@ -128,6 +129,8 @@ def lib() -> ctypes.CDLL:
         L.msc_selective_scan_bwd_workspace_bytes.restype = ctypes.c_size_t
         L.msc_mamba3_siso_saved_states_bytes.argtypes = [_i64] * 5
         L.msc_mamba3_siso_saved_states_bytes.restype = ctypes.c_size_t
+        L.msc_mamba3_siso_scan_fwd_workspace_bytes.argtypes = [_i64] * 5
+        L.msc_mamba3_siso_scan_fwd_workspace_bytes.restype = ctypes.c_size_t
         L.msc_mamba3_siso_scan_bwd_workspace_bytes.argtypes = [_i64] * 7
         L.msc_mamba3_siso_scan_bwd_workspace_bytes.restype = ctypes.c_size_t
         _lib = L
@@ -316,9 +319,15 @@ def msc_mamba3_siso_scan_bwd_workspace_bytes(batch, seqlen, nheads, headdim, dst
                                                                  dstate, ngroups, nangles))
 
 
+def msc_mamba3_siso_scan_fwd_workspace_bytes(batch, seqlen, nheads, headdim, dstate) -> int:
+    return int(lib().msc_mamba3_siso_scan_fwd_workspace_bytes(batch, seqlen, nheads, headdim,
+                                                                 dstate))
+
+
 def msc_mamba3_siso_scan_fwd(x, B, C, alpha, beta, gamma, theta, D=None, z=None, h0=None,
                              out=None, final_state=None, saved_states=None,
-                             want_final_state=True, want_saved_states=True, stream=None):
+                             want_final_state=True, want_saved_states=True, workspace=None,
+                             stream=None):
     """Mamba-3 SISO forward.  x, z [B, L, H, P]; B, C [B, L, G, N]; alpha, beta, gamma
     [B, L, H]; theta [B, L, H, K].  Returns (out, final_state, saved_states)."""
     Bsz, L, H, P = x.shape
@@ -332,9 +341,13 @@ def msc_mamba3_siso_scan_fwd(x, B, C, alpha, beta, gamma, theta, D=None, z=None,
     if saved_states is None and want_saved_states:
         nb = msc_mamba3_siso_saved_states_bytes(Bsz, L, H, P, N)
         saved_states = torch.empty(max(nb // 4, 4), device=dev, dtype=torch.float32)
+    need = msc_mamba3_siso_scan_fwd_workspace_bytes(Bsz, L, H, P, N)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, device=dev, dtype=torch.uint8)
     a = M3FwdArgs(ctypes.sizeof(M3FwdArgs), _io(x), Bsz, L, H, P, N, G, K, _ptr(x), _ptr(z),
                   _ptr(B), _ptr(C), _ptr(alpha), _ptr(beta), _ptr(gamma), _ptr(theta), _ptr(D),
-                  _ptr(h0), _ptr(out), _ptr(final_state), _ptr(saved_states))
+                  _ptr(h0), _ptr(out), _ptr(final_state), _ptr(saved_states), _ptr(workspace),
+                  workspace.numel() * workspace.element_size() if workspace is not None else 0)
     _check(lib().msc_mamba3_siso_scan_fwd(ctypes.byref(a), _stream(stream)))
     return out, final_state, saved_states
 

@@ -135,6 +135,22 @@ def test_m3_rejects_unsupported_headdim():
     assert st == UNSUPPORTED and "headdim" in _err()
 
 
+def test_m3_wide_state_needs_a_workspace():
+    """d_state 128 runs as slabs; the forward then needs its workspace (the call
+    stops at that check, before any launch)."""
+    assert msc.msc_mamba3_siso_scan_fwd_workspace_bytes(2, 100, 3, 64, 64) == 0
+    assert msc.msc_mamba3_siso_scan_fwd_workspace_bytes(2, 100, 3, 64, 128) == 4 * 2 * 100 * 3 * 64
+    a = msc.M3FwdArgs()
+    a.struct_size = ctypes.sizeof(msc.M3FwdArgs)
+    a.io_dtype, a.batch, a.seqlen, a.nheads, a.headdim, a.dstate, a.ngroups, a.nangles = (
+        msc.MSC_BF16, 1, 64, 2, 64, 128, 1, 8)
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: the workspace check fails first
+    for f in ("x", "Bm", "Cm", "alpha", "beta", "gamma", "theta", "out"):
+        setattr(a, f, fake)
+    assert msc.lib().msc_mamba3_siso_scan_fwd(ctypes.byref(a), None) == WORKSPACE
+    assert "workspace" in _err()
+
+
 def test_m3_rejects_too_many_angles():
     a = msc.M3FwdArgs()
     a.struct_size = ctypes.sizeof(msc.M3FwdArgs)
@@ -160,7 +176,8 @@ def _m3su_args(**kw):
 
 @pytest.mark.parametrize("field,value,status,word", [
     ("headdim", 48, UNSUPPORTED, "headdim"),
-    ("dstate", 128, UNSUPPORTED, "dstate"),
+    ("dstate", 96, UNSUPPORTED, "dstate"),
+    ("dstate", 320, UNSUPPORTED, "dstate"),
     ("nangles", 33, INVALID, "nangles"),
     ("ngroups", 3, INVALID, "ngroups"),
     ("nheads", 0, INVALID, "nheads"),

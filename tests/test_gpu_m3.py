@@ -51,6 +51,13 @@ FWD_CASES = [
     (1, 640, 2, 64, 64, 1, 32, "bf16", True, True, True),
     (2, 200, 4, 64, 64, 2, 32, "f16", True, True, True),
     (1, 65, 3, 16, 32, 3, 16, "f16", False, True, True),
+    # d_state above 64: slabs of 64 states (angle pairs split across the slabs,
+    # a slab without angles, a slab with a few)
+    (1, 130, 2, 64, 128, 1, 64, "bf16", True, True, True),
+    (1, 129, 2, 64, 128, 1, 10, "bf16", True, True, False),
+    (2, 70, 2, 32, 256, 2, 100, "f32", True, True, True),
+    (1, 65, 2, 16, 192, 1, 96, "bf16", False, False, True),
+    (1, 64, 2, 64, 128, 1, 10, "f16", True, True, True),
 ]
 
 
@@ -146,6 +153,10 @@ BWD_CASES = [
     (2, 300, 4, 64, 64, 1, 32, "bf16", True, True, False),
     (1, 130, 2, 32, 64, 1, 10, "f16", True, True, True),
     (2, 70, 2, 64, 64, 1, 32, "f16", True, False, True),
+    (1, 130, 2, 64, 128, 1, 64, "bf16", True, True, True),
+    (1, 70, 2, 32, 256, 1, 100, "f32", True, True, True),
+    (2, 65, 2, 16, 128, 2, 20, "f16", True, True, True),
+    (1, 100, 2, 64, 192, 1, 40, "bf16", False, True, False),
 ]
 
 
@@ -212,6 +223,9 @@ SU_CASES = [
     (2, 4, 32, 32, 4, 16, "bf16", True, True, True, 20),
     (3, 4, 64, 64, 1, 32, "f16", True, True, True, 12),
     (2, 6, 16, 32, 2, 8, "f16", False, True, True, 12),
+    (2, 3, 64, 128, 1, 64, "bf16", True, True, True, 10),
+    (2, 4, 16, 256, 2, 100, "f32", True, True, True, 8),
+    (3, 2, 32, 192, 1, 20, "bf16", False, True, True, 8),
 ]
 
 
