@@ -44,9 +44,11 @@ def _load():
         _lib.oracle_m3_fwd.argtypes = [i64] * 7 + [dp] * 12 + [ci]
         _lib.oracle_m3_bwd.argtypes = [i64] * 7 + [dp] * 21 + [ci]
         _lib.oracle_m3_state_update.argtypes = [i64] * 6 + [dp] * 14
+        _lib.oracle_conv1d_fwd.argtypes = [i64] * 4 + [dp] * 6
+        _lib.oracle_conv1d_bwd.argtypes = [i64] * 4 + [dp] * 9
         for f in (_lib.oracle_m1_fwd, _lib.oracle_m1_fwd_tree, _lib.oracle_m1_bwd,
                   _lib.oracle_ssm_state_update, _lib.oracle_m3_fwd, _lib.oracle_m3_bwd,
-                  _lib.oracle_m3_state_update):
+                  _lib.oracle_m3_state_update, _lib.oracle_conv1d_fwd, _lib.oracle_conv1d_bwd):
             f.restype = ctypes.c_int
         _lib.oracle_default_threads.restype = ctypes.c_int
     return _lib
@@ -194,6 +196,36 @@ def m3_state_update(state, x_prev, bt_prev, phi, x, B, C, alpha, beta, gamma, th
     _check(lib.oracle_m3_state_update(Bsz, H, P, N, G, K, *[a.ctypes.data for a in carried],
                                       *[k[1] for k in keep], po))
     return (*carried, out)
+
+
+# ---------------------------------------------------------------------------
+# causal conv1d (+ SiLU) ahead of the Mamba-1 scan
+# ---------------------------------------------------------------------------
+def conv1d_fwd(x, w, bias=None, xs0=None):
+    """x [B, D, L]; w [D, W]; bias [D]; xs0 [B, D, W-1].  Returns (u, xs_final)."""
+    lib = _load()
+    Bsz, Dm, L = x.shape
+    W = w.shape[1]
+    keep = [_in(v) for v in (x, w, bias, xs0)]
+    u, pu = _out((Bsz, Dm, L))
+    xs, px = _out((Bsz, Dm, max(W - 1, 0)))
+    _check(lib.oracle_conv1d_fwd(Bsz, Dm, L, W, *[k[1] for k in keep], pu, px))
+    return u, xs
+
+
+def conv1d_bwd(x, w, du, bias=None, xs0=None):
+    """Gradients of u = silu(conv(x)) for an upstream du [B, D, L].
+    Returns dx, dw, dbias, dxs0."""
+    lib = _load()
+    Bsz, Dm, L = x.shape
+    W = w.shape[1]
+    keep = [_in(v) for v in (x, w, bias, xs0, du)]
+    dx, p1 = _out((Bsz, Dm, L))
+    dw, p2 = _out((Dm, W))
+    db, p3 = _out((Dm,))
+    dxs, p4 = _out((Bsz, Dm, max(W - 1, 0)))
+    _check(lib.oracle_conv1d_bwd(Bsz, Dm, L, W, *[k[1] for k in keep], p1, p2, p3, p4))
+    return dict(dx=dx, dw=dw, dbias=db, dxs0=dxs)
 
 
 # ---------------------------------------------------------------------------

@@ -684,3 +684,101 @@ int oracle_m3_state_update(int64_t Bsz, int64_t H, int64_t P, int64_t N, int64_t
     }
     return 0;
 }
+
+/* ------------------------------------------------------------------ */
+/* Causal depthwise conv1d ahead of the Mamba-1 scan                   */
+/* ------------------------------------------------------------------ */
+/*
+ * The Mamba block's local convolution (the Mamba README, "Usage / Mamba
+ * Block": d_conv, "Local convolution width"; the causal-conv1d extra of its
+ * installation table; MambaState carries d_conv per layer, mamba-rs 0.7.0
+ * README, "Quick start (CPU)"): per channel c, a causal convolution of width
+ * W over time followed by SiLU, giving the scan's input u:
+ *   v[b,c,t] = bias[c] + sum_{k<W} w[c,k] x[b,c,t-(W-1)+k]
+ *   u[b,c,t] = silu(v[b,c,t])
+ * with x at t < 0 taken from the initial conv state xs0[b,c,0..W-2] (the W-1
+ * inputs before the sequence, oldest first) or 0.  The final conv state is
+ * the last W-1 inputs.  Layouts: x, u [B, D, L]; w [D, W]; bias [D];
+ * xs0, xs_final [B, D, W-1].
+ */
+static double conv_x(const double *x, const double *xs0, int64_t row, int64_t L, int64_t W,
+                     int64_t t) {
+    if (t >= 0) return x[row * L + t];
+    return xs0 ? xs0[row * (W - 1) + (W - 1) + t] : 0.0;  /* t in [-(W-1), -1] */
+}
+
+int oracle_conv1d_fwd(int64_t Bsz, int64_t D, int64_t L, int64_t W, const double *x,
+                      const double *w, const double *bias, const double *xs0, double *u,
+                      double *xs_final) {
+    if (W < 1) return -1;
+    for (int64_t row = 0; row < Bsz * D; ++row) {
+        const int64_t c = row % D;
+        for (int64_t t = 0; t < L; ++t) {
+            double v = bias ? bias[c] : 0.0;
+            for (int64_t k = 0; k < W; ++k)
+                v += w[c * W + k] * conv_x(x, xs0, row, L, W, t - (W - 1) + k);
+            u[row * L + t] = silu(v);
+        }
+        if (xs_final)
+            for (int64_t k = 0; k < W - 1; ++k)
+                xs_final[row * (W - 1) + k] = conv_x(x, xs0, row, L, W, L - (W - 1) + k);
+    }
+    return 0;
+}
+
+/*
+ * Backward of the above for an upstream gradient du [B, D, L]:
+ *   dv[t]     = du[t] silu'(v[t])
+ *   dx[t]     = sum_{k<W, t+(W-1)-k < L} w[c,k] dv[t+(W-1)-k]
+ *   dw[c,k]   = sum_{b,t} dv[t] x[t-(W-1)+k]      (x at t < 0 from xs0 or 0)
+ *   dbias[c]  = sum_{b,t} dv[t]
+ *   dxs0[b,c,j] = sum_{k, 0 <= tau+(W-1)-k < L} w[c,k] dv[tau+(W-1)-k]
+ *                 with tau = j-(W-1), the time of initial-state entry j
+ */
+int oracle_conv1d_bwd(int64_t Bsz, int64_t D, int64_t L, int64_t W, const double *x,
+                      const double *w, const double *bias, const double *xs0, const double *du,
+                      double *dx, double *dw, double *dbias, double *dxs0) {
+    if (W < 1) return -1;
+    double *dv = (double *)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
+    for (int64_t i = 0; i < D * W; ++i) dw[i] = 0.0;
+    if (dbias) for (int64_t c = 0; c < D; ++c) dbias[c] = 0.0;
+    for (int64_t row = 0; row < Bsz * D; ++row) {
+        const int64_t c = row % D;
+        for (int64_t t = 0; t < L; ++t) {
+            double v = bias ? bias[c] : 0.0;
+            for (int64_t k = 0; k < W; ++k)
+                v += w[c * W + k] * conv_x(x, xs0, row, L, W, t - (W - 1) + k);
+            dv[t] = du[row * L + t] * dsilu(v);
+        }
+        for (int64_t t = 0; t < L; ++t) {
+            double s = 0.0;
+            for (int64_t k = 0; k < W; ++k) {
+                const int64_t tt = t + (W - 1) - k;
+                if (tt < L) s += w[c * W + k] * dv[tt];
+            }
+            dx[row * L + t] = s;
+        }
+        for (int64_t k = 0; k < W; ++k) {
+            double s = 0.0;
+            for (int64_t t = 0; t < L; ++t) s += dv[t] * conv_x(x, xs0, row, L, W, t - (W - 1) + k);
+            dw[c * W + k] += s;
+        }
+        if (dbias) {
+            double s = 0.0;
+            for (int64_t t = 0; t < L; ++t) s += dv[t];
+            dbias[c] += s;
+        }
+        if (dxs0)
+            for (int64_t j = 0; j < W - 1; ++j) {  /* x at time tau = j - (W-1) */
+                const int64_t tau = j - (W - 1);
+                double s = 0.0;
+                for (int64_t k = 0; k < W; ++k) {
+                    const int64_t tt = tau + (W - 1) - k;
+                    if (tt >= 0 && tt < L) s += w[c * W + k] * dv[tt];
+                }
+                dxs0[row * (W - 1) + j] = s;
+            }
+    }
+    free(dv);
+    return 0;
+}

@@ -442,3 +442,53 @@ def test_m3_state_update_angle_offset_invariance():
             S, xp, bp, ph, a["x"][:, t], a["B"][:, t], a["C"][:, t], a["alpha"][:, t],
             a["beta"][:, t], a["gamma"][:, t], a["theta"][:, t], D=a["D"], z=a["z"][:, t])
         np.testing.assert_allclose(o, o1[:, t], rtol=1e-11, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# causal conv1d (+ SiLU) ahead of the Mamba-1 scan
+# ---------------------------------------------------------------------------
+def test_conv1d_identity_kernel():
+    """w = (0, ..., 0, 1), no bias: u = silu(x)."""
+    x = _rand(2, 3, 11)
+    w = np.zeros((3, 4))
+    w[:, -1] = 1.0
+    u, xs = oracle.conv1d_fwd(x, w)
+    np.testing.assert_allclose(u, _silu(x), rtol=1e-15)
+    np.testing.assert_array_equal(xs, x[:, :, -3:])
+
+
+def test_conv1d_equals_numpy_convolve():
+    """The pre-activation is the causal (zero-padded) convolution of each row
+    with its kernel: numpy.convolve of the row with the kernel taps reversed
+    (tap W-1 multiplies the current step), first L outputs, plus the bias."""
+    Bsz, Dm, L, W = 2, 3, 13, 4
+    x, w, bias = _rand(Bsz, Dm, L), _rand(Dm, W), _rand(Dm)
+    u, _ = oracle.conv1d_fwd(x, w, bias=bias)
+    for b in range(Bsz):
+        for c in range(Dm):
+            v = np.convolve(x[b, c], w[c, ::-1])[:L] + bias[c]
+            np.testing.assert_allclose(u[b, c], _silu(v), rtol=1e-13, atol=1e-15)
+
+
+def test_conv1d_continuation():
+    """Convolving [x1, x2] equals convolving x1, then x2 from x1's final conv state."""
+    Bsz, Dm, W = 1, 4, 4
+    x1, x2, w, bias = _rand(Bsz, Dm, 9), _rand(Bsz, Dm, 7), _rand(Dm, W), _rand(Dm)
+    u, xs = oracle.conv1d_fwd(np.concatenate([x1, x2], axis=2), w, bias=bias)
+    u1, xs1 = oracle.conv1d_fwd(x1, w, bias=bias)
+    u2, xs2 = oracle.conv1d_fwd(x2, w, bias=bias, xs0=xs1)
+    np.testing.assert_allclose(np.concatenate([u1, u2], axis=2), u, rtol=1e-14)
+    np.testing.assert_allclose(xs2, xs, rtol=1e-15)
+
+
+def test_conv1d_backward_finite_differences():
+    Bsz, Dm, L, W = 2, 2, 6, 3
+    x, w, bias, xs0 = _rand(Bsz, Dm, L), _rand(Dm, W), _rand(Dm), _rand(Bsz, Dm, W - 1)
+    du = _rand(Bsz, Dm, L)
+    g = oracle.conv1d_bwd(x, w, du, bias=bias, xs0=xs0)
+    args = dict(x=x, w=w, bias=bias, xs0=xs0)
+    loss = lambda a: float(np.sum(oracle.conv1d_fwd(a["x"], a["w"], bias=a["bias"],
+                                                    xs0=a["xs0"])[0] * du))
+    for key, gk in (("x", "dx"), ("w", "dw"), ("bias", "dbias"), ("xs0", "dxs0")):
+        fd = _fd(loss, args, key)
+        np.testing.assert_allclose(g[gk], fd, rtol=1e-6, atol=1e-8, err_msg=key)
