@@ -234,6 +234,65 @@ typedef struct {
 msc_status msc_ssm_state_update(const msc_su_args *args, msc_stream_t stream);
 
 /* ======================================================================
+ * Causal depthwise conv1d + SiLU ahead of the Mamba-1 scan
+ * ======================================================================
+ * The Mamba block's local convolution (the Mamba README, "Usage / Mamba
+ * Block": d_conv, the "local convolution width"; its causal-conv1d extra;
+ * MambaState carries d_conv per layer, mamba-rs 0.7.0 README, "Quick start
+ * (CPU)"), producing the scan's input u from x:
+ *   v[b,c,t] = bias[c] + sum_{k<W} w[c,k] x[b,c,t-(W-1)+k]
+ *   u[b,c,t] = silu(v[b,c,t])
+ * x before the sequence comes from conv_state_in[b,c,0..W-2] (the W-1 inputs
+ * before t = 0, oldest first) or is 0; conv_state_out receives the last W-1
+ * inputs (the state for the next call).
+ *
+ *   x, u                      io  [B, D, L]
+ *   w                         f32 [D, W]        1 <= W <= 4
+ *   bias                      f32 [D]           optional
+ *   conv_state_in/out         f32 [B, D, W-1]   optional
+ * Backward, for an upstream gradient du (io, [B, D, L]):
+ *   dv = du silu'(v);  dx[t] = sum_k w[c,k] dv[t+(W-1)-k]  (terms with t+(W-1)-k < L)
+ *   dw[c,k] = sum_{b,t} dv[t] x[t-(W-1)+k];  dbias[c] = sum_{b,t} dv[t]
+ *   dconv_state_in[b,c,j] = the gradient of conv_state_in[b,c,j]
+ * dw and dbias are summed over the batch in a fixed order (a workspace of
+ * msc_causal_conv1d_bwd_workspace_bytes() bytes holds the per-row partials).
+ */
+#define MSC_CONV_MAX_WIDTH 4
+typedef struct {
+  uint32_t struct_size;
+  int32_t io_dtype;
+  int64_t batch, dim, seqlen, width;
+  const void *x;
+  const float *w;
+  const float *bias;            /* optional */
+  const float *conv_state_in;   /* optional */
+  void *u;
+  float *conv_state_out;        /* optional */
+} msc_conv_fwd_args;
+
+msc_status msc_causal_conv1d_fwd(const msc_conv_fwd_args *args, msc_stream_t stream);
+
+typedef struct {
+  uint32_t struct_size;
+  int32_t io_dtype;
+  int64_t batch, dim, seqlen, width;
+  const void *x;
+  const float *w;
+  const float *bias;            /* optional */
+  const float *conv_state_in;   /* optional */
+  const void *du;
+  void *dx;
+  float *dw;
+  float *dbias;                 /* optional */
+  float *dconv_state_in;        /* optional */
+} msc_conv_bwd_args;
+
+size_t msc_causal_conv1d_bwd_workspace_bytes(int64_t batch, int64_t dim, int64_t seqlen,
+                                             int64_t width);
+msc_status msc_causal_conv1d_bwd(const msc_conv_bwd_args *args, void *workspace,
+                                 size_t workspace_bytes, msc_stream_t stream);
+
+/* ======================================================================
  * Mamba-3 SISO scan
  * ======================================================================
  * Shapes: B = batch, L = seqlen, H = nheads, P = headdim, N = dstate,

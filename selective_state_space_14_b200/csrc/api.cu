@@ -288,4 +288,104 @@ msc_status msc_ssm_state_update(const msc_su_args *a, msc_stream_t stream) {
   return cuda_status(msc::launch_state_update(p, reinterpret_cast<cudaStream_t>(stream)), fn);
 }
 
+// ============================================ causal conv1d ahead of the scan ====
+size_t msc_causal_conv1d_bwd_workspace_bytes(int64_t batch, int64_t dim, int64_t seqlen,
+                                             int64_t width) {
+  if (batch <= 0 || dim <= 0 || seqlen <= 0 || width < 1 || width > MSC_CONV_MAX_WIDTH) return 0;
+  return msc::conv1d_bwd_workspace_bytes(batch, dim, seqlen, width);
+}
+
+}  // extern "C"
+
+namespace {
+template <typename Args>
+msc_status check_conv(const char *fn, const Args *a) {
+  if (!a) return fail(MSC_ERR_INVALID_ARG, "%s: args is NULL", fn);
+  if (a->struct_size < sizeof(Args))
+    return fail(MSC_ERR_INVALID_ARG, "%s: struct_size %u < sizeof(args) %zu", fn, a->struct_size,
+                sizeof(Args));
+  msc_status st;
+  if ((st = check_dtype(fn, a->io_dtype)) != MSC_OK) return st;
+  if (a->batch < 0 || a->dim < 0 || a->seqlen < 0)
+    return fail(MSC_ERR_INVALID_ARG, "%s: batch, dim and seqlen must be >= 0", fn);
+  if (a->width < 1 || a->width > MSC_CONV_MAX_WIDTH)
+    return fail(MSC_ERR_UNSUPPORTED, "%s: width %lld outside 1..%d", fn, (long long)a->width,
+                MSC_CONV_MAX_WIDTH);
+  REQUIRE_PTR(fn, "w", a->w);
+  OPTIONAL_PTR(fn, "bias", a->bias);
+  OPTIONAL_PTR(fn, "conv_state_in", a->conv_state_in);
+  return MSC_OK;
+}
+}  // namespace
+
+extern "C" {
+
+msc_status msc_causal_conv1d_fwd(const msc_conv_fwd_args *a, msc_stream_t stream) {
+  const char *fn = "msc_causal_conv1d_fwd";
+  msc_status st = check_conv(fn, a);
+  if (st != MSC_OK) return st;
+  OPTIONAL_PTR(fn, "conv_state_out", a->conv_state_out);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t B = a->batch, D = a->dim, L = a->seqlen, W = a->width;
+  if (B == 0 || D == 0) return ok();
+  if (L == 0) {  // no steps: the state passes through
+    if (a->conv_state_out && W > 1) {
+      const size_t bytes = sizeof(float) * (size_t)(B * D * (W - 1));
+      return cuda_status(a->conv_state_in ? cudaMemcpyAsync(a->conv_state_out, a->conv_state_in,
+                                                            bytes, cudaMemcpyDeviceToDevice, s)
+                                          : cudaMemsetAsync(a->conv_state_out, 0, bytes, s),
+                         fn);
+    }
+    return ok();
+  }
+  REQUIRE_PTR(fn, "x", a->x);
+  REQUIRE_PTR(fn, "u", a->u);
+  msc::ConvParams p = {};
+  p.io = a->io_dtype;
+  p.B = B; p.D = D; p.L = L; p.W = W;
+  p.vec = (L * (int64_t)io_size(a->io_dtype)) % 16 == 0;
+  p.x = a->x; p.w = a->w; p.bias = a->bias; p.xs_in = W > 1 ? a->conv_state_in : nullptr;
+  p.u = a->u; p.xs_out = W > 1 ? a->conv_state_out : nullptr;
+  return cuda_status(msc::launch_conv1d_fwd(p, s), fn);
+}
+
+msc_status msc_causal_conv1d_bwd(const msc_conv_bwd_args *a, void *workspace,
+                                 size_t workspace_bytes, msc_stream_t stream) {
+  const char *fn = "msc_causal_conv1d_bwd";
+  msc_status st = check_conv(fn, a);
+  if (st != MSC_OK) return st;
+  REQUIRE_PTR(fn, "dw", a->dw);
+  OPTIONAL_PTR(fn, "dbias", a->dbias);
+  OPTIONAL_PTR(fn, "dconv_state_in", a->dconv_state_in);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t B = a->batch, D = a->dim, L = a->seqlen, W = a->width;
+  if (B == 0 || D == 0 || L == 0) {  // no steps: zero gradients
+    cudaError_t e = D > 0 ? cudaMemsetAsync(a->dw, 0, sizeof(float) * (size_t)(D * W), s)
+                          : cudaSuccess;
+    if (e == cudaSuccess && a->dbias && D > 0)
+      e = cudaMemsetAsync(a->dbias, 0, sizeof(float) * (size_t)D, s);
+    if (e == cudaSuccess && a->dconv_state_in && W > 1 && B * D > 0)
+      e = cudaMemsetAsync(a->dconv_state_in, 0, sizeof(float) * (size_t)(B * D * (W - 1)), s);
+    return cuda_status(e, fn);
+  }
+  REQUIRE_PTR(fn, "x", a->x);
+  REQUIRE_PTR(fn, "du", a->du);
+  REQUIRE_PTR(fn, "dx", a->dx);
+  const size_t need = msc::conv1d_bwd_workspace_bytes(B, D, L, W);
+  if (workspace == nullptr || workspace_bytes < need)
+    return fail(MSC_ERR_WORKSPACE, "%s: workspace of %zu bytes given, %zu required", fn,
+                workspace ? workspace_bytes : (size_t)0, need);
+  if (!aligned16(workspace))
+    return fail(MSC_ERR_ALIGNMENT, "%s: workspace is not 16-byte aligned", fn);
+  msc::ConvParams p = {};
+  p.io = a->io_dtype;
+  p.B = B; p.D = D; p.L = L; p.W = W;
+  p.vec = (L * (int64_t)io_size(a->io_dtype)) % 16 == 0;
+  p.x = a->x; p.w = a->w; p.bias = a->bias; p.xs_in = W > 1 ? a->conv_state_in : nullptr;
+  p.du = a->du; p.dx = a->dx; p.dw = a->dw; p.dbias = a->dbias;
+  p.dxs_in = W > 1 ? a->dconv_state_in : nullptr;
+  p.ws = static_cast<float *>(workspace);
+  return cuda_status(msc::launch_conv1d_bwd(p, s), fn);
+}
+
 }  // extern "C"

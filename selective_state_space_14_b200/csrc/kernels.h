@@ -104,6 +104,25 @@ size_t m3_bwd_workspace_bytes(int64_t B, int64_t L, int64_t H, int64_t P, int64_
                               int64_t K);
 bool m3_supported(int64_t P, int64_t N);
 
+// causal depthwise conv1d + SiLU ahead of the Mamba-1 scan
+struct ConvParams {
+  int io;  // msc_dtype
+  int64_t B, D, L, W;
+  bool vec;  // rows of length L are 16-byte aligned for vector access
+  const void *x;
+  const float *w, *bias, *xs_in;
+  void *u;
+  float *xs_out;
+  // backward
+  const void *du;
+  void *dx;
+  float *dw, *dbias, *dxs_in;
+  float *ws;  // per-run partials of dw, dbias
+};
+cudaError_t launch_conv1d_fwd(const ConvParams &p, cudaStream_t s);
+cudaError_t launch_conv1d_bwd(const ConvParams &p, cudaStream_t s);
+size_t conv1d_bwd_workspace_bytes(int64_t B, int64_t D, int64_t L, int64_t W);
+
 // Mamba-3 SISO single-token state update (decode)
 struct M3SUParams {
   int io;  // msc_dtype: 0 f32, 1 bf16, 2 f16

@@ -89,12 +89,26 @@ class M3SuArgs(ctypes.Structure):
                 ("gamma", _vp), ("theta", _vp), ("D", _vp), ("out", _vp)]
 
 
+class ConvFwdArgs(ctypes.Structure):
+    _fields_ = [("struct_size", _u32), ("io_dtype", _i32), ("batch", _i64), ("dim", _i64),
+                ("seqlen", _i64), ("width", _i64), ("x", _vp), ("w", _vp), ("bias", _vp),
+                ("conv_state_in", _vp), ("u", _vp), ("conv_state_out", _vp)]
+
+
+class ConvBwdArgs(ctypes.Structure):
+    _fields_ = [("struct_size", _u32), ("io_dtype", _i32), ("batch", _i64), ("dim", _i64),
+                ("seqlen", _i64), ("width", _i64), ("x", _vp), ("w", _vp), ("bias", _vp),
+                ("conv_state_in", _vp), ("du", _vp), ("dx", _vp), ("dw", _vp), ("dbias", _vp),
+                ("dconv_state_in", _vp)]
+
+
 EXPORTS = ["msc_last_error", "msc_version", "msc_selective_scan_saved_states_bytes",
            "msc_selective_scan_fwd_workspace_bytes", "msc_selective_scan_fwd", "msc_selective_scan_bwd_workspace_bytes",
            "msc_selective_scan_bwd", "msc_selective_scan_bwd_static", "msc_ssm_state_update",
            "msc_mamba3_siso_saved_states_bytes", "msc_mamba3_siso_scan_fwd_workspace_bytes",
            "msc_mamba3_siso_scan_fwd", "msc_mamba3_siso_scan_bwd_workspace_bytes",
-           "msc_mamba3_siso_scan_bwd", "msc_mamba3_siso_state_update"]
+           "msc_mamba3_siso_scan_bwd", "msc_mamba3_siso_state_update", "msc_causal_conv1d_fwd",
+           "msc_causal_conv1d_bwd_workspace_bytes", "msc_causal_conv1d_bwd"]
 
 _lib = None
 
@@ -117,7 +131,10 @@ def lib() -> ctypes.CDLL:
                            ("msc_mamba3_siso_scan_fwd", [ctypes.POINTER(M3FwdArgs), _vp]),
                            ("msc_mamba3_siso_scan_bwd",
                             [ctypes.POINTER(M3BwdArgs), _vp, ctypes.c_size_t, _vp]),
-                           ("msc_mamba3_siso_state_update", [ctypes.POINTER(M3SuArgs), _vp])):
+                           ("msc_mamba3_siso_state_update", [ctypes.POINTER(M3SuArgs), _vp]),
+                           ("msc_causal_conv1d_fwd", [ctypes.POINTER(ConvFwdArgs), _vp]),
+                           ("msc_causal_conv1d_bwd",
+                            [ctypes.POINTER(ConvBwdArgs), _vp, ctypes.c_size_t, _vp])):
             f = getattr(L, name)
             f.argtypes = argt
             f.restype = ctypes.c_int
@@ -131,6 +148,8 @@ def lib() -> ctypes.CDLL:
         L.msc_mamba3_siso_saved_states_bytes.restype = ctypes.c_size_t
         L.msc_mamba3_siso_scan_fwd_workspace_bytes.argtypes = [_i64] * 5
         L.msc_mamba3_siso_scan_fwd_workspace_bytes.restype = ctypes.c_size_t
+        L.msc_causal_conv1d_bwd_workspace_bytes.argtypes = [_i64] * 4
+        L.msc_causal_conv1d_bwd_workspace_bytes.restype = ctypes.c_size_t
         L.msc_mamba3_siso_scan_bwd_workspace_bytes.argtypes = [_i64] * 7
         L.msc_mamba3_siso_scan_bwd_workspace_bytes.restype = ctypes.c_size_t
         _lib = L
@@ -411,3 +430,51 @@ def msc_mamba3_siso_state_update(state, x_prev, bt_prev, phi, x, B, C, alpha, be
                  _ptr(out))
     _check(lib().msc_mamba3_siso_state_update(ctypes.byref(a), _stream(stream)))
     return out
+
+
+# ---------------------------------------------------------------------------
+# causal conv1d + SiLU ahead of the Mamba-1 scan
+# ---------------------------------------------------------------------------
+def msc_causal_conv1d_fwd(x, w, bias=None, conv_state_in=None, u=None, conv_state_out=None,
+                          want_state=True, stream=None):
+    """u = silu(causal depthwise conv of x).  x [B, D, L] (io); w f32 [D, W];
+    bias f32 [D]; conv states f32 [B, D, W-1].  Returns (u, conv_state_out)."""
+    Bsz, Dm, L = x.shape
+    W = w.shape[1]
+    if u is None:
+        u = torch.empty_like(x)
+    if conv_state_out is None and want_state and W > 1:
+        conv_state_out = torch.empty((Bsz, Dm, W - 1), device=x.device, dtype=torch.float32)
+    a = ConvFwdArgs(ctypes.sizeof(ConvFwdArgs), _io(x), Bsz, Dm, L, W, _ptr(x), _ptr(w),
+                    _ptr(bias), _ptr(conv_state_in), _ptr(u), _ptr(conv_state_out))
+    _check(lib().msc_causal_conv1d_fwd(ctypes.byref(a), _stream(stream)))
+    return u, conv_state_out
+
+
+def msc_causal_conv1d_bwd_workspace_bytes(batch, dim, seqlen, width) -> int:
+    return int(lib().msc_causal_conv1d_bwd_workspace_bytes(batch, dim, seqlen, width))
+
+
+def msc_causal_conv1d_bwd(x, w, du, bias=None, conv_state_in=None, workspace=None,
+                          want_dstate=True, grads=None, stream=None):
+    """Backward of msc_causal_conv1d_fwd for the upstream du.  Returns dict dx, dw,
+    dbias, dconv_state_in."""
+    Bsz, Dm, L = x.shape
+    W = w.shape[1]
+    f32 = dict(device=x.device, dtype=torch.float32)
+    g = dict(grads or {})
+    g.setdefault("dx", torch.empty_like(x))
+    g.setdefault("dw", torch.empty((Dm, W), **f32))
+    g.setdefault("dbias", torch.empty((Dm,), **f32) if bias is not None else None)
+    g.setdefault("dconv_state_in", torch.empty((Bsz, Dm, W - 1), **f32)
+                 if want_dstate and W > 1 else None)
+    if workspace is None:
+        need = msc_causal_conv1d_bwd_workspace_bytes(Bsz, Dm, L, W)
+        workspace = torch.empty(max(need, 16), device=x.device, dtype=torch.uint8)
+    a = ConvBwdArgs(ctypes.sizeof(ConvBwdArgs), _io(x), Bsz, Dm, L, W, _ptr(x), _ptr(w),
+                    _ptr(bias), _ptr(conv_state_in), _ptr(du), _ptr(g["dx"]), _ptr(g["dw"]),
+                    _ptr(g["dbias"]), _ptr(g["dconv_state_in"]))
+    _check(lib().msc_causal_conv1d_bwd(ctypes.byref(a), _ptr(workspace),
+                                       workspace.numel() * workspace.element_size(),
+                                       _stream(stream)))
+    return g

@@ -218,3 +218,36 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(msc, "_lib", None)
     with pytest.raises(RuntimeError, match="missing"):
         msc.lib()
+
+
+def _conv_args(cls, **kw):
+    a = cls()
+    a.struct_size = ctypes.sizeof(cls)
+    a.io_dtype, a.batch, a.dim, a.seqlen, a.width = msc.MSC_BF16, 2, 8, 64, 4
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("field,value,status,word", [
+    ("width", 0, UNSUPPORTED, "width"),
+    ("width", 5, UNSUPPORTED, "width"),
+    ("seqlen", -1, INVALID, "seqlen"),
+    ("io_dtype", 9, INVALID, "io_dtype"),
+    ("struct_size", 4, INVALID, "struct_size"),
+])
+def test_conv_rejects_bad_sizes(field, value, status, word):
+    st = msc.lib().msc_causal_conv1d_fwd(ctypes.byref(_conv_args(msc.ConvFwdArgs, **{field: value})),
+                                         None)
+    assert st == status and word in _err()
+
+
+def test_conv_rejects_missing_weights_and_workspace():
+    """No weights: rejected; backward without a workspace: rejected (the calls
+    stop at the checks, before any launch)."""
+    assert msc.lib().msc_causal_conv1d_fwd(ctypes.byref(_conv_args(msc.ConvFwdArgs)), None) == INVALID
+    assert "w is NULL" in _err()
+    fake = ctypes.c_void_p(1 << 20)
+    a = _conv_args(msc.ConvBwdArgs, w=fake, x=fake, du=fake, dx=fake, dw=fake)
+    assert msc.lib().msc_causal_conv1d_bwd(ctypes.byref(a), None, 0, None) == WORKSPACE
+    assert msc.msc_causal_conv1d_bwd_workspace_bytes(2, 8, 64, 4) == 4 * 2 * 8 * 8 * 5
