@@ -268,6 +268,60 @@ class M1Step:
                                         workspace=self.ws, grads=self.grads, want_dh0=False)
 
 
+class M1ConvStep:
+    """Device-resident causal conv1d + Mamba-1 scan: the fused forward, the
+    unfused forward (conv, then scan), and the two backward calls."""
+
+    def __init__(self, q, msc):
+        import torch
+        self.msc = msc
+        self.q = q
+        self.st = M1Step(q.scan, msc)  # its u is the conv's input x
+        self.x = self.st.a["u"]
+        self.w, self.bias = to_dev(q.w), to_dev(q.bias)
+        self.u = torch.empty_like(self.x)
+        Bsz, D = q.scan.batch, q.scan.dim
+        self.xs = torch.empty((Bsz, D, q.width - 1), device="cuda", dtype=torch.float32)
+        self.scan_a = {k: v for k, v in self.st.a.items() if k != "u"}
+        self.cws = torch.empty(max(msc.msc_causal_conv1d_bwd_workspace_bytes(
+            Bsz, D, q.scan.seqlen, q.width), 16), device="cuda", dtype=torch.uint8)
+        self.cgrads = None
+
+    def fused_fwd(self):
+        """One launch: u = silu(conv(x)) feeds the scan in shared memory (u is
+        also written out for the backward pass)."""
+        self.msc.msc_selective_scan_conv_fwd(
+            self.x, self.w, conv_bias=self.bias, **self.scan_a, u_out=self.u,
+            conv_state_out=self.xs, out=self.st.out, final_state=self.st.fs,
+            saved_states=self.st.saved)
+
+    def conv_fwd(self):
+        self.msc.msc_causal_conv1d_fwd(self.x, self.w, bias=self.bias, u=self.u,
+                                       conv_state_out=self.xs)
+
+    def scan_fwd(self):
+        self.msc.msc_selective_scan_fwd(u=self.u, **self.scan_a, out=self.st.out,
+                                        final_state=self.st.fs, saved_states=self.st.saved)
+
+    def scan_bwd(self):
+        self.msc.msc_selective_scan_bwd(u=self.u, **self.scan_a, saved_states=self.st.saved,
+                                        dout=self.st.dout, workspace=self.st.ws,
+                                        grads=self.st.grads, want_dh0=False)
+
+    def conv_bwd(self):
+        self.cgrads = self.msc.msc_causal_conv1d_bwd(
+            self.x, self.w, self.st.grads["du"], bias=self.bias, workspace=self.cws,
+            grads=self.cgrads)
+
+
+def conv_bytes(Bsz, D, L, W, io_bytes):
+    """Algorithmic HBM bytes of the standalone conv: forward reads x, writes u;
+    backward reads x and du, writes dx (weights, states and the per-run dw
+    partials are small and left out)."""
+    n = Bsz * D * L * io_bytes
+    return 2 * n, 3 * n
+
+
 def time_steps(step_fns, steps, warmup, world, sampler=None):
     """Run warmup, then time `steps` iterations; per-phase CUDA-event times.
     A clock sampler, if given, runs during the timed region only."""
@@ -543,6 +597,36 @@ def extra_workloads(msc, args, world, peaks):
             bwd_hbm_frac=round(bb / b_ms / 1e6 / peaks["hbm_gbs"], 4))
     except Exception as e:  # noqa: BLE001 -- report, keep the headline line
         res["m3_bf16_b8_h24_p64_n64_k32_l2048"] = dict(error=str(e)[:200])
+    torch.cuda.empty_cache()
+    # causal conv1d (width 4) + SiLU ahead of the Mamba-1 scan, the headline's sizes
+    name = "m1conv_bf16_b8_d1536_n16_l2048_w4"
+    try:
+        q = W.make(name)
+        cs = M1ConvStep(q, msc)
+        cs.fused_fwd()
+        cs.scan_bwd()
+        cs.conv_bwd()
+        n = max(3, args.steps // 2)
+        _, (fused_ms, sbwd_ms, cbwd_ms) = time_steps([cs.fused_fwd, cs.scan_bwd, cs.conv_bwd],
+                                                     n, 3, world)
+        _, (conv_ms, sfwd_ms) = time_steps([cs.conv_fwd, cs.scan_fwd], n, 3, world)
+        sp = q.scan
+        fb, _ = m1_bytes(sp.batch, sp.dim, sp.dstate, sp.seqlen, 2)
+        cfb, cbb = conv_bytes(sp.batch, sp.dim, sp.seqlen, q.width, 2)
+        res[name] = dict(
+            fused_fwd_ms=round(fused_ms, 4), unfused_fwd_ms=round(conv_ms + sfwd_ms, 4),
+            conv_fwd_ms=round(conv_ms, 4), scan_fwd_ms=round(sfwd_ms, 4),
+            scan_bwd_ms=round(sbwd_ms, 4), conv_bwd_ms=round(cbwd_ms, 4),
+            value=round(sp.token_channels / ((fused_ms + sbwd_ms + cbwd_ms) / 1e3), 1),
+            unit=UNIT,
+            fused_fwd_hbm_frac=round((fb + sp.batch * sp.dim * sp.seqlen * 2) / fused_ms / 1e6
+                                     / peaks["hbm_gbs"], 4),
+            conv_fwd_hbm_frac=round(cfb / conv_ms / 1e6 / peaks["hbm_gbs"], 4),
+            conv_bwd_hbm_frac=round(cbb / cbwd_ms / 1e6 / peaks["hbm_gbs"], 4),
+            note="value: fused forward + scan backward + conv backward")
+        del cs
+    except Exception as e:  # noqa: BLE001 -- report, keep the headline line
+        res[name] = dict(error=str(e)[:200])
     return res
 
 
@@ -559,7 +643,7 @@ def run_only(args):
     from selective_state_space_14_b200 import msc
     msc.lib()
     phase = args.only
-    if phase.startswith("m1"):
+    if phase in ("m1_fwd", "m1_bwd"):
         p = W.make(args.workload or HEADLINE)
         st = M1Step(p, msc)
         st.fwd()
@@ -584,6 +668,14 @@ def run_only(args):
                 msc.msc_mamba3_siso_scan_bwd(**a, saved_states=saved, dout=dout, workspace=ws,
                                              grads=grads)
         units = m3.token_channels
+    elif phase in ("m1_conv_fwd", "conv_fwd", "conv_bwd"):
+        q = W.make(args.workload or "m1conv_bf16_b8_d1536_n16_l2048_w4")
+        cs = M1ConvStep(q, msc)
+        cs.fused_fwd()
+        cs.scan_bwd()
+        cs.conv_bwd()
+        fn = {"m1_conv_fwd": cs.fused_fwd, "conv_fwd": cs.conv_fwd, "conv_bwd": cs.conv_bwd}[phase]
+        units = q.scan.token_channels
     elif phase == "m3_decode":
         q = W.make(args.workload or "m3su_bf16_b256_h24_p64_n64_k32_x1000")
         carried = [torch.from_numpy(v).cuda() for v in (q.state0, q.x_prev0, q.bt_prev0, q.phi0)]
@@ -664,7 +756,7 @@ def main():
     ap.add_argument("--no-extra", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", choices=["m1_fwd", "m1_bwd", "m3_fwd", "m3_bwd", "decode",
-                                       "m3_decode"],
+                                       "m3_decode", "m1_conv_fwd", "conv_fwd", "conv_bwd"],
                     help="time one phase alone (for profiling); prints no bench line")
     ap.add_argument("--workload", default=None, help="workload name for --only")
     args = ap.parse_args()

@@ -292,6 +292,33 @@ size_t msc_causal_conv1d_bwd_workspace_bytes(int64_t batch, int64_t dim, int64_t
 msc_status msc_causal_conv1d_bwd(const msc_conv_bwd_args *args, void *workspace,
                                  size_t workspace_bytes, msc_stream_t stream);
 
+/*
+ * The conv fused ahead of the Mamba-1 scan forward: one launch computes
+ * u = silu(conv(x)) per token as the scan consumes it, so u never makes a
+ * round trip through memory.  scan->u holds x (the conv's input, io
+ * [B, D, L]); every other field of scan keeps its meaning in
+ * msc_selective_scan_fwd, and conv gives the conv's parameters with the
+ * layouts of msc_conv_fwd_args.  u_out (optional, io [B, D, L]) receives
+ * u = silu(conv(x)), which the backward pass of the scan takes as its u;
+ * the backward stays two calls: msc_selective_scan_bwd (on u_out) and then
+ * msc_causal_conv1d_bwd (with its du).  The fused form is an addition of
+ * this library; its results are those of msc_causal_conv1d_fwd followed by
+ * msc_selective_scan_fwd, bit for bit (the scan takes u rounded to the io
+ * type, as the unfused conv stores it).
+ */
+typedef struct {
+  uint32_t struct_size;
+  int64_t width;                /* 1 <= width <= MSC_CONV_MAX_WIDTH          */
+  const float *w;               /* f32 [D, W]                                */
+  const float *bias;            /* optional, f32 [D]                         */
+  const float *conv_state_in;   /* optional, f32 [B, D, W-1]                 */
+  float *conv_state_out;        /* optional, f32 [B, D, W-1]                 */
+  void *u_out;                  /* optional, io [B, D, L]                    */
+} msc_ss_conv_args;
+
+msc_status msc_selective_scan_conv_fwd(const msc_ss_fwd_args *scan,
+                                       const msc_ss_conv_args *conv, msc_stream_t stream);
+
 /* ======================================================================
  * Mamba-3 SISO scan
  * ======================================================================

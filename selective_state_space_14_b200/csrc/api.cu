@@ -120,8 +120,12 @@ size_t msc_selective_scan_fwd_workspace_bytes(int64_t batch, int64_t dim, int64_
   return sizeof(float) * (size_t)(batch * dim * seqlen);  // the sums over the earlier slabs
 }
 
-msc_status msc_selective_scan_fwd(const msc_ss_fwd_args *a, msc_stream_t stream) {
-  const char *fn = "msc_selective_scan_fwd";
+}  // extern "C"
+
+namespace {
+// the Mamba-1 forward, with the causal conv1d fused ahead when conv is non-null
+msc_status m1_fwd(const char *fn, const msc_ss_fwd_args *a, const msc_ss_conv_args *conv,
+                  msc_stream_t stream) {
   if (!a) return fail(MSC_ERR_INVALID_ARG, "%s: args is NULL", fn);
   // callers built before the workspace fields pass a shorter struct: no workspace
   constexpr size_t kNoWorkspaceSize = offsetof(msc_ss_fwd_args, workspace);
@@ -137,6 +141,21 @@ msc_status msc_selective_scan_fwd(const msc_ss_fwd_args *a, msc_stream_t stream)
   if ((st = check_m1_sizes(fn, a->batch, a->dim, a->dstate, a->seqlen, a->ngroups)) != MSC_OK)
     return st;
   const int64_t B = a->batch, D = a->dim, N = a->dstate, L = a->seqlen;
+  int64_t W = 0;
+  if (conv) {
+    if (conv->struct_size < sizeof(msc_ss_conv_args))
+      return fail(MSC_ERR_INVALID_ARG, "%s: conv struct_size %u < sizeof(msc_ss_conv_args) %zu",
+                  fn, conv->struct_size, sizeof(msc_ss_conv_args));
+    W = conv->width;
+    if (W < 1 || W > MSC_CONV_MAX_WIDTH)
+      return fail(MSC_ERR_UNSUPPORTED, "%s: width %lld outside 1..%d", fn, (long long)W,
+                  MSC_CONV_MAX_WIDTH);
+    REQUIRE_PTR(fn, "w", conv->w);
+    OPTIONAL_PTR(fn, "bias", conv->bias);
+    OPTIONAL_PTR(fn, "conv_state_in", conv->conv_state_in);
+    OPTIONAL_PTR(fn, "conv_state_out", conv->conv_state_out);
+    OPTIONAL_PTR(fn, "u_out", conv->u_out);
+  }
   if (B == 0 || D == 0) return ok();
   REQUIRE_PTR(fn, "A", a->A);
   OPTIONAL_PTR(fn, "D", a->D);
@@ -144,15 +163,20 @@ msc_status msc_selective_scan_fwd(const msc_ss_fwd_args *a, msc_stream_t stream)
   OPTIONAL_PTR(fn, "h0", a->h0);
   OPTIONAL_PTR(fn, "final_state", a->final_state);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (L == 0) {  // no steps: the final state is the initial state
+  if (L == 0) {  // no steps: the final states are the initial states
+    cudaError_t e = cudaSuccess;
     if (a->final_state) {
       const size_t bytes = sizeof(float) * (size_t)(B * D * N);
-      cudaError_t e = a->h0 ? cudaMemcpyAsync(a->final_state, a->h0, bytes,
-                                              cudaMemcpyDeviceToDevice, s)
-                            : cudaMemsetAsync(a->final_state, 0, bytes, s);
-      return cuda_status(e, fn);
+      e = a->h0 ? cudaMemcpyAsync(a->final_state, a->h0, bytes, cudaMemcpyDeviceToDevice, s)
+                : cudaMemsetAsync(a->final_state, 0, bytes, s);
     }
-    return ok();
+    if (e == cudaSuccess && conv && conv->conv_state_out && W > 1) {
+      const size_t bytes = sizeof(float) * (size_t)(B * D * (W - 1));
+      e = conv->conv_state_in ? cudaMemcpyAsync(conv->conv_state_out, conv->conv_state_in, bytes,
+                                                cudaMemcpyDeviceToDevice, s)
+                              : cudaMemsetAsync(conv->conv_state_out, 0, bytes, s);
+    }
+    return cuda_status(e, fn);
   }
   REQUIRE_PTR(fn, "u", a->u);
   REQUIRE_PTR(fn, "delta", a->delta);
@@ -176,7 +200,28 @@ msc_status msc_selective_scan_fwd(const msc_ss_fwd_args *a, msc_stream_t stream)
   p.A = a->A; p.Dp = a->D; p.bias = a->delta_bias; p.h0 = a->h0;
   p.out = a->out; p.final_state = a->final_state; p.saved = a->saved_states;
   p.tok_part = need > 0 ? static_cast<float *>(workspace) : nullptr;
+  if (conv) {
+    p.conv_W = W;
+    p.conv_w = conv->w; p.conv_b = conv->bias;
+    p.conv_xs_in = W > 1 ? conv->conv_state_in : nullptr;
+    p.conv_xs_out = W > 1 ? conv->conv_state_out : nullptr;
+    p.u_out = conv->u_out;
+  }
   return cuda_status(msc::launch_m1_fwd(p, s), fn);
+}
+}  // namespace
+
+extern "C" {
+
+msc_status msc_selective_scan_fwd(const msc_ss_fwd_args *a, msc_stream_t stream) {
+  return m1_fwd("msc_selective_scan_fwd", a, nullptr, stream);
+}
+
+msc_status msc_selective_scan_conv_fwd(const msc_ss_fwd_args *scan,
+                                       const msc_ss_conv_args *conv, msc_stream_t stream) {
+  const char *fn = "msc_selective_scan_conv_fwd";
+  if (!conv) return fail(MSC_ERR_INVALID_ARG, "%s: conv is NULL", fn);
+  return m1_fwd(fn, scan, conv, stream);
 }
 
 size_t msc_selective_scan_bwd_workspace_bytes(int64_t batch, int64_t dim, int64_t dstate,

@@ -16,6 +16,12 @@ struct M1Params {
   bool vec;  // rows of length L are 16-byte aligned for vector access
   const void *u, *delta, *Bm, *Cm, *z;
   const float *A, *Dp, *bias, *h0;
+  // forward with the causal conv1d + SiLU fused ahead (conv_w non-null): u
+  // holds the conv's input x; u_out (optional) receives the scan input u
+  const float *conv_w, *conv_b, *conv_xs_in;
+  float *conv_xs_out;
+  void *u_out;
+  int64_t conv_W;
   // forward outputs
   void *out;
   float *final_state, *saved;

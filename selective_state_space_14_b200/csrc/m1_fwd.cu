@@ -30,7 +30,7 @@ constexpr int kWarps = 4;
 constexpr int kTF = 32;  // steps per forward chunk
 static_assert(kTF % kM1SaveInterval == 0, "chunk must hold whole saved-state intervals");
 
-template <int kN>
+template <int kN, bool kConv>
 struct FwdSmem {
   using Lay = Layout<kN, kWarps>;
   static constexpr int kP = Lay::kP;
@@ -46,7 +46,12 @@ struct FwdSmem {
   static constexpr int ytile = bc + kTF * kP * 4;             // [kWarps][32/kP][kChBlock]
   static constexpr int out = ytile + kWarps * (32 / kP) * kChBlock;  // [kCh][kOut]
   static constexpr int gate = out + kCh * kOut;               // [kCh][kOut] silu(z), last slab
-  static constexpr int raw = (gate + kCh * kOut + 3) / 4 * 4;  // raw inputs (16-byte aligned)
+  // with the conv fused ahead: [2][kCh][4] conv inputs before a chunk and
+  // [2][kCh][kOut] the conv's output u (a chunk's tile is stored out with the
+  // chunk's outputs, while the next chunk fills the other one)
+  static constexpr int halo = gate + kCh * kOut;
+  static constexpr int su = halo + (kConv ? 2 * kCh * 4 : 0);
+  static constexpr int raw = (su + (kConv ? 2 * kCh * kOut : 0) + 3) / 4 * 4;  // 16-byte aligned
   static constexpr int total_floats = raw;
 };
 
@@ -126,8 +131,9 @@ __device__ __forceinline__ void fwd_issue_raw(const M1Params &p, unsigned char *
 // its own and stores the gated outputs.
 template <typename T, int kCh, int kOut>
 __device__ __forceinline__ void store_chunk(const M1Params &p, const float *sout,
-                                            const float *sgate, int64_t c_first, int64_t c_end,
-                                            int64_t b, int64_t tc, int tid, int nthreads) {
+                                            const float *sgate, const float *su,
+                                            int64_t c_first, int64_t c_end, int64_t b,
+                                            int64_t tc, int tid, int nthreads) {
   const int64_t D = p.D, L = p.L;
   for (int u = tid; u < kCh * (kTF / 8); u += nthreads) {
     const int chl = u / (kTF / 8);
@@ -138,6 +144,12 @@ __device__ __forceinline__ void store_chunk(const M1Params &p, const float *sout
     const float4 e = *reinterpret_cast<const float4 *>(sout + chl * kOut + seg * 8 + 4);
     float v[8] = {a.x, a.y, a.z, a.w, e.x, e.y, e.z, e.w};
     const int64_t row = (b * D + c) * L, t0 = tc + seg * 8;
+    if (su) {  // the conv's output u (exact: values already rounded to T)
+      const float4 ua = *reinterpret_cast<const float4 *>(su + chl * kOut + seg * 8);
+      const float4 ue = *reinterpret_cast<const float4 *>(su + chl * kOut + seg * 8 + 4);
+      const float uv[8] = {ua.x, ua.y, ua.z, ua.w, ue.x, ue.y, ue.z, ue.w};
+      store_run<8>(static_cast<T *>(p.u_out) + row, t0, L, p.vec, uv);
+    }
     if (p.slab == kSlabWhole) {
       store_run<8>(static_cast<T *>(p.out) + row, t0, L, p.vec, v);
       continue;
@@ -161,9 +173,12 @@ __device__ __forceinline__ void store_chunk(const M1Params &p, const float *sout
   }
 }
 
-template <typename T, int kN>
+// kConv: the causal conv1d + SiLU fused ahead: the token runs read the conv's
+// input x (from the stage, the W-1 inputs before a chunk from the halo) and
+// turn it into u
+template <typename T, int kN, bool kConv>
 __global__ void __launch_bounds__(kWarps * 32, 6) m1_fwd_kernel(const M1Params p) {
-  using S = FwdSmem<kN>;
+  using S = FwdSmem<kN, kConv>;
   using Lay = Layout<kN, kWarps>;
   constexpr int kP = Lay::kP;
   constexpr int kCh = Lay::kCh;
@@ -174,6 +189,7 @@ __global__ void __launch_bounds__(kWarps * 32, 6) m1_fwd_kernel(const M1Params p
   float4 *sBC = reinterpret_cast<float4 *>(smem + S::bc);
   float *sOut = smem + S::out;
   float *sGate = smem + S::gate;
+  float *sHalo = smem + S::halo;
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -224,6 +240,19 @@ __global__ void __launch_bounds__(kWarps * 32, 6) m1_fwd_kernel(const M1Params p
 
   const T **const rows = reinterpret_cast<const T **>(raw + R::rows);
   fwd_fill_rows<T, kN>(p, rows, b, c_first, c_end, Bg, Cg, tid);
+  if constexpr (kConv) {
+    // the inputs before the sequence: the conv state (entry j holds x at time
+    // j - (W-1)) or zeros
+    const int Wd = (int)p.conv_W;
+    for (int i = tid; i < kCh * 3; i += kThreads) {
+      const int cl = i / 3, k = i % 3, pos = k - 3;
+      const int64_t cc = c_first + cl;
+      float v = 0.f;
+      if (cc < c_end && p.conv_xs_in && pos >= -(Wd - 1))
+        v = p.conv_xs_in[(b * D + cc) * (Wd - 1) + (Wd - 1) + pos];
+      sHalo[cl * 4 + k] = v;
+    }
+  }
   __syncthreads();
   fwd_issue_raw<T, kN>(p, raw, rows, 0, tid);
   for (int64_t ch = 0; ch <= n_chunks; ++ch) {
@@ -231,7 +260,10 @@ __global__ void __launch_bounds__(kWarps * 32, 6) m1_fwd_kernel(const M1Params p
     cp_async_wait<0>();
     __syncthreads();  // this chunk's raw inputs are in; the last chunk is done
     if (ch > 0)
-      store_chunk<T, kCh, S::kOut>(p, sOut, sGate, c_first, c_end, b, tc - kTF, tid, kThreads);
+      store_chunk<T, kCh, S::kOut>(p, sOut, sGate,
+                                   kConv && p.u_out ? smem + S::su + ((ch - 1) & 1) * kCh * S::kOut
+                                                    : nullptr,
+                                   c_first, c_end, b, tc - kTF, tid, kThreads);
     if (ch == n_chunks) break;
     // ---- per-token values: kRun steps of one channel per thread ---------------
     {
@@ -243,6 +275,40 @@ __global__ void __launch_bounds__(kWarps * 32, 6) m1_fwd_kernel(const M1Params p
         x[i] = to_f32(ru[o]);
         v[i] = to_f32(ru[kCh * R::kTokRow + o]);
         zv[i] = p.z ? to_f32(ru[2 * kCh * R::kTokRow + o]) : 0.f;
+      }
+      if constexpr (kConv) {
+        // u = silu(b + sum_k w[k] x[t-(W-1)+k]) over this run; x before the
+        // chunk from the halo, and this chunk's last three inputs become the
+        // next chunk's halo (other parity: this chunk's halo is still read)
+        const float *hl = sHalo + ((ch & 1) * kCh + tcl) * 4;  // x at tc-3 .. tc-1
+        float xs[kRun + 3];  // x at tseg*kRun - 3 .. tseg*kRun + kRun - 1
+#pragma unroll
+        for (int j = 0; j < kRun + 3; ++j) {
+          const int pos = tseg * kRun - 3 + j;
+          xs[j] = pos >= 0 ? to_f32(ru[tcl * R::kTokRow + pos]) : hl[pos + 3];
+        }
+        // tap k of 4 meets x at t-3+k; a width-W conv uses taps 4-W .. 3 (the
+        // taps stay compile-time indexes: xs lives in registers)
+        const int Wd = (int)p.conv_W, k0 = 4 - Wd;
+        float wv[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) wv[k] = (tact && k >= k0) ? p.conv_w[tcc * Wd + k - k0] : 0.f;
+        const float cb = (tact && p.conv_b) ? p.conv_b[tcc] : 0.f;
+#pragma unroll
+        for (int i = 0; i < kRun; ++i) {
+          float a = cb;
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            if (k >= k0) a = fmaf(wv[k], xs[i + k], a);
+          // u rounded to the io type, as the unfused conv would store it
+          x[i] = to_f32(from_f32<T>(silu(a)));
+          smem[S::su + ((ch & 1) * kCh + tcl) * S::kOut + tseg * kRun + i] = x[i];
+        }
+        if (tseg == kTF / kRun - 1) {
+          float *hn = sHalo + (((ch + 1) & 1) * kCh + tcl) * 4;
+#pragma unroll
+          for (int k = 0; k < 3; ++k) hn[k] = xs[kRun + k];
+        }
       }
 #pragma unroll
       for (int i = 0; i < kRun; ++i) {
@@ -326,6 +392,21 @@ __global__ void __launch_bounds__(kWarps * 32, 6) m1_fwd_kernel(const M1Params p
     }
   }
 
+  if constexpr (kConv) {
+    // the conv state for the next call: the last W-1 inputs
+    const int Wd = (int)p.conv_W;
+    if (p.conv_xs_out) {
+      for (int i = tid; i < kCh * (Wd - 1); i += kThreads) {
+        const int cl = i / (Wd - 1), j = i % (Wd - 1);
+        const int64_t cc = c_first + cl;
+        if (cc >= c_end) continue;
+        const int64_t t = L - (Wd - 1) + j;
+        p.conv_xs_out[(b * D + cc) * (Wd - 1) + j] =
+            t >= 0 ? to_f32(static_cast<const T *>(p.u)[(b * D + cc) * L + t])
+                   : (p.conv_xs_in ? p.conv_xs_in[(b * D + cc) * (Wd - 1) + (Wd - 1) + t] : 0.f);
+      }
+    }
+  }
   if (active && p.final_state) {
     float *dst = p.final_state + (b * D + c) * ldN + ns;
     if (n0 < N) dst[n0] = h.x;
@@ -333,17 +414,23 @@ __global__ void __launch_bounds__(kWarps * 32, 6) m1_fwd_kernel(const M1Params p
   }
 }
 
-template <typename T, int kN>
-cudaError_t launch_t(const M1Params &p, cudaStream_t s) {
+template <typename T, int kN, bool kConv>
+cudaError_t launch_c(const M1Params &p, cudaStream_t s) {
   using Lay = Layout<kN, kWarps>;
-  const size_t smem = sizeof(float) * (size_t)FwdSmem<kN>::total_floats + FwdRaw<T, kN>::bytes;
-  cudaError_t e = cudaFuncSetAttribute(m1_fwd_kernel<T, kN>,
+  const size_t smem =
+      sizeof(float) * (size_t)FwdSmem<kN, kConv>::total_floats + FwdRaw<T, kN>::bytes;
+  cudaError_t e = cudaFuncSetAttribute(m1_fwd_kernel<T, kN, kConv>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int64_t per_group = p.D / p.G;
   dim3 grid((unsigned)(p.G * ((per_group + Lay::kCh - 1) / Lay::kCh)), (unsigned)p.B);
-  m1_fwd_kernel<T, kN><<<grid, Lay::kThreads, smem, s>>>(p);
+  m1_fwd_kernel<T, kN, kConv><<<grid, Lay::kThreads, smem, s>>>(p);
   return cudaGetLastError();
+}
+
+template <typename T, int kN>
+cudaError_t launch_t(const M1Params &p, cudaStream_t s) {
+  return p.conv_w ? launch_c<T, kN, true>(p, s) : launch_c<T, kN, false>(p, s);
 }
 
 template <typename T>

@@ -46,6 +46,11 @@ class SsFwdArgs(ctypes.Structure):
                 ("saved_states", _vp), ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t)]
 
 
+class SsConvArgs(ctypes.Structure):
+    _fields_ = [("struct_size", _u32), ("width", _i64), ("w", _vp), ("bias", _vp),
+                ("conv_state_in", _vp), ("conv_state_out", _vp), ("u_out", _vp)]
+
+
 class SsBwdArgs(ctypes.Structure):
     _fields_ = [("struct_size", _u32), ("io_dtype", _i32), ("batch", _i64), ("dim", _i64),
                 ("dstate", _i64), ("seqlen", _i64), ("ngroups", _i64), ("delta_softplus", _i32),
@@ -108,7 +113,8 @@ EXPORTS = ["msc_last_error", "msc_version", "msc_selective_scan_saved_states_byt
            "msc_mamba3_siso_saved_states_bytes", "msc_mamba3_siso_scan_fwd_workspace_bytes",
            "msc_mamba3_siso_scan_fwd", "msc_mamba3_siso_scan_bwd_workspace_bytes",
            "msc_mamba3_siso_scan_bwd", "msc_mamba3_siso_state_update", "msc_causal_conv1d_fwd",
-           "msc_causal_conv1d_bwd_workspace_bytes", "msc_causal_conv1d_bwd"]
+           "msc_causal_conv1d_bwd_workspace_bytes", "msc_causal_conv1d_bwd",
+           "msc_selective_scan_conv_fwd"]
 
 _lib = None
 
@@ -124,6 +130,8 @@ def lib() -> ctypes.CDLL:
         L.msc_last_error.restype = ctypes.c_char_p
         L.msc_version.restype = ctypes.c_char_p
         for name, argt in (("msc_selective_scan_fwd", [ctypes.POINTER(SsFwdArgs), _vp]),
+                           ("msc_selective_scan_conv_fwd",
+                            [ctypes.POINTER(SsFwdArgs), ctypes.POINTER(SsConvArgs), _vp]),
                            ("msc_selective_scan_bwd",
                             [ctypes.POINTER(SsBwdArgs), _vp, ctypes.c_size_t, _vp]),
                            ("msc_selective_scan_bwd_static", [ctypes.POINTER(SsBwdArgs), _vp]),
@@ -212,6 +220,44 @@ def msc_selective_scan_fwd(u, delta, A, B, C, D=None, delta_bias=None, z=None, h
     Above 64 states a workspace is needed (allocated here if not given).
 
     Returns (out, final_state, saved_states)."""
+    a, out, final_state, saved_states, ws = _ss_fwd_args(
+        u, delta, A, B, C, D, delta_bias, z, h0, delta_softplus, out, final_state, saved_states,
+        want_final_state, want_saved_states, workspace)
+    _check(lib().msc_selective_scan_fwd(ctypes.byref(a), _stream(stream)))
+    return out, final_state, saved_states
+
+
+def msc_selective_scan_conv_fwd(x, conv_w, delta, A, B, C, conv_bias=None, conv_state=None,
+                                D=None, delta_bias=None, z=None, h0=None, delta_softplus=True,
+                                want_u=True, want_conv_state=True, want_final_state=True,
+                                want_saved_states=True, u_out=None, conv_state_out=None,
+                                out=None, final_state=None, saved_states=None, workspace=None,
+                                stream=None):
+    """The causal conv1d + SiLU fused ahead of the Mamba-1 forward: x [B, D, L]
+    is the conv's input, conv_w f32 [D, W], conv_bias f32 [D], conv_state
+    f32 [B, D, W-1] (the inputs before x).
+
+    Returns (out, final_state, saved_states, u, conv_state_out); u is the
+    scan's input silu(conv(x)) (what the backward pass takes as u).  Output
+    tensors may be given (u_out, conv_state_out, out, final_state,
+    saved_states); the missing ones are allocated when wanted."""
+    a, out, final_state, saved_states, ws = _ss_fwd_args(
+        x, delta, A, B, C, D, delta_bias, z, h0, delta_softplus, out, final_state, saved_states,
+        want_final_state, want_saved_states, workspace)
+    Bsz, Dm, _L = x.shape
+    W = conv_w.shape[1]
+    u = u_out if u_out is not None else (torch.empty_like(x) if want_u else None)
+    xs_out = conv_state_out
+    if xs_out is None and want_conv_state:
+        xs_out = torch.empty((Bsz, Dm, max(W - 1, 0)), device=x.device, dtype=torch.float32)
+    c = SsConvArgs(ctypes.sizeof(SsConvArgs), W, _ptr(conv_w), _ptr(conv_bias),
+                   _ptr(conv_state), _ptr(xs_out), _ptr(u))
+    _check(lib().msc_selective_scan_conv_fwd(ctypes.byref(a), ctypes.byref(c), _stream(stream)))
+    return out, final_state, saved_states, u, xs_out
+
+
+def _ss_fwd_args(u, delta, A, B, C, D, delta_bias, z, h0, delta_softplus, out, final_state,
+                 saved_states, want_final_state, want_saved_states, workspace):
     Bsz, Dm, L = u.shape
     G, N = B.shape[1], B.shape[2]
     dev = u.device
@@ -230,8 +276,7 @@ def msc_selective_scan_fwd(u, delta, A, B, C, D=None, delta_bias=None, z=None, h
                   _ptr(z), _ptr(h0), _ptr(out), _ptr(final_state), _ptr(saved_states),
                   _ptr(workspace), workspace.numel() * workspace.element_size()
                   if workspace is not None else 0)
-    _check(lib().msc_selective_scan_fwd(ctypes.byref(a), _stream(stream)))
-    return out, final_state, saved_states
+    return a, out, final_state, saved_states, workspace
 
 
 def msc_selective_scan_bwd(u, delta, A, B, C, saved_states, dout, D=None, delta_bias=None, z=None,

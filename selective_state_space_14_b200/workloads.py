@@ -303,6 +303,32 @@ def m3su_problem(batch, nheads, headdim, dstate, ngroups=1, nangles=None, io=BF1
 
 
 # --------------------------------------------------------------------------
+# The causal conv1d ahead of the Mamba-1 scan
+# --------------------------------------------------------------------------
+@dataclass
+class M1ConvProblem:
+    """Conv + scan inputs: ``scan`` is a Mamba-1 problem whose ``u`` is the
+    conv's input x; w f32 [D, W] and bias f32 [D] are the conv's parameters."""
+    scan: M1Problem
+    width: int
+    w: np.ndarray
+    bias: np.ndarray
+
+
+def m1conv_problem(batch, dim, dstate, seqlen, width=4, io=BF16, seed=SEED_BASE + 6,
+                   ngroups=1) -> M1ConvProblem:
+    """The scan inputs of a model-shaped Mamba-1 workload, and conv weights and
+    bias drawn like a fresh depthwise Conv1d layer's: U(-1/sqrt(W), 1/sqrt(W))
+    (one input channel per group, so the fan-in is the width)."""
+    scan = m1_problem(batch, dim, dstate, seqlen, io=io, seed=seed, ngroups=ngroups, bias=True)
+    rng = np.random.Generator(np.random.PCG64(seed + 500))
+    k = 1.0 / np.sqrt(width)
+    w = _uniform(rng, -k, k, (dim, width))
+    bias = _uniform(rng, -k, k, (dim,))
+    return M1ConvProblem(scan, width, w, bias)
+
+
+# --------------------------------------------------------------------------
 # The named workloads
 # --------------------------------------------------------------------------
 WORKLOADS = {
@@ -320,6 +346,9 @@ WORKLOADS = {
     "m3su_bf16_b256_h24_p64_n64_k32_x1000": dict(kind="m3su", batch=256, nheads=24, headdim=64,
                                                  dstate=64, nangles=32, io=BF16, steps=1000,
                                                  seed=SEED_BASE + 5),
+    "m1conv_bf16_b8_d1536_n16_l2048_w4": dict(kind="m1conv", batch=8, dim=1536, dstate=16,
+                                              seqlen=2048, width=4, io=BF16,
+                                              seed=SEED_BASE + 6),
 }
 
 
@@ -338,6 +367,9 @@ def make(name: str, shard: int = 0):
                           nangles=w["nangles"], io=w["io"], seed=w["seed"])
     if kind == "su":
         return su_problem(w["batch"], w["dim"], w["dstate"], io=w["io"], seed=w["seed"])
+    if kind == "m1conv":
+        return m1conv_problem(w["batch"], w["dim"], w["dstate"], w["seqlen"], width=w["width"],
+                              io=w["io"], seed=w["seed"])
     if kind == "m3su":
         return m3su_problem(w["batch"], w["nheads"], w["headdim"], w["dstate"],
                             nangles=w["nangles"], io=w["io"], seed=w["seed"])

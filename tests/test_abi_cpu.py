@@ -250,4 +250,43 @@ def test_conv_rejects_missing_weights_and_workspace():
     fake = ctypes.c_void_p(1 << 20)
     a = _conv_args(msc.ConvBwdArgs, w=fake, x=fake, du=fake, dx=fake, dw=fake)
     assert msc.lib().msc_causal_conv1d_bwd(ctypes.byref(a), None, 0, None) == WORKSPACE
-    assert msc.msc_causal_conv1d_bwd_workspace_bytes(2, 8, 64, 4) == 4 * 2 * 8 * 8 * 5
+    # one f32 partial of (dw, dbias) per row and segment slot: one slot while a
+    # row fits 256 runs of 16 steps, at most 64 slots
+    assert msc.msc_causal_conv1d_bwd_workspace_bytes(2, 8, 64, 4) == 4 * 2 * 8 * 5
+    assert msc.msc_causal_conv1d_bwd_workspace_bytes(2, 8, 8192, 4) == 4 * 2 * 2 * 8 * 5
+    assert msc.msc_causal_conv1d_bwd_workspace_bytes(2, 8, 1 << 20, 3) == 4 * 64 * 2 * 8 * 4
+
+
+def _ss_conv_args(**kw):
+    c = msc.SsConvArgs()
+    c.struct_size = ctypes.sizeof(msc.SsConvArgs)
+    c.width = 4
+    c.w = ctypes.c_void_p(1 << 20)
+    for k, v in kw.items():
+        setattr(c, k, v)
+    return c
+
+
+@pytest.mark.parametrize("field,value,status,word", [
+    ("width", 0, UNSUPPORTED, "width"),
+    ("width", 5, UNSUPPORTED, "width"),
+    ("struct_size", 8, INVALID, "struct_size"),
+    ("w", None, INVALID, "w is NULL"),
+])
+def test_fused_conv_fwd_rejects_bad_conv_args(field, value, status, word):
+    c = _ss_conv_args(**{field: value})
+    st = msc.lib().msc_selective_scan_conv_fwd(ctypes.byref(_fwd_args()), ctypes.byref(c), None)
+    assert st == status and word in _err() and "msc_selective_scan_conv_fwd" in _err()
+
+
+def test_fused_conv_fwd_checks_scan_args_and_null_conv():
+    """A missing conv is rejected; so is a scan argument the plain forward
+    rejects (the call stops at the checks, before any launch)."""
+    st = msc.lib().msc_selective_scan_conv_fwd(ctypes.byref(_fwd_args()), None, None)
+    assert st == INVALID and "conv is NULL" in _err()
+    st = msc.lib().msc_selective_scan_conv_fwd(ctypes.byref(_fwd_args(A=None)),
+                                               ctypes.byref(_ss_conv_args()), None)
+    assert st == INVALID and "A is NULL" in _err()
+    st = msc.lib().msc_selective_scan_conv_fwd(ctypes.byref(_fwd_args(dstate=300)),
+                                               ctypes.byref(_ss_conv_args()), None)
+    assert st == UNSUPPORTED

@@ -41,6 +41,8 @@ CASES = [
     (2, 96, 1000, 4, "bf16", True, True),
     (1, 40, 257, 4, "bf16", True, False),
     (3, 24, 64, 3, "f16", True, True),
+    (2, 3, 8195, 4, "f32", True, True),      # two segments per row
+    (1, 2, 270007, 4, "bf16", True, True),   # 64 segment slots, CTAs loop
 ]
 
 
@@ -118,3 +120,123 @@ def test_conv_deterministic(msc):
     for r in runs[1:]:
         for k in ("dx", "dw", "dbias", "dconv_state_in"):
             assert torch.equal(r[k], runs[0][k]), k
+
+
+# ---------------------------------------------------------------------------
+# the conv fused ahead of the scan forward (one launch)
+FUSED_CASES = [
+    # (B, D, N, L, G, W, io, state)
+    (1, 8, 16, 1, 1, 4, "f32", False),
+    (2, 40, 16, 300, 1, 4, "f32", True),
+    (2, 72, 32, 129, 2, 3, "f32", True),
+    (1, 48, 64, 200, 1, 2, "f32", False),
+    (2, 24, 16, 70, 1, 1, "f32", False),
+    (2, 96, 16, 513, 1, 4, "bf16", True),
+    (1, 64, 128, 130, 1, 4, "bf16", True),
+    (2, 48, 16, 257, 3, 4, "f16", True),
+]
+
+
+def _fused_inputs(case, seed):
+    Bsz, Dm, N, L, G, Wd, io, state = case
+    p = W.m1_problem(Bsz, Dm, N, L, io=io, seed=seed, ngroups=G, bias=True, with_h0=state)
+    x, w, b, xs0, _ = _problem(Bsz, Dm, L, Wd, io, seed + 1, True, state)
+    return p, x, w, b, xs0
+
+
+@pytest.mark.parametrize("case", FUSED_CASES,
+                         ids=[f"B{c[0]}D{c[1]}N{c[2]}L{c[3]}G{c[4]}W{c[5]}{c[6]}"
+                              for c in FUSED_CASES])
+def test_fused_conv_scan_fwd_parity(msc, case):
+    """One launch of conv + SiLU + scan against the oracle's conv followed by
+    its scan (u rounded to the io type between them, as it is stored)."""
+    Bsz, Dm, N, L, G, Wd, io, state = case
+    p, x, w, b, xs0 = _fused_inputs(case, 40 + L)
+    a = m1_device_args(p)
+    a.pop("u")
+    out, fs, saved, u, xs = msc.msc_selective_scan_conv_fwd(
+        dev(x), dev(w), conv_bias=dev(b), conv_state=dev(xs0), **a)
+    torch.cuda.synchronize()
+    f64 = lambda a_: None if a_ is None else np.asarray(a_, np.float64)
+    u_ref, xs_ref = oracle.conv1d_fwd(x.as_f64(), f64(w), bias=f64(b), xs0=f64(xs0))
+    ra = oracle.m1_problem_args(p)
+    ra["u"] = W.store(u_ref.astype(np.float32), io).as_f64()
+    ref = oracle.m1_fwd(**ra)
+    assert_close("u", host(u), u_ref, TOL[io])
+    assert_close("out", host(out), ref["out"], TOL[io])
+    assert_close("final_state", host(fs), ref["final_state"], TOL[io])
+    if Wd > 1:
+        assert_close("conv_state_out", host(xs), xs_ref, TOL["f32"])
+
+
+@pytest.mark.parametrize("case", [FUSED_CASES[1], FUSED_CASES[5], FUSED_CASES[6], FUSED_CASES[7]],
+                         ids=["f32", "bf16", "bf16_n128", "f16_g3"])
+def test_fused_equals_unfused(msc, case):
+    """The fused forward gives, bit for bit, what the standalone conv followed
+    by the scan forward gives."""
+    Bsz, Dm, N, L, G, Wd, io, state = case
+    p, x, w, b, xs0 = _fused_inputs(case, 7)
+    a = m1_device_args(p)
+    a.pop("u")
+    out, fs, saved, u, xs = msc.msc_selective_scan_conv_fwd(
+        dev(x), dev(w), conv_bias=dev(b), conv_state=dev(xs0), **a)
+    u2, xs2 = msc.msc_causal_conv1d_fwd(dev(x), dev(w), bias=dev(b), conv_state_in=dev(xs0))
+    out2, fs2, saved2 = msc.msc_selective_scan_fwd(u=u2, **a)
+    torch.cuda.synchronize()
+    assert torch.equal(u, u2)
+    assert torch.equal(xs, xs2)
+    assert torch.equal(out, out2)
+    assert torch.equal(fs, fs2)
+    assert torch.equal(saved, saved2)
+
+
+def test_fused_conv_scan_train_step(msc):
+    """Fused forward, then the scan backward on its u and the conv backward on
+    the scan's du, against the oracle's chain."""
+    case = (2, 48, 16, 300, 1, 4, "bf16", True)
+    p, x, w, b, xs0 = _fused_inputs(case, 21)
+    a = m1_device_args(p)
+    a.pop("u")
+    out, fs, saved, u, _ = msc.msc_selective_scan_conv_fwd(
+        dev(x), dev(w), conv_bias=dev(b), conv_state=dev(xs0), **a)
+    gs = msc.msc_selective_scan_bwd(u=u, saved_states=saved, dout=dev(p.dout), **a)
+    gc = msc.msc_causal_conv1d_bwd(dev(x), dev(w), gs["du"], bias=dev(b), conv_state_in=dev(xs0))
+    torch.cuda.synchronize()
+    f64 = lambda a_: np.asarray(a_, np.float64)
+    u_ref, _ = oracle.conv1d_fwd(x.as_f64(), f64(w), bias=f64(b), xs0=f64(xs0))
+    ra = oracle.m1_problem_args(p)
+    ra["u"] = W.store(u_ref.astype(np.float32), "bf16").as_f64()
+    refg = oracle.m1_bwd(dout=p.dout.as_f64(), **ra)
+    du_stored = W.store(refg["du"].astype(np.float32), "bf16").as_f64()
+    rc = oracle.conv1d_bwd(x.as_f64(), f64(w), du_stored, bias=f64(b), xs0=f64(xs0))
+    assert_close("dA", host(gs["dA"]), refg["dA"], TOL["bf16"])
+    assert_close("dx", host(gc["dx"]), rc["dx"], TOL["bf16"])
+    assert_close("dw", host(gc["dw"]), rc["dw"], TOL["bf16"])
+    assert_close("dconv_state_in", host(gc["dconv_state_in"]), rc["dxs0"], TOL["bf16"])
+
+
+def test_fused_continuation(msc):
+    """Two fused calls chained through the conv state and the scan state equal
+    one call over both halves."""
+    case = (2, 40, 16, 256, 1, 4, "f32", False)
+    p, x, w, b, _ = _fused_inputs(case, 33)
+    a = m1_device_args(p)
+    for k in ("u", "h0"):
+        a.pop(k)
+    xd, dd, zd = dev(x), a.pop("delta"), a.pop("z")
+    Bd, Cd = a.pop("B"), a.pop("C")
+    cut = 96
+    half = lambda t, lo, hi: t[..., lo:hi].contiguous()
+    out, fs, _, _, xs = msc.msc_selective_scan_conv_fwd(xd, dev(w), dd, B=Bd, C=Cd, z=zd,
+                                                        conv_bias=dev(b), **a)
+    o1, fs1, _, _, xs1 = msc.msc_selective_scan_conv_fwd(
+        half(xd, 0, cut), dev(w), half(dd, 0, cut), B=half(Bd, 0, cut), C=half(Cd, 0, cut),
+        z=half(zd, 0, cut), conv_bias=dev(b), **a)
+    o2, fs2, _, _, xs2 = msc.msc_selective_scan_conv_fwd(
+        half(xd, cut, 256), dev(w), half(dd, cut, 256), B=half(Bd, cut, 256),
+        C=half(Cd, cut, 256), z=half(zd, cut, 256), conv_bias=dev(b), conv_state=xs1, h0=fs1,
+        **a)
+    torch.cuda.synchronize()
+    assert torch.equal(xs2, xs)
+    assert torch.allclose(torch.cat([o1, o2], dim=2), out, rtol=1e-5, atol=1e-5)
+    assert torch.allclose(fs2, fs, rtol=1e-5, atol=1e-5)
