@@ -229,6 +229,86 @@ def conv1d_bwd(x, w, du, bias=None, xs0=None):
 
 
 # ---------------------------------------------------------------------------
+# Mamba-3 SISO discretisation and BCNorm (the stages ahead of the scan)
+# ---------------------------------------------------------------------------
+# Mamba3Scratch (mamba-rs 0.4.2 src/mamba3_siso/cpu/scratch.rs) names the
+# stages: B6 "discretization" turns per-token, per-head dd_dt, dd_a, trap
+# [T * nheads] and per-token raw angles [T * n_angles] into the scan's
+# coefficients, B5 "BCNorm" normalises the raw B and C [T * ngroups *
+# d_state].  The pages print no formulas; these are the exponential-trapezoid
+# discretisation of the cited Mamba-3 paper (Lahoti et al., 2026), read in its
+# plainest form:
+#   dt    = softplus(dd_dt + dt_bias[h])
+#   A     = min(-softplus(dd_a), -A_floor)
+#   alpha = exp(dt * A)
+#   lam   = sigmoid(trap)
+#   beta  = (1 - lam) * dt * alpha      (the x_{t-1} end of the trapezoid,
+#                                        carried through one step of decay)
+#   gamma = lam * dt                    (the x_t end)
+#   theta[k] = dt * angles[k]           (per head: dt is per head)
+#   B = B_raw / sqrt(mean_n B_raw^2 + eps),  C likewise (RMS norm over
+#   d_state per (token, group), no weight)
+def _softplus(v):
+    return np.maximum(v, 0.0) + np.log1p(np.exp(-np.abs(v)))
+
+
+def _sigmoid(v):
+    return 1.0 / (1.0 + np.exp(-v))
+
+
+def m3_discretize(dd_dt, dd_a, trap, angles, B_raw, C_raw, dt_bias=None, A_floor=0.0,
+                  eps=1e-5):
+    """dd_dt, dd_a, trap [B, L, H]; angles [B, L, K]; B_raw, C_raw [B, L, G, N];
+    dt_bias [H].  Returns alpha, beta, gamma [B, L, H], theta [B, L, H, K], B, C
+    (all float64)."""
+    u = dd_dt + (0.0 if dt_bias is None else dt_bias[None, None, :])
+    dt = _softplus(u)
+    A = np.minimum(-_softplus(dd_a), -A_floor)
+    alpha = np.exp(dt * A)
+    lam = _sigmoid(trap)
+    beta = (1.0 - lam) * dt * alpha
+    gamma = lam * dt
+    theta = dt[..., None] * angles[:, :, None, :]
+    B = B_raw / np.sqrt(np.mean(B_raw * B_raw, axis=-1, keepdims=True) + eps)
+    C = C_raw / np.sqrt(np.mean(C_raw * C_raw, axis=-1, keepdims=True) + eps)
+    return dict(alpha=alpha, beta=beta, gamma=gamma, theta=theta, B=B, C=C)
+
+
+def _rms_norm_bwd(v, g, eps):
+    """Gradient of v / sqrt(mean(v^2) + eps) (last axis) for an upstream g."""
+    r = 1.0 / np.sqrt(np.mean(v * v, axis=-1, keepdims=True) + eps)
+    vh = v * r
+    return r * (g - vh * np.mean(g * vh, axis=-1, keepdims=True))
+
+
+def m3_discretize_bwd(dd_dt, dd_a, trap, angles, B_raw, C_raw, dalpha, dbeta, dgamma, dtheta,
+                      dB, dC, dt_bias=None, A_floor=0.0, eps=1e-5):
+    """Chain rule through m3_discretize for upstream gradients of its outputs.
+    Returns ddd_dt, ddd_a, dtrap [B, L, H], dangles [B, L, K], ddt_bias [H],
+    dB_raw, dC_raw [B, L, G, N]."""
+    u = dd_dt + (0.0 if dt_bias is None else dt_bias[None, None, :])
+    dt = _softplus(u)
+    sa = _softplus(dd_a)
+    clamped = -sa > -A_floor          # A = -A_floor there: no gradient to dd_a
+    A = np.where(clamped, -A_floor, -sa)
+    alpha = np.exp(dt * A)
+    lam = _sigmoid(trap)
+    # alpha reaches the loss directly and through beta
+    g_alpha = dalpha + dbeta * (1.0 - lam) * dt
+    d_dt = (g_alpha * alpha * A + dbeta * (1.0 - lam) * alpha + dgamma * lam
+            + np.sum(dtheta * angles[:, :, None, :], axis=-1))
+    d_A = g_alpha * alpha * dt
+    d_lam = dgamma * dt - dbeta * dt * alpha
+    ddd_dt = d_dt * _sigmoid(u)
+    ddd_a = np.where(clamped, 0.0, -d_A * _sigmoid(dd_a))
+    dtrap = d_lam * lam * (1.0 - lam)
+    dangles = np.sum(dtheta * dt[..., None], axis=2)
+    ddt_bias = ddd_dt.sum(axis=(0, 1))
+    return dict(ddd_dt=ddd_dt, ddd_a=ddd_a, dtrap=dtrap, dangles=dangles, ddt_bias=ddt_bias,
+                dB_raw=_rms_norm_bwd(B_raw, dB, eps), dC_raw=_rms_norm_bwd(C_raw, dC, eps))
+
+
+# ---------------------------------------------------------------------------
 # convenience: run on a generated problem (workloads.M1Problem / M3Problem)
 # ---------------------------------------------------------------------------
 def m1_problem_args(p):

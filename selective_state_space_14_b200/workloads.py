@@ -205,6 +205,41 @@ def m3_problem(batch, seqlen, nheads, headdim, dstate, ngroups=1, nangles=None, 
                      h0, dout)
 
 
+@dataclass
+class M3DiscProblem:
+    """Mamba-3 inputs before the discretisation and BCNorm stages: the scan
+    problem ``scan`` (its x, z, D, h0, dout are used; its alpha .. theta, B, C
+    are not) and the raw per-token values those stages take."""
+    scan: M3Problem
+    dd_dt: Tensor      # [B, L, H]
+    dd_a: Tensor       # [B, L, H]
+    trap: Tensor       # [B, L, H]
+    angles: Tensor     # [B, L, K]
+    B_raw: Tensor      # [B, L, G, N]
+    C_raw: Tensor      # [B, L, G, N]
+    dt_bias: np.ndarray  # float32 [H]
+    A_floor: float
+    eps: float
+
+
+def m3disc_problem(batch, seqlen, nheads, headdim, dstate, ngroups=1, nangles=None, io=F32,
+                   seed=SEED_BASE + 7, with_h0=False, A_floor=1e-4, eps=1e-5) -> M3DiscProblem:
+    """Raw projections ~ N(0, 1) (dd_dt scaled by 1/2, as Mamba-1's delta);
+    dt_bias = softplus^-1(dt0) with dt0 log-uniform on [1e-3, 1e-1], the Mamba
+    dt initialisation, so that dt starts in that range."""
+    scan = m3_problem(batch, seqlen, nheads, headdim, dstate, ngroups, nangles, io=io, seed=seed,
+                      with_h0=with_h0)
+    rng = np.random.Generator(np.random.PCG64(seed + 500))
+    Bsz, L, H, N, G, K = batch, seqlen, nheads, dstate, ngroups, scan.nangles
+    dt0 = np.exp(_uniform(rng, np.log(1e-3), np.log(1e-1), (H,)).astype(np.float64))
+    dt_bias = np.log(np.expm1(dt0)).astype(np.float32)
+    return M3DiscProblem(
+        scan, store(0.5 * _normal(rng, (Bsz, L, H)), io), store(_normal(rng, (Bsz, L, H)), io),
+        store(_normal(rng, (Bsz, L, H)), io), store(_normal(rng, (Bsz, L, K)), io),
+        store(_normal(rng, (Bsz, L, G, N)), io), store(_normal(rng, (Bsz, L, G, N)), io),
+        dt_bias, A_floor, eps)
+
+
 # --------------------------------------------------------------------------
 # Single-token state update (decode)
 # --------------------------------------------------------------------------
@@ -346,6 +381,9 @@ WORKLOADS = {
     "m3su_bf16_b256_h24_p64_n64_k32_x1000": dict(kind="m3su", batch=256, nheads=24, headdim=64,
                                                  dstate=64, nangles=32, io=BF16, steps=1000,
                                                  seed=SEED_BASE + 5),
+    "m3disc_bf16_b8_h24_p64_n64_k32_l2048": dict(kind="m3disc", batch=8, seqlen=2048,
+                                                 nheads=24, headdim=64, dstate=64, nangles=32,
+                                                 io=BF16, seed=SEED_BASE + 7),
     "m1conv_bf16_b8_d1536_n16_l2048_w4": dict(kind="m1conv", batch=8, dim=1536, dstate=16,
                                               seqlen=2048, width=4, io=BF16,
                                               seed=SEED_BASE + 6),
@@ -367,6 +405,9 @@ def make(name: str, shard: int = 0):
                           nangles=w["nangles"], io=w["io"], seed=w["seed"])
     if kind == "su":
         return su_problem(w["batch"], w["dim"], w["dstate"], io=w["io"], seed=w["seed"])
+    if kind == "m3disc":
+        return m3disc_problem(w["batch"], w["seqlen"], w["nheads"], w["headdim"], w["dstate"],
+                              nangles=w["nangles"], io=w["io"], seed=w["seed"])
     if kind == "m1conv":
         return m1conv_problem(w["batch"], w["dim"], w["dstate"], w["seqlen"], width=w["width"],
                               io=w["io"], seed=w["seed"])

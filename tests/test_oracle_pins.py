@@ -492,3 +492,128 @@ def test_conv1d_backward_finite_differences():
     for key, gk in (("x", "dx"), ("w", "dw"), ("bias", "dbias"), ("xs0", "dxs0")):
         fd = _fd(loss, args, key)
         np.testing.assert_allclose(g[gk], fd, rtol=1e-6, atol=1e-8, err_msg=key)
+
+
+# ---------------------------------------------------------------------------
+# Mamba-3 discretisation (dt, A, trap, raw angles) and BCNorm ahead of the scan
+# ---------------------------------------------------------------------------
+def _inv_softplus(v):
+    return np.log(np.expm1(v))
+
+
+def _disc_scan(x, dt, a, trap, omega, eps=0.0):
+    """The oracle's discretisation followed by its scan, for one head with
+    P = 1, N = 2 (one angle pair), raw B = C = (1, 0), D = 0, no gate."""
+    L = x.shape[0]
+    ones = np.ones((1, L, 1))
+    d = oracle.m3_discretize(ones * _inv_softplus(dt), ones * _inv_softplus(-a), ones * trap,
+                             np.full((1, L, 1), omega), np.tile([1.0, 0.0], (1, L, 1, 1)),
+                             np.tile([1.0, 0.0], (1, L, 1, 1)), eps=eps)
+    r = oracle.m3_fwd(x.reshape(1, L, 1, 1), d["B"], d["C"], d["alpha"], d["beta"], d["gamma"],
+                      d["theta"])
+    return r["out"][0, :, 0, 0]
+
+
+def _exact_rotating(s, a, omega, Om):
+    """w' = (a - i omega) w + x(s), x = sin(Om s), w(0) = 0, read out as
+    2 Re w (B = C = sqrt(2) after the norm, a pair read as one complex number;
+    the real state rotated by R(phi) is this complex state multiplied by
+    e^{i phi})."""
+    lam = a - 1j * omega
+    w = (Om * np.exp(lam * s) - Om * np.cos(Om * s) - lam * np.sin(Om * s)) / (lam ** 2 + Om ** 2)
+    return 2.0 * w.real
+
+
+@pytest.mark.parametrize("omega", [0.0, 3.0])
+def test_m3_discretisation_is_second_order(omega):
+    """With trap = 0 (lam = 1/2) the discretised scan solves the continuous
+    system to second order in dt (error / 4 when dt halves); the explicit end
+    alone (lam -> 1) is first order.  A beta without its decay factor, a theta
+    not scaled by dt or a wrong alpha breaks the order."""
+    a, Om, T = -1.0, 2.0, 2.0
+
+    def err(dt, trap):
+        L = int(round(T / dt)) + 1
+        s = dt * np.arange(L)
+        y = _disc_scan(np.sin(Om * s), dt, a, trap, omega)
+        return np.max(np.abs(y - _exact_rotating(s, a, omega, Om)))
+
+    r2 = err(0.02, 0.0) / err(0.01, 0.0)
+    assert 3.6 < r2 < 4.4, r2
+    r1 = err(0.02, 40.0) / err(0.01, 40.0)
+    assert 1.7 < r1 < 2.3, r1
+
+
+def test_m3_discretisation_trapezoid_weights():
+    """No decay (A -> 0), constant dt and unit input: S_t = dt (t + lam) per
+    state entry, so y_t = 2 dt (t + lam); lam != 1/2 tells the two ends of
+    the trapezoid apart."""
+    L, dt, trap = 20, 0.1, 1.3
+    lam = 1.0 / (1.0 + np.exp(-trap))
+    ones = np.ones((1, L, 1))
+    d = oracle.m3_discretize(ones * _inv_softplus(dt), ones * -60.0, ones * trap,
+                             np.zeros((1, L, 1)), np.tile([1.0, 0.0], (1, L, 1, 1)),
+                             np.tile([1.0, 0.0], (1, L, 1, 1)), eps=0.0)
+    r = oracle.m3_fwd(np.ones((1, L, 1, 1)), d["B"], d["C"], d["alpha"], d["beta"], d["gamma"],
+                      d["theta"])
+    np.testing.assert_allclose(r["out"][0, :, 0, 0], 2 * dt * (np.arange(L) + lam), rtol=1e-12)
+
+
+def test_m3_discretisation_floor_bias_and_norm():
+    """A_floor bounds the decay rate from below; dt_bias is a per-head shift of
+    dd_dt; BCNorm leaves unit mean square (eps = 0) and ignores the scale of
+    each raw row, but not of another row."""
+    Bsz, L, H, K, G, N = 2, 5, 3, 2, 2, 8
+    dd_dt, dd_a, trap = _rand(Bsz, L, H), _rand(Bsz, L, H), _rand(Bsz, L, H)
+    ang, Br, Cr = _rand(Bsz, L, K), _rand(Bsz, L, G, N), _rand(Bsz, L, G, N)
+    dd_a[0, 0, 0] = -60.0  # softplus ~ 0: the floor holds
+    d = oracle.m3_discretize(dd_dt, dd_a, trap, ang, Br, Cr, A_floor=0.25, eps=0.0)
+    dt = np.log1p(np.exp(dd_dt))
+    assert np.isclose(d["alpha"][0, 0, 0], np.exp(-0.25 * dt[0, 0, 0]), rtol=1e-14)
+    assert np.all(d["alpha"] <= np.exp(-0.25 * dt) * (1 + 1e-15))
+    bias = _rand(H)
+    e = oracle.m3_discretize(dd_dt - bias, dd_a, trap, ang, Br, Cr, dt_bias=bias, A_floor=0.25,
+                             eps=0.0)
+    for k in ("alpha", "beta", "gamma", "theta"):
+        np.testing.assert_allclose(e[k], d[k], rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(np.mean(d["B"] ** 2, axis=-1), 1.0, rtol=1e-13)
+    scale = np.exp(_rand(Bsz, L, G, 1))
+    f = oracle.m3_discretize(dd_dt, dd_a, trap, ang, Br * scale, Cr * scale, eps=0.0)
+    np.testing.assert_allclose(f["B"], d["B"], rtol=1e-12)
+    np.testing.assert_allclose(f["C"], d["C"], rtol=1e-12)
+    assert not np.allclose(f["B"][..., :1], (Br * scale)[..., :1] / np.sqrt(
+        np.mean(Br ** 2, axis=(-1, -2), keepdims=True)))
+
+
+def test_m3_discretisation_backward_finite_differences():
+    """Central differences of a random linear functional of every output with
+    respect to every input (with eps > 0 and a floor that clamps some
+    entries)."""
+    Bsz, L, H, K, G, N = 1, 4, 2, 2, 2, 4
+    ins = dict(dd_dt=_rand(Bsz, L, H), dd_a=_rand(Bsz, L, H) * 2.0, trap=_rand(Bsz, L, H),
+               angles=_rand(Bsz, L, K), B_raw=_rand(Bsz, L, G, N), C_raw=_rand(Bsz, L, G, N),
+               dt_bias=_rand(H))
+    ins["dd_a"][0, 0, 0] = -6.0  # clamped by the floor below
+    kw = dict(A_floor=0.05, eps=1e-3)
+    outs = oracle.m3_discretize(**ins, **kw)
+    w = {k: _rand(*v.shape) for k, v in outs.items()}
+
+    def loss(args):
+        o = oracle.m3_discretize(**args, **kw)
+        return sum(float(np.sum(w[k] * o[k])) for k in o)
+
+    g = oracle.m3_discretize_bwd(**ins, dalpha=w["alpha"], dbeta=w["beta"], dgamma=w["gamma"],
+                                 dtheta=w["theta"], dB=w["B"], dC=w["C"], **kw)
+    names = dict(dd_dt="ddd_dt", dd_a="ddd_a", trap="dtrap", angles="dangles",
+                 dt_bias="ddt_bias", B_raw="dB_raw", C_raw="dC_raw")
+    h = 1e-6
+    for name, gname in names.items():
+        fd = np.zeros_like(ins[name])
+        for i in np.ndindex(ins[name].shape):
+            plus = {k: v.copy() for k, v in ins.items()}
+            minus = {k: v.copy() for k, v in ins.items()}
+            plus[name][i] += h
+            minus[name][i] -= h
+            fd[i] = (loss(plus) - loss(minus)) / (2 * h)
+        np.testing.assert_allclose(g[gname], fd, rtol=1e-6, atol=1e-8, err_msg=name)
+    assert g["ddd_a"][0, 0, 0] == 0.0
