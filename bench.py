@@ -314,12 +314,82 @@ class M1ConvStep:
             grads=self.cgrads)
 
 
+class M3DiscStep:
+    """Device-resident Mamba-3 step from the raw projections: discretisation
+    and BCNorm, the scan forward and backward, the discretisation backward."""
+
+    def __init__(self, q, msc):
+        import torch
+        self.msc, self.q = msc, q
+        s = q.scan
+        self.raw = dict(dd_dt=to_dev(q.dd_dt), dd_a=to_dev(q.dd_a), trap=to_dev(q.trap),
+                        angles=to_dev(q.angles), B_raw=to_dev(q.B_raw), C_raw=to_dev(q.C_raw))
+        self.kw = dict(dt_bias=to_dev(q.dt_bias), A_floor=q.A_floor, eps=q.eps)
+        self.o = msc.msc_mamba3_siso_discretize(**self.raw, **self.kw)
+        self.a = dict(x=to_dev(s.x), B=self.o["B"], C=self.o["C"], alpha=self.o["alpha"],
+                      beta=self.o["beta"], gamma=self.o["gamma"], theta=self.o["theta"],
+                      D=to_dev(s.D), z=to_dev(s.z), h0=None)
+        self.dout = to_dev(s.dout)
+        self.out, _, self.saved = msc.msc_mamba3_siso_scan_fwd(**self.a)
+        self.ws = torch.empty(max(msc.msc_mamba3_siso_scan_bwd_workspace_bytes(
+            s.batch, s.seqlen, s.nheads, s.headdim, s.dstate, s.ngroups, s.nangles), 16),
+            device="cuda", dtype=torch.uint8)
+        self.gs = msc.msc_mamba3_siso_scan_bwd(**self.a, saved_states=self.saved, dout=self.dout,
+                                               workspace=self.ws)
+        self.gd = None
+        self.disc_bwd()
+
+    def disc_fwd(self):
+        self.msc.msc_mamba3_siso_discretize(**self.raw, **self.kw, outs=self.o)
+
+    def scan_fwd(self):
+        self.msc.msc_mamba3_siso_scan_fwd(**self.a, out=self.out, saved_states=self.saved)
+
+    def scan_bwd(self):
+        self.msc.msc_mamba3_siso_scan_bwd(**self.a, saved_states=self.saved, dout=self.dout,
+                                          workspace=self.ws, grads=self.gs)
+
+    def disc_bwd(self):
+        g = self.gs
+        self.gd = self.msc.msc_mamba3_siso_discretize_bwd(
+            **self.raw, dalpha=g["dalpha"], dbeta=g["dbeta"], dgamma=g["dgamma"],
+            dtheta=g["dtheta"], dB=g["dB"], dC=g["dC"], **self.kw, grads=self.gd)
+
+
+def m3disc_bytes(Bsz, L, H, N, G, K, io_bytes):
+    """Algorithmic HBM bytes of the discretisation: forward reads dd_dt, dd_a,
+    trap, angles, B_raw, C_raw and writes alpha, beta, gamma, theta, B, C (io);
+    backward reads the raw inputs (io) and the f32 upstream gradients, writes
+    f32 gradients of the raw inputs."""
+    tok = Bsz * L
+    raw = tok * (3 * H + K + 2 * G * N) * io_bytes
+    fwd = raw + tok * (3 * H + H * K + 2 * G * N) * io_bytes
+    bwd = raw + tok * (3 * H + H * K + 2 * G * N) * 4 + tok * (3 * H + K + 2 * G * N) * 4
+    return fwd, bwd
+
+
 def conv_bytes(Bsz, D, L, W, io_bytes):
     """Algorithmic HBM bytes of the standalone conv: forward reads x, writes u;
     backward reads x and du, writes dx (weights, states and the per-run dw
     partials are small and left out)."""
     n = Bsz * D * L * io_bytes
     return 2 * n, 3 * n
+
+
+def graphed(fn):
+    """fn captured once in a CUDA graph; returns its replay.  For launches
+    shorter than the Python binding's host time, so that CUDA events measure
+    the device, not the gaps between launches.  fn must allocate nothing."""
+    import torch
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        fn()
+    torch.cuda.current_stream().wait_stream(side)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    return g.replay
 
 
 def time_steps(step_fns, steps, warmup, world, sampler=None):
@@ -598,6 +668,26 @@ def extra_workloads(msc, args, world, peaks):
     except Exception as e:  # noqa: BLE001 -- report, keep the headline line
         res["m3_bf16_b8_h24_p64_n64_k32_l2048"] = dict(error=str(e)[:200])
     torch.cuda.empty_cache()
+    # Mamba-3 from the raw projections: discretisation + BCNorm around the scan
+    name = "m3disc_bf16_b8_h24_p64_n64_k32_l2048"
+    try:
+        ds = M3DiscStep(W.make(name), msc)
+        n = max(3, args.steps // 2)
+        _, (dfw, sfw, sbw, dbw) = time_steps([graphed(ds.disc_fwd), ds.scan_fwd, ds.scan_bwd,
+                                              graphed(ds.disc_bwd)], n, 3, world)
+        s = ds.q.scan
+        fb, bb = m3disc_bytes(s.batch, s.seqlen, s.nheads, s.dstate, s.ngroups, s.nangles, 2)
+        res[name] = dict(
+            disc_fwd_ms=round(dfw, 4), scan_fwd_ms=round(sfw, 4), scan_bwd_ms=round(sbw, 4),
+            disc_bwd_ms=round(dbw, 4),
+            value=round(s.token_channels / ((dfw + sfw + sbw + dbw) / 1e3), 1), unit=UNIT,
+            disc_fwd_hbm_frac=round(fb / dfw / 1e6 / peaks["hbm_gbs"], 4),
+            disc_bwd_hbm_frac=round(bb / dbw / 1e6 / peaks["hbm_gbs"], 4),
+            note="value: discretisation + scan forward + scan backward + discretisation backward")
+        del ds
+    except Exception as e:  # noqa: BLE001 -- report, keep the headline line
+        res[name] = dict(error=str(e)[:200])
+    torch.cuda.empty_cache()
     # causal conv1d (width 4) + SiLU ahead of the Mamba-1 scan, the headline's sizes
     name = "m1conv_bf16_b8_d1536_n16_l2048_w4"
     try:
@@ -607,9 +697,9 @@ def extra_workloads(msc, args, world, peaks):
         cs.scan_bwd()
         cs.conv_bwd()
         n = max(3, args.steps // 2)
-        _, (fused_ms, sbwd_ms, cbwd_ms) = time_steps([cs.fused_fwd, cs.scan_bwd, cs.conv_bwd],
-                                                     n, 3, world)
-        _, (conv_ms, sfwd_ms) = time_steps([cs.conv_fwd, cs.scan_fwd], n, 3, world)
+        _, (fused_ms, sbwd_ms, cbwd_ms) = time_steps([cs.fused_fwd, cs.scan_bwd,
+                                                      graphed(cs.conv_bwd)], n, 3, world)
+        _, (conv_ms, sfwd_ms) = time_steps([graphed(cs.conv_fwd), cs.scan_fwd], n, 3, world)
         sp = q.scan
         fb, _ = m1_bytes(sp.batch, sp.dim, sp.dstate, sp.seqlen, 2)
         cfb, cbb = conv_bytes(sp.batch, sp.dim, sp.seqlen, q.width, 2)
@@ -668,6 +758,10 @@ def run_only(args):
                 msc.msc_mamba3_siso_scan_bwd(**a, saved_states=saved, dout=dout, workspace=ws,
                                              grads=grads)
         units = m3.token_channels
+    elif phase in ("m3_disc_fwd", "m3_disc_bwd"):
+        ds = M3DiscStep(W.make(args.workload or "m3disc_bf16_b8_h24_p64_n64_k32_l2048"), msc)
+        fn = ds.disc_fwd if phase == "m3_disc_fwd" else ds.disc_bwd
+        units = ds.q.scan.token_channels
     elif phase in ("m1_conv_fwd", "conv_fwd", "conv_bwd"):
         q = W.make(args.workload or "m1conv_bf16_b8_d1536_n16_l2048_w4")
         cs = M1ConvStep(q, msc)
@@ -700,6 +794,8 @@ def run_only(args):
                                      delta_bias=bias, z=s["z"], out=out)
         units = q.batch * q.dim
     torch.cuda.synchronize()
+    if args.graph:
+        fn = graphed(fn)
     total_ms, (ms,) = time_steps([fn], args.steps, args.warmup, 1)
     print(json.dumps({"only": phase, "workload": args.workload, "ms_per_launch": round(ms, 5),
                       "units_per_s": round(units / (ms / 1e3), 1)}), flush=True)
@@ -756,9 +852,12 @@ def main():
     ap.add_argument("--no-extra", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", choices=["m1_fwd", "m1_bwd", "m3_fwd", "m3_bwd", "decode",
-                                       "m3_decode", "m1_conv_fwd", "conv_fwd", "conv_bwd"],
+                                       "m3_decode", "m1_conv_fwd", "conv_fwd", "conv_bwd",
+                                       "m3_disc_fwd", "m3_disc_bwd"],
                     help="time one phase alone (for profiling); prints no bench line")
     ap.add_argument("--workload", default=None, help="workload name for --only")
+    ap.add_argument("--graph", action="store_true",
+                    help="with --only: replay the launch from a CUDA graph (device time alone)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -466,6 +466,75 @@ typedef struct {
 
 msc_status msc_mamba3_siso_state_update(const msc_m3_su_args *args, msc_stream_t stream);
 
+/* ======================================================================
+ * Mamba-3 SISO discretisation and BCNorm (the stages ahead of the scan)
+ * ======================================================================
+ * Stage B6 "discretization" and stage B5 "BCNorm" of Mamba3Scratch (mamba-rs
+ * 0.4.2 src/mamba3_siso/cpu/scratch.rs: per-token, per-head dd_dt, dd_a,
+ * trap [T * nheads], per-token raw angles [T * n_angles], raw B and C
+ * [T * ngroups * d_state]).  The pages name the buffers but print no
+ * formulas; this library reads them as the exponential-trapezoid
+ * discretisation of the Mamba-3 paper (the README's citation), per (b, t, h):
+ *   dt    = softplus(dd_dt + dt_bias[h])
+ *   A     = min(-softplus(dd_a), -A_floor)
+ *   alpha = exp(dt A),   lam = sigmoid(trap)
+ *   beta  = (1 - lam) dt alpha,   gamma = lam dt
+ *   theta[k] = dt angles[b,t,k]            (k < K; per head through dt)
+ * and per (b, t, g):
+ *   Bm = B_raw / sqrt(mean_n B_raw^2 + eps),   Cm likewise (no weight)
+ * The outputs are the scan's inputs of the same names (io, layouts of
+ * msc_m3_fwd_args).
+ *
+ *   dd_dt, dd_a, trap         io  [B, L, H]
+ *   angles                    io  [B, L, K]      (may be NULL when K = 0)
+ *   dt_bias                   f32 [H]            optional
+ *   B_raw, C_raw              io  [B, L, G, N]
+ *   alpha, beta, gamma        io  [B, L, H]      out
+ *   theta                     io  [B, L, H, K]   out (may be NULL when K = 0)
+ *   Bm, Cm                    io  [B, L, G, N]   out
+ * Any N >= 1 and K with 2K <= N, and H (K + 2) + K <= 6144 (a token's
+ * per-head values and angle gradients are staged in shared memory); A_floor
+ * >= 0, eps >= 0 (eps > 0 unless no raw row is all zeros).
+ */
+typedef struct {
+  uint32_t struct_size;
+  int32_t io_dtype;
+  int64_t batch, seqlen, nheads, dstate, ngroups, nangles;
+  float A_floor, eps;
+  const void *dd_dt, *dd_a, *trap, *angles;
+  const float *dt_bias;    /* optional */
+  const void *B_raw, *C_raw;
+  void *alpha, *beta, *gamma, *theta, *Bm, *Cm;
+} msc_m3_disc_args;
+
+msc_status msc_mamba3_siso_discretize(const msc_m3_disc_args *args, msc_stream_t stream);
+
+/*
+ * Backward of msc_mamba3_siso_discretize for upstream f32 gradients of its
+ * outputs (as msc_mamba3_siso_scan_bwd writes them: dalpha, dbeta, dgamma
+ * [B, L, H], dtheta [B, L, H, K], dB, dC [B, L, G, N]).  Writes, all f32:
+ *   ddd_dt, ddd_a, dtrap      [B, L, H]
+ *   dangles                   [B, L, K]   sum over heads, ascending
+ *   ddt_bias                  [H]         optional; sum over (b, t) of ddd_dt
+ *   dB_raw, dC_raw            [B, L, G, N]
+ * ddd_a is 0 where A is held at -A_floor.  Every output is overwritten.
+ */
+typedef struct {
+  uint32_t struct_size;
+  int32_t io_dtype;
+  int64_t batch, seqlen, nheads, dstate, ngroups, nangles;
+  float A_floor, eps;
+  const void *dd_dt, *dd_a, *trap, *angles;
+  const float *dt_bias;    /* optional */
+  const void *B_raw, *C_raw;
+  const float *dalpha, *dbeta, *dgamma, *dtheta, *dB, *dC;
+  float *ddd_dt, *ddd_a, *dtrap, *dangles;
+  float *ddt_bias;         /* optional */
+  float *dB_raw, *dC_raw;
+} msc_m3_disc_bwd_args;
+
+msc_status msc_mamba3_siso_discretize_bwd(const msc_m3_disc_bwd_args *args, msc_stream_t stream);
+
 #ifdef __cplusplus
 } /* extern "C" */
 #endif

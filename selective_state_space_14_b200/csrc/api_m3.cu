@@ -262,4 +262,113 @@ msc_status msc_mamba3_siso_state_update(const msc_m3_su_args *a, msc_stream_t st
   return api_cuda(msc::launch_m3_state_update(p, reinterpret_cast<cudaStream_t>(stream)), fn);
 }
 
+
+}  // extern "C"
+
+namespace {
+template <typename Args>
+msc_status check_disc(const char *fn, const Args *a) {
+  if (!a) return api_fail(MSC_ERR_INVALID_ARG, "%s: args is NULL", fn);
+  if (a->struct_size < sizeof(Args))
+    return api_fail(MSC_ERR_INVALID_ARG, "%s: struct_size %u is smaller than the struct (%zu)",
+                    fn, a->struct_size, sizeof(Args));
+  if (a->io_dtype != MSC_F32 && a->io_dtype != MSC_BF16 && a->io_dtype != MSC_F16)
+    return api_fail(MSC_ERR_INVALID_ARG,
+                    "%s: io_dtype %d is not MSC_F32 (0), MSC_BF16 (1) or MSC_F16 (2)",
+                    fn, (int)a->io_dtype);
+  if (a->batch < 0 || a->seqlen < 0 || a->nheads < 1 || a->ngroups < 1 || a->dstate < 1 ||
+      a->nangles < 0)
+    return api_fail(MSC_ERR_INVALID_ARG,
+                    "%s: need batch >= 0, seqlen >= 0, nheads >= 1, ngroups >= 1, dstate >= 1, "
+                    "nangles >= 0", fn);
+  if (2 * a->nangles > a->dstate)
+    return api_fail(MSC_ERR_INVALID_ARG, "%s: 2 * nangles (%lld) exceeds dstate (%lld)", fn,
+                    (long long)(2 * a->nangles), (long long)a->dstate);
+  if (!(a->A_floor >= 0.f) || !(a->eps >= 0.f))
+    return api_fail(MSC_ERR_INVALID_ARG, "%s: A_floor and eps must be >= 0", fn);
+  // per-warp shared memory holds a token's per-head dt, its angles and (backward)
+  // its dtheta rows
+  if (a->nheads * (a->nangles + 2) + a->nangles > 6144)
+    return api_fail(MSC_ERR_UNSUPPORTED, "%s: nheads * (nangles + 2) + nangles must be <= 6144",
+                    fn);
+  if (a->batch * a->seqlen == 0) return MSC_OK;
+  M3_REQUIRE(fn, "dd_dt", a->dd_dt);
+  M3_REQUIRE(fn, "dd_a", a->dd_a);
+  M3_REQUIRE(fn, "trap", a->trap);
+  if (a->nangles > 0) M3_REQUIRE(fn, "angles", a->angles);
+  M3_OPTIONAL(fn, "dt_bias", a->dt_bias);
+  M3_REQUIRE(fn, "B_raw", a->B_raw);
+  M3_REQUIRE(fn, "C_raw", a->C_raw);
+  return MSC_OK;
+}
+
+msc::M3DiscParams disc_params(const msc_m3_disc_args *a) {
+  msc::M3DiscParams p = {};
+  p.io = a->io_dtype;
+  p.B = a->batch; p.L = a->seqlen; p.H = a->nheads; p.N = a->dstate; p.G = a->ngroups;
+  p.K = a->nangles; p.A_floor = a->A_floor; p.eps = a->eps;
+  p.dd_dt = a->dd_dt; p.dd_a = a->dd_a; p.trap = a->trap; p.angles = a->angles;
+  p.dt_bias = a->dt_bias; p.B_raw = a->B_raw; p.C_raw = a->C_raw;
+  return p;
+}
+}  // namespace
+
+extern "C" {
+
+msc_status msc_mamba3_siso_discretize(const msc_m3_disc_args *a, msc_stream_t stream) {
+  const char *fn = "msc_mamba3_siso_discretize";
+  msc_status st = check_disc(fn, a);
+  if (st != MSC_OK) return st;
+  if (a->batch * a->seqlen == 0) return api_ok();
+  M3_REQUIRE(fn, "alpha", a->alpha);
+  M3_REQUIRE(fn, "beta", a->beta);
+  M3_REQUIRE(fn, "gamma", a->gamma);
+  if (a->nangles > 0) M3_REQUIRE(fn, "theta", a->theta);
+  M3_REQUIRE(fn, "Bm", a->Bm);
+  M3_REQUIRE(fn, "Cm", a->Cm);
+  msc::M3DiscParams p = disc_params(a);
+  p.alpha = a->alpha; p.beta = a->beta; p.gamma = a->gamma; p.theta = a->theta;
+  p.Bm = a->Bm; p.Cm = a->Cm;
+  return api_cuda(msc::launch_m3_disc_fwd(p, reinterpret_cast<cudaStream_t>(stream)), fn);
+}
+
+msc_status msc_mamba3_siso_discretize_bwd(const msc_m3_disc_bwd_args *a, msc_stream_t stream) {
+  const char *fn = "msc_mamba3_siso_discretize_bwd";
+  msc_status st = check_disc(fn, a);
+  if (st != MSC_OK) return st;
+  M3_OPTIONAL(fn, "ddt_bias", a->ddt_bias);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (a->batch * a->seqlen == 0) {  // no tokens: the bias gradient is 0
+    return a->ddt_bias ? api_cuda(cudaMemsetAsync(a->ddt_bias, 0, sizeof(float) *
+                                                  (size_t)a->nheads, s), fn)
+                       : api_ok();
+  }
+  M3_REQUIRE(fn, "dalpha", a->dalpha);
+  M3_REQUIRE(fn, "dbeta", a->dbeta);
+  M3_REQUIRE(fn, "dgamma", a->dgamma);
+  M3_REQUIRE(fn, "dB", a->dB);
+  M3_REQUIRE(fn, "dC", a->dC);
+  M3_REQUIRE(fn, "ddd_dt", a->ddd_dt);
+  M3_REQUIRE(fn, "ddd_a", a->ddd_a);
+  M3_REQUIRE(fn, "dtrap", a->dtrap);
+  M3_REQUIRE(fn, "dB_raw", a->dB_raw);
+  M3_REQUIRE(fn, "dC_raw", a->dC_raw);
+  if (a->nangles > 0) {
+    M3_REQUIRE(fn, "dtheta", a->dtheta);
+    M3_REQUIRE(fn, "dangles", a->dangles);
+  }
+  msc_m3_disc_args f = {};
+  f.io_dtype = a->io_dtype;
+  f.batch = a->batch; f.seqlen = a->seqlen; f.nheads = a->nheads; f.dstate = a->dstate;
+  f.ngroups = a->ngroups; f.nangles = a->nangles; f.A_floor = a->A_floor; f.eps = a->eps;
+  f.dd_dt = a->dd_dt; f.dd_a = a->dd_a; f.trap = a->trap; f.angles = a->angles;
+  f.dt_bias = a->dt_bias; f.B_raw = a->B_raw; f.C_raw = a->C_raw;
+  msc::M3DiscParams p = disc_params(&f);
+  p.dalpha = a->dalpha; p.dbeta = a->dbeta; p.dgamma = a->dgamma; p.dtheta = a->dtheta;
+  p.dB = a->dB; p.dC = a->dC;
+  p.ddd_dt = a->ddd_dt; p.ddd_a = a->ddd_a; p.dtrap = a->dtrap; p.dangles = a->dangles;
+  p.ddt_bias = a->ddt_bias; p.dB_raw = a->dB_raw; p.dC_raw = a->dC_raw;
+  return api_cuda(msc::launch_m3_disc_bwd(p, s), fn);
+}
+
 }  // extern "C"

@@ -110,6 +110,24 @@ size_t m3_bwd_workspace_bytes(int64_t B, int64_t L, int64_t H, int64_t P, int64_
                               int64_t K);
 bool m3_supported(int64_t P, int64_t N);
 
+// Mamba-3 SISO discretisation (dd_dt, dd_a, trap, angles -> alpha, beta,
+// gamma, theta) and BCNorm (B_raw, C_raw -> Bm, Cm), and their backward
+struct M3DiscParams {
+  int io;  // msc_dtype
+  int64_t B, L, H, N, G, K;
+  float A_floor, eps;
+  const void *dd_dt, *dd_a, *trap, *angles;  // io [B, L, H] x3, [B, L, K]
+  const float *dt_bias;                      // [H] or null
+  const void *B_raw, *C_raw;                 // io [B, L, G, N]
+  // forward outputs (io)
+  void *alpha, *beta, *gamma, *theta, *Bm, *Cm;
+  // backward: upstream f32 gradients and f32 results
+  const float *dalpha, *dbeta, *dgamma, *dtheta, *dB, *dC;
+  float *ddd_dt, *ddd_a, *dtrap, *dangles, *ddt_bias, *dB_raw, *dC_raw;
+};
+cudaError_t launch_m3_disc_fwd(const M3DiscParams &p, cudaStream_t s);
+cudaError_t launch_m3_disc_bwd(const M3DiscParams &p, cudaStream_t s);
+
 // causal depthwise conv1d + SiLU ahead of the Mamba-1 scan
 struct ConvParams {
   int io;  // msc_dtype

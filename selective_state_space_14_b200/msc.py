@@ -94,6 +94,26 @@ class M3SuArgs(ctypes.Structure):
                 ("gamma", _vp), ("theta", _vp), ("D", _vp), ("out", _vp)]
 
 
+class M3DiscArgs(ctypes.Structure):
+    _fields_ = [("struct_size", _u32), ("io_dtype", _i32), ("batch", _i64), ("seqlen", _i64),
+                ("nheads", _i64), ("dstate", _i64), ("ngroups", _i64), ("nangles", _i64),
+                ("A_floor", ctypes.c_float), ("eps", ctypes.c_float), ("dd_dt", _vp),
+                ("dd_a", _vp), ("trap", _vp), ("angles", _vp), ("dt_bias", _vp),
+                ("B_raw", _vp), ("C_raw", _vp), ("alpha", _vp), ("beta", _vp), ("gamma", _vp),
+                ("theta", _vp), ("Bm", _vp), ("Cm", _vp)]
+
+
+class M3DiscBwdArgs(ctypes.Structure):
+    _fields_ = [("struct_size", _u32), ("io_dtype", _i32), ("batch", _i64), ("seqlen", _i64),
+                ("nheads", _i64), ("dstate", _i64), ("ngroups", _i64), ("nangles", _i64),
+                ("A_floor", ctypes.c_float), ("eps", ctypes.c_float), ("dd_dt", _vp),
+                ("dd_a", _vp), ("trap", _vp), ("angles", _vp), ("dt_bias", _vp),
+                ("B_raw", _vp), ("C_raw", _vp), ("dalpha", _vp), ("dbeta", _vp),
+                ("dgamma", _vp), ("dtheta", _vp), ("dB", _vp), ("dC", _vp), ("ddd_dt", _vp),
+                ("ddd_a", _vp), ("dtrap", _vp), ("dangles", _vp), ("ddt_bias", _vp),
+                ("dB_raw", _vp), ("dC_raw", _vp)]
+
+
 class ConvFwdArgs(ctypes.Structure):
     _fields_ = [("struct_size", _u32), ("io_dtype", _i32), ("batch", _i64), ("dim", _i64),
                 ("seqlen", _i64), ("width", _i64), ("x", _vp), ("w", _vp), ("bias", _vp),
@@ -114,7 +134,8 @@ EXPORTS = ["msc_last_error", "msc_version", "msc_selective_scan_saved_states_byt
            "msc_mamba3_siso_scan_fwd", "msc_mamba3_siso_scan_bwd_workspace_bytes",
            "msc_mamba3_siso_scan_bwd", "msc_mamba3_siso_state_update", "msc_causal_conv1d_fwd",
            "msc_causal_conv1d_bwd_workspace_bytes", "msc_causal_conv1d_bwd",
-           "msc_selective_scan_conv_fwd"]
+           "msc_selective_scan_conv_fwd", "msc_mamba3_siso_discretize",
+           "msc_mamba3_siso_discretize_bwd"]
 
 _lib = None
 
@@ -140,6 +161,9 @@ def lib() -> ctypes.CDLL:
                            ("msc_mamba3_siso_scan_bwd",
                             [ctypes.POINTER(M3BwdArgs), _vp, ctypes.c_size_t, _vp]),
                            ("msc_mamba3_siso_state_update", [ctypes.POINTER(M3SuArgs), _vp]),
+                           ("msc_mamba3_siso_discretize", [ctypes.POINTER(M3DiscArgs), _vp]),
+                           ("msc_mamba3_siso_discretize_bwd",
+                            [ctypes.POINTER(M3DiscBwdArgs), _vp]),
                            ("msc_causal_conv1d_fwd", [ctypes.POINTER(ConvFwdArgs), _vp]),
                            ("msc_causal_conv1d_bwd",
                             [ctypes.POINTER(ConvBwdArgs), _vp, ctypes.c_size_t, _vp])):
@@ -477,6 +501,66 @@ def msc_mamba3_siso_state_update(state, x_prev, bt_prev, phi, x, B, C, alpha, be
     return out
 
 
+def msc_mamba3_siso_discretize(dd_dt, dd_a, trap, angles, B_raw, C_raw, dt_bias=None,
+                               A_floor=1e-4, eps=1e-5, outs=None, stream=None):
+    """Discretisation and BCNorm ahead of the Mamba-3 scan.  dd_dt, dd_a, trap
+    [B, L, H]; angles [B, L, K]; B_raw, C_raw [B, L, G, N] (io); dt_bias f32 [H].
+    Returns dict alpha, beta, gamma, theta, B, C (io, the scan's inputs)."""
+    Bsz, L, H = dd_dt.shape
+    G, N = B_raw.shape[2], B_raw.shape[3]
+    K = angles.shape[2] if angles is not None else 0
+    o = dict(outs or {})
+    for k in ("alpha", "beta", "gamma"):
+        if k not in o:
+            o[k] = torch.empty_like(dd_dt)
+    if "theta" not in o:
+        o["theta"] = torch.empty((Bsz, L, H, K), device=dd_dt.device, dtype=dd_dt.dtype)
+    if "B" not in o:
+        o["B"] = torch.empty_like(B_raw)
+    if "C" not in o:
+        o["C"] = torch.empty_like(C_raw)
+    a = M3DiscArgs(ctypes.sizeof(M3DiscArgs), _io(dd_dt), Bsz, L, H, N, G, K, A_floor, eps,
+                   _ptr(dd_dt), _ptr(dd_a), _ptr(trap), _ptr(angles) if K > 0 else None,
+                   _ptr(dt_bias), _ptr(B_raw), _ptr(C_raw), _ptr(o["alpha"]), _ptr(o["beta"]),
+                   _ptr(o["gamma"]), _ptr(o["theta"]) if K > 0 else None, _ptr(o["B"]),
+                   _ptr(o["C"]))
+    _check(lib().msc_mamba3_siso_discretize(ctypes.byref(a), _stream(stream)))
+    return o
+
+
+def msc_mamba3_siso_discretize_bwd(dd_dt, dd_a, trap, angles, B_raw, C_raw, dalpha, dbeta,
+                                   dgamma, dtheta, dB, dC, dt_bias=None, A_floor=1e-4,
+                                   eps=1e-5, want_ddt_bias=True, grads=None, stream=None):
+    """Backward of msc_mamba3_siso_discretize for f32 upstream gradients (as the
+    scan backward returns them).  Returns dict ddd_dt, ddd_a, dtrap, dangles,
+    ddt_bias, dB_raw, dC_raw (f32)."""
+    Bsz, L, H = dd_dt.shape
+    G, N = B_raw.shape[2], B_raw.shape[3]
+    K = angles.shape[2] if angles is not None else 0
+    f32 = dict(device=dd_dt.device, dtype=torch.float32)
+    g = dict(grads or {})
+    for k in ("ddd_dt", "ddd_a", "dtrap"):
+        if k not in g:
+            g[k] = torch.empty((Bsz, L, H), **f32)
+    if "dangles" not in g:
+        g["dangles"] = torch.empty((Bsz, L, K), **f32)
+    if "ddt_bias" not in g:
+        g["ddt_bias"] = torch.empty((H,), **f32) if want_ddt_bias else None
+    if "dB_raw" not in g:
+        g["dB_raw"] = torch.empty((Bsz, L, G, N), **f32)
+    if "dC_raw" not in g:
+        g["dC_raw"] = torch.empty((Bsz, L, G, N), **f32)
+    a = M3DiscBwdArgs(ctypes.sizeof(M3DiscBwdArgs), _io(dd_dt), Bsz, L, H, N, G, K, A_floor,
+                      eps, _ptr(dd_dt), _ptr(dd_a), _ptr(trap), _ptr(angles) if K > 0 else None,
+                      _ptr(dt_bias), _ptr(B_raw), _ptr(C_raw), _ptr(dalpha), _ptr(dbeta),
+                      _ptr(dgamma), _ptr(dtheta) if K > 0 else None, _ptr(dB), _ptr(dC),
+                      _ptr(g["ddd_dt"]), _ptr(g["ddd_a"]), _ptr(g["dtrap"]),
+                      _ptr(g["dangles"]) if K > 0 else None, _ptr(g["ddt_bias"]),
+                      _ptr(g["dB_raw"]), _ptr(g["dC_raw"]))
+    _check(lib().msc_mamba3_siso_discretize_bwd(ctypes.byref(a), _stream(stream)))
+    return g
+
+
 # ---------------------------------------------------------------------------
 # causal conv1d + SiLU ahead of the Mamba-1 scan
 # ---------------------------------------------------------------------------
@@ -508,11 +592,15 @@ def msc_causal_conv1d_bwd(x, w, du, bias=None, conv_state_in=None, workspace=Non
     W = w.shape[1]
     f32 = dict(device=x.device, dtype=torch.float32)
     g = dict(grads or {})
-    g.setdefault("dx", torch.empty_like(x))
-    g.setdefault("dw", torch.empty((Dm, W), **f32))
-    g.setdefault("dbias", torch.empty((Dm,), **f32) if bias is not None else None)
-    g.setdefault("dconv_state_in", torch.empty((Bsz, Dm, W - 1), **f32)
-                 if want_dstate and W > 1 else None)
+    if "dx" not in g:
+        g["dx"] = torch.empty_like(x)
+    if "dw" not in g:
+        g["dw"] = torch.empty((Dm, W), **f32)
+    if "dbias" not in g:
+        g["dbias"] = torch.empty((Dm,), **f32) if bias is not None else None
+    if "dconv_state_in" not in g:
+        g["dconv_state_in"] = (torch.empty((Bsz, Dm, W - 1), **f32)
+                               if want_dstate and W > 1 else None)
     if workspace is None:
         need = msc_causal_conv1d_bwd_workspace_bytes(Bsz, Dm, L, W)
         workspace = torch.empty(max(need, 16), device=x.device, dtype=torch.uint8)

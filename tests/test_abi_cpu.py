@@ -290,3 +290,48 @@ def test_fused_conv_fwd_checks_scan_args_and_null_conv():
     st = msc.lib().msc_selective_scan_conv_fwd(ctypes.byref(_fwd_args(dstate=300)),
                                                ctypes.byref(_ss_conv_args()), None)
     assert st == UNSUPPORTED
+
+
+def _disc_args(cls=None, **kw):
+    cls = cls or msc.M3DiscArgs
+    a = cls()
+    a.struct_size = ctypes.sizeof(cls)
+    a.io_dtype, a.batch, a.seqlen, a.nheads, a.dstate, a.ngroups, a.nangles = (
+        msc.MSC_BF16, 2, 64, 4, 64, 1, 32)
+    a.A_floor, a.eps = 1e-4, 1e-5
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("field,value,status,word", [
+    ("struct_size", 8, INVALID, "struct_size"),
+    ("io_dtype", 7, INVALID, "io_dtype"),
+    ("nheads", 0, INVALID, "nheads"),
+    ("nangles", 33, INVALID, "nangles"),
+    ("eps", -1.0, INVALID, "eps"),
+    ("nheads", 200, UNSUPPORTED, "6144"),
+])
+def test_disc_rejects_bad_sizes(field, value, status, word):
+    for fn, cls in (("msc_mamba3_siso_discretize", msc.M3DiscArgs),
+                    ("msc_mamba3_siso_discretize_bwd", msc.M3DiscBwdArgs)):
+        st = getattr(msc.lib(), fn)(ctypes.byref(_disc_args(cls, **{field: value})), None)
+        assert st == status and word in _err() and fn in _err()
+
+
+def test_disc_rejects_missing_pointers():
+    """Inputs, outputs and upstream gradients are required (the calls stop at
+    the checks, before any launch); no tokens is a no-op."""
+    fake = ctypes.c_void_p(1 << 20)
+    st = msc.lib().msc_mamba3_siso_discretize(ctypes.byref(_disc_args()), None)
+    assert st == INVALID and "dd_dt is NULL" in _err()
+    a = _disc_args(dd_dt=fake, dd_a=fake, trap=fake, angles=fake, B_raw=fake, C_raw=fake)
+    assert msc.lib().msc_mamba3_siso_discretize(ctypes.byref(a), None) == INVALID
+    assert "alpha is NULL" in _err()
+    a.angles = ctypes.c_void_p((1 << 20) + 4)
+    assert msc.lib().msc_mamba3_siso_discretize(ctypes.byref(a), None) == ALIGNMENT
+    b = _disc_args(msc.M3DiscBwdArgs, dd_dt=fake, dd_a=fake, trap=fake, angles=fake, B_raw=fake,
+                   C_raw=fake, dalpha=fake, dbeta=fake, dgamma=fake, dB=fake, dC=fake)
+    assert msc.lib().msc_mamba3_siso_discretize_bwd(ctypes.byref(b), None) == INVALID
+    assert "ddd_dt is NULL" in _err()
+    assert msc.lib().msc_mamba3_siso_discretize(ctypes.byref(_disc_args(batch=0)), None) == OK

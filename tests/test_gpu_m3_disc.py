@@ -1,0 +1,146 @@
+"""GPU parity of the Mamba-3 discretisation and BCNorm stages (forward and
+backward) against the f64 oracle, through the C ABI, and chained with the
+scan: raw projections -> discretisation -> scan -> scan backward ->
+discretisation backward."""
+import numpy as np
+import pytest
+
+import oracle
+from selective_state_space_14_b200 import workloads as W
+from tests._util import TOL, assert_close, dev, host
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+DISC_OUT = ("alpha", "beta", "gamma", "theta", "B", "C")
+DISC_GRADS = ("ddd_dt", "ddd_a", "dtrap", "dangles", "ddt_bias", "dB_raw", "dC_raw")
+
+
+@pytest.fixture(scope="module")
+def msc():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from selective_state_space_14_b200 import msc as m
+    m.lib()
+    return m
+
+
+def _raw(q):
+    return dict(dd_dt=q.dd_dt, dd_a=q.dd_a, trap=q.trap, angles=q.angles, B_raw=q.B_raw,
+                C_raw=q.C_raw)
+
+
+def _oracle_raw(q, bias=True):
+    a = {k: v.as_f64() for k, v in _raw(q).items()}
+    a["dt_bias"] = q.dt_bias.astype(np.float64) if bias else None
+    return a
+
+
+CASES = [
+    # (B, L, H, N, G, K, io, bias, A_floor)
+    (1, 1, 1, 16, 1, 8, "f32", True, 1e-4),
+    (2, 37, 3, 16, 1, 8, "f32", True, 0.3),      # the floor holds for part of the entries
+    (1, 70, 40, 64, 2, 32, "f32", False, 1e-4),  # more heads than lanes
+    (2, 33, 4, 17, 1, 3, "f32", True, 1e-4),     # odd d_state
+    (1, 20, 2, 32, 2, 0, "f32", True, 1e-4),     # no angles
+    (2, 130, 24, 64, 1, 32, "bf16", True, 1e-4),
+    (1, 65, 6, 128, 3, 64, "bf16", True, 1e-4),
+    (2, 48, 8, 64, 2, 16, "f16", True, 1e-4),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=[f"B{c[0]}L{c[1]}H{c[2]}N{c[3]}G{c[4]}K{c[5]}{c[6]}"
+                                             for c in CASES])
+def test_disc_fwd_bwd_parity(msc, case):
+    Bsz, L, H, N, G, K, io, bias, A_floor = case
+    q = W.m3disc_problem(Bsz, L, H, 16, N, ngroups=G, nangles=K, io=io, seed=L + H,
+                         A_floor=A_floor)
+    d = {k: dev(v) for k, v in _raw(q).items()}
+    if K == 0:
+        d["angles"] = None
+    dtb = dev(q.dt_bias) if bias else None
+    o = msc.msc_mamba3_siso_discretize(**d, dt_bias=dtb, A_floor=A_floor, eps=q.eps)
+    rng = np.random.default_rng(L)
+    up = dict(dalpha=rng.standard_normal((Bsz, L, H)), dbeta=rng.standard_normal((Bsz, L, H)),
+              dgamma=rng.standard_normal((Bsz, L, H)),
+              dtheta=rng.standard_normal((Bsz, L, H, K)),
+              dB=rng.standard_normal((Bsz, L, G, N)), dC=rng.standard_normal((Bsz, L, G, N)))
+    up = {k: v.astype(np.float32) for k, v in up.items()}
+    g = msc.msc_mamba3_siso_discretize_bwd(**d, **{k: dev(v) for k, v in up.items()},
+                                           dt_bias=dtb, A_floor=A_floor, eps=q.eps)
+    torch.cuda.synchronize()
+    ra = _oracle_raw(q, bias)
+    ref = oracle.m3_discretize(**ra, A_floor=A_floor, eps=q.eps)
+    refg = oracle.m3_discretize_bwd(**ra, **{k: v.astype(np.float64) for k, v in up.items()},
+                                    A_floor=A_floor, eps=q.eps)
+    for k in DISC_OUT:
+        assert_close(k, host(o[k]), ref[k], TOL[io])
+    # the gradients are f32 from io-rounded inputs: f32 arithmetic throughout
+    for k in DISC_GRADS:
+        assert_close(k, host(g[k]), refg[k], TOL["f32"])
+
+
+def test_disc_chained_with_the_scan(msc):
+    """Raw projections through the discretisation, the scan forward and
+    backward, and the discretisation backward, against the oracle's chain (the
+    scan consuming the discretised values as the io dtype stores them)."""
+    q = W.m3disc_problem(2, 130, 4, 32, 64, nangles=32, io="bf16", seed=5, with_h0=True)
+    s = q.scan
+    d = {k: dev(v) for k, v in _raw(q).items()}
+    o = msc.msc_mamba3_siso_discretize(**d, dt_bias=dev(q.dt_bias), A_floor=q.A_floor, eps=q.eps)
+    a = dict(x=dev(s.x), B=o["B"], C=o["C"], alpha=o["alpha"], beta=o["beta"], gamma=o["gamma"],
+             theta=o["theta"], D=dev(s.D), z=dev(s.z), h0=dev(s.h0))
+    out, fs, saved = msc.msc_mamba3_siso_scan_fwd(**a)
+    gs = msc.msc_mamba3_siso_scan_bwd(**a, saved_states=saved, dout=dev(s.dout))
+    g = msc.msc_mamba3_siso_discretize_bwd(**d, dalpha=gs["dalpha"], dbeta=gs["dbeta"],
+                                           dgamma=gs["dgamma"], dtheta=gs["dtheta"], dB=gs["dB"],
+                                           dC=gs["dC"], dt_bias=dev(q.dt_bias), A_floor=q.A_floor,
+                                           eps=q.eps)
+    torch.cuda.synchronize()
+    ra = _oracle_raw(q)
+    disc = oracle.m3_discretize(**ra, A_floor=q.A_floor, eps=q.eps)
+    stored = {k: W.store(v.astype(np.float32), "bf16").as_f64() for k, v in disc.items()}
+    f64 = lambda a_: None if a_ is None else np.asarray(a_, np.float64)
+    sa = dict(x=s.x.as_f64(), B=stored["B"], C=stored["C"], alpha=stored["alpha"],
+              beta=stored["beta"], gamma=stored["gamma"], theta=stored["theta"], D=f64(s.D),
+              z=s.z.as_f64(), h0=f64(s.h0))
+    ref = oracle.m3_fwd(**sa)
+    refs = oracle.m3_bwd(**sa, dout=s.dout.as_f64())
+    refg = oracle.m3_discretize_bwd(**ra, dalpha=refs["dalpha"], dbeta=refs["dbeta"],
+                                    dgamma=refs["dgamma"], dtheta=refs["dtheta"], dB=refs["dB"],
+                                    dC=refs["dC"], A_floor=q.A_floor, eps=q.eps)
+    assert_close("out", host(out), ref["out"], TOL["bf16"])
+    for k in DISC_GRADS:
+        assert_close(k, host(g[k]), refg[k], TOL["bf16"])
+
+
+def test_disc_full_size_sampled(msc):
+    """The full-size workload (B8 L2048 H24 N64 K32, bf16) through the launch
+    the bench times; a sample of tokens against the oracle (tokens are
+    independent in the forward, so the sample is exact)."""
+    q = W.make("m3disc_bf16_b8_h24_p64_n64_k32_l2048")
+    d = {k: dev(v) for k, v in _raw(q).items()}
+    o = msc.msc_mamba3_siso_discretize(**d, dt_bias=dev(q.dt_bias), A_floor=q.A_floor, eps=q.eps)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(1)
+    bs, ts = rng.integers(0, 8, 64), rng.integers(0, 2048, 64)
+    ra = {k: v[bs, ts][:, None] for k, v in _oracle_raw(q).items() if k != "dt_bias"}
+    ref = oracle.m3_discretize(**ra, dt_bias=q.dt_bias.astype(np.float64), A_floor=q.A_floor,
+                               eps=q.eps)
+    for k in DISC_OUT:
+        got = host(o[k])[bs, ts][:, None]
+        assert_close(k, got, ref[k], TOL["bf16"])
+
+
+def test_disc_bwd_deterministic(msc):
+    q = W.m3disc_problem(4, 512, 24, 16, 64, nangles=32, io="bf16", seed=3)
+    d = {k: dev(v) for k, v in _raw(q).items()}
+    gen = torch.Generator(device="cuda").manual_seed(0)
+    sh = dict(dalpha=(4, 512, 24), dbeta=(4, 512, 24), dgamma=(4, 512, 24),
+              dtheta=(4, 512, 24, 32), dB=(4, 512, 1, 64), dC=(4, 512, 1, 64))
+    up = {k: torch.randn(v, device="cuda", generator=gen) for k, v in sh.items()}
+    runs = [msc.msc_mamba3_siso_discretize_bwd(**d, **up, dt_bias=dev(q.dt_bias)) for _ in range(3)]
+    torch.cuda.synchronize()
+    for r in runs[1:]:
+        for k in DISC_GRADS:
+            assert torch.equal(r[k], runs[0][k]), k
