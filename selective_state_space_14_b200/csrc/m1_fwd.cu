@@ -46,12 +46,17 @@ struct FwdSmem {
   static constexpr int ytile = bc + kTF * kP * 4;             // [kWarps][32/kP][kChBlock]
   static constexpr int out = ytile + kWarps * (32 / kP) * kChBlock;  // [kCh][kOut]
   static constexpr int gate = out + kCh * kOut;               // [kCh][kOut] silu(z), last slab
-  // with the conv fused ahead: [2][kCh][4] conv inputs before a chunk and
-  // [2][kCh][kOut] the conv's output u (a chunk's tile is stored out with the
-  // chunk's outputs, while the next chunk fills the other one)
+  // with the conv fused ahead: [2][kCh][4] conv inputs before a chunk,
+  // [kCh][8] the conv's taps (4, right-aligned: a width-W conv uses taps
+  // 4-W..3) and bias, and [2][kCh][kUOut] the conv's output u (a chunk's tile
+  // is stored out with the chunk's outputs, while the next chunk fills the
+  // other one; the stride of 36 floats makes a warp's 16-byte stores and
+  // loads conflict-free)
+  static constexpr int kUOut = kTF + 4;
   static constexpr int halo = gate + kCh * kOut;
-  static constexpr int su = halo + (kConv ? 2 * kCh * 4 : 0);
-  static constexpr int raw = (su + (kConv ? 2 * kCh * kOut : 0) + 3) / 4 * 4;  // 16-byte aligned
+  static constexpr int cw = halo + (kConv ? 2 * kCh * 4 : 0);
+  static constexpr int su = cw + (kConv ? kCh * 8 : 0);
+  static constexpr int raw = (su + (kConv ? 2 * kCh * kUOut : 0) + 3) / 4 * 4;  // 16-byte aligned
   static constexpr int total_floats = raw;
 };
 
@@ -129,7 +134,7 @@ __device__ __forceinline__ void fwd_issue_raw(const M1Params &p, unsigned char *
 // d_state: the gated outputs.  Slabs: the first writes its sums over its
 // states to tok_part (f32), a middle one adds to them, the last adds them to
 // its own and stores the gated outputs.
-template <typename T, int kCh, int kOut>
+template <typename T, int kCh, int kOut, int kUOut>
 __device__ __forceinline__ void store_chunk(const M1Params &p, const float *sout,
                                             const float *sgate, const float *su,
                                             int64_t c_first, int64_t c_end, int64_t b,
@@ -145,8 +150,8 @@ __device__ __forceinline__ void store_chunk(const M1Params &p, const float *sout
     float v[8] = {a.x, a.y, a.z, a.w, e.x, e.y, e.z, e.w};
     const int64_t row = (b * D + c) * L, t0 = tc + seg * 8;
     if (su) {  // the conv's output u (exact: values already rounded to T)
-      const float4 ua = *reinterpret_cast<const float4 *>(su + chl * kOut + seg * 8);
-      const float4 ue = *reinterpret_cast<const float4 *>(su + chl * kOut + seg * 8 + 4);
+      const float4 ua = *reinterpret_cast<const float4 *>(su + chl * kUOut + seg * 8);
+      const float4 ue = *reinterpret_cast<const float4 *>(su + chl * kUOut + seg * 8 + 4);
       const float uv[8] = {ua.x, ua.y, ua.z, ua.w, ue.x, ue.y, ue.z, ue.w};
       store_run<8>(static_cast<T *>(p.u_out) + row, t0, L, p.vec, uv);
     }
@@ -252,6 +257,16 @@ __global__ void __launch_bounds__(kWarps * 32, 6) m1_fwd_kernel(const M1Params p
         v = p.conv_xs_in[(b * D + cc) * (Wd - 1) + (Wd - 1) + pos];
       sHalo[cl * 4 + k] = v;
     }
+    for (int i = tid; i < kCh * 5; i += kThreads) {  // taps right-aligned, then the bias
+      const int cl = i / 5, k = i % 5, k0 = 4 - Wd;
+      const int64_t cc = c_first + cl;
+      float v = 0.f;
+      if (cc < c_end) {
+        if (k == 4) v = p.conv_b ? p.conv_b[cc] : 0.f;
+        else if (k >= k0) v = p.conv_w[cc * Wd + k - k0];
+      }
+      smem[S::cw + cl * 8 + k] = v;
+    }
   }
   __syncthreads();
   fwd_issue_raw<T, kN>(p, raw, rows, 0, tid);
@@ -260,9 +275,9 @@ __global__ void __launch_bounds__(kWarps * 32, 6) m1_fwd_kernel(const M1Params p
     cp_async_wait<0>();
     __syncthreads();  // this chunk's raw inputs are in; the last chunk is done
     if (ch > 0)
-      store_chunk<T, kCh, S::kOut>(p, sOut, sGate,
-                                   kConv && p.u_out ? smem + S::su + ((ch - 1) & 1) * kCh * S::kOut
-                                                    : nullptr,
+      store_chunk<T, kCh, S::kOut, S::kUOut>(
+          p, sOut, sGate,
+          kConv && p.u_out ? smem + S::su + ((ch - 1) & 1) * kCh * S::kUOut : nullptr,
                                    c_first, c_end, b, tc - kTF, tid, kThreads);
     if (ch == n_chunks) break;
     // ---- per-token values: kRun steps of one channel per thread ---------------
@@ -282,18 +297,35 @@ __global__ void __launch_bounds__(kWarps * 32, 6) m1_fwd_kernel(const M1Params p
         // next chunk's halo (other parity: this chunk's halo is still read)
         const float *hl = sHalo + ((ch & 1) * kCh + tcl) * 4;  // x at tc-3 .. tc-1
         float xs[kRun + 3];  // x at tseg*kRun - 3 .. tseg*kRun + kRun - 1
+        if constexpr (kRun == 4 && sizeof(T) == 2) {
+          // this run and the run before it, 8 bytes each (rows and runs are
+          // 8-byte aligned); the first run takes the chunk's halo
+          const T *row = ru + tcl * R::kTokRow + tseg * 4;
+          float prev[4];
+          const uint2 w1 = *reinterpret_cast<const uint2 *>(row);
+          if (tseg > 0) {
+            const uint2 w0 = *reinterpret_cast<const uint2 *>(row - 4);
+            unpack2<T>(w0.x, prev[0], prev[1]);
+            unpack2<T>(w0.y, prev[2], prev[3]);
+          } else {
+            prev[1] = hl[0]; prev[2] = hl[1]; prev[3] = hl[2];
+          }
+          xs[0] = prev[1]; xs[1] = prev[2]; xs[2] = prev[3];
+          unpack2<T>(w1.x, xs[3], xs[4]);
+          unpack2<T>(w1.y, xs[5], xs[6]);
+        } else {
 #pragma unroll
-        for (int j = 0; j < kRun + 3; ++j) {
-          const int pos = tseg * kRun - 3 + j;
-          xs[j] = pos >= 0 ? to_f32(ru[tcl * R::kTokRow + pos]) : hl[pos + 3];
+          for (int j = 0; j < kRun + 3; ++j) {
+            const int pos = tseg * kRun - 3 + j;
+            xs[j] = pos >= 0 ? to_f32(ru[tcl * R::kTokRow + pos]) : hl[pos + 3];
+          }
         }
         // tap k of 4 meets x at t-3+k; a width-W conv uses taps 4-W .. 3 (the
         // taps stay compile-time indexes: xs lives in registers)
-        const int Wd = (int)p.conv_W, k0 = 4 - Wd;
-        float wv[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) wv[k] = (tact && k >= k0) ? p.conv_w[tcc * Wd + k - k0] : 0.f;
-        const float cb = (tact && p.conv_b) ? p.conv_b[tcc] : 0.f;
+        const int k0 = 4 - (int)p.conv_W;
+        const float4 wq = *reinterpret_cast<const float4 *>(smem + S::cw + tcl * 8);
+        const float wv[4] = {wq.x, wq.y, wq.z, wq.w};
+        const float cb = smem[S::cw + tcl * 8 + 4];
 #pragma unroll
         for (int i = 0; i < kRun; ++i) {
           float a = cb;
@@ -302,7 +334,13 @@ __global__ void __launch_bounds__(kWarps * 32, 6) m1_fwd_kernel(const M1Params p
             if (k >= k0) a = fmaf(wv[k], xs[i + k], a);
           // u rounded to the io type, as the unfused conv would store it
           x[i] = to_f32(from_f32<T>(silu(a)));
-          smem[S::su + ((ch & 1) * kCh + tcl) * S::kOut + tseg * kRun + i] = x[i];
+        }
+        float *ud = smem + S::su + ((ch & 1) * kCh + tcl) * S::kUOut + tseg * kRun;
+        if constexpr (kRun == 4) {
+          *reinterpret_cast<float4 *>(ud) = make_float4(x[0], x[1], x[2], x[3]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < kRun; ++i) ud[i] = x[i];
         }
         if (tseg == kTF / kRun - 1) {
           float *hn = sHalo + (((ch + 1) & 1) * kCh + tcl) * 4;
