@@ -240,3 +240,28 @@ def test_fused_continuation(msc):
     assert torch.equal(xs2, xs)
     assert torch.allclose(torch.cat([o1, o2], dim=2), out, rtol=1e-5, atol=1e-5)
     assert torch.allclose(fs2, fs, rtol=1e-5, atol=1e-5)
+
+
+def test_conv_workload_full_size(msc):
+    """The conv + scan workload (bf16, B8 D1536 N16 L2048, width 4) at full size
+    in the launches the bench times: the fused forward against the oracle's
+    conv followed by its scan over the whole problem, and the standalone conv
+    backward against the oracle's."""
+    q = W.make("m1conv_bf16_b8_d1536_n16_l2048_w4")
+    a = m1_device_args(q.scan)
+    x = a.pop("u")
+    out, fs, _, u, xs = msc.msc_selective_scan_conv_fwd(x, dev(q.w), conv_bias=dev(q.bias), **a)
+    g = msc.msc_causal_conv1d_bwd(x, dev(q.w), dev(q.scan.dout), bias=dev(q.bias))
+    torch.cuda.synchronize()
+    f64 = lambda a_: np.asarray(a_, np.float64)
+    u_ref, xs_ref = oracle.conv1d_fwd(q.scan.u.as_f64(), f64(q.w), bias=f64(q.bias))
+    ra = oracle.m1_problem_args(q.scan)
+    ra["u"] = W.store(u_ref.astype(np.float32), "bf16").as_f64()
+    ref = oracle.m1_fwd(**ra)
+    assert_close("u", host(u), u_ref, TOL["bf16"])
+    assert_close("out", host(out), ref["out"], TOL["bf16"])
+    assert_close("final_state", host(fs), ref["final_state"], TOL["bf16"])
+    assert_close("conv_state_out", host(xs), xs_ref, TOL["f32"])
+    rc = oracle.conv1d_bwd(q.scan.u.as_f64(), f64(q.w), q.scan.dout.as_f64(), bias=f64(q.bias))
+    for k, rk in (("dx", "dx"), ("dw", "dw"), ("dbias", "dbias")):
+        assert_close(k, host(g[k]), rc[rk], TOL["bf16"])

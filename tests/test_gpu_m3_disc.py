@@ -144,3 +144,26 @@ def test_disc_bwd_deterministic(msc):
     for r in runs[1:]:
         for k in DISC_GRADS:
             assert torch.equal(r[k], runs[0][k]), k
+
+
+def test_disc_bwd_full_size(msc):
+    """The full-size workload's discretisation backward (B8 L2048 H24 N64 K32,
+    bf16 inputs, f32 upstream gradients) against the oracle on the whole
+    problem (ddt_bias sums all 16384 tokens)."""
+    q = W.make("m3disc_bf16_b8_h24_p64_n64_k32_l2048")
+    d = {k: dev(v) for k, v in _raw(q).items()}
+    rng = np.random.default_rng(2)
+    Bsz, L, H, K, G, N = 8, 2048, 24, 32, 1, 64
+    up = dict(dalpha=rng.standard_normal((Bsz, L, H)), dbeta=rng.standard_normal((Bsz, L, H)),
+              dgamma=rng.standard_normal((Bsz, L, H)),
+              dtheta=rng.standard_normal((Bsz, L, H, K)),
+              dB=rng.standard_normal((Bsz, L, G, N)), dC=rng.standard_normal((Bsz, L, G, N)))
+    up = {k: v.astype(np.float32) for k, v in up.items()}
+    g = msc.msc_mamba3_siso_discretize_bwd(**d, **{k: dev(v) for k, v in up.items()},
+                                           dt_bias=dev(q.dt_bias), A_floor=q.A_floor, eps=q.eps)
+    torch.cuda.synchronize()
+    refg = oracle.m3_discretize_bwd(**_oracle_raw(q),
+                                    **{k: v.astype(np.float64) for k, v in up.items()},
+                                    A_floor=q.A_floor, eps=q.eps)
+    for k in DISC_GRADS:
+        assert_close(k, host(g[k]), refg[k], TOL["f32"])
