@@ -449,9 +449,25 @@ def cpu_baseline(budget_s=12.0):
         t_total += time.perf_counter() - t0
         reps += 1
     units = nch * p.seqlen * reps
+    # one host thread, forward only, on the first 128 channels of the same row
+    few = {k: (v[:, :128] if k in ("u", "delta", "z") else
+               v[:128] if k in ("A", "D", "delta_bias") else v) for k, v in args.items()}
+    t0 = time.perf_counter()
+    oracle.m1_fwd(**few, nthreads=1)
+    t1 = time.perf_counter() - t0
+    model = ""
+    try:
+        with open("/proc/cpuinfo") as f:
+            model = next((ln.split(":", 1)[1].strip() for ln in f if ln.startswith("model name")),
+                         "")
+    except OSError:
+        pass
     return dict(value=units / t_total, unit=UNIT, cores=threads, kind="oracle",
                 sample=f"batch row 0, channels 0..{nch - 1}, L={p.seqlen}, fwd+bwd, {reps} reps, "
-                       f"{t_total:.1f} s")
+                       f"{t_total:.1f} s",
+                fwd_1thread=dict(value=round(128 * p.seqlen / t1, 1), unit=UNIT,
+                                 sample=f"batch row 0, channels 0..127, L={p.seqlen}, fwd only"),
+                cpu_model=model)
 
 
 def run_e2e(p, msc, steps, warmup, world):
