@@ -470,6 +470,112 @@ def cpu_baseline(budget_s=12.0):
                 cpu_model=model)
 
 
+def _rate(fn, budget_s):
+    """Calls of fn per second over about budget_s seconds (at least one call)."""
+    reps, t = 0, 0.0
+    while reps == 0 or (t < budget_s and reps < 1000):
+        t0 = time.perf_counter()
+        fn()
+        t += time.perf_counter() - t0
+        reps += 1
+    return reps / t, reps, t
+
+
+def oracle_beside(res, budget_s=1.5):
+    """The f64 oracle, as it stands, timed on the host beside each extra
+    workload, on a bounded sample (stated): one row or sequence of the
+    workload's shape drawn with its generator and distributions, in the
+    workload's unit."""
+    import oracle
+    f64 = lambda a: None if a is None else np.asarray(a, np.float64)
+    thr = oracle.default_threads()
+    BF = "bf16"
+
+    def put(name, units_per_call, fn, sample):
+        if name not in res or "error" in res[name]:
+            return
+        r, reps, t = _rate(fn, budget_s)
+        res[name]["oracle"] = dict(value=round(units_per_call * r, 1), unit=res[name]["unit"],
+                                   cores=thr, kind="oracle",
+                                   sample=f"{sample}; {reps} reps, {t:.1f} s")
+
+    # Mamba-1, 2.8B-layer rows: one batch row of 256 channels, L 4096, fwd+bwd
+    p = W.m1_problem(1, 256, 16, 4096, io=BF, bias=True)
+    a = oracle.m1_problem_args(p)
+    dout = p.dout.as_f64()
+    put("m1_bf16_b4_d5120_n16_l4096", 256 * 4096,
+        lambda: (oracle.m1_fwd(**a), oracle.m1_bwd(dout=dout, **a)),
+        "one batch row of 256 channels, L 4096, fwd+bwd")
+    # Mamba-1 decode: 64 channels of one sequence, 10 steps
+    q = W.su_problem(1, 64, 16, n_pool=10)
+    steps = [{k: v.as_f64() for k, v in s_.items()} for s_ in q.steps]
+
+    def su():
+        st = q.state0.astype(np.float64)
+        for s_ in steps:
+            st, _ = oracle.ssm_state_update(st, s_["x"], s_["delta"], f64(q.A), s_["B"], s_["C"],
+                                            D=f64(q.D), delta_bias=f64(q.delta_bias), z=s_["z"])
+    put("su_bf16_b256_d5120_n16_x1000", 64 * 10, su, "64 channels of one sequence, 10 steps")
+    # Mamba-3 SISO: one sequence, one head (P64 N64 K32), L 2048, fwd+bwd
+    m3 = W.m3_problem(1, 2048, 1, 64, 64, nangles=32, io=BF)
+    ms = oracle.m3_problem_args(m3)
+    mdout = m3.dout.as_f64()
+    put("m3_bf16_b8_h24_p64_n64_k32_l2048", 2048 * 64,
+        lambda: (oracle.m3_fwd(**ms), oracle.m3_bwd(dout=mdout, **ms)),
+        "one sequence, one head, L 2048, fwd+bwd")
+    # Mamba-3 decode: one sequence (24 heads), 10 steps
+    q3 = W.m3su_problem(1, 24, 64, 64, nangles=32, n_pool=10)
+    st3 = [{k: v.as_f64() for k, v in s_.items()} for s_ in q3.steps]
+
+    def su3():
+        c = [v.astype(np.float64) for v in (q3.state0, q3.x_prev0, q3.bt_prev0, q3.phi0)]
+        for s_ in st3:
+            *c, _ = oracle.m3_state_update(*c, *[s_[k] for k in ("x", "B", "C", "alpha", "beta",
+                                                                "gamma", "theta")],
+                                           D=f64(q3.D), z=s_["z"])
+    put("m3su_bf16_b256_h24_p64_n64_k32_x1000", 24 * 64 * 10, su3,
+        "one sequence (24 heads), 10 steps")
+    # Mamba-3 from raw projections: one sequence; the discretisation fwd+bwd of
+    # all 24 heads and the scan fwd+bwd of one head, per token-channel of one head
+    d = W.m3disc_problem(1, 2048, 24, 64, 64, nangles=32, io=BF)
+    raw = {k: getattr(d, k).as_f64() for k in ("dd_dt", "dd_a", "trap", "angles", "B_raw",
+                                                "C_raw")}
+    kw = dict(dt_bias=f64(d.dt_bias), A_floor=d.A_floor, eps=d.eps)
+    rng = np.random.default_rng(0)
+    up = dict(dalpha=rng.standard_normal((1, 2048, 24)), dbeta=rng.standard_normal((1, 2048, 24)),
+              dgamma=rng.standard_normal((1, 2048, 24)),
+              dtheta=rng.standard_normal((1, 2048, 24, 32)),
+              dB=rng.standard_normal((1, 2048, 1, 64)), dC=rng.standard_normal((1, 2048, 1, 64)))
+    name = "m3disc_bf16_b8_h24_p64_n64_k32_l2048"
+    if name in res and "error" not in res[name]:
+        # seconds per token-channel: the discretisation's share (all 24 heads)
+        # plus one head's scan
+        rd, nd, td = _rate(lambda: (oracle.m3_discretize(**raw, **kw),
+                                    oracle.m3_discretize_bwd(**raw, **up, **kw)), budget_s)
+        rs, ns, ts = _rate(lambda: (oracle.m3_fwd(**ms), oracle.m3_bwd(dout=mdout, **ms)),
+                           budget_s)
+        per = 1.0 / (rd * 24 * 2048 * 64) + 1.0 / (rs * 2048 * 64)
+        res[name]["oracle"] = dict(
+            value=round(1.0 / per, 1), unit=res[name]["unit"], cores=thr, kind="oracle",
+            sample=f"one sequence: discretisation fwd+bwd of its 24 heads ({nd} reps, {td:.1f} s) "
+                   f"and scan fwd+bwd of one head ({ns} reps, {ts:.1f} s), combined per "
+                   f"token-channel")
+    # conv + Mamba-1 scan: one batch row of 128 channels, conv and scan fwd+bwd
+    c = W.m1conv_problem(1, 128, 16, 2048)
+    cs = oracle.m1_problem_args(c.scan)
+    cx, cw, cb = cs["u"], f64(c.w), f64(c.bias)
+    cdout = c.scan.dout.as_f64()
+
+    def conv_step():
+        u, _ = oracle.conv1d_fwd(cx, cw, bias=cb)
+        sa = dict(cs, u=u)
+        oracle.m1_fwd(**sa)
+        g = oracle.m1_bwd(dout=cdout, **sa)
+        oracle.conv1d_bwd(cx, cw, g["du"], bias=cb)
+    put("m1conv_bf16_b8_d1536_n16_l2048_w4", 128 * 2048, conv_step,
+        "one batch row of 128 channels, conv fwd+bwd and scan fwd+bwd")
+
+
 def run_e2e(p, msc, steps, warmup, world):
     """The step through the C ABI from pinned host buffers, pipelined the way a
     training input pipeline runs: every step copies its inputs host to device
@@ -581,6 +687,8 @@ def run_ours(args):
         line["cpu_baseline"] = cpu_baseline()
     if not args.no_extra:
         line["workloads"] = extra_workloads(msc, args, world, peaks)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            oracle_beside(line["workloads"])
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
