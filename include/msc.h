@@ -13,7 +13,12 @@
  *     "Features"; backward stages B2 output gating, B3 BPTT and B4 RoPE of
  *     Mamba3Scratch in mamba-rs 0.4.2 src/mamba3_siso/cpu/scratch.rs);
  *   - the single-token recurrent state update used in decoding (mamba_step /
- *     GpuMambaBackbone::step, mamba-rs 0.7.0 README, "Quick start").
+ *     GpuMambaBackbone::step, mamba-rs 0.7.0 README, "Quick start"), for
+ *     Mamba-1 and for Mamba-3 SISO (mamba3_step, the same README);
+ *   - the steps either side of the scans: the causal conv1d + SiLU ahead of
+ *     the Mamba-1 scan, standalone and fused into its forward, and the
+ *     Mamba-3 discretisation and BCNorm stages (B6, B5 of Mamba3Scratch),
+ *     each with its backward.
  *
  * Conventions shared by every entry point
  * ---------------------------------------
