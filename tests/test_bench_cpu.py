@@ -60,3 +60,32 @@ def test_clock_sampler_without_gpu():
     s.start()
     r = s.stop()
     assert set(r) >= {"sm_mhz", "sm_max_mhz", "reasons"}
+
+
+def test_conv_and_disc_bytes():
+    # conv: x in, u out (forward); x, du in, dx out (backward), bf16
+    fwd, bwd = bench.conv_bytes(8, 1536, 2048, 4, 2)
+    assert fwd == 2 * 8 * 1536 * 2048 * 2 and bwd == 3 * 8 * 1536 * 2048 * 2
+    # discretisation, per token: dd_dt, dd_a, trap (H each), angles (K), B_raw,
+    # C_raw (G N each) in; alpha, beta, gamma (H each), theta (H K), B, C out
+    tok, H, K, GN = 8 * 2048, 24, 32, 64
+    fwd, bwd = bench.m3disc_bytes(8, 2048, 24, 64, 1, 32, 2)
+    raw = tok * (3 * H + K + 2 * GN) * 2
+    assert fwd == raw + tok * (3 * H + H * K + 2 * GN) * 2
+    assert bwd == raw + tok * (3 * H + H * K + 2 * GN) * 4 + tok * (3 * H + K + 2 * GN) * 4
+    assert round(fwd / 1e6, 1) == 39.3 and round(bwd / 1e6, 1) == 86.2
+
+
+def test_oracle_beside_fills_every_workload():
+    """The oracle timings beside the extra workloads run on the host alone and
+    fill an entry for every workload that ran (none for one that failed)."""
+    names = ["m1_bf16_b4_d5120_n16_l4096", "su_bf16_b256_d5120_n16_x1000",
+             "m3_bf16_b8_h24_p64_n64_k32_l2048", "m3su_bf16_b256_h24_p64_n64_k32_x1000",
+             "m3disc_bf16_b8_h24_p64_n64_k32_l2048", "m1conv_bf16_b8_d1536_n16_l2048_w4"]
+    res = {n: {"unit": "u"} for n in names}
+    res[names[0]] = {"error": "x"}
+    bench.oracle_beside(res, budget_s=0.0)
+    assert "oracle" not in res[names[0]]
+    for n in names[1:]:
+        o = res[n]["oracle"]
+        assert o["kind"] == "oracle" and o["value"] > 0 and o["unit"] == "u" and o["sample"]

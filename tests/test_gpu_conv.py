@@ -265,3 +265,23 @@ def test_conv_workload_full_size(msc):
     rc = oracle.conv1d_bwd(q.scan.u.as_f64(), f64(q.w), q.scan.dout.as_f64(), bias=f64(q.bias))
     for k, rk in (("dx", "dx"), ("dw", "dw"), ("dbias", "dbias")):
         assert_close(k, host(g[k]), rc[rk], TOL["bf16"])
+
+
+def test_conv_empty_sequences(msc):
+    """L = 0: the conv state passes through (or becomes zeros), the gradients of
+    the weights are zero; the fused forward also passes the scan state."""
+    x = torch.empty(2, 3, 0, device="cuda")
+    w = torch.randn(3, 4, device="cuda")
+    xs0 = torch.randn(2, 3, 3, device="cuda")
+    _, xs = msc.msc_causal_conv1d_fwd(x, w, conv_state_in=xs0)
+    _, xz = msc.msc_causal_conv1d_fwd(x, w)
+    g = msc.msc_causal_conv1d_bwd(x, w, x, bias=torch.randn(3, device="cuda"), conv_state_in=xs0)
+    A = -torch.ones(3, 16, device="cuda")
+    Be = torch.empty(2, 1, 16, 0, device="cuda")
+    h0 = torch.randn(2, 3, 16, device="cuda")
+    out, fs, _, u, xs2 = msc.msc_selective_scan_conv_fwd(x, w, x, A, Be, Be, conv_state=xs0, h0=h0)
+    torch.cuda.synchronize()
+    assert torch.equal(xs, xs0) and float(xz.abs().sum()) == 0.0
+    assert float(g["dw"].abs().sum()) == 0.0 and float(g["dbias"].abs().sum()) == 0.0
+    assert float(g["dconv_state_in"].abs().sum()) == 0.0
+    assert torch.equal(fs, h0) and torch.equal(xs2, xs0)

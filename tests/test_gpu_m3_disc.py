@@ -167,3 +167,17 @@ def test_disc_bwd_full_size(msc):
                                     A_floor=q.A_floor, eps=q.eps)
     for k in DISC_GRADS:
         assert_close(k, host(g[k]), refg[k], TOL["f32"])
+
+
+def test_disc_empty_sequence(msc):
+    """L = 0: nothing to discretise; the bias gradient is zero."""
+    e3 = torch.empty(2, 0, 4, device="cuda")
+    ang = torch.empty(2, 0, 8, device="cuda")
+    raw = torch.empty(2, 0, 1, 16, device="cuda")
+    dtb = torch.randn(4, device="cuda")
+    msc.msc_mamba3_siso_discretize(e3, e3, e3, ang, raw, raw, dt_bias=dtb)
+    g = msc.msc_mamba3_siso_discretize_bwd(e3, e3, e3, ang, raw, raw, e3, e3, e3,
+                                           torch.empty(2, 0, 4, 8, device="cuda"), raw, raw,
+                                           dt_bias=dtb)
+    torch.cuda.synchronize()
+    assert float(g["ddt_bias"].abs().sum()) == 0.0
