@@ -535,6 +535,20 @@ def oracle_beside(res, budget_s=1.5):
                                            D=f64(q3.D), z=s_["z"])
     put("m3su_bf16_b256_h24_p64_n64_k32_x1000", 24 * 64 * 10, su3,
         "one sequence (24 heads), 10 steps")
+    # the same decode from raw values: the oracle's discretisation of the token
+    # (values rounded to bf16 as stored) ahead of its step
+    raw_steps, rdtb = W.m3su_raw_steps(1, 24, 64, nangles=32, n_pool=10)
+    rsteps = [{k: v.as_f64()[:, None] for k, v in s_.items()} for s_ in raw_steps]
+
+    def su3_raw():
+        c = [v.astype(np.float64) for v in (q3.state0, q3.x_prev0, q3.bt_prev0, q3.phi0)]
+        for s_, r_ in zip(st3, rsteps):
+            d_ = oracle.m3_discretize(**r_, dt_bias=f64(rdtb), A_floor=1e-4, eps=1e-5)
+            d_ = {k: W.store(v[:, 0].astype(np.float32), BF).as_f64() for k, v in d_.items()}
+            *c, _ = oracle.m3_state_update(*c, s_["x"], d_["B"], d_["C"], d_["alpha"], d_["beta"],
+                                           d_["gamma"], d_["theta"], D=f64(q3.D), z=s_["z"])
+    put("m3su_raw_bf16_b256_h24_p64_n64_k32_x1000", 24 * 64 * 10, su3_raw,
+        "one sequence (24 heads), 10 steps from raw values")
     # Mamba-3 from raw projections: one sequence; the discretisation fwd+bwd of
     # all 24 heads and the scan fwd+bwd of one head, per token-channel of one head
     d = W.m3disc_problem(1, 2048, 24, 64, 64, nangles=32, io=BF)
@@ -754,6 +768,44 @@ def extra_workloads(msc, args, world, peaks):
         unit="token-channel steps/s",
         hbm_frac=round(sb3 * 1000 / (ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
         note="101 MB state: most of it can stay in the 126 MB L2 between steps")
+    # the same decode from raw values: the discretisation fused into the step,
+    # against the discretisation kernel (one token) followed by the plain step
+    raw_steps, dtb = W.m3su_raw_steps(q3.batch, q3.nheads, q3.dstate, nangles=q3.nangles)
+    rawd = [{k: to_dev(v) for k, v in s_.items()} for s_ in raw_steps]
+    dtb_d = to_dev(dtb)
+    one = lambda t: t.view(t.shape[0], 1, *t.shape[1:])
+    disc_out = msc.msc_mamba3_siso_discretize(one(rawd[0]["dd_dt"]), one(rawd[0]["dd_a"]),
+                                              one(rawd[0]["trap"]), one(rawd[0]["angles"]),
+                                              one(rawd[0]["B_raw"]), one(rawd[0]["C_raw"]),
+                                              dt_bias=dtb_d)
+    sq = {k: v[:, 0] for k, v in disc_out.items()}
+
+    def m3_decode_raw_1000():
+        for t in range(1000):
+            r = rawd[t % 8]
+            msc.msc_mamba3_siso_disc_state_update(
+                *carried, pool3[t % 8]["x"], r["dd_dt"], r["dd_a"], r["trap"], r["angles"],
+                r["B_raw"], r["C_raw"], dt_bias=dtb_d, D=D3, z=pool3[t % 8]["z"],
+                out=outs3[t % 8])
+
+    def m3_decode_raw_unfused_1000():
+        for t in range(1000):
+            r = rawd[t % 8]
+            msc.msc_mamba3_siso_discretize(one(r["dd_dt"]), one(r["dd_a"]), one(r["trap"]),
+                                           one(r["angles"]), one(r["B_raw"]), one(r["C_raw"]),
+                                           dt_bias=dtb_d, outs=disc_out)
+            msc.msc_mamba3_siso_state_update(*carried, pool3[t % 8]["x"], sq["B"], sq["C"],
+                                             sq["alpha"], sq["beta"], sq["gamma"], sq["theta"],
+                                             D=D3, z=pool3[t % 8]["z"], out=outs3[t % 8])
+
+    _, (ms_f,) = time_steps([m3_decode_raw_1000], 2, 1, world)
+    _, (ms_u,) = time_steps([m3_decode_raw_unfused_1000], 2, 1, world)
+    res["m3su_raw_bf16_b256_h24_p64_n64_k32_x1000"] = dict(
+        us_per_step=round(ms_f, 3), unfused_us_per_step=round(ms_u, 3),
+        value=round(q3.batch * q3.nheads * q3.headdim * 1000 / (ms_f / 1e3), 1),
+        unit="token-channel steps/s",
+        note="decode from raw dd_dt, dd_a, trap, angles, B_raw, C_raw: the discretisation "
+             "fused into the step vs its own kernel ahead of the plain step")
     del carried, pool3, outs3
     torch.cuda.empty_cache()
     # Mamba-3 SISO

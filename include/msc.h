@@ -471,6 +471,32 @@ typedef struct {
 
 msc_status msc_mamba3_siso_state_update(const msc_m3_su_args *args, msc_stream_t stream);
 
+/*
+ * The same step with the discretisation and BCNorm (msc_mamba3_siso_discretize
+ * below) fused ahead: the step's alpha, beta, gamma, theta, Bm and Cm are
+ * derived in the kernel from this token's raw values instead of being read
+ * (the corresponding fields of `step` are ignored and may be NULL):
+ *   dd_dt, dd_a, trap         io  [B, H]
+ *   angles                    io  [B, K]   (may be NULL when K = 0)
+ *   dt_bias                   f32 [H]      optional
+ *   B_raw, C_raw              io  [B, G, N]
+ * Every derived value is rounded to the io type, so the result equals, bit
+ * for bit, msc_mamba3_siso_discretize over the token followed by
+ * msc_mamba3_siso_state_update.  An addition of this library (one launch per
+ * generated token instead of two).
+ */
+typedef struct {
+  uint32_t struct_size;
+  float A_floor, eps;
+  const void *dd_dt, *dd_a, *trap, *angles;
+  const float *dt_bias;    /* optional */
+  const void *B_raw, *C_raw;
+} msc_m3_disc_step_args;
+
+msc_status msc_mamba3_siso_disc_state_update(const msc_m3_su_args *step,
+                                             const msc_m3_disc_step_args *raw,
+                                             msc_stream_t stream);
+
 /* ======================================================================
  * Mamba-3 SISO discretisation and BCNorm (the stages ahead of the scan)
  * ======================================================================

@@ -208,8 +208,12 @@ msc_status msc_mamba3_siso_scan_bwd(const msc_m3_bwd_args *a, void *workspace,
   return api_cuda(msc::launch_m3_bwd(p, s), fn);
 }
 
-msc_status msc_mamba3_siso_state_update(const msc_m3_su_args *a, msc_stream_t stream) {
-  const char *fn = "msc_mamba3_siso_state_update";
+}  // extern "C"
+
+namespace {
+// the decode step; raw non-null: the discretisation and BCNorm fused ahead
+msc_status m3_step(const char *fn, const msc_m3_su_args *a, const msc_m3_disc_step_args *raw,
+                   msc_stream_t stream) {
   if (!a) return api_fail(MSC_ERR_INVALID_ARG, "%s: args is NULL", fn);
   if (a->struct_size < sizeof(msc_m3_su_args))
     return api_fail(MSC_ERR_INVALID_ARG, "%s: struct_size %u is smaller than the struct (%zu)",
@@ -239,15 +243,28 @@ msc_status msc_mamba3_siso_state_update(const msc_m3_su_args *a, msc_stream_t st
   M3_REQUIRE(fn, "x_prev", a->x_prev);
   M3_REQUIRE(fn, "bt_prev", a->bt_prev);
   M3_REQUIRE(fn, "x", a->x);
-  M3_REQUIRE(fn, "Bm", a->Bm);
-  M3_REQUIRE(fn, "Cm", a->Cm);
-  M3_REQUIRE(fn, "alpha", a->alpha);
-  M3_REQUIRE(fn, "beta", a->beta);
-  M3_REQUIRE(fn, "gamma", a->gamma);
   M3_REQUIRE(fn, "out", a->out);
-  if (a->nangles > 0) {
-    M3_REQUIRE(fn, "phi", a->phi);
-    M3_REQUIRE(fn, "theta", a->theta);
+  if (a->nangles > 0) M3_REQUIRE(fn, "phi", a->phi);
+  if (raw) {
+    if (raw->struct_size < sizeof(msc_m3_disc_step_args))
+      return api_fail(MSC_ERR_INVALID_ARG, "%s: raw struct_size %u is smaller than the struct "
+                      "(%zu)", fn, raw->struct_size, sizeof(msc_m3_disc_step_args));
+    if (!(raw->A_floor >= 0.f) || !(raw->eps >= 0.f))
+      return api_fail(MSC_ERR_INVALID_ARG, "%s: A_floor and eps must be >= 0", fn);
+    M3_REQUIRE(fn, "dd_dt", raw->dd_dt);
+    M3_REQUIRE(fn, "dd_a", raw->dd_a);
+    M3_REQUIRE(fn, "trap", raw->trap);
+    if (a->nangles > 0) M3_REQUIRE(fn, "angles", raw->angles);
+    M3_OPTIONAL(fn, "dt_bias", raw->dt_bias);
+    M3_REQUIRE(fn, "B_raw", raw->B_raw);
+    M3_REQUIRE(fn, "C_raw", raw->C_raw);
+  } else {
+    M3_REQUIRE(fn, "Bm", a->Bm);
+    M3_REQUIRE(fn, "Cm", a->Cm);
+    M3_REQUIRE(fn, "alpha", a->alpha);
+    M3_REQUIRE(fn, "beta", a->beta);
+    M3_REQUIRE(fn, "gamma", a->gamma);
+    if (a->nangles > 0) M3_REQUIRE(fn, "theta", a->theta);
   }
   M3_OPTIONAL(fn, "z", a->z);
   M3_OPTIONAL(fn, "D", a->D);
@@ -259,7 +276,28 @@ msc_status msc_mamba3_siso_state_update(const msc_m3_su_args *a, msc_stream_t st
   p.x = a->x; p.z = a->z; p.Bm = a->Bm; p.Cm = a->Cm;
   p.alpha = a->alpha; p.beta = a->beta; p.gamma = a->gamma; p.theta = a->theta;
   p.Dp = a->D; p.out = a->out;
+  if (raw) {
+    p.raw = true;
+    p.dd_dt = raw->dd_dt; p.dd_a = raw->dd_a; p.trap = raw->trap; p.angles = raw->angles;
+    p.dt_bias = raw->dt_bias; p.B_raw = raw->B_raw; p.C_raw = raw->C_raw;
+    p.A_floor = raw->A_floor; p.eps = raw->eps;
+  }
   return api_cuda(msc::launch_m3_state_update(p, reinterpret_cast<cudaStream_t>(stream)), fn);
+}
+}  // namespace
+
+extern "C" {
+
+msc_status msc_mamba3_siso_state_update(const msc_m3_su_args *a, msc_stream_t stream) {
+  return m3_step("msc_mamba3_siso_state_update", a, nullptr, stream);
+}
+
+msc_status msc_mamba3_siso_disc_state_update(const msc_m3_su_args *step,
+                                             const msc_m3_disc_step_args *raw,
+                                             msc_stream_t stream) {
+  const char *fn = "msc_mamba3_siso_disc_state_update";
+  if (!raw) return api_fail(MSC_ERR_INVALID_ARG, "%s: raw is NULL", fn);
+  return m3_step(fn, step, raw, stream);
 }
 
 

@@ -155,6 +155,13 @@ struct M3SUParams {
   const void *x, *z, *Bm, *Cm, *alpha, *beta, *gamma, *theta;
   const float *Dp;
   void *out;
+  // with the discretisation and BCNorm fused ahead (raw): alpha .. theta, Bm,
+  // Cm are derived in the kernel from these step inputs instead
+  bool raw;
+  const void *dd_dt, *dd_a, *trap, *angles;  // io [B, H] x3, [B, K]
+  const float *dt_bias;                      // [H] or null
+  const void *B_raw, *C_raw;                 // io [B, G, N]
+  float A_floor, eps;
 };
 cudaError_t launch_m3_state_update(const M3SUParams &p, cudaStream_t s);
 

@@ -23,8 +23,8 @@
 // ddt_bias is a second, fixed-order pass over ddd_dt (one CTA per head).
 // Bound: HBM (the theta write dominates the forward, the dtheta read the
 // backward).
-#include "common.cuh"
 #include "kernels.h"
+#include "m3_disc_common.cuh"
 
 namespace msc {
 namespace {
@@ -44,33 +44,15 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-struct HeadCoef {
-  float dt, sig_u, A, dA_dda, alpha, lam;
-};
-
 template <typename T>
-__device__ __forceinline__ HeadCoef head_coef(const M3DiscParams &p, int64_t i, int h) {
-  HeadCoef c;
-  const float u = ldv<T>(p.dd_dt, i) + (p.dt_bias ? p.dt_bias[h] : 0.f);
-  c.dt = softplus(u);
-  c.sig_u = sigmoid(u);
-  const float dda = ldv<T>(p.dd_a, i);
-  const float sa = softplus(dda);
-  const bool clamped = -sa > -p.A_floor;  // A held at -A_floor: no gradient to dd_a
-  c.A = clamped ? -p.A_floor : -sa;
-  c.dA_dda = clamped ? 0.f : -sigmoid(dda);
-  c.alpha = __expf(c.dt * c.A);
-  c.lam = sigmoid(ldv<T>(p.trap, i));
-  return c;
+__device__ __forceinline__ DiscCoef head_coef(const M3DiscParams &p, int64_t i, int h) {
+  return disc_coef(ldv<T>(p.dd_dt, i), p.dt_bias ? p.dt_bias[h] : 0.f, ldv<T>(p.dd_a, i),
+                   ldv<T>(p.trap, i), p.A_floor);
 }
 
 // Row pieces of 8 elements: a B or C row of N = 8 S elements (S a power of
 // two <= 32) is served by S lanes, 32 / S rows per pass, 16-byte accesses.
-__device__ __forceinline__ int row_lanes(int N) {
-  if (N % 8 != 0) return 0;
-  const int s = N / 8;
-  return (s <= 32 && (s & (s - 1)) == 0) ? s : 0;
-}
+__device__ __forceinline__ int row_lanes(int N) { return disc_row_lanes(N); }
 
 // the same sum in every lane of each aligned group of `seg` lanes
 __device__ __forceinline__ float seg_sum(float v, int seg) {
@@ -136,10 +118,10 @@ __global__ void __launch_bounds__(kDiscWarps * 32) m3_disc_fwd_kernel(const M3Di
        tok += (int64_t)gridDim.x * kDiscWarps) {
     for (int h = lane; h < H; h += 32) {
       const int64_t i = tok * H + h;
-      const HeadCoef c = head_coef<T>(p, i, h);
+      const DiscCoef c = head_coef<T>(p, i, h);
       static_cast<T *>(p.alpha)[i] = from_f32<T>(c.alpha);
-      static_cast<T *>(p.beta)[i] = from_f32<T>((1.f - c.lam) * c.dt * c.alpha);
-      static_cast<T *>(p.gamma)[i] = from_f32<T>(c.lam * c.dt);
+      static_cast<T *>(p.beta)[i] = from_f32<T>(disc_beta(c));
+      static_cast<T *>(p.gamma)[i] = from_f32<T>(disc_gamma(c));
       sdt[h] = c.dt;
     }
     for (int k = lane; k < K; k += 32) sang[k] = ldv<T>(p.angles, tok * K + k);
@@ -237,7 +219,7 @@ __global__ void __launch_bounds__(kDiscWarps * 32) m3_disc_bwd_kernel(const M3Di
     }
     for (int h = lane; h < H; h += 32) {
       const int64_t i = tok * H + h;
-      const HeadCoef c = head_coef<T>(p, i, h);
+      const DiscCoef c = head_coef<T>(p, i, h);
       float gth = 0.f;  // sum_k dtheta[h, k] angles[k]
       for (int k = 0; k < K; ++k) gth = fmaf(sth[h * (K + 1) + k], sang[k], gth);
       const float ga = p.dalpha[i], gb = p.dbeta[i], gg = p.dgamma[i];

@@ -19,8 +19,16 @@
 // partials over its N / 16 threads with shuffles in a fixed order.  Wider
 // states (128, 192, 256) are walked in slabs of 64 states with the 64-state
 // layout, y carried across the slabs in registers.
-#include "common.cuh"
+//
+// kRaw fuses the discretisation and BCNorm ahead (m3_disc_common.cuh): the
+// first lanes of a head (its first warp, or half-warp when a warp holds two
+// heads) derive dt, alpha, beta, gamma from dd_dt, dd_a, trap and the RMS
+// scales of the head's raw B and C rows, and the rotating threads take
+// theta = dt angles.  Every derived value is rounded to the io type and the
+// row sums follow the discretisation kernel's order, so the fused step gives
+// the same bits as the discretisation kernel followed by the plain step.
 #include "kernels.h"
+#include "m3_disc_common.cuh"
 
 namespace msc {
 namespace {
@@ -32,14 +40,63 @@ __device__ __forceinline__ float ldf(const void *base, int64_t i) {
   return to_f32(static_cast<const T *>(base)[i]);
 }
 
-template <typename T, int P, int N>
+// The RMS scale 1/sqrt(mean(v^2) + eps) of the raw row at `row` (N entries),
+// its square sum taken in the discretisation kernel's order: in the 16-byte
+// path lane l < S sums its 8 entries in order and the S lanes add with xor
+// shuffles at distances 1, 2, ...; otherwise lane l sums entries l, l + 32, ...
+// and the warp adds at distances 16, 8, ....  Every lane of the warp calls it;
+// lane l of each aligned group of kLW lanes takes the role of lane l there,
+// and the group's lane 0 holds the result.
+template <typename T, int N, int kLW>
+__device__ __forceinline__ float raw_rms_scale(const void *raw, int64_t row, bool live, int lg,
+                                               float eps) {
+  constexpr int kS = disc_row_lanes(N);
+  float ss = 0.f;
+  if constexpr (kS > 0) {
+    static_assert(kS <= kLW, "a row's lanes sit in one group");
+    if (live && lg < kS) {
+      const T *src = static_cast<const T *>(raw) + row + lg * 8;
+      float v[8];
+      if constexpr (sizeof(T) == 2) {
+        const uint4 w = *reinterpret_cast<const uint4 *>(src);
+        unpack2<T>(w.x, v[0], v[1]);
+        unpack2<T>(w.y, v[2], v[3]);
+        unpack2<T>(w.z, v[4], v[5]);
+        unpack2<T>(w.w, v[6], v[7]);
+      } else {
+        const float4 a = reinterpret_cast<const float4 *>(src)[0];
+        const float4 b = reinterpret_cast<const float4 *>(src)[1];
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+        v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) ss = fmaf(v[e], v[e], ss);
+    }
+#pragma unroll
+    for (int m = 1; m < kS; m <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+  } else {
+    static_assert(kLW == 32, "the scalar path uses whole warps");
+    if (live)
+      for (int n = lg; n < N; n += 32) {
+        const float v = ldf<T>(raw, row + n);
+        ss = fmaf(v, v, ss);
+      }
+#pragma unroll
+    for (int m = 16; m > 0; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+  }
+  return rsqrtf(ss / (float)N + eps);
+}
+
+template <typename T, int P, int N, bool kRaw>
 __global__ void __launch_bounds__(kSUThreads) m3_state_update_kernel(const M3SUParams p) {
   constexpr int kSN = N < 64 ? N : 64;     // states per slab (wider states: slabs of 64 in turn)
   constexpr int kNS = N / kSN;             // slabs
   constexpr int kTPR = kSN / 16;           // threads per row of a slab
   constexpr int kTPH = P * kTPR;           // threads per head
   constexpr int kHPC = kSUThreads / kTPH;  // heads per CTA
-  constexpr int kPer = 3 * kSN + P;        // shared floats per head: Bt, Ct, bt_prev (a slab), x_prev
+  constexpr int kLW = kTPH < 32 ? kTPH : 32;  // lanes of a head in its first warp
+  // shared floats per head: Bt, Ct, bt_prev (a slab), x_prev; (kRaw) alpha, beta, gamma
+  constexpr int kPer = 3 * kSN + P + (kRaw ? 4 : 0);
   __shared__ __align__(16) float sm[kHPC * kPer];
 
   const int tid = threadIdx.x;
@@ -55,7 +112,13 @@ __global__ void __launch_bounds__(kSUThreads) m3_state_update_kernel(const M3SUP
   float4 *srow = reinterpret_cast<float4 *>(p.state + (bh * P + row) * N);
 
   float al = 0.f, be = 0.f, ga = 0.f, xv = 0.f;
-  if (live) {
+  float dt = 0.f, rB = 0.f, rC = 0.f;  // kRaw: the head's dt and B, C scales (rotating lanes)
+  if constexpr (kRaw) {
+    if (live) {
+      xv = ldf<T>(p.x, bh * P + row);
+      for (int i = j; i < P; i += kTPH) sXp[i] = p.x_prev[bh * P + i];
+    }
+  } else if (live) {
     al = ldf<T>(p.alpha, bh);
     be = ldf<T>(p.beta, bh);
     ga = ldf<T>(p.gamma, bh);
@@ -72,13 +135,49 @@ __global__ void __launch_bounds__(kSUThreads) m3_state_update_kernel(const M3SUP
     if (live) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) st[i] = srow[n0 / 4 + i * kTPR + q];
+    }
+    if constexpr (kRaw) {
+      // (first slab, after the state loads are under way) the head's dt, alpha,
+      // beta, gamma and the scales of its raw B and C rows
+      if (sl == 0 && j < kLW) {  // the head's first lanes; every lane of their warp is here
+        float *sCoef = sXp + P;
+        if (live) {
+          const DiscCoef c = disc_coef(ldf<T>(p.dd_dt, bh), p.dt_bias ? p.dt_bias[h] : 0.f,
+                                       ldf<T>(p.dd_a, bh), ldf<T>(p.trap, bh), p.A_floor);
+          dt = c.dt;
+          if (j == 0) {
+            sCoef[0] = to_f32(from_f32<T>(c.alpha));
+            sCoef[1] = to_f32(from_f32<T>(disc_beta(c)));
+            sCoef[2] = to_f32(from_f32<T>(disc_gamma(c)));
+          }
+        }
+        const int64_t brow = (b * p.G + g) * N;
+        rB = __shfl_sync(0xffffffffu, raw_rms_scale<T, N, kLW>(p.B_raw, brow, live, j, p.eps),
+                         0, kLW);
+        rC = __shfl_sync(0xffffffffu, raw_rms_scale<T, N, kLW>(p.C_raw, brow, live, j, p.eps),
+                         0, kLW);
+      }
+    }
+    if (live) {
       if (j < kSN / 2) {
         const int ka = n0 / 2 + j;  // global angle pair
         const int64_t o = (b * p.G + g) * N + n0 + 2 * j;
-        float b0 = ldf<T>(p.Bm, o), b1 = ldf<T>(p.Bm, o + 1);
-        float c0 = ldf<T>(p.Cm, o), c1 = ldf<T>(p.Cm, o + 1);
+        float b0, b1, c0, c1;
+        // (kRaw) products in __fmul_rn: with f32 io nothing rounds between them
+        // and their next use, and a contraction into an FMA would change the bits
+        if constexpr (kRaw) {  // normalised as the discretisation kernel stores them
+          b0 = to_f32(from_f32<T>(__fmul_rn(ldf<T>(p.B_raw, o), rB)));
+          b1 = to_f32(from_f32<T>(__fmul_rn(ldf<T>(p.B_raw, o + 1), rB)));
+          c0 = to_f32(from_f32<T>(__fmul_rn(ldf<T>(p.C_raw, o), rC)));
+          c1 = to_f32(from_f32<T>(__fmul_rn(ldf<T>(p.C_raw, o + 1), rC)));
+        } else {
+          b0 = ldf<T>(p.Bm, o); b1 = ldf<T>(p.Bm, o + 1);
+          c0 = ldf<T>(p.Cm, o); c1 = ldf<T>(p.Cm, o + 1);
+        }
         if (ka < K) {
-          const float phi = p.phi[bh * K + ka] + ldf<T>(p.theta, bh * K + ka);
+          const float th = kRaw ? to_f32(from_f32<T>(__fmul_rn(dt, ldf<T>(p.angles, b * K + ka))))
+                                : ldf<T>(p.theta, bh * K + ka);
+          const float phi = p.phi[bh * K + ka] + th;
           p.phi[bh * K + ka] = phi;
           float sn, cs;
           sincosf(phi, &sn, &cs);
@@ -92,6 +191,12 @@ __global__ void __launch_bounds__(kSUThreads) m3_state_update_kernel(const M3SUP
       for (int i = j; i < kSN; i += kTPH) sBp[i] = p.bt_prev[bh * N + n0 + i];
     }
     __syncthreads();
+    if constexpr (kRaw) {
+      if (sl == 0) {
+        const float *sCoef = sXp + P;
+        al = sCoef[0]; be = sCoef[1]; ga = sCoef[2];
+      }
+    }
     if (live) {
       // the carried key of the next step (every read of the old one is done)
       for (int i = j; i < kSN; i += kTPH) p.bt_prev[bh * N + n0 + i] = sBt[i];
@@ -134,7 +239,10 @@ template <typename T, int P, int N>
 cudaError_t launch_pn(const M3SUParams &p, cudaStream_t s) {
   constexpr int kHPC = kSUThreads / (P * (N < 64 ? N : 64) / 16);
   const int64_t blocks = (p.B * p.H + kHPC - 1) / kHPC;
-  m3_state_update_kernel<T, P, N><<<(unsigned)blocks, kSUThreads, 0, s>>>(p);
+  if (p.raw)
+    m3_state_update_kernel<T, P, N, true><<<(unsigned)blocks, kSUThreads, 0, s>>>(p);
+  else
+    m3_state_update_kernel<T, P, N, false><<<(unsigned)blocks, kSUThreads, 0, s>>>(p);
   return cudaGetLastError();
 }
 

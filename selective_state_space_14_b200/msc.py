@@ -94,6 +94,12 @@ class M3SuArgs(ctypes.Structure):
                 ("gamma", _vp), ("theta", _vp), ("D", _vp), ("out", _vp)]
 
 
+class M3DiscStepArgs(ctypes.Structure):
+    _fields_ = [("struct_size", _u32), ("A_floor", ctypes.c_float), ("eps", ctypes.c_float),
+                ("dd_dt", _vp), ("dd_a", _vp), ("trap", _vp), ("angles", _vp), ("dt_bias", _vp),
+                ("B_raw", _vp), ("C_raw", _vp)]
+
+
 class M3DiscArgs(ctypes.Structure):
     _fields_ = [("struct_size", _u32), ("io_dtype", _i32), ("batch", _i64), ("seqlen", _i64),
                 ("nheads", _i64), ("dstate", _i64), ("ngroups", _i64), ("nangles", _i64),
@@ -135,7 +141,7 @@ EXPORTS = ["msc_last_error", "msc_version", "msc_selective_scan_saved_states_byt
            "msc_mamba3_siso_scan_bwd", "msc_mamba3_siso_state_update", "msc_causal_conv1d_fwd",
            "msc_causal_conv1d_bwd_workspace_bytes", "msc_causal_conv1d_bwd",
            "msc_selective_scan_conv_fwd", "msc_mamba3_siso_discretize",
-           "msc_mamba3_siso_discretize_bwd"]
+           "msc_mamba3_siso_discretize_bwd", "msc_mamba3_siso_disc_state_update"]
 
 _lib = None
 
@@ -162,6 +168,8 @@ def lib() -> ctypes.CDLL:
                             [ctypes.POINTER(M3BwdArgs), _vp, ctypes.c_size_t, _vp]),
                            ("msc_mamba3_siso_state_update", [ctypes.POINTER(M3SuArgs), _vp]),
                            ("msc_mamba3_siso_discretize", [ctypes.POINTER(M3DiscArgs), _vp]),
+                           ("msc_mamba3_siso_disc_state_update",
+                            [ctypes.POINTER(M3SuArgs), ctypes.POINTER(M3DiscStepArgs), _vp]),
                            ("msc_mamba3_siso_discretize_bwd",
                             [ctypes.POINTER(M3DiscBwdArgs), _vp]),
                            ("msc_causal_conv1d_fwd", [ctypes.POINTER(ConvFwdArgs), _vp]),
@@ -498,6 +506,29 @@ def msc_mamba3_siso_state_update(state, x_prev, bt_prev, phi, x, B, C, alpha, be
                  _ptr(alpha), _ptr(beta), _ptr(gamma), _ptr(theta) if K > 0 else None, _ptr(D),
                  _ptr(out))
     _check(lib().msc_mamba3_siso_state_update(ctypes.byref(a), _stream(stream)))
+    return out
+
+
+def msc_mamba3_siso_disc_state_update(state, x_prev, bt_prev, phi, x, dd_dt, dd_a, trap, angles,
+                                      B_raw, C_raw, dt_bias=None, A_floor=1e-4, eps=1e-5, D=None,
+                                      z=None, out=None, stream=None):
+    """The Mamba-3 decode step from this token's raw values (the discretisation
+    and BCNorm fused ahead).  Carried state as msc_mamba3_siso_state_update;
+    dd_dt, dd_a, trap [B, H]; angles [B, K]; B_raw, C_raw [B, G, N] (io);
+    dt_bias f32 [H].  Returns out [B, H, P]."""
+    Bsz, H, P, N = state.shape
+    G = B_raw.shape[1]
+    K = phi.shape[2]
+    if out is None:
+        out = torch.empty_like(x)
+    a = M3SuArgs(ctypes.sizeof(M3SuArgs), _io(x), Bsz, H, P, N, G, K, _ptr(state), _ptr(x_prev),
+                 _ptr(bt_prev), _ptr(phi) if K > 0 else None, _ptr(x), _ptr(z), None, None,
+                 None, None, None, None, _ptr(D), _ptr(out))
+    r = M3DiscStepArgs(ctypes.sizeof(M3DiscStepArgs), A_floor, eps, _ptr(dd_dt), _ptr(dd_a),
+                       _ptr(trap), _ptr(angles) if K > 0 else None, _ptr(dt_bias), _ptr(B_raw),
+                       _ptr(C_raw))
+    _check(lib().msc_mamba3_siso_disc_state_update(ctypes.byref(a), ctypes.byref(r),
+                                                   _stream(stream)))
     return out
 
 

@@ -337,6 +337,25 @@ def m3su_problem(batch, nheads, headdim, dstate, ngroups=1, nangles=None, io=BF1
     return M3SUProblem(Bsz, H, P, N, G, K, io, Dp, state0, x_prev0, bt_prev0, phi0, steps)
 
 
+def m3su_raw_steps(batch, nheads, dstate, ngroups=1, nangles=None, io=BF16, seed=SEED_BASE + 8,
+                   n_pool=8):
+    """Raw per-token values for the Mamba-3 decode step with the discretisation
+    fused ahead, drawn like the raw-input scan workload: a pool of ``n_pool``
+    step sets (dd_dt, dd_a, trap [B, H], angles [B, K], B_raw, C_raw [B, G, N])
+    and dt_bias [H]."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    Bsz, H, N, G = batch, nheads, dstate, ngroups
+    K = N // 2 if nangles is None else nangles
+    dt0 = np.exp(_uniform(rng, np.log(1e-3), np.log(1e-1), (H,)).astype(np.float64))
+    dt_bias = np.log(np.expm1(dt0)).astype(np.float32)
+    steps = [dict(dd_dt=store(0.5 * _normal(rng, (Bsz, H)), io),
+                  dd_a=store(_normal(rng, (Bsz, H)), io), trap=store(_normal(rng, (Bsz, H)), io),
+                  angles=store(_normal(rng, (Bsz, K)), io),
+                  B_raw=store(_normal(rng, (Bsz, G, N)), io),
+                  C_raw=store(_normal(rng, (Bsz, G, N)), io)) for _ in range(n_pool)]
+    return steps, dt_bias
+
+
 # --------------------------------------------------------------------------
 # The causal conv1d ahead of the Mamba-1 scan
 # --------------------------------------------------------------------------

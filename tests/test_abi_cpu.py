@@ -335,3 +335,27 @@ def test_disc_rejects_missing_pointers():
     assert msc.lib().msc_mamba3_siso_discretize_bwd(ctypes.byref(b), None) == INVALID
     assert "ddd_dt is NULL" in _err()
     assert msc.lib().msc_mamba3_siso_discretize(ctypes.byref(_disc_args(batch=0)), None) == OK
+
+
+def test_fused_decode_checks_raw_args():
+    """The fused decode step rejects a missing raw struct or raw input before
+    any launch; the plain step's alpha .. Cm are not required."""
+    fake = ctypes.c_void_p(1 << 20)
+    a = msc.M3SuArgs()
+    a.struct_size = ctypes.sizeof(msc.M3SuArgs)
+    a.io_dtype, a.batch, a.nheads, a.headdim, a.dstate, a.ngroups, a.nangles = (
+        msc.MSC_BF16, 2, 4, 64, 64, 1, 32)
+    for f in ("state", "x_prev", "bt_prev", "phi", "x", "out"):
+        setattr(a, f, fake)
+    fn = msc.lib().msc_mamba3_siso_disc_state_update
+    assert fn(ctypes.byref(a), None, None) == INVALID and "raw is NULL" in _err()
+    r = msc.M3DiscStepArgs()
+    r.struct_size = ctypes.sizeof(msc.M3DiscStepArgs)
+    r.A_floor, r.eps = 1e-4, 1e-5
+    assert fn(ctypes.byref(a), ctypes.byref(r), None) == INVALID and "dd_dt is NULL" in _err()
+    r.dd_dt = r.dd_a = r.trap = r.angles = r.B_raw = fake
+    assert fn(ctypes.byref(a), ctypes.byref(r), None) == INVALID and "C_raw is NULL" in _err()
+    r.eps = -1.0
+    assert fn(ctypes.byref(a), ctypes.byref(r), None) == INVALID and "eps" in _err()
+    r.eps, r.struct_size = 1e-5, 4
+    assert fn(ctypes.byref(a), ctypes.byref(r), None) == INVALID and "struct_size" in _err()

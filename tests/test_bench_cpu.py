@@ -81,7 +81,8 @@ def test_oracle_beside_fills_every_workload():
     fill an entry for every workload that ran (none for one that failed)."""
     names = ["m1_bf16_b4_d5120_n16_l4096", "su_bf16_b256_d5120_n16_x1000",
              "m3_bf16_b8_h24_p64_n64_k32_l2048", "m3su_bf16_b256_h24_p64_n64_k32_x1000",
-             "m3disc_bf16_b8_h24_p64_n64_k32_l2048", "m1conv_bf16_b8_d1536_n16_l2048_w4"]
+             "m3disc_bf16_b8_h24_p64_n64_k32_l2048", "m1conv_bf16_b8_d1536_n16_l2048_w4",
+             "m3su_raw_bf16_b256_h24_p64_n64_k32_x1000"]
     res = {n: {"unit": "u"} for n in names}
     res[names[0]] = {"error": "x"}
     bench.oracle_beside(res, budget_s=0.0)

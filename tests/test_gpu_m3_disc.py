@@ -181,3 +181,98 @@ def test_disc_empty_sequence(msc):
                                            dt_bias=dtb)
     torch.cuda.synchronize()
     assert float(g["ddt_bias"].abs().sum()) == 0.0
+
+
+# ---------------------------------------------------------------------------
+# the decode step with the discretisation fused ahead
+# ---------------------------------------------------------------------------
+def _raw_steps(Bsz, H, N, G, K, io, n, seed):
+    rng = np.random.default_rng(seed)
+    st = lambda *sh, s=1.0: W.store((s * rng.standard_normal(sh)).astype(np.float32), io)
+    return [dict(x=None, dd_dt=st(Bsz, H, s=0.5), dd_a=st(Bsz, H), trap=st(Bsz, H),
+                 angles=st(Bsz, K), B_raw=st(Bsz, G, N), C_raw=st(Bsz, G, N), z=None)
+            for _ in range(n)]
+
+
+def _carried(Bsz, H, P, N, K, seed):
+    rng = np.random.default_rng(seed)
+    f = lambda *sh: (0.5 * rng.standard_normal(sh)).astype(np.float32)
+    return [f(Bsz, H, P, N), f(Bsz, H, P), f(Bsz, H, N), f(Bsz, H, K)]
+
+
+DEC_CASES = [
+    # (B, H, P, N, G, K, io)
+    (2, 4, 16, 16, 1, 8, "f32"),
+    (3, 6, 64, 64, 2, 32, "bf16"),
+    (2, 4, 32, 128, 1, 48, "bf16"),
+    (2, 3, 64, 192, 3, 96, "f16"),
+    (1, 2, 16, 32, 1, 0, "f32"),
+]
+
+
+@pytest.mark.parametrize("case", DEC_CASES, ids=[f"B{c[0]}H{c[1]}P{c[2]}N{c[3]}G{c[4]}K{c[5]}{c[6]}"
+                                                 for c in DEC_CASES])
+def test_fused_decode_equals_unfused(msc, case):
+    """Ten chained decode steps from raw values: the fused step gives the bits
+    of the discretisation kernel (one token) followed by the plain step."""
+    Bsz, H, P, N, G, K, io = case
+    rng = np.random.default_rng(N + H)
+    steps = _raw_steps(Bsz, H, N, G, K, io, 10, N)
+    xs = [W.store(rng.standard_normal((Bsz, H, P)).astype(np.float32), io) for _ in steps]
+    zs = [W.store(rng.standard_normal((Bsz, H, P)).astype(np.float32), io) for _ in steps]
+    dtb = dev(rng.standard_normal(H).astype(np.float32))
+    Dp = dev(rng.standard_normal(H).astype(np.float32))
+    c0 = _carried(Bsz, H, P, N, K, 3)
+    ca = [dev(v) for v in c0]
+    cb = [dev(v) for v in c0]
+    for s, x, z in zip(steps, xs, zs):
+        r = {k: dev(v) for k, v in s.items() if v is not None}
+        if K == 0:
+            r["angles"] = None
+        oa = msc.msc_mamba3_siso_disc_state_update(*ca, dev(x), r["dd_dt"], r["dd_a"], r["trap"],
+                                                   r["angles"], r["B_raw"], r["C_raw"],
+                                                   dt_bias=dtb, A_floor=0.05, eps=1e-5, D=Dp,
+                                                   z=dev(z))
+        one = lambda t: None if t is None else t.unsqueeze(1).contiguous()
+        d = msc.msc_mamba3_siso_discretize(one(r["dd_dt"]), one(r["dd_a"]), one(r["trap"]),
+                                           one(r["angles"]) if K else None, one(r["B_raw"]),
+                                           one(r["C_raw"]), dt_bias=dtb, A_floor=0.05, eps=1e-5)
+        ob = msc.msc_mamba3_siso_state_update(*cb, dev(x), d["B"][:, 0].contiguous(),
+                                              d["C"][:, 0].contiguous(), d["alpha"][:, 0].contiguous(),
+                                              d["beta"][:, 0].contiguous(), d["gamma"][:, 0].contiguous(),
+                                              d["theta"][:, 0].contiguous(), D=Dp, z=dev(z))
+        torch.cuda.synchronize()
+        assert torch.equal(oa, ob)
+    for u, v in zip(ca, cb):
+        assert torch.equal(u, v)
+
+
+def test_fused_decode_vs_oracle(msc):
+    """Chained fused decode steps against the oracle's discretisation (each
+    value rounded to the io type, as stored) followed by its decode step."""
+    Bsz, H, P, N, G, K, io = 2, 4, 64, 64, 1, 32, "bf16"
+    rng = np.random.default_rng(9)
+    steps = _raw_steps(Bsz, H, N, G, K, io, 8, 1)
+    dtb = rng.standard_normal(H).astype(np.float32)
+    Dp = rng.standard_normal(H).astype(np.float32)
+    c0 = _carried(Bsz, H, P, N, K, 5)
+    cg = [dev(v) for v in c0]
+    cr = [v.astype(np.float64) for v in c0]
+    for s in steps:
+        x = W.store(rng.standard_normal((Bsz, H, P)).astype(np.float32), io)
+        z = W.store(rng.standard_normal((Bsz, H, P)).astype(np.float32), io)
+        o = msc.msc_mamba3_siso_disc_state_update(
+            *cg, dev(x), dev(s["dd_dt"]), dev(s["dd_a"]), dev(s["trap"]), dev(s["angles"]),
+            dev(s["B_raw"]), dev(s["C_raw"]), dt_bias=dev(dtb), A_floor=1e-4, eps=1e-5,
+            D=dev(Dp), z=dev(z))
+        one = lambda t: t.as_f64()[:, None]
+        d = oracle.m3_discretize(one(s["dd_dt"]), one(s["dd_a"]), one(s["trap"]),
+                                 one(s["angles"]), one(s["B_raw"]), one(s["C_raw"]),
+                                 dt_bias=dtb.astype(np.float64), A_floor=1e-4, eps=1e-5)
+        d = {k: W.store(v[:, 0].astype(np.float32), io).as_f64() for k, v in d.items()}
+        *cr, o_ref = oracle.m3_state_update(*cr, x.as_f64(), d["B"], d["C"], d["alpha"],
+                                            d["beta"], d["gamma"], d["theta"],
+                                            D=Dp.astype(np.float64), z=z.as_f64())
+        torch.cuda.synchronize()
+        assert_close("out", host(o), o_ref, TOL["bf16"])
+    assert_close("state", host(cg[0]), cr[0], TOL["bf16"])
