@@ -24,9 +24,12 @@
 // first lanes of a head (its first warp, or half-warp when a warp holds two
 // heads) derive dt, alpha, beta, gamma from dd_dt, dd_a, trap and the RMS
 // scales of the head's raw B and C rows, and the rotating threads take
-// theta = dt angles.  Every derived value is rounded to the io type and the
-// row sums follow the discretisation kernel's order, so the fused step gives
-// the same bits as the discretisation kernel followed by the plain step.
+// theta = dt angles.  Up to 64 states the rotating lanes hold the whole row,
+// so everything comes from one round of loads and shuffles; wider states
+// take a pass over the raw rows first.  Every derived value is rounded to
+// the io type and the row sums follow the discretisation kernel's order, so
+// the fused step gives the same bits as the discretisation kernel followed
+// by the plain step.
 #include "kernels.h"
 #include "m3_disc_common.cuh"
 
@@ -87,6 +90,28 @@ __device__ __forceinline__ float raw_rms_scale(const void *raw, int64_t row, boo
   return rsqrtf(ss / (float)N + eps);
 }
 
+// The same scale when the row (N = 16, 32 or 64) is held in registers, two
+// consecutive entries (e0, e1) per lane j < N / 2 of a group of kLW lanes:
+// the discretisation kernel's lane l (8 entries) is lanes 4 l .. 4 l + 3 here,
+// so its running sum is passed along those four lanes, and its xor tree over
+// l becomes one over lane distances 4, 8, 16.  Lane 3 of the group ends with
+// the sum and broadcasts the scale.  Every lane of the warp calls it.
+template <int N, int kLW>
+__device__ __forceinline__ float pair_rms_scale(float e0, float e1, int j, float eps) {
+  constexpr int kS = disc_row_lanes(N);
+  static_assert(kS > 0 && 4 * kS <= kLW && N <= 64, "the row sits in one lane group");
+  float s = fmaf(e1, e1, __fmul_rn(e0, e0));
+#pragma unroll
+  for (int r = 1; r < 4; ++r) {
+    const float prev = __shfl_up_sync(0xffffffffu, s, 1);
+    if ((j & 3) == r) s = fmaf(e1, e1, fmaf(e0, e0, prev));
+  }
+#pragma unroll
+  for (int m = 1; m < kS; m <<= 1) s += __shfl_xor_sync(0xffffffffu, s, 4 * m);
+  s = __shfl_sync(0xffffffffu, s, 3, kLW);
+  return rsqrtf(s / (float)N + eps);
+}
+
 template <typename T, int P, int N, bool kRaw>
 __global__ void __launch_bounds__(kSUThreads) m3_state_update_kernel(const M3SUParams p) {
   constexpr int kSN = N < 64 ? N : 64;     // states per slab (wider states: slabs of 64 in turn)
@@ -136,9 +161,9 @@ __global__ void __launch_bounds__(kSUThreads) m3_state_update_kernel(const M3SUP
 #pragma unroll
       for (int i = 0; i < 4; ++i) st[i] = srow[n0 / 4 + i * kTPR + q];
     }
-    if constexpr (kRaw) {
-      // (first slab, after the state loads are under way) the head's dt, alpha,
-      // beta, gamma and the scales of its raw B and C rows
+    if constexpr (kRaw && kNS > 1) {
+      // (wide states; first slab, after the state loads are under way) the
+      // head's dt, alpha, beta, gamma and the scales of its raw B and C rows
       if (sl == 0 && j < kLW) {  // the head's first lanes; every lane of their warp is here
         float *sCoef = sXp + P;
         if (live) {
@@ -158,7 +183,54 @@ __global__ void __launch_bounds__(kSUThreads) m3_state_update_kernel(const M3SUP
                          0, kLW);
       }
     }
-    if (live) {
+    if constexpr (kRaw && kNS == 1) {
+      // the whole row in one slab: the rotating lanes load their raw pairs,
+      // the angle and the head's raw scalars together, derive the coefficients
+      // and the row scales in registers, and rotate
+      if (j < kLW) {  // every lane of the warp is here
+        const bool rot = live && j < kSN / 2;
+        const int64_t o = (b * p.G + g) * N + 2 * j;
+        float e0 = 0.f, e1 = 0.f, f0 = 0.f, f1 = 0.f, ang = 0.f;
+        if (rot) {
+          e0 = ldf<T>(p.B_raw, o); e1 = ldf<T>(p.B_raw, o + 1);
+          f0 = ldf<T>(p.C_raw, o); f1 = ldf<T>(p.C_raw, o + 1);
+          if (j < K) ang = ldf<T>(p.angles, b * K + j);
+        }
+        if (live) {
+          const DiscCoef c = disc_coef(ldf<T>(p.dd_dt, bh), p.dt_bias ? p.dt_bias[h] : 0.f,
+                                       ldf<T>(p.dd_a, bh), ldf<T>(p.trap, bh), p.A_floor);
+          dt = c.dt;
+          if (j == 0) {
+            float *sCoef = sXp + P;
+            sCoef[0] = to_f32(from_f32<T>(c.alpha));
+            sCoef[1] = to_f32(from_f32<T>(disc_beta(c)));
+            sCoef[2] = to_f32(from_f32<T>(disc_gamma(c)));
+          }
+        }
+        rB = pair_rms_scale<N, kLW>(e0, e1, j, p.eps);
+        rC = pair_rms_scale<N, kLW>(f0, f1, j, p.eps);
+        if (rot) {
+          float b0 = to_f32(from_f32<T>(__fmul_rn(e0, rB)));
+          float b1 = to_f32(from_f32<T>(__fmul_rn(e1, rB)));
+          float c0 = to_f32(from_f32<T>(__fmul_rn(f0, rC)));
+          float c1 = to_f32(from_f32<T>(__fmul_rn(f1, rC)));
+          if (j < K) {
+            const float th = to_f32(from_f32<T>(__fmul_rn(dt, ang)));
+            const float phi = p.phi[bh * K + j] + th;
+            p.phi[bh * K + j] = phi;
+            float sn, cs;
+            sincosf(phi, &sn, &cs);
+            const float rb0 = cs * b0 - sn * b1, rb1 = sn * b0 + cs * b1;
+            const float rc0 = cs * c0 - sn * c1, rc1 = sn * c0 + cs * c1;
+            b0 = rb0; b1 = rb1; c0 = rc0; c1 = rc1;
+          }
+          sBt[2 * j] = b0; sBt[2 * j + 1] = b1;
+          sCt[2 * j] = c0; sCt[2 * j + 1] = c1;
+        }
+      }
+      if (live)
+        for (int i = j; i < kSN; i += kTPH) sBp[i] = p.bt_prev[bh * N + n0 + i];
+    } else if (live) {
       if (j < kSN / 2) {
         const int ka = n0 / 2 + j;  // global angle pair
         const int64_t o = (b * p.G + g) * N + n0 + 2 * j;
