@@ -89,11 +89,65 @@ __global__ void __launch_bounds__(256) state_update_kernel(const SUParams p) {
   static_cast<T *>(p.out)[i] = from_f32<T>(y);
 }
 
+// The same step for a compile-time N (16): every load of the row (its
+// state, B, C and A pieces) is issued before the first store, so a thread has
+// all of them in flight at once instead of one 8-state group at a time.  The
+// arithmetic is the kernel above's, operation for operation.
+template <typename T, int kN>
+__global__ void __launch_bounds__(256) state_update_fixed_kernel(const SUParams p) {
+  static_assert(kN % 8 == 0, "rows of 8-element runs");
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t D = p.D;
+  if (i >= p.B * D) return;
+  const int64_t b = i / D, c = i % D, g = c / (D / p.G);
+  const T *Bp = static_cast<const T *>(p.Bm) + (b * p.G + g) * kN;
+  const T *Cp = static_cast<const T *>(p.Cm) + (b * p.G + g) * kN;
+  const float4 *Ap = reinterpret_cast<const float4 *>(p.A + c * kN);
+  float4 *st = reinterpret_cast<float4 *>(p.state + i * kN);
+  float4 h4[kN / 4], A4[kN / 4];
+  float bv[kN / 8][8], cv[kN / 8][8];
+#pragma unroll
+  for (int k = 0; k < kN / 4; ++k) h4[k] = st[k];
+#pragma unroll
+  for (int k = 0; k < kN / 8; ++k) {
+    load_run<8, Cache::kKeep>(Bp, 8 * k, kN, true, bv[k], 0.f);
+    load_run<8, Cache::kKeep>(Cp, 8 * k, kN, true, cv[k], 0.f);
+  }
+#pragma unroll
+  for (int k = 0; k < kN / 4; ++k) A4[k] = __ldg(Ap + k);
+  const float x = to_f32(static_cast<const T *>(p.x)[i]);
+  const float v = to_f32(static_cast<const T *>(p.delta)[i]) + (p.bias ? p.bias[c] : 0.f);
+  const float zv = p.z ? to_f32(static_cast<const T *>(p.z)[i]) : 0.f;
+  const float d = p.softplus ? softplus(v) : v;
+  const float dtx = d * x;
+  float y = (p.Dp ? p.Dp[c] : 0.f) * x;
+#pragma unroll
+  for (int k = 0; k < kN / 4; ++k) {
+    const float *bq = &bv[k / 2][(k & 1) * 4];
+    const float *cq = &cv[k / 2][(k & 1) * 4];
+    float2 h01 = make_float2(h4[k].x, h4[k].y), h23 = make_float2(h4[k].z, h4[k].w);
+    const float2 a01 = ex2_2(mul2(splat2(d), mul2(make_float2(A4[k].x, A4[k].y), splat2(kLog2e))));
+    const float2 a23 = ex2_2(mul2(splat2(d), mul2(make_float2(A4[k].z, A4[k].w), splat2(kLog2e))));
+    h01 = fma2(a01, h01, mul2(splat2(dtx), make_float2(bq[0], bq[1])));
+    h23 = fma2(a23, h23, mul2(splat2(dtx), make_float2(bq[2], bq[3])));
+    y = fmaf(cq[0], h01.x, y);
+    y = fmaf(cq[1], h01.y, y);
+    y = fmaf(cq[2], h23.x, y);
+    y = fmaf(cq[3], h23.y, y);
+    st[k] = make_float4(h01.x, h01.y, h23.x, h23.y);
+  }
+  if (p.z) y *= silu(zv);
+  static_cast<T *>(p.out)[i] = from_f32<T>(y);
+}
+
 template <typename T>
 cudaError_t launch_t(const SUParams &p, cudaStream_t s) {
   const int64_t rows = p.B * p.D;
   const unsigned blocks = (unsigned)((rows + 255) / 256);
-  state_update_kernel<T><<<blocks, 256, 0, s>>>(p);
+  if (p.N == 16)  // (at 32 states the row in registers would halve the occupancy)
+    state_update_fixed_kernel<T, 16><<<blocks, 256, 0, s>>>(p);
+  else
+    state_update_kernel<T><<<blocks, 256, 0, s>>>(p);
   return cudaGetLastError();
 }
 
