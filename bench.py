@@ -946,6 +946,21 @@ def run_only(args):
         cs.conv_bwd()
         fn = {"m1_conv_fwd": cs.fused_fwd, "conv_fwd": cs.conv_fwd, "conv_bwd": cs.conv_bwd}[phase]
         units = q.scan.token_channels
+    elif phase == "m3_decode_raw":
+        q = W.make(args.workload or "m3su_bf16_b256_h24_p64_n64_k32_x1000")
+        carried = [torch.from_numpy(v).cuda() for v in (q.state0, q.x_prev0, q.bt_prev0, q.phi0)]
+        D3 = to_dev(q.D)
+        s = {k: to_dev(v) for k, v in q.steps[0].items()}
+        raw_steps, dtb = W.m3su_raw_steps(q.batch, q.nheads, q.dstate, nangles=q.nangles)
+        r = {k: to_dev(v) for k, v in raw_steps[0].items()}
+        dtb_d = to_dev(dtb)
+        out = torch.empty_like(s["x"])
+
+        def fn():
+            msc.msc_mamba3_siso_disc_state_update(*carried, s["x"], r["dd_dt"], r["dd_a"],
+                                                  r["trap"], r["angles"], r["B_raw"], r["C_raw"],
+                                                  dt_bias=dtb_d, D=D3, z=s["z"], out=out)
+        units = q.batch * q.nheads * q.headdim
     elif phase == "m3_decode":
         q = W.make(args.workload or "m3su_bf16_b256_h24_p64_n64_k32_x1000")
         carried = [torch.from_numpy(v).cuda() for v in (q.state0, q.x_prev0, q.bt_prev0, q.phi0)]
@@ -1029,7 +1044,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", choices=["m1_fwd", "m1_bwd", "m3_fwd", "m3_bwd", "decode",
                                        "m3_decode", "m1_conv_fwd", "conv_fwd", "conv_bwd",
-                                       "m3_disc_fwd", "m3_disc_bwd"],
+                                       "m3_disc_fwd", "m3_disc_bwd", "m3_decode_raw"],
                     help="time one phase alone (for profiling); prints no bench line")
     ap.add_argument("--workload", default=None, help="workload name for --only")
     ap.add_argument("--graph", action="store_true",
