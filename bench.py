@@ -92,6 +92,15 @@ def m3su_bytes(Bsz, H, P, N, G, K, io_bytes):
     return Bsz * H * per_head + 2 * Bsz * G * N * io_bytes
 
 
+def m3su_raw_bytes(Bsz, H, P, N, G, K, io_bytes):
+    """The Mamba-3 decode step from raw values: the plain step's bytes with
+    alpha, beta, gamma, theta per (b, h) and the normalised B, C replaced by
+    dd_dt, dd_a, trap per (b, h), the angles per b and the raw B, C (same
+    size); dt_bias is small."""
+    return (m3su_bytes(Bsz, H, P, N, G, K, io_bytes) - Bsz * H * (3 + K) * io_bytes
+            + Bsz * H * 3 * io_bytes + Bsz * K * io_bytes)
+
+
 # ---------------------------------------------------------------------------
 # DRAM traffic of the dominant kernel from an ncu capture (dram__bytes_read.sum
 # + dram__bytes_write.sum, one launch of the named workload), valid only for
@@ -800,10 +809,12 @@ def extra_workloads(msc, args, world, peaks):
 
     _, (ms_f,) = time_steps([m3_decode_raw_1000], 2, 1, world)
     _, (ms_u,) = time_steps([m3_decode_raw_unfused_1000], 2, 1, world)
+    rb3 = m3su_raw_bytes(q3.batch, q3.nheads, q3.headdim, q3.dstate, q3.ngroups, q3.nangles, 2)
     res["m3su_raw_bf16_b256_h24_p64_n64_k32_x1000"] = dict(
         us_per_step=round(ms_f, 3), unfused_us_per_step=round(ms_u, 3),
         value=round(q3.batch * q3.nheads * q3.headdim * 1000 / (ms_f / 1e3), 1),
         unit="token-channel steps/s",
+        hbm_frac=round(rb3 * 1000 / (ms_f / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
         note="decode from raw dd_dt, dd_a, trap, angles, B_raw, C_raw: the discretisation "
              "fused into the step vs its own kernel ahead of the plain step")
     del carried, pool3, outs3

@@ -90,3 +90,11 @@ def test_oracle_beside_fills_every_workload():
     for n in names[1:]:
         o = res[n]["oracle"]
         assert o["kind"] == "oracle" and o["value"] > 0 and o["unit"] == "u" and o["sample"]
+
+
+def test_m3_decode_raw_bytes():
+    B, H, P, N, G, K, io = 256, 24, 64, 64, 1, 32, 2
+    plain = bench.m3su_bytes(B, H, P, N, G, K, io)
+    raw = bench.m3su_raw_bytes(B, H, P, N, G, K, io)
+    # theta [B, H, K] (and alpha .. gamma) out; dd_dt, dd_a, trap [B, H] and angles [B, K] in
+    assert plain - raw == B * H * K * io - B * K * io
