@@ -299,8 +299,8 @@ msc_status msc_causal_conv1d_bwd(const msc_conv_bwd_args *args, void *workspace,
 
 /*
  * The conv fused ahead of the Mamba-1 scan forward: one launch computes
- * u = silu(conv(x)) per token as the scan consumes it, so u never makes a
- * round trip through memory.  scan->u holds x (the conv's input, io
+ * u = silu(conv(x)) per token as the scan consumes it, so u is never read
+ * back from memory (and written only when u_out asks for it).  scan->u holds x (the conv's input, io
  * [B, D, L]); every other field of scan keeps its meaning in
  * msc_selective_scan_fwd, and conv gives the conv's parameters with the
  * layouts of msc_conv_fwd_args.  u_out (optional, io [B, D, L]) receives
