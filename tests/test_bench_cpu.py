@@ -98,3 +98,22 @@ def test_m3_decode_raw_bytes():
     raw = bench.m3su_raw_bytes(B, H, P, N, G, K, io)
     # theta [B, H, K] (and alpha .. gamma) out; dd_dt, dd_a, trap [B, H] and angles [B, K] in
     assert plain - raw == B * H * K * io - B * K * io
+
+
+def test_reference_arm_prints_one_line():
+    """`bench.py --impl reference` (the oracle on the host) prints one JSON line
+    with the contract's keys, on the headline's metric and workload."""
+    import json
+    import subprocess
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--steps", "1", "--warmup", "3"], capture_output=True, text=True,
+                       timeout=600, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["steps"] == 1 and d["warmup"] >= 3
+    assert d["metric"] == bench.METRIC and d["config"]["workload"] == bench.HEADLINE
+    assert d["value"] > 0 and d["higher_is_better"] is True
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
