@@ -47,6 +47,17 @@ __device__ __forceinline__ float softplus(float v) {
   return __logf(1.f + e);
 }
 
+// sin and cos of a cumulative angle: Cody and Waite's additive reduction by
+// 2 pi, the constant split as 6.28125 (8 significant bits, so n * 6.28125 is
+// exact for |n| < 2^16) plus the remainder 2 pi - 6.28125, then the SFU's sin
+// and cos on [-pi, pi] (absolute error about 2^-21)
+__device__ __forceinline__ void sincos_reduced(float phi, float &sn, float &cs) {
+  const float n = rintf(phi * 0.15915494309189535f);
+  float r = fmaf(-n, 6.28125f, phi);
+  r = fmaf(-n, 1.9353071795864769e-3f, r);
+  __sincosf(r, &sn, &cs);
+}
+
 // sigmoid(v) = 1 / (1 + e^-v), evaluated from e^-|v| so that it stays finite.
 __device__ __forceinline__ float sigmoid(float v) {
   const float e = __expf(-fabsf(v));

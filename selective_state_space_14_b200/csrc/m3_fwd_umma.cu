@@ -110,17 +110,6 @@ __device__ __forceinline__ void put3x2(unsigned char *base, int stride, int off,
   for (int q = 0; q < 3; ++q) *reinterpret_cast<uint32_t *>(base + q * stride + off) = w[q];
 }
 
-// sin and cos of a cumulative angle: Cody and Waite's additive reduction by
-// 2 pi, the constant split as 6.28125 (8 significant bits, so n * 6.28125 is
-// exact for |n| < 2^16) plus the remainder 2 pi - 6.28125, then the SFU's sin
-// and cos on [-pi, pi] (absolute error about 2^-21)
-__device__ __forceinline__ void sincos_reduced(float phi, float &sn, float &cs) {
-  const float n = rintf(phi * 0.15915494309189535f);
-  float r = fmaf(-n, 6.28125f, phi);
-  r = fmaf(-n, 1.9353071795864769e-3f, r);
-  __sincosf(r, &sn, &cs);
-}
-
 // Issue one product into TMEM column `col`: parts of A (nA of them, planes at
 // aA, stride sA, K-major with Ka columns, 64 rows) times parts of B (nB,
 // planes at aB, stride sB; K-major with Kb columns, or with kBMN the same

@@ -219,7 +219,7 @@ __global__ void __launch_bounds__(kSUThreads) m3_state_update_kernel(const M3SUP
             const float phi = p.phi[bh * K + j] + th;
             p.phi[bh * K + j] = phi;
             float sn, cs;
-            sincosf(phi, &sn, &cs);
+            sincos_reduced(phi, sn, cs);
             const float rb0 = cs * b0 - sn * b1, rb1 = sn * b0 + cs * b1;
             const float rc0 = cs * c0 - sn * c1, rc1 = sn * c0 + cs * c1;
             b0 = rb0; b1 = rb1; c0 = rc0; c1 = rc1;
@@ -252,7 +252,7 @@ __global__ void __launch_bounds__(kSUThreads) m3_state_update_kernel(const M3SUP
           const float phi = p.phi[bh * K + ka] + th;
           p.phi[bh * K + ka] = phi;
           float sn, cs;
-          sincosf(phi, &sn, &cs);
+          sincos_reduced(phi, sn, cs);
           const float rb0 = cs * b0 - sn * b1, rb1 = sn * b0 + cs * b1;
           const float rc0 = cs * c0 - sn * c1, rc1 = sn * c0 + cs * c1;
           b0 = rb0; b1 = rb1; c0 = rc0; c1 = rc1;
