@@ -15,7 +15,8 @@
 // four 16-byte pieces interleaved with its row neighbours' (so that the
 // threads of a row read and write one contiguous run per instruction).  A
 // CTA of 256 threads serves 256 / (P N / 16) heads.  Per head, the first N/2
-// threads rotate one pair of B and C each into shared memory; y sums a row's
+// threads rotate one pair of B and C each into shared memory (sin and cos by
+// Cody and Waite's reduction and the SFU, common.cuh); y sums a row's
 // partials over its N / 16 threads with shuffles in a fixed order.  Wider
 // states (128, 192, 256) are walked in slabs of 64 states with the 64-state
 // layout, y carried across the slabs in registers.
