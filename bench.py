@@ -5,8 +5,9 @@
                     [--no-extra] [--no-cpu-baseline]
 
 One step = the Mamba-1 selective scan forward + backward over one batch of the
-Mamba-130M-layer-shaped workload (bf16 storage, f32 accumulation; batch 8,
-d_inner 1536, d_state 16, L 2048), inputs resident in HBM.  Metric:
+Mamba-2.8B-layer-shaped workload (bf16 storage, f32 accumulation; batch 4,
+d_inner 5120, d_state 16, L 4096, final state returned), inputs resident in
+HBM.  Metric:
 tokens*channels per second (B*L*D per step / step time), whole job over all
 ranks.  Under torchrun each rank runs its own batch (independent problems, no
 data-path collective: weak scaling); timing is taken with CUDA events on the
@@ -15,9 +16,11 @@ launching stream, bracketed by a barrier and a synchronize, max over ranks.
 The JSON line also carries: the roofline of the dominant launch (algorithmic
 bytes / measured duration vs the measured HBM copy bandwidth), the e2e figure
 (the same step through the C ABI starting from pinned host buffers, copies
-inside the timed region), the CPU oracle timed on a bounded sample, SM clocks
-sampled during the timed region, and per-workload figures for the other
-workloads (2.8B-layer-shaped Mamba-1, Mamba-3 SISO, decode step).
+inside the timed region), the compute ceiling of the Mamba-1 kernels (their
+2^x count over the SFU rate measured by the library's probe in the same run),
+the CPU oracle timed on a bounded sample, SM clocks sampled during the timed
+region, and per-workload figures for the other workloads (130M-layer-shaped
+Mamba-1, Mamba-3 SISO, decode steps, conv, discretisation).
 
 --impl reference runs the f64 CPU oracle (the reference arm of this build) on a
 bounded sample of the same workload and prints the same metric.
@@ -42,7 +45,7 @@ from selective_state_space_14_b200 import workloads as W  # noqa: E402
 
 METRIC = "selective-scan tokens·channels/s (fwd+bwd) and achieved HBM GB/s vs ~8 TB/s peak"
 UNIT = "tokens*channels/s"
-HEADLINE = "m1_bf16_b8_d1536_n16_l2048"
+HEADLINE = "m1_bf16_b4_d5120_n16_l4096"
 L2_BYTES = 126 * 1024 * 1024
 
 
@@ -68,6 +71,16 @@ def m1_bytes(Bsz, D, N, L, io_bytes, G=1):
     fwd = 4 * io_bytes * tc + 2 * N * io_bytes * bt + params + Bsz * D * N * 4  # x,dt,z,out; B,C; final
     bwd = 7 * io_bytes * tc + 2 * N * io_bytes * bt + 2 * N * 4 * bt + params + D * N * 4 + 2 * D * 4
     return fwd, bwd
+
+
+def m1_sfu_ops(Bsz, D, N, L):
+    """SFU operations of the Mamba-1 kernels: one 2^x per state element and
+    step (its decay; the backward recomputes it once), plus per token the
+    forward's softplus (2^x and a reciprocal or logarithm) and silu gate
+    (2^x and a reciprocal), and the backward's softplus, sigmoid of the gate
+    and sigmoid of the delta pre-activation (two each)."""
+    tc = Bsz * D * L
+    return tc * (N + 4), tc * (N + 6)
 
 
 def m3_bytes(Bsz, L, H, P, N, G, K, io_bytes):
@@ -109,14 +122,14 @@ def m3su_raw_bytes(Bsz, H, P, N, G, K, io_bytes):
 # ---------------------------------------------------------------------------
 NCU_TRAFFIC = {
     # kernel source file: (sha256 prefix of the file, workload, bytes per launch)
-    "m1_bwd.cu": ("4523265612d28912", "m1_bf16_b8_d1536_n16_l2048", 404786688 + 159501312),
+    "m1_bwd.cu": ("4523265612d28912", "m1_bf16_b4_d5120_n16_l4096", 1350000000 + 591390000),
 }
 
 
-def ncu_traffic(src_name):
+def ncu_traffic(src_name, workload):
     import hashlib
     ent = NCU_TRAFFIC.get(src_name)
-    if ent is None:
+    if ent is None or ent[1] != workload:
         return None
     path = os.path.join(ROOT, "selective_state_space_14_b200", "csrc", src_name)
     try:
@@ -435,6 +448,36 @@ def time_steps(step_fns, steps, warmup, world, sampler=None):
     return total_ms, phase_ms
 
 
+def measure_rates(msc, reps=3):
+    """The SFU's 2^x rate and the FMA pipe's (scalar and packed) on this GPU,
+    from the library's probes: 8 CTAs of 256 threads per SM, best of ``reps``
+    CUDA-event timed launches after one warm-up (a burst rate, like the
+    measured copy bandwidth the HBM fraction divides by)."""
+    import torch
+    props = torch.cuda.get_device_properties(torch.cuda.current_device())
+    blocks = props.multi_processor_count * 8
+    out = torch.empty(blocks * int(msc.lib().msc_probe_threads_per_block()), device="cuda",
+                      dtype=torch.float32)
+    stream = torch.cuda.current_stream()
+    rates = {}
+    for kind, iters in (("ex2", 2048), ("ffma", 16384), ("ffma2", 8192)):
+        msc.msc_probe(kind, out, blocks, iters)
+        best = None
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            ops = msc.msc_probe(kind, out, blocks, iters)
+            b.record(stream)
+            b.synchronize()
+            ms = a.elapsed_time(b)
+            best = ms if best is None else min(best, ms)
+        rates[kind] = ops / (best / 1e3)
+    return dict(sfu_ex2_per_s=round(rates["ex2"], 1), ffma_per_s=round(rates["ffma"], 1),
+                ffma2_elem_per_s=round(rates["ffma2"], 1), sms=props.multi_processor_count,
+                how="libmsc probes: 8 CTAs x 256 threads per SM, 8 independent chains per "
+                    "thread, best of 3 CUDA-event timed launches")
+
+
 def cpu_baseline(budget_s=12.0):
     """The f64 oracle (as it stands) on a bounded sample of the headline workload:
     batch row 0 (all its channels, all steps), forward + backward, repeated for
@@ -508,13 +551,13 @@ def oracle_beside(res, budget_s=1.5):
                                    cores=thr, kind="oracle",
                                    sample=f"{sample}; {reps} reps, {t:.1f} s")
 
-    # Mamba-1, 2.8B-layer rows: one batch row of 256 channels, L 4096, fwd+bwd
-    p = W.m1_problem(1, 256, 16, 4096, io=BF, bias=True)
+    # Mamba-1, 130M-layer rows: one batch row of 256 channels, L 2048, fwd+bwd
+    p = W.m1_problem(1, 256, 16, 2048, io=BF, bias=True)
     a = oracle.m1_problem_args(p)
     dout = p.dout.as_f64()
-    put("m1_bf16_b4_d5120_n16_l4096", 256 * 4096,
+    put("m1_bf16_b8_d1536_n16_l2048", 256 * 2048,
         lambda: (oracle.m1_fwd(**a), oracle.m1_bwd(dout=dout, **a)),
-        "one batch row of 256 channels, L 4096, fwd+bwd")
+        "one batch row of 256 channels, L 2048, fwd+bwd")
     # Mamba-1 decode: 64 channels of one sequence, 10 steps
     q = W.su_problem(1, 64, 16, n_pool=10)
     steps = [{k: v.as_f64() for k, v in s_.items()} for s_ in q.steps]
@@ -679,13 +722,25 @@ def run_ours(args):
     dom = "bwd" if bwd_ms >= fwd_ms else "fwd"
     dom_ms, dom_b = (bwd_ms, bwd_b) if dom == "bwd" else (fwd_ms, fwd_b)
     achieved = dom_b / (dom_ms / 1e3) / 1e9
+    # the compute side: the kernels' 2^x count over the measured SFU rate
+    rates = measure_rates(msc)
+    fwd_ops, bwd_ops = m1_sfu_ops(p.batch, p.dim, p.dstate, p.seqlen)
+    sfu = rates["sfu_ex2_per_s"]
+
+    def compute(ops, ms):
+        floor_ms = ops / sfu * 1e3
+        return dict(bound="sfu", sfu_ops=ops, floor_ms=round(floor_ms, 4),
+                    achieved_ops_per_s=round(ops / (ms / 1e3), 1), peak_ops_per_s=sfu,
+                    frac=round(floor_ms / ms, 4))
+    compute_fwd, compute_bwd = compute(fwd_ops, fwd_ms), compute(bwd_ops, bwd_ms)
     roofline = dict(bound="hbm", achieved=round(achieved, 1), peak=peaks["hbm_gbs"], unit="GB/s",
                     frac=round(achieved / peaks["hbm_gbs"], 4),
-                    traffic=ncu_traffic("m1_bwd.cu" if dom == "bwd" else "m1_fwd.cu"),
+                    traffic=ncu_traffic("m1_bwd.cu" if dom == "bwd" else "m1_fwd.cu", HEADLINE),
                     kernel=("msc_selective_scan_bwd (m1_bwd_kernel + m1_bwd_reduce_kernel)"
                             if dom == "bwd" else "msc_selective_scan_fwd (m1_fwd_kernel)"),
                     algorithmic_bytes=dom_b, launch_ms=round(dom_ms, 4),
-                    peak_source=peaks["source"])
+                    peak_source=peaks["source"],
+                    compute=compute_bwd if dom == "bwd" else compute_fwd)
     e2e_ms, h2d, d2h = run_e2e(p, msc, max(2, args.steps // 2), 3, world)
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
@@ -698,6 +753,11 @@ def run_ours(args):
                    "l2": "per-step working set > 126 MB L2 (inputs larger than L2)"},
         "phases_ms": {"fwd": round(fwd_ms, 4), "bwd": round(bwd_ms, 4)},
         "achieved_gbs": {"fwd": round(fwd_b / fwd_ms / 1e6, 1), "bwd": round(bwd_b / bwd_ms / 1e6, 1)},
+        "hbm_frac": {"fwd": round(fwd_b / fwd_ms / 1e6 / peaks["hbm_gbs"], 4),
+                     "bwd": round(bwd_b / bwd_ms / 1e6 / peaks["hbm_gbs"], 4)},
+        "compute_frac": {"fwd": compute_fwd["frac"], "bwd": compute_bwd["frac"]},
+        "compute": {"fwd": compute_fwd, "bwd": compute_bwd},
+        "rates": rates,
         "roofline": roofline,
         "e2e": {"value": round(units * world / (e2e_ms / 1e3), 1), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -709,6 +769,7 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
     if not args.no_extra:
+        args.sfu_rate = rates["sfu_ex2_per_s"]
         line["workloads"] = extra_workloads(msc, args, world, peaks)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             oracle_beside(line["workloads"])
@@ -723,16 +784,23 @@ def extra_workloads(msc, args, world, peaks):
     """Per-workload figures beside the headline (each timed like the headline)."""
     import torch
     res = {}
-    # Mamba-2.8B-layer-shaped Mamba-1 scan (bf16, B4 D5120 N16 L4096, final state)
-    p = W.make("m1_bf16_b4_d5120_n16_l4096")
+    # Mamba-130M-layer-shaped Mamba-1 scan (bf16, B8 D1536 N16 L2048)
+    name = "m1_bf16_b8_d1536_n16_l2048"
+    p = W.make(name)
     st = M1Step(p, msc)
-    total_ms, (fwd_ms, bwd_ms) = time_steps([st.fwd, st.bwd], max(3, args.steps // 2), 3, world)
+    total_ms, (fwd_ms, bwd_ms) = time_steps([st.fwd, st.bwd], max(3, args.steps), 3, world)
     fb, bb = m1_bytes(p.batch, p.dim, p.dstate, p.seqlen, 2)
-    res["m1_bf16_b4_d5120_n16_l4096"] = dict(
+    fo, bo = m1_sfu_ops(p.batch, p.dim, p.dstate, p.seqlen)
+    sfu = getattr(args, "sfu_rate", None)
+    res[name] = dict(
         fwd_ms=round(fwd_ms, 4), bwd_ms=round(bwd_ms, 4),
         value=round(p.token_channels / ((fwd_ms + bwd_ms) / 1e3), 1), unit=UNIT,
         fwd_hbm_frac=round(fb / fwd_ms / 1e6 / peaks["hbm_gbs"], 4),
-        bwd_hbm_frac=round(bb / bwd_ms / 1e6 / peaks["hbm_gbs"], 4))
+        bwd_hbm_frac=round(bb / bwd_ms / 1e6 / peaks["hbm_gbs"], 4),
+        bwd_traffic=ncu_traffic("m1_bwd.cu", name))
+    if sfu:
+        res[name]["fwd_compute_frac"] = round(fo / sfu / (fwd_ms / 1e3), 4)
+        res[name]["bwd_compute_frac"] = round(bo / sfu / (bwd_ms / 1e3), 4)
     del st
     torch.cuda.empty_cache()
     # decode step (B256 D5120 N16, 1000 consecutive steps cycling 8 input sets)

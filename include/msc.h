@@ -202,7 +202,10 @@ msc_status msc_selective_scan_bwd(const msc_ss_bwd_args *args, void *workspace,
  * exceeds it are rejected with MSC_ERR_WORKSPACE (nothing launched).  The
  * first call on a device looks up the array's device address on that device
  * (cudaGetSymbolAddress); make that first call before any stream capture.
- * All calls share the array: calls that may overlap on the GPU race on it
+ * The address is kept for the life of the process, so the entry point must
+ * not be used across a cudaDeviceReset of that device (the reset may move the
+ * array).  Arguments are checked as msc_selective_scan_bwd checks them, before
+ * the scratch size is computed.  All calls share the array: calls that may overlap on the GPU race on it
  * and must be serialised by the caller.  Results equal those of
  * msc_selective_scan_bwd.  Allocates nothing, never synchronises.
  */
@@ -565,6 +568,34 @@ typedef struct {
 } msc_m3_disc_bwd_args;
 
 msc_status msc_mamba3_siso_discretize_bwd(const msc_m3_disc_bwd_args *args, msc_stream_t stream);
+
+/* ======================================================================
+ * Measurement probes: the compute ceiling of the Mamba-1 scans
+ * ======================================================================
+ * Every state element of every step of the Mamba-1 recurrence takes one
+ * 2^x for its decay exp(delta A) (the discretisation of the selective SSM,
+ * Mamba paper, Section 3 / Algorithm 2), so the GPU's rate of 2^x bounds the
+ * scans from below independently of their memory traffic (the pages quote
+ * "the step is dominated by the scan and the other non-GEMM kernels",
+ * mamba-rs 0.7.0 README, "Performance").  These probes measure that rate and
+ * the FMA pipe's, for the roofline's compute side.  They are not part of
+ * the scan path.
+ *
+ * Each launches `blocks` CTAs of msc_probe_threads_per_block() threads; a
+ * thread runs 8 independent chains for `iters` rounds and writes one float
+ * to out[thread] (caller-owned device memory of blocks * threads floats, its
+ * values meaningless).  *ops (host memory) receives the number of
+ * operations the launch performs: 2^x evaluations (ex2.approx.ftz.f32), or
+ * element fused multiply-adds (packed = 1: fma.rn.f32x2, two per
+ * instruction; packed = 0: scalar fma.rn.f32).  Time the launch with events
+ * on `stream`; rate = ops / time.  blocks must be in 1..2^20, iters in
+ * 1..2^24; otherwise MSC_ERR_INVALID_ARG and nothing is launched.
+ */
+int64_t msc_probe_threads_per_block(void);
+msc_status msc_probe_sfu_ex2(float *out, int64_t blocks, int64_t iters, int64_t *ops,
+                             msc_stream_t stream);
+msc_status msc_probe_ffma(float *out, int64_t blocks, int64_t iters, int32_t packed, int64_t *ops,
+                          msc_stream_t stream);
 
 #ifdef __cplusplus
 } /* extern "C" */

@@ -97,6 +97,13 @@ msc_status api_fail(msc_status st, const char *fmt, ...) {
   return st;
 }
 msc_status api_ok() { return ok(); }
+// the backward's checks of dtype, flags and sizes (before any size is computed)
+msc_status m1_bwd_check_sizes(const char *fn, const msc_ss_bwd_args *a) {
+  msc_status st;
+  if ((st = check_dtype(fn, a->io_dtype)) != MSC_OK) return st;
+  if ((st = check_flag(fn, "delta_softplus", a->delta_softplus)) != MSC_OK) return st;
+  return check_m1_sizes(fn, a->batch, a->dim, a->dstate, a->seqlen, a->ngroups);
+}
 msc_status api_cuda(cudaError_t e, const char *what) { return cuda_status(e, what); }
 }  // namespace msc
 
@@ -227,6 +234,8 @@ msc_status msc_selective_scan_conv_fwd(const msc_ss_fwd_args *scan,
 size_t msc_selective_scan_bwd_workspace_bytes(int64_t batch, int64_t dim, int64_t dstate,
                                               int64_t seqlen, int64_t ngroups) {
   if (batch <= 0 || dim <= 0 || dstate <= 0 || seqlen <= 0) return 0;
+  // sizes the backward refuses need no workspace (and ngroups is a divisor)
+  if (dstate > MSC_M1_MAX_DSTATE || ngroups < 1 || dim % ngroups != 0) return 0;
   return msc::m1_bwd_workspace_bytes(batch, dim, dstate, seqlen, ngroups);
 }
 

@@ -15,7 +15,10 @@
 // host-side shadow -- so the device address is looked up with
 // cudaGetSymbolAddress, once per device, with that device current, on the
 // first call made on that device.  Make that first call before any stream
-// capture.  All calls share the one array: calls whose executions overlap on
+// capture.  The address is kept for the life of the process: a
+// cudaDeviceReset (or anything else that tears down and rebuilds the device's
+// primary context) reloads the module and may move the array, so do not use
+// this entry point across such a reset.  All calls share the one array: calls whose executions overlap on
 // the GPU (different streams, or different host threads on one stream without
 // ordering) race on it and must be serialised by the caller.  The backward
 // kernels overwrite every scratch word they later read, so nothing in the
@@ -29,6 +32,7 @@
 
 namespace msc {
 msc_status api_fail(msc_status st, const char *fmt, ...);
+msc_status m1_bwd_check_sizes(const char *fn, const msc_ss_bwd_args *a);
 }  // namespace msc
 
 namespace {
@@ -48,6 +52,10 @@ extern "C" msc_status msc_selective_scan_bwd_static(const msc_ss_bwd_args *args,
   if (args->struct_size < sizeof(msc_ss_bwd_args))
     return msc::api_fail(MSC_ERR_INVALID_ARG, "%s: struct_size %u < sizeof(msc_ss_bwd_args) %zu",
                          fn, args->struct_size, sizeof(msc_ss_bwd_args));
+  // the backward's own argument checks first: the scratch size is computed
+  // from sizes that are known to be valid (ngroups >= 1 and a divisor of dim)
+  const msc_status st = msc::m1_bwd_check_sizes(fn, args);
+  if (st != MSC_OK) return st;
   const size_t need = msc_selective_scan_bwd_workspace_bytes(
       args->batch, args->dim, args->dstate, args->seqlen, args->ngroups);
   if (need > (size_t)MSC_STATIC_SCRATCH_BYTES)

@@ -17,7 +17,15 @@
 //   dgamma_s = sum_{tau>=s} d(tau,s) (Ct_tau.Bt_s)(g_tau.x_s) + alpha_Q d(Q-1,s) v_s
 //   dbeta_s  = sum_{tau>=s} d(tau,s) (Ct_tau.Bt_{s-1})(g_tau.x_{s-1}) + alpha_Q d(Q-1,s) v_{s-1}
 //     (v_s = x_s^T U Bt_s; index -1 is the previous chunk's last step)
-//   dalpha_r = (1/alpha_r) sum_{t>=r} [rowsum_t(E) - colsum_t(E)],  E(tau,s) = d(tau,s) dL/dd(tau,s)
+//   dalpha_s = <Lambda_s, S_{s-1}>, taken without any subtraction: every term of it
+//     carries alpha_s, so with the U row written as tau = Q (d(Q,.) = alpha_Q d(Q-1,.),
+//     c(Q,.) = alpha_Q c(Q-1,.), its "a" = <U, S_in>, "e" = v_{-1}, "M" = v) and
+//     M(tau,j) = (Ct_tau.Bt_j)(g_tau.x_j), a_tau = g_tau^T S_in Ct_tau,
+//     e_tau = (Ct_tau.Bt_prev)(g_tau.x_prev):
+//   dalpha_s = (1/alpha_s) sum_{tau=s..Q} [d(tau,-1) a_tau + beta_0 d(tau,0) e_tau
+//                                          + sum_{j<=s-2} c(tau,j) M(tau,j)]
+//              + gamma_{s-1} dbeta_s                                   (s >= 1)
+//   dalpha_0 = sum_{tau=0..Q} d(tau,0) a_tau
 // The RoPE backward rotates dBt, dCt back (R^T) per head, forms dphi and
 // the reverse cumulative sum dtheta; the per-head dB, dC go to the workspace
 // and a second kernel adds the heads of each group in ascending order.
@@ -347,20 +355,25 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
       }
       sDgam[s] = dg;
       sDbet[s] = db;
-      sColE[s] = sGa[s] * dg + sBe[s] * db;
     }
     for (int tau = tid; tau < kQ; tau += kThreads) {
-      // row tau of E: columns -1..tau
+      // a_tau = g_tau^T S_in Ct_tau
       float gs = 0.f;
       for (int n = 0; n < N; ++n) gs = fmaf(sT3[tau * lMx + n], sCt[tau * lN + n], gs);
-      float r = sDm[tau * (kQ + 1)] * gs;
-      for (int s = 0; s <= tau; ++s) {
-        const float m0 = sCB[tau * lQ + s] * sT2[tau * lMx + s];
-        const float m1 = s > 0 ? sCB[tau * lQ + s - 1] * sT2[tau * lMx + s - 1]
-                               : sCbp[tau] * sGxp[tau];
-        r = fmaf(sDm[tau * (kQ + 1) + s + 1], fmaf(sGa[s], m0, sBe[s] * m1), r);
-      }
-      sRowE[tau] = r;
+      sRowE[tau] = gs;
+    }
+    {
+      // the box sums sum_{tau>=s} sum_{j<=s-2} c(tau,j) M(tau,j) (c o M = W o G X^T),
+      // four threads per s (rows tau = s + part, s + part + 4, ...), added in a
+      // fixed butterfly
+      static_assert(kThreads == 4 * kQ, "four threads per step");
+      const int s = tid >> 2, part = tid & 3;
+      float acc = 0.f;
+      for (int tau = s + part; tau < kQ; tau += 4)
+        for (int j = 0; j <= s - 2; ++j) acc = fmaf(sW[tau * lQ + j], sT2[tau * lMx + j], acc);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+      if (part == 0) sColE[s] = acc;
     }
     __syncthreads();
     // c o G X^T replaces Ct Bt^T
@@ -424,19 +437,32 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
     }
     if (tid == 0) sV[-1] = vm1;
     __syncthreads();
-    float ex = 0.f;
     for (int s = tid; s < kQ; s += kThreads) {
       // parts that reach the next chunk through the last state
       const float dl = sDm[(kQ - 1) * (kQ + 1) + s + 1];
       const float fg = alQ * dl * sV[s], fb = alQ * dl * sV[s - 1];
       sDgam[s] += fg;
       sDbet[s] += fb;
-      sColE[s] += sGa[s] * fg + sBe[s] * fb;
-      ex = fmaf(alQ * dl, fmaf(sGa[s], sV[s], sBe[s] * sV[s - 1]), ex);
     }
-    {
-      const float extra = block_sum(ex, sRed) + alQ * sDm[(kQ - 1) * (kQ + 1)] * us;
-      if (tid == 0) sRowE[kQ - 1] += extra;  // column -1 and the U terms of row Q-1
+    __syncthreads();
+    // dalpha of the chunk (above): the suffix sums over tau, the U row, the
+    // box sums and gamma_{s-1} dbeta_s, each step by one thread in a fixed order
+    for (int s = tid; s < kQ; s += kThreads) {
+      float v;
+      if (s == 0) {
+        v = alQ * sDm[(kQ - 1) * (kQ + 1) + 1] * us;
+        for (int tau = kQ - 1; tau >= 0; --tau) v = fmaf(sDm[tau * (kQ + 1) + 1], sRowE[tau], v);
+      } else {
+        float a1 = alQ * fmaf(sBe[0] * sDm[(kQ - 1) * (kQ + 1) + 1], sV[-1],
+                              sDm[(kQ - 1) * (kQ + 1)] * us);
+        for (int tau = kQ - 1; tau >= s; --tau)
+          a1 += fmaf(sDm[tau * (kQ + 1)], sRowE[tau],
+                     sBe[0] * sDm[tau * (kQ + 1) + 1] * (sCbp[tau] * sGxp[tau]));
+        float bu = 0.f;  // the U row of the box sums: alpha_Q sum_{j<=s-2} c(Q-1,j) v_j
+        for (int j = 0; j <= s - 2; ++j) bu = fmaf(sCrow[j], sV[j], bu);
+        v = (a1 + sColE[s] + alQ * bu) / sAl[s] + sGa[s - 1] * sDbet[s];
+      }
+      sColE[s] = v;
     }
     __syncthreads();
     // ---- G. dCt ---------------------------------------------------------------------
@@ -448,32 +474,21 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
       v = fmaf(sBe[0] * sD0[t] * sGxp[t], sBprev[n], v);
       sT1[t * lMx + n] = v;
     }
-    // dalpha, dbeta, dgamma of this chunk: dalpha_r = (1/alpha_r) sum_{t>=r}
-    // (rowE_t - colE_t), a suffix scan over the chunk in warp 0 (lane l: steps
-    // 2l, 2l+1)
+    // dalpha (sColE), dbeta, dgamma of this chunk, warp 0 (lane l: steps 2l, 2l+1)
     if (tid < 32) {
       const int r0 = 2 * tid, r1 = 2 * tid + 1;
-      const float v0 = sRowE[r0] - sColE[r0], v1 = sRowE[r1] - sColE[r1];
-      float incl = v0 + v1;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const float o = __shfl_down_sync(0xffffffffu, incl, off);
-        if (tid + off < 32) incl += o;
-      }
-      float excl = __shfl_down_sync(0xffffffffu, incl, 1);
-      if (tid == 31) excl = 0.f;
-      const float a1 = excl + v1, a0 = a1 + v0;
+      const float a0 = sColE[r0], a1 = sColE[r1];
       // (slabs after the first add their sums over the states in place)
       const bool add = slab == kSlabMiddle || slab == kSlabLast;
       if (r0 < Qc) {
         const int64_t j = (b * L + t0 + r0) * H + h;
-        p.dalpha[j] = (add ? p.dalpha[j] : 0.f) + a0 / sAl[r0];
+        p.dalpha[j] = (add ? p.dalpha[j] : 0.f) + a0;
         p.dbeta[j] = (add ? p.dbeta[j] : 0.f) + sDbet[r0];
         p.dgamma[j] = (add ? p.dgamma[j] : 0.f) + sDgam[r0];
       }
       if (r1 < Qc) {
         const int64_t j = (b * L + t0 + r1) * H + h;
-        p.dalpha[j] = (add ? p.dalpha[j] : 0.f) + a1 / sAl[r1];
+        p.dalpha[j] = (add ? p.dalpha[j] : 0.f) + a1;
         p.dbeta[j] = (add ? p.dbeta[j] : 0.f) + sDbet[r1];
         p.dgamma[j] = (add ? p.dgamma[j] : 0.f) + sDgam[r1];
       }

@@ -141,7 +141,8 @@ EXPORTS = ["msc_last_error", "msc_version", "msc_selective_scan_saved_states_byt
            "msc_mamba3_siso_scan_bwd", "msc_mamba3_siso_state_update", "msc_causal_conv1d_fwd",
            "msc_causal_conv1d_bwd_workspace_bytes", "msc_causal_conv1d_bwd",
            "msc_selective_scan_conv_fwd", "msc_mamba3_siso_discretize",
-           "msc_mamba3_siso_discretize_bwd", "msc_mamba3_siso_disc_state_update"]
+           "msc_mamba3_siso_discretize_bwd", "msc_mamba3_siso_disc_state_update",
+           "msc_probe_threads_per_block", "msc_probe_sfu_ex2", "msc_probe_ffma"]
 
 _lib = None
 
@@ -192,6 +193,12 @@ def lib() -> ctypes.CDLL:
         L.msc_causal_conv1d_bwd_workspace_bytes.restype = ctypes.c_size_t
         L.msc_mamba3_siso_scan_bwd_workspace_bytes.argtypes = [_i64] * 7
         L.msc_mamba3_siso_scan_bwd_workspace_bytes.restype = ctypes.c_size_t
+        L.msc_probe_threads_per_block.argtypes = []
+        L.msc_probe_threads_per_block.restype = _i64
+        L.msc_probe_sfu_ex2.argtypes = [_vp, _i64, _i64, ctypes.POINTER(_i64), _vp]
+        L.msc_probe_sfu_ex2.restype = ctypes.c_int
+        L.msc_probe_ffma.argtypes = [_vp, _i64, _i64, ctypes.c_int32, ctypes.POINTER(_i64), _vp]
+        L.msc_probe_ffma.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -238,6 +245,23 @@ def msc_selective_scan_saved_states_bytes(batch, dim, dstate, seqlen) -> int:
 
 def msc_selective_scan_bwd_workspace_bytes(batch, dim, dstate, seqlen, ngroups=1) -> int:
     return int(lib().msc_selective_scan_bwd_workspace_bytes(batch, dim, dstate, seqlen, ngroups))
+
+
+def msc_probe(kind, out, blocks, iters, stream=None) -> int:
+    """Launch one rate probe ("ex2", "ffma" or "ffma2") into the float32 device
+    tensor ``out`` (blocks * msc_probe_threads_per_block() elements); returns
+    the number of operations the launch performs."""
+    ops = _i64(0)
+    n = int(lib().msc_probe_threads_per_block()) * blocks
+    if out.numel() < n:
+        raise ValueError(f"out holds {out.numel()} floats, the probe writes {n}")
+    if kind == "ex2":
+        st = lib().msc_probe_sfu_ex2(out.data_ptr(), blocks, iters, ctypes.byref(ops), _stream(stream))
+    else:
+        st = lib().msc_probe_ffma(out.data_ptr(), blocks, iters, 1 if kind == "ffma2" else 0,
+                                  ctypes.byref(ops), _stream(stream))
+    _check(st)
+    return int(ops.value)
 
 
 def msc_selective_scan_fwd_workspace_bytes(batch, dim, dstate, seqlen) -> int:

@@ -34,11 +34,18 @@ F16 = "f16"
 
 
 def round_to_bf16_bits(x: np.ndarray) -> np.ndarray:
-    """float32 -> bfloat16 bit patterns (uint16), round-to-nearest-even."""
+    """float32 -> bfloat16 bit patterns (uint16), round-to-nearest-even.
+
+    The sum below fits in 32 bits for every finite value and every infinity
+    (the largest pattern, 0xFF800000, plus 0x8000 stays below 2^32); only NaN
+    payloads near 0xFFFFFFFF would wrap, and the generators draw none."""
     f = np.ascontiguousarray(x, dtype=np.float32)
-    bits = f.view(np.uint32).astype(np.uint64)
-    bits = (bits + 0x7FFF + ((bits >> 16) & 1)) >> 16
-    return bits.astype(np.uint16)
+    bits = f.view(np.uint32)
+    r = (bits >> 16) & np.uint32(1)
+    r += np.uint32(0x7FFF)
+    r += bits
+    r >>= np.uint32(16)
+    return r.astype(np.uint16)
 
 
 def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:

@@ -212,6 +212,36 @@ def test_size_functions():
         msc.MSC_STATIC_SCRATCH_BYTES
 
 
+def test_bwd_workspace_query_refuses_bad_groups():
+    """ngroups < 1 or not a divisor of dim needs no workspace (the backward
+    refuses it); the query must not divide by it."""
+    assert msc.msc_selective_scan_bwd_workspace_bytes(2, 64, 16, 128, 0) == 0
+    assert msc.msc_selective_scan_bwd_workspace_bytes(2, 64, 16, 128, -2) == 0
+    assert msc.msc_selective_scan_bwd_workspace_bytes(2, 64, 16, 128, 3) == 0
+    assert msc.msc_selective_scan_bwd_workspace_bytes(2, 64, 300, 128, 1) == 0
+
+
+@pytest.mark.parametrize("field,value,status,word", [
+    ("ngroups", 0, INVALID, "ngroups"),
+    ("ngroups", -1, INVALID, "ngroups"),
+    ("ngroups", 3, INVALID, "ngroups"),
+    ("dstate", 0, UNSUPPORTED, "dstate"),
+    ("io_dtype", 9, INVALID, "io_dtype"),
+    ("delta_softplus", 2, INVALID, "delta_softplus"),
+])
+def test_static_backward_checks_arguments_before_sizing(field, value, status, word):
+    """The allocation-free backward validates its arguments the way the
+    workspace backward does, before the scratch size is computed (no host
+    division by ngroups = 0); nothing is launched, so no GPU is needed."""
+    a = msc.SsBwdArgs()
+    a.struct_size = ctypes.sizeof(msc.SsBwdArgs)
+    a.io_dtype, a.batch, a.dim, a.dstate, a.seqlen, a.ngroups = msc.MSC_BF16, 2, 64, 16, 128, 1
+    a.delta_softplus = 1
+    setattr(a, field, value)
+    st = msc.lib().msc_selective_scan_bwd_static(ctypes.byref(a), None)
+    assert st == status and word in _err()
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     """No silent fallback: without libmsc.so the binding raises."""
     monkeypatch.setattr(msc, "LIB_PATH", str(tmp_path / "missing" / "libmsc.so"))

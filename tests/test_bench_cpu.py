@@ -20,7 +20,7 @@ def test_m1_bytes_per_unit():
     params = D * N * 4 + 2 * D * 4
     assert bwd == 7 * io * tc + 2 * N * io * bt + 2 * N * 4 * bt + params + D * N * 4 + 2 * D * 4
     assert fwd == 4 * io * tc + 2 * N * io * bt + params + B * D * N * 4
-    assert bwd == 355688448  # the figure the bench line and DESIGN quote
+    assert bwd == 355688448  # the figure the bench line's roofline divides by
 
 
 def test_m3_bytes_per_unit():
@@ -45,14 +45,15 @@ def test_m3_decode_bytes():
 
 
 def test_traffic_gated_by_source_hash(monkeypatch):
-    assert bench.ncu_traffic("no_such_kernel.cu") is None
+    assert bench.ncu_traffic("no_such_kernel.cu", "w") is None
     monkeypatch.setitem(bench.NCU_TRAFFIC, "m1_fwd.cu", ("0000000000000000", "w", 123))
-    assert bench.ncu_traffic("m1_fwd.cu") is None  # stale capture: not reported
+    assert bench.ncu_traffic("m1_fwd.cu", "w") is None  # stale capture: not reported
     import hashlib
     path = os.path.join(ROOT, "selective_state_space_14_b200", "csrc", "m1_fwd.cu")
     h = hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
     monkeypatch.setitem(bench.NCU_TRAFFIC, "m1_fwd.cu", (h, "w", 123))
-    assert bench.ncu_traffic("m1_fwd.cu") == 123
+    assert bench.ncu_traffic("m1_fwd.cu", "w") == 123
+    assert bench.ncu_traffic("m1_fwd.cu", "another workload") is None  # other sizes: not reported
 
 
 def test_clock_sampler_without_gpu():
@@ -79,10 +80,10 @@ def test_conv_and_disc_bytes():
 def test_oracle_beside_fills_every_workload():
     """The oracle timings beside the extra workloads run on the host alone and
     fill an entry for every workload that ran (none for one that failed)."""
-    names = ["m1_bf16_b4_d5120_n16_l4096", "su_bf16_b256_d5120_n16_x1000",
-             "m3_bf16_b8_h24_p64_n64_k32_l2048", "m3su_bf16_b256_h24_p64_n64_k32_x1000",
-             "m3disc_bf16_b8_h24_p64_n64_k32_l2048", "m1conv_bf16_b8_d1536_n16_l2048_w4",
-             "m3su_raw_bf16_b256_h24_p64_n64_k32_x1000"]
+    names = ["m3su_raw_bf16_b256_h24_p64_n64_k32_x1000", "m1_bf16_b8_d1536_n16_l2048",
+             "su_bf16_b256_d5120_n16_x1000", "m3_bf16_b8_h24_p64_n64_k32_l2048",
+             "m3su_bf16_b256_h24_p64_n64_k32_x1000", "m3disc_bf16_b8_h24_p64_n64_k32_l2048",
+             "m1conv_bf16_b8_d1536_n16_l2048_w4"]
     res = {n: {"unit": "u"} for n in names}
     res[names[0]] = {"error": "x"}
     bench.oracle_beside(res, budget_s=0.0)

@@ -11,6 +11,9 @@ from tests._util import TOL, assert_close, dev, host, m1_device_args
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
 
+# f32 elementwise guards of the Mamba-1 recurrences (tests/_util.py)
+FAMILY = "m1"
+
 
 @pytest.fixture(scope="module")
 def msc():
@@ -56,15 +59,15 @@ def test_conv_fwd_bwd_parity(msc, case):
     f64 = lambda a: None if a is None else np.asarray(a, np.float64)
     u_ref, xs_ref = oracle.conv1d_fwd(x.as_f64(), f64(w), bias=f64(b), xs0=f64(xs0))
     r = oracle.conv1d_bwd(x.as_f64(), f64(w), du.as_f64(), bias=f64(b), xs0=f64(xs0))
-    assert_close("u", host(u), u_ref, TOL[io])
+    assert_close("u", host(u), u_ref, TOL[io], FAMILY)
     if Wd > 1:
-        assert_close("conv_state_out", host(xs), xs_ref, TOL["f32"])
-    assert_close("dx", host(g["dx"]), r["dx"], TOL[io])
-    assert_close("dw", host(g["dw"]), r["dw"], TOL[io])
+        assert_close("conv_state_out", host(xs), xs_ref, TOL["f32"], FAMILY)
+    assert_close("dx", host(g["dx"]), r["dx"], TOL[io], FAMILY)
+    assert_close("dw", host(g["dw"]), r["dw"], TOL[io], FAMILY)
     if bias:
-        assert_close("dbias", host(g["dbias"]), r["dbias"], TOL[io])
+        assert_close("dbias", host(g["dbias"]), r["dbias"], TOL[io], FAMILY)
     if Wd > 1:
-        assert_close("dconv_state_in", host(g["dconv_state_in"]), r["dxs0"], TOL[io])
+        assert_close("dconv_state_in", host(g["dconv_state_in"]), r["dxs0"], TOL[io], FAMILY)
 
 
 @pytest.mark.parametrize("io", ["f32", "bf16"])
@@ -90,10 +93,10 @@ def test_conv_feeding_the_scan(msc, io):
     refg = oracle.m1_bwd(dout=p.dout.as_f64(), **ra)
     du_stored = W.store(refg["du"].astype(np.float32), io).as_f64()
     rc = oracle.conv1d_bwd(x.as_f64(), f64(w), du_stored, bias=f64(b), xs0=f64(xs0))
-    assert_close("out", host(out), ref["out"], TOL[io])
-    assert_close("dx", host(gc["dx"]), rc["dx"], TOL[io])
-    assert_close("dw", host(gc["dw"]), rc["dw"], TOL[io])
-    assert_close("dbias", host(gc["dbias"]), rc["dbias"], TOL[io])
+    assert_close("out", host(out), ref["out"], TOL[io], FAMILY)
+    assert_close("dx", host(gc["dx"]), rc["dx"], TOL[io], FAMILY)
+    assert_close("dw", host(gc["dw"]), rc["dw"], TOL[io], FAMILY)
+    assert_close("dbias", host(gc["dbias"]), rc["dbias"], TOL[io], FAMILY)
 
 
 def test_conv_continuation(msc):
@@ -162,11 +165,11 @@ def test_fused_conv_scan_fwd_parity(msc, case):
     ra = oracle.m1_problem_args(p)
     ra["u"] = W.store(u_ref.astype(np.float32), io).as_f64()
     ref = oracle.m1_fwd(**ra)
-    assert_close("u", host(u), u_ref, TOL[io])
-    assert_close("out", host(out), ref["out"], TOL[io])
-    assert_close("final_state", host(fs), ref["final_state"], TOL[io])
+    assert_close("u", host(u), u_ref, TOL[io], FAMILY)
+    assert_close("out", host(out), ref["out"], TOL[io], FAMILY)
+    assert_close("final_state", host(fs), ref["final_state"], TOL[io], FAMILY)
     if Wd > 1:
-        assert_close("conv_state_out", host(xs), xs_ref, TOL["f32"])
+        assert_close("conv_state_out", host(xs), xs_ref, TOL["f32"], FAMILY)
 
 
 @pytest.mark.parametrize("case", [FUSED_CASES[1], FUSED_CASES[5], FUSED_CASES[6], FUSED_CASES[7]],
@@ -209,10 +212,10 @@ def test_fused_conv_scan_train_step(msc):
     refg = oracle.m1_bwd(dout=p.dout.as_f64(), **ra)
     du_stored = W.store(refg["du"].astype(np.float32), "bf16").as_f64()
     rc = oracle.conv1d_bwd(x.as_f64(), f64(w), du_stored, bias=f64(b), xs0=f64(xs0))
-    assert_close("dA", host(gs["dA"]), refg["dA"], TOL["bf16"])
-    assert_close("dx", host(gc["dx"]), rc["dx"], TOL["bf16"])
-    assert_close("dw", host(gc["dw"]), rc["dw"], TOL["bf16"])
-    assert_close("dconv_state_in", host(gc["dconv_state_in"]), rc["dxs0"], TOL["bf16"])
+    assert_close("dA", host(gs["dA"]), refg["dA"], TOL["bf16"], FAMILY)
+    assert_close("dx", host(gc["dx"]), rc["dx"], TOL["bf16"], FAMILY)
+    assert_close("dw", host(gc["dw"]), rc["dw"], TOL["bf16"], FAMILY)
+    assert_close("dconv_state_in", host(gc["dconv_state_in"]), rc["dxs0"], TOL["bf16"], FAMILY)
 
 
 def test_fused_continuation(msc):
@@ -258,13 +261,13 @@ def test_conv_workload_full_size(msc):
     ra = oracle.m1_problem_args(q.scan)
     ra["u"] = W.store(u_ref.astype(np.float32), "bf16").as_f64()
     ref = oracle.m1_fwd(**ra)
-    assert_close("u", host(u), u_ref, TOL["bf16"])
-    assert_close("out", host(out), ref["out"], TOL["bf16"])
-    assert_close("final_state", host(fs), ref["final_state"], TOL["bf16"])
-    assert_close("conv_state_out", host(xs), xs_ref, TOL["f32"])
+    assert_close("u", host(u), u_ref, TOL["bf16"], FAMILY)
+    assert_close("out", host(out), ref["out"], TOL["bf16"], FAMILY)
+    assert_close("final_state", host(fs), ref["final_state"], TOL["bf16"], FAMILY)
+    assert_close("conv_state_out", host(xs), xs_ref, TOL["f32"], FAMILY)
     rc = oracle.conv1d_bwd(q.scan.u.as_f64(), f64(q.w), q.scan.dout.as_f64(), bias=f64(q.bias))
     for k, rk in (("dx", "dx"), ("dw", "dw"), ("dbias", "dbias")):
-        assert_close(k, host(g[k]), rc[rk], TOL["bf16"])
+        assert_close(k, host(g[k]), rc[rk], TOL["bf16"], FAMILY)
 
 
 def test_conv_empty_sequences(msc):

@@ -10,6 +10,9 @@ from tests._util import TOL, assert_close, dev, host, m1_device_args
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
 
+# f32 elementwise guards of the Mamba-1 recurrences (tests/_util.py)
+FAMILY = "m1"
+
 M1_GRADS = ("du", "ddelta", "dA", "dB", "dC", "dD", "ddelta_bias", "dz", "dh0")
 
 
@@ -49,7 +52,7 @@ def _compare(gpu, ref, tol, skip=()):
     for k, v in gpu.items():
         if k in skip or k not in ref:
             continue
-        errs[k] = assert_close(k, v, ref[k], tol)
+        errs[k] = assert_close(k, v, ref[k], tol, FAMILY)
     return errs
 
 
@@ -115,11 +118,11 @@ def test_determinism(msc):
 def test_resume_is_bit_continuous(msc):
     """A scan over L equals a scan over L1 followed by one over L - L1 started
     from the first one's final state; bit-equal when L1 is a multiple of the
-    forward's 128-step chunk."""
+    forward's 32-step chunk (and so of the 8-step saved-state interval)."""
     p = W.m1_problem(1, 12, 16, 1536, io="f32", seed=9, bias=True)
     a = m1_device_args(p)
     full, fs_full, _ = msc.msc_selective_scan_fwd(**a)
-    L1 = 1024  # a multiple of the 128-step chunk
+    L1 = 1024  # a multiple of the 32-step chunk
     part = {k: (v[..., :L1].contiguous() if k in ("u", "delta", "z") else v) for k, v in a.items()}
     part["B"], part["C"] = a["B"][..., :L1].contiguous(), a["C"][..., :L1].contiguous()
     o1, fs1, _ = msc.msc_selective_scan_fwd(**part)
@@ -167,7 +170,7 @@ def test_2p8b_shaped_full_size_sampled(msc):
                      W.Tensor(p.io, p.dout.data[:1]))
     ref = _run_oracle(p0)
     for k in ("out", "final_state", "du", "ddelta", "dz", "dh0", "dB", "dC"):
-        assert_close(k, g[k][:1], ref[k], TOL["bf16"])
+        assert_close(k, g[k][:1], ref[k], TOL["bf16"], FAMILY)
 
 
 # ---------------------------------------------------------------------------
@@ -203,8 +206,8 @@ def test_state_update_chain(msc, io):
                                                 s["C"].as_f64(), D=q.D.astype(np.float64),
                                                 delta_bias=q.delta_bias.astype(np.float64),
                                                 z=s["z"].as_f64())
-        assert_close("out", host(o), o_ref, TOL[io])
-    assert_close("state", host(st), st_ref, TOL[io])
+        assert_close("out", host(o), o_ref, TOL[io], FAMILY)
+    assert_close("state", host(st), st_ref, TOL[io], FAMILY)
 
 
 def test_state_update_wide_state(msc):
@@ -221,8 +224,8 @@ def test_state_update_wide_state(msc):
                                                 s["C"].as_f64(), D=q.D.astype(np.float64),
                                                 delta_bias=q.delta_bias.astype(np.float64),
                                                 z=s["z"].as_f64())
-        assert_close("out", host(o), o_ref, TOL["bf16"])
-    assert_close("state", host(st), st_ref, TOL["bf16"])
+        assert_close("out", host(o), o_ref, TOL["bf16"], FAMILY)
+    assert_close("state", host(st), st_ref, TOL["bf16"], FAMILY)
 
 
 def test_state_update_decode_workload_sampled(msc):
@@ -266,5 +269,5 @@ def test_state_update_decode_workload_sampled(msc):
             ref_out[r] = o[0, 0]
         for (tt, got) in outs:
             if tt == t:
-                assert_close(f"out@{t}", got, ref_out, TOL["bf16"])
-    assert_close("state", final, st_ref[:, 0, :], TOL["bf16"])
+                assert_close(f"out@{t}", got, ref_out, TOL["bf16"], FAMILY)
+    assert_close("state", final, st_ref[:, 0, :], TOL["bf16"], FAMILY)

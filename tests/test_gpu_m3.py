@@ -10,6 +10,9 @@ from tests._util import TOL, assert_close, dev, host, m3_device_args
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
 
+# f32 elementwise guards of the Mamba-3 recurrences (tests/_util.py)
+FAMILY = "m3"
+
 M3_GRADS = ("dx", "dz", "dB", "dC", "dalpha", "dbeta", "dgamma", "dtheta", "dD", "dh0")
 
 
@@ -69,8 +72,8 @@ def test_fwd_parity_shapes(msc, case):
                      with_D=Dp, with_h0=h0)
     g, _, _ = _gpu_fwd(msc, p)
     r = _oracle_fwd(p)
-    assert_close("out", g["out"], r["out"], TOL[io])
-    assert_close("final_state", g["final_state"], r["final_state"], TOL[io])
+    assert_close("out", g["out"], r["out"], TOL[io], FAMILY)
+    assert_close("final_state", g["final_state"], r["final_state"], TOL[io], FAMILY)
 
 
 @pytest.mark.parametrize("case", [c for c in FWD_CASES if c[7] == "bf16"],
@@ -88,8 +91,8 @@ def test_fwd_without_saved_states(msc, case):
     torch.cuda.synchronize()
     assert sv is None
     r = _oracle_fwd(p)
-    assert_close("out", host(out1), r["out"], TOL[io])
-    assert_close("final_state", host(fs1), r["final_state"], TOL[io])
+    assert_close("out", host(out1), r["out"], TOL[io], FAMILY)
+    assert_close("final_state", host(fs1), r["final_state"], TOL[io], FAMILY)
     assert torch.equal(out1, out2) and torch.equal(fs1, fs2)
 
 
@@ -123,8 +126,8 @@ def test_fwd_model_shaped_full_size(msc):
     p = W.make("m3_bf16_b8_h24_p64_n64_k32_l2048")
     g, _, _ = _gpu_fwd(msc, p)
     r = _oracle_fwd(p)
-    assert_close("out", g["out"], r["out"], TOL["bf16"])
-    assert_close("final_state", g["final_state"], r["final_state"], TOL["bf16"])
+    assert_close("out", g["out"], r["out"], TOL["bf16"], FAMILY)
+    assert_close("final_state", g["final_state"], r["final_state"], TOL["bf16"], FAMILY)
 
 
 # ---------------------------------------------------------------------------
@@ -177,7 +180,7 @@ def test_bwd_parity_shapes(msc, case):
             continue
         if k == "dD" and not Dp:
             continue
-        assert_close(k, g[k], r[k], TOL[io])
+        assert_close(k, g[k], r[k], TOL[io], FAMILY)
 
 
 def test_bwd_determinism(msc):
@@ -200,7 +203,7 @@ def test_bwd_model_shaped_full_size(msc):
                      T(p.theta), p.D, None, T(p.dout))
     r = _oracle_bwd(p0)
     for k in ("dx", "dz", "dB", "dC", "dalpha", "dbeta", "dgamma", "dtheta", "dh0"):
-        assert_close(k, g[k][:1], r[k], TOL["bf16"])
+        assert_close(k, g[k][:1], r[k], TOL["bf16"], FAMILY)
 
 
 # ---------------------------------------------------------------------------
@@ -250,9 +253,9 @@ def test_m3_state_update_chain(msc, case):
                                              f(s["theta"]),
                                              D=None if q.D is None else q.D.astype(np.float64),
                                              z=f(s["z"]))
-        assert_close("out", host(o), o_ref, TOL[io])
+        assert_close("out", host(o), o_ref, TOL[io], FAMILY)
     for name, g, r in zip(("state", "x_prev", "bt_prev", "phi"), (S, xp, bp, ph), ref):
-        assert_close(name, host(g), r, TOL[io])
+        assert_close(name, host(g), r, TOL[io], FAMILY)
 
 
 @pytest.mark.parametrize("io", ["f32", "bf16"])
@@ -275,8 +278,8 @@ def test_m3_state_update_chain_equals_scan(msc, io):
             S, xp, bp, ph, c("x"), c("B"), c("C"), c("alpha"), c("beta"), c("gamma"), c("theta"),
             D=a["D"], z=c("z")))
     torch.cuda.synchronize()
-    assert_close("out", host(torch.stack(outs, dim=1)), host(out), TOL[io])
-    assert_close("final_state", host(S), host(fs), TOL[io])
+    assert_close("out", host(torch.stack(outs, dim=1)), host(out), TOL[io], FAMILY)
+    assert_close("final_state", host(S), host(fs), TOL[io], FAMILY)
 
 
 def test_m3_state_update_deterministic(msc):
@@ -339,7 +342,7 @@ def test_m3_state_update_workload_sampled(msc):
             o_ref[r:r + 1] = res[4]
         ref = new
         if k < len(outs) and outs[k][0] == t:
-            assert_close(f"out@{t}", outs[k][1], o_ref[:, 0], TOL["bf16"])
+            assert_close(f"out@{t}", outs[k][1], o_ref[:, 0], TOL["bf16"], FAMILY)
             k += 1
-    assert_close("state", host(S)[bi, hi], ref[0][:, 0], TOL["bf16"])
-    assert_close("phi", host(ph)[bi, hi], ref[3][:, 0], TOL["bf16"])
+    assert_close("state", host(S)[bi, hi], ref[0][:, 0], TOL["bf16"], FAMILY)
+    assert_close("phi", host(ph)[bi, hi], ref[3][:, 0], TOL["bf16"], FAMILY)
