@@ -106,6 +106,15 @@ constexpr int kM3Slab = 64;  // widest d_state one launch handles
 cudaError_t launch_m3_fwd(const M3Params &p, cudaStream_t s);
 cudaError_t launch_m3_fwd_umma(const M3Params &p, cudaStream_t s);  // bf16 io, tcgen05
 cudaError_t launch_m3_bwd(const M3Params &p, cudaStream_t s);
+cudaError_t launch_m3_bwd_umma(const M3Params &p, cudaStream_t s);  // bf16 io, tcgen05
+// Workspace of the Mamba-3 backward, byte offsets of its regions: per-head dB,
+// dC [B, L, H, N]; per-(b, h, chunk) dD [B, H, nc]; the chunk adjoints V / U
+// [B, H, nc, P, N] and their decays rho [B, H, nc]; the dtheta chunk totals
+// [B, H, nc, K]; above one slab the token sums of y and dx [B, L, H, P].
+struct M3BwdWs {
+  size_t dB, dC, dD, vu, rho, th, tok_y, tok_dx, total;
+};
+M3BwdWs m3_bwd_ws_layout(int64_t B, int64_t L, int64_t H, int64_t P, int64_t N, int64_t K);
 size_t m3_bwd_workspace_bytes(int64_t B, int64_t L, int64_t H, int64_t P, int64_t N, int64_t G,
                               int64_t K);
 bool m3_supported(int64_t P, int64_t N);

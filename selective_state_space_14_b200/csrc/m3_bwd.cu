@@ -1,6 +1,8 @@
-// m3_bwd.cu -- Mamba-3 SISO scan, backward (sm_100a): backward stages B2
-// (output gating), B3 (BPTT through the trapezoidal state) and B4 (RoPE) of
-// Mamba3Scratch in mamba-rs 0.4.2 src/mamba3_siso/cpu/scratch.rs.
+// m3_bwd.cu -- Mamba-3 SISO scan, backward for f32 and f16 io (sm_100a, CUDA
+// cores): backward stages B2 (output gating), B3 (BPTT through the
+// trapezoidal state) and B4 (RoPE) of Mamba3Scratch in mamba-rs 0.4.2
+// src/mamba3_siso/cpu/scratch.rs.  bf16 io runs the chunk-parallel
+// tensor-core backward of m3_bwd_umma.cu, which uses the same chunk algebra.
 //
 // Chunk-local notation as in m3_common.cuh (t, s, tau in [0, Q); g_t the
 // gradient of y_t, i.e. dout_t silu(z_t)).  The state adjoint
@@ -31,28 +33,14 @@
 // and a second kernel adds the heads of each group in ascending order.
 // One CTA per (b, h) walks the chunks from last to first; the chunk-start
 // states come from the forward's saved states, the chunk-start angles from a
-// sequential sum per angle identical to the forward's.
-#include <type_traits>
-
-#include "m3_tc.cuh"
+// sequential sum per angle identical to the forward's.  The contractions are
+// f32 on the CUDA cores (mm in m3_common.cuh).
+#include "m3_common.cuh"
 
 namespace msc {
 namespace {
 
 using namespace m3;
-
-// Chunk contractions: tensor cores (split tf32, f32-class products) for bf16
-// io, f32 on the CUDA cores for f32 io.
-template <typename T, int M, int N, int K, bool kAT, bool kBT, bool kSplitA = true,
-          bool kSplitB = true>
-__device__ __forceinline__ void mmx(float *C, int ldc, const float *A, int lda, const float *B,
-                                    int ldb, const float *rowscale, const float *kscale,
-                                    bool accumulate) {
-  if constexpr (std::is_same_v<T, bf16>)
-    mmt<M, N, K, kAT, kBT, kSplitA, kSplitB>(C, ldc, A, lda, B, ldb, rowscale, kscale, accumulate);
-  else
-    mm<M, N, K, kAT, kBT>(C, ldc, A, lda, B, ldb, rowscale, kscale, accumulate);
-}
 
 // 8 consecutive io elements from global memory at index j (16-byte aligned
 // for bf16), or zeros when !valid
@@ -293,7 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
     }
     __syncthreads();
     // ---- C. Ct Bt^T, per-step vectors, W ---------------------------------------
-    mmx<T, kQ, kQ, N, false, true>(sCB, lQ, sCt, lN, sBt, lN, nullptr, nullptr, false);
+    mm<kQ, kQ, N, false, true>(sCB, lQ, sCt, lN, sBt, lN, nullptr, nullptr, false);
     for (int t = tid; t < kQ; t += kThreads) {
       sD1[t] = sDm[t * (kQ + 1)];
       sD0[t] = sDm[t * (kQ + 1) + 1];
@@ -317,8 +305,8 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
     }
     __syncthreads();
     // ---- D. y (for dz) -----------------------------------------------------------
-    mmx<T, kQ, P, kQ, false, false, true, false>(sT1, lMx, sW, lQ, sX, lP, nullptr, nullptr, false);
-    mmx<T, kQ, P, N, false, true>(sT1, lMx, sCt, lN, sSin, lN, sD1, nullptr, true);
+    mm<kQ, P, kQ, false, false>(sT1, lMx, sW, lQ, sX, lP, nullptr, nullptr, false);
+    mm<kQ, P, N, false, true>(sT1, lMx, sCt, lN, sSin, lN, sD1, nullptr, true);
     __syncthreads();
     if (p.dz) {
       for (int i = tid; i < kQ * P; i += kThreads) {
@@ -340,8 +328,8 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
       }
     }
     // ---- E. G X^T, G S_in; first scalar pass -----------------------------------
-    mmx<T, kQ, kQ, P, false, true, true, false>(sT2, lMx, sG, lP, sX, lP, nullptr, nullptr, false);
-    mmx<T, kQ, N, P, false, false>(sT3, lMx, sG, lP, sSin, lN, nullptr, nullptr, false);
+    mm<kQ, kQ, P, false, true>(sT2, lMx, sG, lP, sX, lP, nullptr, nullptr, false);
+    mm<kQ, N, P, false, false>(sT3, lMx, sG, lP, sSin, lN, nullptr, nullptr, false);
     __syncthreads();
     for (int s = tid; s < kQ; s += kThreads) {
       // column s of E, dgamma_s and dbeta_s (chunk-internal parts)
@@ -387,9 +375,9 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
     }
     __syncthreads();
     // ---- F. dx; X U; dBt; second scalar pass --------------------------------------
-    mmx<T, kQ, P, kQ, true, false>(sT1, lMx, sW, lQ, sG, lP, nullptr, nullptr, false);
-    mmx<T, kQ, P, N, false, true>(sT1, lMx, sBt, lN, sU, lN, sWu, nullptr, true);
-    mmx<T, kQ, N, P, false, false, false, true>(sT2, lMx, sX, lP, sU, lN, nullptr, nullptr, false);
+    mm<kQ, P, kQ, true, false>(sT1, lMx, sW, lQ, sG, lP, nullptr, nullptr, false);
+    mm<kQ, P, N, false, true>(sT1, lMx, sBt, lN, sU, lN, sWu, nullptr, true);
+    mm<kQ, N, P, false, false>(sT2, lMx, sX, lP, sU, lN, nullptr, nullptr, false);
     __syncthreads();
     for (int i = tid; i < kQ * P; i += kThreads) {
       const int t = i / P, pp = i % P;
@@ -406,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
         static_cast<T *>(p.dx)[j] = from_f32<T>(v);
       }
     }
-    mmx<T, kQ, N, kQ, true, false>(sW, lN, sCB, lQ, sCt, lN, nullptr, nullptr, false);
+    mm<kQ, N, kQ, true, false>(sW, lN, sCB, lQ, sCt, lN, nullptr, nullptr, false);
     // v_s = x_s^T U Bt_s (s >= 0), v_{-1} with the previous step; <U, S_in>
     for (int s = tid; s < kQ; s += kThreads) {
       float v = 0.f;
@@ -466,7 +454,7 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
     }
     __syncthreads();
     // ---- G. dCt ---------------------------------------------------------------------
-    mmx<T, kQ, N, kQ, false, false>(sT1, lMx, sCB, lQ, sBt, lN, nullptr, nullptr, false);
+    mm<kQ, N, kQ, false, false>(sT1, lMx, sCB, lQ, sBt, lN, nullptr, nullptr, false);
     __syncthreads();
     for (int i = tid; i < kQ * N; i += kThreads) {
       const int t = i / N, n = i % N;
@@ -495,7 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1) m3_bwd_kernel(const M3Params p, f
     }
     __syncthreads();
     // ---- H. U_prev = G^T diag(d(.,0)) Ct + d(Q-1,0) alpha_Q U --------------------------
-    mmx<T, P, N, kQ, true, false>(sT3, lMx, sG, lP, sCt, lN, nullptr, sD0, false);
+    mm<P, N, kQ, true, false>(sT3, lMx, sG, lP, sCt, lN, nullptr, sD0, false);
     // ---- J. RoPE backward: per-head dB, dC and dphi -----------------------------------
     for (int i = tid; i < kQ * (N / 2); i += kThreads) {
       const int t = i / (N / 2), k = i % (N / 2);
@@ -584,32 +572,13 @@ __global__ void m3_bwd_reduce_kernel(const M3Params p, const float *ws_dB, const
   }
 }
 
-// per-head dB, dC [B, L, H, N]; per-(b, h) dD [B, H]; above one slab the
-// sums over the states of y and dx [B, L, H, P]
-struct WsLayout {
-  size_t dB, dC, dD, tok_y, tok_dx, total;
-};
-
-WsLayout ws_layout(int64_t B, int64_t L, int64_t H, int64_t P, int64_t N) {
-  auto up = [](size_t v) { return (v + 255) / 256 * 256; };
-  WsLayout w;
-  w.dB = 0;
-  w.dC = w.dB + up(sizeof(float) * (size_t)(B * L * H * N));
-  w.dD = w.dC + up(sizeof(float) * (size_t)(B * L * H * N));
-  w.tok_y = w.dD + up(sizeof(float) * (size_t)(B * H));
-  const size_t tok = N > kM3Slab ? up(sizeof(float) * (size_t)(B * L * H * P)) : 0;
-  w.tok_dx = w.tok_y + tok;
-  w.total = w.tok_dx + tok;
-  return w;
-}
-
 template <typename T, int P, int N, bool kSlab>
 cudaError_t launch_t(const M3Params &p, cudaStream_t s) {
   const size_t smem = sizeof(float) * (size_t)BwdSmem<P, N>::total;
   cudaError_t e = cudaFuncSetAttribute(m3_bwd_kernel<T, P, N, kSlab>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const WsLayout w = ws_layout(p.B, p.L, p.H, p.P, p.ldN);
+  const M3BwdWs w = m3_bwd_ws_layout(p.B, p.L, p.H, p.P, p.ldN, p.K);
   char *ws = static_cast<char *>(p.ws);
   float *dB = reinterpret_cast<float *>(ws + w.dB);
   float *dC = reinterpret_cast<float *>(ws + w.dC);
@@ -640,11 +609,12 @@ cudaError_t launch_p(const M3Params &p, cudaStream_t s) {
 
 }  // namespace
 
+// one layout serves both implementations (its regions are a superset of what
+// this one uses), so the size does not depend on the io type
 size_t m3_bwd_workspace_bytes(int64_t B, int64_t L, int64_t H, int64_t P, int64_t N, int64_t G,
                               int64_t K) {
   (void)G;
-  (void)K;
-  return ws_layout(B, L, H, P, N).total;
+  return m3_bwd_ws_layout(B, L, H, P, N, K).total;
 }
 
 // The whole d_state in one launch, or slabs of kM3Slab states in ascending
@@ -652,9 +622,10 @@ size_t m3_bwd_workspace_bytes(int64_t B, int64_t L, int64_t H, int64_t P, int64_
 // dgamma), then the fixed-order sum of dB, dC over the heads of a group and
 // of dD over the batch.
 cudaError_t launch_m3_bwd(const M3Params &p0, cudaStream_t s) {
+  if (p0.io == 1) return launch_m3_bwd_umma(p0, s);  // bf16 io: the tensor-core backward
   const int64_t n_tot = p0.N;
   const int64_t slabs = (n_tot + kM3Slab - 1) / kM3Slab;
-  const WsLayout w = ws_layout(p0.B, p0.L, p0.H, p0.P, n_tot);
+  const M3BwdWs w = m3_bwd_ws_layout(p0.B, p0.L, p0.H, p0.P, n_tot, p0.K);
   char *ws = static_cast<char *>(p0.ws);
   for (int64_t k = 0; k < slabs; ++k) {
     M3Params p = p0;
@@ -667,7 +638,6 @@ cudaError_t launch_m3_bwd(const M3Params &p0, cudaStream_t s) {
     p.tok_dx = slabs > 1 ? reinterpret_cast<float *>(ws + w.tok_dx) : nullptr;
     cudaError_t e;
     switch (p.io) {
-      case 1: e = launch_p<bf16>(p, s); break;
       case 2: e = launch_p<f16>(p, s); break;
       default: e = launch_p<float>(p, s); break;
     }

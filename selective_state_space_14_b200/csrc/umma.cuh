@@ -53,13 +53,14 @@ __device__ __forceinline__ uint64_t desc(uint32_t saddr, uint32_t lbo, uint32_t 
   return d;              // base offset 0, no swizzle
 }
 
-// instruction descriptor: bf16 x bf16 -> f32, M = 64, N columns; A K-major,
-// B K-major (kBMN = false) or MN-major (kBMN = true)
-template <int N, bool kBMN>
+// instruction descriptor: bf16 x bf16 -> f32, M = 64, N columns; A K-major
+// (kAMN = false) or MN-major (bit 15), B K-major (kBMN = false) or MN-major
+// (bit 16)
+template <int N, bool kBMN, bool kAMN = false>
 __device__ __forceinline__ uint32_t idesc_bf16() {
   static_assert(N % 16 == 0 && N >= 16 && N <= 256, "N");
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((kBMN ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) |
-         ((64u >> 4) << 24);
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((kAMN ? 1u : 0u) << 15) | ((kBMN ? 1u : 0u) << 16) |
+         ((uint32_t)(N >> 3) << 17) | ((64u >> 4) << 24);
 }
 
 __device__ __forceinline__ void mma(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc,
