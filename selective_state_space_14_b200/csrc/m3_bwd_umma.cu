@@ -224,11 +224,14 @@ struct Chunk {
   int Kt, k0, K;   // angle pairs: total, this slab's first, this slab's count
 };
 
-__device__ __forceinline__ Chunk chunk_of(const M3Params &p, int P) {
+// unit u of the persistent loop: chunk u % nc of head (u / nc) % H of batch
+// row u / (nc H)
+__device__ __forceinline__ Chunk chunk_of(const M3Params &p, int P, int64_t u) {
   Chunk c;
-  c.ch = blockIdx.x;
-  c.h = blockIdx.y;
-  c.b = blockIdx.z;
+  const int64_t nc = (p.L + kQ - 1) / kQ;
+  c.ch = u % nc;
+  c.h = (u / nc) % p.H;
+  c.b = u / (nc * p.H);
   c.g = c.h / (p.H / p.G);
   c.t0 = c.ch * kQ;
   c.nc = (p.L + kQ - 1) / kQ;
@@ -604,20 +607,32 @@ __global__ void __launch_bounds__(kThreads, 1) m3b_prep_kernel(const M3Params p,
   uint64_t *sMbar = reinterpret_cast<uint64_t *>(sm + S::misc + 8);
   int *sErr = reinterpret_cast<int *>(sm + S::misc + 16);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const Chunk c = chunk_of(p, P);
   const int slab = p.slab;
   const bool finish = slab == kSlabWhole || slab == kSlabLast;
-  const float Dh = (p.Dp && finish) ? p.Dp[c.h] : 0.f;
   const uint32_t base = umma::smem_addr(sm);
   const uint32_t mbar = umma::smem_addr(sMbar);
+  const int64_t n_units = ((p.L + kQ - 1) / kQ) * p.H * p.B;
 
   if (warp == 0) umma::tmem_alloc(sTmem, 256);
   if (tid == 0) {
     umma::mbar_init(mbar);
     *sErr = 0;
   }
+  auto sin_of = [&](const Chunk &c) {
+    return p.saved_in + ((c.b * p.H + c.h) * c.nc + c.ch) * P * c.ldN + c.n0;
+  };
   Loads<P, N, false> ld;
-  ld.issue(p, c, p.saved_in + ((c.b * p.H + c.h) * c.nc + c.ch) * P * c.ldN + c.n0, nullptr);
+  if ((int64_t)blockIdx.x < n_units) {
+    const Chunk c0 = chunk_of(p, P, blockIdx.x);
+    ld.issue(p, c0, sin_of(c0), nullptr);
+  }
+  umma::fence_before();
+  __syncthreads();
+  umma::fence_after();
+  const uint32_t tmem = *sTmem;
+  for (int64_t unit = blockIdx.x; unit < n_units; unit += gridDim.x) {
+  const Chunk c = chunk_of(p, P, unit);
+  const float Dh = (p.Dp && finish) ? p.Dp[c.h] : 0.f;
   stage_small(ld, sv, tPhi, P, N);
   __syncthreads();
   stage_decays(c, sv, tPhi, tD);
@@ -628,11 +643,14 @@ __global__ void __launch_bounds__(kThreads, 1) m3b_prep_kernel(const M3Params p,
     float us = 0.f, vm1 = 0.f;
     stage_state<P, N, false>(ld, sm + S::pS, nullptr, sv, us, vm1);
   }
+  if (unit + gridDim.x < n_units) {  // the next unit's loads fly while this one computes
+    const Chunk cn = chunk_of(p, P, unit + gridDim.x);
+    ld.issue(p, cn, sin_of(cn), nullptr);
+  }
   umma::fence_async_smem();
   umma::fence_before();
   __syncthreads();
   umma::fence_after();
-  const uint32_t tmem = *sTmem;
   if (tid == 0) {
     product<64, false>(tmem, 0, base + S::pC, kParts, N, base + S::pB, kParts, N, N, false);  // Ct Bt^T
     product<P, false>(tmem, 64, base + S::pC, kParts, N, base + S::pS, kParts, N, N, false);  // Ct S_in^T
@@ -729,6 +747,11 @@ __global__ void __launch_bounds__(kThreads, 1) m3b_prep_kernel(const M3Params p,
     }
   }
   umma::fence_before();
+  __syncthreads();  // this unit's TMEM reads and shared-memory uses are done
+  umma::fence_after();
+  if (*sErr) break;  // a tensor-core round never completed: stop (outputs are NaN)
+  }
+  umma::fence_before();
   __syncthreads();
   if (warp == 0) {
     umma::fence_after();
@@ -797,21 +820,30 @@ __global__ void __launch_bounds__(kThreads, 1) m3b_grad_kernel(const M3Params p,
   uint64_t *sMbar = reinterpret_cast<uint64_t *>(sm + S::misc + 8);
   int *sErr = reinterpret_cast<int *>(sm + S::misc + 16);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const Chunk c = chunk_of(p, P);
   const int slab = p.slab;
   const bool finish = slab == kSlabWhole || slab == kSlabLast;
-  const float Dh = (p.Dp && finish) ? p.Dp[c.h] : 0.f;
   const uint32_t base = umma::smem_addr(sm);
   const uint32_t mbar = umma::smem_addr(sMbar);
+  const int64_t n_units = ((p.L + kQ - 1) / kQ) * p.H * p.B;
 
   if (warp == 0) umma::tmem_alloc(sTmem, 512);
   if (tid == 0) {
     umma::mbar_init(mbar);
     *sErr = 0;
   }
+  auto off_of = [&](const Chunk &c) { return ((c.b * p.H + c.h) * c.nc + c.ch) * P * c.ldN + c.n0; };
   Loads<P, N, true> ld;
-  ld.issue(p, c, p.saved_in + ((c.b * p.H + c.h) * c.nc + c.ch) * P * c.ldN + c.n0,
-           vu + ((c.b * p.H + c.h) * c.nc + c.ch) * P * c.ldN + c.n0);
+  if ((int64_t)blockIdx.x < n_units) {
+    const Chunk c0 = chunk_of(p, P, blockIdx.x);
+    ld.issue(p, c0, p.saved_in + off_of(c0), vu + off_of(c0));
+  }
+  umma::fence_before();
+  __syncthreads();
+  umma::fence_after();
+  const uint32_t tmem = *sTmem;
+  for (int64_t unit = blockIdx.x; unit < n_units; unit += gridDim.x) {
+  const Chunk c = chunk_of(p, P, unit);
+  const float Dh = (p.Dp && finish) ? p.Dp[c.h] : 0.f;
   stage_small(ld, sv, tPhi, P, N);
   __syncthreads();
   stage_decays(c, sv, tPhi, tD);
@@ -820,11 +852,14 @@ __global__ void __launch_bounds__(kThreads, 1) m3b_grad_kernel(const M3Params p,
   const float gx_l = stage_xg<P>(ld, p.z != nullptr, sv, sm + S::pX, sm + S::pG, nullptr);
   float us_l = 0.f, vm1_l = 0.f;
   stage_state<P, N, true>(ld, sm + S::pS, sm + S::pU, sv, us_l, vm1_l);
+  if (unit + gridDim.x < n_units) {  // the next unit's loads fly while this one computes
+    const Chunk cn = chunk_of(p, P, unit + gridDim.x);
+    ld.issue(p, cn, p.saved_in + off_of(cn), vu + off_of(cn));
+  }
   umma::fence_async_smem();
   umma::fence_before();
   __syncthreads();
   umma::fence_after();
-  const uint32_t tmem = *sTmem;
   if (tid == 0) {
     product<64, false>(tmem, 0, base + S::pC, kParts, N, base + S::pB, kParts, N, N, false);   // Ct Bt^T
     product<64, false>(tmem, 64, base + S::pG, kParts, P, base + S::pX, 1, P, P, false);       // G X^T
@@ -912,13 +947,11 @@ __global__ void __launch_bounds__(kThreads, 1) m3b_grad_kernel(const M3Params p,
   const float alQ = sv[Vec::al + kQ];
   {
     const int s = tid >> 2, part = tid & 3;
-    float dg = 0.f, db = 0.f, bx = 0.f;
+    float dg = 0.f, db = 0.f;
     for (int tau = s + part; tau < kQ; tau += 4) {
       const float dts = tD[tau * 65 + s + 1];
       dg = fmaf(dts, tM[tau * 65 + s], dg);
       if (s > 0) db = fmaf(dts, tM[tau * 65 + s - 1], db);
-      for (int j = 0; j <= s - 2; ++j)
-        bx = fmaf(tD[tau * 65 + j + 2] * sv[Vec::eps + j], tM[tau * 65 + j], bx);
     }
     if (s == 0) {
       for (int tau = part; tau < kQ; tau += 4)
@@ -928,14 +961,36 @@ __global__ void __launch_bounds__(kThreads, 1) m3b_grad_kernel(const M3Params p,
     for (int o = 1; o < 4; o <<= 1) {
       dg += __shfl_xor_sync(0xffffffffu, dg, o);
       db += __shfl_xor_sync(0xffffffffu, db, o);
-      bx += __shfl_xor_sync(0xffffffffu, bx, o);
     }
     if (part == 0) {
       const float dq = alQ * tD[(kQ - 1) * 65 + s + 1];  // the U row
       sv[Vec::dg + s] = fmaf(dq, sv[Vec::v + s], dg);
       sv[Vec::db + s] = fmaf(dq, s == 0 ? vm1 : sv[Vec::v + s - 1], db);
-      sv[Vec::bx + s] = bx;
     }
+  }
+  __syncthreads();
+  // the box sums BX_s = sum_{tau>=s} sum_{j<=s-2} c(tau,j) M(tau,j): each row's
+  // prefix over j, written over M (a row keeps the two M values it still needs
+  // in registers), then the column sums over tau >= s
+  if (tid < kQ) {
+    const int tau = tid;
+    float run = 0.f, m2 = 0.f, m1 = 0.f;  // M(tau, s-2), M(tau, s-1)
+    for (int s2 = 0; s2 <= tau; ++s2) {
+      const float m0 = tM[tau * 65 + s2];
+      if (s2 >= 2) run = fmaf(tD[tau * 65 + s2] * sv[Vec::eps + s2 - 2], m2, run);  // c(tau, s2-2)
+      tM[tau * 65 + s2] = run;
+      m2 = m1;
+      m1 = m0;
+    }
+  }
+  __syncthreads();
+  {
+    const int s = tid >> 2, part = tid & 3;
+    float bx = 0.f;
+    for (int tau = s + part; tau < kQ; tau += 4) bx += tM[tau * 65 + s];
+    bx += __shfl_xor_sync(0xffffffffu, bx, 1);
+    bx += __shfl_xor_sync(0xffffffffu, bx, 2);
+    if (part == 0) sv[Vec::bx + s] = bx;
   }
   __syncthreads();
   {
@@ -1048,14 +1103,26 @@ __global__ void __launch_bounds__(kThreads, 1) m3b_grad_kernel(const M3Params p,
   __syncthreads();
   // ---- dtheta within the chunk (reverse sum), the chunk's total; dalpha, dbeta,
   // dgamma; dD -----------------------------------------------------------------------
-  if (tid < c.K) {
-    const int k = tid;
-    float acc = 0.f;
-    for (int t = c.Qc - 1; t >= 0; --t) {
-      acc += tPhi[t * 32 + k];
-      p.dtheta[((c.b * p.L + c.t0 + t) * p.H + c.h) * c.Kt + c.k0 + k] = failed ? qnan : acc;
+  if (warp < 2) {
+    // reverse sums over the chunk per angle pair: warp w takes pairs w, w + 2,
+    // ...; lane l holds steps 2l, 2l + 1 (steps past Qc carry zero)
+    const int t0 = 2 * lane, t1 = t0 + 1;
+    for (int k = warp; k < c.K; k += 2) {
+      const float a0 = tPhi[t0 * 32 + k], a1 = tPhi[t1 * 32 + k];
+      float incl = a0 + a1;  // suffix sums: lanes >= l
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float u = __shfl_down_sync(0xffffffffu, incl, o);
+        if (lane + o < 32) incl += u;
+      }
+      float excl = __shfl_down_sync(0xffffffffu, incl, 1);
+      if (lane == 31) excl = 0.f;
+      const float v1 = excl + a1, v0 = v1 + a0;
+      const int64_t j = ((c.b * p.L + c.t0 + t0) * p.H + c.h) * c.Kt + c.k0 + k;
+      if (t0 < c.Qc) p.dtheta[j] = failed ? qnan : v0;
+      if (t1 < c.Qc) p.dtheta[j + p.H * c.Kt] = failed ? qnan : v1;
+      if (lane == 0) ws_th[((c.b * p.H + c.h) * c.nc + c.ch) * c.Kt + c.k0 + k] = v0;
     }
-    ws_th[((c.b * p.H + c.h) * c.nc + c.ch) * c.Kt + c.k0 + k] = acc;
   } else if (tid >= 64 && tid < 64 + kQ) {
     const int s = tid - 64;
     if (s < c.Qc) {
@@ -1069,6 +1136,11 @@ __global__ void __launch_bounds__(kThreads, 1) m3b_grad_kernel(const M3Params p,
     }
   } else if (tid == 128 && finish) {
     ws_dD[(c.b * p.H + c.h) * c.nc + c.ch] = dD;
+  }
+  umma::fence_before();
+  __syncthreads();  // this unit's TMEM reads and shared-memory uses are done
+  umma::fence_after();
+  if (*sErr) break;  // a tensor-core round never completed: stop (outputs are NaN)
   }
   umma::fence_before();
   __syncthreads();
@@ -1134,8 +1206,12 @@ __global__ void m3b_finish_kernel(const M3Params p, const float *ws_dB, const fl
 template <int P, int N>
 cudaError_t launch_chunks(const M3Params &p, char *ws, const M3BwdWs &w, bool prep,
                           cudaStream_t s) {
-  const int64_t nc = (p.L + kQ - 1) / kQ;
-  const dim3 grid((unsigned)nc, (unsigned)p.H, (unsigned)p.B);
+  const int64_t units = ((p.L + kQ - 1) / kQ) * p.H * p.B;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // persistent: one CTA per SM (shared memory admits no second) walking the units
+  const dim3 grid((unsigned)(units < sms ? units : sms));
   float *vu = reinterpret_cast<float *>(ws + w.vu);
   if (prep) {
     const size_t smem = (size_t)PrepSmem::total;
