@@ -123,8 +123,12 @@ size_t msc_selective_scan_saved_states_bytes(int64_t batch, int64_t dim, int64_t
 
 size_t msc_selective_scan_fwd_workspace_bytes(int64_t batch, int64_t dim, int64_t dstate,
                                               int64_t seqlen) {
-  if (batch <= 0 || dim <= 0 || dstate <= msc::kM1Slab || seqlen <= 0) return 0;
-  return sizeof(float) * (size_t)(batch * dim * seqlen);  // the sums over the earlier slabs
+  if (batch <= 0 || dim <= 0 || dstate <= 0 || seqlen <= 0) return 0;
+  if (dstate > msc::kM1Slab)
+    return sizeof(float) * (size_t)(batch * dim * seqlen);  // the sums over the earlier slabs
+  // time segments: per segment and state element a decay product and a state
+  const int64_t n_seg = msc::m1_fwd_segments(batch, dim, dstate, seqlen);
+  return n_seg > 1 ? sizeof(float) * (size_t)(2 * n_seg * batch * dim * dstate) : 0;
 }
 
 }  // extern "C"
@@ -194,8 +198,8 @@ msc_status m1_fwd(const char *fn, const msc_ss_fwd_args *a, const msc_ss_conv_ar
   OPTIONAL_PTR(fn, "saved_states", a->saved_states);
   const size_t need = msc_selective_scan_fwd_workspace_bytes(B, D, N, L);
   if (need > 0 && (workspace == nullptr || workspace_bytes < need))
-    return fail(MSC_ERR_WORKSPACE, "%s: dstate %lld needs a workspace of %zu bytes, %zu given",
-                fn, (long long)N, need, workspace ? workspace_bytes : (size_t)0);
+    return fail(MSC_ERR_WORKSPACE, "%s: these sizes need a workspace of %zu bytes, %zu given",
+                fn, need, workspace ? workspace_bytes : (size_t)0);
   OPTIONAL_PTR(fn, "workspace", workspace);
 
   msc::M1Params p = {};
@@ -206,7 +210,8 @@ msc_status m1_fwd(const char *fn, const msc_ss_fwd_args *a, const msc_ss_conv_ar
   p.u = a->u; p.delta = a->delta; p.Bm = a->Bm; p.Cm = a->Cm; p.z = a->z;
   p.A = a->A; p.Dp = a->D; p.bias = a->delta_bias; p.h0 = a->h0;
   p.out = a->out; p.final_state = a->final_state; p.saved = a->saved_states;
-  p.tok_part = need > 0 ? static_cast<float *>(workspace) : nullptr;
+  p.tok_part = need > 0 && N > msc::kM1Slab ? static_cast<float *>(workspace) : nullptr;
+  p.seg_ws = need > 0 && N <= msc::kM1Slab ? static_cast<float *>(workspace) : nullptr;
   if (conv) {
     p.conv_W = W;
     p.conv_w = conv->w; p.conv_b = conv->bias;

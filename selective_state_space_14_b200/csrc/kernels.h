@@ -41,8 +41,18 @@ struct M1Params {
   int64_t n0, ldN;
   int slab;         // kSlabWhole, kSlabFirst, kSlabMiddle or kSlabLast
   float *tok_part;  // fwd: [B][D][L] (y); bwd: [3][B][D][L] (y, dΔ sum, Σ λ B)
+  // forward in time segments (when the (batch, channel) grid alone cannot
+  // fill the GPU): segment blockIdx.z covers steps [z seg_len, (z+1) seg_len);
+  // seg_ws holds per segment and state element the decay product and the
+  // state reached from zero ([2][S][B][D][N], f32), then the carried state
+  int64_t seg_len;  // 0: the whole sequence in one segment
+  float *seg_ws;
 };
 constexpr int kM1Slab = 64;  // widest d_state one launch handles
+// time segments of the Mamba-1 forward for these sizes (1: none)
+int64_t m1_fwd_segments(int64_t B, int64_t D, int64_t N, int64_t L);
+int64_t m1_fwd_seg_len(int64_t L, int64_t n_seg);
+constexpr int kM1SegSteps = 32;  // segments are whole multiples of the forward's chunk
 constexpr int kSlabWhole = 0, kSlabFirst = 1, kSlabMiddle = 2, kSlabLast = 3;
 
 constexpr int MSC_MAX_N = 256;            // largest Mamba-1 d_state (slabs of 64 above 64)

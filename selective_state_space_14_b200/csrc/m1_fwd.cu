@@ -138,8 +138,8 @@ template <typename T, int kCh, int kOut, int kUOut>
 __device__ __forceinline__ void store_chunk(const M1Params &p, const float *sout,
                                             const float *sgate, const float *su,
                                             int64_t c_first, int64_t c_end, int64_t b,
-                                            int64_t tc, int tid, int nthreads) {
-  const int64_t D = p.D, L = p.L;
+                                            int64_t tc, int64_t t_end, int tid, int nthreads) {
+  const int64_t D = p.D, L = t_end;  // rows are L long; this pass ends at t_end
   for (int u = tid; u < kCh * (kTF / 8); u += nthreads) {
     const int chl = u / (kTF / 8);
     const int seg = u % (kTF / 8);
@@ -148,7 +148,7 @@ __device__ __forceinline__ void store_chunk(const M1Params &p, const float *sout
     const float4 a = *reinterpret_cast<const float4 *>(sout + chl * kOut + seg * 8);
     const float4 e = *reinterpret_cast<const float4 *>(sout + chl * kOut + seg * 8 + 4);
     float v[8] = {a.x, a.y, a.z, a.w, e.x, e.y, e.z, e.w};
-    const int64_t row = (b * D + c) * L, t0 = tc + seg * 8;
+    const int64_t row = (b * D + c) * p.L, t0 = tc + seg * 8;
     if (su) {  // the conv's output u (exact: values already rounded to T)
       const float4 ua = *reinterpret_cast<const float4 *>(su + chl * kUOut + seg * 8);
       const float4 ue = *reinterpret_cast<const float4 *>(su + chl * kUOut + seg * 8 + 4);
@@ -180,8 +180,13 @@ __device__ __forceinline__ void store_chunk(const M1Params &p, const float *sout
 
 // kConv: the causal conv1d + SiLU fused ahead: the token runs read the conv's
 // input x (from the stage, the W-1 inputs before a chunk from the halo) and
-// turn it into u
-template <typename T, int kN, bool kConv>
+// turn it into u.
+// Time segments (p.seg_len > 0): the CTA covers segment blockIdx.z.  kSum:
+// the segment's summary alone, from a zero state -- the product of its decays
+// and the state it reaches, per state element, to seg_ws -- with no outputs;
+// otherwise the segment runs from its carried state (seg_ws, written by the
+// combine kernel; h0 for the first segment) and writes its outputs.
+template <typename T, int kN, bool kConv, bool kSum>
 __global__ void __launch_bounds__(kWarps * 32, 6) m1_fwd_kernel(const M1Params p) {
   using S = FwdSmem<kN, kConv>;
   using Lay = Layout<kN, kWarps>;
@@ -216,18 +221,28 @@ __global__ void __launch_bounds__(kWarps * 32, 6) m1_fwd_kernel(const M1Params p
   const bool active = c < c_end;
   const T *Bg = static_cast<const T *>(p.Bm) + ((b * p.G + g) * ldN + ns) * L;
   const T *Cg = static_cast<const T *>(p.Cm) + ((b * p.G + g) * ldN + ns) * L;
-  const int64_t n_chunks = (L + kTF - 1) / kTF;
+  // this pass's steps [tb, te): the whole sequence, or time segment blockIdx.z
+  const int64_t seg = blockIdx.z, n_seg = gridDim.z;
+  const int64_t tb = p.seg_len > 0 ? seg * p.seg_len : 0;
+  const int64_t te = p.seg_len > 0 && tb + p.seg_len < L ? tb + p.seg_len : L;
+  const int64_t n_chunks = (te - tb + kTF - 1) / kTF;
   const int64_t n_save = (L + kM1SaveInterval - 1) / kM1SaveInterval;
+  const int64_t seg_elems = p.B * D * N;  // state elements (whole d_state: N == ldN)
   using R = FwdRaw<T, kN>;
   unsigned char *raw = reinterpret_cast<unsigned char *>(smem + S::raw);
 
   // this thread's state pair and its A * log2(e)
   const int n0 = 2 * pr, n1 = 2 * pr + 1;
   float2 h = make_float2(0.f, 0.f), A2 = make_float2(0.f, 0.f);
+  float2 decay = make_float2(1.f, 1.f);  // kSum: the product of the segment's decays
   if (active) {
     if (n0 < N) A2.x = p.A[c * ldN + ns + n0] * kLog2e;
     if (n1 < N) A2.y = p.A[c * ldN + ns + n1] * kLog2e;
-    if (p.h0) {
+    if (!kSum && seg > 0) {  // the state carried into this segment
+      const float *cs = p.seg_ws + seg_elems * (n_seg + seg - 1) + (b * D + c) * N;
+      if (n0 < N) h.x = cs[n0];
+      if (n1 < N) h.y = cs[n1];
+    } else if (!kSum && p.h0) {
       if (n0 < N) h.x = p.h0[(b * D + c) * ldN + ns + n0];
       if (n1 < N) h.y = p.h0[(b * D + c) * ldN + ns + n1];
     }
@@ -248,13 +263,16 @@ __global__ void __launch_bounds__(kWarps * 32, 6) m1_fwd_kernel(const M1Params p
   if constexpr (kConv) {
     // the inputs before the sequence: the conv state (entry j holds x at time
     // j - (W-1)) or zeros
+    // (a time segment after the first takes them from x itself)
     const int Wd = (int)p.conv_W;
     for (int i = tid; i < kCh * 3; i += kThreads) {
       const int cl = i / 3, k = i % 3, pos = k - 3;
       const int64_t cc = c_first + cl;
       float v = 0.f;
-      if (cc < c_end && p.conv_xs_in && pos >= -(Wd - 1))
-        v = p.conv_xs_in[(b * D + cc) * (Wd - 1) + (Wd - 1) + pos];
+      if (cc < c_end && pos >= -(Wd - 1)) {
+        if (tb > 0) v = to_f32(static_cast<const T *>(p.u)[(b * D + cc) * L + tb + pos]);
+        else if (p.conv_xs_in) v = p.conv_xs_in[(b * D + cc) * (Wd - 1) + (Wd - 1) + pos];
+      }
       sHalo[cl * 4 + k] = v;
     }
     for (int i = tid; i < kCh * 5; i += kThreads) {  // taps right-aligned, then the bias
@@ -269,16 +287,16 @@ __global__ void __launch_bounds__(kWarps * 32, 6) m1_fwd_kernel(const M1Params p
     }
   }
   __syncthreads();
-  fwd_issue_raw<T, kN>(p, raw, rows, 0, tid);
+  fwd_issue_raw<T, kN>(p, raw, rows, tb, tid);
   for (int64_t ch = 0; ch <= n_chunks; ++ch) {
-    const int64_t tc = ch * kTF;
+    const int64_t tc = tb + ch * kTF;
     cp_async_wait<0>();
     __syncthreads();  // this chunk's raw inputs are in; the last chunk is done
-    if (ch > 0)
+    if (ch > 0 && !kSum)
       store_chunk<T, kCh, S::kOut, S::kUOut>(
           p, sOut, sGate,
           kConv && p.u_out ? smem + S::su + ((ch - 1) & 1) * kCh * S::kUOut : nullptr,
-                                   c_first, c_end, b, tc - kTF, tid, kThreads);
+                                   c_first, c_end, b, tc - kTF, te, tid, kThreads);
     if (ch == n_chunks) break;
     // ---- per-token values: kRun steps of one channel per thread ---------------
     {
@@ -351,7 +369,7 @@ __global__ void __launch_bounds__(kWarps * 32, 6) m1_fwd_kernel(const M1Params p
 #pragma unroll
       for (int i = 0; i < kRun; ++i) {
         float4 tk = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (tact && tc + tseg * kRun + i < L) {
+        if (tact && tc + tseg * kRun + i < te) {
           const float vv = v[i] + tbias;
           const float d = p.softplus ? softplus(vv) : vv;
           tk = make_float4(d, d * x[i], tDc * x[i], p.z ? silu(zv[i]) : 1.f);
@@ -390,15 +408,28 @@ __global__ void __launch_bounds__(kWarps * 32, 6) m1_fwd_kernel(const M1Params p
     }
     __syncthreads();  // tables ready; the raw buffer and the output tile are free
     if (ch + 1 < n_chunks) fwd_issue_raw<T, kN>(p, raw, rows, tc + kTF, tid);
+    if constexpr (kSum) {
+      // no outputs: the state walk alone
+#pragma unroll 1
+      for (int t = 0; t < kTF; ++t) {
+        const float4 tk = sTok[t * kCh + chl];
+        const float4 bcv = sBC[t * kP + pr];
+        const float2 a = ex2_2(mul2(splat2(tk.x), A2));
+        h = fma2(a, h, mul2(splat2(tk.y), make_float2(bcv.x, bcv.y)));
+        decay = mul2(decay, a);
+      }
+      continue;
+    }
 
     // ---- the recurrence over the chunk -------------------------------------
+    if constexpr (!kSum) {
 #pragma unroll 1
     for (int grp = 0; grp < kTF / kP; ++grp) {
       float yp[kP];
 #pragma unroll
       for (int k = 0; k < kP; ++k) {
         const int t = grp * kP + k;
-        if (t % kM1SaveInterval == 0 && active && p.saved && tc + t < L) {
+        if (!kSum && t % kM1SaveInterval == 0 && active && p.saved && tc + t < te) {
           float *dst = p.saved + ((b * D + c) * n_save + (tc + t) / kM1SaveInterval) * ldN + ns;
           if (n0 < N) dst[n0] = h.x;
           if (n1 < N) dst[n1] = h.y;
@@ -428,12 +459,14 @@ __global__ void __launch_bounds__(kWarps * 32, 6) m1_fwd_kernel(const M1Params p
       }
       __syncwarp();
     }
+    }
   }
 
   if constexpr (kConv) {
-    // the conv state for the next call: the last W-1 inputs
+    // the conv state for the next call: the last W-1 inputs (the last
+    // segment's outputs pass writes it)
     const int Wd = (int)p.conv_W;
-    if (p.conv_xs_out) {
+    if (p.conv_xs_out && !kSum && seg == n_seg - 1) {
       for (int i = tid; i < kCh * (Wd - 1); i += kThreads) {
         const int cl = i / (Wd - 1), j = i % (Wd - 1);
         const int64_t cc = c_first + cl;
@@ -445,30 +478,83 @@ __global__ void __launch_bounds__(kWarps * 32, 6) m1_fwd_kernel(const M1Params p
       }
     }
   }
-  if (active && p.final_state) {
+  if (kSum) {
+    if (active) {  // the segment's summary: decays [seg], state [n_seg + seg]
+      float *dd = p.seg_ws + seg_elems * seg + (b * D + c) * N;
+      float *hh = p.seg_ws + seg_elems * (n_seg + seg) + (b * D + c) * N;
+      if (n0 < N) { dd[n0] = decay.x; hh[n0] = h.x; }
+      if (n1 < N) { dd[n1] = decay.y; hh[n1] = h.y; }
+    }
+    return;
+  }
+  if (active && p.final_state && seg == n_seg - 1) {
     float *dst = p.final_state + (b * D + c) * ldN + ns;
     if (n0 < N) dst[n0] = h.x;
     if (n1 < N) dst[n1] = h.y;
   }
 }
 
-template <typename T, int kN, bool kConv>
-cudaError_t launch_c(const M1Params &p, cudaStream_t s) {
+// The segments' summaries combined in time order: for state element e, with
+// segment s taking a state x to decay_s x + state_s, the state entering
+// segment s + 1 is the composition of segments 0..s applied to h0.  A warp
+// takes one element, its lanes the segments (at most 32), and composes them
+// with the warp-shuffle scan of the linear-recurrence monoid
+// (p, h) o (p', h') = (p p', p' h + h'); the result for segment s goes over
+// state_s, which only this warp reads.
+__global__ void m1_seg_combine_kernel(const M1Params p, int n_seg) {
+  const int64_t elems = p.B * p.D * p.N;
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t e = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); e < elems;
+       e += warps) {
+    float dc = 1.f, st = 0.f;  // segments past the last compose as the identity
+    if (lane < n_seg) {
+      dc = p.seg_ws[elems * lane + e];
+      st = p.seg_ws[elems * (n_seg + lane) + e];
+    }
+    float pe, he;
+    warp_scan_fwd(dc, st, pe, he);
+    // inclusive: segments 0..lane, applied to the initial state
+    const float pi = pe * dc, hi = fmaf(dc, he, st);
+    const float x0 = p.h0 ? p.h0[e] : 0.f;
+    if (lane < n_seg - 1) p.seg_ws[elems * (n_seg + lane) + e] = fmaf(pi, x0, hi);
+  }
+}
+
+template <typename T, int kN, bool kConv, bool kSum>
+cudaError_t launch_c(const M1Params &p, int64_t n_seg, cudaStream_t s) {
   using Lay = Layout<kN, kWarps>;
   const size_t smem =
       sizeof(float) * (size_t)FwdSmem<kN, kConv>::total_floats + FwdRaw<T, kN>::bytes;
-  cudaError_t e = cudaFuncSetAttribute(m1_fwd_kernel<T, kN, kConv>,
+  cudaError_t e = cudaFuncSetAttribute(m1_fwd_kernel<T, kN, kConv, kSum>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int64_t per_group = p.D / p.G;
-  dim3 grid((unsigned)(p.G * ((per_group + Lay::kCh - 1) / Lay::kCh)), (unsigned)p.B);
-  m1_fwd_kernel<T, kN, kConv><<<grid, Lay::kThreads, smem, s>>>(p);
+  dim3 grid((unsigned)(p.G * ((per_group + Lay::kCh - 1) / Lay::kCh)), (unsigned)p.B,
+            (unsigned)n_seg);
+  m1_fwd_kernel<T, kN, kConv, kSum><<<grid, Lay::kThreads, smem, s>>>(p);
   return cudaGetLastError();
+}
+
+template <typename T, int kN, bool kConv>
+cudaError_t launch_seg(const M1Params &p, cudaStream_t s) {
+  if (p.seg_len <= 0) return launch_c<T, kN, kConv, false>(p, 1, s);
+  // time segments: summaries, their combination, then every segment from its
+  // carried state
+  const int64_t n_seg = (p.L + p.seg_len - 1) / p.seg_len;
+  cudaError_t e = launch_c<T, kN, kConv, true>(p, n_seg, s);
+  if (e != cudaSuccess) return e;
+  const int64_t elems = p.B * p.D * p.N;
+  int64_t blocks = (elems + 7) / 8;  // 8 warps of 32 per block, a warp per element
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  m1_seg_combine_kernel<<<(unsigned)blocks, 256, 0, s>>>(p, (int)n_seg);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  return launch_c<T, kN, kConv, false>(p, n_seg, s);
 }
 
 template <typename T, int kN>
 cudaError_t launch_t(const M1Params &p, cudaStream_t s) {
-  return p.conv_w ? launch_c<T, kN, true>(p, s) : launch_c<T, kN, false>(p, s);
+  return p.conv_w ? launch_seg<T, kN, true>(p, s) : launch_seg<T, kN, false>(p, s);
 }
 
 template <typename T>
@@ -482,6 +568,31 @@ cudaError_t launch_n(const M1Params &p, cudaStream_t s) {
 
 }  // namespace
 
+// Time segments of the forward: only when the (batch, channel-block) grid
+// gives fewer CTAs than SMs (small batch, few channels), aiming at about two
+// CTAs per SM, each segment at least two chunks long and at most 32 segments
+// (one warp's lanes compose them).  d_state up to one slab; the forward with
+// the conv fused ahead takes the same segments, so that it stays bit-equal to
+// the conv followed by the plain forward.
+int64_t m1_fwd_segments(int64_t B, int64_t D, int64_t N, int64_t L) {
+  if (N > kM1Slab || B <= 0 || D <= 0 || L <= 0) return 1;
+  const int64_t kch = pad_n(N) == 16 ? 16 : (pad_n(N) == 32 ? 8 : 4);  // channels per CTA
+  const int64_t ctas = B * ((D + kch - 1) / kch);
+  constexpr int64_t kSMs = 148;
+  if (ctas >= kSMs) return 1;
+  int64_t n = (2 * kSMs + ctas - 1) / ctas;
+  const int64_t by_len = L / (2 * kM1SegSteps);
+  if (n > by_len) n = by_len;
+  if (n > 32) n = 32;
+  if (n < 2) return 1;
+  return (L + m1_fwd_seg_len(L, n) - 1) / m1_fwd_seg_len(L, n);  // segments of whole chunks
+}
+
+int64_t m1_fwd_seg_len(int64_t L, int64_t n_seg) {
+  const int64_t per = (L + n_seg - 1) / n_seg;
+  return (per + kM1SegSteps - 1) / kM1SegSteps * kM1SegSteps;
+}
+
 // The whole d_state in one launch, or slabs of kM1Slab states in ascending
 // order, the sums over the states carried in tok_part.
 cudaError_t launch_m1_fwd(const M1Params &p0, cudaStream_t s) {
@@ -489,6 +600,11 @@ cudaError_t launch_m1_fwd(const M1Params &p0, cudaStream_t s) {
   const int64_t slabs = (n_tot + kM1Slab - 1) / kM1Slab;
   for (int64_t k = 0; k < slabs; ++k) {
     M1Params p = p0;
+    p.seg_len = 0;
+    if (slabs == 1) {
+      const int64_t n_seg = m1_fwd_segments(p0.B, p0.D, n_tot, p0.L);
+      if (n_seg > 1) p.seg_len = m1_fwd_seg_len(p0.L, n_seg);
+    }
     p.ldN = n_tot;
     p.n0 = k * kM1Slab;
     p.N = n_tot - p.n0 < kM1Slab ? n_tot - p.n0 : kM1Slab;

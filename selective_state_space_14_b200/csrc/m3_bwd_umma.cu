@@ -91,15 +91,6 @@ __device__ __forceinline__ void put2x2(unsigned char *base, int off, float v0, f
     v1 -= hf.y;
   }
 }
-// one element's parts, 2-byte stores (transposed writes)
-__device__ __forceinline__ void put1x2(unsigned char *base, int off, float v) {
-#pragma unroll
-  for (int q = 0; q < kParts; ++q) {
-    const bf16 h = __float2bfloat16_rn(v);
-    *reinterpret_cast<bf16 *>(base + q * kPl + off) = h;
-    v -= __bfloat162float(h);
-  }
-}
 // eight consecutive K elements of one row (16 bytes per part)
 __device__ __forceinline__ void put8x2(unsigned char *base, int off, const float (&v8)[8]) {
   float v[8];

@@ -40,8 +40,10 @@ def _err():
 def _fwd_args(**kw):
     a = msc.SsFwdArgs()
     a.struct_size = ctypes.sizeof(msc.SsFwdArgs)
+    # 2 x 4096 channels fill the GPU with channel blocks: a single pass over
+    # time, which needs no workspace
     a.io_dtype, a.batch, a.dim, a.dstate, a.seqlen, a.ngroups, a.delta_softplus = (
-        msc.MSC_BF16, 2, 64, 16, 128, 1, 1)
+        msc.MSC_BF16, 2, 4096, 16, 128, 1, 1)
     fake = ctypes.c_void_p(1 << 20)  # never dereferenced: the checks fail first
     for f in ("u", "delta", "A", "Bm", "Cm", "out"):
         setattr(a, f, fake)
@@ -90,7 +92,7 @@ def test_fwd_rejects_bad_sizes(field, value, status, word):
 def test_fwd_wide_state_needs_a_workspace():
     """Above 64 states the forward runs in slabs and needs its workspace; the
     call stops at that check (no launch)."""
-    assert msc.msc_selective_scan_fwd_workspace_bytes(2, 64, 64, 128) == 0
+    assert msc.msc_selective_scan_fwd_workspace_bytes(8, 1536, 64, 128) == 0
     assert msc.msc_selective_scan_fwd_workspace_bytes(2, 64, 65, 128) == 4 * 2 * 64 * 128
     assert _call_fwd(_fwd_args(dstate=128)) == WORKSPACE and "workspace" in _err()
 
@@ -210,6 +212,17 @@ def test_size_functions():
         4 * 2 * 3 * 2 * (16 * 32 + 16)
     assert msc.msc_selective_scan_bwd_workspace_bytes(8, 1536, 16, 2048, 1) <= \
         msc.MSC_STATIC_SCRATCH_BYTES
+
+
+def test_fwd_time_segments_workspace():
+    """The forward runs in time segments when its (batch, channel) grid has
+    fewer CTAs than SMs: two floats per segment and state element.  B1 D64
+    N16 L256 gives 4 channel blocks, so 4 segments of 64 steps; grids of 148
+    or more blocks, and d_state above 64 (slabs), take none."""
+    assert msc.msc_selective_scan_fwd_workspace_bytes(1, 64, 16, 256) == 4 * 2 * 4 * 64 * 16
+    assert msc.msc_selective_scan_fwd_workspace_bytes(8, 1536, 16, 2048) == 0
+    assert msc.msc_selective_scan_fwd_workspace_bytes(1, 64, 16, 63) == 0  # too short to split
+    assert msc.msc_selective_scan_fwd_workspace_bytes(1, 8, 128, 4096) == 4 * 1 * 8 * 4096
 
 
 def test_bwd_workspace_query_refuses_bad_groups():

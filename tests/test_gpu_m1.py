@@ -106,6 +106,31 @@ def test_parity_shapes(msc, case):
     _compare(_run_gpu(msc, p), _run_oracle(p), TOL[io])
 
 
+SEG_CASES = [
+    # (B, D, N, L, io): grids of few (batch, channel) blocks, so the forward
+    # runs in time segments combined by the warp-shuffle scan
+    (1, 64, 16, 256, "f32"),
+    (1, 16, 16, 1024, "f32"),
+    # 4096 steps in bf16: over that many steps a step-by-step f32 evaluation
+    # with correctly rounded exp already leaves the final state 1.75e-5 from
+    # the oracle (normwise), above the f32 bound
+    (1, 16, 16, 4096, "bf16"),
+    (2, 40, 32, 2000, "bf16"),
+    (1, 8, 64, 777, "f32"),
+    (1, 512, 16, 2048, "bf16"),
+]
+
+
+@pytest.mark.parametrize("case", SEG_CASES, ids=[f"B{c[0]}D{c[1]}N{c[2]}L{c[3]}{c[4]}" for c in SEG_CASES])
+def test_time_segments_parity(msc, case):
+    """Forward in time segments (and the backward from its saved states)
+    against the oracle: the segment count the workspace query implies is > 1."""
+    Bsz, D, N, L, io = case
+    assert msc.msc_selective_scan_fwd_workspace_bytes(Bsz, D, N, L) > 0
+    p = W.m1_problem(Bsz, D, N, L, io=io, seed=3000 + L, bias=True, with_h0=True)
+    _compare(_run_gpu(msc, p), _run_oracle(p), TOL[io])
+
+
 def test_determinism(msc):
     """Same inputs, same bits: five runs of forward and backward."""
     p = W.m1_problem(2, 130, 16, 700, io="bf16", seed=5, bias=True, with_h0=True)
@@ -118,8 +143,11 @@ def test_determinism(msc):
 def test_resume_is_bit_continuous(msc):
     """A scan over L equals a scan over L1 followed by one over L - L1 started
     from the first one's final state; bit-equal when L1 is a multiple of the
-    forward's 32-step chunk (and so of the 8-step saved-state interval)."""
-    p = W.m1_problem(1, 12, 16, 1536, io="f32", seed=9, bias=True)
+    forward's 32-step chunk (and so of the 8-step saved-state interval).  The
+    sizes fill the GPU with (batch, channel) blocks, so the forward walks time
+    in one pass (no time segments, whose composition rounds differently)."""
+    assert msc.msc_selective_scan_fwd_workspace_bytes(2, 1184, 16, 1536) == 0
+    p = W.m1_problem(2, 1184, 16, 1536, io="f32", seed=9, bias=True)
     a = m1_device_args(p)
     full, fs_full, _ = msc.msc_selective_scan_fwd(**a)
     L1 = 1024  # a multiple of the 32-step chunk
