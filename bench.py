@@ -360,6 +360,25 @@ class M3DiscStep:
                                                workspace=self.ws)
         self.gd = None
         self.disc_bwd()
+        # the same step through the fused entry points (the derived inputs are
+        # made inside the scan's kernels and never stored)
+        self.c = dict(x=self.a["x"], D=self.a["D"], z=self.a["z"], h0=None)
+        self.out_r, _, self.saved_r = msc.msc_mamba3_siso_scan_fwd_raw(**self.c, **self.raw,
+                                                                       **self.kw)
+        self.ws_r = torch.empty(max(msc.msc_mamba3_siso_scan_bwd_raw_workspace_bytes(
+            s.batch, s.seqlen, s.nheads, s.headdim, s.dstate, s.ngroups, s.nangles), 16),
+            device="cuda", dtype=torch.uint8)
+        self.gr = None
+        self.fused_bwd()
+
+    def fused_fwd(self):
+        self.msc.msc_mamba3_siso_scan_fwd_raw(**self.c, **self.raw, **self.kw, out=self.out_r,
+                                              saved_states=self.saved_r)
+
+    def fused_bwd(self):
+        self.gr = self.msc.msc_mamba3_siso_scan_bwd_raw(
+            **self.c, **self.raw, **self.kw, saved_states=self.saved_r, dout=self.dout,
+            workspace=self.ws_r, grads=self.gr)
 
     def disc_fwd(self):
         self.msc.msc_mamba3_siso_discretize(**self.raw, **self.kw, outs=self.o)
@@ -930,15 +949,20 @@ def extra_workloads(msc, args, world, peaks):
         n = max(3, args.steps // 2)
         _, (dfw, sfw, sbw, dbw) = time_steps([graphed(ds.disc_fwd), ds.scan_fwd, ds.scan_bwd,
                                               graphed(ds.disc_bwd)], n, 3, world)
+        _, (ffw, fbw) = time_steps([ds.fused_fwd, ds.fused_bwd], n, 3, world)
         s = ds.q.scan
         fb, bb = m3disc_bytes(s.batch, s.seqlen, s.nheads, s.dstate, s.ngroups, s.nangles, 2)
         res[name] = dict(
+            fused_fwd_ms=round(ffw, 4), fused_bwd_ms=round(fbw, 4),
             disc_fwd_ms=round(dfw, 4), scan_fwd_ms=round(sfw, 4), scan_bwd_ms=round(sbw, 4),
             disc_bwd_ms=round(dbw, 4),
-            value=round(s.token_channels / ((dfw + sfw + sbw + dbw) / 1e3), 1), unit=UNIT,
+            value=round(s.token_channels / ((ffw + fbw) / 1e3), 1), unit=UNIT,
+            unfused_value=round(s.token_channels / ((dfw + sfw + sbw + dbw) / 1e3), 1),
             disc_fwd_hbm_frac=round(fb / dfw / 1e6 / peaks["hbm_gbs"], 4),
             disc_bwd_hbm_frac=round(bb / dbw / 1e6 / peaks["hbm_gbs"], 4),
-            note="value: discretisation + scan forward + scan backward + discretisation backward")
+            note="value: scan forward + backward from raw projections (fused entry points); "
+                 "unfused_value: discretisation + scan forward + scan backward + "
+                 "discretisation backward as four calls")
         del ds
     except Exception as e:  # noqa: BLE001 -- report, keep the headline line
         res[name] = dict(error=str(e)[:200])
@@ -1013,9 +1037,10 @@ def run_only(args):
                 msc.msc_mamba3_siso_scan_bwd(**a, saved_states=saved, dout=dout, workspace=ws,
                                              grads=grads)
         units = m3.token_channels
-    elif phase in ("m3_disc_fwd", "m3_disc_bwd"):
+    elif phase in ("m3_disc_fwd", "m3_disc_bwd", "m3_raw_fwd", "m3_raw_bwd"):
         ds = M3DiscStep(W.make(args.workload or "m3disc_bf16_b8_h24_p64_n64_k32_l2048"), msc)
-        fn = ds.disc_fwd if phase == "m3_disc_fwd" else ds.disc_bwd
+        fn = {"m3_disc_fwd": ds.disc_fwd, "m3_disc_bwd": ds.disc_bwd, "m3_raw_fwd": ds.fused_fwd,
+              "m3_raw_bwd": ds.fused_bwd}[phase]
         units = ds.q.scan.token_channels
     elif phase in ("m1_conv_fwd", "conv_fwd", "conv_bwd"):
         q = W.make(args.workload or "m1conv_bf16_b8_d1536_n16_l2048_w4")
@@ -1123,7 +1148,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", choices=["m1_fwd", "m1_bwd", "m3_fwd", "m3_bwd", "decode",
                                        "m3_decode", "m1_conv_fwd", "conv_fwd", "conv_bwd",
-                                       "m3_disc_fwd", "m3_disc_bwd", "m3_decode_raw"],
+                                       "m3_disc_fwd", "m3_disc_bwd", "m3_raw_fwd", "m3_raw_bwd",
+                                       "m3_decode_raw"],
                     help="time one phase alone (for profiling); prints no bench line")
     ap.add_argument("--workload", default=None, help="workload name for --only")
     ap.add_argument("--graph", action="store_true",

@@ -6,9 +6,9 @@
  *   - the Mamba-1 selective scan, forward and backward (the selective SSM
  *     layer of "Mamba: Linear-Time Sequence Modeling with Selective State
  *     Spaces", Section 3 / Algorithm 2, as the state-spaces/mamba README's
- *     "Usage / Selective SSM" section names it; "Mamba SSM (Gu and Dao,
- *     2023)" with a "full backward pass through the recurrent SSM state" in
- *     the mamba-rs 0.7.0 README, "Features");
+ *     "Usage / Selective SSM" section names it; the mamba-rs 0.7.0 README,
+ *     "Features", lists the Gu and Dao 2023 SSM with backpropagation
+ *     through its recurrent state);
  *   - the Mamba-3 SISO scan, forward and backward (mamba-rs 0.7.0 README,
  *     "Features"; backward stages B2 output gating, B3 BPTT and B4 RoPE of
  *     Mamba3Scratch in mamba-rs 0.4.2 src/mamba3_siso/cpu/scratch.rs);
@@ -570,14 +570,74 @@ typedef struct {
 msc_status msc_mamba3_siso_discretize_bwd(const msc_m3_disc_bwd_args *args, msc_stream_t stream);
 
 /* ======================================================================
+ * Mamba-3 SISO scan from raw projections (discretisation fused in)
+ * ======================================================================
+ * The scan forward and backward with the discretisation and BCNorm above
+ * fused into them (the pages list the stages B6 "discretization" and B5
+ * "BCNorm" of Mamba3Scratch either side of the BPTT and RoPE stages, mamba-rs
+ * 0.4.2 src/mamba3_siso/cpu/scratch.rs).  The kernels derive alpha, beta,
+ * gamma, theta and the normalised Bm, Cm from the raw values as they stage
+ * each chunk, so theta [B, L, H, K] and the other derived inputs are never
+ * written or read in global memory.  Every derived value is rounded to bf16
+ * exactly as msc_mamba3_siso_discretize stores it, so:
+ *   msc_mamba3_siso_scan_fwd_raw  equals, bit for bit,
+ *     msc_mamba3_siso_discretize followed by msc_mamba3_siso_scan_fwd;
+ *   msc_mamba3_siso_scan_bwd_raw  equals, bit for bit,
+ *     msc_mamba3_siso_scan_bwd (on the discretised inputs) followed by
+ *     msc_mamba3_siso_discretize_bwd.
+ * bf16 io and dstate 16, 32 or 64 (the tensor-core kernels; other sizes:
+ * MSC_ERR_UNSUPPORTED -- take the two calls).
+ *
+ * In the scan arguments (msc_m3_fwd_args / msc_m3_bwd_args) alpha, beta,
+ * gamma, theta, Bm and Cm are ignored (may be NULL), and so, in the backward,
+ * are dB, dC, dalpha, dbeta, dgamma and dtheta: the scan's gradients of the
+ * derived inputs live in the workspace (msc_mamba3_siso_scan_bwd_raw
+ * _workspace_bytes), and the raw gradients go to `grads`.  dx, dz, dD and
+ * dh0 are the scan's, as in msc_mamba3_siso_scan_bwd.  Layouts as in
+ * msc_mamba3_siso_discretize:
+ *   dd_dt, dd_a, trap         bf16 [B, L, H]
+ *   angles                    bf16 [B, L, K]      (may be NULL when K = 0)
+ *   dt_bias                   f32  [H]            optional
+ *   B_raw, C_raw              bf16 [B, L, G, N]
+ *   ddd_dt, ddd_a, dtrap      f32  [B, L, H]      out
+ *   dangles                   f32  [B, L, K]      out (may be NULL when K = 0)
+ *   ddt_bias                  f32  [H]            out, optional
+ *   dB_raw, dC_raw            f32  [B, L, G, N]   out
+ */
+typedef struct {
+  uint32_t struct_size;
+  float A_floor, eps;
+  const void *dd_dt, *dd_a, *trap, *angles;
+  const float *dt_bias;    /* optional */
+  const void *B_raw, *C_raw;
+} msc_m3_raw_args;
+
+typedef struct {
+  uint32_t struct_size;
+  float *ddd_dt, *ddd_a, *dtrap, *dangles;
+  float *ddt_bias;         /* optional */
+  float *dB_raw, *dC_raw;
+} msc_m3_raw_grads;
+
+msc_status msc_mamba3_siso_scan_fwd_raw(const msc_m3_fwd_args *scan, const msc_m3_raw_args *raw,
+                                        msc_stream_t stream);
+size_t msc_mamba3_siso_scan_bwd_raw_workspace_bytes(int64_t batch, int64_t seqlen,
+                                                    int64_t nheads, int64_t headdim,
+                                                    int64_t dstate, int64_t ngroups,
+                                                    int64_t nangles);
+msc_status msc_mamba3_siso_scan_bwd_raw(const msc_m3_bwd_args *scan, const msc_m3_raw_args *raw,
+                                        const msc_m3_raw_grads *grads, void *workspace,
+                                        size_t workspace_bytes, msc_stream_t stream);
+
+/* ======================================================================
  * Measurement probes: the compute ceiling of the Mamba-1 scans
  * ======================================================================
  * Every state element of every step of the Mamba-1 recurrence takes one
  * 2^x for its decay exp(delta A) (the discretisation of the selective SSM,
  * Mamba paper, Section 3 / Algorithm 2), so the GPU's rate of 2^x bounds the
- * scans from below independently of their memory traffic (the pages quote
- * "the step is dominated by the scan and the other non-GEMM kernels",
- * mamba-rs 0.7.0 README, "Performance").  These probes measure that rate and
+ * scans from below independently of their memory traffic (mamba-rs 0.7.0
+ * README, "Performance", names the scan and the other kernels outside the
+ * GEMMs as the bulk of a training step).  These probes measure that rate and
  * the FMA pipe's, for the roofline's compute side.  They are not part of
  * the scan path.
  *

@@ -22,8 +22,8 @@
  *       h_t[n]  = exp(delta_t * A[n]) * h_{t-1}[n] + delta_t * B_t[n] * x_t
  *       y_t     = sum_n C_t[n] h_t[n] + D * x_t
  *       out_t   = y_t * silu(z_t)
- *   and its backward pass through the recurrent state ("full backward pass
- *   through the recurrent SSM state", mamba-rs 0.7.0 README, "Features").
+ *   and its backward pass through the recurrent state (backpropagation
+ *   through time over the SSM state, mamba-rs 0.7.0 README, "Features").
  *
  *   Mamba-3 SISO scan (mamba-rs 0.7.0 README, "Features"; backward stages
  *   B2 output gating, B3 BPTT and B4 RoPE of Mamba3Scratch in mamba-rs 0.4.2

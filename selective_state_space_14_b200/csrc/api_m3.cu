@@ -89,8 +89,76 @@ size_t msc_mamba3_siso_scan_fwd_workspace_bytes(int64_t batch, int64_t seqlen, i
   return sizeof(float) * (size_t)(batch * seqlen * nheads * headdim);  // y over the earlier slabs
 }
 
-msc_status msc_mamba3_siso_scan_fwd(const msc_m3_fwd_args *a, msc_stream_t stream) {
-  const char *fn = "msc_mamba3_siso_scan_fwd";
+}  // extern "C"
+
+namespace {
+
+// The raw projections' checks for the fused entry points (after the scan
+// struct's own checks): bf16 io, d_state 16, 32 or 64 (the tensor-core
+// kernels), and the raw rows present wherever there are tokens.
+template <typename Scan>
+msc_status check_raw(const char *fn, const Scan *a, const msc_m3_raw_args *raw) {
+  if (!a) return api_fail(MSC_ERR_INVALID_ARG, "%s: args is NULL", fn);
+  if (!raw) return api_fail(MSC_ERR_INVALID_ARG, "%s: raw is NULL", fn);
+  if (raw->struct_size < sizeof(msc_m3_raw_args))
+    return api_fail(MSC_ERR_INVALID_ARG, "%s: raw struct_size %u is smaller than the struct (%zu)",
+                    fn, raw->struct_size, sizeof(msc_m3_raw_args));
+  if (a->io_dtype != MSC_BF16)
+    return api_fail(MSC_ERR_UNSUPPORTED,
+                    "%s: io_dtype %d: the fused path takes bf16 io (use "
+                    "msc_mamba3_siso_discretize and the scan)", fn, (int)a->io_dtype);
+  // the tensor-core kernels' own sizes: their BCNorm sums runs of 8 states
+  // in the order the discretisation kernel does, and divides by d_state
+  if (a->dstate != 16 && a->dstate != 32 && a->dstate != 64)
+    return api_fail(MSC_ERR_UNSUPPORTED,
+                    "%s: dstate %lld: the fused path takes d_state 16, 32 or 64 (use "
+                    "msc_mamba3_siso_discretize and the scan)", fn, (long long)a->dstate);
+  if (!(raw->A_floor >= 0.f) || !(raw->eps >= 0.f))
+    return api_fail(MSC_ERR_INVALID_ARG, "%s: A_floor and eps must be >= 0", fn);
+  M3_OPTIONAL(fn, "dt_bias", raw->dt_bias);
+  if (a->batch > 0 && a->seqlen > 0) {
+    M3_REQUIRE(fn, "dd_dt", raw->dd_dt);
+    M3_REQUIRE(fn, "dd_a", raw->dd_a);
+    M3_REQUIRE(fn, "trap", raw->trap);
+    if (a->nangles > 0) M3_REQUIRE(fn, "angles", raw->angles);
+    M3_REQUIRE(fn, "B_raw", raw->B_raw);
+    M3_REQUIRE(fn, "C_raw", raw->C_raw);
+  }
+  return MSC_OK;
+}
+
+// The scan arguments with the derived inputs (alpha .. theta, Bm, Cm) taken
+// by the raw rows, so that the scan's own pointer checks test those.
+template <typename Scan>
+Scan with_raw(const Scan *a, const msc_m3_raw_args *raw) {
+  Scan s = *a;
+  s.Bm = raw->B_raw;
+  s.Cm = raw->C_raw;
+  s.alpha = raw->dd_dt;
+  s.beta = raw->dd_a;
+  s.gamma = raw->trap;
+  s.theta = raw->angles;
+  return s;
+}
+
+void set_raw(msc::M3Params &p, const msc_m3_raw_args *raw) {
+  p.raw = true;
+  p.Bm = raw->B_raw;
+  p.Cm = raw->C_raw;
+  p.alpha = p.beta = p.gamma = p.theta = nullptr;
+  p.dd_dt = raw->dd_dt;
+  p.dd_a = raw->dd_a;
+  p.trap = raw->trap;
+  p.angles = raw->angles;
+  p.dt_bias = raw->dt_bias;
+  p.A_floor = raw->A_floor;
+  p.eps = raw->eps;
+}
+
+// the scan forward; raw non-null: from raw projections (the arguments'
+// derived-input pointers already replaced by with_raw)
+msc_status m3_fwd_impl(const char *fn, const msc_m3_fwd_args *a, const msc_m3_raw_args *raw,
+                       msc_stream_t stream) {
   // callers built before the workspace fields pass a shorter struct: no workspace
   msc_status st = check_m3(fn, a, offsetof(msc_m3_fwd_args, workspace));
   if (st != MSC_OK) return st;
@@ -136,7 +204,26 @@ msc_status msc_mamba3_siso_scan_fwd(const msc_m3_fwd_args *a, msc_stream_t strea
   p.Dp = a->D; p.h0 = a->h0; p.out = a->out; p.final_state = a->final_state;
   p.saved = a->saved_states;
   p.tok_y = need > 0 ? static_cast<float *>(workspace) : nullptr;
+  if (raw) set_raw(p, raw);
   return api_cuda(msc::launch_m3_fwd(p, s), fn);
+}
+
+}  // namespace
+
+extern "C" {
+
+msc_status msc_mamba3_siso_scan_fwd(const msc_m3_fwd_args *a, msc_stream_t stream) {
+  return m3_fwd_impl("msc_mamba3_siso_scan_fwd", a, nullptr, stream);
+}
+
+msc_status msc_mamba3_siso_scan_fwd_raw(const msc_m3_fwd_args *a, const msc_m3_raw_args *raw,
+                                        msc_stream_t stream) {
+  const char *fn = "msc_mamba3_siso_scan_fwd_raw";
+  msc_status st = check_m3(fn, a, offsetof(msc_m3_fwd_args, workspace));
+  if (st != MSC_OK) return st;
+  if ((st = check_raw(fn, a, raw)) != MSC_OK) return st;
+  const msc_m3_fwd_args s = with_raw(a, raw);
+  return m3_fwd_impl(fn, &s, raw, stream);
 }
 
 size_t msc_mamba3_siso_scan_bwd_workspace_bytes(int64_t batch, int64_t seqlen, int64_t nheads,
@@ -147,9 +234,16 @@ size_t msc_mamba3_siso_scan_bwd_workspace_bytes(int64_t batch, int64_t seqlen, i
   return msc::m3_bwd_workspace_bytes(batch, seqlen, nheads, headdim, dstate, ngroups, nangles);
 }
 
-msc_status msc_mamba3_siso_scan_bwd(const msc_m3_bwd_args *a, void *workspace,
-                                    size_t workspace_bytes, msc_stream_t stream) {
-  const char *fn = "msc_mamba3_siso_scan_bwd";
+}  // extern "C"
+
+namespace {
+
+// the scan backward; raw non-null: from raw projections (derived-input
+// pointers already replaced by with_raw; the gradients of the derived inputs
+// go where the arguments say -- the fused entry point points them into its
+// workspace)
+msc_status m3_bwd_impl(const char *fn, const msc_m3_bwd_args *a, const msc_m3_raw_args *raw,
+                       void *workspace, size_t workspace_bytes, msc_stream_t stream) {
   msc_status st = check_m3(fn, a);
   if (st != MSC_OK) return st;
   const int64_t B = a->batch, L = a->seqlen, H = a->nheads, P = a->headdim, N = a->dstate;
@@ -205,7 +299,104 @@ msc_status msc_mamba3_siso_scan_bwd(const msc_m3_bwd_args *a, void *workspace,
   p.dx = a->dx; p.dz = a->z ? a->dz : nullptr; p.dB = a->dB; p.dC = a->dC;
   p.dalpha = a->dalpha; p.dbeta = a->dbeta; p.dgamma = a->dgamma; p.dtheta = a->dtheta;
   p.dD = a->dD; p.dh0 = a->dh0; p.ws = workspace; p.ws_bytes = workspace_bytes;
+  if (raw) set_raw(p, raw);
   return api_cuda(msc::launch_m3_bwd(p, s), fn);
+}
+
+// the fused backward's workspace: the scan's own, then the scan's f32
+// gradients of the derived inputs: dalpha, dbeta, dgamma [B, L, H], dtheta
+// [B, L, H, K], dB, dC [B, L, G, N]
+struct RawWs {
+  size_t da, db, dg, dth, dB, dC, total;
+};
+RawWs raw_ws(int64_t B, int64_t L, int64_t H, int64_t P, int64_t N, int64_t G, int64_t K) {
+  auto up = [](size_t v) { return (v + 255) / 256 * 256; };
+  RawWs w;
+  w.da = up(msc::m3_bwd_workspace_bytes(B, L, H, P, N, G, K));
+  const size_t th = up(sizeof(float) * (size_t)(B * L * H));
+  w.db = w.da + th;
+  w.dg = w.db + th;
+  w.dth = w.dg + th;
+  w.dB = w.dth + up(sizeof(float) * (size_t)(B * L * H * (K > 0 ? K : 1)));
+  w.dC = w.dB + up(sizeof(float) * (size_t)(B * L * G * N));
+  w.total = w.dC + up(sizeof(float) * (size_t)(B * L * G * N));
+  return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+msc_status msc_mamba3_siso_scan_bwd(const msc_m3_bwd_args *a, void *workspace,
+                                    size_t workspace_bytes, msc_stream_t stream) {
+  return m3_bwd_impl("msc_mamba3_siso_scan_bwd", a, nullptr, workspace, workspace_bytes, stream);
+}
+
+size_t msc_mamba3_siso_scan_bwd_raw_workspace_bytes(int64_t batch, int64_t seqlen,
+                                                    int64_t nheads, int64_t headdim,
+                                                    int64_t dstate, int64_t ngroups,
+                                                    int64_t nangles) {
+  if (batch <= 0 || seqlen <= 0 || nheads <= 0 || headdim <= 0 || dstate <= 0 || ngroups <= 0 ||
+      nangles < 0)
+    return 0;
+  return raw_ws(batch, seqlen, nheads, headdim, dstate, ngroups, nangles).total;
+}
+
+msc_status msc_mamba3_siso_scan_bwd_raw(const msc_m3_bwd_args *a, const msc_m3_raw_args *raw,
+                                        const msc_m3_raw_grads *grads, void *workspace,
+                                        size_t workspace_bytes, msc_stream_t stream) {
+  const char *fn = "msc_mamba3_siso_scan_bwd_raw";
+  msc_status st = check_m3(fn, a);
+  if (st != MSC_OK) return st;
+  if ((st = check_raw(fn, a, raw)) != MSC_OK) return st;
+  if (!grads) return api_fail(MSC_ERR_INVALID_ARG, "%s: grads is NULL", fn);
+  if (grads->struct_size < sizeof(msc_m3_raw_grads))
+    return api_fail(MSC_ERR_INVALID_ARG,
+                    "%s: grads struct_size %u is smaller than the struct (%zu)", fn,
+                    grads->struct_size, sizeof(msc_m3_raw_grads));
+  M3_OPTIONAL(fn, "ddt_bias", grads->ddt_bias);
+  const int64_t B = a->batch, L = a->seqlen, H = a->nheads, P = a->headdim, N = a->dstate;
+  const int64_t G = a->ngroups, K = a->nangles;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  msc_m3_bwd_args sa = with_raw(a, raw);
+  if (B == 0 || L == 0) {  // no tokens: dD, dh0 and the bias gradient are 0
+    st = m3_bwd_impl(fn, &sa, raw, workspace, workspace_bytes, stream);
+    if (st != MSC_OK || !grads->ddt_bias) return st;
+    return api_cuda(cudaMemsetAsync(grads->ddt_bias, 0, sizeof(float) * (size_t)H, s), fn);
+  }
+  const RawWs w = raw_ws(B, L, H, P, N, G, K);
+  if (workspace == nullptr || workspace_bytes < w.total)
+    return api_fail(MSC_ERR_WORKSPACE, "%s: workspace of %zu bytes given, %zu required", fn,
+                    workspace ? workspace_bytes : (size_t)0, w.total);
+  M3_REQUIRE(fn, "workspace", workspace);
+  M3_REQUIRE(fn, "ddd_dt", grads->ddd_dt);
+  M3_REQUIRE(fn, "ddd_a", grads->ddd_a);
+  M3_REQUIRE(fn, "dtrap", grads->dtrap);
+  if (K > 0) M3_REQUIRE(fn, "dangles", grads->dangles);
+  M3_REQUIRE(fn, "dB_raw", grads->dB_raw);
+  M3_REQUIRE(fn, "dC_raw", grads->dC_raw);
+  char *ws = static_cast<char *>(workspace);
+  sa.dalpha = reinterpret_cast<float *>(ws + w.da);
+  sa.dbeta = reinterpret_cast<float *>(ws + w.db);
+  sa.dgamma = reinterpret_cast<float *>(ws + w.dg);
+  sa.dtheta = reinterpret_cast<float *>(ws + w.dth);
+  sa.dB = reinterpret_cast<float *>(ws + w.dB);
+  sa.dC = reinterpret_cast<float *>(ws + w.dC);
+  st = m3_bwd_impl(fn, &sa, raw, workspace, w.da, stream);
+  if (st != MSC_OK) return st;
+  // the discretisation's backward on the scan's gradients of its outputs
+  msc::M3DiscParams d = {};
+  d.io = a->io_dtype;
+  d.B = B; d.L = L; d.H = H; d.N = N; d.G = G; d.K = K;
+  d.A_floor = raw->A_floor; d.eps = raw->eps;
+  d.dd_dt = raw->dd_dt; d.dd_a = raw->dd_a; d.trap = raw->trap; d.angles = raw->angles;
+  d.dt_bias = raw->dt_bias; d.B_raw = raw->B_raw; d.C_raw = raw->C_raw;
+  d.dalpha = sa.dalpha; d.dbeta = sa.dbeta; d.dgamma = sa.dgamma; d.dtheta = sa.dtheta;
+  d.dB = sa.dB; d.dC = sa.dC;
+  d.ddd_dt = grads->ddd_dt; d.ddd_a = grads->ddd_a; d.dtrap = grads->dtrap;
+  d.dangles = grads->dangles; d.ddt_bias = grads->ddt_bias;
+  d.dB_raw = grads->dB_raw; d.dC_raw = grads->dC_raw;
+  return api_cuda(msc::launch_m3_disc_bwd(d, s), fn);
 }
 
 }  // extern "C"

@@ -111,6 +111,14 @@ struct M3Params {
   int64_t n0, ldN;
   int slab;  // kSlabWhole, kSlabFirst, kSlabMiddle or kSlabLast
   float *tok_y, *tok_dx;  // [B, L, H, P] f32
+  // from raw projections (bf16 io, d_state <= kM3Slab): alpha, beta, gamma,
+  // theta and the normalised B, C are derived in the kernels from these, each
+  // rounded to bf16 as the discretisation kernel stores it (Bm, Cm point at
+  // B_raw, C_raw; alpha .. theta are unused)
+  bool raw;
+  const void *dd_dt, *dd_a, *trap, *angles;  // [B, L, H] x3, [B, L, K]
+  const float *dt_bias;                      // [H] or null
+  float A_floor, eps;
 };
 constexpr int kM3Slab = 64;  // widest d_state one launch handles
 cudaError_t launch_m3_fwd(const M3Params &p, cudaStream_t s);

@@ -1,6 +1,6 @@
 // m1_bwd.cu -- Mamba-1 selective scan, backward through the recurrent state
-// (sm_100a).  "Full backward pass through the recurrent SSM state", mamba-rs
-// 0.7.0 README, "Features".
+// (sm_100a): backpropagation through time over the SSM state, mamba-rs 0.7.0
+// README, "Features".
 //
 // With g_t = dout_t silu(z_t) and a_t[n] = exp(delta_t A[c,n]), the state
 // adjoint runs backwards in time,

@@ -31,6 +31,7 @@
 // steps (lanes 4 i + q hold step i of angle pairs q, q + 4, ...) and the
 // per-warp totals, which is also the layout the rotation writes in.
 #include "m3_common.cuh"
+#include "m3_disc_common.cuh"
 #include "umma.cuh"
 
 namespace msc {
@@ -62,7 +63,8 @@ struct UmFwdSmem {
                        wcd = crow + 256,           // [kG][Q] partial Ct_t . Bt_prev per angle group
                        xprev = wcd + kG * 256,     // [2][P], by chunk parity
                        bprev = xprev + 2 * P * 4,  // [2][N]
-                       misc = bprev + 2 * N * 4;
+                       dtv = bprev + 2 * N * 4,    // [Q] dt of the next chunk's steps (raw input)
+                       misc = dtv + 256;
   static constexpr int total = misc + 32;  // tmem slot, mbarrier, error flag
 };
 
@@ -237,28 +239,92 @@ __global__ void __launch_bounds__(kThreads, 2) m3_fwd_umma_kernel(const M3Params
   // 2 lane, 2 lane + 1)
   float thv[8];
   float pa0, pa1, pb0, pb1, pg0, pg1;
+  // from raw projections: the discretisation of step s (the expressions of
+  // the discretisation kernel, each value rounded to bf16 as it stores them)
+  const float dtb = (p.raw && p.dt_bias) ? p.dt_bias[h] : 0.f;
+  float *sDt = reinterpret_cast<float *>(sm + S::dtv);
+  auto raw_coef = [&](int64_t j, float &a, float &bt, float &gm) {
+    const DiscCoef cf = disc_coef(__bfloat162float(static_cast<const bf16 *>(p.dd_dt)[j]), dtb,
+                                  __bfloat162float(static_cast<const bf16 *>(p.dd_a)[j]),
+                                  __bfloat162float(static_cast<const bf16 *>(p.trap)[j]), p.A_floor);
+    a = to_f32(from_f32<bf16>(cf.alpha));
+    bt = to_f32(from_f32<bf16>(disc_beta(cf)));
+    gm = to_f32(from_f32<bf16>(disc_gamma(cf)));
+    return cf.dt;
+  };
+  // the next chunk's per-step values into registers (and, from raw
+  // projections, warp 0's dt of each step into sDt: the chunk's readers of
+  // sDt are past barrier (C), where this is called, so one buffer serves)
   auto load_small = [&](int64_t t0) {
 #pragma unroll
     for (int m = 0; m < 8; ++m) {
       const int64_t t = t0 + 8 * m + ri;
-      thv[m] = (ka < K && t < L) ? __bfloat162float(th_g[((b * L + t) * H + h) * Kt + k0 + ka]) : 0.f;
+      float v = 0.f;
+      if (ka < K && t < L) {
+        if (p.raw)  // the raw angle (shared by the heads); theta = dt x angle once dt is in
+          v = __bfloat162float(static_cast<const bf16 *>(p.angles)[(b * L + t) * Kt + k0 + ka]);
+        else
+          v = __bfloat162float(th_g[((b * L + t) * H + h) * Kt + k0 + ka]);
+      }
+      thv[m] = v;
     }
     pa0 = pa1 = 1.f;
     pb0 = pb1 = pg0 = pg1 = 0.f;
     if (warp == 0) {
       const int64_t s = t0 + 2 * lane;
+      float dt0 = 0.f, dt1 = 0.f;
       if (s < L) {
         const int64_t j = (b * L + s) * H + h;
-        pa0 = __bfloat162float(al_g[j]);
-        pb0 = __bfloat162float(be_g[j]);
-        pg0 = __bfloat162float(ga_g[j]);
+        if (p.raw) {
+          dt0 = raw_coef(j, pa0, pb0, pg0);
+        } else {
+          pa0 = __bfloat162float(al_g[j]);
+          pb0 = __bfloat162float(be_g[j]);
+          pg0 = __bfloat162float(ga_g[j]);
+        }
       }
       if (s + 1 < L) {
         const int64_t j = (b * L + s + 1) * H + h;
-        pa1 = __bfloat162float(al_g[j]);
-        pb1 = __bfloat162float(be_g[j]);
-        pg1 = __bfloat162float(ga_g[j]);
+        if (p.raw) {
+          dt1 = raw_coef(j, pa1, pb1, pg1);
+        } else {
+          pa1 = __bfloat162float(al_g[j]);
+          pb1 = __bfloat162float(be_g[j]);
+          pg1 = __bfloat162float(ga_g[j]);
+        }
       }
+      if (p.raw) {
+        sDt[2 * lane] = dt0;
+        sDt[2 * lane + 1] = dt1;
+      }
+    }
+  };
+  // BCNorm of the chunk's raw B and C rows in place: R = N / 8 lanes per row,
+  // each with a run of 8 states summed in order, the runs' sums combined by an
+  // xor butterfly over the R lanes (the discretisation kernel's order), every
+  // value rounded to bf16 as that kernel stores it
+  auto norm_rows = [&]() {
+    constexpr int R = N / 8;
+    static_assert((2 * kQ * R) % kThreads == 0, "every thread takes part in each butterfly");
+#pragma unroll
+    for (int u = tid; u < 2 * kQ * R; u += kThreads) {
+      const int row = u / R, run = u % R;
+      unsigned char *rowp = sm + (row < kQ ? S::rB : S::rC) + (row % kQ) * S::kRS + run * 16;
+      uint4 w = *reinterpret_cast<const uint4 *>(rowp);
+      uint32_t *wp = reinterpret_cast<uint32_t *>(&w);
+      float v[8];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) unpack_bf16x2(wp[e], v[2 * e], v[2 * e + 1]);
+      float ss = 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) ss = fmaf(v[e], v[e], ss);
+#pragma unroll
+      for (int m = 1; m < R; m <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+      const float rn = rsqrtf(ss / (float)N + p.eps);
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        wp[e] = bf16pair(from_f32<bf16>(v[2 * e] * rn), from_f32<bf16>(v[2 * e + 1] * rn));
+      *reinterpret_cast<uint4 *>(rowp) = w;
     }
   };
   um_issue_raw<P, N, kSlab>(p, sm, b, h, g, 0);
@@ -279,6 +345,13 @@ __global__ void __launch_bounds__(kThreads, 2) m3_fwd_umma_kernel(const M3Params
     cp_async_wait<0>();
     __syncthreads();  // (A) this chunk's raw inputs are in; the last chunk is done
     if (*sErr) break;
+    if (p.raw) {
+      norm_rows();
+      // theta = dt x angle, rounded to bf16 as the discretisation stores it
+#pragma unroll
+      for (int m = 0; m < 8; ++m) thv[m] = to_f32(from_f32<bf16>(sDt[8 * m + ri] * thv[m]));
+      __syncthreads();  // normalised rows in place
+    }
 
     // ---- 1. state and angles entering the chunk; X^T; per-step vectors ----------
     if (p.saved) {

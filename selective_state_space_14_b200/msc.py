@@ -120,6 +120,17 @@ class M3DiscBwdArgs(ctypes.Structure):
                 ("dB_raw", _vp), ("dC_raw", _vp)]
 
 
+class M3RawArgs(ctypes.Structure):
+    _fields_ = [("struct_size", _u32), ("A_floor", ctypes.c_float), ("eps", ctypes.c_float),
+                ("dd_dt", _vp), ("dd_a", _vp), ("trap", _vp), ("angles", _vp), ("dt_bias", _vp),
+                ("B_raw", _vp), ("C_raw", _vp)]
+
+
+class M3RawGrads(ctypes.Structure):
+    _fields_ = [("struct_size", _u32), ("ddd_dt", _vp), ("ddd_a", _vp), ("dtrap", _vp),
+                ("dangles", _vp), ("ddt_bias", _vp), ("dB_raw", _vp), ("dC_raw", _vp)]
+
+
 class ConvFwdArgs(ctypes.Structure):
     _fields_ = [("struct_size", _u32), ("io_dtype", _i32), ("batch", _i64), ("dim", _i64),
                 ("seqlen", _i64), ("width", _i64), ("x", _vp), ("w", _vp), ("bias", _vp),
@@ -142,7 +153,9 @@ EXPORTS = ["msc_last_error", "msc_version", "msc_selective_scan_saved_states_byt
            "msc_causal_conv1d_bwd_workspace_bytes", "msc_causal_conv1d_bwd",
            "msc_selective_scan_conv_fwd", "msc_mamba3_siso_discretize",
            "msc_mamba3_siso_discretize_bwd", "msc_mamba3_siso_disc_state_update",
-           "msc_probe_threads_per_block", "msc_probe_sfu_ex2", "msc_probe_ffma"]
+           "msc_probe_threads_per_block", "msc_probe_sfu_ex2", "msc_probe_ffma",
+           "msc_mamba3_siso_scan_fwd_raw", "msc_mamba3_siso_scan_bwd_raw_workspace_bytes",
+           "msc_mamba3_siso_scan_bwd_raw"]
 
 _lib = None
 
@@ -173,6 +186,11 @@ def lib() -> ctypes.CDLL:
                             [ctypes.POINTER(M3SuArgs), ctypes.POINTER(M3DiscStepArgs), _vp]),
                            ("msc_mamba3_siso_discretize_bwd",
                             [ctypes.POINTER(M3DiscBwdArgs), _vp]),
+                           ("msc_mamba3_siso_scan_fwd_raw",
+                            [ctypes.POINTER(M3FwdArgs), ctypes.POINTER(M3RawArgs), _vp]),
+                           ("msc_mamba3_siso_scan_bwd_raw",
+                            [ctypes.POINTER(M3BwdArgs), ctypes.POINTER(M3RawArgs),
+                             ctypes.POINTER(M3RawGrads), _vp, ctypes.c_size_t, _vp]),
                            ("msc_causal_conv1d_fwd", [ctypes.POINTER(ConvFwdArgs), _vp]),
                            ("msc_causal_conv1d_bwd",
                             [ctypes.POINTER(ConvBwdArgs), _vp, ctypes.c_size_t, _vp])):
@@ -193,6 +211,8 @@ def lib() -> ctypes.CDLL:
         L.msc_causal_conv1d_bwd_workspace_bytes.restype = ctypes.c_size_t
         L.msc_mamba3_siso_scan_bwd_workspace_bytes.argtypes = [_i64] * 7
         L.msc_mamba3_siso_scan_bwd_workspace_bytes.restype = ctypes.c_size_t
+        L.msc_mamba3_siso_scan_bwd_raw_workspace_bytes.argtypes = [_i64] * 7
+        L.msc_mamba3_siso_scan_bwd_raw_workspace_bytes.restype = ctypes.c_size_t
         L.msc_probe_threads_per_block.argtypes = []
         L.msc_probe_threads_per_block.restype = _i64
         L.msc_probe_sfu_ex2.argtypes = [_vp, _i64, _i64, ctypes.POINTER(_i64), _vp]
@@ -512,6 +532,88 @@ def msc_mamba3_siso_scan_bwd(x, B, C, alpha, beta, gamma, theta, saved_states, d
                   _ptr(g["dgamma"]), _ptr(g["dtheta"]), _ptr(g["dD"]), _ptr(g["dh0"]))
     _check(lib().msc_mamba3_siso_scan_bwd(ctypes.byref(a), _ptr(workspace), workspace.numel(),
                                           _stream(stream)))
+    return g
+
+
+def _m3_raw(dd_dt, dd_a, trap, angles, B_raw, C_raw, dt_bias, A_floor, eps):
+    return M3RawArgs(ctypes.sizeof(M3RawArgs), A_floor, eps, _ptr(dd_dt), _ptr(dd_a), _ptr(trap),
+                     _ptr(angles), _ptr(dt_bias), _ptr(B_raw), _ptr(C_raw))
+
+
+def msc_mamba3_siso_scan_fwd_raw(x, dd_dt, dd_a, trap, angles, B_raw, C_raw, dt_bias=None,
+                                 A_floor=1e-4, eps=1e-5, D=None, z=None, h0=None, out=None,
+                                 final_state=None, saved_states=None, want_final_state=True,
+                                 want_saved_states=True, stream=None):
+    """Mamba-3 SISO forward from raw projections (bf16, d_state <= 64):
+    dd_dt, dd_a, trap [B, L, H]; angles [B, L, K]; B_raw, C_raw [B, L, G, N].
+    Returns (out, final_state, saved_states); equals msc_mamba3_siso_discretize
+    followed by msc_mamba3_siso_scan_fwd bit for bit."""
+    Bsz, L, H, P = x.shape
+    G, N = B_raw.shape[2], B_raw.shape[3]
+    K = angles.shape[2] if angles is not None else 0
+    dev = x.device
+    if out is None:
+        out = torch.empty_like(x)
+    if final_state is None and want_final_state:
+        final_state = torch.empty((Bsz, H, P, N), device=dev, dtype=torch.float32)
+    if saved_states is None and want_saved_states:
+        nb = msc_mamba3_siso_saved_states_bytes(Bsz, L, H, P, N)
+        saved_states = torch.empty(max(nb // 4, 4), device=dev, dtype=torch.float32)
+    a = M3FwdArgs(ctypes.sizeof(M3FwdArgs), _io(x), Bsz, L, H, P, N, G, K, _ptr(x), _ptr(z),
+                  None, None, None, None, None, None, _ptr(D), _ptr(h0), _ptr(out),
+                  _ptr(final_state), _ptr(saved_states), None, 0)
+    r = _m3_raw(dd_dt, dd_a, trap, angles, B_raw, C_raw, dt_bias, A_floor, eps)
+    _check(lib().msc_mamba3_siso_scan_fwd_raw(ctypes.byref(a), ctypes.byref(r), _stream(stream)))
+    return out, final_state, saved_states
+
+
+def msc_mamba3_siso_scan_bwd_raw_workspace_bytes(batch, seqlen, nheads, headdim, dstate,
+                                                 ngroups, nangles) -> int:
+    return int(lib().msc_mamba3_siso_scan_bwd_raw_workspace_bytes(
+        batch, seqlen, nheads, headdim, dstate, ngroups, nangles))
+
+
+def msc_mamba3_siso_scan_bwd_raw(x, dd_dt, dd_a, trap, angles, B_raw, C_raw, saved_states, dout,
+                                 dt_bias=None, A_floor=1e-4, eps=1e-5, D=None, z=None, h0=None,
+                                 workspace=None, want_dh0=True, grads=None, stream=None):
+    """Mamba-3 SISO backward from raw projections (bf16, d_state <= 64).
+    Returns dict dx, dz, dD, dh0 and ddd_dt, ddd_a, dtrap, dangles, ddt_bias,
+    dB_raw, dC_raw; equals the scan's backward followed by
+    msc_mamba3_siso_discretize_bwd bit for bit."""
+    Bsz, L, H, P = x.shape
+    G, N = B_raw.shape[2], B_raw.shape[3]
+    K = angles.shape[2] if angles is not None else 0
+    dev = x.device
+    f32 = dict(device=dev, dtype=torch.float32)
+    g = dict(grads or {})
+    defaults = dict(dx=lambda: torch.empty_like(x),
+                    dz=lambda: torch.empty_like(x) if z is not None else None,
+                    dD=lambda: torch.empty((H,), **f32),
+                    dh0=lambda: torch.empty((Bsz, H, P, N), **f32) if want_dh0 else None,
+                    ddd_dt=lambda: torch.empty((Bsz, L, H), **f32),
+                    ddd_a=lambda: torch.empty((Bsz, L, H), **f32),
+                    dtrap=lambda: torch.empty((Bsz, L, H), **f32),
+                    dangles=lambda: torch.empty((Bsz, L, K), **f32) if K > 0 else None,
+                    ddt_bias=lambda: torch.empty((H,), **f32),
+                    dB_raw=lambda: torch.empty((Bsz, L, G, N), **f32),
+                    dC_raw=lambda: torch.empty((Bsz, L, G, N), **f32))
+    for k, mk in defaults.items():
+        if k not in g:
+            g[k] = mk()
+    need = msc_mamba3_siso_scan_bwd_raw_workspace_bytes(Bsz, L, H, P, N, G, K)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), device=dev, dtype=torch.uint8)
+    a = M3BwdArgs(ctypes.sizeof(M3BwdArgs), _io(x), Bsz, L, H, P, N, G, K, _ptr(x), _ptr(z),
+                  None, None, None, None, None, None, _ptr(D), _ptr(h0), _ptr(saved_states),
+                  _ptr(dout), _ptr(g["dx"]), _ptr(g["dz"]), None, None, None, None, None, None,
+                  _ptr(g["dD"]), _ptr(g["dh0"]))
+    r = _m3_raw(dd_dt, dd_a, trap, angles, B_raw, C_raw, dt_bias, A_floor, eps)
+    gr = M3RawGrads(ctypes.sizeof(M3RawGrads), _ptr(g["ddd_dt"]), _ptr(g["ddd_a"]),
+                    _ptr(g["dtrap"]), _ptr(g["dangles"]), _ptr(g["ddt_bias"]), _ptr(g["dB_raw"]),
+                    _ptr(g["dC_raw"]))
+    _check(lib().msc_mamba3_siso_scan_bwd_raw(ctypes.byref(a), ctypes.byref(r), ctypes.byref(gr),
+                                              _ptr(workspace), workspace.numel(),
+                                              _stream(stream)))
     return g
 
 

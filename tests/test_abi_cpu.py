@@ -402,3 +402,88 @@ def test_fused_decode_checks_raw_args():
     assert fn(ctypes.byref(a), ctypes.byref(r), None) == INVALID and "eps" in _err()
     r.eps, r.struct_size = 1e-5, 4
     assert fn(ctypes.byref(a), ctypes.byref(r), None) == INVALID and "struct_size" in _err()
+
+
+def _m3_raw_scan_args(**kw):
+    a = msc.M3FwdArgs()
+    a.struct_size = ctypes.sizeof(msc.M3FwdArgs)
+    a.io_dtype, a.batch, a.seqlen, a.nheads, a.headdim, a.dstate, a.ngroups, a.nangles = (
+        msc.MSC_BF16, 2, 128, 4, 64, 64, 1, 32)
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: the checks fail first
+    a.x = a.out = fake
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+def _m3_raw(**kw):
+    r = msc.M3RawArgs()
+    r.struct_size = ctypes.sizeof(msc.M3RawArgs)
+    r.A_floor, r.eps = 1e-4, 1e-5
+    fake = ctypes.c_void_p(1 << 20)
+    r.dd_dt = r.dd_a = r.trap = r.angles = r.B_raw = r.C_raw = fake
+    for k, v in kw.items():
+        setattr(r, k, v)
+    return r
+
+
+@pytest.mark.parametrize("field,value,word", [
+    ("io_dtype", msc.MSC_F32, "bf16"),
+    ("io_dtype", msc.MSC_F16, "bf16"),
+    ("dstate", 128, "dstate"),   # a shape the plain scan takes as slabs
+    ("dstate", 48, "dstate"),
+])
+def test_fused_raw_scan_rejects_what_it_does_not_fuse(field, value, word):
+    """The scan from raw projections takes bf16 io and d_state 16, 32 or 64; other
+    shapes are MSC_ERR_UNSUPPORTED (the two-call chain serves them)."""
+    a = _m3_raw_scan_args(**{field: value})
+    st = msc.lib().msc_mamba3_siso_scan_fwd_raw(ctypes.byref(a), ctypes.byref(_m3_raw()), None)
+    assert st == UNSUPPORTED and word in _err()
+
+
+def test_fused_raw_scan_checks_raw_args():
+    fn = msc.lib().msc_mamba3_siso_scan_fwd_raw
+    a = _m3_raw_scan_args()
+    assert fn(ctypes.byref(a), None, None) == INVALID and "raw is NULL" in _err()
+    r = _m3_raw(trap=None)
+    assert fn(ctypes.byref(a), ctypes.byref(r), None) == INVALID and "trap is NULL" in _err()
+    r = _m3_raw(C_raw=None)
+    assert fn(ctypes.byref(a), ctypes.byref(r), None) == INVALID and "C_raw is NULL" in _err()
+    r = _m3_raw(angles=ctypes.c_void_p((1 << 20) + 2))
+    assert fn(ctypes.byref(a), ctypes.byref(r), None) == ALIGNMENT and "angles" in _err()
+    r = _m3_raw(eps=-1.0)
+    assert fn(ctypes.byref(a), ctypes.byref(r), None) == INVALID and "eps" in _err()
+    r = _m3_raw(struct_size=4)
+    assert fn(ctypes.byref(a), ctypes.byref(r), None) == INVALID and "struct_size" in _err()
+    # the scan struct is checked first
+    a.struct_size = 4
+    assert fn(ctypes.byref(a), ctypes.byref(_m3_raw()), None) == INVALID
+    assert "struct_size" in _err()
+
+
+def test_fused_raw_bwd_workspace_and_grads():
+    """The backward from raw projections needs the scan's workspace plus room for
+    the scan's gradients of the derived inputs, and its raw-gradient struct."""
+    B, L, H, P, N, G, K = 2, 128, 4, 64, 64, 1, 32
+    scan = msc.msc_mamba3_siso_scan_bwd_workspace_bytes(B, L, H, P, N, G, K)
+    need = msc.msc_mamba3_siso_scan_bwd_raw_workspace_bytes(B, L, H, P, N, G, K)
+    derived = 4 * B * L * (3 * H + H * K + 2 * G * N)
+    assert need >= scan + derived
+    assert msc.msc_mamba3_siso_scan_bwd_raw_workspace_bytes(B, L, H, P, N, 0, K) == 0
+    fake = ctypes.c_void_p(1 << 20)
+    a = msc.M3BwdArgs()
+    a.struct_size = ctypes.sizeof(msc.M3BwdArgs)
+    a.io_dtype, a.batch, a.seqlen, a.nheads, a.headdim, a.dstate, a.ngroups, a.nangles = (
+        msc.MSC_BF16, B, L, H, P, N, G, K)
+    a.x = a.saved_states = a.dout = a.dx = fake
+    fn = msc.lib().msc_mamba3_siso_scan_bwd_raw
+    r = _m3_raw()
+    assert fn(ctypes.byref(a), ctypes.byref(r), None, fake, need, None) == INVALID
+    assert "grads is NULL" in _err()
+    g = msc.M3RawGrads()
+    g.struct_size = ctypes.sizeof(msc.M3RawGrads)
+    g.ddd_dt = g.ddd_a = g.dtrap = g.dangles = g.dB_raw = g.dC_raw = fake
+    assert fn(ctypes.byref(a), ctypes.byref(r), ctypes.byref(g), fake, need - 16, None) == WORKSPACE
+    g.dangles = None
+    assert fn(ctypes.byref(a), ctypes.byref(r), ctypes.byref(g), fake, need, None) == INVALID
+    assert "dangles is NULL" in _err()

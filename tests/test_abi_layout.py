@@ -17,13 +17,15 @@ PAIRS = [("msc_ss_fwd_args", msc.SsFwdArgs), ("msc_ss_conv_args", msc.SsConvArgs
          ("msc_m3_fwd_args", msc.M3FwdArgs), ("msc_m3_bwd_args", msc.M3BwdArgs),
          ("msc_m3_su_args", msc.M3SuArgs), ("msc_m3_disc_step_args", msc.M3DiscStepArgs),
          ("msc_m3_disc_args", msc.M3DiscArgs), ("msc_m3_disc_bwd_args", msc.M3DiscBwdArgs),
-         ("msc_conv_fwd_args", msc.ConvFwdArgs), ("msc_conv_bwd_args", msc.ConvBwdArgs)]
+         ("msc_conv_fwd_args", msc.ConvFwdArgs), ("msc_conv_bwd_args", msc.ConvBwdArgs),
+         ("msc_m3_raw_args", msc.M3RawArgs), ("msc_m3_raw_grads", msc.M3RawGrads)]
 
 
 def test_every_header_struct_is_bound():
     import re
     text = open(os.path.join(ROOT, "include", "msc.h")).read()
-    assert sorted(re.findall(r"^\} (msc_\w+_args);", text, flags=re.M)) == sorted(c for c, _ in PAIRS)
+    assert sorted(re.findall(r"^\} (msc_\w+_(?:args|grads));", text, flags=re.M)) == \
+        sorted(c for c, _ in PAIRS)
 
 
 def test_struct_layouts_match_the_header(tmp_path):

@@ -279,3 +279,105 @@ def test_fused_decode_vs_oracle(msc):
         torch.cuda.synchronize()
         assert_close("out", host(o), o_ref, TOL["bf16"], FAMILY)
     assert_close("state", host(cg[0]), cr[0], TOL["bf16"], FAMILY)
+
+
+# --------------------------------------------------------------------------
+# The scan from raw projections (discretisation and BCNorm fused into the
+# scan's kernels): bit for bit the two-call chain, and so the oracle's chain
+# --------------------------------------------------------------------------
+SCAN_OUT = ("dx", "dz", "dD", "dh0")
+
+
+def _chain_and_fused(msc, q, bias=True, h0=True, z=True, D=True):
+    """Run discretise -> scan forward -> scan backward -> discretise backward and
+    the two fused entry points on the same inputs."""
+    s = q.scan
+    d = {k: dev(v) for k, v in _raw(q).items()}
+    if s.nangles == 0:
+        d["angles"] = None
+    dtb = dev(q.dt_bias) if bias else None
+    kw = dict(dt_bias=dtb, A_floor=q.A_floor, eps=q.eps)
+    com = dict(x=dev(s.x), D=dev(s.D) if D else None, z=dev(s.z) if z else None,
+               h0=dev(s.h0) if h0 else None)
+    dout = dev(s.dout)
+    o = msc.msc_mamba3_siso_discretize(**d, **kw)
+    der = dict(B=o["B"], C=o["C"], alpha=o["alpha"], beta=o["beta"], gamma=o["gamma"],
+               theta=o["theta"])
+    out, fs, saved = msc.msc_mamba3_siso_scan_fwd(**com, **der)
+    gs = msc.msc_mamba3_siso_scan_bwd(**com, **der, saved_states=saved, dout=dout)
+    g = msc.msc_mamba3_siso_discretize_bwd(**d, dalpha=gs["dalpha"], dbeta=gs["dbeta"],
+                                           dgamma=gs["dgamma"], dtheta=gs["dtheta"],
+                                           dB=gs["dB"], dC=gs["dC"], **kw)
+    chain = dict(out=out, final_state=fs, saved=saved, **{k: gs[k] for k in SCAN_OUT}, **g)
+    out_r, fs_r, saved_r = msc.msc_mamba3_siso_scan_fwd_raw(**com, **d, **kw)
+    gr = msc.msc_mamba3_siso_scan_bwd_raw(**com, **d, **kw, saved_states=saved_r, dout=dout)
+    fused = dict(out=out_r, final_state=fs_r, saved=saved_r, **gr)
+    torch.cuda.synchronize()
+    return chain, fused
+
+
+def _assert_bit_equal(chain, fused, keys):
+    for k in keys:
+        a, b = chain[k], fused[k]
+        if a is None or b is None:  # absent (no angles, no h0): absent or empty on both sides
+            assert all(v is None or v.numel() == 0 for v in (a, b)), k
+            continue
+        assert torch.equal(a, b), (k, (a.float() - b.float()).abs().max().item())
+
+
+FUSED_CASES = [
+    # (B, L, H, P, N, G, K, bias, h0, z, D)
+    (2, 130, 4, 64, 64, 1, 32, True, True, True, True),   # ragged last chunk
+    (1, 200, 6, 32, 32, 2, 16, False, False, True, False),
+    (2, 64, 4, 16, 16, 1, 0, True, True, False, True),    # no angles, one chunk
+    (1, 1, 2, 64, 64, 1, 8, True, False, True, True),     # one step
+    (1, 257, 8, 64, 16, 4, 8, True, True, True, True),    # four groups
+]
+
+
+@pytest.mark.parametrize("case", FUSED_CASES,
+                         ids=[f"B{c[0]}L{c[1]}H{c[2]}P{c[3]}N{c[4]}G{c[5]}K{c[6]}"
+                              for c in FUSED_CASES])
+def test_fused_raw_equals_the_chain(msc, case):
+    Bsz, L, H, P, N, G, K, bias, h0, z, D = case
+    q = W.m3disc_problem(Bsz, L, H, P, N, ngroups=G, nangles=K, io="bf16", seed=L + 3 * H,
+                         with_h0=h0)
+    chain, fused = _chain_and_fused(msc, q, bias=bias, h0=h0, z=z, D=D)
+    _assert_bit_equal(chain, fused, ("out", "final_state", "saved") + SCAN_OUT + DISC_GRADS)
+
+
+def test_fused_raw_against_the_oracle(msc):
+    """The fused entry points against the oracle's chain directly (the scan taking
+    the discretised values as bf16 stores them)."""
+    q = W.m3disc_problem(2, 130, 4, 64, 64, nangles=32, io="bf16", seed=11, with_h0=True)
+    _, fused = _chain_and_fused(msc, q)
+    s = q.scan
+    ra = _oracle_raw(q)
+    disc = oracle.m3_discretize(**ra, A_floor=q.A_floor, eps=q.eps)
+    stored = {k: W.store(v.astype(np.float32), "bf16").as_f64() for k, v in disc.items()}
+    sa = dict(x=s.x.as_f64(), B=stored["B"], C=stored["C"], alpha=stored["alpha"],
+              beta=stored["beta"], gamma=stored["gamma"], theta=stored["theta"],
+              D=np.asarray(s.D, np.float64), z=s.z.as_f64(), h0=np.asarray(s.h0, np.float64))
+    ref = oracle.m3_fwd(**sa)
+    refs = oracle.m3_bwd(**sa, dout=s.dout.as_f64())
+    refg = oracle.m3_discretize_bwd(**ra, dalpha=refs["dalpha"], dbeta=refs["dbeta"],
+                                    dgamma=refs["dgamma"], dtheta=refs["dtheta"], dB=refs["dB"],
+                                    dC=refs["dC"], A_floor=q.A_floor, eps=q.eps)
+    assert_close("out", host(fused["out"]), ref["out"], TOL["bf16"], FAMILY)
+    assert_close("final_state", host(fused["final_state"]), ref["final_state"], TOL["bf16"],
+                 FAMILY)
+    for k in ("dx", "dz"):
+        assert_close(k, host(fused[k]), refs[k], TOL["bf16"], FAMILY)
+    for k in ("dD", "dh0"):
+        assert_close(k, host(fused[k]), refs[k], TOL["bf16"], FAMILY)
+    for k in DISC_GRADS:
+        assert_close(k, host(fused[k]), refg[k], TOL["bf16"], FAMILY)
+
+
+def test_fused_raw_full_size_equals_the_chain(msc):
+    """At the full training shape (B8 L2048 H24 P64 N64 K32, bf16), the launch the
+    bench times: every output bit for bit the two-call chain's, whose own parity
+    the scan's full-size tests establish."""
+    q = W.make("m3disc_bf16_b8_h24_p64_n64_k32_l2048")
+    chain, fused = _chain_and_fused(msc, q, h0=False)
+    _assert_bit_equal(chain, fused, ("out", "final_state", "saved") + SCAN_OUT + DISC_GRADS)
