@@ -278,62 +278,9 @@ __device__ __forceinline__ void cp_async_wait() {
 }
 
 // ---------------------------------------------------------------------------
-// scans of the linear-recurrence monoid over the kW lanes of a lane group
-// (kW = 8: four independent 8-lane groups per warp), on packed pairs
+// warp scan of the linear-recurrence monoid
 //   (p, h) o (p', h') = (p p', p' h + h')   -- "earlier o later"
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ float2 shfl_up2(float2 v, int off, int width) {
-  return make_float2(__shfl_up_sync(0xffffffffu, v.x, off, width),
-                     __shfl_up_sync(0xffffffffu, v.y, off, width));
-}
-__device__ __forceinline__ float2 shfl_down2(float2 v, int off, int width) {
-  return make_float2(__shfl_down_sync(0xffffffffu, v.x, off, width),
-                     __shfl_down_sync(0xffffffffu, v.y, off, width));
-}
-__device__ __forceinline__ float2 shfl2(float2 v, int src, int width) {
-  return make_float2(__shfl_sync(0xffffffffu, v.x, src, width),
-                     __shfl_sync(0xffffffffu, v.y, src, width));
-}
-
-// Exclusive prefix within the group (lane order = time order): (pe, he) is the
-// composition of all earlier lanes of the group, identity for its first lane.
-template <int kW>
-__device__ __forceinline__ void group_scan_fwd2(float2 p, float2 h, int j, float2 &pe, float2 &he) {
-#pragma unroll
-  for (int off = 1; off < kW; off <<= 1) {
-    const float2 pu = shfl_up2(p, off, kW);
-    const float2 hu = shfl_up2(h, off, kW);
-    if (j >= off) {
-      h = fma2(p, hu, h);
-      p = mul2(p, pu);
-    }
-  }
-  pe = shfl_up2(p, 1, kW);
-  he = shfl_up2(h, 1, kW);
-  if (j == 0) { pe = splat2(1.f); he = splat2(0.f); }
-}
-
-// Suffix version for the adjoint: a lane maps the carry entering from its
-// right, mu_in, to p * mu_in + m; (ps, ms) composes all later lanes.
-template <int kW>
-__device__ __forceinline__ void group_scan_rev2(float2 p, float2 m, int j, float2 &ps, float2 &ms) {
-#pragma unroll
-  for (int off = 1; off < kW; off <<= 1) {
-    const float2 pd = shfl_down2(p, off, kW);
-    const float2 md = shfl_down2(m, off, kW);
-    if (j + off < kW) {
-      m = fma2(p, md, m);
-      p = mul2(p, pd);
-    }
-  }
-  ps = shfl_down2(p, 1, kW);
-  ms = shfl_down2(m, 1, kW);
-  if (j == kW - 1) { ps = splat2(1.f); ms = splat2(0.f); }
-}
-
-// ---------------------------------------------------------------------------
-// warp scans of the linear-recurrence monoid
-//   (p, h) o (p', h') = (p p', p' h + h')   -- "earlier o later"
+// (the combine of the Mamba-1 forward's time segments)
 // ---------------------------------------------------------------------------
 // Inclusive prefix over lanes 0..lane (lane order = time order); returns the
 // exclusive prefix in (pe, he) -- identity (1, 0) for lane 0.
@@ -351,25 +298,6 @@ __device__ __forceinline__ void warp_scan_fwd(float p, float h, float &pe, float
   pe = __shfl_up_sync(0xffffffffu, p, 1);
   he = __shfl_up_sync(0xffffffffu, h, 1);
   if (lane == 0) { pe = 1.f; he = 0.f; }
-}
-
-// Suffix (reverse-time) version for the adjoint: a lane's transform maps the
-// carry entering from the right, mu_in, to mu_out = p * mu_in + m.  Returns
-// the composition of all lanes strictly to the right of this lane.
-__device__ __forceinline__ void warp_scan_rev(float p, float m, float &ps, float &ms) {
-  const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    float pd = __shfl_down_sync(0xffffffffu, p, off);
-    float md = __shfl_down_sync(0xffffffffu, m, off);
-    if (lane + off < 32) {
-      m = fmaf(p, md, m);
-      p = p * pd;
-    }
-  }
-  ps = __shfl_down_sync(0xffffffffu, p, 1);
-  ms = __shfl_down_sync(0xffffffffu, m, 1);
-  if (lane == 31) { ps = 1.f; ms = 0.f; }
 }
 
 }  // namespace msc

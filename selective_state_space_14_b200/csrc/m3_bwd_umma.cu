@@ -75,7 +75,7 @@ constexpr int kParts = 3;         // bf16 parts of an f32 operand
 constexpr int kMat = kParts * kPl;  // bytes of the planes of one f32 operand
 
 // ---------------------------------------------------------------------------
-// two-part operand stores (core-matrix layout of umma.cuh)
+// kParts-part operand stores (core-matrix layout of umma.cuh)
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t bits2(__nv_bfloat162 v) {
   return *reinterpret_cast<const uint32_t *>(&v);
@@ -183,15 +183,21 @@ struct Vec {
                        rowb = 1352 /* [8][64] per-run parts of Ct.Bt_prev */,
                        rowx = 1864 /* [8][64] per-run parts of g.x_prev */,
                        nrm = 2376 /* [2][8][64] per-run squares of the raw B, C rows */,
-                       dt = 3400 /* [64] dt (from raw projections) */, total = 3464;
+                       dt = 3400 /* [64] dt (from raw projections) */,
+                       rsc = 3464 /* [2][64] BCNorm scales of the raw B, C rows */, total = 3592;
 };
+
+// Row stride (floats) of the angle table tPhi [t][k]: padded so that the
+// threads of a warp that hold steps 2 lane, 2 lane + 1 (the angle scans) or
+// eight consecutive steps (the rotations) fall on different banks.
+constexpr int kPhS = 33;
 
 struct PrepSmem {
   static constexpr int pC = 0, pB = pC + kMat, pS = pB + kMat, pGd = pS + kMat,
                        pW = pGd + kMat, pX = pW + kMat;
   static constexpr int tD = pX + kPl;                // f32 [64][65]: d(t,-1), d(t,0..63)
-  static constexpr int tPhi = tD + 64 * 65 * 4;      // f32 [64][32] cumulative angles
-  static constexpr int vec = tPhi + 64 * 32 * 4;     // Vec
+  static constexpr int tPhi = tD + 64 * 65 * 4;      // f32 [64][kPhS] cumulative angles
+  static constexpr int vec = tPhi + 64 * kPhS * 4;   // Vec
   static constexpr int misc = vec + Vec::total * 4;  // tmem slot, mbarrier, error flag
   static constexpr int total = misc + 32;
 };
@@ -201,8 +207,8 @@ struct GradSmem {
                        pS = pX + kPl /* S_in, then W */, pU = pS + kMat, pZ = pU + kMat;
   static constexpr int tD = pZ + kMat;                // f32 [64][65]
   static constexpr int tM = tD + 64 * 65 * 4;         // f32 [64][65]: (Ct.Bt)(g.x)
-  static constexpr int tPhi = tM + 64 * 65 * 4;       // f32 [64][32] angles, then dphi
-  static constexpr int vec = tPhi + 64 * 32 * 4;
+  static constexpr int tPhi = tM + 64 * 65 * 4;       // f32 [64][kPhS] angles, then dphi
+  static constexpr int vec = tPhi + 64 * kPhS * 4;
   static constexpr int misc = vec + Vec::total * 4;
   static constexpr int total = misc + 32;
   static_assert(total <= 232448, "one CTA's shared memory");
@@ -258,6 +264,10 @@ struct Loads {
   bf16 al, be, ga, prev;
   bool in_step;
   float phist, bias;
+  // from raw projections: the step's alpha, beta, gamma (rounded to bf16 as
+  // the discretisation stores them) and dt, derived by coef() while the
+  // current unit waits on its tensor cores
+  float ca, cbt, cgm, cdt;
 
   __device__ __forceinline__ void issue(const M3Params &p, const Chunk &c, const float *sin,
                                         const float *usrc) {
@@ -336,11 +346,25 @@ struct Loads {
                         (c.b * p.H + c.h) * c.nc * (c.ldN / 2);
       phist = ps[c.ch * (c.ldN / 2) + c.k0 + tid];
     }
+    ca = 1.f;
+    cbt = cgm = cdt = 0.f;
     prev = nil;
     if (c.t0 > 0 && tid < P + N) {
       prev = tid < P ? x[((c.b * p.L + c.t0 - 1) * p.H + c.h) * P + tid]
                      : Bm[((c.b * p.L + c.t0 - 1) * p.G + c.g) * c.ldN + c.n0 + tid - P];
     }
+  }
+
+  // the discretisation of this thread's step (threads 0 .. Q; padded steps
+  // keep alpha = 1, beta = gamma = 0), once the issued loads have landed
+  __device__ __forceinline__ void coef(const M3Params &p) {
+    if (!p.raw || threadIdx.x > kQ || !in_step) return;
+    const DiscCoef cf = disc_coef(__bfloat162float(al), bias, __bfloat162float(be),
+                                  __bfloat162float(ga), p.A_floor);
+    ca = to_f32(from_f32<bf16>(cf.alpha));
+    cbt = to_f32(from_f32<bf16>(disc_beta(cf)));
+    cgm = to_f32(from_f32<bf16>(disc_gamma(cf)));
+    cdt = cf.dt;
   }
 };
 
@@ -352,23 +376,12 @@ __device__ __forceinline__ void stage_small(const M3Params &p, const Chunk &c, c
                                             float *sv, float *tPhi, int P, int N) {
   const int tid = threadIdx.x;
   if (tid <= kQ) {
-    if (p.raw) {
-      // the discretisation, rounded to bf16 as the discretisation kernel
-      // stores it (padded steps keep alpha = 1, beta = gamma = 0)
-      float a = 1.f, bt = 0.f, gm = 0.f, dt = 0.f;
-      if (ld.in_step) {
-        const DiscCoef cf = disc_coef(__bfloat162float(ld.al), ld.bias, __bfloat162float(ld.be),
-                                      __bfloat162float(ld.ga), p.A_floor);
-        a = to_f32(from_f32<bf16>(cf.alpha));
-        bt = to_f32(from_f32<bf16>(disc_beta(cf)));
-        gm = to_f32(from_f32<bf16>(disc_gamma(cf)));
-        dt = cf.dt;
-      }
-      sv[Vec::al + tid] = a;
-      sv[Vec::be + tid] = bt;
+    if (p.raw) {  // the discretisation, derived ahead by ld.coef()
+      sv[Vec::al + tid] = ld.ca;
+      sv[Vec::be + tid] = ld.cbt;
       if (tid < kQ) {
-        sv[Vec::ga + tid] = gm;
-        sv[Vec::dt + tid] = dt;
+        sv[Vec::ga + tid] = ld.cgm;
+        sv[Vec::dt + tid] = ld.cdt;
       }
     } else {
       sv[Vec::al + tid] = __bfloat162float(ld.al);
@@ -377,7 +390,10 @@ __device__ __forceinline__ void stage_small(const M3Params &p, const Chunk &c, c
     }
   }
 #pragma unroll
-  for (int q = 0; q < LD::kTH; ++q) tPhi[tid + q * kThreads] = __bfloat162float(ld.th[q]);
+  for (int q = 0; q < LD::kTH; ++q) {
+    const int i = tid + q * kThreads;
+    tPhi[(i >> 5) * kPhS + (i & 31)] = __bfloat162float(ld.th[q]);
+  }
   if (tid < 32) sv[Vec::phist + tid] = ld.phist;
   if (tid < P) sv[Vec::xprev + tid] = __bfloat162float(ld.prev);
   else if (tid < P + N) sv[Vec::bprev + tid - P] = __bfloat162float(ld.prev);
@@ -401,6 +417,14 @@ __device__ __forceinline__ void stage_decays(const M3Params &p, const Chunk &c, 
                                              float *tPhi, float *tD) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int t0 = 2 * lane, t1 = t0 + 1;
+  if (p.raw && tid >= kThreads - 2 * kQ) {
+    // BCNorm's scale of raw row r (B rows 0 .. Q-1, then C): the runs' sums of
+    // squares combined in the order of an xor butterfly
+    const int r = tid - (kThreads - 2 * kQ), R = (int)p.N / 8;
+    float part[8];
+    for (int q = 0; q < R; ++q) part[q] = sv[Vec::nrm + (r / kQ) * 512 + q * 64 + r % kQ];
+    sv[Vec::rsc + r] = rsqrtf(tree_sum(part, R) / (float)p.N + p.eps);
+  }
   if (p.raw && warp == 0 && c.t0 > 0) {
     // B_prev is a raw row: normalised as BCNorm would -- lane r < N / 8 sums
     // run r of 8 states in order, then an xor butterfly over the runs (the
@@ -423,11 +447,11 @@ __device__ __forceinline__ void stage_decays(const M3Params &p, const Chunk &c, 
   }
   __syncwarp();
   for (int k = warp; k < c.K; k += kThreads / 32) {
+    float a0 = tPhi[t0 * kPhS + k], a1 = tPhi[t1 * kPhS + k];
     if (p.raw) {  // theta = dt x angle, rounded to bf16 (this thread's two steps)
-      tPhi[t0 * 32 + k] = to_f32(from_f32<bf16>(sv[Vec::dt + t0] * tPhi[t0 * 32 + k]));
-      tPhi[t1 * 32 + k] = to_f32(from_f32<bf16>(sv[Vec::dt + t1] * tPhi[t1 * 32 + k]));
+      a0 = to_f32(from_f32<bf16>(sv[Vec::dt + t0] * a0));
+      a1 = to_f32(from_f32<bf16>(sv[Vec::dt + t1] * a1));
     }
-    const float a0 = tPhi[t0 * 32 + k], a1 = tPhi[t1 * 32 + k];
     float incl = a0 + a1;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -437,8 +461,8 @@ __device__ __forceinline__ void stage_decays(const M3Params &p, const Chunk &c, 
     float excl = __shfl_up_sync(0xffffffffu, incl, 1);
     if (lane == 0) excl = 0.f;
     const float st = sv[Vec::phist + k];
-    tPhi[t0 * 32 + k] = st + (excl + a0);
-    tPhi[t1 * 32 + k] = st + incl;
+    tPhi[t0 * kPhS + k] = st + (excl + a0);
+    tPhi[t1 * kPhS + k] = st + incl;
   }
   if (tid < c.K) {
     float sn, cs;
@@ -486,8 +510,8 @@ __device__ __forceinline__ float cw(const float *tD, const float *sv, int t, int
 
 // Phase 1, from raw projections: BCNorm's sum of squares of each run of 8
 // states of the chunk's raw B and C rows (sequential over its 8), into nrm
-// [run][t]; phase 3 combines the runs of a row in the order of an xor
-// butterfly, as the discretisation kernel does.
+// [run][t]; phase 2 combines the runs of a row in the order of an xor
+// butterfly, as the discretisation kernel does, into the row's scale.
 template <int N, class LD>
 __device__ __forceinline__ void stage_norm_sums(const LD &ld, float *sv) {
   constexpr int kR = N / 8;
@@ -532,15 +556,8 @@ __device__ __forceinline__ void stage_bc(const M3Params &p, const LD &ld, const 
     unpack_bf16x2(ld.bb[k].z, bv[4], bv[5]); unpack_bf16x2(ld.bb[k].w, bv[6], bv[7]);
     unpack_bf16x2(ld.cc[k].x, cv[0], cv[1]); unpack_bf16x2(ld.cc[k].y, cv[2], cv[3]);
     unpack_bf16x2(ld.cc[k].z, cv[4], cv[5]); unpack_bf16x2(ld.cc[k].w, cv[6], cv[7]);
-    if (p.raw) {
-      float pb[kR], pc[kR];
-#pragma unroll
-      for (int q = 0; q < kR; ++q) {
-        pb[q] = sv[Vec::nrm + q * 64 + t];
-        pc[q] = sv[Vec::nrm + 512 + q * 64 + t];
-      }
-      const float rb = rsqrtf(tree_sum(pb, kR) / (float)N + p.eps);
-      const float rc = rsqrtf(tree_sum(pc, kR) / (float)N + p.eps);
+    if (p.raw) {  // BCNorm, the row scales from phase 2
+      const float rb = sv[Vec::rsc + t], rc = sv[Vec::rsc + kQ + t];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         bv[e] = to_f32(from_f32<bf16>(bv[e] * rb));
@@ -553,7 +570,7 @@ __device__ __forceinline__ void stage_bc(const M3Params &p, const LD &ld, const 
       const int kk = r * 4 + q;
       if (kk < c.K) {
         float sn, cs;
-        sincos_reduced(tPhi[t * 32 + kk], sn, cs);
+        sincos_reduced(tPhi[t * kPhS + kk], sn, cs);
         const float b0 = bv[2 * q], b1 = bv[2 * q + 1], c0 = cv[2 * q], c1 = cv[2 * q + 1];
         bv[2 * q] = cs * b0 - sn * b1;
         bv[2 * q + 1] = sn * b0 + cs * b1;
@@ -725,6 +742,7 @@ __global__ void __launch_bounds__(kThreads, 1) m3b_prep_kernel(const M3Params p,
   if ((int64_t)blockIdx.x < n_units) {
     const Chunk c0 = chunk_of(p, P, blockIdx.x);
     ld.issue(p, c0, sin_of(c0), nullptr);
+    ld.coef(p);
   }
   umma::fence_before();
   __syncthreads();
@@ -802,6 +820,7 @@ __global__ void __launch_bounds__(kThreads, 1) m3b_prep_kernel(const M3Params p,
     product<P, true>(tmem, 192, base + S::pW, kParts, 64, base + S::pX, 1, P, 64, false);  // W X
     umma::commit(mbar);
   }
+  ld.coef(p);  // the next unit's discretisation while W X runs
   if (!umma::mbar_wait(mbar, 1)) *sErr = 1;
   umma::fence_after();
   // ---- y and dz ----------------------------------------------------------------------
@@ -949,6 +968,7 @@ __global__ void __launch_bounds__(kThreads, 1) m3b_grad_kernel(const M3Params p,
   if ((int64_t)blockIdx.x < n_units) {
     const Chunk c0 = chunk_of(p, P, blockIdx.x);
     ld.issue(p, c0, p.saved_in + off_of(c0), vu + off_of(c0));
+    ld.coef(p);
   }
   umma::fence_before();
   __syncthreads();
@@ -1137,6 +1157,7 @@ __global__ void __launch_bounds__(kThreads, 1) m3b_grad_kernel(const M3Params p,
       sv[Vec::da + s] = v;
     }
   }
+  ld.coef(p);  // the next unit's discretisation while round 2 may still run
   if (!umma::mbar_wait(mbar, 1)) *sErr = 1;
   umma::fence_after();
   __syncthreads();
@@ -1196,7 +1217,7 @@ __global__ void __launch_bounds__(kThreads, 1) m3b_grad_kernel(const M3Params p,
         float rb0 = db0, rb1 = db1, rc0 = dc0, rc1 = dc1, dphi = 0.f;
         if (kk < c.K) {
           float sn, cs;
-          sincos_reduced(tPhi[t * 32 + kk], sn, cs);
+          sincos_reduced(tPhi[t * kPhS + kk], sn, cs);
           rb0 = cs * db0 + sn * db1;
           rb1 = -sn * db0 + cs * db1;
           rc0 = cs * dc0 + sn * dc1;
@@ -1210,7 +1231,7 @@ __global__ void __launch_bounds__(kThreads, 1) m3b_grad_kernel(const M3Params p,
           *reinterpret_cast<float2 *>(ws_dB + j) = make_float2(rb0, rb1);
           *reinterpret_cast<float2 *>(ws_dC + j) = make_float2(rc0, rc1);
         }
-        if (kk < c.K) tPhi[t * 32 + kk] = dphi;  // this thread alone reads and writes it
+        if (kk < c.K) tPhi[t * kPhS + kk] = dphi;  // this thread alone reads and writes it
       }
     }
   }
@@ -1222,7 +1243,7 @@ __global__ void __launch_bounds__(kThreads, 1) m3b_grad_kernel(const M3Params p,
     // ...; lane l holds steps 2l, 2l + 1 (steps past Qc carry zero)
     const int t0 = 2 * lane, t1 = t0 + 1;
     for (int k = warp; k < c.K; k += 2) {
-      const float a0 = tPhi[t0 * 32 + k], a1 = tPhi[t1 * 32 + k];
+      const float a0 = tPhi[t0 * kPhS + k], a1 = tPhi[t1 * kPhS + k];
       float incl = a0 + a1;  // suffix sums: lanes >= l
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
