@@ -363,8 +363,11 @@ class M3DiscStep:
         # the same step through the fused entry points (the derived inputs are
         # made inside the scan's kernels and never stored)
         self.c = dict(x=self.a["x"], D=self.a["D"], z=self.a["z"], h0=None)
-        self.out_r, _, self.saved_r = msc.msc_mamba3_siso_scan_fwd_raw(**self.c, **self.raw,
-                                                                       **self.kw)
+        self.ws_f = torch.empty(max(msc.msc_mamba3_siso_scan_fwd_raw_workspace_bytes(
+            s.batch, s.seqlen, s.nheads, s.headdim, s.dstate, s.ngroups, s.nangles), 16),
+            device="cuda", dtype=torch.uint8)
+        self.out_r, _, self.saved_r = msc.msc_mamba3_siso_scan_fwd_raw(
+            **self.c, **self.raw, **self.kw, workspace=self.ws_f)
         self.ws_r = torch.empty(max(msc.msc_mamba3_siso_scan_bwd_raw_workspace_bytes(
             s.batch, s.seqlen, s.nheads, s.headdim, s.dstate, s.ngroups, s.nangles), 16),
             device="cuda", dtype=torch.uint8)
@@ -373,7 +376,7 @@ class M3DiscStep:
 
     def fused_fwd(self):
         self.msc.msc_mamba3_siso_scan_fwd_raw(**self.c, **self.raw, **self.kw, out=self.out_r,
-                                              saved_states=self.saved_r)
+                                              saved_states=self.saved_r, workspace=self.ws_f)
 
     def fused_bwd(self):
         self.gr = self.msc.msc_mamba3_siso_scan_bwd_raw(

@@ -572,14 +572,25 @@ msc_status msc_mamba3_siso_discretize_bwd(const msc_m3_disc_bwd_args *args, msc_
 /* ======================================================================
  * Mamba-3 SISO scan from raw projections (discretisation fused in)
  * ======================================================================
- * The scan forward and backward with the discretisation and BCNorm above
- * fused into them (the pages list the stages B6 "discretization" and B5
- * "BCNorm" of Mamba3Scratch either side of the BPTT and RoPE stages, mamba-rs
- * 0.4.2 src/mamba3_siso/cpu/scratch.rs).  The kernels derive alpha, beta,
- * gamma, theta and the normalised Bm, Cm from the raw values as they stage
- * each chunk, so theta [B, L, H, K] and the other derived inputs are never
- * written or read in global memory.  Every derived value is rounded to bf16
- * exactly as msc_mamba3_siso_discretize stores it, so:
+ * The scan forward and backward taking the raw projections of the
+ * discretisation and BCNorm above (the pages list the stages B6
+ * "discretization" and B5 "BCNorm" of Mamba3Scratch either side of the BPTT
+ * and RoPE stages, mamba-rs 0.4.2 src/mamba3_siso/cpu/scratch.rs), so that
+ * nothing derived from them is kept between the forward and the backward.
+ *   forward   the per-head discretisation is fused into the scan's kernel:
+ *             it derives alpha, beta, gamma and theta from dd_dt, dd_a,
+ *             trap and angles as it stages each chunk, so theta
+ *             [B, L, H, K] and alpha .. gamma are never written or read in
+ *             global memory.  BCNorm acts per (b, t, g), on rows the group's
+ *             heads share, so it runs once per row, by the discretisation
+ *             kernel, into the call's workspace, ahead of the scan.
+ *   backward  the discretisation and BCNorm are re-derived once, by the
+ *             discretisation kernel, into the workspace; the scan's backward
+ *             kernels read them there (deriving them inside both of its
+ *             chunk kernels measured slower), and the discretisation's
+ *             backward turns the scan's gradients into the raw ones.
+ * Every derived value is rounded to bf16 exactly as
+ * msc_mamba3_siso_discretize stores it, so:
  *   msc_mamba3_siso_scan_fwd_raw  equals, bit for bit,
  *     msc_mamba3_siso_discretize followed by msc_mamba3_siso_scan_fwd;
  *   msc_mamba3_siso_scan_bwd_raw  equals, bit for bit,
@@ -591,10 +602,15 @@ msc_status msc_mamba3_siso_discretize_bwd(const msc_m3_disc_bwd_args *args, msc_
  * In the scan arguments (msc_m3_fwd_args / msc_m3_bwd_args) alpha, beta,
  * gamma, theta, Bm and Cm are ignored (may be NULL), and so, in the backward,
  * are dB, dC, dalpha, dbeta, dgamma and dtheta: the scan's gradients of the
- * derived inputs live in the workspace (msc_mamba3_siso_scan_bwd_raw
- * _workspace_bytes), and the raw gradients go to `grads`.  dx, dz, dD and
- * dh0 are the scan's, as in msc_mamba3_siso_scan_bwd.  Layouts as in
- * msc_mamba3_siso_discretize:
+ * derived inputs live in the workspace, and the raw gradients go to `grads`.
+ * dx, dz, dD and dh0 are the scan's, as in msc_mamba3_siso_scan_bwd.
+ * Workspaces (device memory, 16-byte aligned, caller-owned, contents
+ * undefined on return; MSC_ERR_WORKSPACE when missing or short):
+ *   forward   the `workspace` fields of msc_m3_fwd_args, at least
+ *             msc_mamba3_siso_scan_fwd_raw_workspace_bytes (BCNorm's rows);
+ *   backward  the `workspace` argument, at least
+ *             msc_mamba3_siso_scan_bwd_raw_workspace_bytes.
+ * Layouts as in msc_mamba3_siso_discretize:
  *   dd_dt, dd_a, trap         bf16 [B, L, H]
  *   angles                    bf16 [B, L, K]      (may be NULL when K = 0)
  *   dt_bias                   f32  [H]            optional
@@ -621,6 +637,10 @@ typedef struct {
 
 msc_status msc_mamba3_siso_scan_fwd_raw(const msc_m3_fwd_args *scan, const msc_m3_raw_args *raw,
                                         msc_stream_t stream);
+size_t msc_mamba3_siso_scan_fwd_raw_workspace_bytes(int64_t batch, int64_t seqlen,
+                                                    int64_t nheads, int64_t headdim,
+                                                    int64_t dstate, int64_t ngroups,
+                                                    int64_t nangles);
 size_t msc_mamba3_siso_scan_bwd_raw_workspace_bytes(int64_t batch, int64_t seqlen,
                                                     int64_t nheads, int64_t headdim,
                                                     int64_t dstate, int64_t ngroups,

@@ -107,8 +107,7 @@ msc_status check_raw(const char *fn, const Scan *a, const msc_m3_raw_args *raw) 
     return api_fail(MSC_ERR_UNSUPPORTED,
                     "%s: io_dtype %d: the fused path takes bf16 io (use "
                     "msc_mamba3_siso_discretize and the scan)", fn, (int)a->io_dtype);
-  // the tensor-core kernels' own sizes: their BCNorm sums runs of 8 states
-  // in the order the discretisation kernel does, and divides by d_state
+  // the tensor-core kernels of one 64-state slab
   if (a->dstate != 16 && a->dstate != 32 && a->dstate != 64)
     return api_fail(MSC_ERR_UNSUPPORTED,
                     "%s: dstate %lld: the fused path takes d_state 16, 32 or 64 (use "
@@ -127,13 +126,37 @@ msc_status check_raw(const char *fn, const Scan *a, const msc_m3_raw_args *raw) 
   return MSC_OK;
 }
 
-// The scan arguments with the derived inputs (alpha .. theta, Bm, Cm) taken
-// by the raw rows, so that the scan's own pointer checks test those.
+// BCNorm's rows in the fused entry points' workspace: Bm, Cm bf16 [B, L, G, N]
+// each, 256-byte aligned.  BCNorm is per (b, t, g), shared by the group's
+// heads, so it runs once per row ahead of the per-head scan kernels.
+size_t bcnorm_bytes(int64_t B, int64_t L, int64_t G, int64_t N) {
+  return (sizeof(uint16_t) * (size_t)(B * L * G * N) + 255) / 256 * 256;
+}
+
+// The BCNorm pass: the discretisation kernel with its B and C outputs alone,
+// so the rows are the bits msc_mamba3_siso_discretize writes.
 template <typename Scan>
-Scan with_raw(const Scan *a, const msc_m3_raw_args *raw) {
+cudaError_t bcnorm_pass(const Scan *a, const msc_m3_raw_args *raw, void *bn, void *cn,
+                        cudaStream_t s) {
+  msc::M3DiscParams d = {};
+  d.io = a->io_dtype;
+  d.B = a->batch; d.L = a->seqlen; d.H = a->nheads; d.N = a->dstate; d.G = a->ngroups;
+  d.K = a->nangles;
+  d.bc_only = true;
+  d.A_floor = raw->A_floor; d.eps = raw->eps;
+  d.B_raw = raw->B_raw; d.C_raw = raw->C_raw;
+  d.Bm = bn; d.Cm = cn;
+  return msc::launch_m3_disc_fwd(d, s);
+}
+
+// The scan arguments with the derived inputs taken by the raw rows (alpha ..
+// theta) and by BCNorm's rows (Bm, Cm), so that the scan's own pointer checks
+// test those.
+template <typename Scan>
+Scan with_raw(const Scan *a, const msc_m3_raw_args *raw, const void *bn, const void *cn) {
   Scan s = *a;
-  s.Bm = raw->B_raw;
-  s.Cm = raw->C_raw;
+  s.Bm = bn;
+  s.Cm = cn;
   s.alpha = raw->dd_dt;
   s.beta = raw->dd_a;
   s.gamma = raw->trap;
@@ -143,8 +166,6 @@ Scan with_raw(const Scan *a, const msc_m3_raw_args *raw) {
 
 void set_raw(msc::M3Params &p, const msc_m3_raw_args *raw) {
   p.raw = true;
-  p.Bm = raw->B_raw;
-  p.Cm = raw->C_raw;
   p.alpha = p.beta = p.gamma = p.theta = nullptr;
   p.dd_dt = raw->dd_dt;
   p.dd_a = raw->dd_a;
@@ -219,11 +240,42 @@ msc_status msc_mamba3_siso_scan_fwd(const msc_m3_fwd_args *a, msc_stream_t strea
 msc_status msc_mamba3_siso_scan_fwd_raw(const msc_m3_fwd_args *a, const msc_m3_raw_args *raw,
                                         msc_stream_t stream) {
   const char *fn = "msc_mamba3_siso_scan_fwd_raw";
-  msc_status st = check_m3(fn, a, offsetof(msc_m3_fwd_args, workspace));
+  msc_status st = check_m3(fn, a);
   if (st != MSC_OK) return st;
   if ((st = check_raw(fn, a, raw)) != MSC_OK) return st;
-  const msc_m3_fwd_args s = with_raw(a, raw);
+  const int64_t B = a->batch, L = a->seqlen, G = a->ngroups, N = a->dstate;
+  if (B == 0 || L == 0) return m3_fwd_impl(fn, a, raw, stream);  // no rows to normalise
+  const size_t rows = bcnorm_bytes(B, L, G, N);
+  if (a->workspace == nullptr || a->workspace_bytes < 2 * rows)
+    return api_fail(MSC_ERR_WORKSPACE, "%s: workspace of %zu bytes given, %zu required", fn,
+                    a->workspace ? a->workspace_bytes : (size_t)0, 2 * rows);
+  M3_REQUIRE(fn, "workspace", a->workspace);
+  char *ws = static_cast<char *>(a->workspace);
+  msc_m3_fwd_args s = with_raw(a, raw, ws, ws + rows);
+  s.workspace = nullptr;  // d_state <= 64: the scan itself needs none
+  s.workspace_bytes = 0;
+  // the scan's own pointer checks, ahead of the BCNorm launch
+  M3_REQUIRE(fn, "x", s.x);
+  M3_REQUIRE(fn, "out", s.out);
+  M3_OPTIONAL(fn, "z", s.z);
+  M3_OPTIONAL(fn, "D", s.D);
+  M3_OPTIONAL(fn, "h0", s.h0);
+  M3_OPTIONAL(fn, "final_state", s.final_state);
+  M3_OPTIONAL(fn, "saved_states", s.saved_states);
+  if ((st = api_cuda(bcnorm_pass(a, raw, ws, ws + rows, reinterpret_cast<cudaStream_t>(stream)),
+                     fn)) != MSC_OK)
+    return st;
   return m3_fwd_impl(fn, &s, raw, stream);
+}
+
+size_t msc_mamba3_siso_scan_fwd_raw_workspace_bytes(int64_t batch, int64_t seqlen,
+                                                    int64_t nheads, int64_t headdim,
+                                                    int64_t dstate, int64_t ngroups,
+                                                    int64_t nangles) {
+  if (batch <= 0 || seqlen <= 0 || nheads <= 0 || headdim <= 0 || dstate <= 0 || ngroups <= 0 ||
+      nangles < 0)
+    return 0;
+  return 2 * bcnorm_bytes(batch, seqlen, ngroups, dstate);
 }
 
 size_t msc_mamba3_siso_scan_bwd_workspace_bytes(int64_t batch, int64_t seqlen, int64_t nheads,
@@ -238,12 +290,10 @@ size_t msc_mamba3_siso_scan_bwd_workspace_bytes(int64_t batch, int64_t seqlen, i
 
 namespace {
 
-// the scan backward; raw non-null: from raw projections (derived-input
-// pointers already replaced by with_raw; the gradients of the derived inputs
-// go where the arguments say -- the fused entry point points them into its
-// workspace)
-msc_status m3_bwd_impl(const char *fn, const msc_m3_bwd_args *a, const msc_m3_raw_args *raw,
-                       void *workspace, size_t workspace_bytes, msc_stream_t stream) {
+// the scan backward (the raw-projection entry point points the derived inputs
+// and their gradients into its workspace)
+msc_status m3_bwd_impl(const char *fn, const msc_m3_bwd_args *a, void *workspace,
+                       size_t workspace_bytes, msc_stream_t stream) {
   msc_status st = check_m3(fn, a);
   if (st != MSC_OK) return st;
   const int64_t B = a->batch, L = a->seqlen, H = a->nheads, P = a->headdim, N = a->dstate;
@@ -299,15 +349,16 @@ msc_status m3_bwd_impl(const char *fn, const msc_m3_bwd_args *a, const msc_m3_ra
   p.dx = a->dx; p.dz = a->z ? a->dz : nullptr; p.dB = a->dB; p.dC = a->dC;
   p.dalpha = a->dalpha; p.dbeta = a->dbeta; p.dgamma = a->dgamma; p.dtheta = a->dtheta;
   p.dD = a->dD; p.dh0 = a->dh0; p.ws = workspace; p.ws_bytes = workspace_bytes;
-  if (raw) set_raw(p, raw);
   return api_cuda(msc::launch_m3_bwd(p, s), fn);
 }
 
-// the fused backward's workspace: the scan's own, then the scan's f32
-// gradients of the derived inputs: dalpha, dbeta, dgamma [B, L, H], dtheta
-// [B, L, H, K], dB, dC [B, L, G, N]
+// the raw-projection backward's workspace: the scan's own, then the scan's
+// f32 gradients of the derived inputs: dalpha, dbeta, dgamma [B, L, H],
+// dtheta [B, L, H, K], dB, dC [B, L, G, N], then the derived inputs
+// themselves (bf16): alpha, beta, gamma [B, L, H], theta [B, L, H, K], Bm,
+// Cm [B, L, G, N]
 struct RawWs {
-  size_t da, db, dg, dth, dB, dC, total;
+  size_t da, db, dg, dth, dB, dC, al, be, ga, th, bn, cn, total;
 };
 RawWs raw_ws(int64_t B, int64_t L, int64_t H, int64_t P, int64_t N, int64_t G, int64_t K) {
   auto up = [](size_t v) { return (v + 255) / 256 * 256; };
@@ -319,7 +370,15 @@ RawWs raw_ws(int64_t B, int64_t L, int64_t H, int64_t P, int64_t N, int64_t G, i
   w.dth = w.dg + th;
   w.dB = w.dth + up(sizeof(float) * (size_t)(B * L * H * (K > 0 ? K : 1)));
   w.dC = w.dB + up(sizeof(float) * (size_t)(B * L * G * N));
-  w.total = w.dC + up(sizeof(float) * (size_t)(B * L * G * N));
+  // the discretisation's outputs, re-derived from the raw projections (bf16)
+  w.al = w.dC + up(sizeof(float) * (size_t)(B * L * G * N));
+  const size_t hb = up(sizeof(uint16_t) * (size_t)(B * L * H));
+  w.be = w.al + hb;
+  w.ga = w.be + hb;
+  w.th = w.ga + hb;
+  w.bn = w.th + up(sizeof(uint16_t) * (size_t)(B * L * H * (K > 0 ? K : 1)));
+  w.cn = w.bn + bcnorm_bytes(B, L, G, N);
+  w.total = w.cn + bcnorm_bytes(B, L, G, N);
   return w;
 }
 
@@ -329,7 +388,7 @@ extern "C" {
 
 msc_status msc_mamba3_siso_scan_bwd(const msc_m3_bwd_args *a, void *workspace,
                                     size_t workspace_bytes, msc_stream_t stream) {
-  return m3_bwd_impl("msc_mamba3_siso_scan_bwd", a, nullptr, workspace, workspace_bytes, stream);
+  return m3_bwd_impl("msc_mamba3_siso_scan_bwd", a, workspace, workspace_bytes, stream);
 }
 
 size_t msc_mamba3_siso_scan_bwd_raw_workspace_bytes(int64_t batch, int64_t seqlen,
@@ -358,9 +417,9 @@ msc_status msc_mamba3_siso_scan_bwd_raw(const msc_m3_bwd_args *a, const msc_m3_r
   const int64_t B = a->batch, L = a->seqlen, H = a->nheads, P = a->headdim, N = a->dstate;
   const int64_t G = a->ngroups, K = a->nangles;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  msc_m3_bwd_args sa = with_raw(a, raw);
+  msc_m3_bwd_args sa = *a;
   if (B == 0 || L == 0) {  // no tokens: dD, dh0 and the bias gradient are 0
-    st = m3_bwd_impl(fn, &sa, raw, workspace, workspace_bytes, stream);
+    st = m3_bwd_impl(fn, &sa, workspace, workspace_bytes, stream);
     if (st != MSC_OK || !grads->ddt_bias) return st;
     return api_cuda(cudaMemsetAsync(grads->ddt_bias, 0, sizeof(float) * (size_t)H, s), fn);
   }
@@ -375,14 +434,40 @@ msc_status msc_mamba3_siso_scan_bwd_raw(const msc_m3_bwd_args *a, const msc_m3_r
   if (K > 0) M3_REQUIRE(fn, "dangles", grads->dangles);
   M3_REQUIRE(fn, "dB_raw", grads->dB_raw);
   M3_REQUIRE(fn, "dC_raw", grads->dC_raw);
+  // the scan's own pointer checks, ahead of the first launch
+  M3_REQUIRE(fn, "x", a->x);
+  M3_REQUIRE(fn, "saved_states", a->saved_states);
+  M3_REQUIRE(fn, "dout", a->dout);
+  M3_REQUIRE(fn, "dx", a->dx);
+  M3_OPTIONAL(fn, "z", a->z);
+  M3_OPTIONAL(fn, "dz", a->dz);
+  M3_OPTIONAL(fn, "D", a->D);
+  M3_OPTIONAL(fn, "h0", a->h0);
+  M3_OPTIONAL(fn, "dD", a->dD);
+  M3_OPTIONAL(fn, "dh0", a->dh0);
   char *ws = static_cast<char *>(workspace);
+  // the discretisation and BCNorm once, into the workspace: the backward's two
+  // chunk kernels then read them (deriving the per-head values inside both
+  // measured slower than this pass and the reads)
+  msc::M3DiscParams f = {};
+  f.io = a->io_dtype;
+  f.B = B; f.L = L; f.H = H; f.N = N; f.G = G; f.K = K;
+  f.A_floor = raw->A_floor; f.eps = raw->eps;
+  f.dd_dt = raw->dd_dt; f.dd_a = raw->dd_a; f.trap = raw->trap; f.angles = raw->angles;
+  f.dt_bias = raw->dt_bias; f.B_raw = raw->B_raw; f.C_raw = raw->C_raw;
+  f.alpha = ws + w.al; f.beta = ws + w.be; f.gamma = ws + w.ga;
+  f.theta = K > 0 ? ws + w.th : nullptr;
+  f.Bm = ws + w.bn; f.Cm = ws + w.cn;
+  if ((st = api_cuda(msc::launch_m3_disc_fwd(f, s), fn)) != MSC_OK) return st;
+  sa.alpha = f.alpha; sa.beta = f.beta; sa.gamma = f.gamma; sa.theta = f.theta;
+  sa.Bm = f.Bm; sa.Cm = f.Cm;
   sa.dalpha = reinterpret_cast<float *>(ws + w.da);
   sa.dbeta = reinterpret_cast<float *>(ws + w.db);
   sa.dgamma = reinterpret_cast<float *>(ws + w.dg);
   sa.dtheta = reinterpret_cast<float *>(ws + w.dth);
   sa.dB = reinterpret_cast<float *>(ws + w.dB);
   sa.dC = reinterpret_cast<float *>(ws + w.dC);
-  st = m3_bwd_impl(fn, &sa, raw, workspace, w.da, stream);
+  st = m3_bwd_impl(fn, &sa, workspace, w.da, stream);
   if (st != MSC_OK) return st;
   // the discretisation's backward on the scan's gradients of its outputs
   msc::M3DiscParams d = {};

@@ -111,10 +111,10 @@ struct M3Params {
   int64_t n0, ldN;
   int slab;  // kSlabWhole, kSlabFirst, kSlabMiddle or kSlabLast
   float *tok_y, *tok_dx;  // [B, L, H, P] f32
-  // from raw projections (bf16 io, d_state <= kM3Slab): alpha, beta, gamma,
-  // theta and the normalised B, C are derived in the kernels from these, each
-  // rounded to bf16 as the discretisation kernel stores it (Bm, Cm point at
-  // B_raw, C_raw; alpha .. theta are unused)
+  // forward from raw projections (bf16 io, d_state <= kM3Slab): alpha, beta,
+  // gamma and theta are derived in the kernel from these, each rounded to
+  // bf16 as the discretisation kernel stores it (alpha .. theta are unused;
+  // Bm, Cm are BCNorm's rows, normalised once per row ahead of the scan)
   bool raw;
   const void *dd_dt, *dd_a, *trap, *angles;  // [B, L, H] x3, [B, L, K]
   const float *dt_bias;                      // [H] or null
@@ -142,6 +142,7 @@ bool m3_supported(int64_t P, int64_t N);
 struct M3DiscParams {
   int io;  // msc_dtype
   int64_t B, L, H, N, G, K;
+  bool bc_only;  // forward: BCNorm alone (Bm, Cm), no alpha .. theta
   float A_floor, eps;
   const void *dd_dt, *dd_a, *trap, *angles;  // io [B, L, H] x3, [B, L, K]
   const float *dt_bias;                      // [H] or null

@@ -42,7 +42,6 @@
 // entries 2 % off.  The bf16 inputs x go as one exact part.  Every sum has a fixed order: the
 // results are the same bits on every run.
 #include "m3_common.cuh"
-#include "m3_disc_common.cuh"
 #include "umma.cuh"
 
 namespace msc {
@@ -181,10 +180,7 @@ struct Vec {
                        bx = 910, da = 975, xprev = 1040, bprev = 1104, phist = 1168,
                        part = 1200 /* [2][64] partial row sums */, red = 1328 /* [3][8] */,
                        rowb = 1352 /* [8][64] per-run parts of Ct.Bt_prev */,
-                       rowx = 1864 /* [8][64] per-run parts of g.x_prev */,
-                       nrm = 2376 /* [2][8][64] per-run squares of the raw B, C rows */,
-                       dt = 3400 /* [64] dt (from raw projections) */,
-                       rsc = 3464 /* [2][64] BCNorm scales of the raw B, C rows */, total = 3592;
+                       rowx = 1864 /* [8][64] per-run parts of g.x_prev */, total = 2376;
 };
 
 // Row stride (floats) of the angle table tPhi [t][k]: padded so that the
@@ -262,12 +258,7 @@ struct Loads {
   float4 s0[kST], s1[kST], u0[kST], u1[kST];
   bf16 th[kTH];
   bf16 al, be, ga, prev;
-  bool in_step;
-  float phist, bias;
-  // from raw projections: the step's alpha, beta, gamma (rounded to bf16 as
-  // the discretisation stores them) and dt, derived by coef() while the
-  // current unit waits on its tensor cores
-  float ca, cbt, cgm, cdt;
+  float phist;
 
   __device__ __forceinline__ void issue(const M3Params &p, const Chunk &c, const float *sin,
                                         const float *usrc) {
@@ -315,29 +306,25 @@ struct Loads {
         }
       }
     }
-    // theta per (t, k) -- or, from raw projections, the raw angles (shared by
-    // the heads)
-    const bf16 *thp = static_cast<const bf16 *>(p.raw ? p.angles : p.theta);
+    const bf16 *thp = static_cast<const bf16 *>(p.theta);
 #pragma unroll
     for (int q = 0; q < kTH; ++q) {
       const int i = tid + q * kThreads, t = i >> 5, k = i & 31;
-      const int64_t row = p.raw ? (c.b * p.L + c.t0 + t) : ((c.b * p.L + c.t0 + t) * p.H + c.h);
-      th[q] = (k < c.K && t < c.Qc) ? thp[row * c.Kt + c.k0 + k] : __float2bfloat16_rn(0.f);
+      th[q] = (k < c.K && t < c.Qc)
+                  ? thp[((c.b * p.L + c.t0 + t) * p.H + c.h) * c.Kt + c.k0 + k]
+                  : __float2bfloat16_rn(0.f);
     }
-    // alpha, beta, gamma -- or dd_dt, dd_a, trap and the head's dt bias
     const bf16 one = __float2bfloat16_rn(1.f), nil = __float2bfloat16_rn(0.f);
-    bias = (p.raw && p.dt_bias && tid <= kQ) ? p.dt_bias[c.h] : 0.f;
     al = one;
     be = ga = nil;
-    in_step = false;
     if (tid <= kQ) {
       const int64_t tg = c.t0 + tid;
-      in_step = tid < kQ ? tid < c.Qc : tg < p.L;  // row Q: the next chunk's first step
+      const bool in = tid < kQ ? tid < c.Qc : tg < p.L;  // row Q: the next chunk's first step
       const int64_t j = (c.b * p.L + tg) * p.H + c.h;
-      if (in_step) {
-        al = static_cast<const bf16 *>(p.raw ? p.dd_dt : p.alpha)[j];
-        be = static_cast<const bf16 *>(p.raw ? p.dd_a : p.beta)[j];
-        ga = static_cast<const bf16 *>(p.raw ? p.trap : p.gamma)[j];
+      if (in) {
+        al = static_cast<const bf16 *>(p.alpha)[j];
+        be = static_cast<const bf16 *>(p.beta)[j];
+        if (tid < kQ) ga = static_cast<const bf16 *>(p.gamma)[j];
       }
     }
     phist = 0.f;
@@ -346,25 +333,11 @@ struct Loads {
                         (c.b * p.H + c.h) * c.nc * (c.ldN / 2);
       phist = ps[c.ch * (c.ldN / 2) + c.k0 + tid];
     }
-    ca = 1.f;
-    cbt = cgm = cdt = 0.f;
     prev = nil;
     if (c.t0 > 0 && tid < P + N) {
       prev = tid < P ? x[((c.b * p.L + c.t0 - 1) * p.H + c.h) * P + tid]
                      : Bm[((c.b * p.L + c.t0 - 1) * p.G + c.g) * c.ldN + c.n0 + tid - P];
     }
-  }
-
-  // the discretisation of this thread's step (threads 0 .. Q; padded steps
-  // keep alpha = 1, beta = gamma = 0), once the issued loads have landed
-  __device__ __forceinline__ void coef(const M3Params &p) {
-    if (!p.raw || threadIdx.x > kQ || !in_step) return;
-    const DiscCoef cf = disc_coef(__bfloat162float(al), bias, __bfloat162float(be),
-                                  __bfloat162float(ga), p.A_floor);
-    ca = to_f32(from_f32<bf16>(cf.alpha));
-    cbt = to_f32(from_f32<bf16>(disc_beta(cf)));
-    cgm = to_f32(from_f32<bf16>(disc_gamma(cf)));
-    cdt = cf.dt;
   }
 };
 
@@ -372,22 +345,12 @@ struct Loads {
 // beta), theta into the angle table, the chunk-start angles, x_prev and B_prev
 // (raw).
 template <class LD>
-__device__ __forceinline__ void stage_small(const M3Params &p, const Chunk &c, const LD &ld,
-                                            float *sv, float *tPhi, int P, int N) {
+__device__ __forceinline__ void stage_small(const LD &ld, float *sv, float *tPhi, int P, int N) {
   const int tid = threadIdx.x;
   if (tid <= kQ) {
-    if (p.raw) {  // the discretisation, derived ahead by ld.coef()
-      sv[Vec::al + tid] = ld.ca;
-      sv[Vec::be + tid] = ld.cbt;
-      if (tid < kQ) {
-        sv[Vec::ga + tid] = ld.cgm;
-        sv[Vec::dt + tid] = ld.cdt;
-      }
-    } else {
-      sv[Vec::al + tid] = __bfloat162float(ld.al);
-      sv[Vec::be + tid] = __bfloat162float(ld.be);
-      if (tid < kQ) sv[Vec::ga + tid] = __bfloat162float(ld.ga);
-    }
+    sv[Vec::al + tid] = __bfloat162float(ld.al);
+    sv[Vec::be + tid] = __bfloat162float(ld.be);
+    if (tid < kQ) sv[Vec::ga + tid] = __bfloat162float(ld.ga);
   }
 #pragma unroll
   for (int q = 0; q < LD::kTH; ++q) {
@@ -404,54 +367,11 @@ __device__ __forceinline__ void stage_small(const M3Params &p, const Chunk &c, c
 // angles, the decay table d(t, s) = prod_{r=s+1..t} alpha_r (column s + 1;
 // column 0: d(t, -1); zero above the diagonal; per column a product scan in
 // the same layout), and the per-step coefficients.
-// The sum of n = 2^j values in the order of an xor butterfly over n lanes
-// (pairs, then pairs of pairs, ...): the order the discretisation kernel's
-// row norms take.
-__device__ __forceinline__ float tree_sum(float *v, int n) {
-  for (int m = 1; m < n; m <<= 1)
-    for (int i = 0; i + m < n; i += 2 * m) v[i] += v[i + m];
-  return v[0];
-}
-
-__device__ __forceinline__ void stage_decays(const M3Params &p, const Chunk &c, float *sv,
-                                             float *tPhi, float *tD) {
+__device__ __forceinline__ void stage_decays(const Chunk &c, float *sv, float *tPhi, float *tD) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int t0 = 2 * lane, t1 = t0 + 1;
-  if (p.raw && tid >= kThreads - 2 * kQ) {
-    // BCNorm's scale of raw row r (B rows 0 .. Q-1, then C): the runs' sums of
-    // squares combined in the order of an xor butterfly
-    const int r = tid - (kThreads - 2 * kQ), R = (int)p.N / 8;
-    float part[8];
-    for (int q = 0; q < R; ++q) part[q] = sv[Vec::nrm + (r / kQ) * 512 + q * 64 + r % kQ];
-    sv[Vec::rsc + r] = rsqrtf(tree_sum(part, R) / (float)p.N + p.eps);
-  }
-  if (p.raw && warp == 0 && c.t0 > 0) {
-    // B_prev is a raw row: normalised as BCNorm would -- lane r < N / 8 sums
-    // run r of 8 states in order, then an xor butterfly over the runs (the
-    // discretisation kernel's order)
-    const int R = (int)p.N / 8;
-    float v[8], ss = 0.f;
-    if (lane < R) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        v[e] = sv[Vec::bprev + 8 * lane + e];
-        ss = fmaf(v[e], v[e], ss);
-      }
-    }
-    for (int m = 1; m < R; m <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
-    const float rn = rsqrtf(ss / (float)p.N + p.eps);
-    if (lane < R) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) sv[Vec::bprev + 8 * lane + e] = to_f32(from_f32<bf16>(v[e] * rn));
-    }
-  }
-  __syncwarp();
   for (int k = warp; k < c.K; k += kThreads / 32) {
-    float a0 = tPhi[t0 * kPhS + k], a1 = tPhi[t1 * kPhS + k];
-    if (p.raw) {  // theta = dt x angle, rounded to bf16 (this thread's two steps)
-      a0 = to_f32(from_f32<bf16>(sv[Vec::dt + t0] * a0));
-      a1 = to_f32(from_f32<bf16>(sv[Vec::dt + t1] * a1));
-    }
+    const float a0 = tPhi[t0 * kPhS + k], a1 = tPhi[t1 * kPhS + k];
     float incl = a0 + a1;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -508,42 +428,12 @@ __device__ __forceinline__ float cw(const float *tD, const float *sv, int t, int
   return s == t ? sv[Vec::ga + t] : (s < t ? tD[t * 65 + s + 2] * sv[Vec::eps + s] : 0.f);
 }
 
-// Phase 1, from raw projections: BCNorm's sum of squares of each run of 8
-// states of the chunk's raw B and C rows (sequential over its 8), into nrm
-// [run][t]; phase 2 combines the runs of a row in the order of an xor
-// butterfly, as the discretisation kernel does, into the row's scale.
-template <int N, class LD>
-__device__ __forceinline__ void stage_norm_sums(const LD &ld, float *sv) {
-  constexpr int kR = N / 8;
-#pragma unroll
-  for (int k = 0; k < LD::kBC; ++k) {
-    const int u = threadIdx.x + k * kThreads;
-    if (u >= kQ * kR) break;
-    int t, r;
-    row_run<kR>(u, t, r);
-    float bv[8], cv[8];
-    unpack_bf16x2(ld.bb[k].x, bv[0], bv[1]); unpack_bf16x2(ld.bb[k].y, bv[2], bv[3]);
-    unpack_bf16x2(ld.bb[k].z, bv[4], bv[5]); unpack_bf16x2(ld.bb[k].w, bv[6], bv[7]);
-    unpack_bf16x2(ld.cc[k].x, cv[0], cv[1]); unpack_bf16x2(ld.cc[k].y, cv[2], cv[3]);
-    unpack_bf16x2(ld.cc[k].z, cv[4], cv[5]); unpack_bf16x2(ld.cc[k].w, cv[6], cv[7]);
-    float sb = 0.f, sc = 0.f;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      sb = fmaf(bv[e], bv[e], sb);
-      sc = fmaf(cv[e], cv[e], sc);
-    }
-    sv[Vec::nrm + r * 64 + t] = sb;
-    sv[Vec::nrm + 512 + r * 64 + t] = sc;
-  }
-}
-
 // Phase 3 (after phase 2): the rotated B and C rows of the chunk into the
 // operand planes; the per-run parts of Ct_t . Bt_prev into rowb (added in run
 // order by row_sums).  A unit is 8 consecutive states of one step.
 template <int N, class LD>
-__device__ __forceinline__ void stage_bc(const M3Params &p, const LD &ld, const Chunk &c,
-                                         float *sv, const float *tPhi, unsigned char *pB,
-                                         unsigned char *pC) {
+__device__ __forceinline__ void stage_bc(const LD &ld, const Chunk &c, float *sv,
+                                         const float *tPhi, unsigned char *pB, unsigned char *pC) {
   constexpr int kR = N / 8;  // runs per row
 #pragma unroll
   for (int k = 0; k < LD::kBC; ++k) {
@@ -556,14 +446,6 @@ __device__ __forceinline__ void stage_bc(const M3Params &p, const LD &ld, const 
     unpack_bf16x2(ld.bb[k].z, bv[4], bv[5]); unpack_bf16x2(ld.bb[k].w, bv[6], bv[7]);
     unpack_bf16x2(ld.cc[k].x, cv[0], cv[1]); unpack_bf16x2(ld.cc[k].y, cv[2], cv[3]);
     unpack_bf16x2(ld.cc[k].z, cv[4], cv[5]); unpack_bf16x2(ld.cc[k].w, cv[6], cv[7]);
-    if (p.raw) {  // BCNorm, the row scales from phase 2
-      const float rb = sv[Vec::rsc + t], rc = sv[Vec::rsc + kQ + t];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        bv[e] = to_f32(from_f32<bf16>(bv[e] * rb));
-        cv[e] = to_f32(from_f32<bf16>(cv[e] * rc));
-      }
-    }
     float dot = 0.f;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -742,7 +624,6 @@ __global__ void __launch_bounds__(kThreads, 1) m3b_prep_kernel(const M3Params p,
   if ((int64_t)blockIdx.x < n_units) {
     const Chunk c0 = chunk_of(p, P, blockIdx.x);
     ld.issue(p, c0, sin_of(c0), nullptr);
-    ld.coef(p);
   }
   umma::fence_before();
   __syncthreads();
@@ -751,12 +632,11 @@ __global__ void __launch_bounds__(kThreads, 1) m3b_prep_kernel(const M3Params p,
   for (int64_t unit = blockIdx.x; unit < n_units; unit += gridDim.x) {
   const Chunk c = chunk_of(p, P, unit);
   const float Dh = (p.Dp && finish) ? p.Dp[c.h] : 0.f;
-  stage_small(p, c, ld, sv, tPhi, P, N);
-  if (p.raw) stage_norm_sums<N>(ld, sv);
+  stage_small(ld, sv, tPhi, P, N);
   __syncthreads();
-  stage_decays(p, c, sv, tPhi, tD);
+  stage_decays(c, sv, tPhi, tD);
   __syncthreads();
-  stage_bc<N>(p, ld, c, sv, tPhi, sm + S::pB, sm + S::pC);
+  stage_bc<N>(ld, c, sv, tPhi, sm + S::pB, sm + S::pC);
   stage_xg<P>(ld, p.z != nullptr, sv, sm + S::pX, nullptr, sm + S::pGd);
   {
     float us = 0.f, vm1 = 0.f;
@@ -820,7 +700,6 @@ __global__ void __launch_bounds__(kThreads, 1) m3b_prep_kernel(const M3Params p,
     product<P, true>(tmem, 192, base + S::pW, kParts, 64, base + S::pX, 1, P, 64, false);  // W X
     umma::commit(mbar);
   }
-  ld.coef(p);  // the next unit's discretisation while W X runs
   if (!umma::mbar_wait(mbar, 1)) *sErr = 1;
   umma::fence_after();
   // ---- y and dz ----------------------------------------------------------------------
@@ -917,19 +796,7 @@ __global__ void __launch_bounds__(256) m3b_carry_kernel(const M3Params p, float 
     }
     if (p.dh0) {
       const int64_t b = bh / p.H, h = bh % p.H;
-      const int64_t j = (b * p.L) * p.H + h;
-      float a0;
-      if (p.raw) {  // alpha_0 from the raw row, rounded as the discretisation stores it
-        const bf16 *dd_dt = static_cast<const bf16 *>(p.dd_dt);
-        const bf16 *dd_a = static_cast<const bf16 *>(p.dd_a);
-        const bf16 *trap = static_cast<const bf16 *>(p.trap);
-        a0 = to_f32(from_f32<bf16>(disc_coef(__bfloat162float(dd_dt[j]),
-                                             p.dt_bias ? p.dt_bias[h] : 0.f,
-                                             __bfloat162float(dd_a[j]), __bfloat162float(trap[j]),
-                                             p.A_floor).alpha));
-      } else {
-        a0 = __bfloat162float(static_cast<const bf16 *>(p.alpha)[j]);
-      }
+      const float a0 = __bfloat162float(static_cast<const bf16 *>(p.alpha)[(b * p.L) * p.H + h]);
       p.dh0[bh * PN + e] = a0 * U;  // alpha_0 Lambda_0
     }
   }
@@ -968,7 +835,6 @@ __global__ void __launch_bounds__(kThreads, 1) m3b_grad_kernel(const M3Params p,
   if ((int64_t)blockIdx.x < n_units) {
     const Chunk c0 = chunk_of(p, P, blockIdx.x);
     ld.issue(p, c0, p.saved_in + off_of(c0), vu + off_of(c0));
-    ld.coef(p);
   }
   umma::fence_before();
   __syncthreads();
@@ -977,12 +843,11 @@ __global__ void __launch_bounds__(kThreads, 1) m3b_grad_kernel(const M3Params p,
   for (int64_t unit = blockIdx.x; unit < n_units; unit += gridDim.x) {
   const Chunk c = chunk_of(p, P, unit);
   const float Dh = (p.Dp && finish) ? p.Dp[c.h] : 0.f;
-  stage_small(p, c, ld, sv, tPhi, P, N);
-  if (p.raw) stage_norm_sums<N>(ld, sv);
+  stage_small(ld, sv, tPhi, P, N);
   __syncthreads();
-  stage_decays(p, c, sv, tPhi, tD);
+  stage_decays(c, sv, tPhi, tD);
   __syncthreads();
-  stage_bc<N>(p, ld, c, sv, tPhi, sm + S::pB, sm + S::pC);
+  stage_bc<N>(ld, c, sv, tPhi, sm + S::pB, sm + S::pC);
   const float gx_l = stage_xg<P>(ld, p.z != nullptr, sv, sm + S::pX, sm + S::pG, nullptr);
   float us_l = 0.f, vm1_l = 0.f;
   stage_state<P, N, true>(ld, sm + S::pS, sm + S::pU, sv, us_l, vm1_l);
@@ -1157,7 +1022,6 @@ __global__ void __launch_bounds__(kThreads, 1) m3b_grad_kernel(const M3Params p,
       sv[Vec::da + s] = v;
     }
   }
-  ld.coef(p);  // the next unit's discretisation while round 2 may still run
   if (!umma::mbar_wait(mbar, 1)) *sErr = 1;
   umma::fence_after();
   __syncthreads();

@@ -116,7 +116,7 @@ __global__ void __launch_bounds__(kDiscWarps * 32) m3_disc_fwd_kernel(const M3Di
   const int64_t ntok = p.B * p.L;
   for (int64_t tok = (int64_t)blockIdx.x * kDiscWarps + warp; tok < ntok;
        tok += (int64_t)gridDim.x * kDiscWarps) {
-    for (int h = lane; h < H; h += 32) {
+    for (int h = lane; h < H && !p.bc_only; h += 32) {
       const int64_t i = tok * H + h;
       const DiscCoef c = head_coef<T>(p, i, h);
       static_cast<T *>(p.alpha)[i] = from_f32<T>(c.alpha);
@@ -124,10 +124,11 @@ __global__ void __launch_bounds__(kDiscWarps * 32) m3_disc_fwd_kernel(const M3Di
       static_cast<T *>(p.gamma)[i] = from_f32<T>(disc_gamma(c));
       sdt[h] = c.dt;
     }
-    for (int k = lane; k < K; k += 32) sang[k] = ldv<T>(p.angles, tok * K + k);
+    const int Kd = p.bc_only ? 0 : K;  // BCNorm alone: no theta
+    for (int k = lane; k < Kd; k += 32) sang[k] = ldv<T>(p.angles, tok * K + k);
     __syncwarp();
     if (vec_theta) {  // 8 angles of one head per lane, one 16-byte store (f32: two)
-      for (int j = 8 * lane; j < H * K; j += 256) {
+      for (int j = 8 * lane; j < H * Kd; j += 256) {
         const int h = j / K, k = j - h * K;
         float v[8];
 #pragma unroll
@@ -135,7 +136,7 @@ __global__ void __launch_bounds__(kDiscWarps * 32) m3_disc_fwd_kernel(const M3Di
         store8<T>(p.theta, tok * H * K + j, v);
       }
     } else {
-      for (int j = lane; j < H * K; j += 32) {
+      for (int j = lane; j < H * Kd; j += 32) {
         const int h = j / K, k = j - h * K;
         static_cast<T *>(p.theta)[tok * H * K + j] = from_f32<T>(sdt[h] * sang[k]);
       }

@@ -137,7 +137,7 @@ __device__ __forceinline__ void issue_product(uint32_t tmem, int col, uint32_t a
 
 // kSlab: one slab of a wider d_state (runtime row length and offsets);
 // otherwise the whole d_state with compile-time strides
-template <int P, int N, bool kSlab>
+template <int P, int N, bool kSlab, bool kRaw>
 __global__ void __launch_bounds__(kThreads, 2) m3_fwd_umma_kernel(const M3Params p) {
   using S = UmFwdSmem<P, N>;
   constexpr int kK = N / 2;
@@ -241,7 +241,7 @@ __global__ void __launch_bounds__(kThreads, 2) m3_fwd_umma_kernel(const M3Params
   float pa0, pa1, pb0, pb1, pg0, pg1;
   // from raw projections: the discretisation of step s (the expressions of
   // the discretisation kernel, each value rounded to bf16 as it stores them)
-  const float dtb = (p.raw && p.dt_bias) ? p.dt_bias[h] : 0.f;
+  const float dtb = (kRaw && p.dt_bias) ? p.dt_bias[h] : 0.f;
   float *sDt = reinterpret_cast<float *>(sm + S::dtv);
   auto raw_coef = [&](int64_t j, float &a, float &bt, float &gm) {
     const DiscCoef cf = disc_coef(__bfloat162float(static_cast<const bf16 *>(p.dd_dt)[j]), dtb,
@@ -261,7 +261,7 @@ __global__ void __launch_bounds__(kThreads, 2) m3_fwd_umma_kernel(const M3Params
       const int64_t t = t0 + 8 * m + ri;
       float v = 0.f;
       if (ka < K && t < L) {
-        if (p.raw)  // the raw angle (shared by the heads); theta = dt x angle once dt is in
+        if constexpr (kRaw)  // the raw angle (shared by the heads); theta = dt x angle once dt is in
           v = __bfloat162float(static_cast<const bf16 *>(p.angles)[(b * L + t) * Kt + k0 + ka]);
         else
           v = __bfloat162float(th_g[((b * L + t) * H + h) * Kt + k0 + ka]);
@@ -275,7 +275,7 @@ __global__ void __launch_bounds__(kThreads, 2) m3_fwd_umma_kernel(const M3Params
       float dt0 = 0.f, dt1 = 0.f;
       if (s < L) {
         const int64_t j = (b * L + s) * H + h;
-        if (p.raw) {
+        if constexpr (kRaw) {
           dt0 = raw_coef(j, pa0, pb0, pg0);
         } else {
           pa0 = __bfloat162float(al_g[j]);
@@ -285,7 +285,7 @@ __global__ void __launch_bounds__(kThreads, 2) m3_fwd_umma_kernel(const M3Params
       }
       if (s + 1 < L) {
         const int64_t j = (b * L + s + 1) * H + h;
-        if (p.raw) {
+        if constexpr (kRaw) {
           dt1 = raw_coef(j, pa1, pb1, pg1);
         } else {
           pa1 = __bfloat162float(al_g[j]);
@@ -293,38 +293,10 @@ __global__ void __launch_bounds__(kThreads, 2) m3_fwd_umma_kernel(const M3Params
           pg1 = __bfloat162float(ga_g[j]);
         }
       }
-      if (p.raw) {
+      if constexpr (kRaw) {
         sDt[2 * lane] = dt0;
         sDt[2 * lane + 1] = dt1;
       }
-    }
-  };
-  // BCNorm of the chunk's raw B and C rows in place: R = N / 8 lanes per row,
-  // each with a run of 8 states summed in order, the runs' sums combined by an
-  // xor butterfly over the R lanes (the discretisation kernel's order), every
-  // value rounded to bf16 as that kernel stores it
-  auto norm_rows = [&]() {
-    constexpr int R = N / 8;
-    static_assert((2 * kQ * R) % kThreads == 0, "every thread takes part in each butterfly");
-#pragma unroll
-    for (int u = tid; u < 2 * kQ * R; u += kThreads) {
-      const int row = u / R, run = u % R;
-      unsigned char *rowp = sm + (row < kQ ? S::rB : S::rC) + (row % kQ) * S::kRS + run * 16;
-      uint4 w = *reinterpret_cast<const uint4 *>(rowp);
-      uint32_t *wp = reinterpret_cast<uint32_t *>(&w);
-      float v[8];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) unpack_bf16x2(wp[e], v[2 * e], v[2 * e + 1]);
-      float ss = 0.f;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) ss = fmaf(v[e], v[e], ss);
-#pragma unroll
-      for (int m = 1; m < R; m <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
-      const float rn = rsqrtf(ss / (float)N + p.eps);
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        wp[e] = bf16pair(from_f32<bf16>(v[2 * e] * rn), from_f32<bf16>(v[2 * e + 1] * rn));
-      *reinterpret_cast<uint4 *>(rowp) = w;
     }
   };
   um_issue_raw<P, N, kSlab>(p, sm, b, h, g, 0);
@@ -345,12 +317,11 @@ __global__ void __launch_bounds__(kThreads, 2) m3_fwd_umma_kernel(const M3Params
     cp_async_wait<0>();
     __syncthreads();  // (A) this chunk's raw inputs are in; the last chunk is done
     if (*sErr) break;
-    if (p.raw) {
-      norm_rows();
+    if constexpr (kRaw) {
       // theta = dt x angle, rounded to bf16 as the discretisation stores it
+      // (sDt was written by warp 0 ahead of barrier (A))
 #pragma unroll
       for (int m = 0; m < 8; ++m) thv[m] = to_f32(from_f32<bf16>(sDt[8 * m + ri] * thv[m]));
-      __syncthreads();  // normalised rows in place
     }
 
     // ---- 1. state and angles entering the chunk; X^T; per-step vectors ----------
@@ -609,21 +580,29 @@ __global__ void __launch_bounds__(kThreads, 2) m3_fwd_umma_kernel(const M3Params
   }
 }
 
-template <int P, int N, bool kSlab>
+template <int P, int N, bool kSlab, bool kRaw = false>
 cudaError_t launch_um(const M3Params &p, cudaStream_t s) {
   // at least 80 KB of shared memory per CTA, so that no more than two CTAs
   // (2 x 256 TMEM columns) share an SM
   const size_t smem = UmFwdSmem<P, N>::total > 80 * 1024 ? (size_t)UmFwdSmem<P, N>::total : 80 * 1024;
-  cudaError_t e = cudaFuncSetAttribute(m3_fwd_umma_kernel<P, N, kSlab>,
+  cudaError_t e = cudaFuncSetAttribute(m3_fwd_umma_kernel<P, N, kSlab, kRaw>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  m3_fwd_umma_kernel<P, N, kSlab><<<dim3((unsigned)p.H, (unsigned)p.B), kThreads, smem, s>>>(p);
+  m3_fwd_umma_kernel<P, N, kSlab, kRaw><<<dim3((unsigned)p.H, (unsigned)p.B), kThreads, smem, s>>>(p);
   return cudaGetLastError();
 }
 
 template <int P>
 cudaError_t launch_um_n(const M3Params &p, cudaStream_t s) {
   if (p.slab != kSlabWhole) return launch_um<P, kM3Slab, true>(p, s);
+  // from raw projections: d_state 16, 32 or 64 (the API refuses others)
+  if (p.raw) {
+    switch (p.N) {
+      case 16: return launch_um<P, 16, false, true>(p, s);
+      case 32: return launch_um<P, 32, false, true>(p, s);
+      default: return launch_um<P, 64, false, true>(p, s);
+    }
+  }
   switch (p.N) {
     case 16: return launch_um<P, 16, false>(p, s);
     case 32: return launch_um<P, 32, false>(p, s);

@@ -154,7 +154,8 @@ EXPORTS = ["msc_last_error", "msc_version", "msc_selective_scan_saved_states_byt
            "msc_selective_scan_conv_fwd", "msc_mamba3_siso_discretize",
            "msc_mamba3_siso_discretize_bwd", "msc_mamba3_siso_disc_state_update",
            "msc_probe_threads_per_block", "msc_probe_sfu_ex2", "msc_probe_ffma",
-           "msc_mamba3_siso_scan_fwd_raw", "msc_mamba3_siso_scan_bwd_raw_workspace_bytes",
+           "msc_mamba3_siso_scan_fwd_raw", "msc_mamba3_siso_scan_fwd_raw_workspace_bytes",
+           "msc_mamba3_siso_scan_bwd_raw_workspace_bytes",
            "msc_mamba3_siso_scan_bwd_raw"]
 
 _lib = None
@@ -211,6 +212,8 @@ def lib() -> ctypes.CDLL:
         L.msc_causal_conv1d_bwd_workspace_bytes.restype = ctypes.c_size_t
         L.msc_mamba3_siso_scan_bwd_workspace_bytes.argtypes = [_i64] * 7
         L.msc_mamba3_siso_scan_bwd_workspace_bytes.restype = ctypes.c_size_t
+        L.msc_mamba3_siso_scan_fwd_raw_workspace_bytes.argtypes = [_i64] * 7
+        L.msc_mamba3_siso_scan_fwd_raw_workspace_bytes.restype = ctypes.c_size_t
         L.msc_mamba3_siso_scan_bwd_raw_workspace_bytes.argtypes = [_i64] * 7
         L.msc_mamba3_siso_scan_bwd_raw_workspace_bytes.restype = ctypes.c_size_t
         L.msc_probe_threads_per_block.argtypes = []
@@ -540,11 +543,17 @@ def _m3_raw(dd_dt, dd_a, trap, angles, B_raw, C_raw, dt_bias, A_floor, eps):
                      _ptr(angles), _ptr(dt_bias), _ptr(B_raw), _ptr(C_raw))
 
 
+def msc_mamba3_siso_scan_fwd_raw_workspace_bytes(batch, seqlen, nheads, headdim, dstate,
+                                                 ngroups, nangles) -> int:
+    return int(lib().msc_mamba3_siso_scan_fwd_raw_workspace_bytes(
+        batch, seqlen, nheads, headdim, dstate, ngroups, nangles))
+
+
 def msc_mamba3_siso_scan_fwd_raw(x, dd_dt, dd_a, trap, angles, B_raw, C_raw, dt_bias=None,
                                  A_floor=1e-4, eps=1e-5, D=None, z=None, h0=None, out=None,
                                  final_state=None, saved_states=None, want_final_state=True,
-                                 want_saved_states=True, stream=None):
-    """Mamba-3 SISO forward from raw projections (bf16, d_state <= 64):
+                                 want_saved_states=True, workspace=None, stream=None):
+    """Mamba-3 SISO forward from raw projections (bf16, d_state 16, 32 or 64):
     dd_dt, dd_a, trap [B, L, H]; angles [B, L, K]; B_raw, C_raw [B, L, G, N].
     Returns (out, final_state, saved_states); equals msc_mamba3_siso_discretize
     followed by msc_mamba3_siso_scan_fwd bit for bit."""
@@ -559,9 +568,12 @@ def msc_mamba3_siso_scan_fwd_raw(x, dd_dt, dd_a, trap, angles, B_raw, C_raw, dt_
     if saved_states is None and want_saved_states:
         nb = msc_mamba3_siso_saved_states_bytes(Bsz, L, H, P, N)
         saved_states = torch.empty(max(nb // 4, 4), device=dev, dtype=torch.float32)
+    if workspace is None:
+        need = msc_mamba3_siso_scan_fwd_raw_workspace_bytes(Bsz, L, H, P, N, G, K)
+        workspace = torch.empty(max(need, 16), device=dev, dtype=torch.uint8)
     a = M3FwdArgs(ctypes.sizeof(M3FwdArgs), _io(x), Bsz, L, H, P, N, G, K, _ptr(x), _ptr(z),
                   None, None, None, None, None, None, _ptr(D), _ptr(h0), _ptr(out),
-                  _ptr(final_state), _ptr(saved_states), None, 0)
+                  _ptr(final_state), _ptr(saved_states), _ptr(workspace), workspace.numel())
     r = _m3_raw(dd_dt, dd_a, trap, angles, B_raw, C_raw, dt_bias, A_floor, eps)
     _check(lib().msc_mamba3_siso_scan_fwd_raw(ctypes.byref(a), ctypes.byref(r), _stream(stream)))
     return out, final_state, saved_states
@@ -576,7 +588,7 @@ def msc_mamba3_siso_scan_bwd_raw_workspace_bytes(batch, seqlen, nheads, headdim,
 def msc_mamba3_siso_scan_bwd_raw(x, dd_dt, dd_a, trap, angles, B_raw, C_raw, saved_states, dout,
                                  dt_bias=None, A_floor=1e-4, eps=1e-5, D=None, z=None, h0=None,
                                  workspace=None, want_dh0=True, grads=None, stream=None):
-    """Mamba-3 SISO backward from raw projections (bf16, d_state <= 64).
+    """Mamba-3 SISO backward from raw projections (bf16, d_state 16, 32 or 64).
     Returns dict dx, dz, dD, dh0 and ddd_dt, ddd_a, dtrap, dangles, ddt_bias,
     dB_raw, dC_raw; equals the scan's backward followed by
     msc_mamba3_siso_discretize_bwd bit for bit."""

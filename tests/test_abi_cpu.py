@@ -461,13 +461,33 @@ def test_fused_raw_scan_checks_raw_args():
     assert "struct_size" in _err()
 
 
+def test_fused_raw_fwd_needs_the_bcnorm_workspace():
+    """BCNorm's rows (bf16 B and C, once per row) live in the forward's
+    workspace; without it the call is refused before any launch."""
+    B, L, H, P, N, G, K = 2, 128, 4, 64, 64, 1, 32
+    need = msc.msc_mamba3_siso_scan_fwd_raw_workspace_bytes(B, L, H, P, N, G, K)
+    assert need >= 2 * 2 * B * L * G * N
+    assert msc.msc_mamba3_siso_scan_fwd_raw_workspace_bytes(B, L, H, P, N, 0, K) == 0
+    fn = msc.lib().msc_mamba3_siso_scan_fwd_raw
+    a = _m3_raw_scan_args()
+    assert fn(ctypes.byref(a), ctypes.byref(_m3_raw()), None) == WORKSPACE
+    assert "workspace" in _err()
+    a.workspace, a.workspace_bytes = ctypes.c_void_p(1 << 20), need - 16
+    assert fn(ctypes.byref(a), ctypes.byref(_m3_raw()), None) == WORKSPACE
+    a.workspace, a.workspace_bytes = ctypes.c_void_p((1 << 20) + 8), need
+    assert fn(ctypes.byref(a), ctypes.byref(_m3_raw()), None) == ALIGNMENT
+    # the scan's pointers are checked before BCNorm launches
+    a.workspace, a.x = ctypes.c_void_p(1 << 20), None
+    assert fn(ctypes.byref(a), ctypes.byref(_m3_raw()), None) == INVALID and "x is NULL" in _err()
+
+
 def test_fused_raw_bwd_workspace_and_grads():
     """The backward from raw projections needs the scan's workspace plus room for
     the scan's gradients of the derived inputs, and its raw-gradient struct."""
     B, L, H, P, N, G, K = 2, 128, 4, 64, 64, 1, 32
     scan = msc.msc_mamba3_siso_scan_bwd_workspace_bytes(B, L, H, P, N, G, K)
     need = msc.msc_mamba3_siso_scan_bwd_raw_workspace_bytes(B, L, H, P, N, G, K)
-    derived = 4 * B * L * (3 * H + H * K + 2 * G * N)
+    derived = 4 * B * L * (3 * H + H * K + 2 * G * N) + 2 * 2 * B * L * G * N  # + BCNorm's rows
     assert need >= scan + derived
     assert msc.msc_mamba3_siso_scan_bwd_raw_workspace_bytes(B, L, H, P, N, 0, K) == 0
     fake = ctypes.c_void_p(1 << 20)
