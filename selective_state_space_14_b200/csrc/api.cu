@@ -312,6 +312,10 @@ msc_status msc_selective_scan_bwd(const msc_ss_bwd_args *a, void *workspace,
   p.ws_bc = reinterpret_cast<float *>(ws + w.bc);
   p.ws_misc = reinterpret_cast<float *>(ws + w.misc);
   p.tok_part = N > msc::kM1Slab ? reinterpret_cast<float *>(ws + w.tok) : nullptr;
+  if (w.n_seg > 1) {
+    p.seg_len = msc::m1_fwd_seg_len(L, w.n_seg);
+    p.seg_ws = reinterpret_cast<float *>(ws + w.seg);
+  }
   return cuda_status(msc::launch_m1_bwd(p, s), fn);
 }
 

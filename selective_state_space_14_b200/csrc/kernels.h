@@ -41,10 +41,12 @@ struct M1Params {
   int64_t n0, ldN;
   int slab;         // kSlabWhole, kSlabFirst, kSlabMiddle or kSlabLast
   float *tok_part;  // fwd: [B][D][L] (y); bwd: [3][B][D][L] (y, dΔ sum, Σ λ B)
-  // forward in time segments (when the (batch, channel) grid alone cannot
-  // fill the GPU): segment blockIdx.z covers steps [z seg_len, (z+1) seg_len);
-  // seg_ws holds per segment and state element the decay product and the
-  // state reached from zero ([2][S][B][D][N], f32), then the carried state
+  // time segments (when the (batch, channel) grid alone cannot fill the
+  // GPU): segment blockIdx.z covers steps [z seg_len, (z+1) seg_len).  seg_ws
+  // holds per segment and state element ([2][S][B][D][N], f32) the decay
+  // product and, forward, the state reached from zero, then the carried
+  // state; backward, the adjoint carry reached from zero at the segment's
+  // left end, then the carry entering it from the right
   int64_t seg_len;  // 0: the whole sequence in one segment
   float *seg_ws;
 };
@@ -66,12 +68,14 @@ inline int64_t m1_bwd_cta_channels(int64_t N) {
 }
 
 int64_t m1_bwd_partials(int64_t D, int64_t N, int64_t G);
+// time segments of the Mamba-1 backward for these sizes (1: none)
+int64_t m1_bwd_segments(int64_t B, int64_t D, int64_t N, int64_t L, int64_t G);
 cudaError_t launch_m1_fwd(const M1Params &p, cudaStream_t s);
 cudaError_t launch_m1_bwd(const M1Params &p, cudaStream_t s);
 size_t m1_bwd_workspace_bytes(int64_t B, int64_t D, int64_t N, int64_t L, int64_t G);
 struct M1BwdWorkspace {
-  int64_t n_part;
-  size_t bc, misc, tok, bytes;  // byte offsets of the regions, total size
+  int64_t n_part, n_seg;
+  size_t bc, misc, tok, seg, bytes;  // byte offsets of the regions, total size
 };
 M1BwdWorkspace m1_bwd_workspace(int64_t B, int64_t D, int64_t N, int64_t L, int64_t G);
 

@@ -241,7 +241,11 @@ __global__ void __launch_bounds__(kWarps * 32, 4) m1_bwd_kernel(const M1Params p
   const T *Bg = static_cast<const T *>(p.Bm) + ((b * p.G + g) * ldN + ns) * L;
   const T *Cg = static_cast<const T *>(p.Cm) + ((b * p.G + g) * ldN + ns) * L;
   const int64_t n_chunks = (L + kS - 1) / kS;
-  const int64_t nb = (L + kBlk - 1) / kBlk;
+  // this CTA's blocks: the whole sequence, or time segment blockIdx.z
+  const int64_t seg = blockIdx.z, n_seg = gridDim.z;
+  const int64_t tb = p.seg_len > 0 ? seg * p.seg_len : 0;
+  const int64_t te = p.seg_len > 0 && tb + p.seg_len < L ? tb + p.seg_len : L;
+  const int64_t kb_lo = tb / kBlk, kb_hi = (te + kBlk - 1) / kBlk;
   const int n0 = 2 * pr, n1 = 2 * pr + 1;
   // this thread's pair of the saved states, one window ahead (windows run
   // backwards: chunk kb * kWin + w)
@@ -264,6 +268,11 @@ __global__ void __launch_bounds__(kWarps * 32, 4) m1_bwd_kernel(const M1Params p
   const float bias_c = (active && p.bias) ? p.bias[c] : 0.f;
   const float D_c = (active && p.Dp && finish) ? p.Dp[c] : 0.f;  // the D terms join once
   float2 mu = make_float2(0.f, 0.f);  // a_{t+1} lambda_{t+1}, handed backwards
+  if (seg < n_seg - 1 && active) {     // the carry entering this segment from the right
+    const float *cs = p.seg_ws + p.B * D * N * (n_seg + seg + 1) + (b * D + c) * N;
+    if (n0 < N) mu.x = cs[n0];
+    if (n1 < N) mu.y = cs[n1];
+  }
   float2 dA = make_float2(0.f, 0.f);  // this (b, c)'s dA for the pair
   float dD_l = 0.f, dbias_l = 0.f;    // per lane (the tokens it finishes)
 
@@ -275,20 +284,20 @@ __global__ void __launch_bounds__(kWarps * 32, 4) m1_bwd_kernel(const M1Params p
   // before, in flight); the first window's saved state ------------------------
   fill_rows<T, kN>(p, rows, b, c_first, c_end, Bg, Cg, tid);
   __syncthreads();
-  issue_stage<T, kN>(p, stage0 + ((nb - 1) & 1) * S::kStageBytes, rows, nb - 1, tid);
-  if (nb >= 2) {
-    issue_stage<T, kN>(p, stage0 + ((nb - 2) & 1) * S::kStageBytes, rows, nb - 2, tid);
+  issue_stage<T, kN>(p, stage0 + ((kb_hi - 1) & 1) * S::kStageBytes, rows, kb_hi - 1, tid);
+  if (kb_hi - kb_lo >= 2) {
+    issue_stage<T, kN>(p, stage0 + ((kb_hi - 2) & 1) * S::kStageBytes, rows, kb_hi - 2, tid);
     cp_async_wait<1>();
   } else {
     cp_async_wait<0>();
   }
-  float2 sv_next = load_saved((nb - 1) * kWin + kWin - 1);
+  float2 sv_next = load_saved((kb_hi - 1) * kWin + kWin - 1);
   __syncthreads();
-  convert_bc<T, kN>(stage0 + ((nb - 1) & 1) * S::kStageBytes, bcf0 + ((nb - 1) & 1) * kBlk * kP,
-                    tid);
+  convert_bc<T, kN>(stage0 + ((kb_hi - 1) & 1) * S::kStageBytes,
+                    bcf0 + ((kb_hi - 1) & 1) * kBlk * kP, tid);
   __syncthreads();
 
-  for (int64_t kb = nb - 1; kb >= 0; --kb) {
+  for (int64_t kb = kb_hi - 1; kb >= kb_lo; --kb) {
     const unsigned char *const st = stage0 + (kb & 1) * S::kStageBytes;
     const float4 *const bcf = bcf0 + (kb & 1) * kBlk * kP;
     float *const acc = acc0 + (kb & 1) * S::kAccFloats;
@@ -423,10 +432,10 @@ __global__ void __launch_bounds__(kWarps * 32, 4) m1_bwd_kernel(const M1Params p
     // ---- end of block: next block's inputs, the cluster's sums in rank order --
     cp_async_wait<0>();  // block kb - 1's inputs (issued one block ago) have landed
     cluster.sync();      // every CTA's accumulators of block kb are complete; block kb's buffers free
-    if (kb >= 1)
+    if (kb - 1 >= kb_lo)
       convert_bc<T, kN>(stage0 + ((kb - 1) & 1) * S::kStageBytes, bcf0 + ((kb - 1) & 1) * kBlk * kP,
                         tid);
-    if (kb >= 2) issue_stage<T, kN>(p, stage0 + (kb & 1) * S::kStageBytes, rows, kb - 2, tid);
+    if (kb - 2 >= kb_lo) issue_stage<T, kN>(p, stage0 + (kb & 1) * S::kStageBytes, rows, kb - 2, tid);
     __syncthreads();  // the new B/C table is visible CTA-wide
     // The peers' accumulators of block kb stay intact until their block kb - 2,
     // which starts after the next cluster barrier: this CTA reaches that
@@ -459,10 +468,10 @@ __global__ void __launch_bounds__(kWarps * 32, 4) m1_bwd_kernel(const M1Params p
     dbias_l += __shfl_xor_sync(0xffffffffu, dbias_l, off, kP);
   }
   if (active) {
-    float *m = p.ws_misc + (b * D + c) * (ldN + 2);
+    float *m = p.ws_misc + ((seg * Bsz + b) * D + c) * (ldN + 2);
     if (n0 < N) m[ns + n0] = dA.x;
     if (n1 < N) m[ns + n1] = dA.y;
-    if (p.dh0) {
+    if (p.dh0 && seg == 0) {
       if (n0 < N) p.dh0[(b * D + c) * ldN + ns + n0] = mu.x;
       if (n1 < N) p.dh0[(b * D + c) * ldN + ns + n1] = mu.y;
     }
@@ -474,7 +483,8 @@ __global__ void __launch_bounds__(kWarps * 32, 4) m1_bwd_kernel(const M1Params p
 }
 
 // dB/dC: sum of a group's partials in ascending order; dA, dD, dbias: sum of
-// the per-(b, c) partials over the batch in ascending order.
+// the per-(segment, b, c) partials over the segments and the batch in
+// ascending order.
 __global__ void m1_bwd_reduce_kernel(const M1Params p) {
   const int64_t Bsz = p.B, D = p.D, N = p.N, L = p.L, G = p.G;
   const int64_t per_group = p.n_part / G;  // partials per group
@@ -497,12 +507,89 @@ __global__ void m1_bwd_reduce_kernel(const M1Params p) {
     } else {
       const int64_t j = i - n_bc;  // (c, k), k < N + 2
       const int64_t c = j / (N + 2), k = j % (N + 2);
+      const int64_t n_seg = p.seg_len > 0 ? (L + p.seg_len - 1) / p.seg_len : 1;
       float s = 0.f;
-      for (int64_t b = 0; b < Bsz; ++b) s += p.ws_misc[(b * D + c) * (N + 2) + k];
+      for (int64_t q = 0; q < n_seg * Bsz; ++q) s += p.ws_misc[(q * D + c) * (N + 2) + k];
       if (k < N) p.dA[c * N + k] = s;
       else if (k == N) { if (p.dD) p.dD[c] = s; }
       else if (p.dbias) p.dbias[c] = s;
     }
+  }
+}
+
+// Time segments, first pass: per state element, segment blockIdx.y walked
+// backwards from a zero adjoint carry, as the backward walks it (mu <- a_t
+// (g_t C_t + mu)), without the states: the product of its decays and the
+// carry it reaches at its left end, to seg_ws.  A thread takes one pair of
+// states of one (b, c).
+template <typename T>
+__global__ void __launch_bounds__(256) m1_bwd_seg_sum_kernel(const M1Params p) {
+  const int64_t N = p.N, D = p.D, L = p.L;
+  const int64_t kPr = (N + 1) / 2;
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= p.B * D * kPr) return;
+  const int64_t q = i % kPr, bc = i / kPr, c = bc % D, b = bc / D;
+  const int64_t seg = blockIdx.y, n_seg = gridDim.y;
+  const int64_t tb = seg * p.seg_len, te = tb + p.seg_len < L ? tb + p.seg_len : L;
+  const int64_t g = c / (D / p.G);
+  const int64_t n0 = 2 * q, n1 = 2 * q + 1;
+  const bool has1 = n1 < N;
+  const float2 A2 = mul2(make_float2(p.A[c * N + n0], has1 ? p.A[c * N + n1] : 0.f),
+                         splat2(kLog2e));
+  const float bias = p.bias ? p.bias[c] : 0.f;
+  const T *drow = static_cast<const T *>(p.delta) + bc * L;
+  const T *yrow = static_cast<const T *>(p.dout) + bc * L;
+  const T *zrow = p.z ? static_cast<const T *>(p.z) + bc * L : nullptr;
+  const T *c0 = static_cast<const T *>(p.Cm) + ((b * p.G + g) * N + n0) * L;
+  const T *c1 = has1 ? c0 + L : c0;
+  float2 mu = make_float2(0.f, 0.f), dec = make_float2(1.f, 1.f);
+#pragma unroll 4
+  for (int64_t t = te - 1; t >= tb; --t) {
+    const float v = to_f32(drow[t]) + bias;
+    const float d = p.softplus ? softplus(v) : v;
+    float gz = to_f32(yrow[t]);
+    if (zrow) {
+      const float zv = to_f32(zrow[t]);
+      gz = gz * (zv * sigmoid(zv));
+    }
+    const float2 a = ex2_2(mul2(splat2(d), A2));
+    const float2 Cv = make_float2(to_f32(c0[t]), has1 ? to_f32(c1[t]) : 0.f);
+    mu = mul2(a, fma2(splat2(gz), Cv, mu));
+    dec = mul2(dec, a);
+  }
+  const int64_t elems = p.B * D * N;
+  float *dd = p.seg_ws + elems * seg + bc * N;
+  float *mm = p.seg_ws + elems * (n_seg + seg) + bc * N;
+  dd[n0] = dec.x;
+  mm[n0] = mu.x;
+  if (has1) {
+    dd[n1] = dec.y;
+    mm[n1] = mu.y;
+  }
+}
+
+// The segments' summaries combined from the sequence's end: segment s takes
+// the carry entering it from the right, x, to decay_s x + carry_s at its left
+// end, so the carry entering segment s is the composition of segments
+// n_seg - 1 .. s + 1 applied to 0.  A warp takes one state element, lane l
+// segment n_seg - 1 - l (lane order = the order of the walk), composed with
+// the warp-shuffle scan of the linear-recurrence monoid; the carry leaving
+// segment s goes over carry_s, which only this warp reads.
+__global__ void m1_bwd_seg_combine_kernel(const M1Params p, int n_seg) {
+  const int64_t elems = p.B * p.D * p.N;
+  const int lane = threadIdx.x & 31;
+  const int s = n_seg - 1 - lane;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t e = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); e < elems;
+       e += warps) {
+    float dc = 1.f, st = 0.f;  // lanes past the segments compose as the identity
+    if (s >= 0) {
+      dc = p.seg_ws[elems * s + e];
+      st = p.seg_ws[elems * (n_seg + s) + e];
+    }
+    float pe, he;
+    warp_scan_fwd(dc, st, pe, he);
+    if (s >= 1) p.seg_ws[elems * (n_seg + s) + e] = fmaf(dc, he, st);  // inclusive, applied to 0
   }
 }
 
@@ -521,7 +608,8 @@ cudaError_t launch_t(const M1Params &p, cudaStream_t s) {
   if (err != cudaSuccess) return err;
   const int64_t grid_x = p.G * ctas_padded_per_group(p.D, kN, p.G);  // the layout's channels per CTA
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)grid_x, (unsigned)p.B);
+  const int64_t n_seg = p.seg_len > 0 ? (p.L + p.seg_len - 1) / p.seg_len : 1;
+  cfg.gridDim = dim3((unsigned)grid_x, (unsigned)p.B, (unsigned)n_seg);
   cfg.blockDim = dim3(Lay::kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
@@ -553,16 +641,36 @@ int64_t m1_bwd_partials(int64_t D, int64_t N, int64_t G) {
   return G * ctas_padded_per_group(D, N > kM1Slab ? kM1Slab : N, G) / kM1BwdCluster;
 }
 
-// Workspace: dB/dC partials [n_part][B][2][N][L], per-(b, c) partials
-// [B][D][N + 2], and above one slab the token sums [3][B][D][L].
+// Time segments of the backward: as the forward's (m1_fwd_segments), only
+// when the CTAs of the (batch, channel-block) grid number fewer than the SMs,
+// aiming at about two CTAs per SM, each segment at least two staged blocks
+// long, at most 32 segments; d_state up to one slab.
+int64_t m1_bwd_segments(int64_t B, int64_t D, int64_t N, int64_t L, int64_t G) {
+  if (N > kM1Slab || B <= 0 || D <= 0 || L <= 0 || G <= 0 || D % G != 0) return 1;
+  const int64_t ctas = B * G * ctas_padded_per_group(D, N, G);
+  constexpr int64_t kSMs = 148;
+  if (ctas >= kSMs) return 1;
+  int64_t n = (2 * kSMs + ctas - 1) / ctas;
+  const int64_t by_len = L / (2 * kBlk);
+  if (n > by_len) n = by_len;
+  if (n > 32) n = 32;
+  if (n < 2) return 1;
+  return (L + m1_fwd_seg_len(L, n) - 1) / m1_fwd_seg_len(L, n);  // segments of whole blocks
+}
+
+// Workspace: dB/dC partials [n_part][B][2][N][L], per-(segment, b, c)
+// partials [S][B][D][N + 2], above one slab the token sums [3][B][D][L], and
+// with time segments their summaries [2][S][B][D][N].
 M1BwdWorkspace m1_bwd_workspace(int64_t B, int64_t D, int64_t N, int64_t L, int64_t G) {
   auto up = [](size_t v) { return (v + 255) / 256 * 256; };
   M1BwdWorkspace w;
   w.n_part = m1_bwd_partials(D, N, G);
+  w.n_seg = m1_bwd_segments(B, D, N, L, G);
   w.bc = 0;
   w.misc = up(sizeof(float) * (size_t)(w.n_part * B * 2 * N * L));
-  w.tok = w.misc + up(sizeof(float) * (size_t)(B * D * (N + 2)));
-  w.bytes = w.tok + (N > kM1Slab ? sizeof(float) * (size_t)(3 * B * D * L) : 0);
+  w.tok = w.misc + up(sizeof(float) * (size_t)(w.n_seg * B * D * (N + 2)));
+  w.seg = w.tok + up(N > kM1Slab ? sizeof(float) * (size_t)(3 * B * D * L) : 0);
+  w.bytes = w.seg + (w.n_seg > 1 ? sizeof(float) * (size_t)(2 * w.n_seg * B * D * N) : 0);
   return w;
 }
 
@@ -576,6 +684,25 @@ size_t m1_bwd_workspace_bytes(int64_t B, int64_t D, int64_t N, int64_t L, int64_
 cudaError_t launch_m1_bwd(const M1Params &p0, cudaStream_t s) {
   const int64_t n_tot = p0.N;
   const int64_t slabs = (n_tot + kM1Slab - 1) / kM1Slab;
+  if (p0.seg_len > 0) {
+    // time segments: each one's summary from a zero carry, then the carries
+    // entering them, composed from the sequence's end
+    const int64_t n_seg = (p0.L + p0.seg_len - 1) / p0.seg_len;
+    const int64_t items = p0.B * p0.D * ((p0.N + 1) / 2);
+    const dim3 grid((unsigned)((items + 255) / 256), (unsigned)n_seg);
+    switch (p0.io) {
+      case 1: m1_bwd_seg_sum_kernel<bf16><<<grid, 256, 0, s>>>(p0); break;
+      case 2: m1_bwd_seg_sum_kernel<f16><<<grid, 256, 0, s>>>(p0); break;
+      default: m1_bwd_seg_sum_kernel<float><<<grid, 256, 0, s>>>(p0); break;
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const int64_t elems = p0.B * p0.D * p0.N;
+    int64_t blocks = (elems + 7) / 8;  // 8 warps of 32 per block, a warp per element
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    m1_bwd_seg_combine_kernel<<<(unsigned)blocks, 256, 0, s>>>(p0, (int)n_seg);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
   for (int64_t k = 0; k < slabs; ++k) {
     M1Params p = p0;
     p.ldN = n_tot;

@@ -225,6 +225,22 @@ def test_fwd_time_segments_workspace():
     assert msc.msc_selective_scan_fwd_workspace_bytes(1, 8, 128, 4096) == 4 * 1 * 8 * 4096
 
 
+def test_bwd_workspace_holds_the_time_segments():
+    """A grid of few (batch, channel) blocks splits the backward into time
+    segments: the workspace then holds per-segment partials and summaries; a
+    model-shaped grid does not split."""
+    def base(B, D, N, L, n_part, n_seg=1):
+        up = lambda v: (v + 255) // 256 * 256
+        return up(4 * n_part * B * 2 * N * L) + up(4 * n_seg * B * D * (N + 2))
+    # 8 CTAs of 12 channels (one cluster): 4 segments of 64 steps
+    got = msc.msc_selective_scan_bwd_workspace_bytes(1, 64, 16, 256, 1)
+    assert got == base(1, 64, 16, 256, 1, 4) + 4 * 2 * 4 * 1 * 64 * 16
+    # the 130M-layer shape fills the GPU: no segments (ceil(1536 / 12) = 128
+    # CTAs per batch row, one partial per cluster of 8)
+    assert msc.msc_selective_scan_bwd_workspace_bytes(8, 1536, 16, 2048, 1) == \
+        base(8, 1536, 16, 2048, 128 // 8)
+
+
 def test_bwd_workspace_query_refuses_bad_groups():
     """ngroups < 1 or not a divisor of dim needs no workspace (the backward
     refuses it); the query must not divide by it."""

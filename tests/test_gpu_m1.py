@@ -123,8 +123,10 @@ SEG_CASES = [
 
 @pytest.mark.parametrize("case", SEG_CASES, ids=[f"B{c[0]}D{c[1]}N{c[2]}L{c[3]}{c[4]}" for c in SEG_CASES])
 def test_time_segments_parity(msc, case):
-    """Forward in time segments (and the backward from its saved states)
-    against the oracle: the segment count the workspace query implies is > 1."""
+    """Forward and backward in time segments against the oracle: the grids of
+    (batch, channel) blocks are small enough that both split time (the
+    forward's workspace query is > 0; the backward's includes the segments'
+    summaries), the summaries composed by the warp-shuffle scan."""
     Bsz, D, N, L, io = case
     assert msc.msc_selective_scan_fwd_workspace_bytes(Bsz, D, N, L) > 0
     p = W.m1_problem(Bsz, D, N, L, io=io, seed=3000 + L, bias=True, with_h0=True)
