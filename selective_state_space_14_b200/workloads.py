@@ -399,6 +399,9 @@ WORKLOADS = {
                                        io=BF16, bias=True, seed=SEED_BASE + 1),
     "m1_bf16_b4_d5120_n16_l4096": dict(kind="m1", batch=4, dim=5120, dstate=16, seqlen=4096,
                                        io=BF16, bias=True, seed=SEED_BASE + 2),
+    # one sequence of few channels: the scans split time into segments
+    "m1_bf16_b1_d256_n16_l4096": dict(kind="m1", batch=1, dim=256, dstate=16, seqlen=4096,
+                                      io=BF16, bias=True, seed=SEED_BASE + 9),
     "m3_bf16_b8_h24_p64_n64_k32_l2048": dict(kind="m3", batch=8, seqlen=2048, nheads=24,
                                              headdim=64, dstate=64, nangles=32, io=BF16,
                                              seed=SEED_BASE + 3),
