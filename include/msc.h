@@ -104,10 +104,15 @@ const char *msc_version(void);
  * starting from h = h0[b,c,:] (or 0).  final_state receives h after the last
  * step.  saved_states receives h at the start of every block of
  * MSC_M1_SAVE_INTERVAL steps (the first is h0); the backward pass needs it.
- * N may be 1..256 ("state dimensions up to 256", mamba-rs README,
- * "Features"); L >= 1.  Above 64 states the scan runs in slabs of 64 states
- * and the forward needs a workspace of msc_selective_scan_fwd_workspace_bytes()
- * bytes (0 up to 64 states) for the sums over the earlier slabs.
+ * N may be 1..256 (the largest state the mamba-rs README lists under
+ * "Features"); L >= 1.  Above 64 states the scan runs in slabs of 64 states;
+ * with few (batch, channel) rows for the GPU's SMs it splits time into
+ * segments whose summaries a warp-shuffle scan composes (the associative
+ * combine of the recurrence).  In both cases the forward needs a workspace
+ * of msc_selective_scan_fwd_workspace_bytes() bytes (0 otherwise): the sums
+ * over the earlier slabs, or the segments' summaries.  The segments change
+ * only the rounding order, not the result's accuracy; every configuration
+ * gives the same bits from run to run.
  */
 #define MSC_M1_SAVE_INTERVAL 8
 #define MSC_M1_MAX_DSTATE 256
@@ -127,11 +132,12 @@ typedef struct {
   void *out;
   float *final_state;      /* optional */
   float *saved_states;     /* optional; required if the backward pass follows */
-  void *workspace;         /* required when dstate > 64, else ignored (may be NULL) */
+  void *workspace;         /* required when the workspace query is > 0, else ignored */
   size_t workspace_bytes;
 } msc_ss_fwd_args;
 
-/* Bytes of the forward's workspace for these sizes (0 when dstate <= 64). */
+/* Bytes of the forward's workspace for these sizes (0 when the forward needs
+ * none: up to 64 states, with enough rows to fill the GPU). */
 size_t msc_selective_scan_fwd_workspace_bytes(int64_t batch, int64_t dim, int64_t dstate,
                                               int64_t seqlen);
 
@@ -159,7 +165,9 @@ msc_status msc_selective_scan_fwd(const msc_ss_fwd_args *args, msc_stream_t stre
  * dD, ddelta_bias, dz and dh0 are optional outputs (NULL: not computed).
  * Every output is overwritten (not accumulated into).
  * Workspace: msc_selective_scan_bwd_workspace_bytes() bytes of device memory,
- * contents on entry irrelevant.
+ * contents on entry irrelevant (the dB/dC partials of each cluster of
+ * channel blocks, and with few (batch, channel) rows the summaries of the
+ * time segments the backward then splits into).
  */
 typedef struct {
   uint32_t struct_size;
