@@ -121,6 +121,32 @@ SEG_CASES = [
 ]
 
 
+SEG_VARIANT_CASES = [
+    # (B, D, N, L, io, G, z, bias, softplus, h0): the branches of the segment
+    # summaries -- groups of B/C, no gate, no bias, raw delta, f16 storage
+    (1, 96, 16, 1024, "bf16", 2, True, True, True, False),
+    (1, 48, 16, 700, "f32", 1, False, False, True, True),
+    (1, 32, 32, 900, "f32", 1, True, False, False, True),
+    (2, 24, 16, 1500, "f16", 3, True, True, True, True),
+]
+
+
+@pytest.mark.parametrize("case", SEG_VARIANT_CASES,
+                         ids=[f"B{c[0]}D{c[1]}N{c[2]}L{c[3]}{c[4]}G{c[5]}z{int(c[6])}b{int(c[7])}"
+                              f"sp{int(c[8])}" for c in SEG_VARIANT_CASES])
+def test_time_segments_variants(msc, case):
+    """Both scans in time segments with groups, without the gate or the bias,
+    with softplus off, and in f16, against the oracle."""
+    Bsz, D, N, L, io, G, z, bias, sp, h0 = case
+    assert msc.msc_selective_scan_fwd_workspace_bytes(Bsz, D, N, L) > 0
+    p = W.m1_problem(Bsz, D, N, L, io=io, seed=3100 + L, ngroups=G, bias=bias, with_z=z,
+                     with_h0=h0, delta_softplus=sp)
+    if not sp:  # softplus off: keep delta positive (no bias) so the state stays bounded
+        p.delta = W.store(np.abs(p.delta.as_f32()) * 0.2, io)
+        p.delta_bias = None
+    _compare(_run_gpu(msc, p), _run_oracle(p), TOL[io])
+
+
 @pytest.mark.parametrize("case", SEG_CASES, ids=[f"B{c[0]}D{c[1]}N{c[2]}L{c[3]}{c[4]}" for c in SEG_CASES])
 def test_time_segments_parity(msc, case):
     """Forward and backward in time segments against the oracle: the grids of

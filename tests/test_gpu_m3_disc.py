@@ -282,8 +282,9 @@ def test_fused_decode_vs_oracle(msc):
 
 
 # --------------------------------------------------------------------------
-# The scan from raw projections (discretisation and BCNorm fused into the
-# scan's kernels): bit for bit the two-call chain, and so the oracle's chain
+# The scan from raw projections (the per-head discretisation fused into the
+# forward kernel, BCNorm once per row ahead of it; the backward re-deriving
+# both): bit for bit the two-call chain, and so the oracle's chain
 # --------------------------------------------------------------------------
 SCAN_OUT = ("dx", "dz", "dD", "dh0")
 
