@@ -382,3 +382,24 @@ def test_fused_raw_full_size_equals_the_chain(msc):
     q = W.make("m3disc_bf16_b8_h24_p64_n64_k32_l2048")
     chain, fused = _chain_and_fused(msc, q, h0=False)
     _assert_bit_equal(chain, fused, ("out", "final_state", "saved") + SCAN_OUT + DISC_GRADS)
+
+
+def test_fused_raw_empty_sequence(msc):
+    """L = 0 from raw projections: the final state is h0; dD, dh0 and the dt
+    bias gradient are zero; nothing else is touched."""
+    Bsz, H, P, N, K = 2, 3, 64, 64, 16
+    bf = dict(device="cuda", dtype=torch.bfloat16)
+    x = torch.empty(Bsz, 0, H, P, **bf)
+    raw = dict(dd_dt=torch.empty(Bsz, 0, H, **bf), dd_a=torch.empty(Bsz, 0, H, **bf),
+               trap=torch.empty(Bsz, 0, H, **bf), angles=torch.empty(Bsz, 0, K, **bf),
+               B_raw=torch.empty(Bsz, 0, 1, N, **bf), C_raw=torch.empty(Bsz, 0, 1, N, **bf))
+    h0 = torch.randn(Bsz, H, P, N, device="cuda")
+    dtb = torch.randn(H, device="cuda")
+    out, fs, saved = msc.msc_mamba3_siso_scan_fwd_raw(x, **raw, dt_bias=dtb, h0=h0)
+    g = msc.msc_mamba3_siso_scan_bwd_raw(x, **raw, dt_bias=dtb, h0=h0, saved_states=saved,
+                                         dout=torch.empty_like(x),
+                                         D=torch.randn(H, device="cuda"))
+    torch.cuda.synchronize()
+    assert out.numel() == 0 and torch.equal(fs, h0)
+    assert torch.count_nonzero(g["dD"]) == 0 and torch.count_nonzero(g["dh0"]) == 0
+    assert torch.count_nonzero(g["ddt_bias"]) == 0
