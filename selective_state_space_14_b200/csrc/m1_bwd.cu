@@ -521,51 +521,93 @@ __global__ void m1_bwd_reduce_kernel(const M1Params p) {
 // backwards from a zero adjoint carry, as the backward walks it (mu <- a_t
 // (g_t C_t + mu)), without the states: the product of its decays and the
 // carry it reaches at its left end, to seg_ws.  A thread takes one pair of
-// states of one (b, c).
-template <typename T>
+// states of one (b, c); the kPw lanes of a channel (kPw the power of two at
+// or above its pairs) take the token values of kPw steps at a time, one step
+// each, and hand them round by shuffles.
+template <typename T, int kPw>
 __global__ void __launch_bounds__(256) m1_bwd_seg_sum_kernel(const M1Params p) {
   const int64_t N = p.N, D = p.D, L = p.L;
   const int64_t kPr = (N + 1) / 2;
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= p.B * D * kPr) return;
-  const int64_t q = i % kPr, bc = i / kPr, c = bc % D, b = bc / D;
+  const int q = (int)(threadIdx.x % kPw);
+  const int64_t bc = i / kPw;
+  const bool live = bc < p.B * D;  // every lane of a warp stays for the shuffles
+  const bool act = live && q < kPr;
+  const int64_t c = live ? bc % D : 0, b = live ? bc / D : 0;
   const int64_t seg = blockIdx.y, n_seg = gridDim.y;
   const int64_t tb = seg * p.seg_len, te = tb + p.seg_len < L ? tb + p.seg_len : L;
   const int64_t g = c / (D / p.G);
-  const int64_t n0 = 2 * q, n1 = 2 * q + 1;
-  const bool has1 = n1 < N;
-  const float2 A2 = mul2(make_float2(p.A[c * N + n0], has1 ? p.A[c * N + n1] : 0.f),
+  const int64_t n0 = 2 * (int64_t)q, n1 = n0 + 1;
+  const bool has0 = act && n0 < N, has1 = act && n1 < N;
+  const float2 A2 = mul2(make_float2(has0 ? p.A[c * N + n0] : 0.f, has1 ? p.A[c * N + n1] : 0.f),
                          splat2(kLog2e));
-  const float bias = p.bias ? p.bias[c] : 0.f;
-  const T *drow = static_cast<const T *>(p.delta) + bc * L;
-  const T *yrow = static_cast<const T *>(p.dout) + bc * L;
-  const T *zrow = p.z ? static_cast<const T *>(p.z) + bc * L : nullptr;
-  const T *c0 = static_cast<const T *>(p.Cm) + ((b * p.G + g) * N + n0) * L;
+  const float bias = (live && p.bias) ? p.bias[c] : 0.f;
+  const int64_t row = (live ? bc : 0) * L;
+  const T *drow = static_cast<const T *>(p.delta) + row;
+  const T *yrow = static_cast<const T *>(p.dout) + row;
+  const T *zrow = p.z ? static_cast<const T *>(p.z) + row : nullptr;
+  const T *c0 = static_cast<const T *>(p.Cm) + ((b * p.G + g) * N + (has0 ? n0 : 0)) * L;
   const T *c1 = has1 ? c0 + L : c0;
   float2 mu = make_float2(0.f, 0.f), dec = make_float2(1.f, 1.f);
-#pragma unroll 4
-  for (int64_t t = te - 1; t >= tb; --t) {
-    const float v = to_f32(drow[t]) + bias;
-    const float d = p.softplus ? softplus(v) : v;
-    float gz = to_f32(yrow[t]);
-    if (zrow) {
-      const float zv = to_f32(zrow[t]);
-      gz = gz * (zv * sigmoid(zv));
+  for (int64_t th = te - 1; th >= tb; th -= kPw) {
+    // this lane's step of the group: th - q
+    const int64_t tq = th - q;
+    float d_own = 0.f, g_own = 0.f;
+    if (live && tq >= tb) {
+      const float v = to_f32(drow[tq]) + bias;
+      d_own = p.softplus ? softplus(v) : v;
+      g_own = to_f32(yrow[tq]);
+      if (zrow) {
+        const float zv = to_f32(zrow[tq]);
+        g_own = g_own * (zv * sigmoid(zv));
+      }
     }
-    const float2 a = ex2_2(mul2(splat2(d), A2));
-    const float2 Cv = make_float2(to_f32(c0[t]), has1 ? to_f32(c1[t]) : 0.f);
-    mu = mul2(a, fma2(splat2(gz), Cv, mu));
-    dec = mul2(dec, a);
+#pragma unroll
+    for (int s = 0; s < kPw; ++s) {
+      const int64_t t = th - s;
+      if (t < tb) break;  // the same for every thread of the block
+      const float d = __shfl_sync(0xffffffffu, d_own, s, kPw);
+      const float gz = __shfl_sync(0xffffffffu, g_own, s, kPw);
+      if (act) {
+        const float2 a = ex2_2(mul2(splat2(d), A2));
+        const float2 Cv = make_float2(has0 ? to_f32(c0[t]) : 0.f, has1 ? to_f32(c1[t]) : 0.f);
+        mu = mul2(a, fma2(splat2(gz), Cv, mu));
+        dec = mul2(dec, a);
+      }
+    }
   }
+  if (!act) return;
   const int64_t elems = p.B * D * N;
   float *dd = p.seg_ws + elems * seg + bc * N;
   float *mm = p.seg_ws + elems * (n_seg + seg) + bc * N;
-  dd[n0] = dec.x;
-  mm[n0] = mu.x;
+  if (has0) {
+    dd[n0] = dec.x;
+    mm[n0] = mu.x;
+  }
   if (has1) {
     dd[n1] = dec.y;
     mm[n1] = mu.y;
   }
+}
+
+// the summary pass: kPw lanes per channel, the power of two at or above its
+// state pairs (d_state <= 64: at most 32)
+template <typename T, int kPw>
+cudaError_t launch_seg_sum_w(const M1Params &p, int64_t n_seg, cudaStream_t s) {
+  const int64_t items = p.B * p.D * kPw;
+  const dim3 grid((unsigned)((items + 255) / 256), (unsigned)n_seg);
+  m1_bwd_seg_sum_kernel<T, kPw><<<grid, 256, 0, s>>>(p);
+  return cudaGetLastError();
+}
+template <typename T>
+cudaError_t launch_seg_sum(const M1Params &p, int64_t n_seg, cudaStream_t s) {
+  const int64_t pr = (p.N + 1) / 2;
+  if (pr <= 1) return launch_seg_sum_w<T, 1>(p, n_seg, s);
+  if (pr <= 2) return launch_seg_sum_w<T, 2>(p, n_seg, s);
+  if (pr <= 4) return launch_seg_sum_w<T, 4>(p, n_seg, s);
+  if (pr <= 8) return launch_seg_sum_w<T, 8>(p, n_seg, s);
+  if (pr <= 16) return launch_seg_sum_w<T, 16>(p, n_seg, s);
+  return launch_seg_sum_w<T, 32>(p, n_seg, s);
 }
 
 // The segments' summaries combined from the sequence's end: segment s takes
@@ -688,14 +730,12 @@ cudaError_t launch_m1_bwd(const M1Params &p0, cudaStream_t s) {
     // time segments: each one's summary from a zero carry, then the carries
     // entering them, composed from the sequence's end
     const int64_t n_seg = (p0.L + p0.seg_len - 1) / p0.seg_len;
-    const int64_t items = p0.B * p0.D * ((p0.N + 1) / 2);
-    const dim3 grid((unsigned)((items + 255) / 256), (unsigned)n_seg);
+    cudaError_t e;
     switch (p0.io) {
-      case 1: m1_bwd_seg_sum_kernel<bf16><<<grid, 256, 0, s>>>(p0); break;
-      case 2: m1_bwd_seg_sum_kernel<f16><<<grid, 256, 0, s>>>(p0); break;
-      default: m1_bwd_seg_sum_kernel<float><<<grid, 256, 0, s>>>(p0); break;
+      case 1: e = launch_seg_sum<bf16>(p0, n_seg, s); break;
+      case 2: e = launch_seg_sum<f16>(p0, n_seg, s); break;
+      default: e = launch_seg_sum<float>(p0, n_seg, s); break;
     }
-    cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const int64_t elems = p0.B * p0.D * p0.N;
     int64_t blocks = (elems + 7) / 8;  // 8 warps of 32 per block, a warp per element
