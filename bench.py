@@ -122,7 +122,7 @@ def m3su_raw_bytes(Bsz, H, P, N, G, K, io_bytes):
 # ---------------------------------------------------------------------------
 NCU_TRAFFIC = {
     # kernel source file: (sha256 prefix of the file, workload, bytes per launch)
-    "m1_bwd.cu": ("50b388afa4bff451", "m1_bf16_b4_d5120_n16_l4096", 1350000000 + 592000000),
+    "m1_bwd.cu": ("aa9e576ab0269254", "m1_bf16_b4_d5120_n16_l4096", 1350000000 + 592440000),
     "m1_fwd.cu": ("cb6f1bfb350b55cd", "m1_bf16_b4_d5120_n16_l4096", 505620000 + 792910000),
 }
 
