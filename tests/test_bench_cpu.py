@@ -118,3 +118,18 @@ def test_reference_arm_prints_one_line():
     assert d["value"] > 0 and d["higher_is_better"] is True
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+
+
+def test_m1_sfu_ops():
+    """The compute ceiling's operation count: one 2^x per state element and step
+    (its decay) plus the per-token transcendentals -- four in the forward
+    (softplus: 2^x and a logarithm or reciprocal; the silu gate: 2^x and a
+    reciprocal), six in the backward (softplus, and the sigmoids of the gate
+    and of the delta pre-activation)."""
+    B, D, N, L = 4, 5120, 16, 4096
+    fwd, bwd = bench.m1_sfu_ops(B, D, N, L)
+    tc = B * D * L
+    assert fwd == tc * (N + 4) and bwd == tc * (N + 6)
+    # at the 2.8B layer: 1.68e9 and 1.85e9 operations, the figures the bench
+    # line's `compute` entries divide by the measured 2^x rate
+    assert fwd == 1677721600 and bwd == 1845493760
